@@ -1,0 +1,139 @@
+"""Float64 CPU oracle for pair-bias multi-query attention (ctypes wrapper).
+
+TEST INFRASTRUCTURE ONLY: tests/, ``__graft_entry__.smoke()`` and the
+cpu_baseline / reference leg of ``bench.py`` are the only callers.  The
+product package never imports this module and shares no code with it.
+
+The arithmetic lives in ``oracle.c`` (plain C, float64, OpenMP).  This
+wrapper only converts inputs to contiguous float64 numpy arrays and calls it.
+The definition it follows is Eq. L_ij of the page "Making Full-Context
+AlphaGenome Fit on an RTX 3090" (section "Why stock FlashAttention was not a
+drop-in replacement"), with the softmax over all keys and natural-log lse.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_c_double_p = ctypes.POINTER(ctypes.c_double)
+_c_int64_p = ctypes.POINTER(ctypes.c_int64)
+
+
+def _f64(x) -> np.ndarray:
+    """Exact widening of a torch tensor (bf16 / fp32 / fp64) or array."""
+    try:
+        import torch
+
+        if isinstance(x, torch.Tensor):
+            x = x.detach().to("cpu", torch.float64).numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(_c_double_p)
+
+
+class Oracle:
+    """Handle on one build of the oracle library (the default or a mutant)."""
+
+    def __init__(self, libpath: str | None = None):
+        if libpath is None:
+            libpath = _build.ensure_built()
+        self.libpath = libpath
+        lib = ctypes.CDLL(libpath)
+        L = ctypes.c_long
+        lib.agref_pair_bias_project.argtypes = [
+            _c_double_p, _c_double_p, _c_double_p, L, L, L, ctypes.c_int]
+        lib.agref_attn_fwd.argtypes = [
+            _c_double_p, _c_double_p, _c_double_p, _c_double_p,
+            L, L, L, L, L, L, ctypes.c_double,
+            _c_double_p, _c_double_p, _c_double_p, ctypes.c_int]
+        lib.agref_attn_rows.argtypes = [
+            _c_double_p, _c_double_p, _c_double_p, _c_double_p,
+            L, L, L, L, L, L, ctypes.c_double,
+            _c_int64_p, L, _c_double_p, _c_double_p, ctypes.c_int]
+        lib.agref_max_threads.argtypes = [ctypes.c_int]
+        for f in ("agref_pair_bias_project", "agref_attn_fwd",
+                  "agref_attn_rows", "agref_max_threads", "agref_mutant_id"):
+            getattr(lib, f).restype = ctypes.c_int
+        self._lib = lib
+        self.mutant = lib.agref_mutant_id()
+
+    def threads(self, nthreads: int = 0) -> int:
+        """Set (if > 0) and return the OpenMP thread count the oracle uses."""
+        return int(self._lib.agref_max_threads(int(nthreads)))
+
+    # -- pair-bias projection -------------------------------------------------
+    def pair_bias_project(self, pair, W, nthreads: int = 0) -> np.ndarray:
+        """bias[h,p,q] = sum_c pair[p,q,c] * W[c,h]; pair [P,P,Cp], W [Cp,H]."""
+        pair = _f64(pair)
+        W = _f64(W)
+        P, P2, Cp = pair.shape
+        assert P == P2 and W.shape[0] == Cp
+        H = W.shape[1]
+        bias = np.empty((H, P, P), dtype=np.float64)
+        rc = self._lib.agref_pair_bias_project(
+            _ptr(pair), _ptr(W), _ptr(bias), P, Cp, H, int(nthreads))
+        if rc != 0:
+            raise ValueError(f"agref_pair_bias_project rc={rc}")
+        return bias
+
+    # -- attention ------------------------------------------------------------
+    def attn_fwd(self, q, k, v, bias, block: int = 16, cap: float = 5.0,
+                 probs: bool = False, nthreads: int = 0):
+        """Full attention: returns (out [B,H,L,Dv], lse [B,H,L]) and, if
+        probs=True, also the softmax weights [B,H,L,L] (tiny inputs only)."""
+        q, k, v, bias = _f64(q), _f64(k), _f64(v), _f64(bias)
+        B, H, L, D = q.shape
+        Dv = v.shape[-1]
+        assert k.shape == (B, L, D) and v.shape == (B, L, Dv)
+        out = np.empty((B, H, L, Dv), dtype=np.float64)
+        lse = np.empty((B, H, L), dtype=np.float64)
+        pr = np.empty((B, H, L, L), dtype=np.float64) if probs else None
+        rc = self._lib.agref_attn_fwd(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(bias), B, H, L, D, Dv, int(block),
+            float(cap), _ptr(out), _ptr(lse),
+            _ptr(pr) if probs else None, int(nthreads))
+        if rc != 0:
+            raise ValueError(f"agref_attn_fwd rc={rc}")
+        return (out, lse, pr) if probs else (out, lse)
+
+    def attn_rows(self, q, k, v, bias, rows, block: int = 16,
+                  cap: float = 5.0, nthreads: int = 0):
+        """Selected rows: rows is an int array [n,3] of (b, h, i).  Returns
+        (out_rows [n,Dv], lse_rows [n])."""
+        q, k, v, bias = _f64(q), _f64(k), _f64(v), _f64(bias)
+        B, H, L, D = q.shape
+        Dv = v.shape[-1]
+        rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
+        n = rows.shape[0]
+        out = np.empty((n, Dv), dtype=np.float64)
+        lse = np.empty((n,), dtype=np.float64)
+        rc = self._lib.agref_attn_rows(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(bias), B, H, L, D, Dv, int(block),
+            float(cap), rows.ctypes.data_as(_c_int64_p), n, _ptr(out),
+            _ptr(lse), int(nthreads))
+        if rc != 0:
+            raise ValueError(f"agref_attn_rows rc={rc}")
+        return out, lse
+
+
+_default: Oracle | None = None
+
+
+def default() -> Oracle:
+    """The oracle built from the unmodified source."""
+    global _default
+    if _default is None:
+        _default = Oracle()
+    return _default
+
+
+INF = math.inf
