@@ -1,0 +1,132 @@
+/*
+ * ag.h -- C ABI of libag, pair-bias multi-query attention for B200 (sm_100a).
+ *
+ * The operation is the sequence attention of the page "Making Full-Context
+ * AlphaGenome Fit on an RTX 3090" (section "Why stock FlashAttention was not
+ * a drop-in replacement", Eq. L_ij): eight query heads share one K/V head,
+ * a compact learned pair bias with one cell per 16 x 16 position square is
+ * added to the scaled dot product, the sum is soft-capped with cap*tanh(./cap)
+ * and a softmax over all keys weights V.  The per-head compact bias comes
+ * from a linear projection of a compact pair representation (same page,
+ * section "Profiling pointed at one very large object").
+ *
+ * Conventions shared by every entry point:
+ *   - Every pointer argument is a DEVICE pointer unless stated otherwise,
+ *     row-major, densely packed.  The caller allocates and owns all buffers;
+ *     the library allocates no device memory and keeps no per-call state.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls are asynchronous on that stream: AG_OK means the work
+ *     was enqueued.  Faults inside a kernel surface at the caller's next
+ *     synchronisation, and bounded-wait timeouts in the device error word
+ *     (ag_device_error).
+ *   - Arguments are validated before anything is launched.  On any error
+ *     the call returns the status and writes nothing.
+ *   - Outputs must not overlap inputs (AG_ERR_ALIAS).
+ *   - The kernels are built for sm_100a only; on any other device the
+ *     compute entry points return AG_ERR_UNSUPPORTED.
+ */
+#ifndef AG_H_
+#define AG_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    AG_OK = 0,
+    AG_ERR_NULL = 1,        /* a required pointer is NULL                     */
+    AG_ERR_SHAPE = 2,       /* a size is negative or sizes are inconsistent   */
+    AG_ERR_ALIGN = 3,       /* a pointer lacks the alignment stated below     */
+    AG_ERR_UNSUPPORTED = 4, /* valid sizes the kernels do not handle, or the
+                               current device is not sm_100                   */
+    AG_ERR_VALUE = 5,       /* a scalar argument is out of range (cap)        */
+    AG_ERR_CUDA = 6,        /* a CUDA runtime or driver call failed           */
+    AG_ERR_ALIAS = 7,       /* an output buffer overlaps an input buffer      */
+    AG_ERR_DEVICE = 8       /* the device error word is set (see below)       */
+} ag_status;
+
+/* Static, human-readable name of a status code (never NULL). */
+const char *ag_status_string(int status);
+
+/* Library version as 10000*major + 100*minor + patch. */
+int ag_version(void);
+
+/*
+ * ag_pair_bias_project -- compact pair representation to per-head bias.
+ *
+ *   bias[h, p, q] = sum_c pair[p, q, c] * W[c, h]
+ *
+ * Source: page "Making Full-Context AlphaGenome Fit on an RTX 3090", section
+ * "Profiling pointed at one very large object" (the dense path projects a
+ * compact pair representation into the attention bias before repeating it
+ * 16x along both sequence axes).  The page gives no further terms; this is
+ * the plain linear map.
+ *
+ *   pair  [P, P, Cp] float32, 16-byte aligned
+ *   W     [Cp, H]    float32,  4-byte aligned
+ *   bias  [H, P, P]  float32,  8-byte aligned (written)
+ *   P >= 0 (P == 0 is a no-op); supported: Cp == 128, H == 8, P <= 4096.
+ * Float32 multiply-add accumulation in a fixed order.
+ */
+ag_status ag_pair_bias_project(const float *pair, const float *W, float *bias,
+                               int64_t P, int64_t Cp, int64_t H, void *stream);
+
+/*
+ * ag_attn_fwd -- fused pair-bias multi-query attention forward.
+ *
+ * For b < B, h < H, query i < L, key j < L (page "Making Full-Context
+ * AlphaGenome Fit on an RTX 3090", section "Why stock FlashAttention was not
+ * a drop-in replacement", Eq. L_ij; online softmax of section "Online
+ * softmax, one block at a time"):
+ *   s_ij   = q[b,h,i,:] . k[b,j,:] / sqrt(D) + bias[h, i/block, j/block]
+ *   L_ij   = cap * tanh(s_ij / cap)       (cap == +INFINITY: L_ij = s_ij)
+ *   lse    = log(sum_j exp(L_ij))         (natural log)   -> lse[b,h,i]
+ *   out    = sum_j exp(L_ij - lse) v[b,j,:]              -> out[b,h,i,:]
+ * No L x L tensor is formed.  No mask (every key attends).
+ *
+ *   q     [B, H, L, D]  bfloat16 bit patterns, 16-byte aligned
+ *   k     [B, L, D]     bfloat16, 16-byte aligned (one head, shared by all H)
+ *   v     [B, L, D]     bfloat16, 16-byte aligned (one head, shared by all H)
+ *   bias  [H, P, P]     float32,   4-byte aligned, P = L / block, shared by
+ *                       every batch item
+ *   out   [B, H, L, D]  float32,  16-byte aligned (written)
+ *   lse   [B, H, L]     float32,   4-byte aligned (written)
+ *   cap   > 0 and not NaN; +INFINITY disables the soft cap.
+ * Supported: H == 8, D == 128, block == 16, L % 16 == 0, L <= 65536,
+ * B * L <= 2^31 / 8.  B == 0 or L == 0 is a no-op (pointers may be NULL).
+ * Products in bf16 with fp32 accumulation (tensor cores); softmax in fp32;
+ * the probabilities are rounded to bf16 for the second product while the
+ * row sums use their fp32 values.
+ */
+ag_status ag_attn_fwd(const void *q, const void *k, const void *v,
+                      const float *bias, int64_t B, int64_t H, int64_t L,
+                      int64_t D, int64_t block, float cap, float *out,
+                      float *lse, void *stream);
+
+/*
+ * Device error word.  Every wait inside the kernels is bounded (about one
+ * second); a wait that runs out makes the kernel stop, release what it
+ * holds and record a code here instead of hanging the GPU.
+ *   code == 0: no error.  Otherwise (site << 8) | kind, kind 1 = wait timeout.
+ * ag_device_error synchronises `device`, copies the word of that device to
+ * *code (host pointer) and clears it if `clear` != 0.  Returns AG_ERR_DEVICE
+ * if the word was set, AG_OK if not, AG_ERR_CUDA/AG_ERR_NULL on failure.
+ */
+ag_status ag_device_error(int device, int *code, int clear);
+
+/*
+ * Self-test of the bounded waits: launches one block whose thread waits on an
+ * mbarrier that nothing ever arrives at, for at most `timeout_ns`
+ * nanoseconds (1 ms .. 10 s), and then records site 255 in the device error
+ * word.  Lets a test check that a wait that runs out is reported and leaves
+ * the context usable.  No fault and no hang: the wait is always bounded.
+ */
+ag_status ag_debug_wait_timeout(uint64_t timeout_ns, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AG_H_ */

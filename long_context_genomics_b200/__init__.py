@@ -1,0 +1,163 @@
+"""Python binding of libag: pair-bias multi-query attention on B200.
+
+Argument marshalling only.  Every step of the computation runs in the CUDA
+kernels of libag.so (see include/ag.h for the C ABI); there is no CPU or
+PyTorch fallback, and importing this package raises if the library is
+missing.  PyTorch supplies device memory and the current stream.
+
+    ag_pair_bias_project(pair[P,P,Cp] f32, W[Cp,H] f32) -> bias[H,P,P] f32
+    ag_attn_fwd(q[B,H,L,D] bf16, k[B,L,D] bf16, v[B,L,D] bf16,
+                bias[H,P,P] f32, cap) -> (out[B,H,L,D] f32, lse[B,H,L] f32)
+
+The operation is Eq. L_ij of the page "Making Full-Context AlphaGenome Fit
+on an RTX 3090" (section "Why stock FlashAttention was not a drop-in
+replacement") with a softmax over all keys.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libag.so")
+
+AG_OK = 0
+STATUS_NAMES = {
+    0: "AG_OK", 1: "AG_ERR_NULL", 2: "AG_ERR_SHAPE", 3: "AG_ERR_ALIGN",
+    4: "AG_ERR_UNSUPPORTED", 5: "AG_ERR_VALUE", 6: "AG_ERR_CUDA",
+    7: "AG_ERR_ALIAS", 8: "AG_ERR_DEVICE",
+}
+
+
+class AgError(RuntimeError):
+    """A libag call returned a status other than AG_OK."""
+
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn}: {ag_status_string(status)} ({status})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with "
+            "`python long_context_genomics_b200/build.py` (or __graft_entry__.build())")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i64, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float
+    lib.ag_status_string.argtypes = [ctypes.c_int]
+    lib.ag_status_string.restype = ctypes.c_char_p
+    lib.ag_version.argtypes = []
+    lib.ag_version.restype = ctypes.c_int
+    lib.ag_pair_bias_project.argtypes = [vp, vp, vp, i64, i64, i64, vp]
+    lib.ag_pair_bias_project.restype = ctypes.c_int
+    lib.ag_attn_fwd.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, f32,
+                                vp, vp, vp]
+    lib.ag_attn_fwd.restype = ctypes.c_int
+    lib.ag_device_error.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int),
+                                    ctypes.c_int]
+    lib.ag_device_error.restype = ctypes.c_int
+    lib.ag_debug_wait_timeout.argtypes = [ctypes.c_uint64, vp]
+    lib.ag_debug_wait_timeout.restype = ctypes.c_int
+    return lib
+
+
+lib = _load()
+
+
+def ag_status_string(status: int) -> str:
+    return lib.ag_status_string(int(status)).decode()
+
+
+def ag_version() -> int:
+    return int(lib.ag_version())
+
+
+def _stream_ptr(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check(t: torch.Tensor, name: str, dtype, ndim: int):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be on a CUDA device")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def ag_pair_bias_project(pair: torch.Tensor, W: torch.Tensor,
+                         bias: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """bias[h,p,q] = sum_c pair[p,q,c] W[c,h] on the GPU (libag kernel)."""
+    _check(pair, "pair", torch.float32, 3)
+    _check(W, "W", torch.float32, 2)
+    P, P2, Cp = pair.shape
+    if P != P2 or W.shape[0] != Cp:
+        raise ValueError("pair must be [P,P,Cp] and W [Cp,H]")
+    H = W.shape[1]
+    if bias is None:
+        bias = torch.empty((H, P, P), dtype=torch.float32, device=pair.device)
+    _check(bias, "bias", torch.float32, 3)
+    if tuple(bias.shape) != (H, P, P):
+        raise ValueError("bias must be [H,P,P]")
+    st = lib.ag_pair_bias_project(pair.data_ptr(), W.data_ptr(), bias.data_ptr(),
+                                  P, Cp, H, _stream_ptr(stream))
+    if st != AG_OK:
+        raise AgError("ag_pair_bias_project", st)
+    return bias
+
+
+def ag_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                bias: torch.Tensor, cap: float = 5.0, block: int = 16,
+                out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                stream=None):
+    """Fused pair-bias MQA attention forward (libag kernel).
+
+    Returns (out [B,H,L,D] fp32, lse [B,H,L] fp32).  cap = math.inf turns the
+    soft cap off."""
+    _check(q, "q", torch.bfloat16, 4)
+    _check(k, "k", torch.bfloat16, 3)
+    _check(v, "v", torch.bfloat16, 3)
+    _check(bias, "bias", torch.float32, 3)
+    B, H, L, D = q.shape
+    if tuple(k.shape) != (B, L, D) or tuple(v.shape) != (B, L, D):
+        raise ValueError("k and v must be [B,L,D] with q [B,H,L,D]")
+    if out is None:
+        out = torch.empty((B, H, L, D), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H, L), dtype=torch.float32, device=q.device)
+    _check(out, "out", torch.float32, 4)
+    _check(lse, "lse", torch.float32, 3)
+    st = lib.ag_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), bias.data_ptr(),
+                         B, H, L, D, int(block), float(cap), out.data_ptr(),
+                         lse.data_ptr(), _stream_ptr(stream))
+    if st != AG_OK:
+        raise AgError("ag_attn_fwd", st)
+    return out, lse
+
+
+def ag_device_error(device: int = 0, clear: bool = True) -> int:
+    """Synchronise `device` and return (and optionally clear) its error word."""
+    code = ctypes.c_int(0)
+    st = lib.ag_device_error(int(device), ctypes.byref(code), 1 if clear else 0)
+    if st not in (AG_OK, 8):
+        raise AgError("ag_device_error", st)
+    return int(code.value)
+
+
+def ag_debug_wait_timeout(timeout_ns: int, stream=None) -> None:
+    """Launch the bounded-wait self-test kernel (see include/ag.h)."""
+    st = lib.ag_debug_wait_timeout(int(timeout_ns), _stream_ptr(stream))
+    if st != AG_OK:
+        raise AgError("ag_debug_wait_timeout", st)
+
+
+INF = math.inf

@@ -1,0 +1,605 @@
+// attn_fwd_sm100.cu -- fused pair-bias multi-query attention forward, sm_100a.
+//
+// Computes, for every batch item b, query head h and query position i
+// (page "Making Full-Context AlphaGenome Fit on an RTX 3090", section "Why
+// stock FlashAttention was not a drop-in replacement", Eq. L_ij):
+//   L_ij = cap * tanh((q_i . k_j / sqrt(D) + bias[h, i/16, j/16]) / cap)
+//   out_i = softmax_j(L_ij) V,  lse_i = log sum_j exp(L_ij)
+// one key tile at a time with the online softmax of section "Online softmax,
+// one block at a time"; no L x L tensor exists at any point.
+//
+// B200 design (not the page's 64 x 64 Pallas tiling, which targeted sm_86):
+//  * A query tile is 128 tensor-core rows = 16 consecutive positions x all 8
+//    heads.  Every row of the tile then shares one 16-position bias row block
+//    and all 8 heads consume the same K/V tile (multi-query sharing), so each
+//    K/V byte staged in shared memory feeds eight heads.
+//  * A persistent CTA per SM owns two such query tiles at a time (A and B).
+//    Warp 8 streams Q tiles and a ring of K and V tiles with TMA; warp 9
+//    issues every tcgen05.mma from one thread; warps 0-3 and 4-7 are the
+//    softmax warpgroups of tiles A and B.  The MMA order per key tile j is
+//    PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), so one warpgroup's softmax runs
+//    while the tensor core works for the other.
+//  * Tensor memory (512 columns): S_A, S_B (fp32 128x128 logits), O_A, O_B
+//    (fp32 128x128 accumulators).  P is written as bf16 over the first 64
+//    columns of its S and fed to the PV product straight from tensor memory.
+//  * Bias: each softmax thread owns one row, so per 128-key tile it needs
+//    just the 8 compact cells bias[h, I, 8j .. 8j+7], read from global (L2)
+//    one tile ahead and kept in registers; the 16x repeat is never built.
+//  * With a finite cap every logit lies in (-cap, cap), so the softmax uses
+//    the fixed shift m = cap (exact: softmax is shift invariant) and needs no
+//    running max and no rescaling of O.  cap > 40 (where exp(-2 cap) would
+//    underflow fp32) and cap = +inf use a running max with lazy rescaling.
+//  * Every wait is bounded (sm100.cuh); on timeout the kernel records the
+//    wait site in the device error word, drains its own copies and MMAs,
+//    frees tensor memory and returns.
+#include "ag_internal.h"
+#include "sm100.cuh"
+
+namespace ag {
+namespace attn {
+
+constexpr int kH = 8;
+constexpr int kD = 128;
+constexpr int kKeys = 128;                  // keys per K/V tile
+constexpr int kStages = 4;                  // K/V ring slots
+constexpr int kTileBytes = 128 * 128 * 2;   // one Q, K or V tile (bf16)
+constexpr int kHalfBytes = kTileBytes / 2;  // one 64-wide (128-byte) half
+constexpr int kNumWarps = 10;
+constexpr int kThreads = kNumWarps * 32;
+constexpr int kWarpLoad = 8;
+constexpr int kWarpMma = 9;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0);  // K-major B (K)
+constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, 1);  // MN-major B (V)
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+// Lazy rescale threshold (log2 units) for the running-max modes.
+constexpr float kRescaleThreshold = 8.0f;
+
+enum Mode { kStaticCap = 0, kOnlineCap = 1, kNoCap = 2 };
+
+// Wait sites recorded in the device error word.
+enum Site : unsigned {
+  kSiteProdQ = 1, kSiteProdKV = 2, kSiteMmaQ = 3, kSiteMmaKV = 4,
+  kSiteMmaP = 5, kSiteSoftS = 6, kSiteSoftO = 7, kSiteDrain = 8
+};
+
+struct __align__(8) Barriers {
+  uint64_t q_full[2], q_empty[2];
+  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t s_full[2], p_full[2], o_full[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+constexpr size_t kSmemBytes =
+    1024 + (2 + kStages) * static_cast<size_t>(kTileBytes) + sizeof(Barriers);
+
+struct Params {
+  const float *bias;
+  float *out;
+  float *lse;
+  unsigned *err;
+  int L, P;
+  int nb;          // 16-position query blocks per batch item (L / 16)
+  int pairs;       // work items per batch item: ceil(nb / 2)
+  int n_items;     // B * pairs
+  int n_kt;        // key tiles: ceil(L / 128)
+  int last_valid;  // valid keys in the last key tile (1..128)
+  float qk_scale;  // multiplies q.k
+  float bias_mul;  // multiplies the compact bias
+  float A;         // capped modes: cap * log2(e)
+};
+
+// --------------------------------------------------------------------------
+// MMA issue helpers (single thread).
+
+// S[128 x 128] = Q[128 x 128] K^T: eight K=16 steps over two 64-wide halves.
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_addr,
+                                         uint32_t k_addr) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+    umma_ss(d_tmem, smem_desc_sw128(q_addr + off, 16, 1024),
+            smem_desc_sw128(k_addr + off, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+  }
+}
+
+// O[128 x 128] (+)= P[128 x 128 keys] V[128 keys x 128]: P from tensor memory
+// (bf16 pairs, 8 columns per 16 keys), V MN-major in shared memory (the two
+// 64-wide halves are 16 KB apart, 8-key row groups 1 KB apart).
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem,
+                                         uint32_t v_addr, bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    umma_ts(d_tmem, p_tmem + kk * 8,
+            smem_desc_sw128(v_addr + kk * 2048, kHalfBytes, 1024), kIdescPV,
+            (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+// Bounded wait used while draining: ignores the abort flag, records nothing.
+__device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
+  const uint32_t a = smem_u32(bar);
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_test(a, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return;
+  }
+}
+
+// --------------------------------------------------------------------------
+// Warp 8, lane 0: TMA producer.
+__device__ __forceinline__ void producer(const CUtensorMap *tm_q,
+                                         const CUtensorMap *tm_k,
+                                         const CUtensorMap *tm_v, uint8_t *q_s,
+                                         uint8_t *kv_s, Barriers *bars,
+                                         const Params &p, volatile int *abort) {
+  const uint64_t pol_q = l2_policy_evict_first();
+  const uint64_t pol_kv = l2_policy_evict_last();
+  uint32_t qcount[2] = {0, 0};
+  uint32_t kv = 0;
+  bool ok = true;
+  for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x) {
+    const int b = w / p.pairs;
+    const int I0 = (w % p.pairs) * 2;
+    const int nX = (I0 + 1 < p.nb) ? 2 : 1;
+    for (int X = 0; X < nX; ++X) {
+      ok = mbar_wait(&bars->q_empty[X], (qcount[X] & 1u) ^ 1u, abort, p.err,
+                     kSiteProdQ);
+      if (!ok) break;
+      mbar_arrive_expect_tx(&bars->q_full[X], kTileBytes);
+      uint8_t *dst = q_s + X * kTileBytes;
+      tma_load_4d(dst, tm_q, &bars->q_full[X], 0, (I0 + X) * 16, 0, b, pol_q);
+      tma_load_4d(dst + kHalfBytes, tm_q, &bars->q_full[X], 64, (I0 + X) * 16,
+                  0, b, pol_q);
+      ++qcount[X];
+    }
+    for (int j = 0; j < p.n_kt && ok; ++j) {
+#pragma unroll 1
+      for (int t = 0; t < 2; ++t) {  // t = 0: K tile j, t = 1: V tile j
+        const uint32_t slot = kv % kStages, ph = (kv / kStages) & 1u;
+        ok = mbar_wait(&bars->kv_empty[slot], ph ^ 1u, abort, p.err, kSiteProdKV);
+        if (!ok) break;
+        mbar_arrive_expect_tx(&bars->kv_full[slot], kTileBytes);
+        uint8_t *dst = kv_s + slot * kTileBytes;
+        const CUtensorMap *tm = t == 0 ? tm_k : tm_v;
+        tma_load_3d(dst, tm, &bars->kv_full[slot], 0, j * kKeys, b, pol_kv);
+        tma_load_3d(dst + kHalfBytes, tm, &bars->kv_full[slot], 64, j * kKeys, b,
+                    pol_kv);
+        ++kv;
+      }
+    }
+  }
+  // Every copy this thread started must land before the CTA exits.
+  for (int X = 0; X < 2; ++X)
+    if (qcount[X] > 0) drain_wait(&bars->q_full[X], (qcount[X] - 1) & 1u);
+  const uint32_t first = kv > kStages ? kv - kStages : 0;
+  for (uint32_t i = first; i < kv; ++i)
+    drain_wait(&bars->kv_full[i % kStages], (i / kStages) & 1u);
+}
+
+// --------------------------------------------------------------------------
+// Warp 9, lane 0: tcgen05.mma issuer.
+__device__ __forceinline__ void mma_issuer(uint8_t *q_s, uint8_t *kv_s,
+                                           Barriers *bars, uint32_t tmem,
+                                           const Params &p, volatile int *abort) {
+  const uint32_t q_addr = smem_u32(q_s);
+  const uint32_t kv_addr = smem_u32(kv_s);
+  uint32_t qcount[2] = {0, 0}, pcount[2] = {0, 0};
+  uint32_t kv = 0;
+  bool ok = true;
+  for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x) {
+    const int I0 = (w % p.pairs) * 2;
+    const int nX = (I0 + 1 < p.nb) ? 2 : 1;
+    for (int X = 0; X < nX && ok; ++X) {
+      ok = mbar_wait(&bars->q_full[X], qcount[X] & 1u, abort, p.err, kSiteMmaQ);
+      ++qcount[X];
+    }
+    if (!ok) break;
+    // Key tile 0: S_X(0) for both query tiles.
+    const uint32_t slot_k0 = kv % kStages;
+    ok = mbar_wait(&bars->kv_full[slot_k0], (kv / kStages) & 1u, abort, p.err,
+                   kSiteMmaKV);
+    if (!ok) break;
+    ++kv;
+    tc_fence_after();
+    for (int X = 0; X < nX; ++X) {
+      issue_qk(tmem + X * 128, q_addr + X * kTileBytes,
+               kv_addr + slot_k0 * kTileBytes);
+      umma_commit(&bars->s_full[X]);
+      if (p.n_kt == 1) umma_commit(&bars->q_empty[X]);
+    }
+    umma_commit(&bars->kv_empty[slot_k0]);
+
+    for (int j = 0; j < p.n_kt && ok; ++j) {
+      const uint32_t slot_v = kv % kStages;
+      ok = mbar_wait(&bars->kv_full[slot_v], (kv / kStages) & 1u, abort, p.err,
+                     kSiteMmaKV);
+      if (!ok) break;
+      ++kv;
+      const bool has_next = j + 1 < p.n_kt;
+      uint32_t slot_k = 0;
+      bool k_ready = false;
+      for (int X = 0; X < nX; ++X) {
+        ok = mbar_wait(&bars->p_full[X], pcount[X] & 1u, abort, p.err, kSiteMmaP);
+        ++pcount[X];
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(tmem + 256 + X * 128, tmem + X * 128,
+                 kv_addr + slot_v * kTileBytes, j > 0);
+        if (!has_next) {
+          umma_commit(&bars->o_full[X]);
+          continue;
+        }
+        if (!k_ready) {
+          slot_k = kv % kStages;
+          ok = mbar_wait(&bars->kv_full[slot_k], (kv / kStages) & 1u, abort,
+                         p.err, kSiteMmaKV);
+          if (!ok) break;
+          ++kv;
+          k_ready = true;
+          tc_fence_after();
+        }
+        issue_qk(tmem + X * 128, q_addr + X * kTileBytes,
+                 kv_addr + slot_k * kTileBytes);
+        umma_commit(&bars->s_full[X]);
+        if (j + 2 == p.n_kt) umma_commit(&bars->q_empty[X]);
+      }
+      if (!ok) break;
+      umma_commit(&bars->kv_empty[slot_v]);
+      if (k_ready) umma_commit(&bars->kv_empty[slot_k]);
+    }
+  }
+  // All MMAs this thread issued complete before tensor memory is released.
+  umma_commit(&bars->drain);
+  drain_wait(&bars->drain, 0);
+}
+
+// --------------------------------------------------------------------------
+// Softmax warpgroups.
+
+__device__ __forceinline__ void load_bias8(const float *brow, int j, int P,
+                                           float (&bn)[8]) {
+  const int J0 = j * 8;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) bn[e] = (J0 + e < P) ? __ldg(brow + J0 + e) : 0.f;
+}
+
+// Static-shift softmax of one 32-column chunk: p = 2^(A tanh(y) - A) with
+// y = s * qk_scale + b / cap.  Returns the partial row sum; writes 16 bf16
+// pairs of P.
+__device__ __forceinline__ float chunk_static(const uint32_t (&s)[32], float b0,
+                                              float b1, float qk_scale, float A,
+                                              int col0, int nvalid,
+                                              uint32_t (&pk)[16]) {
+  float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const int c = 2 * e;
+    const float bb = c < 16 ? b0 : b1;
+    const float y0 = fmaf(__uint_as_float(s[c]), qk_scale, bb);
+    const float y1 = fmaf(__uint_as_float(s[c + 1]), qk_scale, bb);
+    float p0 = ex2_approx(fmaf(tanh_approx(y0), A, -A));
+    float p1 = ex2_approx(fmaf(tanh_approx(y1), A, -A));
+    if (col0 + c >= nvalid) p0 = 0.f;
+    if (col0 + c + 1 >= nvalid) p1 = 0.f;
+    acc0 += p0;
+    acc1 += p1;
+    pk[e] = pack_bf16x2(p0, p1);
+  }
+  return acc0 + acc1;
+}
+
+// Log2-domain logits of one chunk for the running-max modes.
+template <int MODE>
+__device__ __forceinline__ void chunk_logits(const uint32_t (&s)[32], float b0,
+                                             float b1, const Params &p, int col0,
+                                             int nvalid, float (&x)[32]) {
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    const float bb = c < 16 ? b0 : b1;
+    const float y = fmaf(__uint_as_float(s[c]), p.qk_scale, bb);
+    float v = (MODE == kOnlineCap) ? p.A * tanh_approx(y) : y;
+    x[c] = (col0 + c < nvalid) ? v : -INFINITY;
+  }
+}
+
+template <int MODE>
+__device__ __forceinline__ void softmax_role(int X, Barriers *bars, uint32_t tmem,
+                                             const Params &p,
+                                             volatile int *abort) {
+  const int r = threadIdx.x & 127;         // tile row == tensor-memory lane
+  const int wq = r >> 5;                   // warp's lane quarter
+  const int h = r >> 4, il = r & 15;       // head, position inside the block
+  const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+  const uint32_t tS = tmem + X * 128 + lane_base;
+  const uint32_t tO = tmem + 256 + X * 128 + lane_base;
+  uint32_t scount = 0, ocount = 0;
+
+  for (int w = blockIdx.x; w < p.n_items; w += gridDim.x) {
+    const int b = w / p.pairs;
+    const int I = (w % p.pairs) * 2 + X;
+    if (I >= p.nb) continue;  // odd block count: tile B idles on the last pair
+    const float *brow = p.bias + (static_cast<size_t>(h) * p.P + I) * p.P;
+    float m = (MODE == kStaticCap) ? p.A : -INFINITY;  // log2 units
+    float d = 0.f;
+    float bnext[8];
+    load_bias8(brow, 0, p.P, bnext);
+    bool ok = true;
+    for (int j = 0; j < p.n_kt; ++j) {
+      float bj[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) bj[e] = bnext[e] * p.bias_mul;
+      if (j + 1 < p.n_kt) load_bias8(brow, j + 1, p.P, bnext);
+      const int nvalid = (j + 1 == p.n_kt) ? p.last_valid : kKeys;
+
+      ok = mbar_wait(&bars->s_full[X], scount & 1u, abort, p.err, kSiteSoftS);
+      ++scount;
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      tc_fence_after();
+
+      if constexpr (MODE == kStaticCap) {
+        uint32_t sa[32], sb[32], pk[16];
+        float acc = 0.f;
+        tmem_ld32(tS + 0, sa);
+        tmem_wait_ld(sa);
+        tmem_ld32(tS + 32, sb);
+        acc += chunk_static(sa, bj[0], bj[1], p.qk_scale, p.A, 0, nvalid, pk);
+        tmem_st16(tS + 0, pk);
+        tmem_wait_ld(sb);
+        tmem_ld32(tS + 64, sa);
+        acc += chunk_static(sb, bj[2], bj[3], p.qk_scale, p.A, 32, nvalid, pk);
+        tmem_st16(tS + 16, pk);
+        tmem_wait_ld(sa);
+        tmem_ld32(tS + 96, sb);
+        acc += chunk_static(sa, bj[4], bj[5], p.qk_scale, p.A, 64, nvalid, pk);
+        tmem_st16(tS + 32, pk);
+        tmem_wait_ld(sb);
+        acc += chunk_static(sb, bj[6], bj[7], p.qk_scale, p.A, 96, nvalid, pk);
+        tmem_st16(tS + 48, pk);
+        d += acc;
+      } else {
+        // Pass 1: tile max of the log2-domain logits.
+        float mt = -INFINITY;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t s[32];
+          float x[32];
+          tmem_ld32(tS + c * 32, s);
+          tmem_wait_ld(s);
+          chunk_logits<MODE>(s, bj[2 * c], bj[2 * c + 1], p, c * 32, nvalid, x);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) mt = fmaxf(mt, x[e]);
+        }
+        // Lazy rescale: keep the old shift unless the max grew by more than
+        // the threshold (values up to 2^threshold are exact enough in fp32).
+        float factor = 1.f;
+        if (mt > m + kRescaleThreshold || m == -INFINITY) {
+          factor = (m == -INFINITY) ? 0.f : ex2_approx(m - mt);
+          m = mt;
+          d *= factor;
+        }
+        if (j > 0 && __any_sync(0xffffffffu, factor != 1.f)) {
+          // O_X(j-1) is complete: s_full(j) was committed after PV_X(j-1).
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + c * 32, o);
+            tmem_wait_ld(o);
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
+            tmem_st32(tO + c * 32, o);
+          }
+        }
+        // Pass 2: probabilities.
+        float acc = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t s[32], pk[16];
+          float x[32];
+          tmem_ld32(tS + c * 32, s);
+          tmem_wait_ld(s);
+          chunk_logits<MODE>(s, bj[2 * c], bj[2 * c + 1], p, c * 32, nvalid, x);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float p0 = ex2_approx(x[2 * e] - m);
+            const float p1 = ex2_approx(x[2 * e + 1] - m);
+            acc += p0 + p1;
+            pk[e] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(tS + c * 16, pk);
+        }
+        d += acc;
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars->p_full[X]);
+    }
+    if (!ok) break;
+
+    ok = mbar_wait(&bars->o_full[X], ocount & 1u, abort, p.err, kSiteSoftO);
+    ++ocount;
+    if (!__all_sync(0xffffffffu, ok)) break;
+    tc_fence_after();
+
+    // Epilogue: out = O / d (fp32, one 512-byte row per thread), lse.
+    const float inv_d = 1.f / d;
+    const size_t row = (static_cast<size_t>(b) * kH + h) * p.L +
+                       static_cast<size_t>(I) * 16 + il;
+    float4 *orow = reinterpret_cast<float4 *>(p.out + row * kD);
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      uint32_t o[32];
+      tmem_ld32(tO + c * 32, o);
+      tmem_wait_ld(o);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        orow[c * 8 + e] = make_float4(__uint_as_float(o[4 * e]) * inv_d,
+                                      __uint_as_float(o[4 * e + 1]) * inv_d,
+                                      __uint_as_float(o[4 * e + 2]) * inv_d,
+                                      __uint_as_float(o[4 * e + 3]) * inv_d);
+      }
+    }
+    p.lse[row] = (m + lg2_approx(d)) * kLn2;
+    tc_fence_before();
+  }
+}
+
+// --------------------------------------------------------------------------
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  uint8_t *q_s = smem_raw + pad;                 // 2 query tiles
+  uint8_t *kv_s = q_s + 2 * kTileBytes;          // K/V ring
+  Barriers *bars = reinterpret_cast<Barriers *>(kv_s + kStages * kTileBytes);
+  const int warp = threadIdx.x >> 5;
+
+  if (threadIdx.x == 0) {
+    for (int X = 0; X < 2; ++X) {
+      mbar_init(&bars->q_full[X], 1);
+      mbar_init(&bars->q_empty[X], 1);
+      mbar_init(&bars->s_full[X], 1);
+      mbar_init(&bars->p_full[X], 128);
+      mbar_init(&bars->o_full[X], 1);
+    }
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars->kv_full[s], 1);
+      mbar_init(&bars->kv_empty[s], 1);
+    }
+    mbar_init(&bars->drain, 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == kWarpLoad && lane_id() == 0) {
+    prefetch_tensormap(&tm_q);
+    prefetch_tensormap(&tm_k);
+    prefetch_tensormap(&tm_v);
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(&bars->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  volatile int *abort = &bars->abort;
+
+  if (warp == kWarpLoad) {
+    if (lane_id() == 0) producer(&tm_q, &tm_k, &tm_v, q_s, kv_s, bars, p, abort);
+  } else if (warp == kWarpMma) {
+    if (lane_id() == 0) mma_issuer(q_s, kv_s, bars, tmem, p, abort);
+  } else {
+    softmax_role<MODE>(warp >> 2, bars, tmem, p, abort);
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace attn
+
+// --------------------------------------------------------------------------
+// Host launcher.
+
+static bool encode_map(EncodeTiledFn enc, CUtensorMap *map, const void *base,
+                       int rank, const cuuint64_t *dims,
+                       const cuuint64_t *strides, const cuuint32_t *box) {
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank,
+                   const_cast<void *>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int MODE>
+static cudaError_t launch_mode(const CUtensorMap &tq, const CUtensorMap &tk,
+                               const CUtensorMap &tv, const attn::Params &p,
+                               int grid, cudaStream_t stream) {
+  static int configured[64] = {0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!configured[dev]) {
+    e = cudaFuncSetAttribute(attn::attn_fwd_kernel<MODE>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(attn::kSmemBytes));
+    if (e != cudaSuccess) return e;
+    configured[dev] = 1;
+  }
+  attn::attn_fwd_kernel<MODE>
+      <<<grid, attn::kThreads, attn::kSmemBytes, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_fwd(const AttnLaunch &a) {
+  using namespace attn;
+  const int64_t B = a.B, L = a.L;
+  CUtensorMap tq, tk, tv;
+  {
+    const cuuint64_t dims[4] = {kD, static_cast<cuuint64_t>(L), kH,
+                                static_cast<cuuint64_t>(B)};
+    const cuuint64_t strides[3] = {kD * 2, static_cast<cuuint64_t>(L) * kD * 2,
+                                   static_cast<cuuint64_t>(L) * kD * 2 * kH};
+    const cuuint32_t box[4] = {64, 16, kH, 1};
+    if (!encode_map(a.encode, &tq, a.q, 4, dims, strides, box))
+      return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[3] = {kD, static_cast<cuuint64_t>(L),
+                                static_cast<cuuint64_t>(B)};
+    const cuuint64_t strides[2] = {kD * 2, static_cast<cuuint64_t>(L) * kD * 2};
+    const cuuint32_t box[3] = {64, kKeys, 1};
+    if (!encode_map(a.encode, &tk, a.k, 3, dims, strides, box))
+      return cudaErrorInvalidValue;
+    if (!encode_map(a.encode, &tv, a.v, 3, dims, strides, box))
+      return cudaErrorInvalidValue;
+  }
+  Params p;
+  p.bias = a.bias;
+  p.out = a.out;
+  p.lse = a.lse;
+  p.err = a.err;
+  p.L = static_cast<int>(L);
+  p.P = static_cast<int>(L / 16);
+  p.nb = static_cast<int>(L / 16);
+  p.pairs = (p.nb + 1) / 2;
+  p.n_items = static_cast<int>(B) * p.pairs;
+  p.n_kt = static_cast<int>((L + kKeys - 1) / kKeys);
+  p.last_valid = static_cast<int>(L - static_cast<int64_t>(p.n_kt - 1) * kKeys);
+  const float cap = a.cap;
+  const float inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(kD));
+  int mode;
+  if (isinf(cap)) {
+    mode = kNoCap;
+    p.qk_scale = inv_sqrt_d * kLog2e;
+    p.bias_mul = kLog2e;
+    p.A = 0.f;
+  } else {
+    mode = cap <= 40.0f ? kStaticCap : kOnlineCap;
+    p.qk_scale = inv_sqrt_d / cap;
+    p.bias_mul = 1.0f / cap;
+    p.A = cap * kLog2e;
+  }
+  const int grid = p.n_items < a.num_sms ? p.n_items : a.num_sms;
+  switch (mode) {
+    case kStaticCap: return launch_mode<kStaticCap>(tq, tk, tv, p, grid, a.stream);
+    case kOnlineCap: return launch_mode<kOnlineCap>(tq, tk, tv, p, grid, a.stream);
+    default: return launch_mode<kNoCap>(tq, tk, tv, p, grid, a.stream);
+  }
+}
+
+}  // namespace ag

@@ -1,0 +1,97 @@
+"""The C ABI without a GPU: libag loads, exports every function that
+include/ag.h declares, and rejects bad arguments with the documented status
+before touching CUDA.  No call here reaches a kernel launch."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ag.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ag_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def ag():
+    import long_context_genomics_b200 as ag
+
+    return ag
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for required in ("ag_pair_bias_project", "ag_attn_fwd", "ag_status_string",
+                     "ag_device_error"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(ag):
+    lib = ctypes.CDLL(ag.LIB_PATH)
+    missing = [n for n in _declared_functions() if not hasattr(lib, n)]
+    assert not missing, f"declared in ag.h but not exported: {missing}"
+
+
+def test_status_strings(ag):
+    for code, name in ag.STATUS_NAMES.items():
+        assert ag.ag_status_string(code).startswith(name)
+    assert "unknown" in ag.ag_status_string(99)
+    assert ag.ag_version() >= 100
+
+
+# Fake, never-dereferenced device addresses: validation fails before CUDA.
+A16 = 0x10000
+BAD = 0x10004  # 4-byte aligned, not 16
+
+
+def _attn(ag, q=A16, k=A16 * 2, v=A16 * 3, bias=A16 * 4, B=1, H=8, L=256, D=128,
+          block=16, cap=5.0, out=A16 * 1000, lse=A16 * 2000):
+    return ag.lib.ag_attn_fwd(q, k, v, bias, B, H, L, D, block, cap, out, lse, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), 1), (dict(out=None), 1), (dict(lse=None), 1), (dict(bias=None), 1),
+    (dict(B=-1), 2), (dict(L=-16), 2), (dict(L=250), 2), (dict(D=0), 2),
+    (dict(H=4), 4), (dict(D=64), 4), (dict(block=8), 4), (dict(L=65536 + 16), 4),
+    (dict(B=1 << 20, L=65536), 4),
+    (dict(cap=0.0), 5), (dict(cap=-1.0), 5), (dict(cap=math.nan), 5),
+    (dict(q=BAD), 3), (dict(k=BAD), 3), (dict(out=BAD), 3),
+    (dict(out=A16), 7), (dict(lse=A16 * 4), 7),
+])
+def test_attn_validation(ag, kw, status):
+    assert _attn(ag, **kw) == status
+
+
+def test_attn_empty_is_a_noop(ag):
+    assert _attn(ag, B=0, q=None, k=None, v=None, bias=None, out=None, lse=None) == 0
+    assert _attn(ag, L=0, q=None, k=None, v=None, bias=None, out=None, lse=None) == 0
+
+
+@pytest.mark.parametrize("args,status", [
+    ((A16, A16 * 2, A16 * 3, -1, 128, 8), 2),
+    ((A16, A16 * 2, A16 * 3, 16, 0, 8), 2),
+    ((A16, A16 * 2, A16 * 3, 16, 64, 8), 4),
+    ((A16, A16 * 2, A16 * 3, 16, 128, 4), 4),
+    ((A16, A16 * 2, A16 * 3, 8192, 128, 8), 4),
+    ((None, A16 * 2, A16 * 3, 16, 128, 8), 1),
+    ((BAD, A16 * 2, A16 * 3, 16, 128, 8), 3),
+    ((A16, A16 * 2, A16 + 64, 16, 128, 8), 7),
+    ((0, 0, 0, 0, 128, 8), 0),
+])
+def test_projection_validation(ag, args, status):
+    assert ag.lib.ag_pair_bias_project(*args, None) == status
+
+
+def test_binding_rejects_cpu_tensors(ag):
+    import torch
+
+    q = torch.zeros(1, 8, 16, 128, dtype=torch.bfloat16)
+    k = torch.zeros(1, 16, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        ag.ag_attn_fwd(q, k, k, torch.zeros(8, 1, 1))

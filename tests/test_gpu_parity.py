@@ -1,0 +1,218 @@
+"""GPU parity: libag's kernels against the float64 oracle on the same seeded
+inputs (bf16 q/k/v and fp32 bias widened exactly).
+
+Tolerances (bf16 inputs, fp32 accumulation): max |out - oracle| <= 2e-2 and
+max |lse - oracle| <= 1e-3; projection: fp32 sums of 128 products,
+max |bias - oracle| <= 1e-4.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import ag_inputs
+
+pytestmark = pytest.mark.gpu
+
+OUT_TOL = 2e-2
+LSE_TOL = 1e-3
+PROJ_TOL = 1e-4
+
+
+@pytest.fixture(scope="module")
+def ag():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import long_context_genomics_b200 as ag
+
+    return ag
+
+
+def _dev(t):
+    return t.to("cuda").contiguous()
+
+
+def _gpu_attn(ag, inp, cap, bias=None, stream=None):
+    q, k, v = _dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"])
+    b = _dev(inp["bias"]) if bias is None else bias
+    out, lse = ag.ag_attn_fwd(q, k, v, b, cap=cap, stream=stream)
+    torch.cuda.synchronize()
+    assert ag.ag_device_error(0) == 0
+    return out.double().cpu().numpy(), lse.double().cpu().numpy()
+
+
+def _compare(out, lse, ref_out, ref_lse, what):
+    assert np.isfinite(out).all() and np.isfinite(lse).all(), f"{what}: non-finite"
+    eo = float(np.max(np.abs(out - ref_out))) if out.size else 0.0
+    el = float(np.max(np.abs(lse - ref_lse))) if lse.size else 0.0
+    print(f"{what}: max|dout|={eo:.3e} max|dlse|={el:.3e}")
+    assert eo <= OUT_TOL, f"{what}: max|dout| {eo:.3e} > {OUT_TOL}"
+    assert el <= LSE_TOL, f"{what}: max|dlse| {el:.3e} > {LSE_TOL}"
+    return eo, el
+
+
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("P", [1, 3, 5, 32, 128, 512])
+def test_projection_parity(ag, oracle_lib, P):
+    g = torch.Generator().manual_seed(100 + P)
+    pair = torch.randn(P, P, 128, generator=g)
+    W = torch.randn(128, 8, generator=g) / math.sqrt(128)
+    bias = ag.ag_pair_bias_project(_dev(pair), _dev(W))
+    torch.cuda.synchronize()
+    ref = oracle_lib.pair_bias_project(pair, W)
+    err = float(np.max(np.abs(bias.double().cpu().numpy() - ref)))
+    print(f"projection P={P}: max|d|={err:.3e}")
+    assert err <= PROJ_TOL
+
+
+@pytest.mark.parametrize("name", ["tiny", "short", "mid"])
+def test_config_parity_full(ag, oracle_lib, name):
+    w = ag_inputs.WORKLOADS[name]
+    inp = ag_inputs.make_inputs(w)
+    out, lse = _gpu_attn(ag, inp, w.cap)
+    ref_out, ref_lse = oracle_lib.attn_fwd(inp["q"], inp["k"], inp["v"], inp["bias"],
+                                           block=16, cap=w.cap)
+    eo, _ = _compare(out, lse, ref_out, ref_lse, name)
+    if name == "tiny":
+        # For context: the page's standalone L=512 tiled-vs-dense figure was
+        # 2^-9 max abs error (a different pair of bf16 paths, not a bound).
+        print(f"tiny max|dout| {eo:.3e} vs page figure 1.953e-03")
+
+
+def test_full_context_with_projection_sampled(ag, oracle_lib):
+    """L = 8192 with the projected pair bias, exactly as the benchmark runs it;
+    2048 sampled rows against the oracle, every row checked for finiteness."""
+    w = ag_inputs.WORKLOADS["full"]
+    inp = ag_inputs.make_inputs(w)
+    bias = ag.ag_pair_bias_project(_dev(inp["pair"]), _dev(inp["W"]))
+    out, lse = _gpu_attn(ag, inp, w.cap, bias=bias)
+    ref_bias = oracle_lib.pair_bias_project(inp["pair"], inp["W"])
+    assert float(np.max(np.abs(bias.double().cpu().numpy() - ref_bias))) <= PROJ_TOL
+    rows = ag_inputs.sample_rows(w.B, w.H, w.L, 2048, seed=7).numpy()
+    # The oracle uses its own projected bias: the two paths share nothing.
+    ro, rl = oracle_lib.attn_rows(inp["q"], inp["k"], inp["v"], ref_bias, rows,
+                                  block=16, cap=w.cap)
+    b, h, i = rows[:, 0], rows[:, 1], rows[:, 2]
+    _compare(out[b, h, i], lse[b, h, i], ro, rl, "full L=8192 sampled")
+    assert np.isfinite(out).all() and np.isfinite(lse).all()
+    assert (lse <= w.cap + math.log(w.L) + 1e-3).all()
+
+
+def test_nine_block_stack_sampled(ag, oracle_lib):
+    for layer in ag_inputs.nine_block_stack().layers:
+        inp = ag_inputs.make_inputs(layer)
+        bias = ag.ag_pair_bias_project(_dev(inp["pair"]), _dev(inp["W"]))
+        out, lse = _gpu_attn(ag, inp, layer.cap, bias=bias)
+        ref_bias = oracle_lib.pair_bias_project(inp["pair"], inp["W"])
+        rows = ag_inputs.sample_rows(layer.B, layer.H, layer.L, 192,
+                                     seed=layer.seed).numpy()
+        ro, rl = oracle_lib.attn_rows(inp["q"], inp["k"], inp["v"], ref_bias, rows,
+                                      block=16, cap=layer.cap)
+        b, h, i = rows[:, 0], rows[:, 1], rows[:, 2]
+        _compare(out[b, h, i], lse[b, h, i], ro, rl,
+                 f"{layer.name} cap={layer.cap}")
+
+
+@pytest.mark.parametrize("B,L", [(1, 16), (2, 48), (1, 128), (1, 144), (3, 400),
+                                 (1, 1040), (2, 2064)])
+@pytest.mark.parametrize("cap", [5.0, math.inf])
+def test_ragged_and_odd_shapes(ag, oracle_lib, B, L, cap):
+    """L not a multiple of the 128-key tile (masked tail) and odd numbers of
+    16-position blocks (the last pair of a batch item has one tile)."""
+    inp = ag_inputs.random_case(B, 8, L, 128, 128, 16, seed=B * 1000 + L)
+    out, lse = _gpu_attn(ag, inp, cap)
+    ro, rl = oracle_lib.attn_fwd(inp["q"], inp["k"], inp["v"], inp["bias"],
+                                 block=16, cap=cap)
+    _compare(out, lse, ro, rl, f"B={B} L={L} cap={cap}")
+
+
+@pytest.mark.parametrize("cap", [1.0, 5.0, 10.0, 30.0, 40.0, 50.0, 1e4, math.inf])
+def test_cap_modes(ag, oracle_lib, cap):
+    """Static shift (cap <= 40), running max with the cap (cap > 40) and no
+    cap at all."""
+    inp = ag_inputs.random_case(2, 8, 512, 128, 128, 16, seed=int(min(cap, 1e6)) + 3)
+    out, lse = _gpu_attn(ag, inp, cap)
+    ro, rl = oracle_lib.attn_fwd(inp["q"], inp["k"], inp["v"], inp["bias"],
+                                 block=16, cap=cap)
+    _compare(out, lse, ro, rl, f"cap={cap}")
+
+
+@pytest.mark.parametrize("cap", [5.0, 30.0, math.inf])
+def test_large_logits(ag, oracle_lib, cap):
+    """q, k with std 3 and a bias of std 4: logits far beyond the cap
+    (saturated tanh) and, without a cap, a wide softmax range."""
+    inp = ag_inputs.random_case(1, 8, 640, 128, 128, 16, seed=77, bias_std=4.0,
+                                qk_std=3.0)
+    out, lse = _gpu_attn(ag, inp, cap)
+    ro, rl = oracle_lib.attn_fwd(inp["q"], inp["k"], inp["v"], inp["bias"],
+                                 block=16, cap=cap)
+    _compare(out, lse, ro, rl, f"large logits cap={cap}")
+
+
+def test_maximum_length_sampled(ag, oracle_lib):
+    inp = ag_inputs.random_case(1, 8, 65536, 128, 128, 16, seed=5)
+    out, lse = _gpu_attn(ag, inp, 5.0)
+    rows = ag_inputs.sample_rows(1, 8, 65536, 48, seed=3).numpy()
+    ro, rl = oracle_lib.attn_rows(inp["q"], inp["k"], inp["v"], inp["bias"], rows,
+                                  block=16, cap=5.0)
+    b, h, i = rows[:, 0], rows[:, 1], rows[:, 2]
+    _compare(out[b, h, i], lse[b, h, i], ro, rl, "L=65536 sampled")
+
+
+def test_empty_inputs_are_noops(ag):
+    q = torch.empty(0, 8, 64, 128, dtype=torch.bfloat16, device="cuda")
+    k = torch.empty(0, 64, 128, dtype=torch.bfloat16, device="cuda")
+    bias = torch.zeros(8, 4, 4, device="cuda")
+    out, lse = ag.ag_attn_fwd(q, k, k, bias)
+    assert out.shape == (0, 8, 64, 128) and lse.shape == (0, 8, 64)
+    q0 = torch.empty(1, 8, 0, 128, dtype=torch.bfloat16, device="cuda")
+    k0 = torch.empty(1, 0, 128, dtype=torch.bfloat16, device="cuda")
+    ag.ag_attn_fwd(q0, k0, k0, torch.zeros(8, 0, 0, device="cuda"))
+    pair = torch.empty(0, 0, 128, device="cuda")
+    assert ag.ag_pair_bias_project(pair, torch.zeros(128, 8, device="cuda")).numel() == 0
+    torch.cuda.synchronize()
+    assert ag.ag_device_error(0) == 0
+
+
+def test_deterministic_and_stream(ag):
+    inp = ag_inputs.make_inputs(ag_inputs.WORKLOADS["short"])
+    o1, l1 = _gpu_attn(ag, inp, 5.0)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        o2, l2 = _gpu_attn(ag, inp, 5.0, stream=s)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def test_no_quadratic_memory(ag):
+    """The call allocates nothing: peak device memory during it stays at the
+    inputs plus outputs (no L x L logits, no expanded bias)."""
+    w = ag_inputs.WORKLOADS["full"]
+    inp = ag_inputs.make_inputs(w)
+    q, k, v = _dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"])
+    bias = ag.ag_pair_bias_project(_dev(inp["pair"]), _dev(inp["W"]))
+    out = torch.empty(1, 8, w.L, 128, device="cuda")
+    lse = torch.empty(1, 8, w.L, device="cuda")
+    torch.cuda.synchronize()
+    torch.cuda.reset_peak_memory_stats()
+    base = torch.cuda.memory_allocated()
+    ag.ag_attn_fwd(q, k, v, bias, cap=5.0, out=out, lse=lse)
+    torch.cuda.synchronize()
+    assert torch.cuda.max_memory_allocated() == base
+    free, total = torch.cuda.mem_get_info()
+    assert free > 0 and total > 0
+
+
+def test_bounded_wait_reports_and_context_survives(ag, oracle_lib):
+    """A wait that nothing completes runs out after its limit, records
+    (site 255 << 8) | 1 in the error word, and the context stays usable."""
+    assert ag.ag_device_error(0) == 0
+    ag.ag_debug_wait_timeout(20_000_000)
+    code = ag.ag_device_error(0, clear=True)
+    assert code == (255 << 8) | 1
+    assert ag.ag_device_error(0) == 0
+    inp = ag_inputs.random_case(1, 8, 256, 128, 128, 16, seed=9)
+    out, lse = _gpu_attn(ag, inp, 5.0)
+    ro, rl = oracle_lib.attn_fwd(inp["q"], inp["k"], inp["v"], inp["bias"],
+                                 block=16, cap=5.0)
+    _compare(out, lse, ro, rl, "after timeout")
