@@ -1,0 +1,375 @@
+#!/usr/bin/env python
+"""Benchmark of the pair-bias multi-query attention hot path on B200.
+
+One step = the whole path on one batch: ag_pair_bias_project (pair [512,512,128]
+-> bias [8,512,512]) followed by ag_attn_fwd at full context (L = 8192, B = 1,
+8 query heads sharing one K/V head, D = 128, 16x16 bias cells, cap 5).
+The metric counts the attention's 4*B*H*L^2*D tensor FLOPs per step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torchrun, one process per GPU; each rank runs its own
+independent problem (weak scaling, no collective on the data path) and rank 0
+prints one JSON line with the time taken as the maximum over ranks.
+--impl reference times the float64 CPU oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import datetime
+import glob
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import ag_inputs  # noqa: E402
+
+METRIC = "fused pair-bias attention TFLOP/s at L=8192, % of B200 BF16 peak"
+UNIT = "TFLOP/s"
+WORKLOAD = ag_inputs.WORKLOADS["full"]
+FALLBACK_PEAK_TFLOPS = 1590.0
+FLUSH_BYTES = 256 << 20
+KERNEL_SOURCES = ["long_context_genomics_b200/csrc/attn_fwd_sm100.cu",
+                  "long_context_genomics_b200/csrc/sm100.cuh"]
+
+
+def workload_config(w) -> dict:
+    return {
+        "workload": f"full_context_L{w.L}_B{w.B}_projected_pair_bias",
+        "B": w.B, "L": w.L, "H": w.H, "D": w.D, "Dv": w.Dv, "P": w.P, "Cp": w.Cp,
+        "block": w.block, "cap": w.cap, "seed": w.seed,
+        "step": "ag_pair_bias_project + ag_attn_fwd",
+        "l2": "flushed between timed steps (256 MiB write)",
+    }
+
+
+def peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            m = json.load(f)
+        return {"bf16_tflops": float(m["bf16_tflops"]), "hbm_gbs": float(m["hbm_gbs"]),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"bf16_tflops": FALLBACK_PEAK_TFLOPS, "hbm_gbs": 6650.0,
+                "source": "fallback"}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per attention launch from the committed ncu summary, if it
+    was taken on the current kernel source (else None)."""
+    want = kernel_source_hash()
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        fields = {}
+        with open(path) as f:
+            for line in f:
+                if ":" in line and line.strip().startswith(("traffic_bytes_per_launch",
+                                                             "kernel_source_sha256")):
+                    k, v = line.split(":", 1)
+                    fields[k.strip(" -*`")] = v.strip(" `\n")
+        if fields.get("kernel_source_sha256") == want and "traffic_bytes_per_launch" in fields:
+            try:
+                return float(fields["traffic_bytes_per_launch"])
+            except ValueError:
+                return None
+    return None
+
+
+# --------------------------------------------------------------------------
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        self.path = None
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "20", "-i", uuid],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, RuntimeError, AttributeError):
+            self.proc = None
+
+    def stop(self, t0: float, t1: float) -> dict | None:
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) != 8:
+                    continue
+                try:
+                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                    rows.append((ts, float(parts[1]), float(parts[2]), parts[4:]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        inside = [r for r in rows if t0 - 0.05 <= r[0] <= t1 + 0.05] or rows[-5:]
+        if not inside:
+            return None
+        reasons = sorted({name for r in inside for name, v in zip(self.REASONS, r[3])
+                          if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[1] for r in inside),
+                "sm_max_mhz": max(r[2] for r in inside), "reasons": reasons,
+                "samples": len(inside)}
+
+
+# --------------------------------------------------------------------------
+def cpu_baseline(w, target_s: float = 12.0, seed: int = 11) -> dict:
+    """The float64 oracle, as it stands, on a bounded sample of the workload:
+    randomly chosen query rows (all over the batch and heads) against the full
+    key range.  The bias comes from the oracle's own projection (untimed)."""
+    import oracle
+
+    orc = oracle.default()
+    cores = orc.threads(len(os.sched_getaffinity(0)))
+    inp = ag_inputs.make_inputs(w)
+    bias = orc.pair_bias_project(inp["pair"], inp["W"])
+    flops_row = 2.0 * w.L * (w.D + w.Dv)
+
+    def run(n, s):
+        rows = ag_inputs.sample_rows(w.B, w.H, w.L, n, seed=s).numpy()
+        t = time.perf_counter()
+        orc.attn_rows(inp["q"], inp["k"], inp["v"], bias, rows, block=w.block, cap=w.cap)
+        return len(rows), time.perf_counter() - t
+
+    n0, t0 = run(max(4 * cores, 16), seed)
+    n = int(min(w.B * w.H * w.L, max(n0, n0 * target_s / max(t0, 1e-6))))
+    n, t = run(n, seed + 1)
+    return {"value": n * flops_row / t / 1e12, "unit": UNIT, "cores": cores,
+            "kind": "oracle",
+            "sample": f"{n} random query rows of {w.B * w.H * w.L} (b,h,i) at L={w.L}, "
+                      f"full key range, float64, {t:.1f} s; projection untimed"}
+
+
+def run_reference(args, rank: int, world: int) -> None:
+    """The oracle on the host cores: each step is a bounded row sample."""
+    if rank != 0:
+        return
+    import oracle
+
+    w = WORKLOAD
+    orc = oracle.default()
+    cores = orc.threads(len(os.sched_getaffinity(0)))
+    inp = ag_inputs.make_inputs(w)
+    bias = orc.pair_bias_project(inp["pair"], inp["W"])
+    flops_row = 2.0 * w.L * (w.D + w.Dv)
+    per_step_s = min(4.0, 150.0 / max(1, args.steps + args.warmup))
+    rows = ag_inputs.sample_rows(w.B, w.H, w.L, max(4 * cores, 16), seed=0).numpy()
+    t = time.perf_counter()
+    orc.attn_rows(inp["q"], inp["k"], inp["v"], bias, rows, block=w.block, cap=w.cap)
+    n = int(max(len(rows), len(rows) * per_step_s / max(time.perf_counter() - t, 1e-6)))
+    times = []
+    for s in range(args.warmup + args.steps):
+        rows = ag_inputs.sample_rows(w.B, w.H, w.L, n, seed=100 + s).numpy()
+        t = time.perf_counter()
+        orc.attn_rows(inp["q"], inp["k"], inp["v"], bias, rows, block=w.block, cap=w.cap)
+        if s >= args.warmup:
+            times.append(time.perf_counter() - t)
+    total = sum(times)
+    value = len(rows) * flops_row * len(times) / total / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / len(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{len(rows)} random query rows per step at L={w.L}, "
+                                   "full key range, float64"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------
+def run_ours(args, rank: int, world: int, local_rank: int) -> None:
+    import long_context_genomics_b200 as ag
+
+    dist = torch.distributed
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    base = WORKLOAD
+    # Each rank runs its own independent problem (own seed).
+    w = dataclasses.replace(base, seed=base.seed + 1000 * rank)
+    host = ag_inputs.make_inputs(w)
+    pinned = {n: t.pin_memory() for n, t in host.items()}
+    d = {n: t.to(dev) for n, t in host.items()}
+    bias = torch.empty(w.H, w.P, w.P, device=dev)
+    out = torch.empty(w.B, w.H, w.L, w.Dv, device=dev)
+    lse = torch.empty(w.B, w.H, w.L, device=dev)
+    out_h = torch.empty(out.shape, pin_memory=True)
+    lse_h = torch.empty(lse.shape, pin_memory=True)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ag.ag_pair_bias_project(d["pair"], d["W"], bias=bias)
+        ag.ag_attn_fwd(d["q"], d["k"], d["v"], bias, cap=w.cap, out=out, lse=lse)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert ag.ag_device_error(local_rank) == 0
+
+    # ---- device-resident timing --------------------------------------------
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    time.sleep(0.3 if sampler else 0.0)
+    barrier()
+    t_wall0 = time.time()
+    for i in range(K):
+        flush.zero_()                      # untimed: outside the events
+        ev[i][0].record(stream)
+        ag.ag_pair_bias_project(d["pair"], d["W"], bias=bias)
+        ev[i][1].record(stream)
+        ag.ag_attn_fwd(d["q"], d["k"], d["v"], bias, cap=w.cap, out=out, lse=lse)
+        ev[i][2].record(stream)
+    barrier()
+    t_wall1 = time.time()
+    clocks = sampler.stop(t_wall0, t_wall1) if sampler else None
+    step_ms = [e[0].elapsed_time(e[2]) for e in ev]
+    proj_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    total_ms = torch.tensor([sum(step_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(total_ms, op=dist.ReduceOp.MAX)
+    total_s = float(total_ms.item()) / 1e3
+    assert ag.ag_device_error(local_rank) == 0
+
+    # ---- end to end through the public API with host buffers ---------------
+    h2d = sum(pinned[n].numel() * pinned[n].element_size() for n in ("q", "k", "v", "pair", "W"))
+    d2h = out_h.numel() * 4 + lse_h.numel() * 4
+    ee = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    barrier()
+    for i in range(K):
+        flush.zero_()
+        ee[i][0].record(stream)
+        for n in ("q", "k", "v", "pair", "W"):
+            d[n].copy_(pinned[n], non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+        ee[i][1].record(stream)
+    barrier()
+    e2e_ms = torch.tensor([sum(e[0].elapsed_time(e[1]) for e in ee)], dtype=torch.float64,
+                          device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_s = float(e2e_ms.item()) / 1e3
+    assert math.isfinite(float(lse_h[0, 0, 0])) and ag.ag_device_error(local_rank) == 0
+
+    if rank != 0:
+        return
+    flops = w.attn_flops()
+    pk = peaks()
+    value = world * flops * K / total_s / 1e12
+    attn_mean_s = statistics.mean(attn_ms) / 1e3
+    achieved = flops / attn_mean_s / 1e12
+    proj_mean_s = statistics.mean(proj_ms) / 1e3
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": 1e3 * total_s / K,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {**workload_config(w), "parallelism": f"{world} independent replicas"
+                   if world > 1 else "single GPU"},
+        "pct_of_peak": 100.0 * (value / world) / pk["bf16_tflops"],
+        "peak_source": pk["source"],
+        "e2e": {"value": world * flops * K / e2e_s / 1e12, "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 2 * K,
+        "roofline": {"kernel": "attn_fwd_kernel", "bound": "tensor", "achieved": achieved,
+                     "peak": pk["bf16_tflops"], "unit": UNIT,
+                     "frac": achieved / pk["bf16_tflops"], "traffic": profiled_traffic(),
+                     "peak_kind": "bf16 burst (" + pk["source"] + ")"},
+        "attn_ms": {"median": statistics.median(attn_ms),
+                    "p95": sorted(attn_ms)[int(0.95 * (K - 1))]},
+        "projection": {"ms_median": statistics.median(proj_ms),
+                       "achieved_gbs": w.project_bytes() / proj_mean_s / 1e9,
+                       "peak_gbs": pk["hbm_gbs"],
+                       "frac": w.project_bytes() / proj_mean_s / 1e9 / pk["hbm_gbs"]},
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    print(json.dumps(line), flush=True)
+
+
+def main() -> None:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        if world == 1 and args.gpus > 1:
+            sys.exit("--gpus N > 1 must be launched with torchrun (one process per GPU)")
+    if args.impl == "reference":
+        # Rank 0 alone times the oracle; the other ranks exit without work.
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group(
+            backend="nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
