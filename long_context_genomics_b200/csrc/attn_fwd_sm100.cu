@@ -44,10 +44,22 @@ constexpr int kKeys = 128;                  // keys per K/V tile
 constexpr int kStages = 4;                  // K/V ring slots
 constexpr int kTileBytes = 128 * 128 * 2;   // one Q, K or V tile (bf16)
 constexpr int kHalfBytes = kTileBytes / 2;  // one 64-wide (128-byte) half
-constexpr int kNumWarps = 10;
+// Warps 0-7: two softmax warpgroups; warpgroup 2 = warp 8 (TMA producer),
+// warp 9 (MMA issuer) and warps 10-11 (idle, present so that warpgroup 2 is
+// whole for the register re-allocation).
+constexpr int kNumWarps = 12;
 constexpr int kThreads = kNumWarps * 32;
 constexpr int kWarpLoad = 8;
 constexpr int kWarpMma = 9;
+// Registers per thread: the launch gives every thread kRegsLaunch (the cap
+// for 384 threads, which ptxas allocates when setmaxnreg is present); the
+// producer warpgroup drops to kRegsLow and the softmax warpgroups rise to
+// kRegsHigh.  Budget: 2*128*kRegsHigh + 128*kRegsLow <= 384*kRegsLaunch.
+constexpr uint32_t kRegsLaunch = 168;
+constexpr uint32_t kRegsLow = 88;
+constexpr uint32_t kRegsHigh = 208;
+static_assert(2 * 128 * kRegsHigh + 128 * kRegsLow <= kThreads * kRegsLaunch,
+              "register split exceeds the launch allocation");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0);  // K-major B (K)
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, 1);  // MN-major B (V)
@@ -266,29 +278,72 @@ __device__ __forceinline__ void load_bias8(const float *brow, int j, int P,
   for (int e = 0; e < 8; ++e) bn[e] = (J0 + e < P) ? __ldg(brow + J0 + e) : 0.f;
 }
 
+// Column pairs (out of every 8) whose exponential runs on the FMA pipe
+// (exp2_poly2) instead of the special-function unit.  The SFU still computes
+// every tanh, so it does 1 + (8 - kEmuPairs) / 8 operations per logit.
+#ifndef AG_EXP2_EMU_PAIRS
+#define AG_EXP2_EMU_PAIRS 6
+#endif
+constexpr int kEmuPairs = AG_EXP2_EMU_PAIRS;
+
 // Static-shift softmax of one 32-column chunk: p = 2^(A tanh(y) - A) with
-// y = s * qk_scale + b / cap.  Returns the partial row sum; writes 16 bf16
-// pairs of P.
-__device__ __forceinline__ float chunk_static(const uint32_t (&s)[32], float b0,
-                                              float b1, float qk_scale, float A,
-                                              int col0, int nvalid,
-                                              uint32_t (&pk)[16]) {
-  float acc0 = 0.f, acc1 = 0.f;
+// y = s * qk_scale + b / cap, two columns at a time.  Adds the row sum into
+// acc and writes 16 bf16 pairs of P.  kMask zeroes columns >= nvalid (only
+// the last key tile of a ragged length needs it).
+template <bool kMask>
+__device__ __forceinline__ void chunk_static(const uint32_t (&s)[32], float b0,
+                                             float b1, float2 sc, float2 ap,
+                                             float2 an, int col0, int nvalid,
+                                             float2 &acc, uint32_t (&pk)[16]) {
 #pragma unroll
   for (int e = 0; e < 16; ++e) {
-    const int c = 2 * e;
-    const float bb = c < 16 ? b0 : b1;
-    const float y0 = fmaf(__uint_as_float(s[c]), qk_scale, bb);
-    const float y1 = fmaf(__uint_as_float(s[c + 1]), qk_scale, bb);
-    float p0 = ex2_approx(fmaf(tanh_approx(y0), A, -A));
-    float p1 = ex2_approx(fmaf(tanh_approx(y1), A, -A));
-    if (col0 + c >= nvalid) p0 = 0.f;
-    if (col0 + c + 1 >= nvalid) p1 = 0.f;
-    acc0 += p0;
-    acc1 += p1;
-    pk[e] = pack_bf16x2(p0, p1);
+    const float bb = e < 8 ? b0 : b1;
+    const float2 y = __ffma2_rn(
+        make_float2(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1])), sc,
+        make_float2(bb, bb));
+    const float2 t = make_float2(tanh_approx(y.x), tanh_approx(y.y));
+    const float2 x = __ffma2_rn(t, ap, an);
+    float2 p;
+    if ((e & 7) < kEmuPairs) {
+      p = exp2_poly2(x);
+    } else {
+      p = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+    }
+    if (kMask) {
+      if (col0 + 2 * e >= nvalid) p.x = 0.f;
+      if (col0 + 2 * e + 1 >= nvalid) p.y = 0.f;
+    }
+    acc = __fadd2_rn(acc, p);
+    pk[e] = pack_bf16x2(p.x, p.y);
   }
-  return acc0 + acc1;
+}
+
+// One 128-key tile of the static-shift softmax: S from tensor memory in four
+// 32-column chunks (the next chunk's load overlaps this chunk's math), P back
+// over the first 64 columns.  Returns the tile's row sum.
+template <bool kMask>
+__device__ __forceinline__ float tile_static(uint32_t tS, const float (&bj)[8],
+                                             float2 sc, float2 ap, float2 an,
+                                             int nvalid) {
+  uint32_t sa[32], sb[32], pk[16];
+  float2 acc = make_float2(0.f, 0.f);
+  tmem_ld32(tS + 0, sa);
+  tmem_wait_ld(sa);
+  tmem_ld32(tS + 32, sb);
+  chunk_static<kMask>(sa, bj[0], bj[1], sc, ap, an, 0, nvalid, acc, pk);
+  tmem_st16(tS + 0, pk);
+  tmem_wait_ld(sb);
+  tmem_ld32(tS + 64, sa);
+  chunk_static<kMask>(sb, bj[2], bj[3], sc, ap, an, 32, nvalid, acc, pk);
+  tmem_st16(tS + 16, pk);
+  tmem_wait_ld(sa);
+  tmem_ld32(tS + 96, sb);
+  chunk_static<kMask>(sa, bj[4], bj[5], sc, ap, an, 64, nvalid, acc, pk);
+  tmem_st16(tS + 32, pk);
+  tmem_wait_ld(sb);
+  chunk_static<kMask>(sb, bj[6], bj[7], sc, ap, an, 96, nvalid, acc, pk);
+  tmem_st16(tS + 48, pk);
+  return acc.x + acc.y;
 }
 
 // Log2-domain logits of one chunk for the running-max modes.
@@ -340,25 +395,12 @@ __device__ __forceinline__ void softmax_role(int X, Barriers *bars, uint32_t tme
       tc_fence_after();
 
       if constexpr (MODE == kStaticCap) {
-        uint32_t sa[32], sb[32], pk[16];
-        float acc = 0.f;
-        tmem_ld32(tS + 0, sa);
-        tmem_wait_ld(sa);
-        tmem_ld32(tS + 32, sb);
-        acc += chunk_static(sa, bj[0], bj[1], p.qk_scale, p.A, 0, nvalid, pk);
-        tmem_st16(tS + 0, pk);
-        tmem_wait_ld(sb);
-        tmem_ld32(tS + 64, sa);
-        acc += chunk_static(sb, bj[2], bj[3], p.qk_scale, p.A, 32, nvalid, pk);
-        tmem_st16(tS + 16, pk);
-        tmem_wait_ld(sa);
-        tmem_ld32(tS + 96, sb);
-        acc += chunk_static(sa, bj[4], bj[5], p.qk_scale, p.A, 64, nvalid, pk);
-        tmem_st16(tS + 32, pk);
-        tmem_wait_ld(sb);
-        acc += chunk_static(sb, bj[6], bj[7], p.qk_scale, p.A, 96, nvalid, pk);
-        tmem_st16(tS + 48, pk);
-        d += acc;
+        const float2 sc = make_float2(p.qk_scale, p.qk_scale);
+        const float2 ap = make_float2(p.A, p.A), an = make_float2(-p.A, -p.A);
+        if (nvalid == kKeys)
+          d += tile_static<false>(tS, bj, sc, ap, an, nvalid);
+        else
+          d += tile_static<true>(tS, bj, sc, ap, an, nvalid);
       } else {
         // Pass 1: tile max of the log2-domain logits.
         float mt = -INFINITY;
@@ -491,11 +533,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = bars->tmem_base;
   volatile int *abort = &bars->abort;
 
-  if (warp == kWarpLoad) {
-    if (lane_id() == 0) producer(&tm_q, &tm_k, &tm_v, q_s, kv_s, bars, p, abort);
-  } else if (warp == kWarpMma) {
-    if (lane_id() == 0) mma_issuer(q_s, kv_s, bars, tmem, p, abort);
+  if (warp >= kWarpLoad) {
+    regs_dec<kRegsLow>();
+    if (warp == kWarpLoad && lane_id() == 0)
+      producer(&tm_q, &tm_k, &tm_v, q_s, kv_s, bars, p, abort);
+    else if (warp == kWarpMma && lane_id() == 0)
+      mma_issuer(q_s, kv_s, bars, tmem, p, abort);
   } else {
+    regs_inc<kRegsHigh>();
     softmax_role<MODE>(warp >> 2, bars, tmem, p, abort);
   }
   __syncwarp();

@@ -135,6 +135,18 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
 
 // ---------------------------------------------------------------------------
 // tcgen05: tensor memory and the 5th-generation tensor core.
+// Per-warpgroup register re-allocation (every warp of the warpgroup executes
+// the same instruction).  The increases must fit in what the decreases free
+// from the block's launch allocation, or the increasing warps wait forever.
+template <uint32_t kRegs>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+template <uint32_t kRegs>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+
 __device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {
   asm volatile(
       "tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -292,6 +304,28 @@ __device__ __forceinline__ float lg2_approx(float x) {
   float y;
   asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA pipe (two lanes at once) for x in [-126, 0], used to take
+// part of the exponentials off the special-function unit.  Range reduction
+// x = j + f with j = floor(x): adding 1.5 * 2^23 with round-toward-minus-
+// infinity leaves j in the low mantissa bits of t (integers are exact there).
+// 2^f for f in [0, 1) is a degree-3 polynomial with minimax relative error
+// 7.5e-5 (coefficients fitted for this library), and 2^j is added into the
+// exponent field: the bits of t shifted left by 23 equal j << 23 modulo 2^32.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c0 = 0.9999252557754517f, c1 = 0.695833683013916f,
+                  c2 = 0.22606664896011353f, c3 = 0.07802490144968033f;
+  const float2 t = __fadd2_rd(x, make_float2(kShift, kShift));
+  const float2 j = __fadd2_rn(t, make_float2(-kShift, -kShift));
+  const float2 f = __ffma2_rn(j, make_float2(-1.f, -1.f), x);
+  float2 p = __ffma2_rn(make_float2(c3, c3), f, make_float2(c2, c2));
+  p = __ffma2_rn(p, f, make_float2(c1, c1));
+  p = __ffma2_rn(p, f, make_float2(c0, c0));
+  return make_float2(
+      __int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+      __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
