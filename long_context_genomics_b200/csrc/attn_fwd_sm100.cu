@@ -61,6 +61,9 @@ constexpr uint32_t kRegsHigh = 208;
 static_assert(2 * 128 * kRegsHigh + 128 * kRegsLow <= kThreads * kRegsLaunch,
               "register split exceeds the launch allocation");
 constexpr uint32_t kTmemCols = 512;
+// P (bf16 pairs) of a tile occupies tensor-memory columns [kPCol, kPCol + 64)
+// of that tile's S region (see the softmax section).
+constexpr uint32_t kPCol = 32;
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0);  // K-major B (K)
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, 1);  // MN-major B (V)
 constexpr float kLog2e = 1.4426950408889634f;
@@ -73,20 +76,23 @@ enum Mode { kStaticCap = 0, kOnlineCap = 1, kNoCap = 2 };
 // Wait sites recorded in the device error word.
 enum Site : unsigned {
   kSiteProdQ = 1, kSiteProdKV = 2, kSiteMmaQ = 3, kSiteMmaKV = 4,
-  kSiteMmaP = 5, kSiteSoftS = 6, kSiteSoftO = 7, kSiteDrain = 8
+  kSiteMmaP = 5, kSiteSoftS = 6, kSiteSoftO = 7, kSiteDrain = 8,
+  kSiteXchg = 9
 };
 
 struct __align__(8) Barriers {
   uint64_t q_full[2], q_empty[2];
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t s_full[2], p_full[2], o_full[2];
+  uint64_t xm[2], xd[2];  // row-max / row-sum exchange between warpgroups
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
 };
 
-constexpr size_t kSmemBytes =
-    1024 + (2 + kStages) * static_cast<size_t>(kTileBytes) + sizeof(Barriers);
+constexpr size_t kXchgBytes = 2 * 2 * 2 * 128 * sizeof(float);
+constexpr size_t kSmemBytes = 1024 + (2 + kStages) * static_cast<size_t>(kTileBytes) +
+                              sizeof(Barriers) + kXchgBytes;
 
 struct Params {
   const float *bias;
@@ -238,7 +244,7 @@ __device__ __forceinline__ void mma_issuer(uint8_t *q_s, uint8_t *kv_s,
         ++pcount[X];
         if (!ok) break;
         tc_fence_after();
-        issue_pv(tmem + 256 + X * 128, tmem + X * 128,
+        issue_pv(tmem + 256 + X * 128, tmem + X * 128 + kPCol,
                  kv_addr + slot_v * kTileBytes, j > 0);
         if (!has_next) {
           umma_commit(&bars->o_full[X]);
@@ -270,19 +276,53 @@ __device__ __forceinline__ void mma_issuer(uint8_t *q_s, uint8_t *kv_s,
 
 // --------------------------------------------------------------------------
 // Softmax warpgroups.
+//
+// All eight softmax warps work on query tile A, then all eight on tile B, then
+// A again: warpgroup g (0 or 1) takes keys [64g, 64g + 64) of every 128-key
+// tile for all 128 rows (thread r of each warpgroup owns tensor-memory lane r).
+// While the warps run one tile's softmax the tensor core runs the other
+// tile's PV and next QK^T, so the two alternate without further
+// synchronisation.  Each row's sum is split between its two threads and
+// combined through shared memory once per work item.
+//
+// P of a tile is written as bf16 over columns [32, 96) of its S region:
+// warpgroup 0 (S columns 0-63) writes P columns 32-63 and warpgroup 1
+// (S columns 64-127) writes P columns 64-95, so each warpgroup only ever
+// overwrites S columns it has already read itself.
 
-__device__ __forceinline__ void load_bias8(const float *brow, int j, int P,
-                                           float (&bn)[8]) {
-  const int J0 = j * 8;
+
+// Softmax-side shared memory (row-sum and row-max exchange between the two
+// threads of a row).
+struct Xchg {
+  float dpart[2][2][128];  // [tile][warpgroup][row]
+  float mpart[2][2][128];
+};
+
+// Publish this thread's value, then wait (bounded) until all 256 softmax
+// threads have published theirs.  The mbarrier's arrive/wait order the
+// shared-memory writes before the partner's read.
+__device__ __forceinline__ bool exchange(uint64_t *bar, uint32_t &count,
+                                         volatile int *abort, unsigned *err) {
+  mbar_arrive(bar);
+  const bool ok = mbar_wait(bar, count & 1u, abort, err, kSiteXchg);
+  ++count;
+  return __all_sync(0xffffffffu, ok);
+}
+
+// The 4 compact bias cells of this warpgroup's key half of key tile j:
+// bias[h, I, 8j + 4g .. 8j + 4g + 3].
+__device__ __forceinline__ void load_bias4(const float *brow, int j, int g, int P,
+                                           float (&bn)[4]) {
+  const int J0 = j * 8 + g * 4;
 #pragma unroll
-  for (int e = 0; e < 8; ++e) bn[e] = (J0 + e < P) ? __ldg(brow + J0 + e) : 0.f;
+  for (int e = 0; e < 4; ++e) bn[e] = (J0 + e < P) ? __ldg(brow + J0 + e) : 0.f;
 }
 
 // Column pairs (out of every 8) whose exponential runs on the FMA pipe
 // (exp2_poly2) instead of the special-function unit.  The SFU still computes
 // every tanh, so it does 1 + (8 - kEmuPairs) / 8 operations per logit.
 #ifndef AG_EXP2_EMU_PAIRS
-#define AG_EXP2_EMU_PAIRS 6
+#define AG_EXP2_EMU_PAIRS 7
 #endif
 constexpr int kEmuPairs = AG_EXP2_EMU_PAIRS;
 
@@ -318,31 +358,26 @@ __device__ __forceinline__ void chunk_static(const uint32_t (&s)[32], float b0,
   }
 }
 
-// One 128-key tile of the static-shift softmax: S from tensor memory in four
-// 32-column chunks (the next chunk's load overlaps this chunk's math), P back
-// over the first 64 columns.  Returns the tile's row sum.
+// This warpgroup's 64-key half of one tile, static shift: two 32-column
+// chunks of S in, 32 columns of P out.  Returns the half-row sum.  The first
+// chunk's P is stored only after the second chunk's load has completed
+// (for warpgroup 0 it lands on the second chunk's S columns).
 template <bool kMask>
-__device__ __forceinline__ float tile_static(uint32_t tS, const float (&bj)[8],
-                                             float2 sc, float2 ap, float2 an,
-                                             int nvalid) {
-  uint32_t sa[32], sb[32], pk[16];
+__device__ __forceinline__ float half_tile_static(uint32_t tS, int g,
+                                                  const float (&bj)[4], float2 sc,
+                                                  float2 ap, float2 an,
+                                                  int nvalid) {
+  uint32_t sa[32], sb[32], pa[16], pb[16];
   float2 acc = make_float2(0.f, 0.f);
-  tmem_ld32(tS + 0, sa);
+  const uint32_t c0 = g * 64;
+  tmem_ld32(tS + c0, sa);
   tmem_wait_ld(sa);
-  tmem_ld32(tS + 32, sb);
-  chunk_static<kMask>(sa, bj[0], bj[1], sc, ap, an, 0, nvalid, acc, pk);
-  tmem_st16(tS + 0, pk);
+  tmem_ld32(tS + c0 + 32, sb);
+  chunk_static<kMask>(sa, bj[0], bj[1], sc, ap, an, c0, nvalid, acc, pa);
   tmem_wait_ld(sb);
-  tmem_ld32(tS + 64, sa);
-  chunk_static<kMask>(sb, bj[2], bj[3], sc, ap, an, 32, nvalid, acc, pk);
-  tmem_st16(tS + 16, pk);
-  tmem_wait_ld(sa);
-  tmem_ld32(tS + 96, sb);
-  chunk_static<kMask>(sa, bj[4], bj[5], sc, ap, an, 64, nvalid, acc, pk);
-  tmem_st16(tS + 32, pk);
-  tmem_wait_ld(sb);
-  chunk_static<kMask>(sb, bj[6], bj[7], sc, ap, an, 96, nvalid, acc, pk);
-  tmem_st16(tS + 48, pk);
+  tmem_st16(tS + kPCol + g * 32, pa);
+  chunk_static<kMask>(sb, bj[2], bj[3], sc, ap, an, c0 + 32, nvalid, acc, pb);
+  tmem_st16(tS + kPCol + g * 32 + 16, pb);
   return acc.x + acc.y;
 }
 
@@ -360,132 +395,171 @@ __device__ __forceinline__ void chunk_logits(const uint32_t (&s)[32], float b0,
   }
 }
 
+// This warpgroup's half of one tile with a running maximum shared by the two
+// threads of each row (exchanged through shared memory).  Rescales this
+// warpgroup's half of O when the maximum grows past the lazy threshold.
 template <int MODE>
-__device__ __forceinline__ void softmax_role(int X, Barriers *bars, uint32_t tmem,
-                                             const Params &p,
+__device__ __forceinline__ bool half_tile_online(uint32_t tS, uint32_t tO, int g,
+                                                 int r, int X, int j,
+                                                 const float (&bj)[4],
+                                                 const Params &p, int nvalid,
+                                                 Xchg *xc, uint64_t *xbar,
+                                                 uint32_t &xcount,
+                                                 volatile int *abort, float &m,
+                                                 float &d) {
+  const uint32_t c0 = g * 64;
+  float mt = -INFINITY;
+#pragma unroll 1
+  for (int c = 0; c < 2; ++c) {
+    uint32_t s[32];
+    float x[32];
+    tmem_ld32(tS + c0 + c * 32, s);
+    tmem_wait_ld(s);
+    chunk_logits<MODE>(s, bj[2 * c], bj[2 * c + 1], p, c0 + c * 32, nvalid, x);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) mt = fmaxf(mt, x[e]);
+  }
+  xc->mpart[X][g][r] = mt;
+  if (!exchange(xbar, xcount, abort, p.err)) return false;
+  mt = fmaxf(mt, xc->mpart[X][g ^ 1][r]);
+  float factor = 1.f;
+  if (mt > m + kRescaleThreshold || m == -INFINITY) {
+    factor = (m == -INFINITY) ? 0.f : ex2_approx(m - mt);
+    m = mt;
+    d *= factor;
+  }
+  if (j > 0 && __any_sync(0xffffffffu, factor != 1.f)) {
+    // O(j-1) is complete: s_full(j) was committed after PV(j-1).
+#pragma unroll 1
+    for (int c = 0; c < 2; ++c) {
+      uint32_t o[32];
+      tmem_ld32(tO + c0 + c * 32, o);
+      tmem_wait_ld(o);
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
+      tmem_st32(tO + c0 + c * 32, o);
+    }
+  }
+  uint32_t pk[2][16];
+  float acc = 0.f;
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    uint32_t s[32];
+    float x[32];
+    tmem_ld32(tS + c0 + c * 32, s);
+    tmem_wait_ld(s);
+    chunk_logits<MODE>(s, bj[2 * c], bj[2 * c + 1], p, c0 + c * 32, nvalid, x);
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float p0 = ex2_approx(x[2 * e] - m);
+      const float p1 = ex2_approx(x[2 * e + 1] - m);
+      acc += p0 + p1;
+      pk[c][e] = pack_bf16x2(p0, p1);
+    }
+  }
+  // Both S chunks are read: P may now overwrite them.
+  tmem_st16(tS + kPCol + g * 32, pk[0]);
+  tmem_st16(tS + kPCol + g * 32 + 16, pk[1]);
+  d += acc;
+  return true;
+}
+
+template <int MODE>
+__device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc,
+                                             uint32_t tmem, const Params &p,
                                              volatile int *abort) {
-  const int r = threadIdx.x & 127;         // tile row == tensor-memory lane
-  const int wq = r >> 5;                   // warp's lane quarter
-  const int h = r >> 4, il = r & 15;       // head, position inside the block
+  const int g = (threadIdx.x >> 7) & 1;   // key half of every tile
+  const int r = threadIdx.x & 127;        // tile row == tensor-memory lane
+  const int wq = r >> 5;                  // warp's lane quarter
+  const int h = r >> 4, il = r & 15;      // head, position inside the block
   const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
-  const uint32_t tS = tmem + X * 128 + lane_base;
-  const uint32_t tO = tmem + 256 + X * 128 + lane_base;
-  uint32_t scount = 0, ocount = 0;
+  const float2 sc = make_float2(p.qk_scale, p.qk_scale);
+  const float2 ap = make_float2(p.A, p.A), an = make_float2(-p.A, -p.A);
+  uint32_t scount[2] = {0, 0}, ocount[2] = {0, 0};
+  uint32_t xmcount[2] = {0, 0}, xdcount[2] = {0, 0};
+  bool ok = true;
 
-  for (int w = blockIdx.x; w < p.n_items; w += gridDim.x) {
+  for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x) {
     const int b = w / p.pairs;
-    const int I = (w % p.pairs) * 2 + X;
-    if (I >= p.nb) continue;  // odd block count: tile B idles on the last pair
-    const float *brow = p.bias + (static_cast<size_t>(h) * p.P + I) * p.P;
-    float m = (MODE == kStaticCap) ? p.A : -INFINITY;  // log2 units
-    float d = 0.f;
-    float bnext[8];
-    load_bias8(brow, 0, p.P, bnext);
-    bool ok = true;
-    for (int j = 0; j < p.n_kt; ++j) {
-      float bj[8];
+    const int I0 = (w % p.pairs) * 2;
+    const int nX = (I0 + 1 < p.nb) ? 2 : 1;
+    const float *brow[2];
+    float m[2], d[2] = {0.f, 0.f};
+    float bn[2][4];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) bj[e] = bnext[e] * p.bias_mul;
-      if (j + 1 < p.n_kt) load_bias8(brow, j + 1, p.P, bnext);
+    for (int X = 0; X < 2; ++X) {
+      m[X] = (MODE == kStaticCap) ? p.A : -INFINITY;  // log2 units
+      brow[X] = p.bias + (static_cast<size_t>(h) * p.P + (I0 + (X < nX ? X : 0))) * p.P;
+      load_bias4(brow[X], 0, g, p.P, bn[X]);
+    }
+    for (int j = 0; j < p.n_kt && ok; ++j) {
       const int nvalid = (j + 1 == p.n_kt) ? p.last_valid : kKeys;
+#pragma unroll
+      for (int X = 0; X < 2; ++X) {
+        if (X >= nX) break;
+        float bj[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) bj[e] = bn[X][e] * p.bias_mul;
+        if (j + 1 < p.n_kt) load_bias4(brow[X], j + 1, g, p.P, bn[X]);
 
-      ok = mbar_wait(&bars->s_full[X], scount & 1u, abort, p.err, kSiteSoftS);
-      ++scount;
-      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-      tc_fence_after();
-
-      if constexpr (MODE == kStaticCap) {
-        const float2 sc = make_float2(p.qk_scale, p.qk_scale);
-        const float2 ap = make_float2(p.A, p.A), an = make_float2(-p.A, -p.A);
-        if (nvalid == kKeys)
-          d += tile_static<false>(tS, bj, sc, ap, an, nvalid);
-        else
-          d += tile_static<true>(tS, bj, sc, ap, an, nvalid);
-      } else {
-        // Pass 1: tile max of the log2-domain logits.
-        float mt = -INFINITY;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t s[32];
-          float x[32];
-          tmem_ld32(tS + c * 32, s);
-          tmem_wait_ld(s);
-          chunk_logits<MODE>(s, bj[2 * c], bj[2 * c + 1], p, c * 32, nvalid, x);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) mt = fmaxf(mt, x[e]);
+        ok = mbar_wait(&bars->s_full[X], scount[X] & 1u, abort, p.err, kSiteSoftS);
+        ++scount[X];
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t tS = tmem + X * 128 + lane_base;
+        if constexpr (MODE == kStaticCap) {
+          if (nvalid == kKeys)
+            d[X] += half_tile_static<false>(tS, g, bj, sc, ap, an, nvalid);
+          else
+            d[X] += half_tile_static<true>(tS, g, bj, sc, ap, an, nvalid);
+        } else {
+          const uint32_t tO = tmem + 256 + X * 128 + lane_base;
+          ok = half_tile_online<MODE>(tS, tO, g, r, X, j, bj, p, nvalid, xc,
+                                      &bars->xm[X], xmcount[X], abort, m[X], d[X]);
+          if (!ok) break;
         }
-        // Lazy rescale: keep the old shift unless the max grew by more than
-        // the threshold (values up to 2^threshold are exact enough in fp32).
-        float factor = 1.f;
-        if (mt > m + kRescaleThreshold || m == -INFINITY) {
-          factor = (m == -INFINITY) ? 0.f : ex2_approx(m - mt);
-          m = mt;
-          d *= factor;
-        }
-        if (j > 0 && __any_sync(0xffffffffu, factor != 1.f)) {
-          // O_X(j-1) is complete: s_full(j) was committed after PV_X(j-1).
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tO + c * 32, o);
-            tmem_wait_ld(o);
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-              o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
-            tmem_st32(tO + c * 32, o);
-          }
-        }
-        // Pass 2: probabilities.
-        float acc = 0.f;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t s[32], pk[16];
-          float x[32];
-          tmem_ld32(tS + c * 32, s);
-          tmem_wait_ld(s);
-          chunk_logits<MODE>(s, bj[2 * c], bj[2 * c + 1], p, c * 32, nvalid, x);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float p0 = ex2_approx(x[2 * e] - m);
-            const float p1 = ex2_approx(x[2 * e + 1] - m);
-            acc += p0 + p1;
-            pk[e] = pack_bf16x2(p0, p1);
-          }
-          tmem_st16(tS + c * 16, pk);
-        }
-        d += acc;
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars->p_full[X]);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&bars->p_full[X]);
     }
     if (!ok) break;
 
-    ok = mbar_wait(&bars->o_full[X], ocount & 1u, abort, p.err, kSiteSoftO);
-    ++ocount;
-    if (!__all_sync(0xffffffffu, ok)) break;
-    tc_fence_after();
-
-    // Epilogue: out = O / d (fp32, one 512-byte row per thread), lse.
-    const float inv_d = 1.f / d;
-    const size_t row = (static_cast<size_t>(b) * kH + h) * p.L +
-                       static_cast<size_t>(I) * 16 + il;
-    float4 *orow = reinterpret_cast<float4 *>(p.out + row * kD);
-#pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-      uint32_t o[32];
-      tmem_ld32(tO + c * 32, o);
-      tmem_wait_ld(o);
+    // Epilogue: d = both halves' sums; out = O / d (this warpgroup's 64
+    // columns of the row, 256 bytes), lse from warpgroup 0.
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        orow[c * 8 + e] = make_float4(__uint_as_float(o[4 * e]) * inv_d,
-                                      __uint_as_float(o[4 * e + 1]) * inv_d,
-                                      __uint_as_float(o[4 * e + 2]) * inv_d,
-                                      __uint_as_float(o[4 * e + 3]) * inv_d);
+    for (int X = 0; X < 2; ++X) {
+      if (X >= nX) break;
+      ok = mbar_wait(&bars->o_full[X], ocount[X] & 1u, abort, p.err, kSiteSoftO);
+      ++ocount[X];
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      tc_fence_after();
+      xc->dpart[X][g][r] = d[X];
+      ok = exchange(&bars->xd[X], xdcount[X], abort, p.err);
+      if (!ok) break;
+      const float dsum = d[X] + xc->dpart[X][g ^ 1][r];
+      const float inv_d = 1.f / dsum;
+      const size_t row = (static_cast<size_t>(b) * kH + h) * p.L +
+                         static_cast<size_t>(I0 + X) * 16 + il;
+      float4 *orow = reinterpret_cast<float4 *>(p.out + row * kD + g * 64);
+      const uint32_t tO = tmem + 256 + X * 128 + lane_base + g * 64;
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tO + c * 32, o);
+        tmem_wait_ld(o);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          orow[c * 8 + e] = make_float4(__uint_as_float(o[4 * e]) * inv_d,
+                                        __uint_as_float(o[4 * e + 1]) * inv_d,
+                                        __uint_as_float(o[4 * e + 2]) * inv_d,
+                                        __uint_as_float(o[4 * e + 3]) * inv_d);
+        }
       }
+      if (g == 0) p.lse[row] = (m[X] + lg2_approx(dsum)) * kLn2;
+      tc_fence_before();
     }
-    p.lse[row] = (m + lg2_approx(d)) * kLn2;
-    tc_fence_before();
   }
 }
 
@@ -500,6 +574,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *q_s = smem_raw + pad;                 // 2 query tiles
   uint8_t *kv_s = q_s + 2 * kTileBytes;          // K/V ring
   Barriers *bars = reinterpret_cast<Barriers *>(kv_s + kStages * kTileBytes);
+  auto *xc = reinterpret_cast<struct Xchg *>(reinterpret_cast<uint8_t *>(bars) +
+                                             sizeof(Barriers));
   const int warp = threadIdx.x >> 5;
 
   if (threadIdx.x == 0) {
@@ -507,7 +583,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->q_full[X], 1);
       mbar_init(&bars->q_empty[X], 1);
       mbar_init(&bars->s_full[X], 1);
-      mbar_init(&bars->p_full[X], 128);
+      mbar_init(&bars->p_full[X], 256);
+      mbar_init(&bars->xm[X], 256);
+      mbar_init(&bars->xd[X], 256);
       mbar_init(&bars->o_full[X], 1);
     }
     for (int s = 0; s < kStages; ++s) {
@@ -541,7 +619,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_issuer(q_s, kv_s, bars, tmem, p, abort);
   } else {
     regs_inc<kRegsHigh>();
-    softmax_role<MODE>(warp >> 2, bars, tmem, p, abort);
+    softmax_role<MODE>(bars, xc, tmem, p, abort);
   }
   __syncwarp();
   tc_fence_before();
