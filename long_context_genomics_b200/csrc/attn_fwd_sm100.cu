@@ -44,26 +44,32 @@ constexpr int kKeys = 128;                  // keys per K/V tile
 constexpr int kStages = 4;                  // K/V ring slots
 constexpr int kTileBytes = 128 * 128 * 2;   // one Q, K or V tile (bf16)
 constexpr int kHalfBytes = kTileBytes / 2;  // one 64-wide (128-byte) half
-// Warps 0-7: two softmax warpgroups; warpgroup 2 = warp 8 (TMA producer),
-// warp 9 (MMA issuer) and warps 10-11 (idle, present so that warpgroup 2 is
-// whole for the register re-allocation).
-constexpr int kNumWarps = 12;
+// Softmax warpgroups (2 or 4).  Warps 0 .. 4*kWG-1 run the softmax; the next
+// warpgroup holds the TMA producer warp, the MMA warp and two idle warps
+// (present so that it is whole for the register re-allocation).
+#ifndef AG_SOFTMAX_WARPGROUPS
+#define AG_SOFTMAX_WARPGROUPS 4
+#endif
+constexpr int kWG = AG_SOFTMAX_WARPGROUPS;
+static_assert(kWG == 2 || kWG == 4, "two or four softmax warpgroups");
+constexpr int kChunks = 4 / kWG;             // 32-column chunks per warpgroup
+constexpr int kSoftThreads = 128 * kWG;
+constexpr int kNumWarps = 4 * kWG + 4;
 constexpr int kThreads = kNumWarps * 32;
-constexpr int kWarpLoad = 8;
-constexpr int kWarpMma = 9;
+constexpr int kWarpLoad = 4 * kWG;
+constexpr int kWarpMma = 4 * kWG + 1;
 // Registers per thread: the launch gives every thread kRegsLaunch (the cap
-// for 384 threads, which ptxas allocates when setmaxnreg is present); the
-// producer warpgroup drops to kRegsLow and the softmax warpgroups rise to
-// kRegsHigh.  Budget: 2*128*kRegsHigh + 128*kRegsLow <= 384*kRegsLaunch.
-constexpr uint32_t kRegsLaunch = 168;
-constexpr uint32_t kRegsLow = 88;
-constexpr uint32_t kRegsHigh = 208;
-static_assert(2 * 128 * kRegsHigh + 128 * kRegsLow <= kThreads * kRegsLaunch,
+// for this block size, which ptxas allocates when setmaxnreg is present; the
+// launcher checks it); the producer warpgroup then drops to kRegsLow and the
+// softmax warpgroups rise to kRegsHigh.
+constexpr uint32_t kRegsLaunch = kWG == 2 ? 168 : 96;
+constexpr uint32_t kRegsLow = kWG == 2 ? 88 : 64;
+constexpr uint32_t kRegsHigh = kWG == 2 ? 208 : 104;
+static_assert(kSoftThreads * kRegsHigh + 128 * kRegsLow <= kThreads * kRegsLaunch,
               "register split exceeds the launch allocation");
 constexpr uint32_t kTmemCols = 512;
-// P (bf16 pairs) of a tile occupies tensor-memory columns [kPCol, kPCol + 64)
-// of that tile's S region (see the softmax section).
-constexpr uint32_t kPCol = 32;
+// P (bf16 pairs) of a tile: keys [32c, 32c + 32) of chunk c are written over
+// the first 16 columns of that chunk's own S columns, [32c, 32c + 16).
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0);  // K-major B (K)
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, 1);  // MN-major B (V)
 constexpr float kLog2e = 1.4426950408889634f;
@@ -90,7 +96,7 @@ struct __align__(8) Barriers {
   int abort;
 };
 
-constexpr size_t kXchgBytes = 2 * 2 * 2 * 128 * sizeof(float);
+constexpr size_t kXchgBytes = 2 * 2 * kWG * 128 * sizeof(float);
 constexpr size_t kSmemBytes = 1024 + (2 + kStages) * static_cast<size_t>(kTileBytes) +
                               sizeof(Barriers) + kXchgBytes;
 
@@ -125,13 +131,14 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_addr,
 }
 
 // O[128 x 128] (+)= P[128 x 128 keys] V[128 keys x 128]: P from tensor memory
-// (bf16 pairs, 8 columns per 16 keys), V MN-major in shared memory (the two
-// 64-wide halves are 16 KB apart, 8-key row groups 1 KB apart).
-__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem,
+// (bf16 pairs, 8 columns per 16 keys; keys 32c.. of chunk c start at column
+// 32c of the S region), V MN-major in shared memory (the two 64-wide halves
+// are 16 KB apart, 8-key row groups 1 KB apart).
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t s_tmem,
                                          uint32_t v_addr, bool accumulate) {
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk) {
-    umma_ts(d_tmem, p_tmem + kk * 8,
+    umma_ts(d_tmem, s_tmem + 32 * (kk >> 1) + 8 * (kk & 1),
             smem_desc_sw128(v_addr + kk * 2048, kHalfBytes, 1024), kIdescPV,
             (accumulate || kk > 0) ? 1u : 0u);
   }
@@ -147,7 +154,7 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // --------------------------------------------------------------------------
-// Warp 8, lane 0: TMA producer.
+// Producer warp, lane 0: TMA loads.
 __device__ __forceinline__ void producer(const CUtensorMap *tm_q,
                                          const CUtensorMap *tm_k,
                                          const CUtensorMap *tm_v, uint8_t *q_s,
@@ -198,7 +205,7 @@ __device__ __forceinline__ void producer(const CUtensorMap *tm_q,
 }
 
 // --------------------------------------------------------------------------
-// Warp 9, lane 0: tcgen05.mma issuer.
+// MMA warp, lane 0: tcgen05.mma issuer.
 __device__ __forceinline__ void mma_issuer(uint8_t *q_s, uint8_t *kv_s,
                                            Barriers *bars, uint32_t tmem,
                                            const Params &p, volatile int *abort) {
@@ -244,7 +251,7 @@ __device__ __forceinline__ void mma_issuer(uint8_t *q_s, uint8_t *kv_s,
         ++pcount[X];
         if (!ok) break;
         tc_fence_after();
-        issue_pv(tmem + 256 + X * 128, tmem + X * 128 + kPCol,
+        issue_pv(tmem + 256 + X * 128, tmem + X * 128,
                  kv_addr + slot_v * kTileBytes, j > 0);
         if (!has_next) {
           umma_commit(&bars->o_full[X]);
@@ -277,30 +284,26 @@ __device__ __forceinline__ void mma_issuer(uint8_t *q_s, uint8_t *kv_s,
 // --------------------------------------------------------------------------
 // Softmax warpgroups.
 //
-// All eight softmax warps work on query tile A, then all eight on tile B, then
-// A again: warpgroup g (0 or 1) takes keys [64g, 64g + 64) of every 128-key
-// tile for all 128 rows (thread r of each warpgroup owns tensor-memory lane r).
-// While the warps run one tile's softmax the tensor core runs the other
-// tile's PV and next QK^T, so the two alternate without further
-// synchronisation.  Each row's sum is split between its two threads and
-// combined through shared memory once per work item.
-//
-// P of a tile is written as bf16 over columns [32, 96) of its S region:
-// warpgroup 0 (S columns 0-63) writes P columns 32-63 and warpgroup 1
-// (S columns 64-127) writes P columns 64-95, so each warpgroup only ever
+// All softmax warps work on query tile A, then all on tile B, then A again:
+// warpgroup g takes the kChunks 32-key chunks starting at key 32*kChunks*g of
+// every 128-key tile, for all 128 rows (thread r of every warpgroup owns
+// tensor-memory lane r).  While the warps run one tile's softmax the tensor
+// core runs the other tile's PV and next QK^T, so the two alternate without
+// further synchronisation.  A row's sum is split between its kWG threads and
+// combined through shared memory once per work item.  Each chunk's P goes over
+// the first half of that chunk's own S columns, so a warpgroup only ever
 // overwrites S columns it has already read itself.
 
-
-// Softmax-side shared memory (row-sum and row-max exchange between the two
-// threads of a row).
+// Softmax-side shared memory: row-sum and row-max exchange between the kWG
+// threads of a row.
 struct Xchg {
-  float dpart[2][2][128];  // [tile][warpgroup][row]
-  float mpart[2][2][128];
+  float dpart[2][kWG][128];  // [tile][warpgroup][row]
+  float mpart[2][kWG][128];
 };
 
-// Publish this thread's value, then wait (bounded) until all 256 softmax
-// threads have published theirs.  The mbarrier's arrive/wait order the
-// shared-memory writes before the partner's read.
+// Publish this thread's value, then wait (bounded) until every softmax thread
+// has published its own.  The mbarrier's arrive/wait order the shared-memory
+// writes before the partners' reads.
 __device__ __forceinline__ bool exchange(uint64_t *bar, uint32_t &count,
                                          volatile int *abort, unsigned *err) {
   mbar_arrive(bar);
@@ -309,20 +312,21 @@ __device__ __forceinline__ bool exchange(uint64_t *bar, uint32_t &count,
   return __all_sync(0xffffffffu, ok);
 }
 
-// The 4 compact bias cells of this warpgroup's key half of key tile j:
-// bias[h, I, 8j + 4g .. 8j + 4g + 3].
-__device__ __forceinline__ void load_bias4(const float *brow, int j, int g, int P,
-                                           float (&bn)[4]) {
-  const int J0 = j * 8 + g * 4;
+// The compact bias cells of this warpgroup's keys of key tile j (two per
+// 32-key chunk): bias[h, I, 8j + 2*kChunks*g + e].
+__device__ __forceinline__ void load_bias(const float *brow, int j, int g, int P,
+                                          float (&bn)[2 * kChunks]) {
+  const int J0 = j * 8 + g * 2 * kChunks;
 #pragma unroll
-  for (int e = 0; e < 4; ++e) bn[e] = (J0 + e < P) ? __ldg(brow + J0 + e) : 0.f;
+  for (int e = 0; e < 2 * kChunks; ++e)
+    bn[e] = (J0 + e < P) ? __ldg(brow + J0 + e) : 0.f;
 }
 
 // Column pairs (out of every 8) whose exponential runs on the FMA pipe
 // (exp2_poly2) instead of the special-function unit.  The SFU still computes
 // every tanh, so it does 1 + (8 - kEmuPairs) / 8 operations per logit.
 #ifndef AG_EXP2_EMU_PAIRS
-#define AG_EXP2_EMU_PAIRS 7
+#define AG_EXP2_EMU_PAIRS 6
 #endif
 constexpr int kEmuPairs = AG_EXP2_EMU_PAIRS;
 
@@ -358,26 +362,34 @@ __device__ __forceinline__ void chunk_static(const uint32_t (&s)[32], float b0,
   }
 }
 
-// This warpgroup's 64-key half of one tile, static shift: two 32-column
-// chunks of S in, 32 columns of P out.  Returns the half-row sum.  The first
-// chunk's P is stored only after the second chunk's load has completed
-// (for warpgroup 0 it lands on the second chunk's S columns).
+// This warpgroup's chunks of one tile, static shift: S in, P out over the
+// first 16 columns of each chunk.  Returns the partial row sum.
 template <bool kMask>
-__device__ __forceinline__ float half_tile_static(uint32_t tS, int g,
-                                                  const float (&bj)[4], float2 sc,
-                                                  float2 ap, float2 an,
+__device__ __forceinline__ float part_tile_static(uint32_t tS, int g,
+                                                  const float (&bj)[2 * kChunks],
+                                                  float2 sc, float2 ap, float2 an,
                                                   int nvalid) {
-  uint32_t sa[32], sb[32], pa[16], pb[16];
   float2 acc = make_float2(0.f, 0.f);
-  const uint32_t c0 = g * 64;
-  tmem_ld32(tS + c0, sa);
-  tmem_wait_ld(sa);
-  tmem_ld32(tS + c0 + 32, sb);
-  chunk_static<kMask>(sa, bj[0], bj[1], sc, ap, an, c0, nvalid, acc, pa);
-  tmem_wait_ld(sb);
-  tmem_st16(tS + kPCol + g * 32, pa);
-  chunk_static<kMask>(sb, bj[2], bj[3], sc, ap, an, c0 + 32, nvalid, acc, pb);
-  tmem_st16(tS + kPCol + g * 32 + 16, pb);
+  uint32_t pk[16];
+  if constexpr (kChunks == 1) {
+    uint32_t sa[32];
+    const uint32_t c0 = 32 * g;
+    tmem_ld32(tS + c0, sa);
+    tmem_wait_ld(sa);
+    chunk_static<kMask>(sa, bj[0], bj[1], sc, ap, an, c0, nvalid, acc, pk);
+    tmem_st16(tS + c0, pk);
+  } else {
+    uint32_t sa[32], sb[32];
+    const uint32_t c0 = 64 * g;
+    tmem_ld32(tS + c0, sa);
+    tmem_wait_ld(sa);
+    tmem_ld32(tS + c0 + 32, sb);
+    chunk_static<kMask>(sa, bj[0], bj[1], sc, ap, an, c0, nvalid, acc, pk);
+    tmem_st16(tS + c0, pk);
+    tmem_wait_ld(sb);
+    chunk_static<kMask>(sb, bj[2], bj[3], sc, ap, an, c0 + 32, nvalid, acc, pk);
+    tmem_st16(tS + c0 + 32, pk);
+  }
   return acc.x + acc.y;
 }
 
@@ -395,22 +407,22 @@ __device__ __forceinline__ void chunk_logits(const uint32_t (&s)[32], float b0,
   }
 }
 
-// This warpgroup's half of one tile with a running maximum shared by the two
-// threads of each row (exchanged through shared memory).  Rescales this
-// warpgroup's half of O when the maximum grows past the lazy threshold.
+// This warpgroup's chunks of one tile with a running maximum shared by the
+// kWG threads of each row (exchanged through shared memory).  Rescales this
+// warpgroup's columns of O when the maximum grows past the lazy threshold.
 template <int MODE>
-__device__ __forceinline__ bool half_tile_online(uint32_t tS, uint32_t tO, int g,
+__device__ __forceinline__ bool part_tile_online(uint32_t tS, uint32_t tO, int g,
                                                  int r, int X, int j,
-                                                 const float (&bj)[4],
+                                                 const float (&bj)[2 * kChunks],
                                                  const Params &p, int nvalid,
                                                  Xchg *xc, uint64_t *xbar,
                                                  uint32_t &xcount,
                                                  volatile int *abort, float &m,
                                                  float &d) {
-  const uint32_t c0 = g * 64;
+  const uint32_t c0 = 32 * kChunks * g;
   float mt = -INFINITY;
 #pragma unroll 1
-  for (int c = 0; c < 2; ++c) {
+  for (int c = 0; c < kChunks; ++c) {
     uint32_t s[32];
     float x[32];
     tmem_ld32(tS + c0 + c * 32, s);
@@ -421,7 +433,8 @@ __device__ __forceinline__ bool half_tile_online(uint32_t tS, uint32_t tO, int g
   }
   xc->mpart[X][g][r] = mt;
   if (!exchange(xbar, xcount, abort, p.err)) return false;
-  mt = fmaxf(mt, xc->mpart[X][g ^ 1][r]);
+#pragma unroll
+  for (int q = 0; q < kWG; ++q) mt = fmaxf(mt, xc->mpart[X][q][r]);
   float factor = 1.f;
   if (mt > m + kRescaleThreshold || m == -INFINITY) {
     factor = (m == -INFINITY) ? 0.f : ex2_approx(m - mt);
@@ -431,7 +444,7 @@ __device__ __forceinline__ bool half_tile_online(uint32_t tS, uint32_t tO, int g
   if (j > 0 && __any_sync(0xffffffffu, factor != 1.f)) {
     // O(j-1) is complete: s_full(j) was committed after PV(j-1).
 #pragma unroll 1
-    for (int c = 0; c < 2; ++c) {
+    for (int c = 0; c < kChunks; ++c) {
       uint32_t o[32];
       tmem_ld32(tO + c0 + c * 32, o);
       tmem_wait_ld(o);
@@ -441,11 +454,10 @@ __device__ __forceinline__ bool half_tile_online(uint32_t tS, uint32_t tO, int g
       tmem_st32(tO + c0 + c * 32, o);
     }
   }
-  uint32_t pk[2][16];
   float acc = 0.f;
-#pragma unroll
-  for (int c = 0; c < 2; ++c) {
-    uint32_t s[32];
+#pragma unroll 1
+  for (int c = 0; c < kChunks; ++c) {
+    uint32_t s[32], pk[16];
     float x[32];
     tmem_ld32(tS + c0 + c * 32, s);
     tmem_wait_ld(s);
@@ -455,12 +467,10 @@ __device__ __forceinline__ bool half_tile_online(uint32_t tS, uint32_t tO, int g
       const float p0 = ex2_approx(x[2 * e] - m);
       const float p1 = ex2_approx(x[2 * e + 1] - m);
       acc += p0 + p1;
-      pk[c][e] = pack_bf16x2(p0, p1);
+      pk[e] = pack_bf16x2(p0, p1);
     }
+    tmem_st16(tS + c0 + c * 32, pk);
   }
-  // Both S chunks are read: P may now overwrite them.
-  tmem_st16(tS + kPCol + g * 32, pk[0]);
-  tmem_st16(tS + kPCol + g * 32 + 16, pk[1]);
   d += acc;
   return true;
 }
@@ -469,7 +479,7 @@ template <int MODE>
 __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc,
                                              uint32_t tmem, const Params &p,
                                              volatile int *abort) {
-  const int g = (threadIdx.x >> 7) & 1;   // key half of every tile
+  const int g = threadIdx.x >> 7;         // warpgroup: which key chunks
   const int r = threadIdx.x & 127;        // tile row == tensor-memory lane
   const int wq = r >> 5;                  // warp's lane quarter
   const int h = r >> 4, il = r & 15;      // head, position inside the block
@@ -486,22 +496,22 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc,
     const int nX = (I0 + 1 < p.nb) ? 2 : 1;
     const float *brow[2];
     float m[2], d[2] = {0.f, 0.f};
-    float bn[2][4];
+    float bn[2][2 * kChunks];
 #pragma unroll
     for (int X = 0; X < 2; ++X) {
       m[X] = (MODE == kStaticCap) ? p.A : -INFINITY;  // log2 units
       brow[X] = p.bias + (static_cast<size_t>(h) * p.P + (I0 + (X < nX ? X : 0))) * p.P;
-      load_bias4(brow[X], 0, g, p.P, bn[X]);
+      load_bias(brow[X], 0, g, p.P, bn[X]);
     }
     for (int j = 0; j < p.n_kt && ok; ++j) {
       const int nvalid = (j + 1 == p.n_kt) ? p.last_valid : kKeys;
 #pragma unroll
       for (int X = 0; X < 2; ++X) {
         if (X >= nX) break;
-        float bj[4];
+        float bj[2 * kChunks];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) bj[e] = bn[X][e] * p.bias_mul;
-        if (j + 1 < p.n_kt) load_bias4(brow[X], j + 1, g, p.P, bn[X]);
+        for (int e = 0; e < 2 * kChunks; ++e) bj[e] = bn[X][e] * p.bias_mul;
+        if (j + 1 < p.n_kt) load_bias(brow[X], j + 1, g, p.P, bn[X]);
 
         ok = mbar_wait(&bars->s_full[X], scount[X] & 1u, abort, p.err, kSiteSoftS);
         ++scount[X];
@@ -510,12 +520,12 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc,
         const uint32_t tS = tmem + X * 128 + lane_base;
         if constexpr (MODE == kStaticCap) {
           if (nvalid == kKeys)
-            d[X] += half_tile_static<false>(tS, g, bj, sc, ap, an, nvalid);
+            d[X] += part_tile_static<false>(tS, g, bj, sc, ap, an, nvalid);
           else
-            d[X] += half_tile_static<true>(tS, g, bj, sc, ap, an, nvalid);
+            d[X] += part_tile_static<true>(tS, g, bj, sc, ap, an, nvalid);
         } else {
           const uint32_t tO = tmem + 256 + X * 128 + lane_base;
-          ok = half_tile_online<MODE>(tS, tO, g, r, X, j, bj, p, nvalid, xc,
+          ok = part_tile_online<MODE>(tS, tO, g, r, X, j, bj, p, nvalid, xc,
                                       &bars->xm[X], xmcount[X], abort, m[X], d[X]);
           if (!ok) break;
         }
@@ -526,8 +536,8 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc,
     }
     if (!ok) break;
 
-    // Epilogue: d = both halves' sums; out = O / d (this warpgroup's 64
-    // columns of the row, 256 bytes), lse from warpgroup 0.
+    // Epilogue: d = sum of the kWG partial sums; out = O / d (this
+    // warpgroup's 32*kChunks columns of the row), lse from warpgroup 0.
 #pragma unroll
     for (int X = 0; X < 2; ++X) {
       if (X >= nX) break;
@@ -538,14 +548,17 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc,
       xc->dpart[X][g][r] = d[X];
       ok = exchange(&bars->xd[X], xdcount[X], abort, p.err);
       if (!ok) break;
-      const float dsum = d[X] + xc->dpart[X][g ^ 1][r];
+      float dsum = 0.f;
+#pragma unroll
+      for (int q = 0; q < kWG; ++q) dsum += xc->dpart[X][q][r];
       const float inv_d = 1.f / dsum;
       const size_t row = (static_cast<size_t>(b) * kH + h) * p.L +
                          static_cast<size_t>(I0 + X) * 16 + il;
-      float4 *orow = reinterpret_cast<float4 *>(p.out + row * kD + g * 64);
-      const uint32_t tO = tmem + 256 + X * 128 + lane_base + g * 64;
+      const int c0 = 32 * kChunks * g;
+      float4 *orow = reinterpret_cast<float4 *>(p.out + row * kD + c0);
+      const uint32_t tO = tmem + 256 + X * 128 + lane_base + c0;
 #pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < kChunks; ++c) {
         uint32_t o[32];
         tmem_ld32(tO + c * 32, o);
         tmem_wait_ld(o);
@@ -583,9 +596,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->q_full[X], 1);
       mbar_init(&bars->q_empty[X], 1);
       mbar_init(&bars->s_full[X], 1);
-      mbar_init(&bars->p_full[X], 256);
-      mbar_init(&bars->xm[X], 256);
-      mbar_init(&bars->xd[X], 256);
+      mbar_init(&bars->p_full[X], kSoftThreads);
+      mbar_init(&bars->xm[X], kSoftThreads);
+      mbar_init(&bars->xd[X], kSoftThreads);
       mbar_init(&bars->o_full[X], 1);
     }
     for (int s = 0; s < kStages; ++s) {
@@ -657,6 +670,14 @@ static cudaError_t launch_mode(const CUtensorMap &tq, const CUtensorMap &tk,
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!configured[dev]) {
+    // setmaxnreg.inc waits until the registers it asks for are free: refuse
+    // to launch a build whose launch allocation cannot cover the split.
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, attn::attn_fwd_kernel<MODE>);
+    if (e != cudaSuccess) return e;
+    if (static_cast<uint32_t>(fa.numRegs) * attn::kThreads <
+        attn::kSoftThreads * attn::kRegsHigh + 128 * attn::kRegsLow)
+      return cudaErrorInvalidConfiguration;
     e = cudaFuncSetAttribute(attn::attn_fwd_kernel<MODE>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(attn::kSmemBytes));
