@@ -12,8 +12,9 @@
  *
  * Conventions shared by every entry point:
  *   - Every pointer argument is a DEVICE pointer unless stated otherwise,
- *     row-major, densely packed.  The caller allocates and owns all buffers;
- *     the library allocates no device memory and keeps no per-call state.
+ *     row-major, densely packed.  The caller allocates and owns all inputs
+ *     and outputs.  The only memory the library allocates itself is the
+ *     attention scratch described at ag_attn_fwd.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Calls are asynchronous on that stream: AG_OK means the work
  *     was enqueued.  Faults inside a kernel surface at the caller's next
@@ -95,10 +96,19 @@ ag_status ag_pair_bias_project(const float *pair, const float *W, float *bias,
  *   lse   [B, H, L]     float32,   4-byte aligned (written)
  *   cap   > 0 and not NaN; +INFINITY disables the soft cap.
  * Supported: H == 8, D == 128, block == 16, L % 16 == 0, L <= 65536,
- * B * L <= 2^31 / 8.  B == 0 or L == 0 is a no-op (pointers may be NULL).
+ * B * L <= 2^28 and B * ceil(L/32) * ceil(L/128) <= 2^30 (B * L^2 up to
+ * about 2^42).  B == 0 or L == 0 is a no-op (pointers may be NULL).
  * Products in bf16 with fp32 accumulation (tensor cores); softmax in fp32;
  * the probabilities are rounded to bf16 for the second product while the
  * row sums use their fp32 values.
+ *
+ * Scratch: to keep every SM busy to the end, a pair of query tiles may have
+ * its keys split between SMs; each piece's partial result goes through a
+ * scratch buffer of 132,096 bytes per SM (19.6 MB on a 148-SM B200) and a
+ * second kernel on the same stream merges the pieces (by log-sum-exp).  The
+ * first call on a device allocates that buffer with cudaMalloc; it is kept
+ * until the process exits.  Calls whose kernels overlap on the device (e.g.
+ * on two streams at once) must not run concurrently, because they share it.
  */
 ag_status ag_attn_fwd(const void *q, const void *k, const void *v,
                       const float *bias, int64_t B, int64_t H, int64_t L,

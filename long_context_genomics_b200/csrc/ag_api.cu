@@ -26,6 +26,7 @@ struct DeviceInfo {
   bool sm100 = false;
   int num_sms = 0;
   unsigned *err = nullptr;  // device address of g_device_error_word
+  void *scratch = nullptr;  // attention split-pair scratch (one slot per SM)
 };
 
 std::mutex g_mu;
@@ -60,6 +61,20 @@ ag_status device_info(DeviceInfo **out) {
   }
   if (!d.sm100) return AG_ERR_UNSUPPORTED;
   *out = &d;
+  return AG_OK;
+}
+
+// The attention kernel's scratch, allocated with cudaMalloc on the first call
+// that needs it on this device and kept until the process exits.
+ag_status device_scratch(DeviceInfo *d, void **out) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!d->scratch) {
+    void *p = nullptr;
+    const size_t bytes = attn_scratch_bytes(d->num_sms);
+    if (cudaMalloc(&p, bytes) != cudaSuccess) return AG_ERR_CUDA;
+    d->scratch = p;
+  }
+  *out = d->scratch;
   return AG_OK;
 }
 
@@ -157,7 +172,7 @@ ag_status ag_pair_bias_project(const float *pair, const float *W, float *bias,
   ag_status st = ag::device_info(&dev);
   if (st != AG_OK) return st;
   return ag::from_cuda(ag::launch_pair_bias_project(
-      pair, W, bias, P, dev->num_sms, static_cast<cudaStream_t>(stream)));
+      pair, W, bias, P, dev->num_sms, dev->err, static_cast<cudaStream_t>(stream)));
 }
 
 ag_status ag_attn_fwd(const void *q, const void *k, const void *v,
@@ -169,6 +184,9 @@ ag_status ag_attn_fwd(const void *q, const void *k, const void *v,
   if (std::isnan(cap) || !(cap > 0.0f)) return AG_ERR_VALUE;
   if (H != 8 || D != 128 || block != 16 || L > 65536) return AG_ERR_UNSUPPORTED;
   if (B > 0 && L > 0 && B * L > (int64_t(1) << 28)) return AG_ERR_UNSUPPORTED;
+  // Work steps (pairs of query tiles x key tiles) must stay below 2^30.
+  if (B > 0 && L > 0 && B * ((L / 16 + 1) / 2) * ((L + 127) / 128) > (int64_t(1) << 30))
+    return AG_ERR_UNSUPPORTED;
   if (B == 0 || L == 0) return AG_OK;
   if (!q || !k || !v || !bias || !out || !lse) return AG_ERR_NULL;
   if (!ag::aligned(q, 16) || !ag::aligned(k, 16) || !ag::aligned(v, 16) ||
@@ -192,6 +210,9 @@ ag_status ag_attn_fwd(const void *q, const void *k, const void *v,
   ag::EncodeTiledFn enc = nullptr;
   st = ag::get_encoder(&enc);
   if (st != AG_OK) return st;
+  void *scratch = nullptr;
+  st = ag::device_scratch(dev, &scratch);
+  if (st != AG_OK) return st;
   ag::AttnLaunch a;
   a.q = q;
   a.k = k;
@@ -204,6 +225,8 @@ ag_status ag_attn_fwd(const void *q, const void *k, const void *v,
   a.cap = cap;
   a.err = dev->err;
   a.num_sms = dev->num_sms;
+  a.scratch = scratch;
+  a.scratch_slots = dev->num_sms;
   a.encode = enc;
   a.stream = static_cast<cudaStream_t>(stream);
   return ag::from_cuda(ag::launch_attn_fwd(a));

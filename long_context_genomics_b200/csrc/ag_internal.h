@@ -14,6 +14,15 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType,
                                    CUtensorMapSwizzle, CUtensorMapL2promotion,
                                    CUtensorMapFloatOOBfill);
 
+// Scratch of the attention kernel for pairs of query tiles whose key range is
+// split between CTAs: per CTA slot a partial output [2][128][128] fp32 and a
+// partial log-sum-exp [2][128] fp32.  Nothing in it must be initialised.
+constexpr size_t kAttnSlotOutBytes = 2 * 128 * 128 * sizeof(float);
+constexpr size_t kAttnSlotLseBytes = 2 * 128 * sizeof(float);
+inline size_t attn_scratch_bytes(int slots) {
+  return static_cast<size_t>(slots) * (kAttnSlotOutBytes + kAttnSlotLseBytes);
+}
+
 struct AttnLaunch {
   const void *q, *k, *v;
   const float *bias;
@@ -22,6 +31,8 @@ struct AttnLaunch {
   float cap;
   unsigned *err;        // device error word
   int num_sms;
+  void *scratch;        // attn_scratch_bytes(scratch_slots) bytes, 256-aligned
+  int scratch_slots;    // CTAs the grid may use (>= 1)
   EncodeTiledFn encode;
   cudaStream_t stream;
 };
@@ -32,7 +43,7 @@ cudaError_t launch_attn_fwd(const AttnLaunch &a);
 
 cudaError_t launch_pair_bias_project(const float *pair, const float *W,
                                      float *bias, int64_t P, int num_sms,
-                                     cudaStream_t stream);
+                                     unsigned *err, cudaStream_t stream);
 
 cudaError_t launch_wait_timeout_probe(uint64_t timeout_ns, unsigned *err,
                                       cudaStream_t stream);

@@ -13,18 +13,23 @@
 //    heads.  Every row of the tile then shares one 16-position bias row block
 //    and all 8 heads consume the same K/V tile (multi-query sharing), so each
 //    K/V byte staged in shared memory feeds eight heads.
-//  * A persistent CTA per SM owns two such query tiles at a time (A and B).
-//    Warp 8 streams Q tiles and a ring of K and V tiles with TMA; warp 9
-//    issues every tcgen05.mma from one thread; warps 0-3 and 4-7 are the
-//    softmax warpgroups of tiles A and B.  The MMA order per key tile j is
-//    PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), so one warpgroup's softmax runs
-//    while the tensor core works for the other.
+//  * Work is a pair of query tiles (A and B) against a range of key tiles.
+//    One persistent CTA per SM takes a contiguous, equal share of all
+//    (pair, key tile) steps, so the grid finishes together; a pair whose key
+//    range is split between CTAs is merged exactly from the pieces' partial
+//    results by log-sum-exp (see "Split pairs" below).
+//  * Inside a CTA the producer warp streams Q tiles and a ring of K and V
+//    tiles with TMA; the MMA warp issues every tcgen05.mma from one thread;
+//    four softmax warpgroups each own one 32-key chunk of every key tile.
+//    The MMA order per key tile j is PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), so
+//    the softmax warps work on one tile while the tensor core works on the
+//    other.
 //  * Tensor memory (512 columns): S_A, S_B (fp32 128x128 logits), O_A, O_B
-//    (fp32 128x128 accumulators).  P is written as bf16 over the first 64
-//    columns of its S and fed to the PV product straight from tensor memory.
+//    (fp32 128x128 accumulators).  P is written as bf16 over part of its S
+//    and fed to the PV product straight from tensor memory.
 //  * Bias: each softmax thread owns one row, so per 128-key tile it needs
-//    just the 8 compact cells bias[h, I, 8j .. 8j+7], read from global (L2)
-//    one tile ahead and kept in registers; the 16x repeat is never built.
+//    just the compact cells of its key chunk, read from global (L2) one tile
+//    ahead and kept in registers; the 16x repeat is never built.
 //  * With a finite cap every logit lies in (-cap, cap), so the softmax uses
 //    the fixed shift m = cap (exact: softmax is shift invariant) and needs no
 //    running max and no rescaling of O.  cap > 40 (where exp(-2 cap) would
@@ -94,6 +99,7 @@ struct __align__(8) Barriers {
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
+  int range_begin, range_end;  // this CTA's (pair, key tile) steps
 };
 
 constexpr size_t kXchgBytes = 2 * 2 * kWG * 128 * sizeof(float);
@@ -105,28 +111,67 @@ struct Params {
   float *out;
   float *lse;
   unsigned *err;
+  // Split-pair scratch (see "Split pairs"): one slot per CTA.
+  float *ws_out;       // [grid][2][128][128] partial outputs
+  float *ws_lse;       // [grid][2][128] partial log-sum-exps
   int L, P;
   int nb;          // 16-position query blocks per batch item (L / 16)
-  int pairs;       // work items per batch item: ceil(nb / 2)
+  int pairs;       // query-tile pairs per batch item: ceil(nb / 2)
   int n_items;     // B * pairs
   int n_kt;        // key tiles: ceil(L / 128)
   int last_valid;  // valid keys in the last key tile (1..128)
+  int whole;       // 1: CTA ranges hold whole pairs (no split pairs)
   float qk_scale;  // multiplies q.k
   float bias_mul;  // multiplies the compact bias
   float A;         // capped modes: cap * log2(e)
 };
 
 // --------------------------------------------------------------------------
+// Work split.  The W = n_items * n_kt (pair, key tile) steps are cut into
+// gridDim.x contiguous ranges [W c / G, W (c+1) / G).  A CTA walks its range
+// as segments: one pair and a run of its key tiles.  A pair covered by more
+// than one CTA is "split"; its pieces are merged by the last one to finish.
+struct Segment {
+  int item, kb, ke;  // pair index and key tiles [kb, ke)
+};
+
+// W = n_items * n_kt <= 2^30 (checked by the launcher), so steps fit in int;
+// only the range bounds need a 64-bit product.  With p.whole the bounds are
+// rounded to whole pairs: CTA c gets pairs [n_items c / G, n_items (c+1) / G).
+__device__ __forceinline__ int range_start(const Params &p, int c) {
+  if (p.whole)
+    return static_cast<int>(static_cast<long long>(p.n_items) * c /
+                            static_cast<long long>(gridDim.x)) * p.n_kt;
+  return static_cast<int>(static_cast<long long>(p.n_items) * p.n_kt * c /
+                          static_cast<long long>(gridDim.x));
+}
+
+__device__ __forceinline__ Segment segment_at(const Params &p, int t, int end) {
+  Segment sg;
+  sg.item = t / p.n_kt;
+  sg.kb = t - sg.item * p.n_kt;
+  const int left = end - t;
+  sg.ke = left < p.n_kt - sg.kb ? sg.kb + left : p.n_kt;
+  return sg;
+}
+
+// --------------------------------------------------------------------------
 // MMA issue helpers (single thread).
+
+// Shared-memory descriptors: every operand here has 8-row groups 1 KB apart,
+// so all share one high word; the low word (start address and leading
+// offset) is built once per tile base and each K step adds a constant to its
+// start-address field (addresses stay below 2^18: no carry out of the field).
+constexpr uint32_t kDescHi = desc_sw128_hi(1024);
 
 // S[128 x 128] = Q[128 x 128] K^T: eight K=16 steps over two 64-wide halves.
 __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_addr,
                                          uint32_t k_addr) {
+  const uint32_t q_lo = desc_sw128_lo(q_addr, 16), k_lo = desc_sw128_lo(k_addr, 16);
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk) {
-    const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-    umma_ss(d_tmem, smem_desc_sw128(q_addr + off, 16, 1024),
-            smem_desc_sw128(k_addr + off, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+    const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+    umma_ss_lo(d_tmem, q_lo + off, k_lo + off, kDescHi, kIdescQK, kk > 0 ? 1u : 0u);
   }
 }
 
@@ -136,11 +181,12 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_addr,
 // are 16 KB apart, 8-key row groups 1 KB apart).
 __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t s_tmem,
                                          uint32_t v_addr, bool accumulate) {
+  const uint32_t v_lo = desc_sw128_lo(v_addr, kHalfBytes);
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk) {
-    umma_ts(d_tmem, s_tmem + 32 * (kk >> 1) + 8 * (kk & 1),
-            smem_desc_sw128(v_addr + kk * 2048, kHalfBytes, 1024), kIdescPV,
-            (accumulate || kk > 0) ? 1u : 0u);
+    umma_ts_lo(d_tmem, s_tmem + 32 * (kk >> 1) + 8 * (kk & 1),
+               v_lo + ((kk * 2048) >> 4), kDescHi, kIdescPV,
+               (accumulate || kk > 0) ? 1u : 0u);
   }
 }
 
@@ -165,9 +211,12 @@ __device__ __forceinline__ void producer(const CUtensorMap *tm_q,
   uint32_t qcount[2] = {0, 0};
   uint32_t kv = 0;
   bool ok = true;
-  for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x) {
-    const int b = w / p.pairs;
-    const int I0 = (w % p.pairs) * 2;
+  const int end = bars->range_end;
+  for (int t = bars->range_begin; t < end && ok;) {
+    const Segment sg = segment_at(p, t, end);
+    t += sg.ke - sg.kb;
+    const int b = sg.item / p.pairs;
+    const int I0 = (sg.item % p.pairs) * 2;
     const int nX = (I0 + 1 < p.nb) ? 2 : 1;
     for (int X = 0; X < nX; ++X) {
       ok = mbar_wait(&bars->q_empty[X], (qcount[X] & 1u) ^ 1u, abort, p.err,
@@ -180,15 +229,15 @@ __device__ __forceinline__ void producer(const CUtensorMap *tm_q,
                   0, b, pol_q);
       ++qcount[X];
     }
-    for (int j = 0; j < p.n_kt && ok; ++j) {
+    for (int j = sg.kb; j < sg.ke && ok; ++j) {
 #pragma unroll 1
-      for (int t = 0; t < 2; ++t) {  // t = 0: K tile j, t = 1: V tile j
+      for (int u = 0; u < 2; ++u) {  // u = 0: K tile j, u = 1: V tile j
         const uint32_t slot = kv % kStages, ph = (kv / kStages) & 1u;
         ok = mbar_wait(&bars->kv_empty[slot], ph ^ 1u, abort, p.err, kSiteProdKV);
         if (!ok) break;
         mbar_arrive_expect_tx(&bars->kv_full[slot], kTileBytes);
         uint8_t *dst = kv_s + slot * kTileBytes;
-        const CUtensorMap *tm = t == 0 ? tm_k : tm_v;
+        const CUtensorMap *tm = u == 0 ? tm_k : tm_v;
         tma_load_3d(dst, tm, &bars->kv_full[slot], 0, j * kKeys, b, pol_kv);
         tma_load_3d(dst + kHalfBytes, tm, &bars->kv_full[slot], 64, j * kKeys, b,
                     pol_kv);
@@ -214,15 +263,18 @@ __device__ __forceinline__ void mma_issuer(uint8_t *q_s, uint8_t *kv_s,
   uint32_t qcount[2] = {0, 0}, pcount[2] = {0, 0};
   uint32_t kv = 0;
   bool ok = true;
-  for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x) {
-    const int I0 = (w % p.pairs) * 2;
+  const int end = bars->range_end;
+  for (int t = bars->range_begin; t < end && ok;) {
+    const Segment sg = segment_at(p, t, end);
+    t += sg.ke - sg.kb;
+    const int I0 = (sg.item % p.pairs) * 2;
     const int nX = (I0 + 1 < p.nb) ? 2 : 1;
     for (int X = 0; X < nX && ok; ++X) {
       ok = mbar_wait(&bars->q_full[X], qcount[X] & 1u, abort, p.err, kSiteMmaQ);
       ++qcount[X];
     }
     if (!ok) break;
-    // Key tile 0: S_X(0) for both query tiles.
+    // First key tile of the segment: S_X(kb) for both query tiles.
     const uint32_t slot_k0 = kv % kStages;
     ok = mbar_wait(&bars->kv_full[slot_k0], (kv / kStages) & 1u, abort, p.err,
                    kSiteMmaKV);
@@ -233,17 +285,17 @@ __device__ __forceinline__ void mma_issuer(uint8_t *q_s, uint8_t *kv_s,
       issue_qk(tmem + X * 128, q_addr + X * kTileBytes,
                kv_addr + slot_k0 * kTileBytes);
       umma_commit(&bars->s_full[X]);
-      if (p.n_kt == 1) umma_commit(&bars->q_empty[X]);
+      if (sg.ke - sg.kb == 1) umma_commit(&bars->q_empty[X]);
     }
     umma_commit(&bars->kv_empty[slot_k0]);
 
-    for (int j = 0; j < p.n_kt && ok; ++j) {
+    for (int j = sg.kb; j < sg.ke && ok; ++j) {
       const uint32_t slot_v = kv % kStages;
       ok = mbar_wait(&bars->kv_full[slot_v], (kv / kStages) & 1u, abort, p.err,
                      kSiteMmaKV);
       if (!ok) break;
       ++kv;
-      const bool has_next = j + 1 < p.n_kt;
+      const bool has_next = j + 1 < sg.ke;
       uint32_t slot_k = 0;
       bool k_ready = false;
       for (int X = 0; X < nX; ++X) {
@@ -252,7 +304,7 @@ __device__ __forceinline__ void mma_issuer(uint8_t *q_s, uint8_t *kv_s,
         if (!ok) break;
         tc_fence_after();
         issue_pv(tmem + 256 + X * 128, tmem + X * 128,
-                 kv_addr + slot_v * kTileBytes, j > 0);
+                 kv_addr + slot_v * kTileBytes, j > sg.kb);
         if (!has_next) {
           umma_commit(&bars->o_full[X]);
           continue;
@@ -269,7 +321,7 @@ __device__ __forceinline__ void mma_issuer(uint8_t *q_s, uint8_t *kv_s,
         issue_qk(tmem + X * 128, q_addr + X * kTileBytes,
                  kv_addr + slot_k * kTileBytes);
         umma_commit(&bars->s_full[X]);
-        if (j + 2 == p.n_kt) umma_commit(&bars->q_empty[X]);
+        if (j + 2 == sg.ke) umma_commit(&bars->q_empty[X]);
       }
       if (!ok) break;
       umma_commit(&bars->kv_empty[slot_v]);
@@ -475,6 +527,15 @@ __device__ __forceinline__ bool part_tile_online(uint32_t tS, uint32_t tO, int g
   return true;
 }
 
+// --------------------------------------------------------------------------
+// Split pairs.  Every segment of a split pair finishes like a whole pair but
+// over its own key range: a normalised partial output and the partial
+// log-sum-exp.  The first segment (key tile 0) writes them to out / lse, the
+// others to the scratch slot of their CTA (a CTA starts at most one segment in
+// the middle of a pair).  attn_merge_kernel, launched right after on the same
+// stream, then merges the pieces of every split pair:
+//   lse = log sum_s exp(lse_s),  out = sum_s exp(lse_s - lse) out_s.
+
 template <int MODE>
 __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc,
                                              uint32_t tmem, const Params &p,
@@ -489,21 +550,25 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc,
   uint32_t scount[2] = {0, 0}, ocount[2] = {0, 0};
   uint32_t xmcount[2] = {0, 0}, xdcount[2] = {0, 0};
   bool ok = true;
+  const int end = bars->range_end;
 
-  for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x) {
-    const int b = w / p.pairs;
-    const int I0 = (w % p.pairs) * 2;
+  for (int t = bars->range_begin; t < end && ok;) {
+    const Segment sg = segment_at(p, t, end);
+    t += sg.ke - sg.kb;
+    const int b = sg.item / p.pairs;
+    const int I0 = (sg.item % p.pairs) * 2;
     const int nX = (I0 + 1 < p.nb) ? 2 : 1;
-    const float *brow[2];
+    const float *const brow[2] = {
+        p.bias + (static_cast<size_t>(h) * p.P + I0) * p.P,
+        p.bias + (static_cast<size_t>(h) * p.P + (I0 + (nX > 1 ? 1 : 0))) * p.P};
     float m[2], d[2] = {0.f, 0.f};
     float bn[2][2 * kChunks];
 #pragma unroll
     for (int X = 0; X < 2; ++X) {
       m[X] = (MODE == kStaticCap) ? p.A : -INFINITY;  // log2 units
-      brow[X] = p.bias + (static_cast<size_t>(h) * p.P + (I0 + (X < nX ? X : 0))) * p.P;
-      load_bias(brow[X], 0, g, p.P, bn[X]);
+      load_bias(brow[X], sg.kb, g, p.P, bn[X]);
     }
-    for (int j = 0; j < p.n_kt && ok; ++j) {
+    for (int j = sg.kb; j < sg.ke && ok; ++j) {
       const int nvalid = (j + 1 == p.n_kt) ? p.last_valid : kKeys;
 #pragma unroll
       for (int X = 0; X < 2; ++X) {
@@ -511,7 +576,7 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc,
         float bj[2 * kChunks];
 #pragma unroll
         for (int e = 0; e < 2 * kChunks; ++e) bj[e] = bn[X][e] * p.bias_mul;
-        if (j + 1 < p.n_kt) load_bias(brow[X], j + 1, g, p.P, bn[X]);
+        if (j + 1 < sg.ke) load_bias(brow[X], j + 1, g, p.P, bn[X]);
 
         ok = mbar_wait(&bars->s_full[X], scount[X] & 1u, abort, p.err, kSiteSoftS);
         ++scount[X];
@@ -536,8 +601,10 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc,
     }
     if (!ok) break;
 
-    // Epilogue: d = sum of the kWG partial sums; out = O / d (this
-    // warpgroup's 32*kChunks columns of the row), lse from warpgroup 0.
+    // Epilogue: d = sum of the kWG partial sums; out = O / d over this
+    // segment's keys (this warpgroup's 32*kChunks columns of the row) and
+    // lse, to out / lse or, for a later piece of a split pair, to this CTA's
+    // scratch slot.
 #pragma unroll
     for (int X = 0; X < 2; ++X) {
       if (X >= nX) break;
@@ -555,7 +622,17 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc,
       const size_t row = (static_cast<size_t>(b) * kH + h) * p.L +
                          static_cast<size_t>(I0 + X) * 16 + il;
       const int c0 = 32 * kChunks * g;
-      float4 *orow = reinterpret_cast<float4 *>(p.out + row * kD + c0);
+      float *orow_base;
+      float *lse_dst;
+      if (sg.kb == 0) {
+        orow_base = p.out + row * kD;
+        lse_dst = p.lse + row;
+      } else {
+        const size_t slot = (static_cast<size_t>(blockIdx.x) * 2 + X) * 128 + r;
+        orow_base = p.ws_out + slot * kD;
+        lse_dst = p.ws_lse + slot;
+      }
+      float4 *orow = reinterpret_cast<float4 *>(orow_base + c0);
       const uint32_t tO = tmem + 256 + X * 128 + lane_base + c0;
 #pragma unroll 1
       for (int c = 0; c < kChunks; ++c) {
@@ -570,7 +647,7 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc,
                                         __uint_as_float(o[4 * e + 3]) * inv_d);
         }
       }
-      if (g == 0) p.lse[row] = (m[X] + lg2_approx(dsum)) * kLn2;
+      if (g == 0) *lse_dst = (m[X] + lg2_approx(dsum)) * kLn2;
       tc_fence_before();
     }
   }
@@ -607,6 +684,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
+    bars->range_begin = range_start(p, blockIdx.x);
+    bars->range_end = range_start(p, blockIdx.x + 1);
     fence_mbar_init();
   }
   if (warp == kWarpLoad && lane_id() == 0) {
@@ -641,6 +720,74 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+}
+
+// --------------------------------------------------------------------------
+// Split-pair merge.  One block per CTA boundary; the block whose boundary is
+// the first one inside a pair merges that pair.  Thread t takes query tile
+// t / 128 and row t % 128 and merges the whole 128-column row, so it reads
+// the first piece's lse before it overwrites it.
+constexpr int kMergeThreads = 256;
+
+__global__ void __launch_bounds__(kMergeThreads)
+    attn_merge_kernel(const Params p, int grid) {
+  const int c = blockIdx.x + 1;  // boundary between CTA c - 1 and CTA c
+  const int W = p.n_items * p.n_kt;
+  auto start = [&](int cc) {
+    return static_cast<int>(static_cast<long long>(W) * cc / grid);
+  };
+  const int tb = start(c);
+  if (tb % p.n_kt == 0) return;  // the boundary falls between pairs
+  const int item = tb / p.n_kt;
+  const int prev = start(c - 1);
+  if (c > 1 && prev / p.n_kt == item && prev % p.n_kt != 0) return;  // merged by an earlier block
+  auto owner = [&](int t) {
+    return static_cast<int>(((static_cast<long long>(t) + 1) * grid - 1) / W);
+  };
+  const int c_first = owner(item * p.n_kt);
+  const int n_seg = owner(item * p.n_kt + p.n_kt - 1) - c_first + 1;
+  const int b = item / p.pairs;
+  const int I0 = (item % p.pairs) * 2;
+  const int nX = (I0 + 1 < p.nb) ? 2 : 1;
+  const int X = threadIdx.x >> 7, r = threadIdx.x & 127;
+  if (X >= nX) return;
+  const int h = r >> 4, il = r & 15;
+  const size_t row = (static_cast<size_t>(b) * kH + h) * p.L +
+                     static_cast<size_t>(I0 + X) * 16 + il;
+  auto slot = [&](int s) {
+    return (static_cast<size_t>(c_first + s) * 2 + X) * 128 + r;
+  };
+  float M = -INFINITY;
+  for (int s = 0; s < n_seg; ++s)
+    M = fmaxf(M, s == 0 ? p.lse[row] : p.ws_lse[slot(s)]);
+  float sum = 0.f;
+  for (int s = 0; s < n_seg; ++s)
+    sum += ex2_approx(((s == 0 ? p.lse[row] : p.ws_lse[slot(s)]) - M) * kLog2e);
+  const float lse = M + lg2_approx(sum) * kLn2;
+  float4 *dst = reinterpret_cast<float4 *>(p.out + row * kD);
+#pragma unroll 1
+  for (int part = 0; part < kD / 16; ++part) {
+    float4 acc[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < n_seg; ++s) {
+      const float l = s == 0 ? p.lse[row] : p.ws_lse[slot(s)];
+      const float wgt = ex2_approx((l - lse) * kLog2e);
+      const float4 *src = reinterpret_cast<const float4 *>(
+          s == 0 ? p.out + row * kD : p.ws_out + slot(s) * kD);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float4 v = src[part * 4 + e];
+        acc[e].x = fmaf(wgt, v.x, acc[e].x);
+        acc[e].y = fmaf(wgt, v.y, acc[e].y);
+        acc[e].z = fmaf(wgt, v.z, acc[e].z);
+        acc[e].w = fmaf(wgt, v.w, acc[e].w);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dst[part * 4 + e] = acc[e];
+  }
+  p.lse[row] = lse;
 }
 
 }  // namespace attn
@@ -738,12 +885,35 @@ cudaError_t launch_attn_fwd(const AttnLaunch &a) {
     p.bias_mul = 1.0f / cap;
     p.A = cap * kLog2e;
   }
-  const int grid = p.n_items < a.num_sms ? p.n_items : a.num_sms;
-  switch (mode) {
-    case kStaticCap: return launch_mode<kStaticCap>(tq, tk, tv, p, grid, a.stream);
-    case kOnlineCap: return launch_mode<kOnlineCap>(tq, tk, tv, p, grid, a.stream);
-    default: return launch_mode<kNoCap>(tq, tk, tv, p, grid, a.stream);
+  // One CTA per SM, never more CTAs than (pair, key tile) steps or scratch
+  // slots.  Whole pairs per CTA unless that leaves the grid badly balanced:
+  // a split pair costs a second pass over its rows (partial results, then
+  // the merge), so whole pairs win while the busiest CTA's extra work stays
+  // below kSplitGain pairs.
+  const long long steps = static_cast<long long>(p.n_items) * p.n_kt;
+  if (steps > (1ll << 30)) return cudaErrorInvalidValue;
+  int grid = a.num_sms < a.scratch_slots ? a.num_sms : a.scratch_slots;
+  if (steps < grid) grid = static_cast<int>(steps);
+  if (grid < 1) return cudaErrorInvalidValue;
+  {
+    constexpr double kSplitGain = 0.5;
+    const long long per = (p.n_items + grid - 1) / grid;  // pairs, busiest CTA
+    const double even = static_cast<double>(p.n_items) / grid;
+    p.whole = (per - even <= kSplitGain) ? 1 : 0;
+    if (p.whole && p.n_items < grid) grid = p.n_items;
   }
+  char *base = static_cast<char *>(a.scratch);
+  p.ws_out = reinterpret_cast<float *>(base);
+  p.ws_lse = reinterpret_cast<float *>(base + a.scratch_slots * kAttnSlotOutBytes);
+  cudaError_t e;
+  switch (mode) {
+    case kStaticCap: e = launch_mode<kStaticCap>(tq, tk, tv, p, grid, a.stream); break;
+    case kOnlineCap: e = launch_mode<kOnlineCap>(tq, tk, tv, p, grid, a.stream); break;
+    default: e = launch_mode<kNoCap>(tq, tk, tv, p, grid, a.stream); break;
+  }
+  if (e != cudaSuccess || grid < 2 || p.whole) return e;
+  attn_merge_kernel<<<grid - 1, kMergeThreads, 0, a.stream>>>(p, grid);
+  return cudaGetLastError();
 }
 
 }  // namespace ag
