@@ -45,7 +45,9 @@ typedef enum {
     AG_ERR_VALUE = 5,       /* a scalar argument is out of range (cap)        */
     AG_ERR_CUDA = 6,        /* a CUDA runtime or driver call failed           */
     AG_ERR_ALIAS = 7,       /* an output buffer overlaps an input buffer      */
-    AG_ERR_DEVICE = 8       /* the device error word is set (see below)       */
+    AG_ERR_DEVICE = 8,      /* the device error word is set (see below)       */
+    AG_ERR_SCRATCH = 9      /* ag_attn_fwd_noalloc: the call needs more scratch
+                               than its static buffer holds                   */
 } ag_status;
 
 /* Static, human-readable name of a status code (never NULL). */
@@ -114,6 +116,34 @@ ag_status ag_attn_fwd(const void *q, const void *k, const void *v,
                       const float *bias, int64_t B, int64_t H, int64_t L,
                       int64_t D, int64_t block, float cap, float *out,
                       float *lse, void *stream);
+
+/*
+ * ag_attn_fwd_noalloc -- ag_attn_fwd for callers that cannot allocate device
+ * memory (the pages have no counterpart; this is a library convenience).
+ *
+ * Same arguments, checks, results and stream behaviour as ag_attn_fwd, but
+ * it never calls cudaMalloc or cudaFree: its split-pair scratch is a static
+ * device array compiled into the library, 148 slots of 132,096 bytes
+ * (19,550,208 bytes), which every GPU that loads the library holds until the
+ * process exits.  Useful where an allocation is not allowed or not wanted,
+ * e.g. code that must not touch the allocator while a CUDA graph is being
+ * captured, or a framework that has handed all device memory to its own pool.
+ *
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - Returns AG_ERR_SCRATCH, launching nothing, when the call would use more
+ *     than 148 slots (one per CTA of its grid: min(SM count, work steps)),
+ *     i.e. on a device with more than 148 SMs.
+ *   - Every call shares the one array and it keeps the last call's contents;
+ *     nothing in it needs to start at zero.  Calls that overlap on the GPU
+ *     (two streams at once, or together with ag_attn_fwd's kernels on another
+ *     stream of the same device) race on it and must not be issued.
+ */
+ag_status ag_attn_fwd_noalloc(const void *q, const void *k, const void *v,
+                              const float *bias, int64_t B, int64_t H, int64_t L,
+                              int64_t D, int64_t block, float cap, float *out,
+                              float *lse, void *stream);
 
 /*
  * Device error word.  Every wait inside the kernels is bounded (about one

@@ -28,7 +28,7 @@ AG_OK = 0
 STATUS_NAMES = {
     0: "AG_OK", 1: "AG_ERR_NULL", 2: "AG_ERR_SHAPE", 3: "AG_ERR_ALIGN",
     4: "AG_ERR_UNSUPPORTED", 5: "AG_ERR_VALUE", 6: "AG_ERR_CUDA",
-    7: "AG_ERR_ALIAS", 8: "AG_ERR_DEVICE",
+    7: "AG_ERR_ALIAS", 8: "AG_ERR_DEVICE", 9: "AG_ERR_SCRATCH",
 }
 
 
@@ -56,6 +56,9 @@ def _load() -> ctypes.CDLL:
     lib.ag_attn_fwd.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, f32,
                                 vp, vp, vp]
     lib.ag_attn_fwd.restype = ctypes.c_int
+    lib.ag_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64,
+                                        f32, vp, vp, vp]
+    lib.ag_attn_fwd_noalloc.restype = ctypes.c_int
     lib.ag_device_error.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int),
                                     ctypes.c_int]
     lib.ag_device_error.restype = ctypes.c_int
@@ -141,6 +144,27 @@ def ag_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                          lse.data_ptr(), _stream_ptr(stream))
     if st != AG_OK:
         raise AgError("ag_attn_fwd", st)
+    return out, lse
+
+
+def ag_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                        bias: torch.Tensor, out: torch.Tensor, lse: torch.Tensor,
+                        cap: float = 5.0, block: int = 16, stream=None):
+    """ag_attn_fwd through the entry point that allocates nothing (static
+    scratch inside the library).  The caller passes the outputs."""
+    _check(q, "q", torch.bfloat16, 4)
+    _check(k, "k", torch.bfloat16, 3)
+    _check(v, "v", torch.bfloat16, 3)
+    _check(bias, "bias", torch.float32, 3)
+    _check(out, "out", torch.float32, 4)
+    _check(lse, "lse", torch.float32, 3)
+    B, H, L, D = q.shape
+    st = lib.ag_attn_fwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                 bias.data_ptr(), B, H, L, D, int(block),
+                                 float(cap), out.data_ptr(), lse.data_ptr(),
+                                 _stream_ptr(stream))
+    if st != AG_OK:
+        raise AgError("ag_attn_fwd_noalloc", st)
     return out, lse
 
 

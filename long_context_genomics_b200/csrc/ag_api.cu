@@ -27,6 +27,7 @@ struct DeviceInfo {
   int num_sms = 0;
   unsigned *err = nullptr;  // device address of g_device_error_word
   void *scratch = nullptr;  // attention split-pair scratch (one slot per SM)
+  void *static_scratch = nullptr;  // device address of g_static_attn_scratch
 };
 
 std::mutex g_mu;
@@ -93,6 +94,28 @@ ag_status get_encoder(EncodeTiledFn *fn) {
   return AG_OK;
 }
 
+// Scratch for ag_attn_fwd_noalloc: the same split-pair slots as the
+// allocated scratch, for at most kStaticScratchSlots CTAs, in a file-scope
+// array that every device loading this library holds until the process exits.
+constexpr int kStaticScratchSlots = 148;
+constexpr size_t kStaticScratchBytes =
+    kStaticScratchSlots * (kAttnSlotOutBytes + kAttnSlotLseBytes);
+static __device__ __align__(256) unsigned char g_static_attn_scratch[kStaticScratchBytes];
+
+// Device address of g_static_attn_scratch for the current device, looked up
+// once per device (host code may not use the symbol itself as an address).
+ag_status static_scratch(DeviceInfo *d, void **out) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!d->static_scratch) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_attn_scratch) != cudaSuccess || !p)
+      return AG_ERR_CUDA;
+    d->static_scratch = p;
+  }
+  *out = d->static_scratch;
+  return AG_OK;
+}
+
 bool aligned(const void *p, uintptr_t a) {
   return (reinterpret_cast<uintptr_t>(p) % a) == 0;
 }
@@ -149,6 +172,8 @@ const char *ag_status_string(int s) {
     case AG_ERR_CUDA: return "AG_ERR_CUDA: a CUDA call failed";
     case AG_ERR_ALIAS: return "AG_ERR_ALIAS: an output overlaps an input";
     case AG_ERR_DEVICE: return "AG_ERR_DEVICE: the device error word is set";
+    case AG_ERR_SCRATCH:
+      return "AG_ERR_SCRATCH: the call needs more scratch than the static buffer holds";
     default: return "unknown ag_status";
   }
 }
@@ -227,6 +252,69 @@ ag_status ag_attn_fwd(const void *q, const void *k, const void *v,
   a.num_sms = dev->num_sms;
   a.scratch = scratch;
   a.scratch_slots = dev->num_sms;
+  a.encode = enc;
+  a.stream = static_cast<cudaStream_t>(stream);
+  return ag::from_cuda(ag::launch_attn_fwd(a));
+}
+
+ag_status ag_attn_fwd_noalloc(const void *q, const void *k, const void *v,
+                              const float *bias, int64_t B, int64_t H, int64_t L,
+                              int64_t D, int64_t block, float cap, float *out,
+                              float *lse, void *stream) {
+  // The same checks, in the same order, as ag_attn_fwd.
+  if (B < 0 || H <= 0 || L < 0 || D <= 0 || block <= 0) return AG_ERR_SHAPE;
+  if (L % block != 0) return AG_ERR_SHAPE;
+  if (std::isnan(cap) || !(cap > 0.0f)) return AG_ERR_VALUE;
+  if (H != 8 || D != 128 || block != 16 || L > 65536) return AG_ERR_UNSUPPORTED;
+  if (B > 0 && L > 0 && B * L > (int64_t(1) << 28)) return AG_ERR_UNSUPPORTED;
+  if (B > 0 && L > 0 && B * ((L / 16 + 1) / 2) * ((L + 127) / 128) > (int64_t(1) << 30))
+    return AG_ERR_UNSUPPORTED;
+  if (B == 0 || L == 0) return AG_OK;
+  if (!q || !k || !v || !bias || !out || !lse) return AG_ERR_NULL;
+  if (!ag::aligned(q, 16) || !ag::aligned(k, 16) || !ag::aligned(v, 16) ||
+      !ag::aligned(bias, 4) || !ag::aligned(out, 16) || !ag::aligned(lse, 4))
+    return AG_ERR_ALIGN;
+  const uint64_t P = static_cast<uint64_t>(L / block);
+  const uint64_t qb = static_cast<uint64_t>(B) * H * L * D * 2;
+  const uint64_t kb = static_cast<uint64_t>(B) * L * D * 2;
+  const uint64_t bb = static_cast<uint64_t>(H) * P * P * 4;
+  const uint64_t ob = static_cast<uint64_t>(B) * H * L * D * 4;
+  const uint64_t lb = static_cast<uint64_t>(B) * H * L * 4;
+  const void *ins[4] = {q, k, v, bias};
+  const uint64_t insz[4] = {qb, kb, kb, bb};
+  for (int t = 0; t < 4; ++t)
+    if (ag::overlap(out, ob, ins[t], insz[t]) || ag::overlap(lse, lb, ins[t], insz[t]))
+      return AG_ERR_ALIAS;
+  if (ag::overlap(out, ob, lse, lb)) return AG_ERR_ALIAS;
+  ag::DeviceInfo *dev = nullptr;
+  ag_status st = ag::device_info(&dev);
+  if (st != AG_OK) return st;
+  // One scratch slot per CTA; the grid is one CTA per SM (fewer for tiny
+  // problems).  A device whose grid would need more slots than the static
+  // buffer holds is refused rather than given a slower grid.
+  const int64_t steps = B * ((L / 16 + 1) / 2) * ((L + 127) / 128);
+  const int64_t slots = steps < dev->num_sms ? steps : dev->num_sms;
+  if (slots > ag::kStaticScratchSlots) return AG_ERR_SCRATCH;
+  ag::EncodeTiledFn enc = nullptr;
+  st = ag::get_encoder(&enc);
+  if (st != AG_OK) return st;
+  void *scratch = nullptr;
+  st = ag::static_scratch(dev, &scratch);
+  if (st != AG_OK) return st;
+  ag::AttnLaunch a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.bias = bias;
+  a.out = out;
+  a.lse = lse;
+  a.B = B;
+  a.L = L;
+  a.cap = cap;
+  a.err = dev->err;
+  a.num_sms = dev->num_sms;
+  a.scratch = scratch;
+  a.scratch_slots = ag::kStaticScratchSlots;
   a.encode = enc;
   a.stream = static_cast<cudaStream_t>(stream);
   return ag::from_cuda(ag::launch_attn_fwd(a));
