@@ -353,12 +353,22 @@ struct Xchg {
   float mpart[2][kWG][128];
 };
 
+// Softmax-side barriers count warps: each warp arrives once, from lane 0,
+// after __syncwarp has ordered its lanes' prior work (one arrival per warp
+// instead of 32 keeps the mbarrier off the shared-memory pipe).
+constexpr uint32_t kSoftWarps = kSoftThreads / 32;
+
+__device__ __forceinline__ void warp_arrive(uint64_t *bar) {
+  __syncwarp();
+  if (lane_id() == 0) mbar_arrive(bar);
+}
+
 // Publish this thread's value, then wait (bounded) until every softmax thread
-// has published its own.  The mbarrier's arrive/wait order the shared-memory
-// writes before the partners' reads.
+// has published its own.  The warp barrier and the mbarrier's arrive/wait
+// order the shared-memory writes before the partners' reads.
 __device__ __forceinline__ bool exchange(uint64_t *bar, uint32_t &count,
                                          volatile int *abort, unsigned *err) {
-  mbar_arrive(bar);
+  warp_arrive(bar);
   const bool ok = mbar_wait(bar, count & 1u, abort, err, kSiteXchg);
   ++count;
   return __all_sync(0xffffffffu, ok);
@@ -596,7 +606,7 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc,
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bars->p_full[X]);
+        warp_arrive(&bars->p_full[X]);
       }
     }
     if (!ok) break;
@@ -673,9 +683,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->q_full[X], 1);
       mbar_init(&bars->q_empty[X], 1);
       mbar_init(&bars->s_full[X], 1);
-      mbar_init(&bars->p_full[X], kSoftThreads);
-      mbar_init(&bars->xm[X], kSoftThreads);
-      mbar_init(&bars->xd[X], kSoftThreads);
+      mbar_init(&bars->p_full[X], kSoftWarps);
+      mbar_init(&bars->xm[X], kSoftWarps);
+      mbar_init(&bars->xd[X], kSoftWarps);
       mbar_init(&bars->o_full[X], 1);
     }
     for (int s = 0; s < kStages; ++s) {
