@@ -84,10 +84,11 @@ def profiled_traffic():
         fields = {}
         with open(path) as f:
             for line in f:
-                if ":" in line and line.strip().startswith(("traffic_bytes_per_launch",
-                                                             "kernel_source_sha256")):
-                    k, v = line.split(":", 1)
-                    fields[k.strip(" -*`")] = v.strip(" `\n")
+                item = line.strip().lstrip("-* ").strip("`")
+                if ":" in item and item.startswith(("traffic_bytes_per_launch",
+                                                    "kernel_source_sha256")):
+                    k, v = item.split(":", 1)
+                    fields[k.strip(" `")] = v.strip(" `")
         if fields.get("kernel_source_sha256") == want and "traffic_bytes_per_launch" in fields:
             try:
                 return float(fields["traffic_bytes_per_launch"])
@@ -219,6 +220,29 @@ def run_reference(args, rank: int, world: int) -> None:
 
 
 # --------------------------------------------------------------------------
+# Multi-rank plumbing (one process per GPU, launched by torchrun).  The ranks
+# share no data: each runs its own independent problem, so the only
+# collectives are the timing reductions below.
+def rank_workload(base, rank: int):
+    """Rank r's problem: the same shapes with its own input seed."""
+    return dataclasses.replace(base, seed=base.seed + 1000 * rank)
+
+
+def max_over_ranks(seconds: float, device, world: int) -> float:
+    """The slowest rank's time: every rank calls this with its own device
+    time (a collective, so all ranks must call it in the same order)."""
+    t = torch.tensor([seconds], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_rate(world: int, units_per_step: float, steps: int, seconds: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest
+    rank's time (weak scaling: every rank does the same work per step)."""
+    return world * units_per_step * steps / seconds
+
+
 def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     import long_context_genomics_b200 as ag
 
@@ -227,7 +251,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     torch.cuda.set_device(dev)
     base = WORKLOAD
     # Each rank runs its own independent problem (own seed).
-    w = dataclasses.replace(base, seed=base.seed + 1000 * rank)
+    w = rank_workload(base, rank)
     host = ag_inputs.make_inputs(w)
     pinned = {n: t.pin_memory() for n, t in host.items()}
     d = {n: t.to(dev) for n, t in host.items()}
@@ -274,10 +298,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     step_ms = [e[0].elapsed_time(e[2]) for e in ev]
     proj_ms = [e[0].elapsed_time(e[1]) for e in ev]
     attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
-    total_ms = torch.tensor([sum(step_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(total_ms, op=dist.ReduceOp.MAX)
-    total_s = float(total_ms.item()) / 1e3
+    total_s = max_over_ranks(sum(step_ms) / 1e3, dev, world)
     assert ag.ag_device_error(local_rank) == 0
 
     # ---- end to end through the public API with host buffers ---------------
@@ -295,18 +316,14 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         lse_h.copy_(lse, non_blocking=True)
         ee[i][1].record(stream)
     barrier()
-    e2e_ms = torch.tensor([sum(e[0].elapsed_time(e[1]) for e in ee)], dtype=torch.float64,
-                          device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_s = float(e2e_ms.item()) / 1e3
+    e2e_s = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ee) / 1e3, dev, world)
     assert math.isfinite(float(lse_h[0, 0, 0])) and ag.ag_device_error(local_rank) == 0
 
     if rank != 0:
         return
     flops = w.attn_flops()
     pk = peaks()
-    value = world * flops * K / total_s / 1e12
+    value = aggregate_rate(world, flops, K, total_s) / 1e12
     attn_mean_s = statistics.mean(attn_ms) / 1e3
     achieved = flops / attn_mean_s / 1e12
     proj_mean_s = statistics.mean(proj_ms) / 1e3
@@ -319,7 +336,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
                    if world > 1 else "single GPU"},
         "pct_of_peak": 100.0 * (value / world) / pk["bf16_tflops"],
         "peak_source": pk["source"],
-        "e2e": {"value": world * flops * K / e2e_s / 1e12, "unit": UNIT,
+        "e2e": {"value": aggregate_rate(world, flops, K, e2e_s) / 1e12, "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 2 * K,
         "roofline": {"kernel": "attn_fwd_kernel", "bound": "tensor", "achieved": achieved,

@@ -210,7 +210,7 @@ ag_status ag_attn_fwd(const void *q, const void *k, const void *v,
   if (H != 8 || D != 128 || block != 16 || L > 65536) return AG_ERR_UNSUPPORTED;
   if (B > 0 && L > 0 && B * L > (int64_t(1) << 28)) return AG_ERR_UNSUPPORTED;
   // Work steps (pairs of query tiles x key tiles) must stay below 2^30.
-  if (B > 0 && L > 0 && B * ((L / 16 + 1) / 2) * ((L + 127) / 128) > (int64_t(1) << 30))
+  if (B > 0 && L > 0 && ag::attn_work_steps(B, L) > (int64_t(1) << 30))
     return AG_ERR_UNSUPPORTED;
   if (B == 0 || L == 0) return AG_OK;
   if (!q || !k || !v || !bias || !out || !lse) return AG_ERR_NULL;
@@ -267,7 +267,7 @@ ag_status ag_attn_fwd_noalloc(const void *q, const void *k, const void *v,
   if (std::isnan(cap) || !(cap > 0.0f)) return AG_ERR_VALUE;
   if (H != 8 || D != 128 || block != 16 || L > 65536) return AG_ERR_UNSUPPORTED;
   if (B > 0 && L > 0 && B * L > (int64_t(1) << 28)) return AG_ERR_UNSUPPORTED;
-  if (B > 0 && L > 0 && B * ((L / 16 + 1) / 2) * ((L + 127) / 128) > (int64_t(1) << 30))
+  if (B > 0 && L > 0 && ag::attn_work_steps(B, L) > (int64_t(1) << 30))
     return AG_ERR_UNSUPPORTED;
   if (B == 0 || L == 0) return AG_OK;
   if (!q || !k || !v || !bias || !out || !lse) return AG_ERR_NULL;
@@ -292,7 +292,7 @@ ag_status ag_attn_fwd_noalloc(const void *q, const void *k, const void *v,
   // One scratch slot per CTA; the grid is one CTA per SM (fewer for tiny
   // problems).  A device whose grid would need more slots than the static
   // buffer holds is refused rather than given a slower grid.
-  const int64_t steps = B * ((L / 16 + 1) / 2) * ((L + 127) / 128);
+  const int64_t steps = ag::attn_work_steps(B, L);
   const int64_t slots = steps < dev->num_sms ? steps : dev->num_sms;
   if (slots > ag::kStaticScratchSlots) return AG_ERR_SCRATCH;
   ag::EncodeTiledFn enc = nullptr;

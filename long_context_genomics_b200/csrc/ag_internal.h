@@ -23,6 +23,14 @@ inline size_t attn_scratch_bytes(int slots) {
   return static_cast<size_t>(slots) * (kAttnSlotOutBytes + kAttnSlotLseBytes);
 }
 
+// Keys per K/V tile of the attention kernel, and its work steps: pairs of
+// 128-row query tiles (16 positions x 8 heads each) times key tiles.  The
+// kernel indexes steps with int, so callers keep this at or below 2^30.
+constexpr int64_t kAttnKeyTile = 128;
+inline int64_t attn_work_steps(int64_t B, int64_t L) {
+  return B * ((L / 16 + 1) / 2) * ((L + kAttnKeyTile - 1) / kAttnKeyTile);
+}
+
 struct AttnLaunch {
   const void *q, *k, *v;
   const float *bias;

@@ -45,7 +45,8 @@ namespace attn {
 
 constexpr int kH = 8;
 constexpr int kD = 128;
-constexpr int kKeys = 128;                  // keys per K/V tile
+constexpr int kKeys = static_cast<int>(kAttnKeyTile);  // keys per K/V tile
+static_assert(kKeys == 128, "the tile layout below assumes 128-key tiles");
 constexpr int kStages = 4;                  // K/V ring slots
 constexpr int kTileBytes = 128 * 128 * 2;   // one Q, K or V tile (bf16)
 constexpr int kHalfBytes = kTileBytes / 2;  // one 64-wide (128-byte) half
@@ -65,11 +66,13 @@ constexpr int kWarpLoad = 4 * kWG;
 constexpr int kWarpMma = 4 * kWG + 1;
 // Registers per thread: the launch gives every thread kRegsLaunch (the cap
 // for this block size, which ptxas allocates when setmaxnreg is present; the
-// launcher checks it); the producer warpgroup then drops to kRegsLow and the
-// softmax warpgroups rise to kRegsHigh.
+// launcher checks it).  The producer warpgroup then drops to kRegsLow and,
+// where kRegsHigh exceeds the launch count, the softmax warpgroups rise to
+// it.  (With four softmax warpgroups the softmax needs no more than the
+// launch count, and a producer cap below 80 makes the MMA warp spill.)
 constexpr uint32_t kRegsLaunch = kWG == 2 ? 168 : 96;
-constexpr uint32_t kRegsLow = kWG == 2 ? 88 : 64;
-constexpr uint32_t kRegsHigh = kWG == 2 ? 208 : 104;
+constexpr uint32_t kRegsLow = kWG == 2 ? 88 : 80;
+constexpr uint32_t kRegsHigh = kWG == 2 ? 208 : 96;
 static_assert(kSoftThreads * kRegsHigh + 128 * kRegsLow <= kThreads * kRegsLaunch,
               "register split exceeds the launch allocation");
 constexpr uint32_t kTmemCols = 512;
@@ -218,7 +221,9 @@ __device__ __forceinline__ void producer(const CUtensorMap *tm_q,
     const int b = sg.item / p.pairs;
     const int I0 = (sg.item % p.pairs) * 2;
     const int nX = (I0 + 1 < p.nb) ? 2 : 1;
-    for (int X = 0; X < nX; ++X) {
+#pragma unroll
+    for (int X = 0; X < 2; ++X) {
+      if (X >= nX) break;
       ok = mbar_wait(&bars->q_empty[X], (qcount[X] & 1u) ^ 1u, abort, p.err,
                      kSiteProdQ);
       if (!ok) break;
@@ -269,42 +274,49 @@ __device__ __forceinline__ void mma_issuer(uint8_t *q_s, uint8_t *kv_s,
     t += sg.ke - sg.kb;
     const int I0 = (sg.item % p.pairs) * 2;
     const int nX = (I0 + 1 < p.nb) ? 2 : 1;
-    for (int X = 0; X < nX && ok; ++X) {
+#pragma unroll
+    for (int X = 0; X < 2; ++X) {
+      if (X >= nX || !ok) break;
       ok = mbar_wait(&bars->q_full[X], qcount[X] & 1u, abort, p.err, kSiteMmaQ);
       ++qcount[X];
     }
     if (!ok) break;
     // First key tile of the segment: S_X(kb) for both query tiles.
+    const int n = sg.ke - sg.kb;
     const uint32_t slot_k0 = kv % kStages;
     ok = mbar_wait(&bars->kv_full[slot_k0], (kv / kStages) & 1u, abort, p.err,
                    kSiteMmaKV);
     if (!ok) break;
     ++kv;
     tc_fence_after();
-    for (int X = 0; X < nX; ++X) {
+#pragma unroll
+    for (int X = 0; X < 2; ++X) {
+      if (X >= nX) break;
       issue_qk(tmem + X * 128, q_addr + X * kTileBytes,
                kv_addr + slot_k0 * kTileBytes);
       umma_commit(&bars->s_full[X]);
-      if (sg.ke - sg.kb == 1) umma_commit(&bars->q_empty[X]);
+      if (n == 1) umma_commit(&bars->q_empty[X]);
     }
     umma_commit(&bars->kv_empty[slot_k0]);
 
-    for (int j = sg.kb; j < sg.ke && ok; ++j) {
+    for (int i = 0; i < n && ok; ++i) {
       const uint32_t slot_v = kv % kStages;
       ok = mbar_wait(&bars->kv_full[slot_v], (kv / kStages) & 1u, abort, p.err,
                      kSiteMmaKV);
       if (!ok) break;
       ++kv;
-      const bool has_next = j + 1 < sg.ke;
+      const bool has_next = i + 1 < n;
       uint32_t slot_k = 0;
       bool k_ready = false;
-      for (int X = 0; X < nX; ++X) {
+#pragma unroll
+      for (int X = 0; X < 2; ++X) {
+        if (X >= nX) break;
         ok = mbar_wait(&bars->p_full[X], pcount[X] & 1u, abort, p.err, kSiteMmaP);
         ++pcount[X];
         if (!ok) break;
         tc_fence_after();
         issue_pv(tmem + 256 + X * 128, tmem + X * 128,
-                 kv_addr + slot_v * kTileBytes, j > sg.kb);
+                 kv_addr + slot_v * kTileBytes, i > 0);
         if (!has_next) {
           umma_commit(&bars->o_full[X]);
           continue;
@@ -321,7 +333,7 @@ __device__ __forceinline__ void mma_issuer(uint8_t *q_s, uint8_t *kv_s,
         issue_qk(tmem + X * 128, q_addr + X * kTileBytes,
                  kv_addr + slot_k * kTileBytes);
         umma_commit(&bars->s_full[X]);
-        if (j + 2 == sg.ke) umma_commit(&bars->q_empty[X]);
+        if (i + 2 == n) umma_commit(&bars->q_empty[X]);
       }
       if (!ok) break;
       umma_commit(&bars->kv_empty[slot_v]);
@@ -474,7 +486,7 @@ __device__ __forceinline__ void chunk_logits(const uint32_t (&s)[32], float b0,
 // warpgroup's columns of O when the maximum grows past the lazy threshold.
 template <int MODE>
 __device__ __forceinline__ bool part_tile_online(uint32_t tS, uint32_t tO, int g,
-                                                 int r, int X, int j,
+                                                 int r, int X, int i,
                                                  const float (&bj)[2 * kChunks],
                                                  const Params &p, int nvalid,
                                                  Xchg *xc, uint64_t *xbar,
@@ -503,8 +515,9 @@ __device__ __forceinline__ bool part_tile_online(uint32_t tS, uint32_t tO, int g
     m = mt;
     d *= factor;
   }
-  if (j > 0 && __any_sync(0xffffffffu, factor != 1.f)) {
-    // O(j-1) is complete: s_full(j) was committed after PV(j-1).
+  if (i > 0 && __any_sync(0xffffffffu, factor != 1.f)) {
+    // The previous tile's PV into O is complete: this tile's s_full was
+    // committed after it.  (Before the first tile O holds nothing yet.)
 #pragma unroll 1
     for (int c = 0; c < kChunks; ++c) {
       uint32_t o[32];
@@ -578,7 +591,7 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc,
       m[X] = (MODE == kStaticCap) ? p.A : -INFINITY;  // log2 units
       load_bias(brow[X], sg.kb, g, p.P, bn[X]);
     }
-    for (int j = sg.kb; j < sg.ke && ok; ++j) {
+    for (int j = sg.kb, i = 0; j < sg.ke && ok; ++j, ++i) {
       const int nvalid = (j + 1 == p.n_kt) ? p.last_valid : kKeys;
 #pragma unroll
       for (int X = 0; X < 2; ++X) {
@@ -600,7 +613,7 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc,
             d[X] += part_tile_static<true>(tS, g, bj, sc, ap, an, nvalid);
         } else {
           const uint32_t tO = tmem + 256 + X * 128 + lane_base;
-          ok = part_tile_online<MODE>(tS, tO, g, r, X, j, bj, p, nvalid, xc,
+          ok = part_tile_online<MODE>(tS, tO, g, r, X, i, bj, p, nvalid, xc,
                                       &bars->xm[X], xmcount[X], abort, m[X], d[X]);
           if (!ok) break;
         }
@@ -720,7 +733,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     else if (warp == kWarpMma && lane_id() == 0)
       mma_issuer(q_s, kv_s, bars, tmem, p, abort);
   } else {
-    regs_inc<kRegsHigh>();
+    if constexpr (kRegsHigh > kRegsLaunch) regs_inc<kRegsHigh>();
     softmax_role<MODE>(bars, xc, tmem, p, abort);
   }
   __syncwarp();
@@ -901,7 +914,8 @@ cudaError_t launch_attn_fwd(const AttnLaunch &a) {
   // the merge), so whole pairs win while the busiest CTA's extra work stays
   // below kSplitGain pairs.
   const long long steps = static_cast<long long>(p.n_items) * p.n_kt;
-  if (steps > (1ll << 30)) return cudaErrorInvalidValue;
+  if (steps != attn_work_steps(B, L) || steps > (1ll << 30))
+    return cudaErrorInvalidValue;
   int grid = a.num_sms < a.scratch_slots ? a.num_sms : a.scratch_slots;
   if (steps < grid) grid = static_cast<int>(steps);
   if (grid < 1) return cudaErrorInvalidValue;

@@ -60,6 +60,8 @@ def _attn(ag, q=A16, k=A16 * 2, v=A16 * 3, bias=A16 * 4, B=1, H=8, L=256, D=128,
     (dict(B=-1), 2), (dict(L=-16), 2), (dict(L=250), 2), (dict(D=0), 2),
     (dict(H=4), 4), (dict(D=64), 4), (dict(block=8), 4), (dict(L=65536 + 16), 4),
     (dict(B=1 << 20, L=65536), 4),
+    # B * L = 2^27 is allowed, but B * ceil(L/32) * ceil(L/128) = 2^31 work steps is not.
+    (dict(B=2048, L=65536), 4), (dict(B=1024, L=65536, q=None), 1),
     (dict(cap=0.0), 5), (dict(cap=-1.0), 5), (dict(cap=math.nan), 5),
     (dict(q=BAD), 3), (dict(k=BAD), 3), (dict(out=BAD), 3),
     (dict(out=A16), 7), (dict(lse=A16 * 4), 7),
