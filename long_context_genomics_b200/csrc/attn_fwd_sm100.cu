@@ -10,32 +10,38 @@
 //
 // B200 design (not the page's 64 x 64 Pallas tiling, which targeted sm_86):
 //  * A query tile is 128 tensor-core rows = 16 consecutive positions x all 8
-//    heads.  Every row of the tile then shares one 16-position bias row block
-//    and all 8 heads consume the same K/V tile (multi-query sharing), so each
-//    K/V byte staged in shared memory feeds eight heads.
-//  * Work is a pair of query tiles (A and B) against a range of key tiles.
-//    One persistent CTA per SM takes a contiguous, equal share of all
-//    (pair, key tile) steps, so the grid finishes together; a pair whose key
-//    range is split between CTAs is merged exactly from the pieces' partial
-//    results by log-sum-exp (see "Split pairs" below).
-//  * Inside a CTA the producer warp streams Q tiles and a ring of K and V
-//    tiles with TMA; the MMA warp issues every tcgen05.mma from one thread;
-//    four softmax warpgroups each own one 32-key chunk of every key tile.
-//    The MMA order per key tile j is PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), so
-//    the softmax warps work on one tile while the tensor core works on the
-//    other.
-//  * Tensor memory (512 columns): S_A, S_B (fp32 128x128 logits), O_A, O_B
-//    (fp32 128x128 accumulators).  P is written as bf16 over part of its S
-//    and fed to the PV product straight from tensor memory.
-//  * Bias: each softmax thread owns one row, so per 128-key tile it needs
-//    just the compact cells of its key chunk, read from global (L2) one tile
+//    heads.  Every row of the tile shares one 16-position bias row block and
+//    all 8 heads consume the same K/V tile (multi-query sharing).
+//  * Two SMs work as a pair (a 2-CTA cluster) on a pair of query tiles: each
+//    CTA holds one tile, and one thread of the even CTA issues tcgen05.mma
+//    with cta_group::2, M = 256 rows over both SMs.  Each CTA stages only half
+//    of every K tile (64 of its 128 keys) and half of every V tile (64 of the
+//    128 value columns), so a K/V byte loaded from L2 feeds 16 query rows per
+//    SM pair position, and one MMA instruction keeps both tensor cores busy.
+//  * One persistent cluster per SM pair takes a contiguous, equal share of all
+//    (pair, key tile) steps; a pair whose key range is split between clusters
+//    is merged exactly from the pieces' partial results by log-sum-exp (see
+//    "Split pairs" below).
+//  * Inside each CTA: a producer warp streams its Q tile and a ring of K and V
+//    halves with TMA (no multicast); four softmax warpgroups each own one
+//    32-key chunk of every key tile.  In the odd CTA the MMA warp relays
+//    "loaded" to the even CTA (a cluster-scope arrive), so each CTA's copies
+//    complete on its own barriers and can be drained locally.
+//  * Tensor memory (per CTA): two 128-column S buffers (fp32 logits of
+//    alternate key tiles) and the 128-column O accumulator.  P is written as
+//    bf16 over part of its S buffer and fed to the PV product straight from
+//    tensor memory.  With S double-buffered the MMA order per key tile is
+//    PV(j), S(j+2): the logits a softmax warp needs next were computed while
+//    it worked on the current ones.
+//  * Bias: each softmax thread owns one row, so per key tile it needs just
+//    the two compact cells of its 32 keys, read from global (L2) one tile
 //    ahead and kept in registers; the 16x repeat is never built.
 //  * With a finite cap every logit lies in (-cap, cap), so the softmax uses
 //    the fixed shift m = cap (exact: softmax is shift invariant) and needs no
 //    running max and no rescaling of O.  cap > 40 (where exp(-2 cap) would
 //    underflow fp32) and cap = +inf use a running max with lazy rescaling.
-//  * Every wait is bounded (sm100.cuh); on timeout the kernel records the
-//    wait site in the device error word, drains its own copies and MMAs,
+//  * Every mbarrier wait is bounded (sm100.cuh); on timeout the kernel records
+//    the wait site in the device error word, drains its own copies and MMAs,
 //    frees tensor memory and returns.
 #include "ag_internal.h"
 #include "sm100.cuh"
@@ -45,41 +51,41 @@ namespace attn {
 
 constexpr int kH = 8;
 constexpr int kD = 128;
-constexpr int kKeys = static_cast<int>(kAttnKeyTile);  // keys per K/V tile
+constexpr int kKeys = static_cast<int>(kAttnKeyTile);  // keys per key tile
 static_assert(kKeys == 128, "the tile layout below assumes 128-key tiles");
-constexpr int kStages = 4;                  // K/V ring slots
-constexpr int kTileBytes = 128 * 128 * 2;   // one Q, K or V tile (bf16)
-constexpr int kHalfBytes = kTileBytes / 2;  // one 64-wide (128-byte) half
-// Softmax warpgroups (2 or 4).  Warps 0 .. 4*kWG-1 run the softmax; the next
-// warpgroup holds the TMA producer warp, the MMA warp and two idle warps
-// (present so that it is whole for the register re-allocation).
-#ifndef AG_SOFTMAX_WARPGROUPS
-#define AG_SOFTMAX_WARPGROUPS 4
-#endif
-constexpr int kWG = AG_SOFTMAX_WARPGROUPS;
-static_assert(kWG == 2 || kWG == 4, "two or four softmax warpgroups");
-constexpr int kChunks = 4 / kWG;             // 32-column chunks per warpgroup
+constexpr int kQTileBytes = 128 * kD * 2;     // this CTA's query tile (bf16)
+constexpr int kQHalfBytes = kQTileBytes / 2;  // one 64-wide (128-byte) half
+// A ring slot holds what one key-tile step needs from this CTA: its half of
+// a V tile (128 keys x 64 value columns, 16 KB) and its half of the K tile
+// two steps ahead (64 keys x 128, two 64-wide halves of 8 KB), or, first in
+// a segment, the halves of the segment's first two K tiles.
+constexpr int kPartBytes = 16384;            // one K half or one V half
+constexpr int kKHalfBytes = kPartBytes / 2;  // a K half's 64-wide half
+constexpr int kSlotBytes = 2 * kPartBytes;
+constexpr int kStages = 5;
+constexpr int kWG = 4;                      // softmax warpgroups
 constexpr int kSoftThreads = 128 * kWG;
+constexpr int kSoftWarps = 4 * kWG;         // per CTA
+constexpr int kPairSoftWarps = 2 * kSoftWarps;
 constexpr int kNumWarps = 4 * kWG + 4;
 constexpr int kThreads = kNumWarps * 32;
-constexpr int kWarpLoad = 4 * kWG;
-constexpr int kWarpMma = 4 * kWG + 1;
+constexpr int kWarpLoad = 4 * kWG;          // TMA producer
+constexpr int kWarpMma = 4 * kWG + 1;       // MMA issuer (even CTA) / relay (odd)
 // Registers per thread: the launch gives every thread kRegsLaunch (the cap
 // for this block size, which ptxas allocates when setmaxnreg is present; the
-// launcher checks it).  The producer warpgroup then drops to kRegsLow and,
-// where kRegsHigh exceeds the launch count, the softmax warpgroups rise to
-// it.  (With four softmax warpgroups the softmax needs no more than the
-// launch count, and a producer cap below 80 makes the MMA warp spill.)
-constexpr uint32_t kRegsLaunch = kWG == 2 ? 168 : 96;
-constexpr uint32_t kRegsLow = kWG == 2 ? 88 : 80;
-constexpr uint32_t kRegsHigh = kWG == 2 ? 208 : 96;
-static_assert(kSoftThreads * kRegsHigh + 128 * kRegsLow <= kThreads * kRegsLaunch,
+// launcher checks it); the producer warpgroup then drops to kRegsLow (below
+// 80 the MMA warp spills).  The softmax needs no more than the launch count.
+constexpr uint32_t kRegsLaunch = 96;
+constexpr uint32_t kRegsLow = 80;
+static_assert(kSoftThreads * kRegsLaunch + 128 * kRegsLow <= kThreads * kRegsLaunch,
               "register split exceeds the launch allocation");
 constexpr uint32_t kTmemCols = 512;
-// P (bf16 pairs) of a tile: keys [32c, 32c + 32) of chunk c are written over
-// the first 16 columns of that chunk's own S columns, [32c, 32c + 16).
-constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0);  // K-major B (K)
-constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, 1);  // MN-major B (V)
+// Tensor-memory columns: S buffer u at 128 u, O at 256.  P (bf16 pairs) of
+// chunk c (keys [32c, 32c + 32) of the tile) is written over the first 16
+// columns of that chunk's own S columns, [32c, 32c + 16).
+constexpr uint32_t kColO = 256;
+constexpr uint32_t kIdescQK = idesc_bf16_f32(256, kKeys, 0);  // K-major B (K)
+constexpr uint32_t kIdescPV = idesc_bf16_f32(256, kD, 1);     // MN-major B (V)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 // Lazy rescale threshold (log2 units) for the running-max modes.
@@ -91,39 +97,54 @@ enum Mode { kStaticCap = 0, kOnlineCap = 1, kNoCap = 2 };
 enum Site : unsigned {
   kSiteProdQ = 1, kSiteProdKV = 2, kSiteMmaQ = 3, kSiteMmaKV = 4,
   kSiteMmaP = 5, kSiteSoftS = 6, kSiteSoftO = 7, kSiteDrain = 8,
-  kSiteXchg = 9
+  kSiteXchg = 9, kSiteSoftPV = 10, kSiteRelay = 11
 };
 
+// Per-CTA barriers.  q_peer, kv_peer and p_full are used in the even CTA
+// only (the odd CTA's relay and softmax warps arrive on them remotely);
+// q_empty, kv_empty, s_full, pv_done and o_full are signalled in both CTAs
+// by the even CTA's MMA commits.
 struct __align__(8) Barriers {
-  uint64_t q_full[2], q_empty[2];
-  uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t s_full[2], p_full[2], o_full[2];
-  uint64_t xm[2], xd[2];  // row-max / row-sum exchange between warpgroups
+  uint64_t q_full, q_peer, q_empty;
+  uint64_t kv_full[kStages], kv_peer[kStages], kv_empty[kStages];
+  // s_full / p_full by S buffer: a softmax may finish key tile j + 1 before
+  // the MMA warp has taken key tile j's arrivals.
+  uint64_t s_full[2], p_full[2];
+  uint64_t pv_done, o_full;
+  uint64_t xm, xd;  // row-max / row-sum exchange between the warpgroups
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
-  int range_begin, range_end;  // this CTA's (pair, key tile) steps
+  int range_begin, range_end;  // this cluster's (pair, key tile) steps
 };
 
-constexpr size_t kXchgBytes = 2 * 2 * kWG * 128 * sizeof(float);
-constexpr size_t kSmemBytes = 1024 + (2 + kStages) * static_cast<size_t>(kTileBytes) +
-                              sizeof(Barriers) + kXchgBytes;
+// Softmax-side shared memory: row-max (per step, double-buffered by step
+// parity) and row-sum (per segment) exchange between the four chunks.
+struct Xchg {
+  float mpart[2][kWG][128];  // [step parity][chunk][row]
+  float dpart[kWG][128];     // [chunk][row]
+};
+
+constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kQTileBytes) +
+                              kStages * static_cast<size_t>(kSlotBytes) +
+                              sizeof(Barriers) + sizeof(Xchg);
+static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
 struct Params {
   const float *bias;
   float *out;
   float *lse;
   unsigned *err;
-  // Split-pair scratch (see "Split pairs"): one slot per CTA.
-  float *ws_out;       // [grid][2][128][128] partial outputs
-  float *ws_lse;       // [grid][2][128] partial log-sum-exps
+  // Split-pair scratch (see "Split pairs"): one slot per cluster.
+  float *ws_out;       // [clusters][2][128][128] partial outputs
+  float *ws_lse;       // [clusters][2][128] partial log-sum-exps
   int L, P;
   int nb;          // 16-position query blocks per batch item (L / 16)
   int pairs;       // query-tile pairs per batch item: ceil(nb / 2)
   int n_items;     // B * pairs
   int n_kt;        // key tiles: ceil(L / 128)
-  int last_valid;  // valid keys in the last key tile (1..128)
-  int whole;       // 1: CTA ranges hold whole pairs (no split pairs)
+  int last_valid;  // valid keys in the last key tile (16..128)
+  int whole;       // 1: cluster ranges hold whole pairs (no split pairs)
   float qk_scale;  // multiplies q.k
   float bias_mul;  // multiplies the compact bias
   float A;         // capped modes: cap * log2(e)
@@ -131,22 +152,24 @@ struct Params {
 
 // --------------------------------------------------------------------------
 // Work split.  The W = n_items * n_kt (pair, key tile) steps are cut into
-// gridDim.x contiguous ranges [W c / G, W (c+1) / G).  A CTA walks its range
-// as segments: one pair and a run of its key tiles.  A pair covered by more
-// than one CTA is "split"; its pieces are merged by the last one to finish.
+// one contiguous range per cluster, [W c / G, W (c+1) / G) for cluster c of
+// G.  Both CTAs of a cluster walk the range as segments: one pair and a run
+// of its key tiles.  A pair covered by more than one cluster is "split".
 struct Segment {
   int item, kb, ke;  // pair index and key tiles [kb, ke)
 };
 
+__device__ __forceinline__ int num_clusters() { return static_cast<int>(gridDim.x >> 1); }
+__device__ __forceinline__ int cluster_index() { return static_cast<int>(blockIdx.x >> 1); }
+
 // W = n_items * n_kt <= 2^30 (checked by the launcher), so steps fit in int;
 // only the range bounds need a 64-bit product.  With p.whole the bounds are
-// rounded to whole pairs: CTA c gets pairs [n_items c / G, n_items (c+1) / G).
+// rounded to whole pairs: cluster c gets pairs [n_items c / G, n_items (c+1) / G).
 __device__ __forceinline__ int range_start(const Params &p, int c) {
+  const long long G = num_clusters();
   if (p.whole)
-    return static_cast<int>(static_cast<long long>(p.n_items) * c /
-                            static_cast<long long>(gridDim.x)) * p.n_kt;
-  return static_cast<int>(static_cast<long long>(p.n_items) * p.n_kt * c /
-                          static_cast<long long>(gridDim.x));
+    return static_cast<int>(static_cast<long long>(p.n_items) * c / G) * p.n_kt;
+  return static_cast<int>(static_cast<long long>(p.n_items) * p.n_kt * c / G);
 }
 
 __device__ __forceinline__ Segment segment_at(const Params &p, int t, int end) {
@@ -158,8 +181,22 @@ __device__ __forceinline__ Segment segment_at(const Params &p, int t, int end) {
   return sg;
 }
 
+// K/V ring order, shared by the producers, the relay and the MMA warp: for a
+// segment with key tiles [kb, ke), slot load 0 holds K(kb) (part 0) and
+// K(kb+1) (part 1); slot load i = 1 .. n holds K(kb+i+1) (part 0, while it
+// exists) and V(kb+i-1) (part 1).  S runs two key tiles ahead of PV.
+// f(i, k_tile or -1, second part: is_v ? v_tile : k_tile or -1, is_v).
+template <typename F>
+__device__ __forceinline__ bool for_each_ring_load(const Segment &sg, F &&f) {
+  const int n = sg.ke - sg.kb;
+  bool ok = f(sg.kb, n > 1 ? sg.kb + 1 : -1, false);
+  for (int i = 1; i <= n && ok; ++i)
+    ok = f(sg.kb + i + 1 < sg.ke ? sg.kb + i + 1 : -1, sg.kb + i - 1, true);
+  return ok;
+}
+
 // --------------------------------------------------------------------------
-// MMA issue helpers (single thread).
+// MMA issue helpers (single thread of the even CTA).
 
 // Shared-memory descriptors: every operand here has 8-row groups 1 KB apart,
 // so all share one high word; the low word (start address and leading
@@ -167,29 +204,31 @@ __device__ __forceinline__ Segment segment_at(const Params &p, int t, int end) {
 // start-address field (addresses stay below 2^18: no carry out of the field).
 constexpr uint32_t kDescHi = desc_sw128_hi(1024);
 
-// S[128 x 128] = Q[128 x 128] K^T: eight K=16 steps over two 64-wide halves.
+// S[256 x 128] = Q[256 x 128] K^T over the pair: eight K=16 steps over the two
+// 64-wide halves of each CTA's Q tile (16 KB apart) and K half (8 KB apart).
 __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_addr,
                                          uint32_t k_addr) {
   const uint32_t q_lo = desc_sw128_lo(q_addr, 16), k_lo = desc_sw128_lo(k_addr, 16);
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk) {
-    const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
-    umma_ss_lo(d_tmem, q_lo + off, k_lo + off, kDescHi, kIdescQK, kk > 0 ? 1u : 0u);
+    const uint32_t qo = ((kk >> 2) * kQHalfBytes + (kk & 3) * 32) >> 4;
+    const uint32_t ko = ((kk >> 2) * kKHalfBytes + (kk & 3) * 32) >> 4;
+    umma2_ss_lo(d_tmem, q_lo + qo, k_lo + ko, kDescHi, kIdescQK, kk > 0 ? 1u : 0u);
   }
 }
 
-// O[128 x 128] (+)= P[128 x 128 keys] V[128 keys x 128]: P from tensor memory
-// (bf16 pairs, 8 columns per 16 keys; keys 32c.. of chunk c start at column
-// 32c of the S region), V MN-major in shared memory (the two 64-wide halves
-// are 16 KB apart, 8-key row groups 1 KB apart).
+// O[256 x 128] (+)= P[256 x 128 keys] V[128 keys x 128]: P from each CTA's
+// tensor memory (bf16 pairs, 8 columns per 16 keys; keys 32c.. of chunk c
+// start at column 32c of the S buffer), V MN-major: each CTA holds 64 value
+// columns (one 128-byte atom) for all 128 keys, 8-key row groups 1 KB apart.
 __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t s_tmem,
                                          uint32_t v_addr, bool accumulate) {
-  const uint32_t v_lo = desc_sw128_lo(v_addr, kHalfBytes);
+  const uint32_t v_lo = desc_sw128_lo(v_addr, kPartBytes / 2);
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk) {
-    umma_ts_lo(d_tmem, s_tmem + 32 * (kk >> 1) + 8 * (kk & 1),
-               v_lo + ((kk * 2048) >> 4), kDescHi, kIdescPV,
-               (accumulate || kk > 0) ? 1u : 0u);
+    umma2_ts_lo(d_tmem, s_tmem + 32 * (kk >> 1) + 8 * (kk & 1),
+                v_lo + ((kk * 2048) >> 4), kDescHi, kIdescPV,
+                (accumulate || kk > 0) ? 1u : 0u);
   }
 }
 
@@ -202,17 +241,26 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
   }
 }
 
+// The query block this CTA's tile covers in pair item I0 / 2: I0 + rank, or
+// (past the end of an odd count) a copy of block I0 whose results are not
+// written.
+__device__ __forceinline__ int tile_block(const Params &p, int I0, uint32_t rank) {
+  const int I = I0 + static_cast<int>(rank);
+  return I < p.nb ? I : I0;
+}
+
 // --------------------------------------------------------------------------
-// Producer warp, lane 0: TMA loads.
+// Producer warp, lane 0 (each CTA): TMA loads of this CTA's Q tile and of its
+// halves of the K and V tiles.
 __device__ __forceinline__ void producer(const CUtensorMap *tm_q,
                                          const CUtensorMap *tm_k,
                                          const CUtensorMap *tm_v, uint8_t *q_s,
                                          uint8_t *kv_s, Barriers *bars,
-                                         const Params &p, volatile int *abort) {
+                                         const Params &p, uint32_t rank,
+                                         volatile int *abort) {
   const uint64_t pol_q = l2_policy_evict_first();
   const uint64_t pol_kv = l2_policy_evict_last();
-  uint32_t qcount[2] = {0, 0};
-  uint32_t kv = 0;
+  uint32_t qcount = 0, kv = 0;
   bool ok = true;
   const int end = bars->range_end;
   for (int t = bars->range_begin; t < end && ok;) {
@@ -220,164 +268,169 @@ __device__ __forceinline__ void producer(const CUtensorMap *tm_q,
     t += sg.ke - sg.kb;
     const int b = sg.item / p.pairs;
     const int I0 = (sg.item % p.pairs) * 2;
-    const int nX = (I0 + 1 < p.nb) ? 2 : 1;
-#pragma unroll
-    for (int X = 0; X < 2; ++X) {
-      if (X >= nX) break;
-      ok = mbar_wait(&bars->q_empty[X], (qcount[X] & 1u) ^ 1u, abort, p.err,
-                     kSiteProdQ);
-      if (!ok) break;
-      mbar_arrive_expect_tx(&bars->q_full[X], kTileBytes);
-      uint8_t *dst = q_s + X * kTileBytes;
-      tma_load_4d(dst, tm_q, &bars->q_full[X], 0, (I0 + X) * 16, 0, b, pol_q);
-      tma_load_4d(dst + kHalfBytes, tm_q, &bars->q_full[X], 64, (I0 + X) * 16,
-                  0, b, pol_q);
-      ++qcount[X];
-    }
-    for (int j = sg.kb; j < sg.ke && ok; ++j) {
-#pragma unroll 1
-      for (int u = 0; u < 2; ++u) {  // u = 0: K tile j, u = 1: V tile j
-        const uint32_t slot = kv % kStages, ph = (kv / kStages) & 1u;
-        ok = mbar_wait(&bars->kv_empty[slot], ph ^ 1u, abort, p.err, kSiteProdKV);
-        if (!ok) break;
-        mbar_arrive_expect_tx(&bars->kv_full[slot], kTileBytes);
-        uint8_t *dst = kv_s + slot * kTileBytes;
-        const CUtensorMap *tm = u == 0 ? tm_k : tm_v;
-        tma_load_3d(dst, tm, &bars->kv_full[slot], 0, j * kKeys, b, pol_kv);
-        tma_load_3d(dst + kHalfBytes, tm, &bars->kv_full[slot], 64, j * kKeys, b,
-                    pol_kv);
-        ++kv;
-      }
-    }
+    ok = mbar_wait(&bars->q_empty, (qcount & 1u) ^ 1u, abort, p.err, kSiteProdQ);
+    if (!ok) break;
+    mbar_arrive_expect_tx(&bars->q_full, kQTileBytes);
+    const int qrow = tile_block(p, I0, rank) * 16;
+    tma_load_4d(q_s, tm_q, &bars->q_full, 0, qrow, 0, b, pol_q);
+    tma_load_4d(q_s + kQHalfBytes, tm_q, &bars->q_full, 64, qrow, 0, b, pol_q);
+    ++qcount;
+    ok = for_each_ring_load(sg, [&](int k_tile, int second, bool is_v) {
+      const uint32_t slot = kv % kStages, ph = (kv / kStages) & 1u;
+      if (!mbar_wait(&bars->kv_empty[slot], ph ^ 1u, abort, p.err, kSiteProdKV))
+        return false;
+      const uint32_t bytes = (k_tile >= 0 ? kPartBytes : 0) +
+                             (second >= 0 ? kPartBytes : 0);
+      mbar_arrive_expect_tx(&bars->kv_full[slot], bytes);
+      uint8_t *dst = kv_s + slot * kSlotBytes;
+      // A K half: keys [128 j + 64 rank, +64), all 128 columns.
+      auto load_k = [&](uint8_t *to, int j) {
+        const int key0 = j * kKeys + 64 * static_cast<int>(rank);
+        tma_load_3d(to, tm_k, &bars->kv_full[slot], 0, key0, b, pol_kv);
+        tma_load_3d(to + kKHalfBytes, tm_k, &bars->kv_full[slot], 64, key0, b, pol_kv);
+      };
+      if (k_tile >= 0) load_k(dst, k_tile);
+      if (is_v)  // keys [128 j, +128), value columns [64 rank, +64)
+        tma_load_3d(dst + kPartBytes, tm_v, &bars->kv_full[slot],
+                    64 * static_cast<int>(rank), second * kKeys, b, pol_kv);
+      else if (second >= 0)
+        load_k(dst + kPartBytes, second);
+      ++kv;
+      return true;
+    });
   }
   // Every copy this thread started must land before the CTA exits.
-  for (int X = 0; X < 2; ++X)
-    if (qcount[X] > 0) drain_wait(&bars->q_full[X], (qcount[X] - 1) & 1u);
+  if (qcount > 0) drain_wait(&bars->q_full, (qcount - 1) & 1u);
   const uint32_t first = kv > kStages ? kv - kStages : 0;
   for (uint32_t i = first; i < kv; ++i)
     drain_wait(&bars->kv_full[i % kStages], (i / kStages) & 1u);
 }
 
 // --------------------------------------------------------------------------
-// MMA warp, lane 0: tcgen05.mma issuer.
-__device__ __forceinline__ void mma_issuer(uint8_t *q_s, uint8_t *kv_s,
-                                           Barriers *bars, uint32_t tmem,
-                                           const Params &p, volatile int *abort) {
-  const uint32_t q_addr = smem_u32(q_s);
-  const uint32_t kv_addr = smem_u32(kv_s);
-  uint32_t qcount[2] = {0, 0}, pcount[2] = {0, 0};
-  uint32_t kv = 0;
+// MMA warp of the odd CTA, lane 0: tells the even CTA's MMA thread, in ring
+// order, that this CTA's half of each Q / K / V load has landed.
+__device__ __forceinline__ void relay(Barriers *bars, const Params &p,
+                                      volatile int *abort) {
+  const uint32_t q_peer = cluster_addr(&bars->q_peer, 0);
+  uint32_t qcount = 0, kv = 0;
   bool ok = true;
   const int end = bars->range_end;
   for (int t = bars->range_begin; t < end && ok;) {
     const Segment sg = segment_at(p, t, end);
     t += sg.ke - sg.kb;
-    const int I0 = (sg.item % p.pairs) * 2;
-    const int nX = (I0 + 1 < p.nb) ? 2 : 1;
-#pragma unroll
-    for (int X = 0; X < 2; ++X) {
-      if (X >= nX || !ok) break;
-      ok = mbar_wait(&bars->q_full[X], qcount[X] & 1u, abort, p.err, kSiteMmaQ);
-      ++qcount[X];
-    }
+    ok = mbar_wait(&bars->q_full, qcount & 1u, abort, p.err, kSiteRelay);
+    ++qcount;
     if (!ok) break;
-    // First key tile of the segment: S_X(kb) for both query tiles.
-    const int n = sg.ke - sg.kb;
-    const uint32_t slot_k0 = kv % kStages;
-    ok = mbar_wait(&bars->kv_full[slot_k0], (kv / kStages) & 1u, abort, p.err,
-                   kSiteMmaKV);
-    if (!ok) break;
-    ++kv;
-    tc_fence_after();
-#pragma unroll
-    for (int X = 0; X < 2; ++X) {
-      if (X >= nX) break;
-      issue_qk(tmem + X * 128, q_addr + X * kTileBytes,
-               kv_addr + slot_k0 * kTileBytes);
-      umma_commit(&bars->s_full[X]);
-      if (n == 1) umma_commit(&bars->q_empty[X]);
-    }
-    umma_commit(&bars->kv_empty[slot_k0]);
-
-    for (int i = 0; i < n && ok; ++i) {
-      const uint32_t slot_v = kv % kStages;
-      ok = mbar_wait(&bars->kv_full[slot_v], (kv / kStages) & 1u, abort, p.err,
-                     kSiteMmaKV);
-      if (!ok) break;
+    mbar_arrive_cluster(q_peer);
+    ok = for_each_ring_load(sg, [&](int, int, bool) {
+      const uint32_t slot = kv % kStages;
+      if (!mbar_wait(&bars->kv_full[slot], (kv / kStages) & 1u, abort, p.err,
+                     kSiteRelay))
+        return false;
       ++kv;
-      const bool has_next = i + 1 < n;
-      uint32_t slot_k = 0;
-      bool k_ready = false;
-#pragma unroll
-      for (int X = 0; X < 2; ++X) {
-        if (X >= nX) break;
-        ok = mbar_wait(&bars->p_full[X], pcount[X] & 1u, abort, p.err, kSiteMmaP);
-        ++pcount[X];
-        if (!ok) break;
-        tc_fence_after();
-        issue_pv(tmem + 256 + X * 128, tmem + X * 128,
-                 kv_addr + slot_v * kTileBytes, i > 0);
-        if (!has_next) {
-          umma_commit(&bars->o_full[X]);
-          continue;
-        }
-        if (!k_ready) {
-          slot_k = kv % kStages;
-          ok = mbar_wait(&bars->kv_full[slot_k], (kv / kStages) & 1u, abort,
-                         p.err, kSiteMmaKV);
-          if (!ok) break;
-          ++kv;
-          k_ready = true;
-          tc_fence_after();
-        }
-        issue_qk(tmem + X * 128, q_addr + X * kTileBytes,
-                 kv_addr + slot_k * kTileBytes);
-        umma_commit(&bars->s_full[X]);
-        if (i + 2 == n) umma_commit(&bars->q_empty[X]);
-      }
+      mbar_arrive_cluster(cluster_addr(&bars->kv_peer[slot], 0));
+      return true;
+    });
+  }
+}
+
+// --------------------------------------------------------------------------
+// MMA warp of the even CTA, lane 0: tcgen05.mma issuer for the pair.
+// kPvDone: also signal pv_done after every PV but the segment's last (the
+// running-max modes rescale O and must know when the previous PV finished).
+template <bool kPvDone>
+__device__ __forceinline__ void mma_issuer(uint8_t *q_s, uint8_t *kv_s,
+                                           Barriers *bars, uint32_t tmem,
+                                           const Params &p, volatile int *abort) {
+  const uint32_t q_addr = smem_u32(q_s);
+  const uint32_t kv_addr = smem_u32(kv_s);
+  uint32_t qcount = 0, kv = 0;
+  uint32_t pbits = 0;  // bit u: parity of the next p_full[u] phase
+  bool ok = true;
+  // Both halves of the next ring load: this CTA's copy and the peer's relay.
+  auto wait_kv = [&](uint32_t &slot) {
+    slot = kv % kStages;
+    const uint32_t ph = (kv / kStages) & 1u;
+    ++kv;
+    return mbar_wait(&bars->kv_full[slot], ph, abort, p.err, kSiteMmaKV) &&
+           mbar_wait_cluster(&bars->kv_peer[slot], ph, abort, p.err, kSiteMmaKV);
+  };
+  const int end = bars->range_end;
+  for (int t = bars->range_begin; t < end && ok;) {
+    const Segment sg = segment_at(p, t, end);
+    t += sg.ke - sg.kb;
+    const int n = sg.ke - sg.kb;
+    ok = mbar_wait(&bars->q_full, qcount & 1u, abort, p.err, kSiteMmaQ) &&
+         mbar_wait_cluster(&bars->q_peer, qcount & 1u, abort, p.err, kSiteMmaQ);
+    ++qcount;
+    if (!ok) break;
+    // Slot load 0: S(kb) into buffer 0 and S(kb+1) into buffer 1.
+    {
+      uint32_t slot;
+      ok = wait_kv(slot);
       if (!ok) break;
-      umma_commit(&bars->kv_empty[slot_v]);
-      if (k_ready) umma_commit(&bars->kv_empty[slot_k]);
+      tc_fence_after();
+      const uint32_t base = kv_addr + slot * kSlotBytes;
+      for (int u = 0; u < 2 && u < n; ++u) {
+        issue_qk(tmem + 128u * u, q_addr, base + u * kPartBytes);
+        umma2_commit_both(&bars->s_full[u]);
+        if (u == n - 1) umma2_commit_both(&bars->q_empty);
+      }
+      umma2_commit_both(&bars->kv_empty[slot]);
+    }
+
+    for (int j = sg.kb; j < sg.ke; ++j) {
+      const uint32_t u = static_cast<uint32_t>(j - sg.kb) & 1u;
+      uint32_t slot;  // V(j) in part 1, K(j+2) (while it exists) in part 0
+      ok = wait_kv(slot);
+      if (!ok) break;
+      ok = mbar_wait_cluster(&bars->p_full[u], (pbits >> u) & 1u, abort, p.err,
+                             kSiteMmaP);
+      pbits ^= 1u << u;
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t base = kv_addr + slot * kSlotBytes;
+      issue_pv(tmem + kColO, tmem + 128u * u, base + kPartBytes, j > sg.kb);
+      if (j + 1 == sg.ke)
+        umma2_commit_both(&bars->o_full);
+      else if (kPvDone)
+        umma2_commit_both(&bars->pv_done);
+      if (j + 2 < sg.ke) {
+        // S(j+2) over buffer u: issued after PV(j), which reads P(j) from the
+        // same columns (the tensor core runs one thread's MMAs in order).
+        issue_qk(tmem + 128u * u, q_addr, base);
+        umma2_commit_both(&bars->s_full[u]);
+        if (j + 3 == sg.ke) umma2_commit_both(&bars->q_empty);
+      }
+      umma2_commit_both(&bars->kv_empty[slot]);
     }
   }
   // All MMAs this thread issued complete before tensor memory is released.
-  umma_commit(&bars->drain);
+  umma2_commit_self(&bars->drain);
   drain_wait(&bars->drain, 0);
 }
 
 // --------------------------------------------------------------------------
-// Softmax warpgroups.
+// Softmax warpgroups (each CTA, its own query tile).
 //
-// All softmax warps work on query tile A, then all on tile B, then A again:
-// warpgroup g takes the kChunks 32-key chunks starting at key 32*kChunks*g of
-// every 128-key tile, for all 128 rows (thread r of every warpgroup owns
-// tensor-memory lane r).  While the warps run one tile's softmax the tensor
-// core runs the other tile's PV and next QK^T, so the two alternate without
-// further synchronisation.  A row's sum is split between its kWG threads and
-// combined through shared memory once per work item.  Each chunk's P goes over
-// the first half of that chunk's own S columns, so a warpgroup only ever
-// overwrites S columns it has already read itself.
-
-// Softmax-side shared memory: row-sum and row-max exchange between the kWG
-// threads of a row.
-struct Xchg {
-  float dpart[2][kWG][128];  // [tile][warpgroup][row]
-  float mpart[2][kWG][128];
-};
+// Warpgroup g owns keys [32g, 32g + 32) of every 128-key tile, for all 128
+// rows (thread r of the warpgroup owns tensor-memory lane r).  A row's sum is
+// split between its four threads and combined through shared memory once per
+// work item (and, in the running-max modes, its maximum once per key tile).
+// Each chunk's P goes over the first 16 of its own S columns, so a
+// warpgroup only ever overwrites S columns it has already read itself.
 
 // Softmax-side barriers count warps: each warp arrives once, from lane 0,
 // after __syncwarp has ordered its lanes' prior work (one arrival per warp
 // instead of 32 keeps the mbarrier off the shared-memory pipe).
-constexpr uint32_t kSoftWarps = kSoftThreads / 32;
-
 __device__ __forceinline__ void warp_arrive(uint64_t *bar) {
   __syncwarp();
   if (lane_id() == 0) mbar_arrive(bar);
 }
 
 // Publish this thread's value, then wait (bounded) until every softmax thread
-// has published its own.  The warp barrier and the mbarrier's arrive/wait
-// order the shared-memory writes before the partners' reads.
+// of the CTA has published its own.  The warp barrier and the mbarrier's
+// arrive/wait order the shared-memory writes before the partners' reads.
 __device__ __forceinline__ bool exchange(uint64_t *bar, uint32_t &count,
                                          volatile int *abort, unsigned *err) {
   warp_arrive(bar);
@@ -386,14 +439,13 @@ __device__ __forceinline__ bool exchange(uint64_t *bar, uint32_t &count,
   return __all_sync(0xffffffffu, ok);
 }
 
-// The compact bias cells of this warpgroup's keys of key tile j (two per
-// 32-key chunk): bias[h, I, 8j + 2*kChunks*g + e].
+// The compact bias cells of chunk g of key tile j (two per 32-key chunk):
+// bias[h, I, 8j + 2g + e] (0 past the end: those keys are masked).
 __device__ __forceinline__ void load_bias(const float *brow, int j, int g, int P,
-                                          float (&bn)[2 * kChunks]) {
-  const int J0 = j * 8 + g * 2 * kChunks;
+                                          float (&bn)[2]) {
+  const int J0 = j * 8 + g * 2;
 #pragma unroll
-  for (int e = 0; e < 2 * kChunks; ++e)
-    bn[e] = (J0 + e < P) ? __ldg(brow + J0 + e) : 0.f;
+  for (int e = 0; e < 2; ++e) bn[e] = (J0 + e < P) ? __ldg(brow + J0 + e) : 0.f;
 }
 
 // Column pairs (out of every 8) whose exponential runs on the FMA pipe
@@ -421,131 +473,93 @@ __device__ __forceinline__ void chunk_static(const uint32_t (&s)[32], float b0,
         make_float2(bb, bb));
     const float2 t = make_float2(tanh_approx(y.x), tanh_approx(y.y));
     const float2 x = __ffma2_rn(t, ap, an);
-    float2 p;
+    float2 pr;
     if ((e & 7) < kEmuPairs) {
-      p = exp2_poly2(x);
+      pr = exp2_poly2(x);
     } else {
-      p = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+      pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
     }
     if (kMask) {
-      if (col0 + 2 * e >= nvalid) p.x = 0.f;
-      if (col0 + 2 * e + 1 >= nvalid) p.y = 0.f;
+      if (col0 + 2 * e >= nvalid) pr.x = 0.f;
+      if (col0 + 2 * e + 1 >= nvalid) pr.y = 0.f;
     }
-    acc = __fadd2_rn(acc, p);
-    pk[e] = pack_bf16x2(p.x, p.y);
+    acc = __fadd2_rn(acc, pr);
+    pk[e] = pack_bf16x2(pr.x, pr.y);
   }
 }
 
-// This warpgroup's chunks of one tile, static shift: S in, P out over the
-// first 16 columns of each chunk.  Returns the partial row sum.
+// One key tile, static shift: S in, P out over the first 16 columns of this
+// warpgroup's chunk.  Returns the partial row sum.
 template <bool kMask>
-__device__ __forceinline__ float part_tile_static(uint32_t tS, int g,
-                                                  const float (&bj)[2 * kChunks],
-                                                  float2 sc, float2 ap, float2 an,
-                                                  int nvalid) {
+__device__ __forceinline__ float tile_static(uint32_t tS, int col0, float b0,
+                                             float b1, float2 sc, float2 ap,
+                                             float2 an, int nvalid) {
   float2 acc = make_float2(0.f, 0.f);
-  uint32_t pk[16];
-  if constexpr (kChunks == 1) {
-    uint32_t sa[32];
-    const uint32_t c0 = 32 * g;
-    tmem_ld32(tS + c0, sa);
-    tmem_wait_ld(sa);
-    chunk_static<kMask>(sa, bj[0], bj[1], sc, ap, an, c0, nvalid, acc, pk);
-    tmem_st16(tS + c0, pk);
-  } else {
-    uint32_t sa[32], sb[32];
-    const uint32_t c0 = 64 * g;
-    tmem_ld32(tS + c0, sa);
-    tmem_wait_ld(sa);
-    tmem_ld32(tS + c0 + 32, sb);
-    chunk_static<kMask>(sa, bj[0], bj[1], sc, ap, an, c0, nvalid, acc, pk);
-    tmem_st16(tS + c0, pk);
-    tmem_wait_ld(sb);
-    chunk_static<kMask>(sb, bj[2], bj[3], sc, ap, an, c0 + 32, nvalid, acc, pk);
-    tmem_st16(tS + c0 + 32, pk);
-  }
+  uint32_t s[32], pk[16];
+  tmem_ld32(tS, s);
+  tmem_wait_ld(s);
+  chunk_static<kMask>(s, b0, b1, sc, ap, an, col0, nvalid, acc, pk);
+  tmem_st16(tS, pk);
   return acc.x + acc.y;
 }
 
-// Log2-domain logits of one chunk for the running-max modes.
+// One key tile with a running maximum shared by the four threads of each row
+// (exchanged through shared memory).  When the maximum grows past the lazy
+// threshold, this warpgroup's 32 columns of O are rescaled, after the
+// previous PV into O has finished (pv_done).
 template <int MODE>
-__device__ __forceinline__ void chunk_logits(const uint32_t (&s)[32], float b0,
-                                             float b1, const Params &p, int col0,
-                                             int nvalid, float (&x)[32]) {
-#pragma unroll
-  for (int c = 0; c < 32; ++c) {
-    const float bb = c < 16 ? b0 : b1;
-    const float y = fmaf(__uint_as_float(s[c]), p.qk_scale, bb);
-    float v = (MODE == kOnlineCap) ? p.A * tanh_approx(y) : y;
-    x[c] = (col0 + c < nvalid) ? v : -INFINITY;
-  }
-}
-
-// This warpgroup's chunks of one tile with a running maximum shared by the
-// kWG threads of each row (exchanged through shared memory).  Rescales this
-// warpgroup's columns of O when the maximum grows past the lazy threshold.
-template <int MODE>
-__device__ __forceinline__ bool part_tile_online(uint32_t tS, uint32_t tO, int g,
-                                                 int r, int X, int i,
-                                                 const float (&bj)[2 * kChunks],
-                                                 const Params &p, int nvalid,
-                                                 Xchg *xc, uint64_t *xbar,
-                                                 uint32_t &xcount,
-                                                 volatile int *abort, float &m,
-                                                 float &d) {
-  const uint32_t c0 = 32 * kChunks * g;
+__device__ __forceinline__ bool tile_online(uint32_t tS, uint32_t tO, int g,
+                                            int r, uint32_t par, bool o_live,
+                                            uint32_t pv_parity, float b0,
+                                            float b1, const Params &p, int nvalid,
+                                            Xchg *xc, Barriers *bars,
+                                            uint32_t &xcount, volatile int *abort,
+                                            float &m, float &d) {
+  uint32_t s[32];
+  float x[32];
+  tmem_ld32(tS, s);
+  tmem_wait_ld(s);
   float mt = -INFINITY;
-#pragma unroll 1
-  for (int c = 0; c < kChunks; ++c) {
-    uint32_t s[32];
-    float x[32];
-    tmem_ld32(tS + c0 + c * 32, s);
-    tmem_wait_ld(s);
-    chunk_logits<MODE>(s, bj[2 * c], bj[2 * c + 1], p, c0 + c * 32, nvalid, x);
 #pragma unroll
-    for (int e = 0; e < 32; ++e) mt = fmaxf(mt, x[e]);
+  for (int e = 0; e < 32; ++e) {
+    const float bb = e < 16 ? b0 : b1;
+    const float y = fmaf(__uint_as_float(s[e]), p.qk_scale, bb);
+    const float v = (MODE == kOnlineCap) ? p.A * tanh_approx(y) : y;
+    x[e] = (32 * g + e < nvalid) ? v : -INFINITY;
+    mt = fmaxf(mt, x[e]);
   }
-  xc->mpart[X][g][r] = mt;
-  if (!exchange(xbar, xcount, abort, p.err)) return false;
+  xc->mpart[par][g][r] = mt;
+  if (!exchange(&bars->xm, xcount, abort, p.err)) return false;
 #pragma unroll
-  for (int q = 0; q < kWG; ++q) mt = fmaxf(mt, xc->mpart[X][q][r]);
+  for (int q = 0; q < kWG; ++q) mt = fmaxf(mt, xc->mpart[par][q][r]);
   float factor = 1.f;
   if (mt > m + kRescaleThreshold || m == -INFINITY) {
     factor = (m == -INFINITY) ? 0.f : ex2_approx(m - mt);
     m = mt;
     d *= factor;
   }
-  if (i > 0 && __any_sync(0xffffffffu, factor != 1.f)) {
-    // The previous tile's PV into O is complete: this tile's s_full was
-    // committed after it.  (Before the first tile O holds nothing yet.)
-#pragma unroll 1
-    for (int c = 0; c < kChunks; ++c) {
-      uint32_t o[32];
-      tmem_ld32(tO + c0 + c * 32, o);
-      tmem_wait_ld(o);
+  if (o_live && __any_sync(0xffffffffu, factor != 1.f)) {
+    const bool ok = mbar_wait(&bars->pv_done, pv_parity, abort, p.err, kSiteSoftPV);
+    if (!__all_sync(0xffffffffu, ok)) return false;
+    tc_fence_after();
+    uint32_t o[32];
+    tmem_ld32(tO, o);
+    tmem_wait_ld(o);
 #pragma unroll
-      for (int e = 0; e < 32; ++e)
-        o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
-      tmem_st32(tO + c0 + c * 32, o);
-    }
+    for (int e = 0; e < 32; ++e)
+      o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
+    tmem_st32(tO, o);
   }
   float acc = 0.f;
-#pragma unroll 1
-  for (int c = 0; c < kChunks; ++c) {
-    uint32_t s[32], pk[16];
-    float x[32];
-    tmem_ld32(tS + c0 + c * 32, s);
-    tmem_wait_ld(s);
-    chunk_logits<MODE>(s, bj[2 * c], bj[2 * c + 1], p, c0 + c * 32, nvalid, x);
+  uint32_t pk[16];
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const float p0 = ex2_approx(x[2 * e] - m);
-      const float p1 = ex2_approx(x[2 * e + 1] - m);
-      acc += p0 + p1;
-      pk[e] = pack_bf16x2(p0, p1);
-    }
-    tmem_st16(tS + c0 + c * 32, pk);
+  for (int e = 0; e < 16; ++e) {
+    const float p0 = ex2_approx(x[2 * e] - m);
+    const float p1 = ex2_approx(x[2 * e + 1] - m);
+    acc += p0 + p1;
+    pk[e] = pack_bf16x2(p0, p1);
   }
+  tmem_st16(tS, pk);
   d += acc;
   return true;
 }
@@ -554,24 +568,132 @@ __device__ __forceinline__ bool part_tile_online(uint32_t tS, uint32_t tO, int g
 // Split pairs.  Every segment of a split pair finishes like a whole pair but
 // over its own key range: a normalised partial output and the partial
 // log-sum-exp.  The first segment (key tile 0) writes them to out / lse, the
-// others to the scratch slot of their CTA (a CTA starts at most one segment in
-// the middle of a pair).  attn_merge_kernel, launched right after on the same
-// stream, then merges the pieces of every split pair:
+// others to the scratch slot of their cluster (a cluster starts at most one
+// segment in the middle of a pair).  attn_merge_kernel, launched right after
+// on the same stream, then merges the pieces of every split pair:
 //   lse = log sum_s exp(lse_s),  out = sum_s exp(lse_s - lse) out_s.
+
+// Static-cap mode: the warps split into two groups that take alternate key
+// tiles (group q = warpgroups 2q, 2q+1 takes the tiles in S buffer q), each
+// warpgroup 64 keys of its group's tiles.  Both S buffers are then in work
+// at once, so one group's waits (for its logits, for its tensor-memory
+// stores, for its arrival) are covered by the other group's arithmetic.
+__device__ __forceinline__ void load_bias4(const float *brow, int j, int hk, int P,
+                                           float (&bn)[4]) {
+  const int J0 = j * 8 + hk * 4;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) bn[e] = (J0 + e < P) ? __ldg(brow + J0 + e) : 0.f;
+}
+
+__device__ __forceinline__ bool segment_static(const Segment &sg, const float *brow,
+                                               uint32_t tmem, uint32_t lane_base,
+                                               int g, const Params &p,
+                                               Barriers *bars, uint32_t rank,
+                                               uint32_t pf_remote, uint32_t &scount,
+                                               volatile int *abort, float &d) {
+  const int q = g >> 1, hk = g & 1;  // group (S buffer) and key half
+  const float2 sc = make_float2(p.qk_scale, p.qk_scale);
+  const float2 ap = make_float2(p.A, p.A), an = make_float2(-p.A, -p.A);
+  const int j0 = sg.kb + q;
+  // Bias cells of this group's next two tiles; the cells of tile j + 4 are
+  // requested right after tile j's arrival.
+  float bc[4] = {0.f, 0.f, 0.f, 0.f}, bn[4] = {0.f, 0.f, 0.f, 0.f};
+  if (j0 < sg.ke) load_bias4(brow, j0, hk, p.P, bc);
+  if (j0 + 2 < sg.ke) load_bias4(brow, j0 + 2, hk, p.P, bn);
+  for (int j = j0; j < sg.ke; j += 2) {
+    const int nvalid = (j + 1 == p.n_kt) ? p.last_valid : kKeys;
+    bool ok = mbar_wait(&bars->s_full[q], scount & 1u, abort, p.err, kSiteSoftS);
+    ++scount;
+    if (!__all_sync(0xffffffffu, ok)) return false;
+    tc_fence_after();
+    const uint32_t tS = tmem + 128u * q + 64 * hk + lane_base;
+    const float m = p.bias_mul;
+    if (nvalid == kKeys) {
+      d += tile_static<false>(tS, 64 * hk, bc[0] * m, bc[1] * m, sc, ap, an, nvalid);
+      d += tile_static<false>(tS + 32, 64 * hk + 32, bc[2] * m, bc[3] * m, sc, ap, an,
+                              nvalid);
+    } else {
+      d += tile_static<true>(tS, 64 * hk, bc[0] * m, bc[1] * m, sc, ap, an, nvalid);
+      d += tile_static<true>(tS + 32, 64 * hk + 32, bc[2] * m, bc[3] * m, sc, ap, an,
+                             nvalid);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane_id() == 0) {
+      if (rank == 0)
+        mbar_arrive(&bars->p_full[q]);
+      else
+        mbar_arrive_cluster(pf_remote);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) bc[e] = bn[e];
+    if (j + 4 < sg.ke) load_bias4(brow, j + 4, hk, p.P, bn);
+  }
+  return true;
+}
+
+// Running-max modes: every warpgroup takes every key tile (32 keys each),
+// the four threads of a row sharing its maximum per tile.
+template <int MODE>
+__device__ __forceinline__ bool segment_online(const Segment &sg, const float *brow,
+                                               uint32_t tmem, uint32_t lane_base,
+                                               int g, int r, const Params &p,
+                                               Barriers *bars, Xchg *xc,
+                                               uint32_t rank, uint32_t pf_remote0,
+                                               uint32_t pf_remote1, uint32_t &scount0,
+                                               uint32_t &scount1, uint32_t &xmcount,
+                                               uint32_t pvd, volatile int *abort,
+                                               float &m, float &d) {
+  float bc[2], bn[2] = {0.f, 0.f};
+  load_bias(brow, sg.kb, g, p.P, bc);
+  if (sg.kb + 1 < sg.ke) load_bias(brow, sg.kb + 1, g, p.P, bn);
+  for (int j = sg.kb; j < sg.ke; ++j) {
+    const uint32_t u = static_cast<uint32_t>(j - sg.kb) & 1u;
+    const int nvalid = (j + 1 == p.n_kt) ? p.last_valid : kKeys;
+    const float b0 = bc[0] * p.bias_mul, b1 = bc[1] * p.bias_mul;
+    const uint32_t sphase = u ? scount1++ : scount0++;
+    bool ok = mbar_wait(&bars->s_full[u], sphase & 1u, abort, p.err, kSiteSoftS);
+    if (!__all_sync(0xffffffffu, ok)) return false;
+    tc_fence_after();
+    const uint32_t tS = tmem + 128u * u + 32 * g + lane_base;
+    const uint32_t tO = tmem + kColO + 32 * g + lane_base;
+    // PV(j-1) is pv_done phase pvd + (j - 1 - kb); PV(j-2) has finished
+    // (s_full(j) was committed after it), so that phase is the current or
+    // the last completed one and its parity identifies it.
+    const uint32_t pv_parity = (pvd + static_cast<uint32_t>(j - 1 - sg.kb)) & 1u;
+    if (!tile_online<MODE>(tS, tO, g, r, u, j > sg.kb, pv_parity, b0, b1, p, nvalid,
+                           xc, bars, xmcount, abort, m, d))
+      return false;
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane_id() == 0) {
+      if (rank == 0)
+        mbar_arrive(&bars->p_full[u]);
+      else
+        mbar_arrive_cluster(u ? pf_remote1 : pf_remote0);
+    }
+    bc[0] = bn[0];
+    bc[1] = bn[1];
+    if (j + 2 < sg.ke) load_bias(brow, j + 2, g, p.P, bn);
+  }
+  return true;
+}
 
 template <int MODE>
 __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc,
                                              uint32_t tmem, const Params &p,
-                                             volatile int *abort) {
-  const int g = threadIdx.x >> 7;         // warpgroup: which key chunks
+                                             uint32_t rank, volatile int *abort) {
+  const int g = threadIdx.x >> 7;         // warpgroup
   const int r = threadIdx.x & 127;        // tile row == tensor-memory lane
-  const int wq = r >> 5;                  // warp's lane quarter
   const int h = r >> 4, il = r & 15;      // head, position inside the block
-  const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
-  const float2 sc = make_float2(p.qk_scale, p.qk_scale);
-  const float2 ap = make_float2(p.A, p.A), an = make_float2(-p.A, -p.A);
-  uint32_t scount[2] = {0, 0}, ocount[2] = {0, 0};
-  uint32_t xmcount[2] = {0, 0}, xdcount[2] = {0, 0};
+  const uint32_t lane_base = static_cast<uint32_t>(r >> 5) << 21;  // (32 * quarter) << 16
+  const uint32_t pf_remote0 = cluster_addr(&bars->p_full[0], 0);
+  const uint32_t pf_remote1 = cluster_addr(&bars->p_full[1], 0);
+  uint32_t scount0 = 0, scount1 = 0;  // s_full waits per S buffer
+  uint32_t ocount = 0, xmcount = 0, xdcount = 0;
+  uint32_t pvd = 0;  // pv_done phases completed before this segment
   bool ok = true;
   const int end = bars->range_end;
 
@@ -580,135 +702,109 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc,
     t += sg.ke - sg.kb;
     const int b = sg.item / p.pairs;
     const int I0 = (sg.item % p.pairs) * 2;
-    const int nX = (I0 + 1 < p.nb) ? 2 : 1;
-    const float *const brow[2] = {
-        p.bias + (static_cast<size_t>(h) * p.P + I0) * p.P,
-        p.bias + (static_cast<size_t>(h) * p.P + (I0 + (nX > 1 ? 1 : 0))) * p.P};
-    float m[2], d[2] = {0.f, 0.f};
-    float bn[2][2 * kChunks];
-#pragma unroll
-    for (int X = 0; X < 2; ++X) {
-      m[X] = (MODE == kStaticCap) ? p.A : -INFINITY;  // log2 units
-      load_bias(brow[X], sg.kb, g, p.P, bn[X]);
-    }
-    for (int j = sg.kb, i = 0; j < sg.ke && ok; ++j, ++i) {
-      const int nvalid = (j + 1 == p.n_kt) ? p.last_valid : kKeys;
-#pragma unroll
-      for (int X = 0; X < 2; ++X) {
-        if (X >= nX) break;
-        float bj[2 * kChunks];
-#pragma unroll
-        for (int e = 0; e < 2 * kChunks; ++e) bj[e] = bn[X][e] * p.bias_mul;
-        if (j + 1 < sg.ke) load_bias(brow[X], j + 1, g, p.P, bn[X]);
-
-        ok = mbar_wait(&bars->s_full[X], scount[X] & 1u, abort, p.err, kSiteSoftS);
-        ++scount[X];
-        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t tS = tmem + X * 128 + lane_base;
-        if constexpr (MODE == kStaticCap) {
-          if (nvalid == kKeys)
-            d[X] += part_tile_static<false>(tS, g, bj, sc, ap, an, nvalid);
-          else
-            d[X] += part_tile_static<true>(tS, g, bj, sc, ap, an, nvalid);
-        } else {
-          const uint32_t tO = tmem + 256 + X * 128 + lane_base;
-          ok = part_tile_online<MODE>(tS, tO, g, r, X, i, bj, p, nvalid, xc,
-                                      &bars->xm[X], xmcount[X], abort, m[X], d[X]);
-          if (!ok) break;
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        warp_arrive(&bars->p_full[X]);
-      }
+    const int I = tile_block(p, I0, rank);
+    const bool valid = I0 + static_cast<int>(rank) < p.nb;
+    const float *brow = p.bias + (static_cast<size_t>(h) * p.P + I) * p.P;
+    float m = (MODE == kStaticCap) ? p.A : -INFINITY;  // log2 units
+    float d = 0.f;
+    if constexpr (MODE == kStaticCap) {
+      // A thread of group q only ever waits on S buffer q: scount0 counts
+      // those waits.
+      ok = segment_static(sg, brow, tmem, lane_base, g, p, bars, rank,
+                          (g >> 1) ? pf_remote1 : pf_remote0, scount0, abort, d);
+    } else {
+      ok = segment_online<MODE>(sg, brow, tmem, lane_base, g, r, p, bars, xc, rank,
+                                pf_remote0, pf_remote1, scount0, scount1, xmcount,
+                                pvd, abort, m, d);
     }
     if (!ok) break;
+    pvd += static_cast<uint32_t>(sg.ke - sg.kb - 1);
 
-    // Epilogue: d = sum of the kWG partial sums; out = O / d over this
-    // segment's keys (this warpgroup's 32*kChunks columns of the row) and
-    // lse, to out / lse or, for a later piece of a split pair, to this CTA's
-    // scratch slot.
+    // Epilogue: d = sum of the four warpgroups' partial sums; out = O / d
+    // over this segment's keys (warpgroup g writes columns [32g, 32g + 32)
+    // of the row) and lse, to out / lse or, for a later piece of a split
+    // pair, to this cluster's scratch slot.  The copy of block I0 in an odd
+    // CTA past the end of an odd block count writes nothing.
+    ok = mbar_wait(&bars->o_full, ocount & 1u, abort, p.err, kSiteSoftO);
+    ++ocount;
+    if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+    tc_fence_after();
+    xc->dpart[g][r] = d;
+    ok = exchange(&bars->xd, xdcount, abort, p.err);
+    if (!ok) break;
+    float dsum = 0.f;
 #pragma unroll
-    for (int X = 0; X < 2; ++X) {
-      if (X >= nX) break;
-      ok = mbar_wait(&bars->o_full[X], ocount[X] & 1u, abort, p.err, kSiteSoftO);
-      ++ocount[X];
-      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-      tc_fence_after();
-      xc->dpart[X][g][r] = d[X];
-      ok = exchange(&bars->xd[X], xdcount[X], abort, p.err);
-      if (!ok) break;
-      float dsum = 0.f;
-#pragma unroll
-      for (int q = 0; q < kWG; ++q) dsum += xc->dpart[X][q][r];
-      const float inv_d = 1.f / dsum;
+    for (int q = 0; q < kWG; ++q) dsum += xc->dpart[q][r];
+    const float inv_d = 1.f / dsum;
+    uint32_t o[32];
+    tmem_ld32(tmem + kColO + 32 * g + lane_base, o);
+    tmem_wait_ld(o);
+    if (valid) {
       const size_t row = (static_cast<size_t>(b) * kH + h) * p.L +
-                         static_cast<size_t>(I0 + X) * 16 + il;
-      const int c0 = 32 * kChunks * g;
+                         static_cast<size_t>(I) * 16 + il;
       float *orow_base;
       float *lse_dst;
       if (sg.kb == 0) {
         orow_base = p.out + row * kD;
         lse_dst = p.lse + row;
       } else {
-        const size_t slot = (static_cast<size_t>(blockIdx.x) * 2 + X) * 128 + r;
+        const size_t slot =
+            (static_cast<size_t>(cluster_index()) * 2 + rank) * 128 + r;
         orow_base = p.ws_out + slot * kD;
         lse_dst = p.ws_lse + slot;
       }
-      float4 *orow = reinterpret_cast<float4 *>(orow_base + c0);
-      const uint32_t tO = tmem + 256 + X * 128 + lane_base + c0;
-#pragma unroll 1
-      for (int c = 0; c < kChunks; ++c) {
-        uint32_t o[32];
-        tmem_ld32(tO + c * 32, o);
-        tmem_wait_ld(o);
+      float4 *orow = reinterpret_cast<float4 *>(orow_base + 32 * g);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          orow[c * 8 + e] = make_float4(__uint_as_float(o[4 * e]) * inv_d,
-                                        __uint_as_float(o[4 * e + 1]) * inv_d,
-                                        __uint_as_float(o[4 * e + 2]) * inv_d,
-                                        __uint_as_float(o[4 * e + 3]) * inv_d);
-        }
+      for (int e = 0; e < 8; ++e) {
+        orow[e] = make_float4(__uint_as_float(o[4 * e]) * inv_d,
+                              __uint_as_float(o[4 * e + 1]) * inv_d,
+                              __uint_as_float(o[4 * e + 2]) * inv_d,
+                              __uint_as_float(o[4 * e + 3]) * inv_d);
       }
-      if (g == 0) *lse_dst = (m[X] + lg2_approx(dsum)) * kLn2;
-      tc_fence_before();
+      if (g == 0) *lse_dst = (m + lg2_approx(dsum)) * kLn2;
     }
+    tc_fence_before();
   }
 }
 
 // --------------------------------------------------------------------------
 template <int MODE>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
-  uint8_t *q_s = smem_raw + pad;                 // 2 query tiles
-  uint8_t *kv_s = q_s + 2 * kTileBytes;          // K/V ring
-  Barriers *bars = reinterpret_cast<Barriers *>(kv_s + kStages * kTileBytes);
-  auto *xc = reinterpret_cast<struct Xchg *>(reinterpret_cast<uint8_t *>(bars) +
-                                             sizeof(Barriers));
+  uint8_t *q_s = smem_raw + pad;             // this CTA's query tile
+  uint8_t *kv_s = q_s + kQTileBytes;         // K/V ring
+  Barriers *bars = reinterpret_cast<Barriers *>(kv_s + kStages * kSlotBytes);
+  auto *xc = reinterpret_cast<Xchg *>(reinterpret_cast<uint8_t *>(bars) +
+                                      sizeof(Barriers));
   const int warp = threadIdx.x >> 5;
+  const uint32_t rank = cluster_ctarank();
 
   if (threadIdx.x == 0) {
-    for (int X = 0; X < 2; ++X) {
-      mbar_init(&bars->q_full[X], 1);
-      mbar_init(&bars->q_empty[X], 1);
-      mbar_init(&bars->s_full[X], 1);
-      mbar_init(&bars->p_full[X], kSoftWarps);
-      mbar_init(&bars->xm[X], kSoftWarps);
-      mbar_init(&bars->xd[X], kSoftWarps);
-      mbar_init(&bars->o_full[X], 1);
-    }
+    mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->q_peer, 1);
+    mbar_init(&bars->q_empty, 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars->kv_full[s], 1);
+      mbar_init(&bars->kv_peer[s], 1);
       mbar_init(&bars->kv_empty[s], 1);
     }
+    for (int u = 0; u < 2; ++u) {
+      mbar_init(&bars->s_full[u], 1);
+      // Static cap: one warp group per S buffer; otherwise every warp.
+      mbar_init(&bars->p_full[u], MODE == kStaticCap ? kPairSoftWarps / 2 : kPairSoftWarps);
+    }
+    mbar_init(&bars->pv_done, 1);
+    mbar_init(&bars->o_full, 1);
+    mbar_init(&bars->xm, kSoftWarps);
+    mbar_init(&bars->xd, kSoftWarps);
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
-    bars->range_begin = range_start(p, blockIdx.x);
-    bars->range_end = range_start(p, blockIdx.x + 1);
+    bars->range_begin = range_start(p, cluster_index());
+    bars->range_end = range_start(p, cluster_index() + 1);
     fence_mbar_init();
   }
   if (warp == kWarpLoad && lane_id() == 0) {
@@ -717,44 +813,52 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tensormap(&tm_v);
   }
   if (warp == kWarpMma) {
-    tmem_alloc(&bars->tmem_base, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc2(&bars->tmem_base, kTmemCols);
+    tmem_relinquish2();
   }
+  // Both CTAs' barriers are initialised and their tensor memory allocated
+  // before either CTA signals the other.
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   volatile int *abort = &bars->abort;
 
   if (warp >= kWarpLoad) {
     regs_dec<kRegsLow>();
-    if (warp == kWarpLoad && lane_id() == 0)
-      producer(&tm_q, &tm_k, &tm_v, q_s, kv_s, bars, p, abort);
-    else if (warp == kWarpMma && lane_id() == 0)
-      mma_issuer(q_s, kv_s, bars, tmem, p, abort);
+    if (warp == kWarpLoad && lane_id() == 0) {
+      producer(&tm_q, &tm_k, &tm_v, q_s, kv_s, bars, p, rank, abort);
+    } else if (warp == kWarpMma && lane_id() == 0) {
+      if (rank == 0)
+        mma_issuer<MODE != kStaticCap>(q_s, kv_s, bars, tmem, p, abort);
+      else
+        relay(bars, p, abort);
+    }
   } else {
-    if constexpr (kRegsHigh > kRegsLaunch) regs_inc<kRegsHigh>();
-    softmax_role<MODE>(bars, xc, tmem, p, abort);
+    softmax_role<MODE>(bars, xc, tmem, p, rank, abort);
   }
   __syncwarp();
+  // No CTA leaves while the other may still use its shared or tensor memory:
+  // the even CTA's MMAs have drained and the odd CTA's remote arrivals are
+  // done once every thread of both CTAs is here.
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();
   if (warp == kWarpMma) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc2(tmem, kTmemCols);
   }
 }
 
 // --------------------------------------------------------------------------
-// Split-pair merge.  One block per CTA boundary; the block whose boundary is
-// the first one inside a pair merges that pair.  Thread t takes query tile
-// t / 128 and row t % 128 and merges the whole 128-column row, so it reads
-// the first piece's lse before it overwrites it.
+// Split-pair merge.  One block per cluster boundary; the block whose boundary
+// is the first one inside a pair merges that pair.  Thread t takes query
+// tile t / 128 and row t % 128 and merges the whole 128-column row, so it
+// reads the first piece's lse before it overwrites it.
 constexpr int kMergeThreads = 256;
 
 __global__ void __launch_bounds__(kMergeThreads)
     attn_merge_kernel(const Params p, int grid) {
-  const int c = blockIdx.x + 1;  // boundary between CTA c - 1 and CTA c
+  const int c = blockIdx.x + 1;  // boundary between cluster c - 1 and cluster c
   const int W = p.n_items * p.n_kt;
   auto start = [&](int cc) {
     return static_cast<int>(static_cast<long long>(W) * cc / grid);
@@ -830,11 +934,12 @@ static bool encode_map(EncodeTiledFn enc, CUtensorMap *map, const void *base,
   return r == CUDA_SUCCESS;
 }
 
+// One-time per-device setup of a mode's kernel: shared-memory opt-in, the
+// register check, and how many 2-CTA clusters can be resident at once.
 template <int MODE>
-static cudaError_t launch_mode(const CUtensorMap &tq, const CUtensorMap &tk,
-                               const CUtensorMap &tv, const attn::Params &p,
-                               int grid, cudaStream_t stream) {
+static cudaError_t configure_mode(int *max_clusters) {
   static int configured[64] = {0};
+  static int clusters[64] = {0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -845,17 +950,33 @@ static cudaError_t launch_mode(const CUtensorMap &tq, const CUtensorMap &tk,
     cudaFuncAttributes fa;
     e = cudaFuncGetAttributes(&fa, attn::attn_fwd_kernel<MODE>);
     if (e != cudaSuccess) return e;
-    if (static_cast<uint32_t>(fa.numRegs) * attn::kThreads <
-        attn::kSoftThreads * attn::kRegsHigh + 128 * attn::kRegsLow)
+    if (static_cast<uint32_t>(fa.numRegs) < attn::kRegsLaunch)
       return cudaErrorInvalidConfiguration;
     e = cudaFuncSetAttribute(attn::attn_fwd_kernel<MODE>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(attn::kSmemBytes));
     if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(attn::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = attn::kSmemBytes;
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, attn::attn_fwd_kernel<MODE>, &cfg);
+    if (e != cudaSuccess) return e;
+    if (n < 1) return cudaErrorInvalidConfiguration;
+    clusters[dev] = n;
     configured[dev] = 1;
   }
+  *max_clusters = clusters[dev];
+  return cudaSuccess;
+}
+
+template <int MODE>
+static cudaError_t launch_mode(const CUtensorMap &tq, const CUtensorMap &tk,
+                               const CUtensorMap &tv, const attn::Params &p,
+                               int clusters, cudaStream_t stream) {
   attn::attn_fwd_kernel<MODE>
-      <<<grid, attn::kThreads, attn::kSmemBytes, stream>>>(tq, tk, tv, p);
+      <<<2 * clusters, attn::kThreads, attn::kSmemBytes, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 
@@ -876,10 +997,11 @@ cudaError_t launch_attn_fwd(const AttnLaunch &a) {
     const cuuint64_t dims[3] = {kD, static_cast<cuuint64_t>(L),
                                 static_cast<cuuint64_t>(B)};
     const cuuint64_t strides[2] = {kD * 2, static_cast<cuuint64_t>(L) * kD * 2};
-    const cuuint32_t box[3] = {64, kKeys, 1};
-    if (!encode_map(a.encode, &tk, a.k, 3, dims, strides, box))
+    const cuuint32_t kbox[3] = {64, kKeys / 2, 1};  // a CTA's 64 keys, one 64-wide half
+    const cuuint32_t vbox[3] = {64, kKeys, 1};      // a CTA's 64 value columns, 128 keys
+    if (!encode_map(a.encode, &tk, a.k, 3, dims, strides, kbox))
       return cudaErrorInvalidValue;
-    if (!encode_map(a.encode, &tv, a.v, 3, dims, strides, box))
+    if (!encode_map(a.encode, &tv, a.v, 3, dims, strides, vbox))
       return cudaErrorInvalidValue;
   }
   Params p;
@@ -908,35 +1030,44 @@ cudaError_t launch_attn_fwd(const AttnLaunch &a) {
     p.bias_mul = 1.0f / cap;
     p.A = cap * kLog2e;
   }
-  // One CTA per SM, never more CTAs than (pair, key tile) steps or scratch
-  // slots.  Whole pairs per CTA unless that leaves the grid badly balanced:
-  // a split pair costs a second pass over its rows (partial results, then
-  // the merge), so whole pairs win while the busiest CTA's extra work stays
-  // below kSplitGain pairs.
+  int max_clusters = 0;
+  cudaError_t e;
+  switch (mode) {
+    case kStaticCap: e = configure_mode<kStaticCap>(&max_clusters); break;
+    case kOnlineCap: e = configure_mode<kOnlineCap>(&max_clusters); break;
+    default: e = configure_mode<kNoCap>(&max_clusters); break;
+  }
+  if (e != cudaSuccess) return e;
+  // One cluster per resident SM pair, never more clusters than (pair, key
+  // tile) steps or scratch slots.  Whole pairs per cluster unless that
+  // leaves the grid badly balanced: a split pair costs a second pass over
+  // its rows (partial results, then the merge), so whole pairs win while the
+  // busiest cluster's extra work stays below kSplitGain pairs.
   const long long steps = static_cast<long long>(p.n_items) * p.n_kt;
   if (steps != attn_work_steps(B, L) || steps > (1ll << 30))
     return cudaErrorInvalidValue;
-  int grid = a.num_sms < a.scratch_slots ? a.num_sms : a.scratch_slots;
-  if (steps < grid) grid = static_cast<int>(steps);
-  if (grid < 1) return cudaErrorInvalidValue;
+  int clusters = a.num_sms / 2;
+  if (max_clusters < clusters) clusters = max_clusters;
+  if (a.scratch_slots < clusters) clusters = a.scratch_slots;
+  if (steps < clusters) clusters = static_cast<int>(steps);
+  if (clusters < 1) return cudaErrorInvalidValue;
   {
     constexpr double kSplitGain = 0.5;
-    const long long per = (p.n_items + grid - 1) / grid;  // pairs, busiest CTA
-    const double even = static_cast<double>(p.n_items) / grid;
+    const long long per = (p.n_items + clusters - 1) / clusters;  // busiest cluster
+    const double even = static_cast<double>(p.n_items) / clusters;
     p.whole = (per - even <= kSplitGain) ? 1 : 0;
-    if (p.whole && p.n_items < grid) grid = p.n_items;
+    if (p.whole && p.n_items < clusters) clusters = p.n_items;
   }
   char *base = static_cast<char *>(a.scratch);
   p.ws_out = reinterpret_cast<float *>(base);
   p.ws_lse = reinterpret_cast<float *>(base + a.scratch_slots * kAttnSlotOutBytes);
-  cudaError_t e;
   switch (mode) {
-    case kStaticCap: e = launch_mode<kStaticCap>(tq, tk, tv, p, grid, a.stream); break;
-    case kOnlineCap: e = launch_mode<kOnlineCap>(tq, tk, tv, p, grid, a.stream); break;
-    default: e = launch_mode<kNoCap>(tq, tk, tv, p, grid, a.stream); break;
+    case kStaticCap: e = launch_mode<kStaticCap>(tq, tk, tv, p, clusters, a.stream); break;
+    case kOnlineCap: e = launch_mode<kOnlineCap>(tq, tk, tv, p, clusters, a.stream); break;
+    default: e = launch_mode<kNoCap>(tq, tk, tv, p, clusters, a.stream); break;
   }
-  if (e != cudaSuccess || grid < 2 || p.whole) return e;
-  attn_merge_kernel<<<grid - 1, kMergeThreads, 0, a.stream>>>(p, grid);
+  if (e != cudaSuccess || clusters < 2 || p.whole) return e;
+  attn_merge_kernel<<<clusters - 1, kMergeThreads, 0, a.stream>>>(p, clusters);
   return cudaGetLastError();
 }
 
