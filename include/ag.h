@@ -105,9 +105,10 @@ ag_status ag_pair_bias_project(const float *pair, const float *W, float *bias,
  * row sums use their fp32 values.
  *
  * Scratch: to keep every SM busy to the end, a pair of query tiles may have
- * its keys split between SMs; each piece's partial result goes through a
- * scratch buffer of 132,096 bytes per SM (19.6 MB on a 148-SM B200) and a
- * second kernel on the same stream merges the pieces (by log-sum-exp).  The
+ * its keys split between SM pairs (the kernel runs on 2-CTA clusters); each
+ * piece's partial result goes through a scratch buffer of 132,096 bytes per
+ * SM (19.6 MB on a 148-SM B200; half of it is used) and a second kernel on
+ * the same stream merges the pieces (by log-sum-exp).  The
  * first call on a device allocates that buffer with cudaMalloc; it is kept
  * until the process exits.  Calls whose kernels overlap on the device (e.g.
  * on two streams at once) must not run concurrently, because they share it.
@@ -133,8 +134,8 @@ ag_status ag_attn_fwd(const void *q, const void *k, const void *v,
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before any stream capture.
  *   - Returns AG_ERR_SCRATCH, launching nothing, when the call would use more
- *     than 148 slots (one per CTA of its grid: min(SM count, work steps)),
- *     i.e. on a device with more than 148 SMs.
+ *     than 148 slots (one per 2-CTA cluster of its grid: min(SM count / 2,
+ *     work steps)), i.e. on a device with more than 296 SMs.
  *   - Every call shares the one array and it keeps the last call's contents;
  *     nothing in it needs to start at zero.  Calls that overlap on the GPU
  *     (two streams at once, or together with ag_attn_fwd's kernels on another

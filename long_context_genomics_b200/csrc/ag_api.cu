@@ -95,7 +95,7 @@ ag_status get_encoder(EncodeTiledFn *fn) {
 }
 
 // Scratch for ag_attn_fwd_noalloc: the same split-pair slots as the
-// allocated scratch, for at most kStaticScratchSlots CTAs, in a file-scope
+// allocated scratch, for at most kStaticScratchSlots clusters, in a file-scope
 // array that every device loading this library holds until the process exits.
 constexpr int kStaticScratchSlots = 148;
 constexpr size_t kStaticScratchBytes =
@@ -289,11 +289,12 @@ ag_status ag_attn_fwd_noalloc(const void *q, const void *k, const void *v,
   ag::DeviceInfo *dev = nullptr;
   ag_status st = ag::device_info(&dev);
   if (st != AG_OK) return st;
-  // One scratch slot per CTA; the grid is one CTA per SM (fewer for tiny
-  // problems).  A device whose grid would need more slots than the static
-  // buffer holds is refused rather than given a slower grid.
+  // One scratch slot per cluster; the grid is one 2-CTA cluster per SM pair
+  // (fewer for tiny problems).  A device whose grid would need more slots
+  // than the static buffer holds is refused rather than given a slower grid.
   const int64_t steps = ag::attn_work_steps(B, L);
-  const int64_t slots = steps < dev->num_sms ? steps : dev->num_sms;
+  const int64_t pairs_of_sms = dev->num_sms / 2;
+  const int64_t slots = steps < pairs_of_sms ? steps : pairs_of_sms;
   if (slots > ag::kStaticScratchSlots) return AG_ERR_SCRATCH;
   ag::EncodeTiledFn enc = nullptr;
   st = ag::get_encoder(&enc);

@@ -73,10 +73,10 @@ constexpr int kWarpLoad = 4 * kWG;          // TMA producer
 constexpr int kWarpMma = 4 * kWG + 1;       // MMA issuer (even CTA) / relay (odd)
 // Registers per thread: the launch gives every thread kRegsLaunch (the cap
 // for this block size, which ptxas allocates when setmaxnreg is present; the
-// launcher checks it); the producer warpgroup then drops to kRegsLow (below
-// 80 the MMA warp spills).  The softmax needs no more than the launch count.
+// launcher checks it); the producer warpgroup then drops to kRegsLow (with
+// fewer the MMA and relay threads spill).  The softmax keeps the launch count.
 constexpr uint32_t kRegsLaunch = 96;
-constexpr uint32_t kRegsLow = 80;
+constexpr uint32_t kRegsLow = 88;
 static_assert(kSoftThreads * kRegsLaunch + 128 * kRegsLow <= kThreads * kRegsLaunch,
               "register split exceeds the launch allocation");
 constexpr uint32_t kTmemCols = 512;
@@ -100,13 +100,15 @@ enum Site : unsigned {
   kSiteXchg = 9, kSiteSoftPV = 10, kSiteRelay = 11
 };
 
-// Per-CTA barriers.  q_peer, kv_peer and p_full are used in the even CTA
-// only (the odd CTA's relay and softmax warps arrive on them remotely);
-// q_empty, kv_empty, s_full, pv_done and o_full are signalled in both CTAs
-// by the even CTA's MMA commits.
+// Per-CTA barriers.  In the even CTA, q_full and kv_full also count the odd
+// CTA's relay (two arrivals: the local producer's, with the byte count, and
+// the relay's), so the MMA thread waits once for both halves of a load;
+// p_full is used in the even CTA only (the odd CTA's softmax warps arrive on
+// it remotely).  q_empty, kv_empty, s_full, pv_done and o_full are signalled
+// in both CTAs by the even CTA's MMA commits.
 struct __align__(8) Barriers {
-  uint64_t q_full, q_peer, q_empty;
-  uint64_t kv_full[kStages], kv_peer[kStages], kv_empty[kStages];
+  uint64_t q_full, q_empty;
+  uint64_t kv_full[kStages], kv_empty[kStages];
   // s_full / p_full by S buffer: a softmax may finish key tile j + 1 before
   // the MMA warp has taken key tile j's arrivals.
   uint64_t s_full[2], p_full[2];
@@ -311,7 +313,7 @@ __device__ __forceinline__ void producer(const CUtensorMap *tm_q,
 // order, that this CTA's half of each Q / K / V load has landed.
 __device__ __forceinline__ void relay(Barriers *bars, const Params &p,
                                       volatile int *abort) {
-  const uint32_t q_peer = cluster_addr(&bars->q_peer, 0);
+  const uint32_t q_leader = cluster_addr(&bars->q_full, 0);
   uint32_t qcount = 0, kv = 0;
   bool ok = true;
   const int end = bars->range_end;
@@ -321,14 +323,14 @@ __device__ __forceinline__ void relay(Barriers *bars, const Params &p,
     ok = mbar_wait(&bars->q_full, qcount & 1u, abort, p.err, kSiteRelay);
     ++qcount;
     if (!ok) break;
-    mbar_arrive_cluster(q_peer);
+    mbar_arrive_cluster(q_leader);
     ok = for_each_ring_load(sg, [&](int, int, bool) {
       const uint32_t slot = kv % kStages;
       if (!mbar_wait(&bars->kv_full[slot], (kv / kStages) & 1u, abort, p.err,
                      kSiteRelay))
         return false;
       ++kv;
-      mbar_arrive_cluster(cluster_addr(&bars->kv_peer[slot], 0));
+      mbar_arrive_cluster(cluster_addr(&bars->kv_full[slot], 0));
       return true;
     });
   }
@@ -347,21 +349,23 @@ __device__ __forceinline__ void mma_issuer(uint8_t *q_s, uint8_t *kv_s,
   uint32_t qcount = 0, kv = 0;
   uint32_t pbits = 0;  // bit u: parity of the next p_full[u] phase
   bool ok = true;
-  // Both halves of the next ring load: this CTA's copy and the peer's relay.
+  // Both halves of the next ring load: this CTA's copy and the peer's relay
+  // (both arrive on this CTA's kv_full).  The odd CTA's arrivals here (relay,
+  // softmax) are relaxed (see mbar_arrive_cluster), so these waits acquire at
+  // CTA scope: a cluster-scope acquire would order nothing more and costs
+  // about 180 cycles per wait on this thread (measured).
   auto wait_kv = [&](uint32_t &slot) {
     slot = kv % kStages;
     const uint32_t ph = (kv / kStages) & 1u;
     ++kv;
-    return mbar_wait(&bars->kv_full[slot], ph, abort, p.err, kSiteMmaKV) &&
-           mbar_wait_cluster(&bars->kv_peer[slot], ph, abort, p.err, kSiteMmaKV);
+    return mbar_wait(&bars->kv_full[slot], ph, abort, p.err, kSiteMmaKV);
   };
   const int end = bars->range_end;
   for (int t = bars->range_begin; t < end && ok;) {
     const Segment sg = segment_at(p, t, end);
     t += sg.ke - sg.kb;
     const int n = sg.ke - sg.kb;
-    ok = mbar_wait(&bars->q_full, qcount & 1u, abort, p.err, kSiteMmaQ) &&
-         mbar_wait_cluster(&bars->q_peer, qcount & 1u, abort, p.err, kSiteMmaQ);
+    ok = mbar_wait(&bars->q_full, qcount & 1u, abort, p.err, kSiteMmaQ);
     ++qcount;
     if (!ok) break;
     // Slot load 0: S(kb) into buffer 0 and S(kb+1) into buffer 1.
@@ -384,8 +388,7 @@ __device__ __forceinline__ void mma_issuer(uint8_t *q_s, uint8_t *kv_s,
       uint32_t slot;  // V(j) in part 1, K(j+2) (while it exists) in part 0
       ok = wait_kv(slot);
       if (!ok) break;
-      ok = mbar_wait_cluster(&bars->p_full[u], (pbits >> u) & 1u, abort, p.err,
-                             kSiteMmaP);
+      ok = mbar_wait(&bars->p_full[u], (pbits >> u) & 1u, abort, p.err, kSiteMmaP);
       pbits ^= 1u << u;
       if (!ok) break;
       tc_fence_after();
@@ -595,11 +598,11 @@ __device__ __forceinline__ bool segment_static(const Segment &sg, const float *b
   const float2 sc = make_float2(p.qk_scale, p.qk_scale);
   const float2 ap = make_float2(p.A, p.A), an = make_float2(-p.A, -p.A);
   const int j0 = sg.kb + q;
-  // Bias cells of this group's next two tiles; the cells of tile j + 4 are
-  // requested right after tile j's arrival.
-  float bc[4] = {0.f, 0.f, 0.f, 0.f}, bn[4] = {0.f, 0.f, 0.f, 0.f};
+  // Bias cells of this group's next tile.  The cells of tile j + 2 are
+  // requested right after tile j's arrival (a load in flight would hold up
+  // that arrival); they land while the group waits for tile j + 2's logits.
+  float bc[4] = {0.f, 0.f, 0.f, 0.f};
   if (j0 < sg.ke) load_bias4(brow, j0, hk, p.P, bc);
-  if (j0 + 2 < sg.ke) load_bias4(brow, j0 + 2, hk, p.P, bn);
   for (int j = j0; j < sg.ke; j += 2) {
     const int nvalid = (j + 1 == p.n_kt) ? p.last_valid : kKeys;
     bool ok = mbar_wait(&bars->s_full[q], scount & 1u, abort, p.err, kSiteSoftS);
@@ -626,9 +629,7 @@ __device__ __forceinline__ bool segment_static(const Segment &sg, const float *b
       else
         mbar_arrive_cluster(pf_remote);
     }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) bc[e] = bn[e];
-    if (j + 4 < sg.ke) load_bias4(brow, j + 4, hk, p.P, bn);
+    if (j + 2 < sg.ke) load_bias4(brow, j + 2, hk, p.P, bc);
   }
   return true;
 }
@@ -784,12 +785,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t rank = cluster_ctarank();
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars->q_full, 1);
-    mbar_init(&bars->q_peer, 1);
+    const uint32_t loads = rank == 0 ? 2 : 1;  // producer (+ relay, even CTA)
+    mbar_init(&bars->q_full, loads);
     mbar_init(&bars->q_empty, 1);
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bars->kv_full[s], 1);
-      mbar_init(&bars->kv_peer[s], 1);
+      mbar_init(&bars->kv_full[s], loads);
       mbar_init(&bars->kv_empty[s], 1);
     }
     for (int u = 0; u < 2; ++u) {
@@ -850,15 +850,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 }
 
 // --------------------------------------------------------------------------
-// Split-pair merge.  One block per cluster boundary; the block whose boundary
-// is the first one inside a pair merges that pair.  Thread t takes query
-// tile t / 128 and row t % 128 and merges the whole 128-column row, so it
-// reads the first piece's lse before it overwrites it.
+// Split-pair merge.  kMergeBlocksPerBoundary blocks per cluster boundary; only
+// the boundary that is the first one inside a pair merges that pair.  One
+// warp per output row (query tile row / 128, row % 128): lane l merges
+// columns [4l, 4l + 4) over the pieces, and lane 0 writes the merged lse
+// once every lane has read the first piece's.
 constexpr int kMergeThreads = 256;
+constexpr int kMergeRowsPerBlock = kMergeThreads / 32;
+constexpr int kMergeBlocksPerBoundary = 2 * 128 / kMergeRowsPerBlock;
 
 __global__ void __launch_bounds__(kMergeThreads)
     attn_merge_kernel(const Params p, int grid) {
-  const int c = blockIdx.x + 1;  // boundary between cluster c - 1 and cluster c
+  const int c = blockIdx.x / kMergeBlocksPerBoundary + 1;  // boundary between clusters c-1, c
   const int W = p.n_items * p.n_kt;
   auto start = [&](int cc) {
     return static_cast<int>(static_cast<long long>(W) * cc / grid);
@@ -867,7 +870,7 @@ __global__ void __launch_bounds__(kMergeThreads)
   if (tb % p.n_kt == 0) return;  // the boundary falls between pairs
   const int item = tb / p.n_kt;
   const int prev = start(c - 1);
-  if (c > 1 && prev / p.n_kt == item && prev % p.n_kt != 0) return;  // merged by an earlier block
+  if (c > 1 && prev / p.n_kt == item && prev % p.n_kt != 0) return;  // merged at an earlier boundary
   auto owner = [&](int t) {
     return static_cast<int>(((static_cast<long long>(t) + 1) * grid - 1) / W);
   };
@@ -876,8 +879,11 @@ __global__ void __launch_bounds__(kMergeThreads)
   const int b = item / p.pairs;
   const int I0 = (item % p.pairs) * 2;
   const int nX = (I0 + 1 < p.nb) ? 2 : 1;
-  const int X = threadIdx.x >> 7, r = threadIdx.x & 127;
+  const int tr = (blockIdx.x % kMergeBlocksPerBoundary) * kMergeRowsPerBlock +
+                 static_cast<int>(threadIdx.x >> 5);  // 0 .. 255
+  const int X = tr >> 7, r = tr & 127;
   if (X >= nX) return;
+  const int lane = static_cast<int>(threadIdx.x & 31);
   const int h = r >> 4, il = r & 15;
   const size_t row = (static_cast<size_t>(b) * kH + h) * p.L +
                      static_cast<size_t>(I0 + X) * 16 + il;
@@ -891,30 +897,20 @@ __global__ void __launch_bounds__(kMergeThreads)
   for (int s = 0; s < n_seg; ++s)
     sum += ex2_approx(((s == 0 ? p.lse[row] : p.ws_lse[slot(s)]) - M) * kLog2e);
   const float lse = M + lg2_approx(sum) * kLn2;
-  float4 *dst = reinterpret_cast<float4 *>(p.out + row * kD);
-#pragma unroll 1
-  for (int part = 0; part < kD / 16; ++part) {
-    float4 acc[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) acc[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < n_seg; ++s) {
-      const float l = s == 0 ? p.lse[row] : p.ws_lse[slot(s)];
-      const float wgt = ex2_approx((l - lse) * kLog2e);
-      const float4 *src = reinterpret_cast<const float4 *>(
-          s == 0 ? p.out + row * kD : p.ws_out + slot(s) * kD);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float4 v = src[part * 4 + e];
-        acc[e].x = fmaf(wgt, v.x, acc[e].x);
-        acc[e].y = fmaf(wgt, v.y, acc[e].y);
-        acc[e].z = fmaf(wgt, v.z, acc[e].z);
-        acc[e].w = fmaf(wgt, v.w, acc[e].w);
-      }
-    }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) dst[part * 4 + e] = acc[e];
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = 0; s < n_seg; ++s) {
+    const float l = s == 0 ? p.lse[row] : p.ws_lse[slot(s)];
+    const float wgt = ex2_approx((l - lse) * kLog2e);
+    const float4 v = reinterpret_cast<const float4 *>(
+        s == 0 ? p.out + row * kD : p.ws_out + slot(s) * kD)[lane];
+    acc.x = fmaf(wgt, v.x, acc.x);
+    acc.y = fmaf(wgt, v.y, acc.y);
+    acc.z = fmaf(wgt, v.z, acc.z);
+    acc.w = fmaf(wgt, v.w, acc.w);
   }
-  p.lse[row] = lse;
+  reinterpret_cast<float4 *>(p.out + row * kD)[lane] = acc;
+  __syncwarp();  // every lane has read p.lse[row]
+  if (lane == 0) p.lse[row] = lse;
 }
 
 }  // namespace attn
@@ -1067,7 +1063,8 @@ cudaError_t launch_attn_fwd(const AttnLaunch &a) {
     default: e = launch_mode<kNoCap>(tq, tk, tv, p, clusters, a.stream); break;
   }
   if (e != cudaSuccess || clusters < 2 || p.whole) return e;
-  attn_merge_kernel<<<clusters - 1, kMergeThreads, 0, a.stream>>>(p, clusters);
+  attn_merge_kernel<<<(clusters - 1) * kMergeBlocksPerBoundary, kMergeThreads, 0,
+                      a.stream>>>(p, clusters);
   return cudaGetLastError();
 }
 

@@ -316,37 +316,6 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
                    cluster_bar)
                : "memory");
 }
-// As mbar_test, with acquire at cluster scope (pairs with arrivals made by
-// the other CTA of the pair).
-__device__ __forceinline__ bool mbar_test_cluster(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0u;
-}
-// Bounded wait (as mbar_wait) for barriers that the other CTA arrives at.
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity,
-                                                  volatile int *abort,
-                                                  unsigned *err, unsigned site) {
-  const uint32_t a = smem_u32(bar);
-  if (mbar_test_cluster(a, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (true) {
-    if (mbar_test_cluster(a, parity)) return true;
-    if (*abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-      *abort = 1;
-      if (err) atomicCAS(err, 0u, (site << 8) | kErrTimeout);
-      return false;
-    }
-  }
-}
-
 // tcgen05 with .cta_group::2: one warp of each CTA of the pair allocates
 // (and later frees) the same columns in both CTAs' tensor memory; one thread
 // of the even CTA issues MMAs of M = 256 whose A rows 0..127 come from the
