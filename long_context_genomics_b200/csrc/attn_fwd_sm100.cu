@@ -55,14 +55,18 @@ constexpr int kKeys = static_cast<int>(kAttnKeyTile);  // keys per key tile
 static_assert(kKeys == 128, "the tile layout below assumes 128-key tiles");
 constexpr int kQTileBytes = 128 * kD * 2;     // this CTA's query tile (bf16)
 constexpr int kQHalfBytes = kQTileBytes / 2;  // one 64-wide (128-byte) half
-// A ring slot holds what one key-tile step needs from this CTA: its half of
-// a V tile (128 keys x 64 value columns, 16 KB) and its half of the K tile
-// two steps ahead (64 keys x 128, two 64-wide halves of 8 KB), or, first in
-// a segment, the halves of the segment's first two K tiles.
+// A step load is what one key-tile step needs from this CTA: its half of a
+// V tile (128 keys x 64 value columns, 16 KB) and its half of the K tile two
+// steps ahead (64 keys x 128, two 64-wide halves of 8 KB), or, first in a
+// segment, the halves of the segment's first two K tiles.  A ring slot holds
+// two consecutive step loads, so the MMA thread waits for data and releases
+// it once per two steps (each mbarrier operation costs it about 180 cycles
+// while the tensor core is busy, measured).
 constexpr int kPartBytes = 16384;            // one K half or one V half
 constexpr int kKHalfBytes = kPartBytes / 2;  // a K half's 64-wide half
-constexpr int kSlotBytes = 2 * kPartBytes;
-constexpr int kStages = 5;
+constexpr int kStepBytes = 2 * kPartBytes;
+constexpr int kSlotBytes = 2 * kStepBytes;
+constexpr int kStages = 2;
 constexpr int kWG = 4;                      // softmax warpgroups
 constexpr int kSoftThreads = 128 * kWG;
 constexpr int kSoftWarps = 4 * kWG;         // per CTA
@@ -184,16 +188,26 @@ __device__ __forceinline__ Segment segment_at(const Params &p, int t, int end) {
 }
 
 // K/V ring order, shared by the producers, the relay and the MMA warp: for a
-// segment with key tiles [kb, ke), slot load 0 holds K(kb) (part 0) and
-// K(kb+1) (part 1); slot load i = 1 .. n holds K(kb+i+1) (part 0, while it
-// exists) and V(kb+i-1) (part 1).  S runs two key tiles ahead of PV.
-// f(i, k_tile or -1, second part: is_v ? v_tile : k_tile or -1, is_v).
-template <typename F>
-__device__ __forceinline__ bool for_each_ring_load(const Segment &sg, F &&f) {
+// segment with key tiles [kb, ke) (n of them), step load 0 holds K(kb) (part
+// 0) and K(kb+1) (part 1); step load i = 1 .. n holds K(kb+i+1) (part 0,
+// while it exists) and V(kb+i-1) (part 1).  S runs two key tiles ahead of PV.
+// Step loads 2d and 2d+1 share ring slot load d (the last may be alone).
+struct StepLoad {
+  int k_tile;  // K tile in part 0, or -1
+  int second;  // V tile (is_v) or K tile in part 1, or -1
+  bool is_v;
+};
+__device__ __forceinline__ StepLoad step_load(const Segment &sg, int i) {
   const int n = sg.ke - sg.kb;
-  bool ok = f(sg.kb, n > 1 ? sg.kb + 1 : -1, false);
-  for (int i = 1; i <= n && ok; ++i)
-    ok = f(sg.kb + i + 1 < sg.ke ? sg.kb + i + 1 : -1, sg.kb + i - 1, true);
+  if (i == 0) return {sg.kb, n > 1 ? sg.kb + 1 : -1, false};
+  return {sg.kb + i + 1 < sg.ke ? sg.kb + i + 1 : -1, sg.kb + i - 1, true};
+}
+// f(first step load, last step load) for every ring slot load of the segment.
+template <typename F>
+__device__ __forceinline__ bool for_each_slot_load(const Segment &sg, F &&f) {
+  const int n = sg.ke - sg.kb;
+  bool ok = true;
+  for (int i = 0; i <= n && ok; i += 2) ok = f(i, i + 1 <= n ? i + 1 : i);
   return ok;
 }
 
@@ -277,26 +291,32 @@ __device__ __forceinline__ void producer(const CUtensorMap *tm_q,
     tma_load_4d(q_s, tm_q, &bars->q_full, 0, qrow, 0, b, pol_q);
     tma_load_4d(q_s + kQHalfBytes, tm_q, &bars->q_full, 64, qrow, 0, b, pol_q);
     ++qcount;
-    ok = for_each_ring_load(sg, [&](int k_tile, int second, bool is_v) {
+    ok = for_each_slot_load(sg, [&](int i0, int i1) {
       const uint32_t slot = kv % kStages, ph = (kv / kStages) & 1u;
       if (!mbar_wait(&bars->kv_empty[slot], ph ^ 1u, abort, p.err, kSiteProdKV))
         return false;
-      const uint32_t bytes = (k_tile >= 0 ? kPartBytes : 0) +
-                             (second >= 0 ? kPartBytes : 0);
+      uint32_t bytes = 0;
+      for (int i = i0; i <= i1; ++i) {
+        const StepLoad sl = step_load(sg, i);
+        bytes += (sl.k_tile >= 0 ? kPartBytes : 0) + (sl.second >= 0 ? kPartBytes : 0);
+      }
       mbar_arrive_expect_tx(&bars->kv_full[slot], bytes);
-      uint8_t *dst = kv_s + slot * kSlotBytes;
       // A K half: keys [128 j + 64 rank, +64), all 128 columns.
       auto load_k = [&](uint8_t *to, int j) {
         const int key0 = j * kKeys + 64 * static_cast<int>(rank);
         tma_load_3d(to, tm_k, &bars->kv_full[slot], 0, key0, b, pol_kv);
         tma_load_3d(to + kKHalfBytes, tm_k, &bars->kv_full[slot], 64, key0, b, pol_kv);
       };
-      if (k_tile >= 0) load_k(dst, k_tile);
-      if (is_v)  // keys [128 j, +128), value columns [64 rank, +64)
-        tma_load_3d(dst + kPartBytes, tm_v, &bars->kv_full[slot],
-                    64 * static_cast<int>(rank), second * kKeys, b, pol_kv);
-      else if (second >= 0)
-        load_k(dst + kPartBytes, second);
+      for (int i = i0; i <= i1; ++i) {
+        const StepLoad sl = step_load(sg, i);
+        uint8_t *dst = kv_s + slot * kSlotBytes + (i & 1) * kStepBytes;
+        if (sl.k_tile >= 0) load_k(dst, sl.k_tile);
+        if (sl.is_v)  // keys [128 j, +128), value columns [64 rank, +64)
+          tma_load_3d(dst + kPartBytes, tm_v, &bars->kv_full[slot],
+                      64 * static_cast<int>(rank), sl.second * kKeys, b, pol_kv);
+        else if (sl.second >= 0)
+          load_k(dst + kPartBytes, sl.second);
+      }
       ++kv;
       return true;
     });
@@ -324,7 +344,7 @@ __device__ __forceinline__ void relay(Barriers *bars, const Params &p,
     ++qcount;
     if (!ok) break;
     mbar_arrive_cluster(q_leader);
-    ok = for_each_ring_load(sg, [&](int, int, bool) {
+    ok = for_each_slot_load(sg, [&](int, int) {
       const uint32_t slot = kv % kStages;
       if (!mbar_wait(&bars->kv_full[slot], (kv / kStages) & 1u, abort, p.err,
                      kSiteRelay))
@@ -368,31 +388,34 @@ __device__ __forceinline__ void mma_issuer(uint8_t *q_s, uint8_t *kv_s,
     ok = mbar_wait(&bars->q_full, qcount & 1u, abort, p.err, kSiteMmaQ);
     ++qcount;
     if (!ok) break;
-    // Slot load 0: S(kb) into buffer 0 and S(kb+1) into buffer 1.
+    // Step load 0: S(kb) into buffer 0 and S(kb+1) into buffer 1.
+    uint32_t slot;
+    ok = wait_kv(slot);
+    if (!ok) break;
+    tc_fence_after();
     {
-      uint32_t slot;
-      ok = wait_kv(slot);
-      if (!ok) break;
-      tc_fence_after();
       const uint32_t base = kv_addr + slot * kSlotBytes;
       for (int u = 0; u < 2 && u < n; ++u) {
         issue_qk(tmem + 128u * u, q_addr, base + u * kPartBytes);
         umma2_commit_both(&bars->s_full[u]);
         if (u == n - 1) umma2_commit_both(&bars->q_empty);
       }
-      umma2_commit_both(&bars->kv_empty[slot]);
     }
 
+    // Step load i = j - kb + 1: V(j) in part 1, K(j+2) (while it exists) in
+    // part 0; a new ring slot starts at every even i.
     for (int j = sg.kb; j < sg.ke; ++j) {
+      const int i = j - sg.kb + 1;
       const uint32_t u = static_cast<uint32_t>(j - sg.kb) & 1u;
-      uint32_t slot;  // V(j) in part 1, K(j+2) (while it exists) in part 0
-      ok = wait_kv(slot);
-      if (!ok) break;
+      if ((i & 1) == 0) {
+        ok = wait_kv(slot);
+        if (!ok) break;
+      }
       ok = mbar_wait(&bars->p_full[u], (pbits >> u) & 1u, abort, p.err, kSiteMmaP);
       pbits ^= 1u << u;
       if (!ok) break;
       tc_fence_after();
-      const uint32_t base = kv_addr + slot * kSlotBytes;
+      const uint32_t base = kv_addr + slot * kSlotBytes + (i & 1) * kStepBytes;
       issue_pv(tmem + kColO, tmem + 128u * u, base + kPartBytes, j > sg.kb);
       if (j + 1 == sg.ke)
         umma2_commit_both(&bars->o_full);
@@ -405,8 +428,10 @@ __device__ __forceinline__ void mma_issuer(uint8_t *q_s, uint8_t *kv_s,
         umma2_commit_both(&bars->s_full[u]);
         if (j + 3 == sg.ke) umma2_commit_both(&bars->q_empty);
       }
-      umma2_commit_both(&bars->kv_empty[slot]);
+      if ((i & 1) == 1 || j + 1 == sg.ke) umma2_commit_both(&bars->kv_empty[slot]);
     }
+    // A segment of one key tile: its only slot holds step loads 0 and 1 and
+    // was released above; otherwise the last slot was released in the loop.
   }
   // All MMAs this thread issued complete before tensor memory is released.
   umma2_commit_self(&bars->drain);
