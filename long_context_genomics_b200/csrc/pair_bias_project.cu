@@ -12,7 +12,8 @@
 // 4-stage shared-memory ring with untiled bulk copies issued by one producer
 // lane, so 128 KB per SM are in flight.  Eight consumer warps take 8 cells
 // each per chunk.  Lane l reads channels 4l..4l+3 of a cell (one conflict-free
-// 16-byte shared load per cell) and keeps W[4l..4l+3, 0..7] in registers; the
+// 16-byte shared load per cell) and keeps W[4l..4l+3, 0..7] in registers
+// (products for two heads per packed fp32x2 instruction); the
 // 64 partial sums (8 heads x 8 cells) are reduced across the warp by a
 // butterfly reduce-scatter (offsets 16, 8, 4, 2, 1), after which lane l holds
 // the two finished values of head l/4 for cells 2(l%4) and 2(l%4)+1: a float2
@@ -36,14 +37,21 @@ constexpr size_t kSmemBytes = 1024 + kStages * kChunkBytes + 2 * kStages * 8 + 1
 enum Site : unsigned { kSiteFull = 20, kSiteEmpty = 21 };
 
 // One reduce-scatter level: lanes with bit `o` set keep the upper half of
-// the first 2*n values, the others the lower half; each adds its partner's.
+// the first 2*n values, the others the lower half; each adds its partner's
+// (two values per packed add).
 template <int n>
 __device__ __forceinline__ void rs_level(float (&a)[64], int o, bool upper) {
 #pragma unroll
-  for (int j = 0; j < n; ++j) {
-    const float keep = upper ? a[j + n] : a[j];
-    const float send = upper ? a[j] : a[j + n];
-    a[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+  for (int j = 0; j < n; j += 2) {
+    const float2 keep = upper ? make_float2(a[j + n], a[j + n + 1])
+                              : make_float2(a[j], a[j + 1]);
+    const float2 send = upper ? make_float2(a[j], a[j + 1])
+                              : make_float2(a[j + n], a[j + n + 1]);
+    const float2 recv = make_float2(__shfl_xor_sync(0xffffffffu, send.x, o),
+                                    __shfl_xor_sync(0xffffffffu, send.y, o));
+    const float2 sum = __fadd2_rn(keep, recv);
+    a[j] = sum.x;
+    a[j + 1] = sum.y;
   }
 }
 
@@ -94,11 +102,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    float w[4][kH];
+    // W[4l + i, h] for heads in pairs (2p, 2p + 1).
+    float2 w[4][kH / 2];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int h = 0; h < kH; ++h) w[i][h] = __ldg(W + (4 * lane + i) * kH + h);
+      for (int hp = 0; hp < kH / 2; ++hp)
+        w[i][hp] = make_float2(__ldg(W + (4 * lane + i) * kH + 2 * hp),
+                               __ldg(W + (4 * lane + i) * kH + 2 * hp + 1));
     const int h_out = lane >> 2;       // head this lane finishes
     const int n_out = 2 * (lane & 3);  // first of its two cells
     uint32_t it = 0;
@@ -117,14 +128,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[slot]);  // this warp is done with the slot
       if (c0 >= n_cells) continue;
-      float a[64];  // a[h * 8 + n]
+      float a[64];  // a[h * 8 + n]: the same products and order as
+                    // fmaf(x.w, w3, fmaf(x.z, w2, fmaf(x.y, w1, x.x * w0))),
+                    // two heads per packed instruction
 #pragma unroll
-      for (int h = 0; h < kH; ++h)
+      for (int hp = 0; hp < kH / 2; ++hp)
 #pragma unroll
-        for (int n = 0; n < 8; ++n)
-          a[h * 8 + n] = fmaf(
-              x[n].w, w[3][h],
-              fmaf(x[n].z, w[2][h], fmaf(x[n].y, w[1][h], x[n].x * w[0][h])));
+        for (int n = 0; n < 8; ++n) {
+          float2 v = __fmul2_rn(make_float2(x[n].x, x[n].x), w[0][hp]);
+          v = __ffma2_rn(make_float2(x[n].y, x[n].y), w[1][hp], v);
+          v = __ffma2_rn(make_float2(x[n].z, x[n].z), w[2][hp], v);
+          v = __ffma2_rn(make_float2(x[n].w, x[n].w), w[3][hp], v);
+          a[(2 * hp) * 8 + n] = v.x;
+          a[(2 * hp + 1) * 8 + n] = v.y;
+        }
       rs_level<32>(a, 16, lane & 16);
       rs_level<16>(a, 8, lane & 8);
       rs_level<8>(a, 4, lane & 4);
