@@ -339,7 +339,9 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         "peak_source": pk["source"],
         "e2e": {"value": aggregate_rate(world, flops, K, e2e_s) / 1e12, "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 2 * K,
+        # Our kernels in the timed region: the projection, and the attention
+        # with its split-pair merge when the grid splits pairs.
+        "gpu_launches": K * (1 + ag.ag_attn_fwd_launch_count(w.B, w.L, w.cap)),
         "roofline": {"kernel": "attn_fwd_kernel", "bound": "tensor", "achieved": achieved,
                      "peak": pk["bf16_tflops"], "unit": UNIT,
                      "frac": achieved / pk["bf16_tflops"], "traffic": profiled_traffic(),

@@ -147,6 +147,18 @@ ag_status ag_attn_fwd_noalloc(const void *q, const void *k, const void *v,
                               float *lse, void *stream);
 
 /*
+ * ag_attn_fwd_launch_count -- how many kernels ag_attn_fwd (or
+ * ag_attn_fwd_noalloc) launches for these sizes on the current device: 0 for
+ * an empty call, 1, or 2 when some pair of query tiles has its keys split
+ * between SM pairs and the merge kernel runs as well (a library convenience
+ * for callers that count launches; the pages have no counterpart).
+ * Same size and value checks, and statuses, as ag_attn_fwd; count is a host
+ * pointer (AG_ERR_NULL if NULL).  Launches nothing.
+ */
+ag_status ag_attn_fwd_launch_count(int64_t B, int64_t H, int64_t L, int64_t D,
+                                   int64_t block, float cap, int *count);
+
+/*
  * Device error word.  Every wait inside the kernels is bounded (about one
  * second); a wait that runs out makes the kernel stop, release what it
  * holds and record a code here instead of hanging the GPU.

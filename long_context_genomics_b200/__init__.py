@@ -59,6 +59,9 @@ def _load() -> ctypes.CDLL:
     lib.ag_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64,
                                         f32, vp, vp, vp]
     lib.ag_attn_fwd_noalloc.restype = ctypes.c_int
+    lib.ag_attn_fwd_launch_count.argtypes = [i64, i64, i64, i64, i64, f32,
+                                             ctypes.POINTER(ctypes.c_int)]
+    lib.ag_attn_fwd_launch_count.restype = ctypes.c_int
     lib.ag_device_error.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int),
                                     ctypes.c_int]
     lib.ag_device_error.restype = ctypes.c_int
@@ -166,6 +169,17 @@ def ag_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     if st != AG_OK:
         raise AgError("ag_attn_fwd_noalloc", st)
     return out, lse
+
+
+def ag_attn_fwd_launch_count(B: int, L: int, cap: float = 5.0, H: int = 8,
+                             D: int = 128, block: int = 16) -> int:
+    """How many kernels ag_attn_fwd launches for these sizes (see include/ag.h)."""
+    n = ctypes.c_int(-1)
+    st = lib.ag_attn_fwd_launch_count(int(B), int(H), int(L), int(D), int(block),
+                                      float(cap), ctypes.byref(n))
+    if st != AG_OK:
+        raise AgError("ag_attn_fwd_launch_count", st)
+    return int(n.value)
 
 
 def ag_device_error(device: int = 0, clear: bool = True) -> int:

@@ -200,18 +200,29 @@ ag_status ag_pair_bias_project(const float *pair, const float *W, float *bias,
       pair, W, bias, P, dev->num_sms, dev->err, static_cast<cudaStream_t>(stream)));
 }
 
-ag_status ag_attn_fwd(const void *q, const void *k, const void *v,
-                      const float *bias, int64_t B, int64_t H, int64_t L,
-                      int64_t D, int64_t block, float cap, float *out,
-                      float *lse, void *stream) {
+namespace ag {
+// Size and value checks shared by the attention entry points, in order:
+// shapes, then cap, then what the kernels support (including the work-step
+// bound: pairs of query tiles x key tiles must stay below 2^30).
+static ag_status check_attn_sizes(int64_t B, int64_t H, int64_t L, int64_t D,
+                                  int64_t block, float cap) {
   if (B < 0 || H <= 0 || L < 0 || D <= 0 || block <= 0) return AG_ERR_SHAPE;
   if (L % block != 0) return AG_ERR_SHAPE;
   if (std::isnan(cap) || !(cap > 0.0f)) return AG_ERR_VALUE;
   if (H != 8 || D != 128 || block != 16 || L > 65536) return AG_ERR_UNSUPPORTED;
   if (B > 0 && L > 0 && B * L > (int64_t(1) << 28)) return AG_ERR_UNSUPPORTED;
-  // Work steps (pairs of query tiles x key tiles) must stay below 2^30.
-  if (B > 0 && L > 0 && ag::attn_work_steps(B, L) > (int64_t(1) << 30))
+  if (B > 0 && L > 0 && attn_work_steps(B, L) > (int64_t(1) << 30))
     return AG_ERR_UNSUPPORTED;
+  return AG_OK;
+}
+}  // namespace ag
+
+ag_status ag_attn_fwd(const void *q, const void *k, const void *v,
+                      const float *bias, int64_t B, int64_t H, int64_t L,
+                      int64_t D, int64_t block, float cap, float *out,
+                      float *lse, void *stream) {
+  const ag_status vs = ag::check_attn_sizes(B, H, L, D, block, cap);
+  if (vs != AG_OK) return vs;
   if (B == 0 || L == 0) return AG_OK;
   if (!q || !k || !v || !bias || !out || !lse) return AG_ERR_NULL;
   if (!ag::aligned(q, 16) || !ag::aligned(k, 16) || !ag::aligned(v, 16) ||
@@ -262,13 +273,8 @@ ag_status ag_attn_fwd_noalloc(const void *q, const void *k, const void *v,
                               int64_t D, int64_t block, float cap, float *out,
                               float *lse, void *stream) {
   // The same checks, in the same order, as ag_attn_fwd.
-  if (B < 0 || H <= 0 || L < 0 || D <= 0 || block <= 0) return AG_ERR_SHAPE;
-  if (L % block != 0) return AG_ERR_SHAPE;
-  if (std::isnan(cap) || !(cap > 0.0f)) return AG_ERR_VALUE;
-  if (H != 8 || D != 128 || block != 16 || L > 65536) return AG_ERR_UNSUPPORTED;
-  if (B > 0 && L > 0 && B * L > (int64_t(1) << 28)) return AG_ERR_UNSUPPORTED;
-  if (B > 0 && L > 0 && ag::attn_work_steps(B, L) > (int64_t(1) << 30))
-    return AG_ERR_UNSUPPORTED;
+  const ag_status vs = ag::check_attn_sizes(B, H, L, D, block, cap);
+  if (vs != AG_OK) return vs;
   if (B == 0 || L == 0) return AG_OK;
   if (!q || !k || !v || !bias || !out || !lse) return AG_ERR_NULL;
   if (!ag::aligned(q, 16) || !ag::aligned(k, 16) || !ag::aligned(v, 16) ||
@@ -319,6 +325,25 @@ ag_status ag_attn_fwd_noalloc(const void *q, const void *k, const void *v,
   a.encode = enc;
   a.stream = static_cast<cudaStream_t>(stream);
   return ag::from_cuda(ag::launch_attn_fwd(a));
+}
+
+ag_status ag_attn_fwd_launch_count(int64_t B, int64_t H, int64_t L, int64_t D,
+                                   int64_t block, float cap, int *count) {
+  if (!count) return AG_ERR_NULL;
+  const ag_status vs = ag::check_attn_sizes(B, H, L, D, block, cap);
+  if (vs != AG_OK) return vs;
+  if (B == 0 || L == 0) {
+    *count = 0;
+    return AG_OK;
+  }
+  ag::DeviceInfo *dev = nullptr;
+  ag_status st = ag::device_info(&dev);
+  if (st != AG_OK) return st;
+  int n = 0;
+  st = ag::from_cuda(ag::attn_fwd_kernel_count(B, L, cap, dev->num_sms, dev->num_sms, &n));
+  if (st != AG_OK) return st;
+  *count = n;
+  return AG_OK;
 }
 
 ag_status ag_device_error(int device, int *code, int clear) {

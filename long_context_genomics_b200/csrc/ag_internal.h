@@ -49,6 +49,11 @@ struct AttnLaunch {
 // encoding is reported as cudaErrorInvalidValue.
 cudaError_t launch_attn_fwd(const AttnLaunch &a);
 
+// How many kernels launch_attn_fwd launches for these sizes on the current
+// device (0 for an empty call, 1, or 2 when split pairs need the merge).
+cudaError_t attn_fwd_kernel_count(int64_t B, int64_t L, float cap, int num_sms,
+                                  int scratch_slots, int *count);
+
 cudaError_t launch_pair_bias_project(const float *pair, const float *W,
                                      float *bias, int64_t P, int num_sms,
                                      unsigned *err, cudaStream_t stream);

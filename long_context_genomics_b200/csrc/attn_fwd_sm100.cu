@@ -1001,6 +1001,63 @@ static cudaError_t launch_mode(const CUtensorMap &tq, const CUtensorMap &tk,
   return cudaGetLastError();
 }
 
+// Grid of a call: one 2-CTA cluster per resident SM pair, never more
+// clusters than (pair, key tile) steps or scratch slots.  Whole pairs per
+// cluster unless that leaves the grid badly balanced: a split pair costs a
+// second pass over its rows (partial results, then the merge), so whole pairs
+// win while the busiest cluster's extra work stays below kSplitGain pairs.
+static cudaError_t plan_grid(int mode, int n_items, int n_kt, int num_sms,
+                             int scratch_slots, int *clusters_out, int *whole_out) {
+  using namespace attn;
+  int max_clusters = 0;
+  cudaError_t e;
+  switch (mode) {
+    case kStaticCap: e = configure_mode<kStaticCap>(&max_clusters); break;
+    case kOnlineCap: e = configure_mode<kOnlineCap>(&max_clusters); break;
+    default: e = configure_mode<kNoCap>(&max_clusters); break;
+  }
+  if (e != cudaSuccess) return e;
+  const long long steps = static_cast<long long>(n_items) * n_kt;
+  if (steps > (1ll << 30)) return cudaErrorInvalidValue;
+  int clusters = num_sms / 2;
+  if (max_clusters < clusters) clusters = max_clusters;
+  if (scratch_slots < clusters) clusters = scratch_slots;
+  if (steps < clusters) clusters = static_cast<int>(steps);
+  if (clusters < 1) return cudaErrorInvalidValue;
+  constexpr double kSplitGain = 0.5;
+  const long long per = (n_items + clusters - 1) / clusters;  // busiest cluster
+  const double even = static_cast<double>(n_items) / clusters;
+  const int whole = (per - even <= kSplitGain) ? 1 : 0;
+  if (whole && n_items < clusters) clusters = n_items;
+  *clusters_out = clusters;
+  *whole_out = whole;
+  return cudaSuccess;
+}
+
+static int attn_mode(float cap) {
+  using namespace attn;
+  if (isinf(cap)) return kNoCap;
+  return cap <= 40.0f ? kStaticCap : kOnlineCap;
+}
+
+cudaError_t attn_fwd_kernel_count(int64_t B, int64_t L, float cap, int num_sms,
+                                  int scratch_slots, int *count) {
+  using namespace attn;
+  if (B == 0 || L == 0) {
+    *count = 0;
+    return cudaSuccess;
+  }
+  const int nb = static_cast<int>(L / 16);
+  const int n_items = static_cast<int>(B) * ((nb + 1) / 2);
+  const int n_kt = static_cast<int>((L + kKeys - 1) / kKeys);
+  int clusters = 0, whole = 0;
+  cudaError_t e = plan_grid(attn_mode(cap), n_items, n_kt, num_sms, scratch_slots,
+                            &clusters, &whole);
+  if (e != cudaSuccess) return e;
+  *count = (clusters < 2 || whole) ? 1 : 2;
+  return cudaSuccess;
+}
+
 cudaError_t launch_attn_fwd(const AttnLaunch &a) {
   using namespace attn;
   const int64_t B = a.B, L = a.L;
@@ -1039,46 +1096,22 @@ cudaError_t launch_attn_fwd(const AttnLaunch &a) {
   p.last_valid = static_cast<int>(L - static_cast<int64_t>(p.n_kt - 1) * kKeys);
   const float cap = a.cap;
   const float inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(kD));
-  int mode;
-  if (isinf(cap)) {
-    mode = kNoCap;
+  const int mode = attn_mode(cap);
+  if (mode == kNoCap) {
     p.qk_scale = inv_sqrt_d * kLog2e;
     p.bias_mul = kLog2e;
     p.A = 0.f;
   } else {
-    mode = cap <= 40.0f ? kStaticCap : kOnlineCap;
     p.qk_scale = inv_sqrt_d / cap;
     p.bias_mul = 1.0f / cap;
     p.A = cap * kLog2e;
   }
-  int max_clusters = 0;
-  cudaError_t e;
-  switch (mode) {
-    case kStaticCap: e = configure_mode<kStaticCap>(&max_clusters); break;
-    case kOnlineCap: e = configure_mode<kOnlineCap>(&max_clusters); break;
-    default: e = configure_mode<kNoCap>(&max_clusters); break;
-  }
+  int clusters = 0;
+  cudaError_t e = plan_grid(mode, p.n_items, p.n_kt, a.num_sms, a.scratch_slots,
+                            &clusters, &p.whole);
   if (e != cudaSuccess) return e;
-  // One cluster per resident SM pair, never more clusters than (pair, key
-  // tile) steps or scratch slots.  Whole pairs per cluster unless that
-  // leaves the grid badly balanced: a split pair costs a second pass over
-  // its rows (partial results, then the merge), so whole pairs win while the
-  // busiest cluster's extra work stays below kSplitGain pairs.
-  const long long steps = static_cast<long long>(p.n_items) * p.n_kt;
-  if (steps != attn_work_steps(B, L) || steps > (1ll << 30))
+  if (static_cast<long long>(p.n_items) * p.n_kt != attn_work_steps(B, L))
     return cudaErrorInvalidValue;
-  int clusters = a.num_sms / 2;
-  if (max_clusters < clusters) clusters = max_clusters;
-  if (a.scratch_slots < clusters) clusters = a.scratch_slots;
-  if (steps < clusters) clusters = static_cast<int>(steps);
-  if (clusters < 1) return cudaErrorInvalidValue;
-  {
-    constexpr double kSplitGain = 0.5;
-    const long long per = (p.n_items + clusters - 1) / clusters;  // busiest cluster
-    const double even = static_cast<double>(p.n_items) / clusters;
-    p.whole = (per - even <= kSplitGain) ? 1 : 0;
-    if (p.whole && p.n_items < clusters) clusters = p.n_items;
-  }
   char *base = static_cast<char *>(a.scratch);
   p.ws_out = reinterpret_cast<float *>(base);
   p.ws_lse = reinterpret_cast<float *>(base + a.scratch_slots * kAttnSlotOutBytes);

@@ -70,6 +70,17 @@ def test_attn_validation(ag, kw, status):
     assert _attn(ag, **kw) == status
 
 
+def test_launch_count_checks_before_the_device(ag):
+    import ctypes
+    n = ctypes.c_int(-1)
+    f = ag.lib.ag_attn_fwd_launch_count
+    assert f(1, 8, 256, 128, 16, 5.0, None) == 1                    # AG_ERR_NULL
+    assert f(1, 8, 250, 128, 16, 5.0, ctypes.byref(n)) == 2         # AG_ERR_SHAPE
+    assert f(1, 8, 256, 64, 16, 5.0, ctypes.byref(n)) == 4          # AG_ERR_UNSUPPORTED
+    assert f(1, 8, 256, 128, 16, -1.0, ctypes.byref(n)) == 5        # AG_ERR_VALUE
+    assert f(0, 8, 256, 128, 16, 5.0, ctypes.byref(n)) == 0 and n.value == 0
+
+
 def test_attn_empty_is_a_noop(ag):
     assert _attn(ag, B=0, q=None, k=None, v=None, bias=None, out=None, lse=None) == 0
     assert _attn(ag, L=0, q=None, k=None, v=None, bias=None, out=None, lse=None) == 0

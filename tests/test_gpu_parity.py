@@ -216,3 +216,14 @@ def test_bounded_wait_reports_and_context_survives(ag, oracle_lib):
     ro, rl = oracle_lib.attn_fwd(inp["q"], inp["k"], inp["v"], inp["bias"],
                                  block=16, cap=5.0)
     _compare(out, lse, ro, rl, "after timeout")
+
+
+def test_launch_count_matches_the_grid_policy(ag):
+    """ag_attn_fwd_launch_count reports 1 or 2 kernels for real sizes and 0 for
+    empty ones; at full context on a 148-SM B200 the 256 tile pairs do not
+    divide evenly over the 74 SM pairs, so pairs are split and merged (2)."""
+    assert ag.ag_attn_fwd_launch_count(0, 8192) == 0
+    for B, L in [(1, 512), (1, 2048), (2, 8192)]:
+        assert ag.ag_attn_fwd_launch_count(B, L) in (1, 2)
+    if torch.cuda.get_device_properties(0).multi_processor_count == 148:
+        assert ag.ag_attn_fwd_launch_count(1, 8192) == 2
