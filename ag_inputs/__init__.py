@@ -124,15 +124,18 @@ def make_inputs(w: Workload) -> dict:
 
 def random_case(B: int, H: int, L: int, D: int, Dv: int, block: int,
                 seed: int, bias_std: float = 1.0, qk_std: float = 1.0,
-                dtype=torch.bfloat16) -> dict:
+                dtype=torch.bfloat16, batched_bias: bool = False) -> dict:
     """Small seeded case with free sizes (tests).  Same draw order as
-    make_inputs: q, k, v, then bias."""
+    make_inputs: q, k, v, then bias.  L need not be a multiple of the block
+    (P = ceil(L / block) compact cells per side); batched_bias draws one bias
+    per batch item, [B, H, P, P], instead of one shared [H, P, P]."""
     g = torch.Generator(device="cpu").manual_seed(int(seed))
-    P = L // block
+    P = -(-L // block)
     q = (torch.randn(B, H, L, D, generator=g) * qk_std).to(dtype)
     k = (torch.randn(B, L, D, generator=g) * qk_std).to(dtype)
     v = torch.randn(B, L, Dv, generator=g).to(dtype)
-    bias = torch.randn(H, P, P, generator=g) * bias_std
+    shape = (B, H, P, P) if batched_bias else (H, P, P)
+    bias = torch.randn(*shape, generator=g) * bias_std
     return {"q": q, "k": k, "v": v, "bias": bias}
 
 

@@ -51,17 +51,17 @@ class Oracle:
         L = ctypes.c_long
         lib.agref_pair_bias_project.argtypes = [
             _c_double_p, _c_double_p, _c_double_p, L, L, L, ctypes.c_int]
-        lib.agref_attn_fwd.argtypes = [
-            _c_double_p, _c_double_p, _c_double_p, _c_double_p,
+        lib.agref_attn_fwd_ex.argtypes = [
+            _c_double_p, _c_double_p, _c_double_p, _c_double_p, L,
             L, L, L, L, L, L, ctypes.c_double,
             _c_double_p, _c_double_p, _c_double_p, ctypes.c_int]
-        lib.agref_attn_rows.argtypes = [
-            _c_double_p, _c_double_p, _c_double_p, _c_double_p,
+        lib.agref_attn_rows_ex.argtypes = [
+            _c_double_p, _c_double_p, _c_double_p, _c_double_p, L,
             L, L, L, L, L, L, ctypes.c_double,
             _c_int64_p, L, _c_double_p, _c_double_p, ctypes.c_int]
         lib.agref_max_threads.argtypes = [ctypes.c_int]
-        for f in ("agref_pair_bias_project", "agref_attn_fwd",
-                  "agref_attn_rows", "agref_max_threads", "agref_mutant_id"):
+        for f in ("agref_pair_bias_project", "agref_attn_fwd_ex",
+                  "agref_attn_rows_ex", "agref_max_threads", "agref_mutant_id"):
             getattr(lib, f).restype = ctypes.c_int
         self._lib = lib
         self.mutant = lib.agref_mutant_id()
@@ -86,19 +86,33 @@ class Oracle:
         return bias
 
     # -- attention ------------------------------------------------------------
+    @staticmethod
+    def _bias_stride(bias, B, H, L, block) -> int:
+        """bias is [H,P,P] (shared by the batch) or [B,H,P,P] (one per item),
+        P = ceil(L / block); returns the batch stride in doubles."""
+        P = -(-L // block) if block > 0 else 0
+        if bias.ndim == 3 and bias.shape == (H, P, P):
+            return 0
+        if bias.ndim == 4 and bias.shape == (B, H, P, P):
+            return H * P * P
+        raise ValueError(f"bias shape {bias.shape} is neither ({H},{P},{P}) "
+                         f"nor ({B},{H},{P},{P})")
+
     def attn_fwd(self, q, k, v, bias, block: int = 16, cap: float = 5.0,
                  probs: bool = False, nthreads: int = 0):
         """Full attention: returns (out [B,H,L,Dv], lse [B,H,L]) and, if
-        probs=True, also the softmax weights [B,H,L,L] (tiny inputs only)."""
+        probs=True, also the softmax weights [B,H,L,L] (tiny inputs only).
+        bias: [H,P,P] shared, or [B,H,P,P] per batch item; P = ceil(L/block)."""
         q, k, v, bias = _f64(q), _f64(k), _f64(v), _f64(bias)
         B, H, L, D = q.shape
         Dv = v.shape[-1]
         assert k.shape == (B, L, D) and v.shape == (B, L, Dv)
+        bstride = self._bias_stride(bias, B, H, L, int(block))
         out = np.empty((B, H, L, Dv), dtype=np.float64)
         lse = np.empty((B, H, L), dtype=np.float64)
         pr = np.empty((B, H, L, L), dtype=np.float64) if probs else None
-        rc = self._lib.agref_attn_fwd(
-            _ptr(q), _ptr(k), _ptr(v), _ptr(bias), B, H, L, D, Dv, int(block),
+        rc = self._lib.agref_attn_fwd_ex(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(bias), bstride, B, H, L, D, Dv, int(block),
             float(cap), _ptr(out), _ptr(lse),
             _ptr(pr) if probs else None, int(nthreads))
         if rc != 0:
@@ -112,12 +126,13 @@ class Oracle:
         q, k, v, bias = _f64(q), _f64(k), _f64(v), _f64(bias)
         B, H, L, D = q.shape
         Dv = v.shape[-1]
+        bstride = self._bias_stride(bias, B, H, L, int(block))
         rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
         n = rows.shape[0]
         out = np.empty((n, Dv), dtype=np.float64)
         lse = np.empty((n,), dtype=np.float64)
-        rc = self._lib.agref_attn_rows(
-            _ptr(q), _ptr(k), _ptr(v), _ptr(bias), B, H, L, D, Dv, int(block),
+        rc = self._lib.agref_attn_rows_ex(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(bias), bstride, B, H, L, D, Dv, int(block),
             float(cap), rows.ctypes.data_as(_c_int64_p), n, _ptr(out),
             _ptr(lse), int(nthreads))
         if rc != 0:

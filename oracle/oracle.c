@@ -20,6 +20,13 @@
  * The compact bias holds one cell per block x block square of (query, key)
  * positions and the dense model repeats each cell over its square; the
  * oracle builds that repeated row literally, one query row at a time.
+ * Lengths that are not a multiple of the block end in a partial block whose
+ * compact cell applies as it does to the others (P = ceil(L/block)); the page
+ * lists tails among what is not yet supported (section "What has not yet
+ * been demonstrated") and tail handling as next work (section "Where I would
+ * take it next"), and floor(i/block) is the plain reading for them.  The bias
+ * may also be one per batch item, [B,H,P,P], since each sequence has its own
+ * pair representation (section "Profiling pointed at one very large object").
  * No mask: every key is attended (section "What this does -- and does not --
  * mean" lists masks among the unsupported features).  The softmax is written as the plain
  * two-pass definition (max, then sum), not the tiled online recurrence of
@@ -109,6 +116,7 @@ typedef struct {
     const double *q, *k, *v, *bias;
     long B, H, L, D, Dv, block, P;
     double cap;
+    long bias_bstride; /* doubles between batch items' bias; 0 = one shared bias */
 } attn_args;
 
 /* The soft cap of Eq. L_ij; cap = +inf means no cap. */
@@ -144,7 +152,14 @@ static void attn_row(const attn_args *a, long b, long h, long i, double *logit,
 #endif
 
     /* The compact bias row for query block floor(i/block), repeated over each
-       key block: brow[j] = bias[h, floor(i/block), floor(j/block)]. */
+       key block: brow[j] = bias[b, h, floor(i/block), floor(j/block)].  A
+       length that is not a multiple of the block ends in a partial block,
+       which uses its compact cell like any other (P = ceil(L / block)). */
+#if AGREF_MUTANT == 13
+    const double *bias_b = a->bias; /* every item reads item 0's bias */
+#else
+    const double *bias_b = a->bias + b * a->bias_bstride;
+#endif
 #if AGREF_MUTANT == 5
     const long I = (i / blk + 1) % P; /* query block off by one */
 #else
@@ -153,9 +168,9 @@ static void attn_row(const attn_args *a, long b, long h, long i, double *logit,
     for (long j = 0; j < L; ++j) {
         const long J = j / blk;
 #if AGREF_MUTANT == 1
-        brow[j] = a->bias[(h * P + J) * P + I]; /* bias transposed */
+        brow[j] = bias_b[(h * P + J) * P + I]; /* bias transposed */
 #else
-        brow[j] = a->bias[(h * P + I) * P + J];
+        brow[j] = bias_b[(h * P + I) * P + J];
 #endif
     }
 
@@ -206,7 +221,6 @@ static int check_args(const attn_args *a) {
     if (a->B < 0 || a->H <= 0 || a->L < 0 || a->D <= 0 || a->Dv <= 0 ||
         a->block <= 0)
         return AGREF_EINVAL;
-    if (a->L % a->block != 0) return AGREF_EINVAL;
     if (isnan(a->cap) || a->cap <= 0.0) return AGREF_EINVAL;
     if (a->B == 0 || a->L == 0) return AGREF_OK;
     if (!a->q || !a->k || !a->v || !a->bias) return AGREF_EINVAL;
@@ -214,20 +228,31 @@ static int check_args(const attn_args *a) {
 }
 
 /*
- * Full attention.  q [B,H,L,D], k [B,L,D], v [B,L,Dv], bias [H,P,P] with
- * P = L/block, all row-major float64.  Writes out [B,H,L,Dv] and lse [B,H,L].
- * If probs is not NULL it must hold B*H*L*L doubles and receives the softmax
- * weights (tiny inputs only).
+ * Full attention.  q [B,H,L,D], k [B,L,D], v [B,L,Dv], bias [H,P,P] (or, with
+ * bias_bstride = H*P*P, [B,H,P,P]: one bias per batch item, as each sequence
+ * has its own pair representation) with P = ceil(L/block), all row-major
+ * float64.  Any L >= 0: a last partial block uses its compact cell.  Writes
+ * out [B,H,L,Dv] and lse [B,H,L].  If probs is not NULL it must hold B*H*L*L
+ * doubles and receives the softmax weights (tiny inputs only).
  */
-int agref_attn_fwd(const double *q, const double *k, const double *v,
-                   const double *bias, long B, long H, long L, long D, long Dv,
-                   long block, double cap, double *out, double *lse,
-                   double *probs, int nthreads) {
-    attn_args a = {q, k, v, bias, B, H, L, D, Dv, block, 0, cap};
+/* Compact cells per side for a length: ceil(L / block). */
+static long cells(long L, long block) {
+#if AGREF_MUTANT == 14
+    return L / block; /* partial last block dropped */
+#else
+    return (L + block - 1) / block;
+#endif
+}
+
+int agref_attn_fwd_ex(const double *q, const double *k, const double *v,
+                      const double *bias, long bias_bstride, long B, long H,
+                      long L, long D, long Dv, long block, double cap,
+                      double *out, double *lse, double *probs, int nthreads) {
+    attn_args a = {q, k, v, bias, B, H, L, D, Dv, block, 0, cap, bias_bstride};
     int rc = check_args(&a);
     if (rc != AGREF_OK || B == 0 || L == 0) return rc;
-    if (!out || !lse) return AGREF_EINVAL;
-    a.P = L / block;
+    if (!out || !lse || bias_bstride < 0) return AGREF_EINVAL;
+    a.P = cells(L, block);
     set_threads(nthreads);
     const long rows = B * H * L;
     int failed = 0;
@@ -259,11 +284,12 @@ int agref_attn_fwd(const double *q, const double *k, const double *v,
  * Selected rows only: rows holds n triples (b, h, i).  out_rows [n, Dv],
  * lse_rows [n].  Used to check full-size outputs on a sample of rows.
  */
-int agref_attn_rows(const double *q, const double *k, const double *v,
-                    const double *bias, long B, long H, long L, long D, long Dv,
-                    long block, double cap, const int64_t *rows, long n,
-                    double *out_rows, double *lse_rows, int nthreads) {
-    attn_args a = {q, k, v, bias, B, H, L, D, Dv, block, 0, cap};
+int agref_attn_rows_ex(const double *q, const double *k, const double *v,
+                       const double *bias, long bias_bstride, long B, long H,
+                       long L, long D, long Dv, long block, double cap,
+                       const int64_t *rows, long n, double *out_rows,
+                       double *lse_rows, int nthreads) {
+    attn_args a = {q, k, v, bias, B, H, L, D, Dv, block, 0, cap, bias_bstride};
     int rc = check_args(&a);
     if (rc != AGREF_OK) return rc;
     if (n == 0) return AGREF_OK;
@@ -272,7 +298,8 @@ int agref_attn_rows(const double *q, const double *k, const double *v,
         const int64_t b = rows[3 * t], h = rows[3 * t + 1], i = rows[3 * t + 2];
         if (b < 0 || b >= B || h < 0 || h >= H || i < 0 || i >= L) return AGREF_EINVAL;
     }
-    a.P = L / block;
+    if (bias_bstride < 0) return AGREF_EINVAL;
+    a.P = cells(L, block);
     set_threads(nthreads);
     int failed = 0;
 #pragma omp parallel
@@ -294,4 +321,21 @@ int agref_attn_rows(const double *q, const double *k, const double *v,
         free(brow);
     }
     return failed ? AGREF_ENOMEM : AGREF_OK;
+}
+
+/* The entry points with one bias shared by every batch item. */
+int agref_attn_fwd(const double *q, const double *k, const double *v,
+                   const double *bias, long B, long H, long L, long D, long Dv,
+                   long block, double cap, double *out, double *lse,
+                   double *probs, int nthreads) {
+    return agref_attn_fwd_ex(q, k, v, bias, 0, B, H, L, D, Dv, block, cap, out,
+                             lse, probs, nthreads);
+}
+
+int agref_attn_rows(const double *q, const double *k, const double *v,
+                    const double *bias, long B, long H, long L, long D, long Dv,
+                    long block, double cap, const int64_t *rows, long n,
+                    double *out_rows, double *lse_rows, int nthreads) {
+    return agref_attn_rows_ex(q, k, v, bias, 0, B, H, L, D, Dv, block, cap, rows,
+                              n, out_rows, lse_rows, nthreads);
 }

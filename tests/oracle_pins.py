@@ -33,17 +33,23 @@ import ag_inputs
 CAPS = (5.0, 30.0, math.inf)
 
 
-def _case(B=2, H=3, L=64, D=8, Dv=6, block=16, seed=0, bias_std=1.0, qk_std=1.0):
+def _case(B=2, H=3, L=64, D=8, Dv=6, block=16, seed=0, bias_std=1.0, qk_std=1.0,
+          batched_bias=False):
     c = ag_inputs.random_case(B, H, L, D, Dv, block, seed, bias_std=bias_std,
-                              qk_std=qk_std, dtype=torch.float64)
+                              qk_std=qk_std, dtype=torch.float64,
+                              batched_bias=batched_bias)
     return {n: t.to(torch.float64).numpy() for n, t in c.items()}
 
 
 def dense_bruteforce(q, k, v, bias, block, cap):
-    """Dense evaluation with the literal block repeat of the compact bias."""
+    """Dense evaluation with the literal block repeat of the compact bias,
+    cropped to L when L is not a multiple of the block.  bias is [H,P,P], or
+    [B,H,P,P] with one bias per batch item."""
     D = q.shape[-1]
-    bexp = np.repeat(np.repeat(bias, block, axis=1), block, axis=2)  # [H,L,L]
-    s = np.einsum("bhid,bjd->bhij", q, k) / np.sqrt(D) + bexp[None]
+    L = q.shape[2]
+    b4 = bias if bias.ndim == 4 else bias[None]
+    bexp = np.repeat(np.repeat(b4, block, axis=2), block, axis=3)[:, :, :L, :L]
+    s = np.einsum("bhid,bjd->bhij", q, k) / np.sqrt(D) + bexp
     logits = s if math.isinf(cap) else cap * np.tanh(s / cap)
     lse = logsumexp(logits, axis=-1)
     p = np.exp(logits - lse[..., None])
@@ -71,6 +77,31 @@ def pin_bruteforce(o):
             _close(out, ro, 1e-12, f"out block={block} cap={cap}")
             _close(lse, rl, 1e-12, f"lse block={block} cap={cap}")
             _close(p, rp, 1e-12, f"probs block={block} cap={cap}")
+
+
+def pin_bruteforce_tails_and_batched_bias(o):
+    """Oracle == dense brute force for lengths that end in a partial block
+    and for one bias per batch item."""
+    for L, block in ((40, 16), (23, 4), (17, 16)):
+        for cap in CAPS:
+            for batched in (False, True):
+                c = _case(B=3, L=L, block=block, seed=L + block, batched_bias=batched)
+                out, lse, p = o.attn_fwd(c["q"], c["k"], c["v"], c["bias"],
+                                         block=block, cap=cap, probs=True)
+                ro, rl, rp = dense_bruteforce(c["q"], c["k"], c["v"], c["bias"],
+                                              block, cap)
+                what = f"L={L} block={block} cap={cap} batched={batched}"
+                _close(out, ro, 1e-12, "out " + what)
+                _close(lse, rl, 1e-12, "lse " + what)
+                _close(p, rp, 1e-12, "probs " + what)
+    # Rows of a batched-bias case agree with the full evaluation.
+    c = _case(B=2, L=40, block=16, seed=3, batched_bias=True)
+    out, lse = o.attn_fwd(c["q"], c["k"], c["v"], c["bias"], block=16, cap=5.0)
+    rows = [[0, 0, 0], [1, 2, 39], [1, 0, 33], [0, 1, 16]]
+    ro, rl = o.attn_rows(c["q"], c["k"], c["v"], c["bias"], rows, block=16, cap=5.0)
+    for t, (b, h, i) in enumerate(rows):
+        _close(ro[t], out[b, h, i], 1e-13, f"row {b},{h},{i} out")
+        _close(rl[t], lse[b, h, i], 1e-13, f"row {b},{h},{i} lse")
 
 
 def pin_sdpa(o):
@@ -237,6 +268,6 @@ def pin_projection(o):
 
 
 ALL_PINS = [
-    pin_bruteforce, pin_sdpa, pin_identical_keys, pin_block_bias_closed_form,
+    pin_bruteforce, pin_bruteforce_tails_and_batched_bias, pin_sdpa, pin_identical_keys, pin_block_bias_closed_form,
     pin_cap_limit, pin_probabilities, pin_invariances, pin_rows, pin_projection,
 ]

@@ -22,6 +22,8 @@ MUTANTS = {
     10: "values read from K",
     11: "every head uses query head 0",
     12: "soft cap dropped",
+    13: "every batch item reads item 0's bias",
+    14: "partial last block dropped from the bias layout",
 }
 
 

@@ -26,8 +26,10 @@ def test_oracle_rejects_bad_arguments(oracle_lib):
     for cap in (0.0, -1.0, math.nan):
         with pytest.raises(ValueError):
             oracle_lib.attn_fwd(q, k, v, bias, block=16, cap=cap)
-    with pytest.raises(ValueError):  # L not a multiple of the block
-        oracle_lib.attn_fwd(q[:, :, :30], k[:, :30], v[:, :30], bias, block=16, cap=5.0)
+    with pytest.raises(ValueError):  # bias not [H, ceil(L/block), ...]
+        oracle_lib.attn_fwd(q, k, v, np.zeros((1, 3, 3)), block=16, cap=5.0)
+    with pytest.raises(ValueError):  # per-item bias for the wrong batch size
+        oracle_lib.attn_fwd(q, k, v, np.zeros((2, 1, 2, 2)), block=16, cap=5.0)
     with pytest.raises(ValueError):  # row index out of range
         oracle_lib.attn_rows(q, k, v, bias, [[0, 0, 32]], block=16, cap=5.0)
 
