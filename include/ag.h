@@ -92,14 +92,18 @@ ag_status ag_pair_bias_project(const float *pair, const float *W, float *bias,
  *   q     [B, H, L, D]  bfloat16 bit patterns, 16-byte aligned
  *   k     [B, L, D]     bfloat16, 16-byte aligned (one head, shared by all H)
  *   v     [B, L, D]     bfloat16, 16-byte aligned (one head, shared by all H)
- *   bias  [H, P, P]     float32,   4-byte aligned, P = L / block, shared by
- *                       every batch item
+ *   bias  [H, P, P]     float32,   4-byte aligned, P = ceil(L / block),
+ *                       shared by every batch item (one bias per item:
+ *                       ag_attn_fwd_strided_bias)
  *   out   [B, H, L, D]  float32,  16-byte aligned (written)
  *   lse   [B, H, L]     float32,   4-byte aligned (written)
  *   cap   > 0 and not NaN; +INFINITY disables the soft cap.
- * Supported: H == 8, D == 128, block == 16, L % 16 == 0, L <= 65536,
- * B * L <= 2^28 and B * ceil(L/32) * ceil(L/128) <= 2^30 (B * L^2 up to
- * about 2^42).  B == 0 or L == 0 is a no-op (pointers may be NULL).
+ * Supported: H == 8, D == 128, block == 16, any L <= 65536 (a length that
+ * is not a multiple of 16 ends in a partial block, which uses its compact
+ * bias cell like the others: the page lists tails among what its kernel does
+ * not support yet, section "What has not yet been demonstrated"),
+ * B * L <= 2^28 and B * ceil(ceil(L/16)/2) * ceil(L/128) <= 2^30 (B * L^2 up
+ * to about 2^42).  B == 0 or L == 0 is a no-op (pointers may be NULL).
  * Products in bf16 with fp32 accumulation (tensor cores); softmax in fp32;
  * the probabilities are rounded to bf16 for the second product while the
  * row sums use their fp32 values.
@@ -117,6 +121,24 @@ ag_status ag_attn_fwd(const void *q, const void *k, const void *v,
                       const float *bias, int64_t B, int64_t H, int64_t L,
                       int64_t D, int64_t block, float cap, float *out,
                       float *lse, void *stream);
+
+/*
+ * ag_attn_fwd_strided_bias -- ag_attn_fwd with one bias per batch item.
+ *
+ * Each sequence has its own compact pair representation, hence its own bias
+ * (page "Making Full-Context AlphaGenome Fit on an RTX 3090", section
+ * "Profiling pointed at one very large object").  Batch item b reads
+ * bias + b * bias_batch_stride, a [H, P, P] float32 block (P = ceil(L /
+ * block)); bias_batch_stride is in floats, 0 (one bias shared by every item:
+ * exactly ag_attn_fwd) or at least H * P * P (e.g. H * P * P for a dense
+ * [B, H, P, P] tensor); anything else returns AG_ERR_SHAPE.  Everything else
+ * -- arguments, checks, results, scratch, stream behaviour -- as ag_attn_fwd.
+ */
+ag_status ag_attn_fwd_strided_bias(const void *q, const void *k, const void *v,
+                                   const float *bias, int64_t bias_batch_stride,
+                                   int64_t B, int64_t H, int64_t L, int64_t D,
+                                   int64_t block, float cap, float *out,
+                                   float *lse, void *stream);
 
 /*
  * ag_attn_fwd_noalloc -- ag_attn_fwd for callers that cannot allocate device

@@ -207,7 +207,6 @@ namespace ag {
 static ag_status check_attn_sizes(int64_t B, int64_t H, int64_t L, int64_t D,
                                   int64_t block, float cap) {
   if (B < 0 || H <= 0 || L < 0 || D <= 0 || block <= 0) return AG_ERR_SHAPE;
-  if (L % block != 0) return AG_ERR_SHAPE;
   if (std::isnan(cap) || !(cap > 0.0f)) return AG_ERR_VALUE;
   if (H != 8 || D != 128 || block != 16 || L > 65536) return AG_ERR_UNSUPPORTED;
   if (B > 0 && L > 0 && B * L > (int64_t(1) << 28)) return AG_ERR_UNSUPPORTED;
@@ -221,17 +220,29 @@ ag_status ag_attn_fwd(const void *q, const void *k, const void *v,
                       const float *bias, int64_t B, int64_t H, int64_t L,
                       int64_t D, int64_t block, float cap, float *out,
                       float *lse, void *stream) {
+  return ag_attn_fwd_strided_bias(q, k, v, bias, 0, B, H, L, D, block, cap, out,
+                                  lse, stream);
+}
+
+ag_status ag_attn_fwd_strided_bias(const void *q, const void *k, const void *v,
+                                   const float *bias, int64_t bias_batch_stride,
+                                   int64_t B, int64_t H, int64_t L, int64_t D,
+                                   int64_t block, float cap, float *out,
+                                   float *lse, void *stream) {
   const ag_status vs = ag::check_attn_sizes(B, H, L, D, block, cap);
   if (vs != AG_OK) return vs;
+  const int64_t P = block > 0 ? (L + block - 1) / block : 0;
+  if (bias_batch_stride < 0 || (bias_batch_stride > 0 && bias_batch_stride < H * P * P))
+    return AG_ERR_SHAPE;
   if (B == 0 || L == 0) return AG_OK;
   if (!q || !k || !v || !bias || !out || !lse) return AG_ERR_NULL;
   if (!ag::aligned(q, 16) || !ag::aligned(k, 16) || !ag::aligned(v, 16) ||
       !ag::aligned(bias, 4) || !ag::aligned(out, 16) || !ag::aligned(lse, 4))
     return AG_ERR_ALIGN;
-  const uint64_t P = static_cast<uint64_t>(L / block);
   const uint64_t qb = static_cast<uint64_t>(B) * H * L * D * 2;
   const uint64_t kb = static_cast<uint64_t>(B) * L * D * 2;
-  const uint64_t bb = static_cast<uint64_t>(H) * P * P * 4;
+  const uint64_t bb = (static_cast<uint64_t>(B - 1) * bias_batch_stride +
+                       static_cast<uint64_t>(H) * P * P) * 4;
   const uint64_t ob = static_cast<uint64_t>(B) * H * L * D * 4;
   const uint64_t lb = static_cast<uint64_t>(B) * H * L * 4;
   const void *ins[4] = {q, k, v, bias};
@@ -254,6 +265,7 @@ ag_status ag_attn_fwd(const void *q, const void *k, const void *v,
   a.k = k;
   a.v = v;
   a.bias = bias;
+  a.bias_bstride = bias_batch_stride;
   a.out = out;
   a.lse = lse;
   a.B = B;
@@ -280,7 +292,7 @@ ag_status ag_attn_fwd_noalloc(const void *q, const void *k, const void *v,
   if (!ag::aligned(q, 16) || !ag::aligned(k, 16) || !ag::aligned(v, 16) ||
       !ag::aligned(bias, 4) || !ag::aligned(out, 16) || !ag::aligned(lse, 4))
     return AG_ERR_ALIGN;
-  const uint64_t P = static_cast<uint64_t>(L / block);
+  const uint64_t P = static_cast<uint64_t>((L + block - 1) / block);
   const uint64_t qb = static_cast<uint64_t>(B) * H * L * D * 2;
   const uint64_t kb = static_cast<uint64_t>(B) * L * D * 2;
   const uint64_t bb = static_cast<uint64_t>(H) * P * P * 4;
@@ -313,6 +325,7 @@ ag_status ag_attn_fwd_noalloc(const void *q, const void *k, const void *v,
   a.k = k;
   a.v = v;
   a.bias = bias;
+  a.bias_bstride = 0;
   a.out = out;
   a.lse = lse;
   a.B = B;

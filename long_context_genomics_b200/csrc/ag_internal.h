@@ -28,12 +28,14 @@ inline size_t attn_scratch_bytes(int slots) {
 // kernel indexes steps with int, so callers keep this at or below 2^30.
 constexpr int64_t kAttnKeyTile = 128;
 inline int64_t attn_work_steps(int64_t B, int64_t L) {
-  return B * ((L / 16 + 1) / 2) * ((L + kAttnKeyTile - 1) / kAttnKeyTile);
+  const int64_t blocks = (L + 15) / 16;  // the last may be partial
+  return B * ((blocks + 1) / 2) * ((L + kAttnKeyTile - 1) / kAttnKeyTile);
 }
 
 struct AttnLaunch {
   const void *q, *k, *v;
   const float *bias;
+  int64_t bias_bstride;  // floats between batch items' bias (0: shared)
   float *out, *lse;
   int64_t B, L;
   float cap;

@@ -138,6 +138,7 @@ static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
 struct Params {
   const float *bias;
+  long long bias_bstride;  // floats between batch items' bias (0: shared)
   float *out;
   float *lse;
   unsigned *err;
@@ -145,11 +146,11 @@ struct Params {
   float *ws_out;       // [clusters][2][128][128] partial outputs
   float *ws_lse;       // [clusters][2][128] partial log-sum-exps
   int L, P;
-  int nb;          // 16-position query blocks per batch item (L / 16)
+  int nb;          // 16-position query blocks per batch item, ceil(L / 16)
   int pairs;       // query-tile pairs per batch item: ceil(nb / 2)
   int n_items;     // B * pairs
   int n_kt;        // key tiles: ceil(L / 128)
-  int last_valid;  // valid keys in the last key tile (16..128)
+  int last_valid;  // valid keys in the last key tile (1..128)
   int whole;       // 1: cluster ranges hold whole pairs (no split pairs)
   float qk_scale;  // multiplies q.k
   float bias_mul;  // multiplies the compact bias
@@ -730,7 +731,9 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc,
     const int I0 = (sg.item % p.pairs) * 2;
     const int I = tile_block(p, I0, rank);
     const bool valid = I0 + static_cast<int>(rank) < p.nb;
-    const float *brow = p.bias + (static_cast<size_t>(h) * p.P + I) * p.P;
+    const int pos = I * 16 + il;  // this thread's query position
+    const float *brow = p.bias + static_cast<long long>(b) * p.bias_bstride +
+                        (static_cast<size_t>(h) * p.P + I) * p.P;
     float m = (MODE == kStaticCap) ? p.A : -INFINITY;  // log2 units
     float d = 0.f;
     if constexpr (MODE == kStaticCap) {
@@ -765,9 +768,9 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc,
     uint32_t o[32];
     tmem_ld32(tmem + kColO + 32 * g + lane_base, o);
     tmem_wait_ld(o);
-    if (valid) {
+    if (valid && pos < p.L) {  // rows past the end of a partial block: none
       const size_t row = (static_cast<size_t>(b) * kH + h) * p.L +
-                         static_cast<size_t>(I) * 16 + il;
+                         static_cast<size_t>(pos);
       float *orow_base;
       float *lse_dst;
       if (sg.kb == 0) {
@@ -910,8 +913,10 @@ __global__ void __launch_bounds__(kMergeThreads)
   if (X >= nX) return;
   const int lane = static_cast<int>(threadIdx.x & 31);
   const int h = r >> 4, il = r & 15;
+  const int pos = (I0 + X) * 16 + il;
+  if (pos >= p.L) return;  // past the end of a partial last block
   const size_t row = (static_cast<size_t>(b) * kH + h) * p.L +
-                     static_cast<size_t>(I0 + X) * 16 + il;
+                     static_cast<size_t>(pos);
   auto slot = [&](int s) {
     return (static_cast<size_t>(c_first + s) * 2 + X) * 128 + r;
   };
@@ -1047,7 +1052,7 @@ cudaError_t attn_fwd_kernel_count(int64_t B, int64_t L, float cap, int num_sms,
     *count = 0;
     return cudaSuccess;
   }
-  const int nb = static_cast<int>(L / 16);
+  const int nb = static_cast<int>((L + 15) / 16);
   const int n_items = static_cast<int>(B) * ((nb + 1) / 2);
   const int n_kt = static_cast<int>((L + kKeys - 1) / kKeys);
   int clusters = 0, whole = 0;
@@ -1088,8 +1093,9 @@ cudaError_t launch_attn_fwd(const AttnLaunch &a) {
   p.lse = a.lse;
   p.err = a.err;
   p.L = static_cast<int>(L);
-  p.P = static_cast<int>(L / 16);
-  p.nb = static_cast<int>(L / 16);
+  p.P = static_cast<int>((L + 15) / 16);
+  p.nb = p.P;
+  p.bias_bstride = a.bias_bstride;
   p.pairs = (p.nb + 1) / 2;
   p.n_items = static_cast<int>(B) * p.pairs;
   p.n_kt = static_cast<int>((L + kKeys - 1) / kKeys);

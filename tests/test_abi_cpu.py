@@ -57,7 +57,7 @@ def _attn(ag, q=A16, k=A16 * 2, v=A16 * 3, bias=A16 * 4, B=1, H=8, L=256, D=128,
 
 @pytest.mark.parametrize("kw,status", [
     (dict(q=None), 1), (dict(out=None), 1), (dict(lse=None), 1), (dict(bias=None), 1),
-    (dict(B=-1), 2), (dict(L=-16), 2), (dict(L=250), 2), (dict(D=0), 2),
+    (dict(B=-1), 2), (dict(L=-16), 2), (dict(D=0), 2),
     (dict(H=4), 4), (dict(D=64), 4), (dict(block=8), 4), (dict(L=65536 + 16), 4),
     (dict(B=1 << 20, L=65536), 4),
     # B * L = 2^27 is allowed, but B * ceil(L/32) * ceil(L/128) = 2^31 work steps is not.
@@ -75,10 +75,29 @@ def test_launch_count_checks_before_the_device(ag):
     n = ctypes.c_int(-1)
     f = ag.lib.ag_attn_fwd_launch_count
     assert f(1, 8, 256, 128, 16, 5.0, None) == 1                    # AG_ERR_NULL
-    assert f(1, 8, 250, 128, 16, 5.0, ctypes.byref(n)) == 2         # AG_ERR_SHAPE
+    assert f(1, 8, -1, 128, 16, 5.0, ctypes.byref(n)) == 2          # AG_ERR_SHAPE
     assert f(1, 8, 256, 64, 16, 5.0, ctypes.byref(n)) == 4          # AG_ERR_UNSUPPORTED
     assert f(1, 8, 256, 128, 16, -1.0, ctypes.byref(n)) == 5        # AG_ERR_VALUE
     assert f(0, 8, 256, 128, 16, 5.0, ctypes.byref(n)) == 0 and n.value == 0
+
+
+def _attn_strided(ag, stride, q=A16, k=A16 * 2, v=A16 * 3, bias=A16 * 4, B=2, H=8,
+                  L=250, D=128, block=16, cap=5.0, out=A16 * 1000, lse=A16 * 2000):
+    return ag.lib.ag_attn_fwd_strided_bias(q, k, v, bias, stride, B, H, L, D, block,
+                                           cap, out, lse, None)
+
+
+def test_strided_bias_validation(ag):
+    # L = 250 ends in a partial block: P = 16 cells per side.
+    P = 16
+    assert _attn_strided(ag, -1) == 2                      # negative stride
+    assert _attn_strided(ag, 8 * P * P - 1) == 2           # overlapping items
+    assert _attn_strided(ag, 8 * P * P, q=None) == 1       # a dense [B,H,P,P]: passes to NULL check
+    assert _attn_strided(ag, 0, q=None) == 1               # shared bias
+    assert _attn_strided(ag, 8 * P * P, bias=BAD + 1) == 3  # bias not 4-byte aligned
+    # The per-item bias span (B-1)*stride + H*P*P floats must not overlap out.
+    span = (1 * 10 * 8 * P * P + 8 * P * P) * 4
+    assert _attn_strided(ag, 10 * 8 * P * P, bias=A16 * 1000 - span + 16) == 7
 
 
 def test_attn_empty_is_a_noop(ag):

@@ -127,6 +127,71 @@ def test_ragged_and_odd_shapes(ag, oracle_lib, B, L, cap):
     _compare(out, lse, ro, rl, f"B={B} L={L} cap={cap}")
 
 
+@pytest.mark.parametrize("B,L", [(1, 1), (1, 17), (2, 100), (1, 1000), (3, 2049),
+                                 (1, 4095)])
+@pytest.mark.parametrize("cap", [5.0, 50.0, math.inf])
+def test_lengths_with_a_partial_block(ag, oracle_lib, B, L, cap):
+    """L not a multiple of 16: the last query block and the last bias cell
+    cover fewer than 16 positions (P = ceil(L/16)); rows past L are never
+    written."""
+    inp = ag_inputs.random_case(B, 8, L, 128, 128, 16, seed=B * 7919 + L)
+    q, k, v = _dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"])
+    bias = _dev(inp["bias"])
+    out = torch.full((B, 8, L, 128), float("nan"), device="cuda")
+    lse = torch.full((B, 8, L), float("nan"), device="cuda")
+    ag.ag_attn_fwd(q, k, v, bias, cap=cap, out=out, lse=lse)
+    torch.cuda.synchronize()
+    assert ag.ag_device_error(0) == 0
+    ro, rl = oracle_lib.attn_fwd(inp["q"], inp["k"], inp["v"], inp["bias"],
+                                 block=16, cap=cap)
+    _compare(out.double().cpu().numpy(), lse.double().cpu().numpy(), ro, rl,
+             f"B={B} L={L} cap={cap}")
+
+
+@pytest.mark.parametrize("B,L", [(3, 1040), (2, 333), (2, 8192)])
+@pytest.mark.parametrize("cap", [5.0, math.inf])
+def test_one_bias_per_batch_item(ag, oracle_lib, B, L, cap):
+    """bias [B,H,P,P] (ag_attn_fwd_strided_bias): each batch item reads its
+    own bias; full outputs against the oracle (sampled rows at L = 8192)."""
+    inp = ag_inputs.random_case(B, 8, L, 128, 128, 16, seed=B * 31 + L,
+                                batched_bias=True)
+    out, lse = _gpu_attn(ag, inp, cap)
+    if L <= 2048:
+        ro, rl = oracle_lib.attn_fwd(inp["q"], inp["k"], inp["v"], inp["bias"],
+                                     block=16, cap=cap)
+        _compare(out, lse, ro, rl, f"per-item bias B={B} L={L} cap={cap}")
+    else:
+        rows = ag_inputs.sample_rows(B, 8, L, 384, seed=L).numpy()
+        ro, rl = oracle_lib.attn_rows(inp["q"], inp["k"], inp["v"], inp["bias"], rows,
+                                      block=16, cap=cap)
+        b, h, i = rows[:, 0], rows[:, 1], rows[:, 2]
+        _compare(out[b, h, i], lse[b, h, i], ro, rl, f"per-item bias B={B} L={L} sampled")
+
+
+def test_strided_bias_with_padding_between_items(ag, oracle_lib):
+    """A bias batch stride larger than H*P*P (padded items) through the C ABI."""
+    import ctypes
+    B, L = 2, 400
+    P = 25
+    inp = ag_inputs.random_case(B, 8, L, 128, 128, 16, seed=5, batched_bias=True)
+    stride = 8 * P * P + 96
+    padded = torch.full((B, stride), float("nan"))
+    padded[:, : 8 * P * P] = inp["bias"].reshape(B, -1)
+    q, k, v, bp = _dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"]), _dev(padded)
+    out = torch.empty(B, 8, L, 128, device="cuda")
+    lse = torch.empty(B, 8, L, device="cuda")
+    st = ag.lib.ag_attn_fwd_strided_bias(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), bp.data_ptr(), stride, B, 8, L, 128,
+        16, ctypes.c_float(5.0), out.data_ptr(), lse.data_ptr(), None)
+    assert st == 0
+    torch.cuda.synchronize()
+    assert ag.ag_device_error(0) == 0
+    ro, rl = oracle_lib.attn_fwd(inp["q"], inp["k"], inp["v"], inp["bias"], block=16,
+                                 cap=5.0)
+    _compare(out.double().cpu().numpy(), lse.double().cpu().numpy(), ro, rl,
+             "padded per-item bias")
+
+
 @pytest.mark.parametrize("cap", [1.0, 5.0, 10.0, 30.0, 40.0, 50.0, 1e4, math.inf])
 def test_cap_modes(ag, oracle_lib, cap):
     """Static shift (cap <= 40), running max with the cap (cap > 40) and no
