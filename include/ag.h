@@ -110,9 +110,9 @@ ag_status ag_pair_bias_project(const float *pair, const float *W, float *bias,
  *
  * Scratch: to keep every SM busy to the end, a pair of query tiles may have
  * its keys split between SM pairs (the kernel runs on 2-CTA clusters); each
- * piece's partial result goes through a scratch buffer of 132,096 bytes per
- * SM (19.6 MB on a 148-SM B200; half of it is used) and a second kernel on
- * the same stream merges the pieces (by log-sum-exp).  The
+ * piece's partial result goes through a scratch buffer of 197,632 bytes per
+ * SM (29.2 MB on a 148-SM B200; at most half of it is used) and a second
+ * kernel on the same stream merges the pieces (by log-sum-exp).  The
  * first call on a device allocates that buffer with cudaMalloc; it is kept
  * until the process exits.  Calls whose kernels overlap on the device (e.g.
  * on two streams at once) must not run concurrently, because they share it.
@@ -141,13 +141,27 @@ ag_status ag_attn_fwd_strided_bias(const void *q, const void *k, const void *v,
                                    float *lse, void *stream);
 
 /*
+ * ag_attn_fwd_ex -- ag_attn_fwd_strided_bias with a value width Dv of its
+ * own: v [B, L, Dv] and out [B, H, L, Dv].  The page's checkpoint has
+ * Dv = 192 against D = 128 (section "Why stock FlashAttention was not a
+ * drop-in replacement", tensors Q, K, V); the scale stays 1 / sqrt(D).
+ * Supported: Dv == 128 or Dv == 192 (AG_ERR_UNSUPPORTED otherwise,
+ * AG_ERR_SHAPE if Dv <= 0); v 16-byte aligned.  Everything else as
+ * ag_attn_fwd_strided_bias, which is this call with Dv = D.
+ */
+ag_status ag_attn_fwd_ex(const void *q, const void *k, const void *v,
+                         const float *bias, int64_t bias_batch_stride, int64_t B,
+                         int64_t H, int64_t L, int64_t D, int64_t Dv, int64_t block,
+                         float cap, float *out, float *lse, void *stream);
+
+/*
  * ag_attn_fwd_noalloc -- ag_attn_fwd for callers that cannot allocate device
  * memory (the pages have no counterpart; this is a library convenience).
  *
  * Same arguments, checks, results and stream behaviour as ag_attn_fwd, but
  * it never calls cudaMalloc or cudaFree: its split-pair scratch is a static
- * device array compiled into the library, 148 slots of 132,096 bytes
- * (19,550,208 bytes), which every GPU that loads the library holds until the
+ * device array compiled into the library, 148 slots of 197,632 bytes
+ * (29,249,536 bytes), which every GPU that loads the library holds until the
  * process exits.  Useful where an allocation is not allowed or not wanted,
  * e.g. code that must not touch the allocator while a CUDA graph is being
  * captured, or a framework that has handed all device memory to its own pool.

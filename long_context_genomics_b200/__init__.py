@@ -59,6 +59,9 @@ def _load() -> ctypes.CDLL:
     lib.ag_attn_fwd_strided_bias.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64,
                                              i64, i64, f32, vp, vp, vp]
     lib.ag_attn_fwd_strided_bias.restype = ctypes.c_int
+    lib.ag_attn_fwd_ex.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, i64,
+                                   i64, f32, vp, vp, vp]
+    lib.ag_attn_fwd_ex.restype = ctypes.c_int
     lib.ag_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64,
                                         f32, vp, vp, vp]
     lib.ag_attn_fwd_noalloc.restype = ctypes.c_int
@@ -130,27 +133,29 @@ def ag_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                 stream=None):
     """Fused pair-bias MQA attention forward (libag kernel).
 
-    bias is [H,P,P] (shared by the batch; ag_attn_fwd) or [B,H,P,P] (one per
-    batch item; ag_attn_fwd_strided_bias), P = ceil(L / block).  Returns
-    (out [B,H,L,D] fp32, lse [B,H,L] fp32).  cap = math.inf turns the soft cap
-    off."""
+    bias is [H,P,P] (shared by the batch) or [B,H,P,P] (one per batch item),
+    P = ceil(L / block); v is [B,L,Dv] with Dv = D or 192 (the page's
+    checkpoint).  Calls ag_attn_fwd_ex.  Returns (out [B,H,L,Dv] fp32,
+    lse [B,H,L] fp32).  cap = math.inf turns the soft cap off."""
     _check(q, "q", torch.bfloat16, 4)
     _check(k, "k", torch.bfloat16, 3)
     _check(v, "v", torch.bfloat16, 3)
     B, H, L, D = q.shape
-    if tuple(k.shape) != (B, L, D) or tuple(v.shape) != (B, L, D):
-        raise ValueError("k and v must be [B,L,D] with q [B,H,L,D]")
+    Dv = v.shape[-1]
+    if tuple(k.shape) != (B, L, D) or tuple(v.shape) != (B, L, Dv):
+        raise ValueError("k must be [B,L,D] and v [B,L,Dv] with q [B,H,L,D]")
     bstride = _bias_stride(bias, B, H, L, block)
     if out is None:
-        out = torch.empty((B, H, L, D), dtype=torch.float32, device=q.device)
+        out = torch.empty((B, H, L, Dv), dtype=torch.float32, device=q.device)
     if lse is None:
         lse = torch.empty((B, H, L), dtype=torch.float32, device=q.device)
-    _check_out(out, lse, B, H, L, D)
-    st = lib.ag_attn_fwd_strided_bias(
+    _check_out(out, lse, B, H, L, Dv)
+    st = lib.ag_attn_fwd_ex(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), bias.data_ptr(), bstride, B, H, L,
-        D, int(block), float(cap), out.data_ptr(), lse.data_ptr(), _stream_ptr(stream))
+        D, Dv, int(block), float(cap), out.data_ptr(), lse.data_ptr(),
+        _stream_ptr(stream))
     if st != AG_OK:
-        raise AgError("ag_attn_fwd" if bstride == 0 else "ag_attn_fwd_strided_bias", st)
+        raise AgError("ag_attn_fwd_ex", st)
     return out, lse
 
 
@@ -166,11 +171,11 @@ def _bias_stride(bias: torch.Tensor, B: int, H: int, L: int, block: int) -> int:
     raise ValueError(f"bias must be [{H},{P},{P}] or [{B},{H},{P},{P}], got {tuple(bias.shape)}")
 
 
-def _check_out(out: torch.Tensor, lse: torch.Tensor, B: int, H: int, L: int, D: int):
+def _check_out(out: torch.Tensor, lse: torch.Tensor, B: int, H: int, L: int, Dv: int):
     _check(out, "out", torch.float32, 4)
     _check(lse, "lse", torch.float32, 3)
-    if tuple(out.shape) != (B, H, L, D) or tuple(lse.shape) != (B, H, L):
-        raise ValueError("out must be [B,H,L,D] and lse [B,H,L]")
+    if tuple(out.shape) != (B, H, L, Dv) or tuple(lse.shape) != (B, H, L):
+        raise ValueError("out must be [B,H,L,Dv] and lse [B,H,L]")
 
 
 def ag_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,

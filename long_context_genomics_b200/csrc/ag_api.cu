@@ -229,8 +229,18 @@ ag_status ag_attn_fwd_strided_bias(const void *q, const void *k, const void *v,
                                    int64_t B, int64_t H, int64_t L, int64_t D,
                                    int64_t block, float cap, float *out,
                                    float *lse, void *stream) {
+  return ag_attn_fwd_ex(q, k, v, bias, bias_batch_stride, B, H, L, D, D, block, cap,
+                        out, lse, stream);
+}
+
+ag_status ag_attn_fwd_ex(const void *q, const void *k, const void *v,
+                         const float *bias, int64_t bias_batch_stride, int64_t B,
+                         int64_t H, int64_t L, int64_t D, int64_t Dv, int64_t block,
+                         float cap, float *out, float *lse, void *stream) {
   const ag_status vs = ag::check_attn_sizes(B, H, L, D, block, cap);
   if (vs != AG_OK) return vs;
+  if (Dv <= 0) return AG_ERR_SHAPE;
+  if (Dv != 128 && Dv != 192) return AG_ERR_UNSUPPORTED;
   const int64_t P = block > 0 ? (L + block - 1) / block : 0;
   if (bias_batch_stride < 0 || (bias_batch_stride > 0 && bias_batch_stride < H * P * P))
     return AG_ERR_SHAPE;
@@ -241,12 +251,13 @@ ag_status ag_attn_fwd_strided_bias(const void *q, const void *k, const void *v,
     return AG_ERR_ALIGN;
   const uint64_t qb = static_cast<uint64_t>(B) * H * L * D * 2;
   const uint64_t kb = static_cast<uint64_t>(B) * L * D * 2;
+  const uint64_t vb = static_cast<uint64_t>(B) * L * Dv * 2;
   const uint64_t bb = (static_cast<uint64_t>(B - 1) * bias_batch_stride +
                        static_cast<uint64_t>(H) * P * P) * 4;
-  const uint64_t ob = static_cast<uint64_t>(B) * H * L * D * 4;
+  const uint64_t ob = static_cast<uint64_t>(B) * H * L * Dv * 4;
   const uint64_t lb = static_cast<uint64_t>(B) * H * L * 4;
   const void *ins[4] = {q, k, v, bias};
-  const uint64_t insz[4] = {qb, kb, kb, bb};
+  const uint64_t insz[4] = {qb, kb, vb, bb};
   for (int t = 0; t < 4; ++t)
     if (ag::overlap(out, ob, ins[t], insz[t]) || ag::overlap(lse, lb, ins[t], insz[t]))
       return AG_ERR_ALIAS;
@@ -270,6 +281,7 @@ ag_status ag_attn_fwd_strided_bias(const void *q, const void *k, const void *v,
   a.lse = lse;
   a.B = B;
   a.L = L;
+  a.Dv = Dv;
   a.cap = cap;
   a.err = dev->err;
   a.num_sms = dev->num_sms;
@@ -330,6 +342,7 @@ ag_status ag_attn_fwd_noalloc(const void *q, const void *k, const void *v,
   a.lse = lse;
   a.B = B;
   a.L = L;
+  a.Dv = D;
   a.cap = cap;
   a.err = dev->err;
   a.num_sms = dev->num_sms;
@@ -353,7 +366,7 @@ ag_status ag_attn_fwd_launch_count(int64_t B, int64_t H, int64_t L, int64_t D,
   ag_status st = ag::device_info(&dev);
   if (st != AG_OK) return st;
   int n = 0;
-  st = ag::from_cuda(ag::attn_fwd_kernel_count(B, L, cap, dev->num_sms, dev->num_sms, &n));
+  st = ag::from_cuda(ag::attn_fwd_kernel_count(B, L, D, cap, dev->num_sms, dev->num_sms, &n));
   if (st != AG_OK) return st;
   *count = n;
   return AG_OK;

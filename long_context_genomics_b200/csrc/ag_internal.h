@@ -15,9 +15,10 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType,
                                    CUtensorMapFloatOOBfill);
 
 // Scratch of the attention kernel for pairs of query tiles whose key range is
-// split between CTAs: per CTA slot a partial output [2][128][128] fp32 and a
-// partial log-sum-exp [2][128] fp32.  Nothing in it must be initialised.
-constexpr size_t kAttnSlotOutBytes = 2 * 128 * 128 * sizeof(float);
+// split between clusters: per slot a partial output [2][128][Dv] fp32 (sized
+// for the widest Dv, 192) and a partial log-sum-exp [2][128] fp32.  Nothing
+// in it must be initialised.
+constexpr size_t kAttnSlotOutBytes = 2 * 128 * 192 * sizeof(float);
 constexpr size_t kAttnSlotLseBytes = 2 * 128 * sizeof(float);
 inline size_t attn_scratch_bytes(int slots) {
   return static_cast<size_t>(slots) * (kAttnSlotOutBytes + kAttnSlotLseBytes);
@@ -38,6 +39,7 @@ struct AttnLaunch {
   int64_t bias_bstride;  // floats between batch items' bias (0: shared)
   float *out, *lse;
   int64_t B, L;
+  int64_t Dv;           // value width: 128 or 192
   float cap;
   unsigned *err;        // device error word
   int num_sms;
@@ -53,8 +55,8 @@ cudaError_t launch_attn_fwd(const AttnLaunch &a);
 
 // How many kernels launch_attn_fwd launches for these sizes on the current
 // device (0 for an empty call, 1, or 2 when split pairs need the merge).
-cudaError_t attn_fwd_kernel_count(int64_t B, int64_t L, float cap, int num_sms,
-                                  int scratch_slots, int *count);
+cudaError_t attn_fwd_kernel_count(int64_t B, int64_t L, int64_t Dv, float cap,
+                                  int num_sms, int scratch_slots, int *count);
 
 cudaError_t launch_pair_bias_project(const float *pair, const float *W,
                                      float *bias, int64_t P, int num_sms,

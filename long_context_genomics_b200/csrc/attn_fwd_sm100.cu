@@ -62,11 +62,36 @@ constexpr int kQHalfBytes = kQTileBytes / 2;  // one 64-wide (128-byte) half
 // two consecutive step loads, so the MMA thread waits for data and releases
 // it once per two steps (each mbarrier operation costs it about 180 cycles
 // while the tensor core is busy, measured).
-constexpr int kPartBytes = 16384;            // one K half or one V half
+constexpr int kPartBytes = 16384;            // one K half
 constexpr int kKHalfBytes = kPartBytes / 2;  // a K half's 64-wide half
-constexpr int kStepBytes = 2 * kPartBytes;
-constexpr int kSlotBytes = 2 * kStepBytes;
 constexpr int kStages = 2;
+
+// This CTA's half of a V tile, 128 keys x DV/2 value columns, MN-major for
+// the PV product.  DV = 128: one 128-byte-swizzled 64-column box.  DV = 192
+// (the value width of the page's checkpoint, section "Why stock
+// FlashAttention was not a drop-in replacement", tensor V): 96 columns, which
+// 64-column atoms cannot tile, so three 64-byte-swizzled 32-column boxes
+// 8 KB apart.
+template <int DV> struct VLayout;
+template <> struct VLayout<128> {
+  static constexpr int kBoxes = 1, kBoxCols = 64;
+  static constexpr int kPartBytes = 128 * 64 * 2;       // 16 KB
+  static constexpr uint32_t kDescHi = desc_sw128_hi(1024);
+  static constexpr uint32_t kAtomBytes = 16384;         // LBO (one atom: unused)
+  static constexpr uint32_t kKStepBytes = 16 * 128;     // 16 keys x 128 B
+};
+template <> struct VLayout<192> {
+  static constexpr int kBoxes = 3, kBoxCols = 32;
+  static constexpr int kPartBytes = 128 * 96 * 2;       // 24 KB
+  static constexpr uint32_t kDescHi = desc_sw64_hi(512);
+  static constexpr uint32_t kAtomBytes = 8192;          // LBO: 32-column atoms
+  static constexpr uint32_t kKStepBytes = 16 * 64;      // 16 keys x 64 B
+};
+// A step load: a K half (part 0) and a V half or a second K half (part 1).
+template <int DV> constexpr int step_bytes() { return kPartBytes + VLayout<DV>::kPartBytes; }
+template <int DV> constexpr int slot_bytes() { return 2 * step_bytes<DV>(); }
+static_assert(step_bytes<128>() >= 2 * kPartBytes && step_bytes<192>() >= 2 * kPartBytes,
+              "step load 0 holds two K halves");
 constexpr int kWG = 4;                      // softmax warpgroups
 constexpr int kSoftThreads = 128 * kWG;
 constexpr int kSoftWarps = 4 * kWG;         // per CTA
@@ -84,12 +109,12 @@ constexpr uint32_t kRegsLow = 88;
 static_assert(kSoftThreads * kRegsLaunch + 128 * kRegsLow <= kThreads * kRegsLaunch,
               "register split exceeds the launch allocation");
 constexpr uint32_t kTmemCols = 512;
-// Tensor-memory columns: S buffer u at 128 u, O at 256.  P (bf16 pairs) of
+// Tensor-memory columns: S buffer u at 128 u, O at 256 (DV columns).  P (bf16 pairs) of
 // chunk c (keys [32c, 32c + 32) of the tile) is written over the first 16
 // columns of that chunk's own S columns, [32c, 32c + 16).
 constexpr uint32_t kColO = 256;
 constexpr uint32_t kIdescQK = idesc_bf16_f32(256, kKeys, 0);  // K-major B (K)
-constexpr uint32_t kIdescPV = idesc_bf16_f32(256, kD, 1);     // MN-major B (V)
+template <int DV> constexpr uint32_t idesc_pv() { return idesc_bf16_f32(256, DV, 1); }
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 // Lazy rescale threshold (log2 units) for the running-max modes.
@@ -131,10 +156,13 @@ struct Xchg {
   float dpart[kWG][128];     // [chunk][row]
 };
 
-constexpr size_t kSmemBytes = 1024 + static_cast<size_t>(kQTileBytes) +
-                              kStages * static_cast<size_t>(kSlotBytes) +
-                              sizeof(Barriers) + sizeof(Xchg);
-static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+template <int DV> constexpr size_t smem_bytes() {
+  return 1024 + static_cast<size_t>(kQTileBytes) +
+         kStages * static_cast<size_t>(slot_bytes<DV>()) + sizeof(Barriers) +
+         sizeof(Xchg);
+}
+static_assert(smem_bytes<128>() <= 227 * 1024 && smem_bytes<192>() <= 227 * 1024,
+              "shared memory budget");
 
 struct Params {
   const float *bias;
@@ -143,7 +171,7 @@ struct Params {
   float *lse;
   unsigned *err;
   // Split-pair scratch (see "Split pairs"): one slot per cluster.
-  float *ws_out;       // [clusters][2][128][128] partial outputs
+  float *ws_out;       // [clusters][2][128][DV] partial outputs
   float *ws_lse;       // [clusters][2][128] partial log-sum-exps
   int L, P;
   int nb;          // 16-position query blocks per batch item, ceil(L / 16)
@@ -234,17 +262,19 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_addr,
   }
 }
 
-// O[256 x 128] (+)= P[256 x 128 keys] V[128 keys x 128]: P from each CTA's
+// O[256 x DV] (+)= P[256 x 128 keys] V[128 keys x DV]: P from each CTA's
 // tensor memory (bf16 pairs, 8 columns per 16 keys; keys 32c.. of chunk c
-// start at column 32c of the S buffer), V MN-major: each CTA holds 64 value
-// columns (one 128-byte atom) for all 128 keys, 8-key row groups 1 KB apart.
+// start at column 32c of the S buffer), V MN-major: each CTA holds DV/2 value
+// columns for all 128 keys (VLayout).
+template <int DV>
 __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t s_tmem,
                                          uint32_t v_addr, bool accumulate) {
-  const uint32_t v_lo = desc_sw128_lo(v_addr, kPartBytes / 2);
+  using VL = VLayout<DV>;
+  const uint32_t v_lo = desc_sw128_lo(v_addr, VL::kAtomBytes);
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk) {
     umma2_ts_lo(d_tmem, s_tmem + 32 * (kk >> 1) + 8 * (kk & 1),
-                v_lo + ((kk * 2048) >> 4), kDescHi, kIdescPV,
+                v_lo + ((kk * VL::kKStepBytes) >> 4), VL::kDescHi, idesc_pv<DV>(),
                 (accumulate || kk > 0) ? 1u : 0u);
   }
 }
@@ -269,6 +299,7 @@ __device__ __forceinline__ int tile_block(const Params &p, int I0, uint32_t rank
 // --------------------------------------------------------------------------
 // Producer warp, lane 0 (each CTA): TMA loads of this CTA's Q tile and of its
 // halves of the K and V tiles.
+template <int DV>
 __device__ __forceinline__ void producer(const CUtensorMap *tm_q,
                                          const CUtensorMap *tm_k,
                                          const CUtensorMap *tm_v, uint8_t *q_s,
@@ -299,7 +330,8 @@ __device__ __forceinline__ void producer(const CUtensorMap *tm_q,
       uint32_t bytes = 0;
       for (int i = i0; i <= i1; ++i) {
         const StepLoad sl = step_load(sg, i);
-        bytes += (sl.k_tile >= 0 ? kPartBytes : 0) + (sl.second >= 0 ? kPartBytes : 0);
+        bytes += (sl.k_tile >= 0 ? kPartBytes : 0) +
+                 (sl.second < 0 ? 0 : sl.is_v ? VLayout<DV>::kPartBytes : kPartBytes);
       }
       mbar_arrive_expect_tx(&bars->kv_full[slot], bytes);
       // A K half: keys [128 j + 64 rank, +64), all 128 columns.
@@ -310,13 +342,18 @@ __device__ __forceinline__ void producer(const CUtensorMap *tm_q,
       };
       for (int i = i0; i <= i1; ++i) {
         const StepLoad sl = step_load(sg, i);
-        uint8_t *dst = kv_s + slot * kSlotBytes + (i & 1) * kStepBytes;
+        uint8_t *dst = kv_s + slot * slot_bytes<DV>() + (i & 1) * step_bytes<DV>();
         if (sl.k_tile >= 0) load_k(dst, sl.k_tile);
-        if (sl.is_v)  // keys [128 j, +128), value columns [64 rank, +64)
-          tma_load_3d(dst + kPartBytes, tm_v, &bars->kv_full[slot],
-                      64 * static_cast<int>(rank), sl.second * kKeys, b, pol_kv);
-        else if (sl.second >= 0)
+        if (sl.is_v) {  // keys [128 j, +128), value columns [DV/2 rank, +DV/2)
+#pragma unroll
+          for (int a = 0; a < VLayout<DV>::kBoxes; ++a)
+            tma_load_3d(dst + kPartBytes + a * VLayout<DV>::kAtomBytes, tm_v,
+                        &bars->kv_full[slot],
+                        (DV / 2) * static_cast<int>(rank) + a * VLayout<DV>::kBoxCols,
+                        sl.second * kKeys, b, pol_kv);
+        } else if (sl.second >= 0) {
           load_k(dst + kPartBytes, sl.second);
+        }
       }
       ++kv;
       return true;
@@ -361,7 +398,7 @@ __device__ __forceinline__ void relay(Barriers *bars, const Params &p,
 // MMA warp of the even CTA, lane 0: tcgen05.mma issuer for the pair.
 // kPvDone: also signal pv_done after every PV but the segment's last (the
 // running-max modes rescale O and must know when the previous PV finished).
-template <bool kPvDone>
+template <bool kPvDone, int DV>
 __device__ __forceinline__ void mma_issuer(uint8_t *q_s, uint8_t *kv_s,
                                            Barriers *bars, uint32_t tmem,
                                            const Params &p, volatile int *abort) {
@@ -395,7 +432,7 @@ __device__ __forceinline__ void mma_issuer(uint8_t *q_s, uint8_t *kv_s,
     if (!ok) break;
     tc_fence_after();
     {
-      const uint32_t base = kv_addr + slot * kSlotBytes;
+      const uint32_t base = kv_addr + slot * slot_bytes<DV>();
       for (int u = 0; u < 2 && u < n; ++u) {
         issue_qk(tmem + 128u * u, q_addr, base + u * kPartBytes);
         umma2_commit_both(&bars->s_full[u]);
@@ -416,8 +453,8 @@ __device__ __forceinline__ void mma_issuer(uint8_t *q_s, uint8_t *kv_s,
       pbits ^= 1u << u;
       if (!ok) break;
       tc_fence_after();
-      const uint32_t base = kv_addr + slot * kSlotBytes + (i & 1) * kStepBytes;
-      issue_pv(tmem + kColO, tmem + 128u * u, base + kPartBytes, j > sg.kb);
+      const uint32_t base = kv_addr + slot * slot_bytes<DV>() + (i & 1) * step_bytes<DV>();
+      issue_pv<DV>(tmem + kColO, tmem + 128u * u, base + kPartBytes, j > sg.kb);
       if (j + 1 == sg.ke)
         umma2_commit_both(&bars->o_full);
       else if (kPvDone)
@@ -534,9 +571,9 @@ __device__ __forceinline__ float tile_static(uint32_t tS, int col0, float b0,
 
 // One key tile with a running maximum shared by the four threads of each row
 // (exchanged through shared memory).  When the maximum grows past the lazy
-// threshold, this warpgroup's 32 columns of O are rescaled, after the
+// threshold, this warpgroup's DV/4 columns of O are rescaled, after the
 // previous PV into O has finished (pv_done).
-template <int MODE>
+template <int MODE, int DV>
 __device__ __forceinline__ bool tile_online(uint32_t tS, uint32_t tO, int g,
                                             int r, uint32_t par, bool o_live,
                                             uint32_t pv_parity, float b0,
@@ -578,6 +615,15 @@ __device__ __forceinline__ bool tile_online(uint32_t tS, uint32_t tO, int g,
     for (int e = 0; e < 32; ++e)
       o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
     tmem_st32(tO, o);
+    if constexpr (DV == 192) {  // columns 32 .. 47 of this warpgroup's 48
+      uint32_t o2[16];
+      tmem_ld16(tO + 32, o2);
+      tmem_wait_ld16(o2);
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        o2[e] = __float_as_uint(__uint_as_float(o2[e]) * factor);
+      tmem_st16(tO + 32, o2);
+    }
   }
   float acc = 0.f;
   uint32_t pk[16];
@@ -662,7 +708,7 @@ __device__ __forceinline__ bool segment_static(const Segment &sg, const float *b
 
 // Running-max modes: every warpgroup takes every key tile (32 keys each),
 // the four threads of a row sharing its maximum per tile.
-template <int MODE>
+template <int MODE, int DV>
 __device__ __forceinline__ bool segment_online(const Segment &sg, const float *brow,
                                                uint32_t tmem, uint32_t lane_base,
                                                int g, int r, const Params &p,
@@ -684,12 +730,12 @@ __device__ __forceinline__ bool segment_online(const Segment &sg, const float *b
     if (!__all_sync(0xffffffffu, ok)) return false;
     tc_fence_after();
     const uint32_t tS = tmem + 128u * u + 32 * g + lane_base;
-    const uint32_t tO = tmem + kColO + 32 * g + lane_base;
+    const uint32_t tO = tmem + kColO + (DV / 4) * g + lane_base;
     // PV(j-1) is pv_done phase pvd + (j - 1 - kb); PV(j-2) has finished
     // (s_full(j) was committed after it), so that phase is the current or
     // the last completed one and its parity identifies it.
     const uint32_t pv_parity = (pvd + static_cast<uint32_t>(j - 1 - sg.kb)) & 1u;
-    if (!tile_online<MODE>(tS, tO, g, r, u, j > sg.kb, pv_parity, b0, b1, p, nvalid,
+    if (!tile_online<MODE, DV>(tS, tO, g, r, u, j > sg.kb, pv_parity, b0, b1, p, nvalid,
                            xc, bars, xmcount, abort, m, d))
       return false;
     tmem_wait_st();
@@ -708,7 +754,7 @@ __device__ __forceinline__ bool segment_online(const Segment &sg, const float *b
   return true;
 }
 
-template <int MODE>
+template <int MODE, int DV>
 __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc,
                                              uint32_t tmem, const Params &p,
                                              uint32_t rank, volatile int *abort) {
@@ -742,7 +788,7 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc,
       ok = segment_static(sg, brow, tmem, lane_base, g, p, bars, rank,
                           (g >> 1) ? pf_remote1 : pf_remote0, scount0, abort, d);
     } else {
-      ok = segment_online<MODE>(sg, brow, tmem, lane_base, g, r, p, bars, xc, rank,
+      ok = segment_online<MODE, DV>(sg, brow, tmem, lane_base, g, r, p, bars, xc, rank,
                                 pf_remote0, pf_remote1, scount0, scount1, xmcount,
                                 pvd, abort, m, d);
     }
@@ -750,10 +796,10 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc,
     pvd += static_cast<uint32_t>(sg.ke - sg.kb - 1);
 
     // Epilogue: d = sum of the four warpgroups' partial sums; out = O / d
-    // over this segment's keys (warpgroup g writes columns [32g, 32g + 32)
-    // of the row) and lse, to out / lse or, for a later piece of a split
-    // pair, to this cluster's scratch slot.  The copy of block I0 in an odd
-    // CTA past the end of an odd block count writes nothing.
+    // over this segment's keys (warpgroup g writes columns [g DV/4, (g+1)
+    // DV/4) of the row) and lse, to out / lse or, for a later piece of a
+    // split pair, to this cluster's scratch slot.  The copy of block I0 in an
+    // odd CTA past the end of an odd block count writes nothing.
     ok = mbar_wait(&bars->o_full, ocount & 1u, abort, p.err, kSiteSoftO);
     ++ocount;
     if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
@@ -765,30 +811,45 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc,
 #pragma unroll
     for (int q = 0; q < kWG; ++q) dsum += xc->dpart[q][r];
     const float inv_d = 1.f / dsum;
+    const uint32_t tO = tmem + kColO + (DV / 4) * g + lane_base;
     uint32_t o[32];
-    tmem_ld32(tmem + kColO + 32 * g + lane_base, o);
+    tmem_ld32(tO, o);
     tmem_wait_ld(o);
+    uint32_t o2[16];  // columns 32 .. 47 of this warpgroup's 48 (DV = 192)
+    if constexpr (DV == 192) {
+      tmem_ld16(tO + 32, o2);
+      tmem_wait_ld16(o2);
+    }
     if (valid && pos < p.L) {  // rows past the end of a partial block: none
       const size_t row = (static_cast<size_t>(b) * kH + h) * p.L +
                          static_cast<size_t>(pos);
       float *orow_base;
       float *lse_dst;
       if (sg.kb == 0) {
-        orow_base = p.out + row * kD;
+        orow_base = p.out + row * DV;
         lse_dst = p.lse + row;
       } else {
         const size_t slot =
             (static_cast<size_t>(cluster_index()) * 2 + rank) * 128 + r;
-        orow_base = p.ws_out + slot * kD;
+        orow_base = p.ws_out + slot * DV;
         lse_dst = p.ws_lse + slot;
       }
-      float4 *orow = reinterpret_cast<float4 *>(orow_base + 32 * g);
+      float4 *orow = reinterpret_cast<float4 *>(orow_base + (DV / 4) * g);
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         orow[e] = make_float4(__uint_as_float(o[4 * e]) * inv_d,
                               __uint_as_float(o[4 * e + 1]) * inv_d,
                               __uint_as_float(o[4 * e + 2]) * inv_d,
                               __uint_as_float(o[4 * e + 3]) * inv_d);
+      }
+      if constexpr (DV == 192) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          orow[8 + e] = make_float4(__uint_as_float(o2[4 * e]) * inv_d,
+                                    __uint_as_float(o2[4 * e + 1]) * inv_d,
+                                    __uint_as_float(o2[4 * e + 2]) * inv_d,
+                                    __uint_as_float(o2[4 * e + 3]) * inv_d);
+        }
       }
       if (g == 0) *lse_dst = (m + lg2_approx(dsum)) * kLn2;
     }
@@ -797,7 +858,7 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc,
 }
 
 // --------------------------------------------------------------------------
-template <int MODE>
+template <int MODE, int DV>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
@@ -806,7 +867,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t *q_s = smem_raw + pad;             // this CTA's query tile
   uint8_t *kv_s = q_s + kQTileBytes;         // K/V ring
-  Barriers *bars = reinterpret_cast<Barriers *>(kv_s + kStages * kSlotBytes);
+  Barriers *bars = reinterpret_cast<Barriers *>(kv_s + kStages * slot_bytes<DV>());
   auto *xc = reinterpret_cast<Xchg *>(reinterpret_cast<uint8_t *>(bars) +
                                       sizeof(Barriers));
   const int warp = threadIdx.x >> 5;
@@ -855,15 +916,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (warp >= kWarpLoad) {
     regs_dec<kRegsLow>();
     if (warp == kWarpLoad && lane_id() == 0) {
-      producer(&tm_q, &tm_k, &tm_v, q_s, kv_s, bars, p, rank, abort);
+      producer<DV>(&tm_q, &tm_k, &tm_v, q_s, kv_s, bars, p, rank, abort);
     } else if (warp == kWarpMma && lane_id() == 0) {
       if (rank == 0)
-        mma_issuer<MODE != kStaticCap>(q_s, kv_s, bars, tmem, p, abort);
+        mma_issuer<MODE != kStaticCap, DV>(q_s, kv_s, bars, tmem, p, abort);
       else
         relay(bars, p, abort);
     }
   } else {
-    softmax_role<MODE>(bars, xc, tmem, p, rank, abort);
+    softmax_role<MODE, DV>(bars, xc, tmem, p, rank, abort);
   }
   __syncwarp();
   // No CTA leaves while the other may still use its shared or tensor memory:
@@ -880,13 +941,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 // --------------------------------------------------------------------------
 // Split-pair merge.  kMergeBlocksPerBoundary blocks per cluster boundary; only
 // the boundary that is the first one inside a pair merges that pair.  One
-// warp per output row (query tile row / 128, row % 128): lane l merges
-// columns [4l, 4l + 4) over the pieces, and lane 0 writes the merged lse
-// once every lane has read the first piece's.
+// warp per output row (query tile row / 128, row % 128): lane l merges the
+// 4-column groups l, l + 32, ... of the row's DV columns over the pieces, and
+// lane 0 writes the merged lse once every lane has read the first piece's.
 constexpr int kMergeThreads = 256;
 constexpr int kMergeRowsPerBlock = kMergeThreads / 32;
 constexpr int kMergeBlocksPerBoundary = 2 * 128 / kMergeRowsPerBlock;
 
+template <int DV>
 __global__ void __launch_bounds__(kMergeThreads)
     attn_merge_kernel(const Params p, int grid) {
   const int c = blockIdx.x / kMergeBlocksPerBoundary + 1;  // boundary between clusters c-1, c
@@ -927,18 +989,21 @@ __global__ void __launch_bounds__(kMergeThreads)
   for (int s = 0; s < n_seg; ++s)
     sum += ex2_approx(((s == 0 ? p.lse[row] : p.ws_lse[slot(s)]) - M) * kLog2e);
   const float lse = M + lg2_approx(sum) * kLn2;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = 0; s < n_seg; ++s) {
-    const float l = s == 0 ? p.lse[row] : p.ws_lse[slot(s)];
-    const float wgt = ex2_approx((l - lse) * kLog2e);
-    const float4 v = reinterpret_cast<const float4 *>(
-        s == 0 ? p.out + row * kD : p.ws_out + slot(s) * kD)[lane];
-    acc.x = fmaf(wgt, v.x, acc.x);
-    acc.y = fmaf(wgt, v.y, acc.y);
-    acc.z = fmaf(wgt, v.z, acc.z);
-    acc.w = fmaf(wgt, v.w, acc.w);
+#pragma unroll
+  for (int c = lane; c < DV / 4; c += 32) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < n_seg; ++s) {
+      const float l = s == 0 ? p.lse[row] : p.ws_lse[slot(s)];
+      const float wgt = ex2_approx((l - lse) * kLog2e);
+      const float4 v = reinterpret_cast<const float4 *>(
+          s == 0 ? p.out + row * DV : p.ws_out + slot(s) * DV)[c];
+      acc.x = fmaf(wgt, v.x, acc.x);
+      acc.y = fmaf(wgt, v.y, acc.y);
+      acc.z = fmaf(wgt, v.z, acc.z);
+      acc.w = fmaf(wgt, v.w, acc.w);
+    }
+    reinterpret_cast<float4 *>(p.out + row * DV)[c] = acc;
   }
-  reinterpret_cast<float4 *>(p.out + row * kD)[lane] = acc;
   __syncwarp();  // every lane has read p.lse[row]
   if (lane == 0) p.lse[row] = lse;
 }
@@ -950,19 +1015,20 @@ __global__ void __launch_bounds__(kMergeThreads)
 
 static bool encode_map(EncodeTiledFn enc, CUtensorMap *map, const void *base,
                        int rank, const cuuint64_t *dims,
-                       const cuuint64_t *strides, const cuuint32_t *box) {
+                       const cuuint64_t *strides, const cuuint32_t *box,
+                       CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank,
                    const_cast<void *>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
-// One-time per-device setup of a mode's kernel: shared-memory opt-in, the
-// register check, and how many 2-CTA clusters can be resident at once.
-template <int MODE>
+// One-time per-device setup of a kernel (mode, value width): shared-memory
+// opt-in, the register check, and how many 2-CTA clusters can be resident.
+template <int MODE, int DV>
 static cudaError_t configure_mode(int *max_clusters) {
   static int configured[64] = {0};
   static int clusters[64] = {0};
@@ -971,23 +1037,23 @@ static cudaError_t configure_mode(int *max_clusters) {
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!configured[dev]) {
-    // setmaxnreg.inc waits until the registers it asks for are free: refuse
-    // to launch a build whose launch allocation cannot cover the split.
+    // setmaxnreg.dec must lower the count the launch allocated: refuse a
+    // build whose allocation is below the launch count the split assumes.
     cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, attn::attn_fwd_kernel<MODE>);
+    e = cudaFuncGetAttributes(&fa, attn::attn_fwd_kernel<MODE, DV>);
     if (e != cudaSuccess) return e;
     if (static_cast<uint32_t>(fa.numRegs) < attn::kRegsLaunch)
       return cudaErrorInvalidConfiguration;
-    e = cudaFuncSetAttribute(attn::attn_fwd_kernel<MODE>,
+    e = cudaFuncSetAttribute(attn::attn_fwd_kernel<MODE, DV>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(attn::kSmemBytes));
+                             static_cast<int>(attn::smem_bytes<DV>()));
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2, 1, 1);
     cfg.blockDim = dim3(attn::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = attn::kSmemBytes;
+    cfg.dynamicSmemBytes = attn::smem_bytes<DV>();
     int n = 0;
-    e = cudaOccupancyMaxActiveClusters(&n, attn::attn_fwd_kernel<MODE>, &cfg);
+    e = cudaOccupancyMaxActiveClusters(&n, attn::attn_fwd_kernel<MODE, DV>, &cfg);
     if (e != cudaSuccess) return e;
     if (n < 1) return cudaErrorInvalidConfiguration;
     clusters[dev] = n;
@@ -997,13 +1063,23 @@ static cudaError_t configure_mode(int *max_clusters) {
   return cudaSuccess;
 }
 
-template <int MODE>
+template <int MODE, int DV>
 static cudaError_t launch_mode(const CUtensorMap &tq, const CUtensorMap &tk,
                                const CUtensorMap &tv, const attn::Params &p,
                                int clusters, cudaStream_t stream) {
-  attn::attn_fwd_kernel<MODE>
-      <<<2 * clusters, attn::kThreads, attn::kSmemBytes, stream>>>(tq, tk, tv, p);
+  attn::attn_fwd_kernel<MODE, DV>
+      <<<2 * clusters, attn::kThreads, attn::smem_bytes<DV>(), stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
+}
+
+template <int DV>
+static cudaError_t configure_any(int mode, int *max_clusters) {
+  using namespace attn;
+  switch (mode) {
+    case kStaticCap: return configure_mode<kStaticCap, DV>(max_clusters);
+    case kOnlineCap: return configure_mode<kOnlineCap, DV>(max_clusters);
+    default: return configure_mode<kNoCap, DV>(max_clusters);
+  }
 }
 
 // Grid of a call: one 2-CTA cluster per resident SM pair, never more
@@ -1011,16 +1087,11 @@ static cudaError_t launch_mode(const CUtensorMap &tq, const CUtensorMap &tk,
 // cluster unless that leaves the grid badly balanced: a split pair costs a
 // second pass over its rows (partial results, then the merge), so whole pairs
 // win while the busiest cluster's extra work stays below kSplitGain pairs.
-static cudaError_t plan_grid(int mode, int n_items, int n_kt, int num_sms,
+static cudaError_t plan_grid(int mode, int dv, int n_items, int n_kt, int num_sms,
                              int scratch_slots, int *clusters_out, int *whole_out) {
-  using namespace attn;
   int max_clusters = 0;
-  cudaError_t e;
-  switch (mode) {
-    case kStaticCap: e = configure_mode<kStaticCap>(&max_clusters); break;
-    case kOnlineCap: e = configure_mode<kOnlineCap>(&max_clusters); break;
-    default: e = configure_mode<kNoCap>(&max_clusters); break;
-  }
+  cudaError_t e = dv == 192 ? configure_any<192>(mode, &max_clusters)
+                            : configure_any<128>(mode, &max_clusters);
   if (e != cudaSuccess) return e;
   const long long steps = static_cast<long long>(n_items) * n_kt;
   if (steps > (1ll << 30)) return cudaErrorInvalidValue;
@@ -1045,8 +1116,8 @@ static int attn_mode(float cap) {
   return cap <= 40.0f ? kStaticCap : kOnlineCap;
 }
 
-cudaError_t attn_fwd_kernel_count(int64_t B, int64_t L, float cap, int num_sms,
-                                  int scratch_slots, int *count) {
+cudaError_t attn_fwd_kernel_count(int64_t B, int64_t L, int64_t Dv, float cap,
+                                  int num_sms, int scratch_slots, int *count) {
   using namespace attn;
   if (B == 0 || L == 0) {
     *count = 0;
@@ -1056,8 +1127,8 @@ cudaError_t attn_fwd_kernel_count(int64_t B, int64_t L, float cap, int num_sms,
   const int n_items = static_cast<int>(B) * ((nb + 1) / 2);
   const int n_kt = static_cast<int>((L + kKeys - 1) / kKeys);
   int clusters = 0, whole = 0;
-  cudaError_t e = plan_grid(attn_mode(cap), n_items, n_kt, num_sms, scratch_slots,
-                            &clusters, &whole);
+  cudaError_t e = plan_grid(attn_mode(cap), static_cast<int>(Dv), n_items, n_kt,
+                            num_sms, scratch_slots, &clusters, &whole);
   if (e != cudaSuccess) return e;
   *count = (clusters < 2 || whole) ? 1 : 2;
   return cudaSuccess;
@@ -1081,10 +1152,19 @@ cudaError_t launch_attn_fwd(const AttnLaunch &a) {
                                 static_cast<cuuint64_t>(B)};
     const cuuint64_t strides[2] = {kD * 2, static_cast<cuuint64_t>(L) * kD * 2};
     const cuuint32_t kbox[3] = {64, kKeys / 2, 1};  // a CTA's 64 keys, one 64-wide half
-    const cuuint32_t vbox[3] = {64, kKeys, 1};      // a CTA's 64 value columns, 128 keys
     if (!encode_map(a.encode, &tk, a.k, 3, dims, strides, kbox))
       return cudaErrorInvalidValue;
-    if (!encode_map(a.encode, &tv, a.v, 3, dims, strides, vbox))
+    // V [B, L, Dv]: a box is one swizzle atom column of a CTA's value half.
+    const cuuint64_t vdims[3] = {static_cast<cuuint64_t>(a.Dv),
+                                 static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(B)};
+    const cuuint64_t vstrides[2] = {static_cast<cuuint64_t>(a.Dv) * 2,
+                                    static_cast<cuuint64_t>(L) * a.Dv * 2};
+    const bool dv192 = a.Dv == 192;
+    const cuuint32_t vbox[3] = {
+        static_cast<cuuint32_t>(dv192 ? VLayout<192>::kBoxCols : VLayout<128>::kBoxCols),
+        kKeys, 1};
+    if (!encode_map(a.encode, &tv, a.v, 3, vdims, vstrides, vbox,
+                    dv192 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   }
   Params p;
@@ -1112,8 +1192,10 @@ cudaError_t launch_attn_fwd(const AttnLaunch &a) {
     p.bias_mul = 1.0f / cap;
     p.A = cap * kLog2e;
   }
+  if (a.Dv != 128 && a.Dv != 192) return cudaErrorInvalidValue;
+  const int dv = static_cast<int>(a.Dv);
   int clusters = 0;
-  cudaError_t e = plan_grid(mode, p.n_items, p.n_kt, a.num_sms, a.scratch_slots,
+  cudaError_t e = plan_grid(mode, dv, p.n_items, p.n_kt, a.num_sms, a.scratch_slots,
                             &clusters, &p.whole);
   if (e != cudaSuccess) return e;
   if (static_cast<long long>(p.n_items) * p.n_kt != attn_work_steps(B, L))
@@ -1121,14 +1203,25 @@ cudaError_t launch_attn_fwd(const AttnLaunch &a) {
   char *base = static_cast<char *>(a.scratch);
   p.ws_out = reinterpret_cast<float *>(base);
   p.ws_lse = reinterpret_cast<float *>(base + a.scratch_slots * kAttnSlotOutBytes);
-  switch (mode) {
-    case kStaticCap: e = launch_mode<kStaticCap>(tq, tk, tv, p, clusters, a.stream); break;
-    case kOnlineCap: e = launch_mode<kOnlineCap>(tq, tk, tv, p, clusters, a.stream); break;
-    default: e = launch_mode<kNoCap>(tq, tk, tv, p, clusters, a.stream); break;
+  if (dv == 192) {
+    switch (mode) {
+      case kStaticCap: e = launch_mode<kStaticCap, 192>(tq, tk, tv, p, clusters, a.stream); break;
+      case kOnlineCap: e = launch_mode<kOnlineCap, 192>(tq, tk, tv, p, clusters, a.stream); break;
+      default: e = launch_mode<kNoCap, 192>(tq, tk, tv, p, clusters, a.stream); break;
+    }
+  } else {
+    switch (mode) {
+      case kStaticCap: e = launch_mode<kStaticCap, 128>(tq, tk, tv, p, clusters, a.stream); break;
+      case kOnlineCap: e = launch_mode<kOnlineCap, 128>(tq, tk, tv, p, clusters, a.stream); break;
+      default: e = launch_mode<kNoCap, 128>(tq, tk, tv, p, clusters, a.stream); break;
+    }
   }
   if (e != cudaSuccess || clusters < 2 || p.whole) return e;
-  attn_merge_kernel<<<(clusters - 1) * kMergeBlocksPerBoundary, kMergeThreads, 0,
-                      a.stream>>>(p, clusters);
+  const int merge_blocks = (clusters - 1) * kMergeBlocksPerBoundary;
+  if (dv == 192)
+    attn_merge_kernel<192><<<merge_blocks, kMergeThreads, 0, a.stream>>>(p, clusters);
+  else
+    attn_merge_kernel<128><<<merge_blocks, kMergeThreads, 0, a.stream>>>(p, clusters);
   return cudaGetLastError();
 }
 

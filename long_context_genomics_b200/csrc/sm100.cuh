@@ -251,6 +251,10 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr,
 __host__ __device__ constexpr uint32_t desc_sw128_hi(uint32_t sbo) {
   return ((sbo >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
 }
+// The same for a 64-byte-swizzled operand (swizzle mode 4).
+__host__ __device__ constexpr uint32_t desc_sw64_hi(uint32_t sbo) {
+  return ((sbo >> 4) & 0x3FFFu) | (1u << 14) | (4u << 29);
+}
 __device__ __forceinline__ uint32_t desc_sw128_lo(uint32_t saddr, uint32_t lbo) {
   return ((saddr >> 4) & 0x3FFFu) | (((lbo >> 4) & 0x3FFFu) << 16);
 }
@@ -403,6 +407,20 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 __device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;"
                : AG_P8(r, 0), AG_P8(r, 8), AG_P8(r, 16), AG_P8(r, 24)
+               :
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : AG_R8(r, 0), AG_R8(r, 8)
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld16(uint32_t (&r)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : AG_P8(r, 0), AG_P8(r, 8)
                :
                : "memory");
 }

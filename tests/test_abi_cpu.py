@@ -100,6 +100,17 @@ def test_strided_bias_validation(ag):
     assert _attn_strided(ag, 10 * 8 * P * P, bias=A16 * 1000 - span + 16) == 7
 
 
+def test_value_width_validation(ag):
+    f = ag.lib.ag_attn_fwd_ex
+    args = lambda Dv, **kw: (kw.get("q", A16), A16 * 2, A16 * 3, A16 * 4, 0, 1, 8, 256,
+                             128, Dv, 16, 5.0, A16 * 1000, A16 * 2000, None)
+    assert f(*args(0)) == 2          # AG_ERR_SHAPE
+    assert f(*args(64)) == 4         # AG_ERR_UNSUPPORTED
+    assert f(*args(160)) == 4
+    assert f(*args(192, q=None)) == 1  # supported width: on to the NULL check
+    assert f(*args(128, q=None)) == 1
+
+
 def test_attn_empty_is_a_noop(ag):
     assert _attn(ag, B=0, q=None, k=None, v=None, bias=None, out=None, lse=None) == 0
     assert _attn(ag, L=0, q=None, k=None, v=None, bias=None, out=None, lse=None) == 0

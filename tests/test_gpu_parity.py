@@ -168,6 +168,33 @@ def test_one_bias_per_batch_item(ag, oracle_lib, B, L, cap):
         _compare(out[b, h, i], lse[b, h, i], ro, rl, f"per-item bias B={B} L={L} sampled")
 
 
+@pytest.mark.parametrize("B,L", [(1, 512), (2, 1040), (1, 2049)])
+@pytest.mark.parametrize("cap", [5.0, 50.0, math.inf])
+def test_value_width_192(ag, oracle_lib, B, L, cap):
+    """Dv = 192 (the page's checkpoint value width) through ag_attn_fwd_ex:
+    v [B,L,192], out [B,H,L,192], scale still 1/sqrt(128)."""
+    inp = ag_inputs.random_case(B, 8, L, 128, 192, 16, seed=B * 97 + L)
+    out, lse = _gpu_attn(ag, inp, cap)
+    assert out.shape == (B, 8, L, 192)
+    ro, rl = oracle_lib.attn_fwd(inp["q"], inp["k"], inp["v"], inp["bias"],
+                                 block=16, cap=cap)
+    _compare(out, lse, ro, rl, f"Dv=192 B={B} L={L} cap={cap}")
+
+
+def test_value_width_192_full_context_sampled(ag, oracle_lib):
+    """Dv = 192 at L = 8192 with one bias per batch item (B = 2): split pairs
+    and the merge run; sampled rows against the oracle."""
+    B, L = 2, 8192
+    inp = ag_inputs.random_case(B, 8, L, 128, 192, 16, seed=192, batched_bias=True)
+    out, lse = _gpu_attn(ag, inp, 5.0)
+    rows = ag_inputs.sample_rows(B, 8, L, 512, seed=19).numpy()
+    ro, rl = oracle_lib.attn_rows(inp["q"], inp["k"], inp["v"], inp["bias"], rows,
+                                  block=16, cap=5.0)
+    b, h, i = rows[:, 0], rows[:, 1], rows[:, 2]
+    _compare(out[b, h, i], lse[b, h, i], ro, rl, "Dv=192 L=8192 sampled")
+    assert np.isfinite(out).all() and np.isfinite(lse).all()
+
+
 def test_strided_bias_with_padding_between_items(ag, oracle_lib):
     """A bias batch stride larger than H*P*P (padded items) through the C ABI."""
     import ctypes
