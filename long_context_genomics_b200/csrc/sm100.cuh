@@ -148,75 +148,20 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
 
 // ---------------------------------------------------------------------------
 // tcgen05: tensor memory and the 5th-generation tensor core.
-// Per-warpgroup register re-allocation (every warp of the warpgroup executes
-// the same instruction).  The increases must fit in what the decreases free
-// from the block's launch allocation, or the increasing warps wait forever.
+// Per-warpgroup register release (every warp of the warpgroup executes the
+// same instruction): lowers the warpgroup's register count below the launch
+// allocation.  (The matching increase is not used: an increase that the
+// decreases cannot cover waits forever.)
 template <uint32_t kRegs>
 __device__ __forceinline__ void regs_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
 }
-template <uint32_t kRegs>
-__device__ __forceinline__ void regs_inc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
-}
 
-__device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {
-  asm volatile(
-      "tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-          smem_u32(dst_smem)),
-      "r"(ncols)
-      : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::
-                   : "memory");
-}
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(
-                   taddr),
-               "r"(ncols)
-               : "memory");
-}
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-// D[tmem] (+)= A[smem] * B[smem]^T, kind::f16 (bf16 in, fp32 accumulate).
-__device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc,
-                                        uint64_t b_desc, uint32_t idesc,
-                                        uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(
-          d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// D[tmem] (+)= A[tmem] * B[smem]^T, kind::f16.
-__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem,
-                                        uint64_t b_desc, uint32_t idesc,
-                                        uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(
-          d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Arrive (once) on `bar` when every tcgen05 operation this thread issued so
-// far has completed.
-__device__ __forceinline__ void umma_commit(uint64_t *bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 "
-      "[%0];" ::"r"(smem_u32(bar))
-      : "memory");
 }
 
 // Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B,
@@ -231,21 +176,8 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N,
          | ((M >> 4) << 24);      // M / 16
 }
 
-// Shared-memory matrix descriptor for a 128-byte-swizzled operand.
-//   lbo: leading-dimension byte offset, sbo: stride-dimension byte offset.
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr,
-                                                    uint32_t lbo,
-                                                    uint32_t sbo) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
-  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
-  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
-  d |= 1ull << 46;  // descriptor version for sm_100
-  d |= 2ull << 61;  // 128-byte swizzle
-  return d;
-}
-
-// Split form of smem_desc_sw128 for operands whose upper word is shared:
+// Shared-memory matrix descriptor of a 128-byte-swizzled operand, split for
+// operands whose upper word is shared:
 // the low word holds the start address and the leading-dimension offset, the
 // high word the stride offset, version and swizzle mode.
 __host__ __device__ constexpr uint32_t desc_sw128_hi(uint32_t sbo) {
@@ -257,32 +189,6 @@ __host__ __device__ constexpr uint32_t desc_sw64_hi(uint32_t sbo) {
 }
 __device__ __forceinline__ uint32_t desc_sw128_lo(uint32_t saddr, uint32_t lbo) {
   return ((saddr >> 4) & 0x3FFFu) | (((lbo >> 4) & 0x3FFFu) << 16);
-}
-
-// As umma_ss / umma_ts, with each shared-memory descriptor given as its low
-// word plus one shared high word.
-__device__ __forceinline__ void umma_ss_lo(uint32_t d_tmem, uint32_t a_lo,
-                                           uint32_t b_lo, uint32_t hi,
-                                           uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
-      "mov.b64 da, {%1, %3};\n\t"
-      "mov.b64 db, {%2, %3};\n\t"
-      "setp.ne.b32 p, %5, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_lo), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void umma_ts_lo(uint32_t d_tmem, uint32_t a_tmem,
-                                           uint32_t b_lo, uint32_t hi,
-                                           uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
-      "mov.b64 db, {%2, %3};\n\t"
-      "setp.ne.b32 p, %5, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)
-      : "memory");
 }
 
 // ---------------------------------------------------------------------------
