@@ -15,20 +15,21 @@
 //  * Two SMs work as a pair (a 2-CTA cluster) on a pair of query tiles: each
 //    CTA holds one tile, and one thread of the even CTA issues tcgen05.mma
 //    with cta_group::2, M = 256 rows over both SMs.  Each CTA stages only half
-//    of every K tile (64 of its 128 keys) and half of every V tile (64 of the
-//    128 value columns), so a K/V byte loaded from L2 feeds 16 query rows per
-//    SM pair position, and one MMA instruction keeps both tensor cores busy.
+//    of every K tile (64 of its 128 keys) and half of every V tile (DV/2 of
+//    the DV value columns), so each K/V byte crosses from L2 into one SM only
+//    and serves the 256 query rows of the pair, and one MMA instruction keeps
+//    both tensor cores busy.  DV (value width) is 128 or 192.
 //  * One persistent cluster per SM pair takes a contiguous, equal share of all
 //    (pair, key tile) steps; a pair whose key range is split between clusters
 //    is merged exactly from the pieces' partial results by log-sum-exp (see
 //    "Split pairs" below).
 //  * Inside each CTA: a producer warp streams its Q tile and a ring of K and V
-//    halves with TMA (no multicast); four softmax warpgroups each own one
-//    32-key chunk of every key tile.  In the odd CTA the MMA warp relays
+//    halves with TMA (no multicast); the softmax warpgroups own 32- or 64-key
+//    chunks of the key tiles (see "Softmax warpgroups").  In the odd CTA the MMA warp relays
 //    "loaded" to the even CTA (a cluster-scope arrive), so each CTA's copies
 //    complete on its own barriers and can be drained locally.
 //  * Tensor memory (per CTA): two 128-column S buffers (fp32 logits of
-//    alternate key tiles) and the 128-column O accumulator.  P is written as
+//    alternate key tiles) and the DV-column O accumulator.  P is written as
 //    bf16 over part of its S buffer and fed to the PV product straight from
 //    tensor memory.  With S double-buffered the MMA order per key tile is
 //    PV(j), S(j+2): the logits a softmax warp needs next were computed while
@@ -56,8 +57,8 @@ static_assert(kKeys == 128, "the tile layout below assumes 128-key tiles");
 constexpr int kQTileBytes = 128 * kD * 2;     // this CTA's query tile (bf16)
 constexpr int kQHalfBytes = kQTileBytes / 2;  // one 64-wide (128-byte) half
 // A step load is what one key-tile step needs from this CTA: its half of a
-// V tile (128 keys x 64 value columns, 16 KB) and its half of the K tile two
-// steps ahead (64 keys x 128, two 64-wide halves of 8 KB), or, first in a
+// V tile (128 keys x DV/2 value columns; VLayout below) and its half of the K
+// tile two steps ahead (64 keys x 128, two 64-wide halves of 8 KB), or, first in a
 // segment, the halves of the segment's first two K tiles.  A ring slot holds
 // two consecutive step loads, so the MMA thread waits for data and releases
 // it once per two steps (each mbarrier operation costs it about 180 cycles
@@ -109,9 +110,9 @@ constexpr uint32_t kRegsLow = 88;
 static_assert(kSoftThreads * kRegsLaunch + 128 * kRegsLow <= kThreads * kRegsLaunch,
               "register split exceeds the launch allocation");
 constexpr uint32_t kTmemCols = 512;
-// Tensor-memory columns: S buffer u at 128 u, O at 256 (DV columns).  P (bf16 pairs) of
-// chunk c (keys [32c, 32c + 32) of the tile) is written over the first 16
-// columns of that chunk's own S columns, [32c, 32c + 16).
+// Tensor-memory columns: S buffer u at 128 u, O at 256 (DV columns).  P (bf16
+// pairs) of chunk c (keys [32c, 32c + 32) of the tile) is written over the
+// first 16 columns of that chunk's own S columns, [32c, 32c + 16).
 constexpr uint32_t kColO = 256;
 constexpr uint32_t kIdescQK = idesc_bf16_f32(256, kKeys, 0);  // K-major B (K)
 template <int DV> constexpr uint32_t idesc_pv() { return idesc_bf16_f32(256, DV, 1); }
@@ -479,12 +480,14 @@ __device__ __forceinline__ void mma_issuer(uint8_t *q_s, uint8_t *kv_s,
 // --------------------------------------------------------------------------
 // Softmax warpgroups (each CTA, its own query tile).
 //
-// Warpgroup g owns keys [32g, 32g + 32) of every 128-key tile, for all 128
-// rows (thread r of the warpgroup owns tensor-memory lane r).  A row's sum is
-// split between its four threads and combined through shared memory once per
-// work item (and, in the running-max modes, its maximum once per key tile).
-// Each chunk's P goes over the first 16 of its own S columns, so a
-// warpgroup only ever overwrites S columns it has already read itself.
+// Thread r of a warpgroup owns tensor-memory lane r, i.e. row r of the tile.
+// Static-cap mode: warpgroups 2q and 2q+1 take the key tiles in S buffer q,
+// 64 keys each.  Running-max modes: warpgroup g takes keys [32g, 32g + 32) of
+// every key tile.  Either way a row's sum is split between four threads and
+// combined through shared memory once per work item (and, in the running-max
+// modes, its maximum once per key tile).  Each 32-key chunk's P goes over
+// the first 16 of its own S columns, so a warpgroup only ever overwrites S
+// columns it has already read itself.
 
 // Softmax-side barriers count warps: each warp arrives once, from lane 0,
 // after __syncwarp has ordered its lanes' prior work (one arrival per warp
