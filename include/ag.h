@@ -131,7 +131,8 @@ ag_status ag_attn_fwd(const void *q, const void *k, const void *v,
  * bias + b * bias_batch_stride, a [H, P, P] float32 block (P = ceil(L /
  * block)); bias_batch_stride is in floats, 0 (one bias shared by every item:
  * exactly ag_attn_fwd) or at least H * P * P (e.g. H * P * P for a dense
- * [B, H, P, P] tensor); anything else returns AG_ERR_SHAPE.  Everything else
+ * [B, H, P, P] tensor); anything else returns AG_ERR_SHAPE, as does a span
+ * (B - 1) * bias_batch_stride + H * P * P above 2^56 floats.  Everything else
  * -- arguments, checks, results, scratch, stream behaviour -- as ag_attn_fwd.
  */
 ag_status ag_attn_fwd_strided_bias(const void *q, const void *k, const void *v,

@@ -244,6 +244,11 @@ ag_status ag_attn_fwd_ex(const void *q, const void *k, const void *v,
   const int64_t P = block > 0 ? (L + block - 1) / block : 0;
   if (bias_batch_stride < 0 || (bias_batch_stride > 0 && bias_batch_stride < H * P * P))
     return AG_ERR_SHAPE;
+  // The items' bias span, (B - 1) * stride + H * P * P floats, must stay far
+  // below 2^63 bytes so that the alias check and the kernel's offsets are exact.
+  constexpr int64_t kMaxBiasSpan = int64_t(1) << 56;
+  if (B > 1 && bias_batch_stride > (kMaxBiasSpan - H * P * P) / (B - 1))
+    return AG_ERR_SHAPE;
   if (B == 0 || L == 0) return AG_OK;
   if (!q || !k || !v || !bias || !out || !lse) return AG_ERR_NULL;
   if (!ag::aligned(q, 16) || !ag::aligned(k, 16) || !ag::aligned(v, 16) ||

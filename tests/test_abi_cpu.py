@@ -98,6 +98,10 @@ def test_strided_bias_validation(ag):
     # The per-item bias span (B-1)*stride + H*P*P floats must not overlap out.
     span = (1 * 10 * 8 * P * P + 8 * P * P) * 4
     assert _attn_strided(ag, 10 * 8 * P * P, bias=A16 * 1000 - span + 16) == 7
+    # A span beyond 2^56 floats is refused before its size can overflow.
+    assert _attn_strided(ag, 1 << 62, q=None) == 2
+    assert _attn_strided(ag, (1 << 56) // 9, B=10, q=None) == 2
+    assert _attn_strided(ag, (1 << 56) // 10, B=10, q=None) == 1
 
 
 def test_value_width_validation(ag):
