@@ -59,9 +59,20 @@ class Oracle:
             _c_double_p, _c_double_p, _c_double_p, _c_double_p, L,
             L, L, L, L, L, L, ctypes.c_double,
             _c_int64_p, L, _c_double_p, _c_double_p, ctypes.c_int]
+        lib.agref_attn_bwd_ex.argtypes = [
+            _c_double_p, _c_double_p, _c_double_p, _c_double_p, L, _c_double_p,
+            L, L, L, L, L, L, ctypes.c_double,
+            _c_double_p, _c_double_p, _c_double_p, _c_double_p, _c_double_p,
+            _c_double_p, ctypes.c_int]
+        lib.agref_attn_bwd_sample.argtypes = [
+            _c_double_p, _c_double_p, _c_double_p, _c_double_p, L, _c_double_p,
+            L, L, L, L, L, L, ctypes.c_double,
+            _c_int64_p, L, _c_double_p, _c_int64_p, L, _c_double_p, _c_double_p,
+            _c_int64_p, L, _c_double_p, ctypes.c_int]
         lib.agref_max_threads.argtypes = [ctypes.c_int]
         for f in ("agref_pair_bias_project", "agref_attn_fwd_ex",
-                  "agref_attn_rows_ex", "agref_max_threads", "agref_mutant_id"):
+                  "agref_attn_rows_ex", "agref_attn_bwd_ex", "agref_attn_bwd_sample",
+                  "agref_max_threads", "agref_mutant_id"):
             getattr(lib, f).restype = ctypes.c_int
         self._lib = lib
         self.mutant = lib.agref_mutant_id()
@@ -138,6 +149,59 @@ class Oracle:
         if rc != 0:
             raise ValueError(f"agref_attn_rows rc={rc}")
         return out, lse
+
+    # -- attention backward ---------------------------------------------------
+    def attn_bwd(self, q, k, v, bias, dout, block: int = 16, cap: float = 5.0,
+                 nthreads: int = 0):
+        """Gradients of out for the upstream gradient dout [B,H,L,Dv]: returns
+        (dq [B,H,L,D], dk [B,L,D], dv [B,L,Dv], dbias (bias's shape; a shared
+        [H,P,P] bias gets the sum over the batch), lse [B,H,L], delta [B,H,L])
+        with delta_i = sum_j p_ij * (dout_i . v_j)."""
+        q, k, v, bias, dout = _f64(q), _f64(k), _f64(v), _f64(bias), _f64(dout)
+        B, H, L, D = q.shape
+        Dv = v.shape[-1]
+        assert k.shape == (B, L, D) and v.shape == (B, L, Dv)
+        assert dout.shape == (B, H, L, Dv)
+        bstride = self._bias_stride(bias, B, H, L, int(block))
+        dq = np.zeros((B, H, L, D))
+        dk = np.zeros((B, L, D))
+        dv = np.zeros((B, L, Dv))
+        dbias = np.zeros(bias.shape)
+        lse = np.zeros((B, H, L))
+        delta = np.zeros((B, H, L))
+        rc = self._lib.agref_attn_bwd_ex(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(bias), bstride, _ptr(dout),
+            B, H, L, D, Dv, int(block), float(cap), _ptr(dq), _ptr(dk), _ptr(dv),
+            _ptr(dbias), _ptr(lse), _ptr(delta), int(nthreads))
+        if rc != 0:
+            raise ValueError(f"agref_attn_bwd_ex rc={rc}")
+        return dq, dk, dv, dbias, lse, delta
+
+    def attn_bwd_sample(self, q, k, v, bias, dout, rows=(), keys=(), cells=(),
+                        block: int = 16, cap: float = 5.0, nthreads: int = 0):
+        """Selected gradients: rows (b,h,i) -> dq rows [n,D]; keys (b,j) ->
+        dk rows [n,D] and dv rows [n,Dv]; cells (b,h,I,J) -> dbias values [n]
+        (b ignored for a shared bias)."""
+        q, k, v, bias, dout = _f64(q), _f64(k), _f64(v), _f64(bias), _f64(dout)
+        B, H, L, D = q.shape
+        Dv = v.shape[-1]
+        bstride = self._bias_stride(bias, B, H, L, int(block))
+        rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
+        keys = np.ascontiguousarray(np.asarray(keys, dtype=np.int64).reshape(-1, 2))
+        cells = np.ascontiguousarray(np.asarray(cells, dtype=np.int64).reshape(-1, 4))
+        dq = np.zeros((rows.shape[0], D))
+        dk = np.zeros((keys.shape[0], D))
+        dv = np.zeros((keys.shape[0], Dv))
+        db = np.zeros((cells.shape[0],))
+        rc = self._lib.agref_attn_bwd_sample(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(bias), bstride, _ptr(dout),
+            B, H, L, D, Dv, int(block), float(cap),
+            rows.ctypes.data_as(_c_int64_p), rows.shape[0], _ptr(dq),
+            keys.ctypes.data_as(_c_int64_p), keys.shape[0], _ptr(dk), _ptr(dv),
+            cells.ctypes.data_as(_c_int64_p), cells.shape[0], _ptr(db), int(nthreads))
+        if rc != 0:
+            raise ValueError(f"agref_attn_bwd_sample rc={rc}")
+        return dq, dk, dv, db
 
 
 _default: Oracle | None = None

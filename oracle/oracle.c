@@ -40,6 +40,12 @@
  * read as a plain linear map without bias term or activation (the page names
  * no other term).
  *
+ * Backward (agref_attn_bwd_ex, agref_attn_bwd_sample): the gradients of out
+ * with respect to q, k, v and the compact bias by the chain rule through the
+ * softmax and the soft cap, written out at the end of this file.  The page
+ * lists a backward pass only as later work for fine-tuning (section "Where I
+ * would take it next").
+ *
  * Everything is float64.  Callers widen the exact bf16 / fp32 bit patterns
  * that the GPU receives to float64 before calling.
  *
@@ -338,4 +344,324 @@ int agref_attn_rows(const double *q, const double *k, const double *v,
                     double *out_rows, double *lse_rows, int nthreads) {
     return agref_attn_rows_ex(q, k, v, bias, 0, B, H, L, D, Dv, block, cap, rows,
                               n, out_rows, lse_rows, nthreads);
+}
+
+/* ---- attention backward ------------------------------------------------ */
+/*
+ * Gradients of the attention map above with respect to q, k, v and the
+ * compact bias, for an upstream gradient dout [B,H,L,Dv] of out.  The page
+ * names a backward pass only as later work for fine-tuning (section "Where I
+ * would take it next"); what it must compute is the chain rule applied to
+ * Eq. L_ij and the softmax.  With
+ *   p_ij    = exp(L_ij - lse_i)                        softmax weight
+ *   dp_ij   = sum_c dout[i,c] * v[j,c]
+ *   delta_i = sum_j p_ij * dp_ij
+ *   dL_ij   = p_ij * (dp_ij - delta_i)                 softmax Jacobian
+ *   ds_ij   = dL_ij * (1 - tanh^2(s_ij / cap))         cap = +inf: ds = dL
+ *           = dL_ij * (1 - (L_ij / cap)^2)
+ * the gradients are
+ *   dq[b,h,i,:]  = sum_j ds_ij * k[b,j,:] / sqrt(D)
+ *   dk[b,j,:]    = sum_{h,i} ds_ij * q[b,h,i,:] / sqrt(D)   (K shared by the heads)
+ *   dv[b,j,:]    = sum_{h,i} p_ij * dout[b,h,i,:]          (V shared by the heads)
+ *   dbias cell (h, I, J) = sum_{i in block I, j in block J} ds_ij, summed over
+ *                  the batch items that share the bias (bias_bstride = 0) or
+ *                  kept per item (bias_bstride > 0, same layout as bias).
+ * Three passes, each parallel over what it writes, so that no two threads
+ * add into one value: rows (lse, delta, dq), keys (dk, dv), bias cells.
+ */
+
+/* lse_i and delta_i of row (b, h, i), from the forward row and its weights.
+   logit, brow, prob are caller scratch of length L; orow of length Dv. */
+static void bwd_row_stats(const attn_args *a, const double *dout, long b, long h,
+                          long i, double *logit, double *brow, double *prob,
+                          double *orow, double *lse_out, double *delta_out) {
+    double lse = 0.0;
+    attn_row(a, b, h, i, logit, brow, orow, &lse, prob);
+    const long L = a->L, Dv = a->Dv;
+    const double *gi = dout + ((b * a->H + h) * L + i) * Dv;
+    const double *vb = a->v + b * L * Dv;
+    double delta = 0.0;
+    for (long j = 0; j < L; ++j) {
+        double dp = 0.0;
+        for (long c = 0; c < Dv; ++c) dp += gi[c] * vb[j * Dv + c];
+        delta += prob[j] * dp;
+    }
+    *lse_out = lse;
+    *delta_out = delta;
+}
+
+/* p_ij and ds_ij of one (query, key) pair, given the row's lse and delta. */
+static void bwd_pair(const attn_args *a, const double *dout, long b, long h,
+                     long i, long j, double lse, double delta, double *p_out,
+                     double *ds_out) {
+    const long L = a->L, D = a->D, Dv = a->Dv, blk = a->block, P = a->P;
+    const double *qi = a->q + ((b * a->H + h) * L + i) * D;
+    const double *kj = a->k + (b * L + j) * D;
+    const double *vj = a->v + (b * L + j) * Dv;
+    const double *gi = dout + ((b * a->H + h) * L + i) * Dv;
+    const double *bias_b = a->bias + b * a->bias_bstride;
+    double dot = 0.0;
+    for (long d = 0; d < D; ++d) dot += qi[d] * kj[d];
+    const double s = dot / sqrt((double)D) + bias_b[(h * P + i / blk) * P + j / blk];
+    const double l = soft_cap(s, a->cap);
+    const double p = exp(l - lse);
+    double dp = 0.0;
+    for (long c = 0; c < Dv; ++c) dp += gi[c] * vj[c];
+#if AGREF_MUTANT == 16
+    const double dl = p * dp; /* softmax Jacobian without the delta term */
+    (void)delta;
+#else
+    const double dl = p * (dp - delta);
+#endif
+#if AGREF_MUTANT == 15
+    const double g = 1.0; /* derivative of the soft cap dropped */
+#else
+    const double g = isinf(a->cap) ? 1.0 : 1.0 - (l / a->cap) * (l / a->cap);
+#endif
+    *p_out = p;
+    *ds_out = dl * g;
+}
+
+/* dk and dv of key (b, j): sums over every head and query row. */
+static void bwd_key(const attn_args *a, const double *dout, const double *lse,
+                    const double *delta, long b, long j, double *dk_row,
+                    double *dv_row) {
+    const long L = a->L, D = a->D, Dv = a->Dv, H = a->H;
+    for (long d = 0; d < D; ++d) dk_row[d] = 0.0;
+    for (long c = 0; c < Dv; ++c) dv_row[c] = 0.0;
+#if AGREF_MUTANT == 17
+    const double scale = 1.0; /* 1/sqrt(D) missing from dk */
+#else
+    const double scale = 1.0 / sqrt((double)D);
+#endif
+    for (long h = 0; h < H; ++h) {
+        for (long i = 0; i < L; ++i) {
+            const long r = (b * H + h) * L + i;
+            double p, ds;
+            bwd_pair(a, dout, b, h, i, j, lse[r], delta[r], &p, &ds);
+            const double *qi = a->q + r * D;
+            const double *gi = dout + r * Dv;
+            for (long d = 0; d < D; ++d) dk_row[d] += ds * qi[d] * scale;
+            for (long c = 0; c < Dv; ++c) dv_row[c] += p * gi[c];
+        }
+    }
+}
+
+/* One compact bias cell (h, I, J) of item b's bias; with a shared bias
+   (bias_bstride = 0) the sum runs over every item and b is ignored. */
+static double bwd_cell(const attn_args *a, const double *dout, const double *lse,
+                       const double *delta, long b, long h, long I, long J) {
+    const long L = a->L, blk = a->block, H = a->H;
+#if AGREF_MUTANT == 18
+    const long b0 = a->bias_bstride ? b : 0, b1 = b0 + 1; /* shared: item 0 only */
+#else
+    const long b0 = a->bias_bstride ? b : 0, b1 = a->bias_bstride ? b + 1 : a->B;
+#endif
+    double acc = 0.0;
+    for (long bb = b0; bb < b1; ++bb) {
+        for (long i = I * blk; i < (I + 1) * blk && i < L; ++i) {
+            const long r = (bb * H + h) * L + i;
+            for (long j = J * blk; j < (J + 1) * blk && j < L; ++j) {
+                double p, ds;
+                bwd_pair(a, dout, bb, h, i, j, lse[r], delta[r], &p, &ds);
+                acc += ds;
+            }
+        }
+    }
+    return acc;
+}
+
+/* lse and delta for every row (b, h, i). */
+static int bwd_all_row_stats(const attn_args *a, const double *dout, double *lse,
+                             double *delta) {
+    const long rows = a->B * a->H * a->L, L = a->L;
+    int failed = 0;
+#pragma omp parallel
+    {
+        double *logit = (double *)malloc(sizeof(double) * (size_t)L);
+        double *brow = (double *)malloc(sizeof(double) * (size_t)L);
+        double *prob = (double *)malloc(sizeof(double) * (size_t)L);
+        double *orow = (double *)malloc(sizeof(double) * (size_t)a->Dv);
+        if (!logit || !brow || !prob || !orow) {
+#pragma omp atomic write
+            failed = 1;
+        } else {
+            long r;
+#pragma omp for schedule(dynamic, 16)
+            for (r = 0; r < rows; ++r) {
+                bwd_row_stats(a, dout, r / (L * a->H), (r / L) % a->H, r % L, logit,
+                              brow, prob, orow, lse + r, delta + r);
+            }
+        }
+        free(logit);
+        free(brow);
+        free(prob);
+        free(orow);
+    }
+    return failed ? AGREF_ENOMEM : AGREF_OK;
+}
+
+/*
+ * Full backward.  Inputs as agref_attn_fwd_ex plus dout [B,H,L,Dv].  Writes
+ * dq [B,H,L,D], dk [B,L,D], dv [B,L,Dv] and dbias in the layout of bias
+ * ([H,P,P] when bias_bstride = 0, else item b at dbias + b*bias_bstride);
+ * lse_out and delta_out [B,H,L] are optional.
+ */
+int agref_attn_bwd_ex(const double *q, const double *k, const double *v,
+                      const double *bias, long bias_bstride, const double *dout,
+                      long B, long H, long L, long D, long Dv, long block,
+                      double cap, double *dq, double *dk, double *dv,
+                      double *dbias, double *lse_out, double *delta_out,
+                      int nthreads) {
+    attn_args a = {q, k, v, bias, B, H, L, D, Dv, block, 0, cap, bias_bstride};
+    int rc = check_args(&a);
+    if (rc != AGREF_OK || B == 0 || L == 0) return rc;
+    if (!dout || !dq || !dk || !dv || !dbias || bias_bstride < 0) return AGREF_EINVAL;
+    a.P = cells(L, block);
+    set_threads(nthreads);
+    const long rows = B * H * L, P = a.P;
+    double *lse = (double *)malloc(sizeof(double) * (size_t)rows);
+    double *delta = (double *)malloc(sizeof(double) * (size_t)rows);
+    if (!lse || !delta) {
+        free(lse);
+        free(delta);
+        return AGREF_ENOMEM;
+    }
+    rc = bwd_all_row_stats(&a, dout, lse, delta);
+    if (rc == AGREF_OK) {
+        const double scale = 1.0 / sqrt((double)D);
+        long r;
+#pragma omp parallel for schedule(dynamic, 16)
+        for (r = 0; r < rows; ++r) {
+            const long i = r % L, h = (r / L) % H, b = r / (L * H);
+            double *dqi = dq + r * D;
+            for (long d = 0; d < D; ++d) dqi[d] = 0.0;
+            for (long j = 0; j < L; ++j) {
+                double p, ds;
+                bwd_pair(&a, dout, b, h, i, j, lse[r], delta[r], &p, &ds);
+                const double *kj = k + (b * L + j) * D;
+                for (long d = 0; d < D; ++d) dqi[d] += ds * kj[d] * scale;
+            }
+        }
+        long t;
+#pragma omp parallel for schedule(dynamic, 4)
+        for (t = 0; t < B * L; ++t)
+            bwd_key(&a, dout, lse, delta, t / L, t % L, dk + t * D, dv + t * Dv);
+        const long items = bias_bstride ? B : 1;
+        long c;
+#pragma omp parallel for schedule(dynamic, 4)
+        for (c = 0; c < items * H * P * P; ++c) {
+            const long J = c % P, I = (c / P) % P, h = (c / (P * P)) % H,
+                       b = c / (P * P * H);
+            dbias[b * bias_bstride + (h * P + I) * P + J] =
+                bwd_cell(&a, dout, lse, delta, b, h, I, J);
+        }
+        if (lse_out) memcpy(lse_out, lse, sizeof(double) * (size_t)rows);
+        if (delta_out) memcpy(delta_out, delta, sizeof(double) * (size_t)rows);
+    }
+    free(lse);
+    free(delta);
+    return rc;
+}
+
+/*
+ * Selected gradients only, to check full-size results on a sample:
+ * rows (b,h,i) x n_rows -> dq_rows [n_rows, D]; keys (b,j) x n_keys ->
+ * dk_rows [n_keys, D], dv_rows [n_keys, Dv]; cells (b,h,I,J) x n_cells ->
+ * dbias_cells [n_cells] (b ignored for a shared bias).  Row statistics are
+ * computed for every row when keys or cells are asked for (they sum over all
+ * rows), else only for the rows asked for.
+ */
+int agref_attn_bwd_sample(const double *q, const double *k, const double *v,
+                          const double *bias, long bias_bstride, const double *dout,
+                          long B, long H, long L, long D, long Dv, long block,
+                          double cap, const int64_t *rows, long n_rows,
+                          double *dq_rows, const int64_t *keys, long n_keys,
+                          double *dk_rows, double *dv_rows, const int64_t *cellv,
+                          long n_cells, double *dbias_cells, int nthreads) {
+    attn_args a = {q, k, v, bias, B, H, L, D, Dv, block, 0, cap, bias_bstride};
+    int rc = check_args(&a);
+    if (rc != AGREF_OK) return rc;
+    if (B == 0 || L == 0 || !dout || bias_bstride < 0) return AGREF_EINVAL;
+    a.P = cells(L, block);
+    const long P = a.P;
+    for (long t = 0; t < n_rows; ++t)
+        if (rows[3 * t] < 0 || rows[3 * t] >= B || rows[3 * t + 1] < 0 ||
+            rows[3 * t + 1] >= H || rows[3 * t + 2] < 0 || rows[3 * t + 2] >= L)
+            return AGREF_EINVAL;
+    for (long t = 0; t < n_keys; ++t)
+        if (keys[2 * t] < 0 || keys[2 * t] >= B || keys[2 * t + 1] < 0 ||
+            keys[2 * t + 1] >= L)
+            return AGREF_EINVAL;
+    for (long t = 0; t < n_cells; ++t)
+        if (cellv[4 * t] < 0 || cellv[4 * t] >= B || cellv[4 * t + 1] < 0 ||
+            cellv[4 * t + 1] >= H || cellv[4 * t + 2] < 0 || cellv[4 * t + 2] >= P ||
+            cellv[4 * t + 3] < 0 || cellv[4 * t + 3] >= P)
+            return AGREF_EINVAL;
+    set_threads(nthreads);
+    const long nr = B * H * L;
+    double *lse = (double *)malloc(sizeof(double) * (size_t)nr);
+    double *delta = (double *)malloc(sizeof(double) * (size_t)nr);
+    if (!lse || !delta) {
+        free(lse);
+        free(delta);
+        return AGREF_ENOMEM;
+    }
+    if (n_keys > 0 || n_cells > 0) {
+        rc = bwd_all_row_stats(&a, dout, lse, delta);
+    } else {
+        int failed = 0;
+#pragma omp parallel
+        {
+            double *logit = (double *)malloc(sizeof(double) * (size_t)L);
+            double *brow = (double *)malloc(sizeof(double) * (size_t)L);
+            double *prob = (double *)malloc(sizeof(double) * (size_t)L);
+            double *orow = (double *)malloc(sizeof(double) * (size_t)Dv);
+            if (!logit || !brow || !prob || !orow) {
+#pragma omp atomic write
+                failed = 1;
+            } else {
+                long t;
+#pragma omp for schedule(dynamic, 1)
+                for (t = 0; t < n_rows; ++t) {
+                    const long b = rows[3 * t], h = rows[3 * t + 1], i = rows[3 * t + 2];
+                    const long r = (b * H + h) * L + i;
+                    bwd_row_stats(&a, dout, b, h, i, logit, brow, prob, orow, lse + r,
+                                  delta + r);
+                }
+            }
+            free(logit);
+            free(brow);
+            free(prob);
+            free(orow);
+        }
+        rc = failed ? AGREF_ENOMEM : AGREF_OK;
+    }
+    if (rc == AGREF_OK) {
+        const double scale = 1.0 / sqrt((double)D);
+        long t;
+#pragma omp parallel for schedule(dynamic, 1)
+        for (t = 0; t < n_rows; ++t) {
+            const long b = rows[3 * t], h = rows[3 * t + 1], i = rows[3 * t + 2];
+            const long r = (b * H + h) * L + i;
+            double *dqi = dq_rows + t * D;
+            for (long d = 0; d < D; ++d) dqi[d] = 0.0;
+            for (long j = 0; j < L; ++j) {
+                double p, ds;
+                bwd_pair(&a, dout, b, h, i, j, lse[r], delta[r], &p, &ds);
+                for (long d = 0; d < D; ++d) dqi[d] += ds * k[(b * L + j) * D + d] * scale;
+            }
+        }
+#pragma omp parallel for schedule(dynamic, 1)
+        for (t = 0; t < n_keys; ++t)
+            bwd_key(&a, dout, lse, delta, keys[2 * t], keys[2 * t + 1], dk_rows + t * D,
+                    dv_rows + t * Dv);
+#pragma omp parallel for schedule(dynamic, 1)
+        for (t = 0; t < n_cells; ++t)
+            dbias_cells[t] = bwd_cell(&a, dout, lse, delta, cellv[4 * t],
+                                      cellv[4 * t + 1], cellv[4 * t + 2], cellv[4 * t + 3]);
+    }
+    free(lse);
+    free(delta);
+    return rc;
 }

@@ -267,7 +267,124 @@ def pin_projection(o):
            1e-12, "linearity")
 
 
+# ---- backward ---------------------------------------------------------------
+def torch_dense_grads(q, k, v, bias, dout, block, cap):
+    """Gradients of sum(out * dout) by torch autograd (float64, CPU) through a
+    dense evaluation of its own: the compact bias is repeated with
+    repeat_interleave, so its gradient is autograd's sum over each cell."""
+    t = {n: torch.tensor(x, dtype=torch.float64, requires_grad=True)
+         for n, x in (("q", q), ("k", k), ("v", v), ("bias", bias))}
+    L, D = q.shape[2], q.shape[3]
+    b4 = t["bias"] if bias.ndim == 4 else t["bias"][None]
+    bexp = b4.repeat_interleave(block, 2).repeat_interleave(block, 3)[:, :, :L, :L]
+    s = torch.einsum("bhid,bjd->bhij", t["q"], t["k"]) / math.sqrt(D) + bexp
+    logits = s if math.isinf(cap) else cap * torch.tanh(s / cap)
+    out = torch.einsum("bhij,bjc->bhic", torch.softmax(logits, -1), t["v"])
+    (out * torch.from_numpy(dout)).sum().backward()
+    return [t[n].grad.numpy() for n in ("q", "k", "v", "bias")]
+
+
+def _bwd_case(B=2, H=3, L=40, D=8, Dv=6, block=16, seed=0, batched_bias=False):
+    c = _case(B=B, H=H, L=L, D=D, Dv=Dv, block=block, seed=seed, batched_bias=batched_bias)
+    c["dout"] = np.random.default_rng(seed + 100).normal(size=(B, H, L, Dv))
+    return c
+
+
+def pin_bwd_autograd(o):
+    """Oracle gradients == torch autograd of a dense evaluation, for several
+    blocks and caps, a partial last block, a bias shared by two items (its
+    gradient sums over them) and one bias per item."""
+    cases = [dict(L=64, block=16), dict(L=40, block=16), dict(L=23, block=4),
+             dict(L=32, block=1), dict(L=48, block=16, batched_bias=True)]
+    for n, kw in enumerate(cases):
+        for cap in CAPS:
+            c = _bwd_case(seed=n, **kw)
+            got = o.attn_bwd(c["q"], c["k"], c["v"], c["bias"], c["dout"],
+                             block=kw["block"], cap=cap)
+            want = torch_dense_grads(c["q"], c["k"], c["v"], c["bias"], c["dout"],
+                                     kw["block"], cap)
+            for name, g, w in zip(("dq", "dk", "dv", "dbias"), got[:4], want):
+                _close(g, w, 1e-11, f"{name} {kw} cap={cap}")
+
+
+def pin_bwd_finite_differences(o):
+    """Directional derivatives of f = sum(out * dout) by central differences of
+    the forward oracle match the backward oracle's gradients."""
+    c = _bwd_case(B=2, H=2, L=40, D=8, Dv=5, block=16, seed=21)
+    rng = np.random.default_rng(22)
+    for cap in (5.0, math.inf):
+        dq, dk, dv, db, _, _ = o.attn_bwd(c["q"], c["k"], c["v"], c["bias"], c["dout"],
+                                          block=16, cap=cap)
+        grads = {"q": dq, "k": dk, "v": dv, "bias": db}
+        for name in ("q", "k", "v", "bias"):
+            u = rng.normal(size=c[name].shape)
+            eps = 1e-5
+
+            def f(sign):
+                x = dict(c)
+                x[name] = c[name] + sign * eps * u
+                out, _ = o.attn_fwd(x["q"], x["k"], x["v"], x["bias"], block=16, cap=cap)
+                return float(np.sum(out * c["dout"]))
+
+            fd = (f(+1) - f(-1)) / (2 * eps)
+            an = float(np.sum(grads[name] * u))
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), \
+                f"d/d{name} cap={cap}: finite difference {fd:.10g} vs gradient {an:.10g}"
+
+
+def pin_bwd_closed_forms(o):
+    """(a) All keys equal and no bias: the softmax is uniform and its logits
+    are equal, so dq = 0 and dv_j = (1/L) sum_{h,i} dout_i for every key.
+    (b) No cap: adding a constant to one query block's bias row changes
+    nothing, so each row of dbias sums to 0 over the key blocks.
+    (c) delta_i = dout_i . out_i (sum_j p_ij v_j = out_i)."""
+    rng = np.random.default_rng(31)
+    B, H, L, D, Dv = 1, 2, 48, 8, 5
+    q = rng.normal(size=(B, H, L, D)) * 2.0
+    k = np.broadcast_to(rng.normal(size=(1, 1, D)), (B, L, D)).copy()
+    v = rng.normal(size=(B, L, Dv))
+    dout = rng.normal(size=(B, H, L, Dv))
+    bias = np.zeros((H, L // 16, L // 16))
+    for cap in (5.0, math.inf):
+        dq, _, dv, _, _, _ = o.attn_bwd(q, k, v, bias, dout, block=16, cap=cap)
+        _close(dq, np.zeros_like(dq), 1e-12, f"identical keys dq cap={cap}")
+        want = np.broadcast_to(dout.sum(axis=(1, 2))[:, None, :] / L, dv.shape)
+        _close(dv, want, 1e-12, f"identical keys dv cap={cap}")
+    c = _bwd_case(B=2, H=3, L=40, D=8, Dv=6, block=16, seed=32)
+    _, _, _, db, _, delta = o.attn_bwd(c["q"], c["k"], c["v"], c["bias"], c["dout"],
+                                       block=16, cap=math.inf)
+    _close(db.sum(axis=-1), np.zeros(db.shape[:-1]), 1e-12, "no-cap dbias row sums")
+    out, _ = o.attn_fwd(c["q"], c["k"], c["v"], c["bias"], block=16, cap=5.0)
+    _, _, _, _, _, delta5 = o.attn_bwd(c["q"], c["k"], c["v"], c["bias"], c["dout"],
+                                       block=16, cap=5.0)
+    _close(delta5, np.einsum("bhic,bhic->bhi", c["dout"], out), 1e-12, "delta = dout . out")
+
+
+def pin_bwd_sample(o):
+    """The sampled backward entry returns exactly the full backward's values,
+    for a shared bias (cells summed over the items) and one bias per item."""
+    for batched in (False, True):
+        c = _bwd_case(B=2, H=3, L=40, D=8, Dv=6, block=16, seed=41, batched_bias=batched)
+        dq, dk, dv, db, _, _ = o.attn_bwd(c["q"], c["k"], c["v"], c["bias"], c["dout"],
+                                          block=16, cap=5.0)
+        rows = [[0, 0, 0], [1, 2, 39], [0, 1, 17]]
+        keys = [[0, 0], [1, 39], [1, 16]]
+        cells = [[0, 0, 0, 0], [1, 2, 2, 1], [1, 1, 0, 2]]
+        sq, sk, sv, sb = o.attn_bwd_sample(c["q"], c["k"], c["v"], c["bias"], c["dout"],
+                                           rows=rows, keys=keys, cells=cells,
+                                           block=16, cap=5.0)
+        for t, (b, h, i) in enumerate(rows):
+            _close(sq[t], dq[b, h, i], 1e-13, f"sample dq {b},{h},{i}")
+        for t, (b, j) in enumerate(keys):
+            _close(sk[t], dk[b, j], 1e-13, f"sample dk {b},{j}")
+            _close(sv[t], dv[b, j], 1e-13, f"sample dv {b},{j}")
+        for t, (b, h, I, J) in enumerate(cells):
+            want = db[b, h, I, J] if batched else db[h, I, J]
+            _close(sb[t], want, 1e-13, f"sample dbias {b},{h},{I},{J}")
+
+
 ALL_PINS = [
     pin_bruteforce, pin_bruteforce_tails_and_batched_bias, pin_sdpa, pin_identical_keys, pin_block_bias_closed_form,
     pin_cap_limit, pin_probabilities, pin_invariances, pin_rows, pin_projection,
+    pin_bwd_autograd, pin_bwd_finite_differences, pin_bwd_closed_forms, pin_bwd_sample,
 ]

@@ -24,6 +24,10 @@ MUTANTS = {
     12: "soft cap dropped",
     13: "every batch item reads item 0's bias",
     14: "partial last block dropped from the bias layout",
+    15: "backward: derivative of the soft cap dropped",
+    16: "backward: softmax Jacobian without the delta term",
+    17: "backward: 1/sqrt(D) missing from dk",
+    18: "backward: a shared bias's gradient taken from item 0 only",
 }
 
 
