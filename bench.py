@@ -431,16 +431,103 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     print(json.dumps(line), flush=True)
 
 
+def backward_flops(w) -> float:
+    """Algorithmic FLOPs of one backward call, the usual count of five L x L
+    products: S = Q K^T (recomputed), dP = dO V^T, dV = P^T dO, dQ = dS K,
+    dK = dS^T Q, i.e. 2 B H L^2 (3 D + 2 Dv)."""
+    return 2.0 * w.B * w.H * w.L * w.L * (3 * w.D + 2 * w.Dv)
+
+
+def backward_executed_flops(w) -> float:
+    """FLOPs the two backward kernels execute: the delta pass 2 (D + Dv), the
+    dq pass 2 (D + Dv) + 2 D and the key kernel 2 (D + Dv) + 2 D + 2 Dv per
+    (item, head, query, key)."""
+    return 2.0 * w.B * w.H * w.L * w.L * (3 * (w.D + w.Dv) + 2 * w.D + w.Dv)
+
+
+def run_backward(args) -> None:
+    """One GPU: ag_attn_bwd on the full-context workload (projected bias, the
+    forward's lse), timed per call with CUDA events, L2 flushed between."""
+    import long_context_genomics_b200 as ag
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = WORKLOAD
+    host = ag_inputs.make_inputs(w)
+    d = {n: t.to(dev) for n, t in host.items()}
+    bias = ag.ag_pair_bias_project(d["pair"], d["W"])
+    _, lse = ag.ag_attn_fwd(d["q"], d["k"], d["v"], bias, cap=w.cap)
+    g = torch.Generator(device="cpu").manual_seed(w.seed + 500)
+    dout = torch.randn(w.B, w.H, w.L, w.Dv, generator=g).to(dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        flush.zero_()
+        ag.ag_attn_bwd(d["q"], d["k"], d["v"], bias, lse, dout, cap=w.cap)
+    torch.cuda.synchronize()
+    assert ag.ag_device_error(0) == 0
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    sampler = ClockSampler(0)
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    t0 = time.time()
+    for i in range(K):
+        flush.zero_()
+        ev[i][0].record(stream)
+        ag.ag_attn_bwd(d["q"], d["k"], d["v"], bias, lse, dout, cap=w.cap)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop(t0, time.time())
+    assert ag.ag_device_error(0) == 0
+    ms = [e[0].elapsed_time(e[1]) for e in ev]
+    mean_s = statistics.mean(ms) / 1e3
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    max_mhz = (clocks or {}).get("sm_max_mhz") or 1965.0
+    # FP32 FMA pipe: 128 lanes per SM, 2 FLOPs per FMA, at the maximum SM clock.
+    fp32_peak = sms * 128 * 2 * max_mhz * 1e6 / 1e12
+    alg = backward_flops(w) / mean_s / 1e12
+    exe = backward_executed_flops(w) / mean_s / 1e12
+    line = {
+        "metric": "pair-bias attention backward TFLOP/s at L=8192", "value": alg,
+        "unit": "TFLOP/s", "n_gpus": 1, "steps": K, "warmup": args.warmup,
+        "ms_per_step": 1e3 * mean_s, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {**workload_config(w), "step": "ag_attn_bwd (given the forward's lse)",
+                   "parallelism": "single GPU"},
+        "gpu_launches": K * ag.ag_attn_bwd_launch_count(),
+        "roofline": {"kernel": "attn_bwd_q_kernel + attn_bwd_kv_kernel", "bound": "alu",
+                     "achieved": alg, "peak": fp32_peak, "unit": "TFLOP/s",
+                     "frac": alg / fp32_peak, "traffic": None,
+                     "peak_kind": f"fp32 FMA pipe, {sms} SMs x 128 lanes x 2 x {max_mhz:.0f} MHz",
+                     "executed_tflops": exe, "frac_executed": exe / fp32_peak},
+        "ms": {"median": statistics.median(ms), "p95": sorted(ms)[int(0.95 * (K - 1))]},
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main() -> None:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default 1000; 20 with --path backward)")
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--path", choices=["forward", "backward"], default="forward",
+                    help="forward: projection + attention (the default step); "
+                         "backward: the attention backward alone, one GPU")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
+    if args.steps is None:
+        args.steps = 20 if args.path == "backward" else 1000
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.path == "backward":
+        if args.gpus != 1 or args.impl != "ours":
+            ap.error("--path backward runs our kernels on one GPU")
+        run_backward(args)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

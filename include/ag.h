@@ -196,6 +196,50 @@ ag_status ag_attn_fwd_launch_count(int64_t B, int64_t H, int64_t L, int64_t D,
                                    int64_t block, float cap, int *count);
 
 /*
+ * ag_attn_bwd -- gradients of ag_attn_fwd_ex's out for an upstream gradient
+ * dout: the chain rule through Eq. L_ij and the softmax (page "Making
+ * Full-Context AlphaGenome Fit on an RTX 3090", section "Why stock
+ * FlashAttention was not a drop-in replacement"; the page lists a backward
+ * pass as later work for fine-tuning, section "Where I would take it next").
+ * With x_ij the biased score, p_ij = exp(L_ij - lse_i) and
+ * dp_ij = dout_i . v_j:
+ *   delta_i = sum_j p_ij dp_ij,
+ *   ds_ij   = p_ij (dp_ij - delta_i) (1 - tanh^2(x_ij / cap))  (no cap: 1),
+ *   dq_i = sum_j ds_ij k_j / sqrt(D),  dk_j = sum_{h,i} ds_ij q_i / sqrt(D),
+ *   dv_j = sum_{h,i} p_ij dout_i,  dbias cell = sum of ds_ij over the cell.
+ *
+ * Inputs (device, caller-owned, read only): q, k, v, bias,
+ *   bias_batch_stride, B, H, L, D, Dv, block, cap exactly as
+ *   ag_attn_fwd_ex; lse [B,H,L] float32 as written by the forward call on
+ *   the same inputs; dout [B,H,L,Dv] float32.
+ * Outputs (device, caller-owned, written, float32): dq [B,H,L,D],
+ *   dk [B,L,D], dv [B,L,Dv] (K and V are shared by the heads, so their
+ *   gradients sum over the heads), dbias in the layout of bias (with
+ *   bias_batch_stride = 0 the one shared bias gets the sum over the items;
+ *   otherwise item b's cells at dbias + b * bias_batch_stride, the padding
+ *   between items untouched), delta [B,H,L].
+ * Alignment: q, k, v 2 bytes, the float32 arrays 4 bytes (AG_ERR_ALIGN).
+ *   No output may overlap an input or another output (AG_ERR_ALIAS).  Size
+ *   and value checks and their statuses as ag_attn_fwd_ex; B == 0 or
+ *   L == 0 is a no-op.
+ * Two kernels on `stream` (asynchronous); no device memory is allocated;
+ * every output value is written by one thread in a fixed order, so results
+ * are bitwise reproducible.  The arithmetic is float32 on the CUDA cores.
+ */
+ag_status ag_attn_bwd(const void *q, const void *k, const void *v, const float *bias,
+                      int64_t bias_batch_stride, const float *lse, const float *dout,
+                      int64_t B, int64_t H, int64_t L, int64_t D, int64_t Dv,
+                      int64_t block, float cap, float *dq, float *dk, float *dv,
+                      float *dbias, float *delta, void *stream);
+
+/*
+ * ag_attn_bwd_launch_count -- how many kernels a non-empty ag_attn_bwd call
+ * launches (a library convenience; the pages have no counterpart).  count
+ * is a host pointer (AG_ERR_NULL if NULL).  Launches nothing.
+ */
+ag_status ag_attn_bwd_launch_count(int *count);
+
+/*
  * Device error word.  Every wait inside the kernels is bounded (about one
  * second); a wait that runs out makes the kernel stop, release what it
  * holds and record a code here instead of hanging the GPU.

@@ -68,6 +68,11 @@ def _load() -> ctypes.CDLL:
     lib.ag_attn_fwd_launch_count.argtypes = [i64, i64, i64, i64, i64, f32,
                                              ctypes.POINTER(ctypes.c_int)]
     lib.ag_attn_fwd_launch_count.restype = ctypes.c_int
+    lib.ag_attn_bwd.argtypes = [vp, vp, vp, vp, i64, vp, vp, i64, i64, i64, i64, i64,
+                                i64, f32, vp, vp, vp, vp, vp, vp]
+    lib.ag_attn_bwd.restype = ctypes.c_int
+    lib.ag_attn_bwd_launch_count.argtypes = [ctypes.POINTER(ctypes.c_int)]
+    lib.ag_attn_bwd_launch_count.restype = ctypes.c_int
     lib.ag_device_error.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int),
                                     ctypes.c_int]
     lib.ag_device_error.restype = ctypes.c_int
@@ -210,6 +215,51 @@ def ag_attn_fwd_launch_count(B: int, L: int, cap: float = 5.0, H: int = 8,
                                       float(cap), ctypes.byref(n))
     if st != AG_OK:
         raise AgError("ag_attn_fwd_launch_count", st)
+    return int(n.value)
+
+
+def ag_attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, bias: torch.Tensor,
+                lse: torch.Tensor, dout: torch.Tensor, cap: float = 5.0, block: int = 16,
+                stream=None):
+    """Backward of ag_attn_fwd (libag kernels): gradients of out for the
+    upstream gradient dout [B,H,L,Dv] fp32, given the forward's lse.
+    Returns (dq [B,H,L,D], dk [B,L,D], dv [B,L,Dv], dbias (bias's shape; a
+    shared [H,P,P] bias gets the sum over the batch), delta [B,H,L]), all
+    fp32 and newly allocated."""
+    _check(q, "q", torch.bfloat16, 4)
+    _check(k, "k", torch.bfloat16, 3)
+    _check(v, "v", torch.bfloat16, 3)
+    _check(lse, "lse", torch.float32, 3)
+    _check(dout, "dout", torch.float32, 4)
+    B, H, L, D = q.shape
+    Dv = v.shape[-1]
+    if tuple(k.shape) != (B, L, D) or tuple(v.shape) != (B, L, Dv):
+        raise ValueError("k must be [B,L,D] and v [B,L,Dv] with q [B,H,L,D]")
+    if tuple(lse.shape) != (B, H, L) or tuple(dout.shape) != (B, H, L, Dv):
+        raise ValueError("lse must be [B,H,L] and dout [B,H,L,Dv]")
+    bstride = _bias_stride(bias, B, H, L, block)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    dq = torch.empty((B, H, L, D), **f32)
+    dk = torch.empty((B, L, D), **f32)
+    dv = torch.empty((B, L, Dv), **f32)
+    dbias = torch.empty(tuple(bias.shape), **f32)
+    delta = torch.empty((B, H, L), **f32)
+    st = lib.ag_attn_bwd(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), bias.data_ptr(), bstride,
+        lse.data_ptr(), dout.data_ptr(), B, H, L, D, Dv, int(block), float(cap),
+        dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), dbias.data_ptr(), delta.data_ptr(),
+        _stream_ptr(stream))
+    if st != AG_OK:
+        raise AgError("ag_attn_bwd", st)
+    return dq, dk, dv, dbias, delta
+
+
+def ag_attn_bwd_launch_count() -> int:
+    """How many kernels a non-empty ag_attn_bwd call launches."""
+    n = ctypes.c_int(-1)
+    st = lib.ag_attn_bwd_launch_count(ctypes.byref(n))
+    if st != AG_OK:
+        raise AgError("ag_attn_bwd_launch_count", st)
     return int(n.value)
 
 

@@ -214,6 +214,23 @@ static ag_status check_attn_sizes(int64_t B, int64_t H, int64_t L, int64_t D,
     return AG_ERR_UNSUPPORTED;
   return AG_OK;
 }
+
+// The value width and the per-item bias stride (after check_attn_sizes).
+static ag_status check_value_width_and_bias_stride(int64_t B, int64_t H, int64_t L,
+                                                   int64_t Dv, int64_t block,
+                                                   int64_t bias_batch_stride) {
+  if (Dv <= 0) return AG_ERR_SHAPE;
+  if (Dv != 128 && Dv != 192) return AG_ERR_UNSUPPORTED;
+  const int64_t P = (L + block - 1) / block;
+  if (bias_batch_stride < 0 || (bias_batch_stride > 0 && bias_batch_stride < H * P * P))
+    return AG_ERR_SHAPE;
+  // The items' bias span, (B - 1) * stride + H * P * P floats, must stay far
+  // below 2^63 bytes so that the alias check and the kernel's offsets are exact.
+  constexpr int64_t kMaxBiasSpan = int64_t(1) << 56;
+  if (B > 1 && bias_batch_stride > (kMaxBiasSpan - H * P * P) / (B - 1))
+    return AG_ERR_SHAPE;
+  return AG_OK;
+}
 }  // namespace ag
 
 ag_status ag_attn_fwd(const void *q, const void *k, const void *v,
@@ -239,16 +256,10 @@ ag_status ag_attn_fwd_ex(const void *q, const void *k, const void *v,
                          float cap, float *out, float *lse, void *stream) {
   const ag_status vs = ag::check_attn_sizes(B, H, L, D, block, cap);
   if (vs != AG_OK) return vs;
-  if (Dv <= 0) return AG_ERR_SHAPE;
-  if (Dv != 128 && Dv != 192) return AG_ERR_UNSUPPORTED;
-  const int64_t P = block > 0 ? (L + block - 1) / block : 0;
-  if (bias_batch_stride < 0 || (bias_batch_stride > 0 && bias_batch_stride < H * P * P))
-    return AG_ERR_SHAPE;
-  // The items' bias span, (B - 1) * stride + H * P * P floats, must stay far
-  // below 2^63 bytes so that the alias check and the kernel's offsets are exact.
-  constexpr int64_t kMaxBiasSpan = int64_t(1) << 56;
-  if (B > 1 && bias_batch_stride > (kMaxBiasSpan - H * P * P) / (B - 1))
-    return AG_ERR_SHAPE;
+  const ag_status ws = ag::check_value_width_and_bias_stride(B, H, L, Dv, block,
+                                                             bias_batch_stride);
+  if (ws != AG_OK) return ws;
+  const int64_t P = (L + block - 1) / block;
   if (B == 0 || L == 0) return AG_OK;
   if (!q || !k || !v || !bias || !out || !lse) return AG_ERR_NULL;
   if (!ag::aligned(q, 16) || !ag::aligned(k, 16) || !ag::aligned(v, 16) ||
@@ -374,6 +385,72 @@ ag_status ag_attn_fwd_launch_count(int64_t B, int64_t H, int64_t L, int64_t D,
   st = ag::from_cuda(ag::attn_fwd_kernel_count(B, L, D, cap, dev->num_sms, dev->num_sms, &n));
   if (st != AG_OK) return st;
   *count = n;
+  return AG_OK;
+}
+
+ag_status ag_attn_bwd(const void *q, const void *k, const void *v, const float *bias,
+                      int64_t bias_batch_stride, const float *lse, const float *dout,
+                      int64_t B, int64_t H, int64_t L, int64_t D, int64_t Dv,
+                      int64_t block, float cap, float *dq, float *dk, float *dv,
+                      float *dbias, float *delta, void *stream) {
+  ag_status st = ag::check_attn_sizes(B, H, L, D, block, cap);
+  if (st != AG_OK) return st;
+  st = ag::check_value_width_and_bias_stride(B, H, L, Dv, block, bias_batch_stride);
+  if (st != AG_OK) return st;
+  if (B == 0 || L == 0) return AG_OK;
+  if (!q || !k || !v || !bias || !lse || !dout || !dq || !dk || !dv || !dbias || !delta)
+    return AG_ERR_NULL;
+  if (!ag::aligned(q, 2) || !ag::aligned(k, 2) || !ag::aligned(v, 2) ||
+      !ag::aligned(bias, 4) || !ag::aligned(lse, 4) || !ag::aligned(dout, 4) ||
+      !ag::aligned(dq, 4) || !ag::aligned(dk, 4) || !ag::aligned(dv, 4) ||
+      !ag::aligned(dbias, 4) || !ag::aligned(delta, 4))
+    return AG_ERR_ALIGN;
+  const uint64_t P = static_cast<uint64_t>((L + block - 1) / block);
+  const uint64_t rows = static_cast<uint64_t>(B) * H * L;
+  const uint64_t bias_bytes =
+      (static_cast<uint64_t>(B - 1) * bias_batch_stride + H * P * P) * 4;
+  const uint64_t bias_span = bias_batch_stride ? bias_bytes : H * P * P * 4;
+  const void *ins[6] = {q, k, v, bias, lse, dout};
+  const uint64_t insz[6] = {rows * D * 2, static_cast<uint64_t>(B) * L * D * 2,
+                            static_cast<uint64_t>(B) * L * Dv * 2, bias_span, rows * 4,
+                            rows * Dv * 4};
+  const void *outs[5] = {dq, dk, dv, dbias, delta};
+  const uint64_t outsz[5] = {rows * D * 4, static_cast<uint64_t>(B) * L * D * 4,
+                             static_cast<uint64_t>(B) * L * Dv * 4, bias_span, rows * 4};
+  for (int o = 0; o < 5; ++o) {
+    for (int t = 0; t < 6; ++t)
+      if (ag::overlap(outs[o], outsz[o], ins[t], insz[t])) return AG_ERR_ALIAS;
+    for (int u = o + 1; u < 5; ++u)
+      if (ag::overlap(outs[o], outsz[o], outs[u], outsz[u])) return AG_ERR_ALIAS;
+  }
+  ag::DeviceInfo *dev = nullptr;
+  st = ag::device_info(&dev);
+  if (st != AG_OK) return st;
+  ag::AttnBwdLaunch a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.bias = bias;
+  a.bias_bstride = bias_batch_stride;
+  a.lse = lse;
+  a.dout = dout;
+  a.delta = delta;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.dbias = dbias;
+  a.B = B;
+  a.H = H;
+  a.L = L;
+  a.Dv = Dv;
+  a.cap = cap;
+  a.stream = static_cast<cudaStream_t>(stream);
+  return ag::from_cuda(ag::launch_attn_bwd(a));
+}
+
+ag_status ag_attn_bwd_launch_count(int *count) {
+  if (!count) return AG_ERR_NULL;
+  *count = ag::attn_bwd_kernel_count();
   return AG_OK;
 }
 

@@ -58,6 +58,21 @@ cudaError_t launch_attn_fwd(const AttnLaunch &a);
 cudaError_t attn_fwd_kernel_count(int64_t B, int64_t L, int64_t Dv, float cap,
                                   int num_sms, int scratch_slots, int *count);
 
+// Backward of the attention (attn_bwd.cu): two kernels, the query kernel
+// (delta, dq) then the key kernel (dk, dv, dbias), on `stream`.
+struct AttnBwdLaunch {
+  const void *q, *k, *v;  // bf16 [B,H,L,128], [B,L,128], [B,L,Dv]
+  const float *bias;
+  int64_t bias_bstride;   // floats between batch items' bias (0: shared)
+  const float *lse, *dout;
+  float *delta, *dq, *dk, *dv, *dbias;
+  int64_t B, H, L, Dv;
+  float cap;              // > 0, +inf for no cap
+  cudaStream_t stream;
+};
+cudaError_t launch_attn_bwd(const AttnBwdLaunch &a);
+int attn_bwd_kernel_count();
+
 cudaError_t launch_pair_bias_project(const float *pair, const float *W,
                                      float *bias, int64_t P, int num_sms,
                                      unsigned *err, cudaStream_t stream);

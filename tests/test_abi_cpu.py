@@ -142,3 +142,39 @@ def test_binding_rejects_cpu_tensors(ag):
     k = torch.zeros(1, 16, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         ag.ag_attn_fwd(q, k, k, torch.zeros(8, 1, 1))
+
+
+def _bwd(ag, q=A16, k=A16 * 2, v=A16 * 3, bias=A16 * 4, stride=0, lse=A16 * 5,
+         dout=A16 * 6, B=1, H=8, L=256, D=128, Dv=128, block=16, cap=5.0,
+         dq=A16 * 1000, dk=A16 * 2000, dv=A16 * 3000, dbias=A16 * 4000, delta=A16 * 5000):
+    return ag.lib.ag_attn_bwd(q, k, v, bias, stride, lse, dout, B, H, L, D, Dv, block,
+                              cap, dq, dk, dv, dbias, delta, None)
+
+
+def test_backward_validation(ag):
+    assert _bwd(ag, L=-1) == 2                    # AG_ERR_SHAPE
+    assert _bwd(ag, D=64) == 4                    # AG_ERR_UNSUPPORTED
+    assert _bwd(ag, H=4) == 4
+    assert _bwd(ag, cap=float("nan")) == 5        # AG_ERR_VALUE
+    assert _bwd(ag, cap=0.0) == 5
+    assert _bwd(ag, Dv=0) == 2
+    assert _bwd(ag, Dv=96) == 4
+    assert _bwd(ag, stride=-1) == 2
+    assert _bwd(ag, stride=8 * 16 * 16 - 1) == 2  # items' bias would overlap
+    assert _bwd(ag, B=0, q=None, dq=None) == 0    # empty: a no-op
+    assert _bwd(ag, L=0, dout=None) == 0
+    for name in ("q", "k", "v", "bias", "lse", "dout", "dq", "dk", "dv", "dbias", "delta"):
+        assert _bwd(ag, **{name: None}) == 1, name  # AG_ERR_NULL
+    assert _bwd(ag, q=A16 + 1) == 3               # bf16 needs 2-byte alignment
+    assert _bwd(ag, lse=A16 + 2) == 3             # fp32 needs 4-byte alignment
+    # Outputs overlapping an input or one another.
+    assert _bwd(ag, dq=A16 * 6) == 7              # dq on dout
+    assert _bwd(ag, delta=A16 * 1000 + 64) == 7   # delta inside dq
+    assert _bwd(ag, dbias=A16 * 4) == 7           # dbias on bias
+
+
+def test_backward_launch_count(ag):
+    n = ctypes.c_int(-1)
+    assert ag.lib.ag_attn_bwd_launch_count(ctypes.byref(n)) == 0 and n.value == 2
+    assert ag.lib.ag_attn_bwd_launch_count(None) == 1
+    assert ag.ag_attn_bwd_launch_count() == 2
