@@ -48,7 +48,8 @@ KERNEL_SOURCES = ["long_context_genomics_b200/csrc/attn_fwd_sm100.cu",
 
 def workload_config(w) -> dict:
     return {
-        "workload": f"full_context_L{w.L}_B{w.B}_projected_pair_bias",
+        "workload": (f"full_context_L{w.L}_B{w.B}_projected_pair_bias"
+                     if w.bias_mode == "pair" else f"{w.name}_L{w.L}_B{w.B}_direct_bias"),
         "B": w.B, "L": w.L, "H": w.H, "D": w.D, "Dv": w.Dv, "P": w.P, "Cp": w.Cp,
         "block": w.block, "cap": w.cap, "seed": w.seed,
         "step": "ag_pair_bias_project + ag_attn_fwd",
@@ -446,16 +447,17 @@ def backward_executed_flops(w) -> float:
 
 
 def run_backward(args) -> None:
-    """One GPU: ag_attn_bwd on the full-context workload (projected bias, the
-    forward's lse), timed per call with CUDA events, L2 flushed between."""
+    """One GPU: ag_attn_bwd on one workload (by default the full-context one
+    with its projected bias), given the forward's lse, timed per call with
+    CUDA events, L2 flushed between calls."""
     import long_context_genomics_b200 as ag
 
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    w = WORKLOAD
+    w = ag_inputs.WORKLOADS[args.workload]
     host = ag_inputs.make_inputs(w)
     d = {n: t.to(dev) for n, t in host.items()}
-    bias = ag.ag_pair_bias_project(d["pair"], d["W"])
+    bias = ag.ag_pair_bias_project(d["pair"], d["W"]) if "pair" in d else d["bias"]
     _, lse = ag.ag_attn_fwd(d["q"], d["k"], d["v"], bias, cap=w.cap)
     g = torch.Generator(device="cpu").manual_seed(w.seed + 500)
     dout = torch.randn(w.B, w.H, w.L, w.Dv, generator=g).to(dev)
@@ -489,7 +491,7 @@ def run_backward(args) -> None:
     alg = backward_flops(w) / mean_s / 1e12
     exe = backward_executed_flops(w) / mean_s / 1e12
     line = {
-        "metric": "pair-bias attention backward TFLOP/s at L=8192", "value": alg,
+        "metric": f"pair-bias attention backward TFLOP/s at L={w.L}", "value": alg,
         "unit": "TFLOP/s", "n_gpus": 1, "steps": K, "warmup": args.warmup,
         "ms_per_step": 1e3 * mean_s, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
@@ -517,6 +519,8 @@ def main() -> None:
     ap.add_argument("--path", choices=["forward", "backward"], default="forward",
                     help="forward: projection + attention (the default step); "
                          "backward: the attention backward alone, one GPU")
+    ap.add_argument("--workload", choices=sorted(ag_inputs.WORKLOADS), default="full",
+                    help="with --path backward: which workload (default full, L=8192)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.steps is None:
@@ -526,6 +530,9 @@ def main() -> None:
     if args.path == "backward":
         if args.gpus != 1 or args.impl != "ours":
             ap.error("--path backward runs our kernels on one GPU")
+    elif args.workload != "full":
+        ap.error("--workload applies to --path backward only")
+    if args.path == "backward":
         run_backward(args)
         return
     world = int(os.environ.get("WORLD_SIZE", "1"))
