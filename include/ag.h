@@ -190,7 +190,9 @@ ag_status ag_attn_fwd_noalloc(const void *q, const void *k, const void *v,
  * between SM pairs and the merge kernel runs as well (a library convenience
  * for callers that count launches; the pages have no counterpart).
  * Same size and value checks, and statuses, as ag_attn_fwd; count is a host
- * pointer (AG_ERR_NULL if NULL).  Launches nothing.
+ * pointer (AG_ERR_NULL if NULL).  Launches nothing.  The count holds for
+ * ag_attn_fwd_ex at either value width too: both widths run one CTA per SM,
+ * so they get the same grid.
  */
 ag_status ag_attn_fwd_launch_count(int64_t B, int64_t H, int64_t L, int64_t D,
                                    int64_t block, float cap, int *count);
