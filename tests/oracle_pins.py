@@ -246,7 +246,8 @@ def pin_rows(o):
 def pin_projection(o):
     """Pair projection: one-hot W columns pick a channel (fixes the [H,P,P]
     orientation and the W[c,h] indexing), a constant pair gives the column
-    sums of W, and the map is linear in W."""
+    sums of W, the map is linear in W, and it equals numpy's einsum of the
+    same contraction."""
     rng = np.random.default_rng(2)
     P, Cp, H = 6, 5, 3
     pair = rng.normal(size=(P, P, Cp))
@@ -265,6 +266,9 @@ def pin_projection(o):
     lin = o.pair_bias_project(pair, W2 + W3)
     _close(lin, o.pair_bias_project(pair, W2) + o.pair_bias_project(pair, W3),
            1e-12, "linearity")
+    # A library contraction of the same definition (numpy einsum).
+    _close(o.pair_bias_project(pair, W3), np.einsum("pqc,ch->hpq", pair, W3), 1e-12,
+           "einsum")
 
 
 # ---- backward ---------------------------------------------------------------
