@@ -98,6 +98,17 @@ def _stream_ptr(stream) -> int:
     return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
 
 
+def _one_device(*tensors: torch.Tensor) -> torch.device:
+    """The one device that every tensor of a call lives on.  The kernels run
+    on that device (made current for the call), so a tensor elsewhere would
+    reach them as a pointer they cannot read: refuse it here."""
+    dev = tensors[0].device
+    for t in tensors[1:]:
+        if t.device != dev:
+            raise ValueError(f"all tensors of a call must be on {dev}; one is on {t.device}")
+    return dev
+
+
 def _check(t: torch.Tensor, name: str, dtype, ndim: int):
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
@@ -125,8 +136,9 @@ def ag_pair_bias_project(pair: torch.Tensor, W: torch.Tensor,
     _check(bias, "bias", torch.float32, 3)
     if tuple(bias.shape) != (H, P, P):
         raise ValueError("bias must be [H,P,P]")
-    st = lib.ag_pair_bias_project(pair.data_ptr(), W.data_ptr(), bias.data_ptr(),
-                                  P, Cp, H, _stream_ptr(stream))
+    with torch.cuda.device(_one_device(pair, W, bias)):
+        st = lib.ag_pair_bias_project(pair.data_ptr(), W.data_ptr(), bias.data_ptr(),
+                                      P, Cp, H, _stream_ptr(stream))
     if st != AG_OK:
         raise AgError("ag_pair_bias_project", st)
     return bias
@@ -155,10 +167,11 @@ def ag_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     if lse is None:
         lse = torch.empty((B, H, L), dtype=torch.float32, device=q.device)
     _check_out(out, lse, B, H, L, Dv)
-    st = lib.ag_attn_fwd_ex(
-        q.data_ptr(), k.data_ptr(), v.data_ptr(), bias.data_ptr(), bstride, B, H, L,
-        D, Dv, int(block), float(cap), out.data_ptr(), lse.data_ptr(),
-        _stream_ptr(stream))
+    with torch.cuda.device(_one_device(q, k, v, bias, out, lse)):
+        st = lib.ag_attn_fwd_ex(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), bias.data_ptr(), bstride, B, H, L,
+            D, Dv, int(block), float(cap), out.data_ptr(), lse.data_ptr(),
+            _stream_ptr(stream))
     if st != AG_OK:
         raise AgError("ag_attn_fwd_ex", st)
     return out, lse
@@ -198,10 +211,11 @@ def ag_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     if _bias_stride(bias, B, H, L, block) != 0:
         raise ValueError("ag_attn_fwd_noalloc takes one bias shared by the batch")
     _check_out(out, lse, B, H, L, D)
-    st = lib.ag_attn_fwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                                 bias.data_ptr(), B, H, L, D, int(block),
-                                 float(cap), out.data_ptr(), lse.data_ptr(),
-                                 _stream_ptr(stream))
+    with torch.cuda.device(_one_device(q, k, v, bias, out, lse)):
+        st = lib.ag_attn_fwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                     bias.data_ptr(), B, H, L, D, int(block),
+                                     float(cap), out.data_ptr(), lse.data_ptr(),
+                                     _stream_ptr(stream))
     if st != AG_OK:
         raise AgError("ag_attn_fwd_noalloc", st)
     return out, lse
@@ -238,17 +252,19 @@ def ag_attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, bias: torch.T
     if tuple(lse.shape) != (B, H, L) or tuple(dout.shape) != (B, H, L, Dv):
         raise ValueError("lse must be [B,H,L] and dout [B,H,L,Dv]")
     bstride = _bias_stride(bias, B, H, L, block)
-    f32 = dict(dtype=torch.float32, device=q.device)
+    dev = _one_device(q, k, v, bias, lse, dout)
+    f32 = dict(dtype=torch.float32, device=dev)
     dq = torch.empty((B, H, L, D), **f32)
     dk = torch.empty((B, L, D), **f32)
     dv = torch.empty((B, L, Dv), **f32)
     dbias = torch.empty(tuple(bias.shape), **f32)
     delta = torch.empty((B, H, L), **f32)
-    st = lib.ag_attn_bwd(
-        q.data_ptr(), k.data_ptr(), v.data_ptr(), bias.data_ptr(), bstride,
-        lse.data_ptr(), dout.data_ptr(), B, H, L, D, Dv, int(block), float(cap),
-        dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), dbias.data_ptr(), delta.data_ptr(),
-        _stream_ptr(stream))
+    with torch.cuda.device(dev):
+        st = lib.ag_attn_bwd(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), bias.data_ptr(), bstride,
+            lse.data_ptr(), dout.data_ptr(), B, H, L, D, Dv, int(block), float(cap),
+            dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), dbias.data_ptr(),
+            delta.data_ptr(), _stream_ptr(stream))
     if st != AG_OK:
         raise AgError("ag_attn_bwd", st)
     return dq, dk, dv, dbias, delta

@@ -144,6 +144,15 @@ def test_binding_rejects_cpu_tensors(ag):
         ag.ag_attn_fwd(q, k, k, torch.zeros(8, 1, 1))
 
 
+def test_binding_refuses_tensors_on_different_devices(ag):
+    import torch
+
+    a, b = torch.zeros(2), torch.zeros(2, device="meta")
+    assert ag._one_device(a, torch.ones(3)) == torch.device("cpu")
+    with pytest.raises(ValueError, match="must be on"):
+        ag._one_device(a, b)
+
+
 def _bwd(ag, q=A16, k=A16 * 2, v=A16 * 3, bias=A16 * 4, stride=0, lse=A16 * 5,
          dout=A16 * 6, B=1, H=8, L=256, D=128, Dv=128, block=16, cap=5.0,
          dq=A16 * 1000, dk=A16 * 2000, dv=A16 * 3000, dbias=A16 * 4000, delta=A16 * 5000):
