@@ -7,7 +7,12 @@ One step = the whole path on one batch: ag_pair_bias_project (pair [512,512,128]
 The metric counts the attention's 4*B*H*L^2*D tensor FLOPs per step.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config tiny|short|mid|full|nine_block|all]
 
+--config picks another of the workloads (default full, the headline line):
+tiny/short/mid are L = 512/2048/4096 with a directly drawn bias, nine_block
+runs nine independent L = 8192, B = 2 layers per step (each with its own
+projected bias and cap); "all" prints one line per workload.
 N > 1 runs under torchrun, one process per GPU; each rank runs its own
 independent problem (weak scaling, no collective on the data path) and rank 0
 prints one JSON line with the time taken as the maximum over ranks.
@@ -46,15 +51,43 @@ KERNEL_SOURCES = ["long_context_genomics_b200/csrc/attn_fwd_sm100.cu",
                   "long_context_genomics_b200/csrc/sm100.cuh"]
 
 
+CONFIGS = ("tiny", "short", "mid", "full", "nine_block")
+
+
 def workload_config(w) -> dict:
     return {
         "workload": (f"full_context_L{w.L}_B{w.B}_projected_pair_bias"
                      if w.bias_mode == "pair" else f"{w.name}_L{w.L}_B{w.B}_direct_bias"),
         "B": w.B, "L": w.L, "H": w.H, "D": w.D, "Dv": w.Dv, "P": w.P, "Cp": w.Cp,
         "block": w.block, "cap": w.cap, "seed": w.seed,
-        "step": "ag_pair_bias_project + ag_attn_fwd",
+        "step": ("ag_pair_bias_project + ag_attn_fwd" if w.bias_mode == "pair"
+                 else "ag_attn_fwd"),
         "l2": "flushed between timed steps (256 MiB write)",
     }
+
+
+def config_layers(name: str) -> list:
+    """The layers one step of a workload runs, in order."""
+    if name == "nine_block":
+        return list(ag_inputs.nine_block_stack().layers)
+    return [ag_inputs.WORKLOADS[name]]
+
+
+def job_config(name: str, layers: list, world: int) -> dict:
+    """The line's config: the workload and, for the stack, every layer's cap
+    and seed.  Both arms print the same keys."""
+    if len(layers) == 1:
+        cfg = workload_config(layers[0])
+    else:
+        w = layers[0]
+        cfg = {"workload": f"nine_block_stack_L{w.L}_B{w.B}_projected_pair_bias",
+               "layers": len(layers), "B": w.B, "L": w.L, "H": w.H, "D": w.D,
+               "Dv": w.Dv, "P": w.P, "Cp": w.Cp, "block": w.block,
+               "caps": [l.cap for l in layers], "seeds": [l.seed for l in layers],
+               "step": f"{len(layers)} x (ag_pair_bias_project + ag_attn_fwd)",
+               "l2": "flushed between timed steps (256 MiB write)"}
+    cfg["parallelism"] = f"{world} independent replicas" if world > 1 else "single GPU"
+    return cfg
 
 
 def peaks() -> dict:
@@ -153,68 +186,78 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------
-def cpu_baseline(w, target_s: float = 12.0, seed: int = 11) -> dict:
-    """The float64 oracle, as it stands, on a bounded sample of the workload:
-    randomly chosen query rows (all over the batch and heads) against the full
-    key range.  The bias comes from the oracle's own projection (untimed)."""
+def _oracle_bias(orc, w, inp):
+    return orc.pair_bias_project(inp["pair"], inp["W"]) if w.bias_mode == "pair" else inp["bias"]
+
+
+def cpu_baseline(layers, min_s: float = 2.0) -> dict:
+    """The float64 oracle, as it stands, on the host cores: one full pass over
+    the first layer of the workload (every query row against every key;
+    repeated while it takes under min_s, so that tiny workloads still get a
+    stable time).  The bias comes from the oracle's own projection (untimed)."""
     import oracle
 
     orc = oracle.default()
     cores = orc.threads(len(os.sched_getaffinity(0)))
+    w = layers[0]
     inp = ag_inputs.make_inputs(w)
-    bias = orc.pair_bias_project(inp["pair"], inp["W"])
-    flops_row = 2.0 * w.L * (w.D + w.Dv)
-
-    def run(n, s):
-        rows = ag_inputs.sample_rows(w.B, w.H, w.L, n, seed=s).numpy()
-        t = time.perf_counter()
-        orc.attn_rows(inp["q"], inp["k"], inp["v"], bias, rows, block=w.block, cap=w.cap)
-        return len(rows), time.perf_counter() - t
-
-    n0, t0 = run(max(4 * cores, 16), seed)
-    n = int(min(w.B * w.H * w.L, max(n0, n0 * target_s / max(t0, 1e-6))))
-    n, t = run(n, seed + 1)
-    return {"value": n * flops_row / t / 1e12, "unit": UNIT, "cores": cores,
+    bias = _oracle_bias(orc, w, inp)
+    passes, t = 0, 0.0
+    while t < min_s:
+        t0 = time.perf_counter()
+        orc.attn_fwd(inp["q"], inp["k"], inp["v"], bias, block=w.block, cap=w.cap)
+        t += time.perf_counter() - t0
+        passes += 1
+    what = "layer 1 of 9" if len(layers) > 1 else "the workload"
+    return {"value": passes * w.attn_flops() / t / 1e12, "unit": UNIT, "cores": cores,
             "kind": "oracle",
-            "sample": f"{n} random query rows of {w.B * w.H * w.L} (b,h,i) at L={w.L}, "
-                      f"full key range, float64, {t:.1f} s; projection untimed"}
+            "sample": f"{passes} full pass(es) over {what} (B={w.B}, L={w.L}: every query "
+                      f"row against every key), float64, {t:.1f} s; projection untimed"}
 
 
 def run_reference(args, rank: int, world: int) -> None:
-    """The oracle on the host cores: each step is a bounded row sample."""
+    """The oracle on the host cores: each step is a bounded row sample of the
+    workload's layers (full key range), sized so the whole run takes about
+    two and a half minutes."""
     if rank != 0:
         return
     import oracle
 
-    w = WORKLOAD
+    layers = config_layers(args.config)
     orc = oracle.default()
     cores = orc.threads(len(os.sched_getaffinity(0)))
-    inp = ag_inputs.make_inputs(w)
-    bias = orc.pair_bias_project(inp["pair"], inp["W"])
-    flops_row = 2.0 * w.L * (w.D + w.Dv)
-    per_step_s = min(4.0, 150.0 / max(1, args.steps + args.warmup))
-    rows = ag_inputs.sample_rows(w.B, w.H, w.L, max(4 * cores, 16), seed=0).numpy()
+    inps = [ag_inputs.make_inputs(w) for w in layers]
+    biases = [_oracle_bias(orc, w, inp) for w, inp in zip(layers, inps)]
+    w0 = layers[0]
+    flops_row = 2.0 * w0.L * (w0.D + w0.Dv)
+    per_step_s = min(6.0, 150.0 / max(1, args.steps + args.warmup))
+    rows = ag_inputs.sample_rows(w0.B, w0.H, w0.L, max(4 * cores, 16), seed=0).numpy()
     t = time.perf_counter()
-    orc.attn_rows(inp["q"], inp["k"], inp["v"], bias, rows, block=w.block, cap=w.cap)
+    orc.attn_rows(inps[0]["q"], inps[0]["k"], inps[0]["v"], biases[0], rows, block=w0.block,
+                  cap=w0.cap)
     n = int(max(len(rows), len(rows) * per_step_s / max(time.perf_counter() - t, 1e-6)))
-    times = []
+    n = min(n, w0.B * w0.H * w0.L)
+    times, count = [], 0
     for s in range(args.warmup + args.steps):
+        li = s % len(layers)  # the stack's layers take turns
+        w, inp = layers[li], inps[li]
         rows = ag_inputs.sample_rows(w.B, w.H, w.L, n, seed=100 + s).numpy()
         t = time.perf_counter()
-        orc.attn_rows(inp["q"], inp["k"], inp["v"], bias, rows, block=w.block, cap=w.cap)
+        orc.attn_rows(inp["q"], inp["k"], inp["v"], biases[li], rows, block=w.block, cap=w.cap)
         if s >= args.warmup:
             times.append(time.perf_counter() - t)
+            count += len(rows)
     total = sum(times)
-    value = len(rows) * flops_row * len(times) / total / 1e12
+    value = count * flops_row / total / 1e12
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total / len(times), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(w),
+        "config": job_config(args.config, layers, world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": f"{len(rows)} random query rows per step at L={w.L}, "
-                                   "full key range, float64"},
+                         "sample": f"{n} random query rows per step (full key range) of "
+                                   f"the workload's layers, float64"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -245,24 +288,39 @@ def aggregate_rate(world: int, units_per_step: float, steps: int, seconds: float
     return world * units_per_step * steps / seconds
 
 
-E2E_INPUTS = ("q", "k", "v", "pair", "W")
+def _e2e_inputs(w) -> tuple:
+    """The per-layer host inputs an end-to-end step uploads."""
+    return ("q", "k", "v", "pair", "W") if w.bias_mode == "pair" else ("q", "k", "v", "bias")
 
 
-def pipelined_e2e(ag, w, pinned: dict, dev, steps: int):
-    """Runs `steps` steps through the public API with each step's inputs
-    uploaded from pinned host memory and its out and lse downloaded again, as
-    a pipeline: uploads, compute and downloads go on three streams, so step
-    i+1's upload and step i-1's download overlap step i's kernels.  Two device
-    buffer sets keep an upload from overwriting inputs that a step still reads
-    and a step from overwriting outputs that a download still reads.
+def _forward(ag, w, d, bias, out, lse):
+    """One layer through the public API: the projection (pair mode) and the
+    attention."""
+    if w.bias_mode == "pair":
+        ag.ag_pair_bias_project(d["pair"], d["W"], bias=bias)
+    else:
+        bias = d["bias"]
+    ag.ag_attn_fwd(d["q"], d["k"], d["v"], bias, cap=w.cap, out=out, lse=lse)
+
+
+def pipelined_e2e(ag, layers, pinned: list, dev, steps: int):
+    """Runs `steps` steps (every layer once per step) through the public API
+    with each layer's inputs uploaded from pinned host memory and its out and
+    lse downloaded again, as a pipeline: uploads, compute and downloads go on
+    three streams, so one layer's upload and the previous one's download
+    overlap the kernels in between.  Two device buffer sets keep an upload
+    from overwriting inputs that a layer still reads and a layer from
+    overwriting outputs that a download still reads.
     Returns (seconds from the first upload to the last download, the last
-    step's host lse)."""
+    layer's host lse)."""
     s_up, s_comp, s_down = (torch.cuda.Stream(dev) for _ in range(3))
-    din = [{n: torch.empty(pinned[n].shape, dtype=pinned[n].dtype, device=dev)
-            for n in E2E_INPUTS} for _ in range(2)]
-    bias = torch.empty(w.H, w.P, w.P, device=dev)   # produced and read on s_comp only
-    dout = [torch.empty(w.B, w.H, w.L, w.Dv, device=dev) for _ in range(2)]
-    dlse = [torch.empty(w.B, w.H, w.L, device=dev) for _ in range(2)]
+    w0 = layers[0]
+    names = _e2e_inputs(w0)
+    din = [{n: torch.empty(pinned[0][n].shape, dtype=pinned[0][n].dtype, device=dev)
+            for n in names} for _ in range(2)]
+    bias = torch.empty(w0.H, w0.P, w0.P, device=dev)   # produced and read on s_comp only
+    dout = [torch.empty(w0.B, w0.H, w0.L, w0.Dv, device=dev) for _ in range(2)]
+    dlse = [torch.empty(w0.B, w0.H, w0.L, device=dev) for _ in range(2)]
     hout = [torch.empty(dout[0].shape, pin_memory=True) for _ in range(2)]
     hlse = [torch.empty(dlse[0].shape, pin_memory=True) for _ in range(2)]
     in_ready, in_free, out_ready, out_free = (
@@ -271,31 +329,32 @@ def pipelined_e2e(ag, w, pinned: dict, dev, steps: int):
     t1 = torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize(dev)
     t0.record(s_up)
-    for i in range(steps):
-        u = i % 2
-        # A wait on an event not yet recorded (the first two steps) is a no-op.
-        s_up.wait_event(in_free[u])          # step i-2 has read din[u]
-        with torch.cuda.stream(s_up):
-            for n in E2E_INPUTS:
-                din[u][n].copy_(pinned[n], non_blocking=True)
-        in_ready[u].record(s_up)
-        s_comp.wait_event(in_ready[u])
-        s_comp.wait_event(out_free[u])       # step i-2's outputs are on the host
-        with torch.cuda.stream(s_comp):
-            ag.ag_pair_bias_project(din[u]["pair"], din[u]["W"], bias=bias)
-            ag.ag_attn_fwd(din[u]["q"], din[u]["k"], din[u]["v"], bias, cap=w.cap,
-                           out=dout[u], lse=dlse[u])
-        in_free[u].record(s_comp)
-        out_ready[u].record(s_comp)
-        s_down.wait_event(out_ready[u])
-        with torch.cuda.stream(s_down):
-            hout[u].copy_(dout[u], non_blocking=True)
-            hlse[u].copy_(dlse[u], non_blocking=True)
-        out_free[u].record(s_down)
+    n = 0
+    for _ in range(steps):
+        for li, w in enumerate(layers):
+            u = n % 2
+            n += 1
+            # A wait on an event not yet recorded (the first two) is a no-op.
+            s_up.wait_event(in_free[u])          # the layer two back has read din[u]
+            with torch.cuda.stream(s_up):
+                for name in names:
+                    din[u][name].copy_(pinned[li][name], non_blocking=True)
+            in_ready[u].record(s_up)
+            s_comp.wait_event(in_ready[u])
+            s_comp.wait_event(out_free[u])       # its outputs are on the host
+            with torch.cuda.stream(s_comp):
+                _forward(ag, w, din[u], bias, dout[u], dlse[u])
+            in_free[u].record(s_comp)
+            out_ready[u].record(s_comp)
+            s_down.wait_event(out_ready[u])
+            with torch.cuda.stream(s_down):
+                hout[u].copy_(dout[u], non_blocking=True)
+                hlse[u].copy_(dlse[u], non_blocking=True)
+            out_free[u].record(s_down)
     # The last download waits on every earlier stage, so t1 closes the run.
     t1.record(s_down)
     torch.cuda.synchronize(dev)
-    return t0.elapsed_time(t1) / 1e3, hlse[(steps - 1) % 2]
+    return t0.elapsed_time(t1) / 1e3, hlse[(n - 1) % 2]
 
 
 def run_ours(args, rank: int, world: int, local_rank: int) -> None:
@@ -304,23 +363,25 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     dist = torch.distributed
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    base = WORKLOAD
-    # Each rank runs its own independent problem (own seed).
-    w = rank_workload(base, rank)
-    host = ag_inputs.make_inputs(w)
-    pinned = {n: t.pin_memory() for n, t in host.items()}
-    d = {n: t.to(dev) for n, t in host.items()}
-    bias = torch.empty(w.H, w.P, w.P, device=dev)
-    out = torch.empty(w.B, w.H, w.L, w.Dv, device=dev)
-    lse = torch.empty(w.B, w.H, w.L, device=dev)
+    # Each rank runs its own independent problem (own seeds).
+    layers = [rank_workload(w, rank) for w in config_layers(args.config)]
+    hosts = [ag_inputs.make_inputs(w) for w in layers]
+    pinned = [{n: t.pin_memory() for n, t in h.items()} for h in hosts]
+    d = [{n: t.to(dev) for n, t in h.items()} for h in hosts]
+    w0 = layers[0]
+    biases = [torch.empty(w.H, w.P, w.P, device=dev) if w.bias_mode == "pair" else x["bias"]
+              for w, x in zip(layers, d)]
+    out = torch.empty(w0.B, w0.H, w0.L, w0.Dv, device=dev)
+    lse = torch.empty(w0.B, w0.H, w0.L, device=dev)
     out_h = torch.empty(out.shape, pin_memory=True)
     lse_h = torch.empty(lse.shape, pin_memory=True)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
+    pair_mode = w0.bias_mode == "pair"
 
     def step():
-        ag.ag_pair_bias_project(d["pair"], d["W"], bias=bias)
-        ag.ag_attn_fwd(d["q"], d["k"], d["v"], bias, cap=w.cap, out=out, lse=lse)
+        for w, x, b in zip(layers, d, biases):
+            _forward(ag, w, x, b, out, lse)
 
     def barrier():
         if world > 1:
@@ -334,8 +395,11 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     assert ag.ag_device_error(local_rank) == 0
 
     # ---- device-resident timing --------------------------------------------
+    # Events per step: start, then after each layer's projection and after
+    # its attention.
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    nl = len(layers)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(1 + 2 * nl)] for _ in range(K)]
     sampler = ClockSampler(local_rank) if rank == 0 else None
     time.sleep(0.3 if sampler else 0.0)
     barrier()
@@ -343,60 +407,68 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     for i in range(K):
         flush.zero_()                      # untimed: outside the events
         ev[i][0].record(stream)
-        ag.ag_pair_bias_project(d["pair"], d["W"], bias=bias)
-        ev[i][1].record(stream)
-        ag.ag_attn_fwd(d["q"], d["k"], d["v"], bias, cap=w.cap, out=out, lse=lse)
-        ev[i][2].record(stream)
+        for li, (w, x, b) in enumerate(zip(layers, d, biases)):
+            if pair_mode:
+                ag.ag_pair_bias_project(x["pair"], x["W"], bias=b)
+            ev[i][1 + 2 * li].record(stream)
+            ag.ag_attn_fwd(x["q"], x["k"], x["v"], b, cap=w.cap, out=out, lse=lse)
+            ev[i][2 + 2 * li].record(stream)
     barrier()
     t_wall1 = time.time()
     clocks = sampler.stop(t_wall0, t_wall1) if sampler else None
-    step_ms = [e[0].elapsed_time(e[2]) for e in ev]
-    proj_ms = [e[0].elapsed_time(e[1]) for e in ev]
-    attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    step_ms = [e[0].elapsed_time(e[-1]) for e in ev]
+    proj_ms = [sum((e[2 * li] if li else e[0]).elapsed_time(e[1 + 2 * li]) for li in range(nl))
+               for e in ev]
+    attn_ms = [sum(e[1 + 2 * li].elapsed_time(e[2 + 2 * li]) for li in range(nl)) for e in ev]
     total_s = max_over_ranks(sum(step_ms) / 1e3, dev, world)
     assert ag.ag_device_error(local_rank) == 0
 
     # ---- end to end through the public API with host buffers ---------------
-    h2d = sum(pinned[n].numel() * pinned[n].element_size() for n in E2E_INPUTS)
-    d2h = out_h.numel() * 4 + lse_h.numel() * 4
+    names = _e2e_inputs(w0)
+    h2d = sum(pinned[li][n].numel() * pinned[li][n].element_size()
+              for li in range(nl) for n in names)
+    d2h = nl * (out_h.numel() * 4 + lse_h.numel() * 4)
     # (1) Pipelined, as a serving loop runs it: every step's copies are inside
-    # the timed region, overlapped with the neighbouring steps' kernels.
-    pipelined_e2e(ag, w, pinned, dev, args.warmup)
+    # the timed region, overlapped with the neighbouring layers' kernels.
+    pipelined_e2e(ag, layers, pinned, dev, max(1, min(args.warmup, 3)))
     barrier()
-    e2e_s, e2e_lse = pipelined_e2e(ag, w, pinned, dev, K)
+    e2e_s, e2e_lse = pipelined_e2e(ag, layers, pinned, dev, K)
     e2e_s = max_over_ranks(e2e_s, dev, world)
-    assert math.isfinite(float(e2e_lse[0, 0, 0])) and ag.ag_device_error(local_rank) == 0
-    # (2) One step at a time on one stream: upload, compute, download.
+    assert math.isfinite(float(e2e_lse.flatten()[0])) and ag.ag_device_error(local_rank) == 0
+    # (2) One layer at a time on one stream: upload, compute, download.
     ee = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     barrier()
     for i in range(K):
         flush.zero_()
         ee[i][0].record(stream)
-        for n in E2E_INPUTS:
-            d[n].copy_(pinned[n], non_blocking=True)
-        step()
-        out_h.copy_(out, non_blocking=True)
-        lse_h.copy_(lse, non_blocking=True)
+        for li, (w, x, b) in enumerate(zip(layers, d, biases)):
+            for n in names:
+                x[n].copy_(pinned[li][n], non_blocking=True)
+            _forward(ag, w, x, b, out, lse)
+            out_h.copy_(out, non_blocking=True)
+            lse_h.copy_(lse, non_blocking=True)
         ee[i][1].record(stream)
     barrier()
     serial_s = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ee) / 1e3, dev, world)
-    assert math.isfinite(float(lse_h[0, 0, 0])) and ag.ag_device_error(local_rank) == 0
+    assert math.isfinite(float(lse_h.flatten()[0])) and ag.ag_device_error(local_rank) == 0
 
     if rank != 0:
         return
-    flops = w.attn_flops()
+    flops = sum(w.attn_flops() for w in layers)
+    attn_bytes = sum(w.attn_bytes() for w in layers)
+    proj_bytes = sum(w.project_bytes() for w in layers) if pair_mode else 0
     pk = peaks()
     value = aggregate_rate(world, flops, K, total_s) / 1e12
     attn_mean_s = statistics.mean(attn_ms) / 1e3
+    attn_med_s = statistics.median(attn_ms) / 1e3
     achieved = flops / attn_mean_s / 1e12
-    proj_mean_s = statistics.mean(proj_ms) / 1e3
+    launches = sum(ag.ag_attn_fwd_launch_count(w.B, w.L, w.cap) for w in layers)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": 1e3 * total_s / K,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
-        "config": {**workload_config(w), "parallelism": f"{world} independent replicas"
-                   if world > 1 else "single GPU"},
+        "config": job_config(args.config, layers, world),
         "pct_of_peak": 100.0 * (value / world) / pk["bf16_tflops"],
         "peak_source": pk["source"],
         "e2e": {"value": aggregate_rate(world, flops, K, e2e_s) / 1e12, "unit": UNIT,
@@ -404,13 +476,13 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
                 "ms_per_step": 1e3 * e2e_s / K,
                 "schedule": "pipelined: uploads, compute and downloads on three "
                             "streams, two device buffer sets",
-                "l2": "inputs uploaded every step (155 MB, more than L2); no flush"},
+                "l2": f"inputs uploaded every step ({h2d / 1e6:.0f} MB); no flush"},
         "e2e_serial": {"value": aggregate_rate(world, flops, K, serial_s) / 1e12,
                        "unit": UNIT, "ms_per_step": 1e3 * serial_s / K,
-                       "schedule": "one stream: upload, compute, download per step"},
-        # Our kernels in the timed region: the projection, and the attention
-        # with its split-pair merge when the grid splits pairs.
-        "gpu_launches": K * (1 + ag.ag_attn_fwd_launch_count(w.B, w.L, w.cap)),
+                       "schedule": "one stream: upload, compute, download per layer"},
+        # Our kernels in the timed region: per layer the projection (pair
+        # mode) and the attention's one or two launches.
+        "gpu_launches": K * ((nl if pair_mode else 0) + launches),
         "roofline": {"kernel": "attn_fwd_kernel", "bound": "tensor", "achieved": achieved,
                      "peak": pk["bf16_tflops"], "unit": UNIT,
                      "frac": achieved / pk["bf16_tflops"], "traffic": profiled_traffic(),
@@ -419,16 +491,21 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
                      # (a GEMM looped for seconds at the 1 kW limit).
                      "frac_of_sustained": (achieved / pk["bf16_tflops_sustained"]
                                            if pk["bf16_tflops_sustained"] else None)},
-        "attn_ms": {"median": statistics.median(attn_ms),
-                    "p95": sorted(attn_ms)[int(0.95 * (K - 1))]},
-        "projection": {"ms_median": statistics.median(proj_ms),
-                       "achieved_gbs": w.project_bytes() / proj_mean_s / 1e9,
-                       "peak_gbs": pk["hbm_gbs"],
-                       "frac": w.project_bytes() / proj_mean_s / 1e9 / pk["hbm_gbs"]},
+        "attn_ms": {"median": 1e3 * attn_med_s,
+                    "p95": sorted(attn_ms)[int(0.95 * (K - 1))],
+                    "tflops_median": flops / attn_med_s / 1e12,
+                    "pct_of_peak_median": 100.0 * flops / attn_med_s / 1e12 / pk["bf16_tflops"],
+                    "algorithmic_gbs": attn_bytes / attn_med_s / 1e9},
         "clocks": clocks,
     }
+    if pair_mode:
+        proj_mean_s = statistics.mean(proj_ms) / 1e3
+        line["projection"] = {"ms_median": statistics.median(proj_ms),
+                              "achieved_gbs": proj_bytes / proj_mean_s / 1e9,
+                              "peak_gbs": pk["hbm_gbs"],
+                              "frac": proj_bytes / proj_mean_s / 1e9 / pk["hbm_gbs"]}
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w)
+        line["cpu_baseline"] = cpu_baseline(layers)
     print(json.dumps(line), flush=True)
 
 
@@ -521,6 +598,8 @@ def main() -> None:
                          "backward: the attention backward alone, one GPU")
     ap.add_argument("--workload", choices=sorted(ag_inputs.WORKLOADS), default="full",
                     help="with --path backward: which workload (default full, L=8192)")
+    ap.add_argument("--config", choices=CONFIGS + ("all",), default="full",
+                    help="forward workload (default full: L=8192, B=1, the headline line)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.steps is None:
@@ -532,6 +611,8 @@ def main() -> None:
             ap.error("--path backward runs our kernels on one GPU")
     elif args.workload != "full":
         ap.error("--workload applies to --path backward only")
+    if args.path == "backward" and args.config != "full":
+        ap.error("--config applies to --path forward")
     if args.path == "backward":
         run_backward(args)
         return
@@ -541,16 +622,20 @@ def main() -> None:
     if world != args.gpus:
         if world == 1 and args.gpus > 1:
             sys.exit("--gpus N > 1 must be launched with torchrun (one process per GPU)")
+    configs = CONFIGS if args.config == "all" else (args.config,)
     if args.impl == "reference":
         # Rank 0 alone times the oracle; the other ranks exit without work.
-        run_reference(args, rank, world)
+        for c in configs:
+            run_reference(argparse.Namespace(**{**vars(args), "config": c}), rank, world)
         return
     if world > 1:
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group(
             backend="nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        run_ours(args, rank, world, local_rank)
+        for c in configs:
+            run_ours(argparse.Namespace(**{**vars(args), "config": c}), rank, world, local_rank)
+            torch.cuda.empty_cache()
     finally:
         if world > 1:
             torch.distributed.barrier()

@@ -13,8 +13,10 @@
  * Conventions shared by every entry point:
  *   - Every pointer argument is a DEVICE pointer unless stated otherwise,
  *     row-major, densely packed.  The caller allocates and owns all inputs
- *     and outputs.  The only memory the library allocates itself is the
- *     attention scratch described at ag_attn_fwd.
+ *     and outputs.  The library allocates no device memory: calls keep no
+ *     state on the device besides the error word below (and the static array
+ *     of ag_attn_fwd_noalloc), so independent calls may run concurrently on
+ *     different streams.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Calls are asynchronous on that stream: AG_OK means the work
  *     was enqueued.  Faults inside a kernel surface at the caller's next
@@ -108,14 +110,15 @@ ag_status ag_pair_bias_project(const float *pair, const float *W, float *bias,
  * the probabilities are rounded to bf16 for the second product while the
  * row sums use their fp32 values.
  *
- * Scratch: to keep every SM busy to the end, a pair of query tiles may have
- * its keys split between SM pairs (the kernel runs on 2-CTA clusters); each
- * piece's partial result goes through a scratch buffer of 197,632 bytes per
- * SM (29.2 MB on a 148-SM B200; at most half of it is used) and a second
- * kernel on the same stream merges the pieces (by log-sum-exp).  The
- * first call on a device allocates that buffer with cudaMalloc; it is kept
- * until the process exits.  Calls whose kernels overlap on the device (e.g.
- * on two streams at once) must not run concurrently, because they share it.
+ * Schedule: the kernel runs one 2-CTA cluster per SM pair, each taking
+ * whole pairs of 16-position query blocks.  When those do not divide evenly
+ * over the SM pairs (e.g. L = 8192, B = 1: 256 pairs on 74 SM pairs), some
+ * pairs have their keys split in two: the first piece runs in the first
+ * launch and writes its normalised partial result to out/lse, the second
+ * piece runs in a second launch on the same stream (programmatic dependent
+ * launch, so it starts on the SMs the first launch frees) and merges the
+ * first piece's result with its own by log-sum-exp.  No scratch memory is
+ * used, so calls on different streams may overlap freely.
  */
 ag_status ag_attn_fwd(const void *q, const void *k, const void *v,
                       const float *bias, int64_t B, int64_t H, int64_t L,
@@ -156,27 +159,31 @@ ag_status ag_attn_fwd_ex(const void *q, const void *k, const void *v,
                          float cap, float *out, float *lse, void *stream);
 
 /*
- * ag_attn_fwd_noalloc -- ag_attn_fwd for callers that cannot allocate device
- * memory (the pages have no counterpart; this is a library convenience).
+ * ag_attn_fwd_noalloc -- the attention forward on the range schedule, for
+ * callers that cannot allocate device memory (the pages have no counterpart;
+ * this is a library convenience).
  *
- * Same arguments, checks, results and stream behaviour as ag_attn_fwd, but
- * it never calls cudaMalloc or cudaFree: its split-pair scratch is a static
- * device array compiled into the library, 148 slots of 197,632 bytes
- * (29,249,536 bytes), which every GPU that loads the library holds until the
- * process exits.  Useful where an allocation is not allowed or not wanted,
- * e.g. code that must not touch the allocator while a CUDA graph is being
- * captured, or a framework that has handed all device memory to its own pool.
+ * Same arguments, checks and stream behaviour as ag_attn_fwd, and the same
+ * results within the tolerances of the forward (the schedule differs, so the
+ * fp32 sums are grouped differently).  Its schedule cuts the (pair, key tile)
+ * steps into equal contiguous runs, one per SM pair, and merges the pieces of
+ * split pairs in a second kernel; those pieces need scratch, which here is a
+ * static device array compiled into the library, 148 slots of 197,632 bytes
+ * (29,249,536 bytes).  Callers for whom a library must not allocate: a
+ * framework that has handed all device memory to its own pool, or a process
+ * whose device memory budget is fixed at start-up.  The array is loaded with
+ * the library's module for this entry point (lazy module loading: on the
+ * first call) and stays on that GPU until the process exits.
  *
  *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     (cudaGetSymbolAddress) with that device current.
  *   - Returns AG_ERR_SCRATCH, launching nothing, when the call would use more
  *     than 148 slots (one per 2-CTA cluster of its grid: min(SM count / 2,
  *     work steps)), i.e. on a device with more than 296 SMs.
  *   - Every call shares the one array and it keeps the last call's contents;
- *     nothing in it needs to start at zero.  Calls that overlap on the GPU
- *     (two streams at once, or together with ag_attn_fwd's kernels on another
- *     stream of the same device) race on it and must not be issued.
+ *     nothing in it needs to start at zero.  Calls of this entry point that
+ *     overlap on the GPU (two streams at once) race on it and must not be
+ *     issued; calls of the other entry points do not touch it.
  */
 ag_status ag_attn_fwd_noalloc(const void *q, const void *k, const void *v,
                               const float *bias, int64_t B, int64_t H, int64_t L,
@@ -184,18 +191,42 @@ ag_status ag_attn_fwd_noalloc(const void *q, const void *k, const void *v,
                               float *lse, void *stream);
 
 /*
- * ag_attn_fwd_launch_count -- how many kernels ag_attn_fwd (or
- * ag_attn_fwd_noalloc) launches for these sizes on the current device: 0 for
- * an empty call, 1, or 2 when some pair of query tiles has its keys split
- * between SM pairs and the merge kernel runs as well (a library convenience
- * for callers that count launches; the pages have no counterpart).
- * Same size and value checks, and statuses, as ag_attn_fwd; count is a host
- * pointer (AG_ERR_NULL if NULL).  Launches nothing.  The count holds for
- * ag_attn_fwd_ex at either value width too: both widths run one CTA per SM,
- * so they get the same grid.
+ * ag_attn_fwd_launch_count -- how many kernels ag_attn_fwd (and
+ * ag_attn_fwd_strided_bias, ag_attn_fwd_ex) launches for these sizes on the
+ * current device: 0 for an empty call, 1, or 2 when some pairs of query tiles
+ * have their keys split in two and a second launch merges them (a library
+ * convenience for callers that count launches; the pages have no
+ * counterpart).  Same size and value checks, and statuses, as ag_attn_fwd;
+ * count is a host pointer (AG_ERR_NULL if NULL).  Launches nothing.  The
+ * count holds at either value width: both widths run one CTA per SM, so
+ * they get the same grid.
  */
 ag_status ag_attn_fwd_launch_count(int64_t B, int64_t H, int64_t L, int64_t D,
                                    int64_t block, float cap, int *count);
+
+/*
+ * ag_attn_fwd_schedule -- the work schedule of the attention forward for B
+ * items of length L on a device with sm_pairs resident 2-CTA clusters (a
+ * library convenience for inspecting and testing the host-side planner; the
+ * pages have no counterpart).  Pure host logic: needs no GPU, launches
+ * nothing.  Work unit: a "pair" is two 16-position query blocks of one item
+ * (B * ceil(ceil(L/16)/2) pairs), each over n_kt = ceil(L/128) key tiles.
+ *   with_scratch == 0 (ag_attn_fwd, _strided_bias, _ex): *sched = 1.  The
+ *     first launch has *clusters clusters; cluster c runs whole pairs
+ *     [wb[c], wb[c+1]) and then the first pieces (key tiles [0, *split_at))
+ *     of split pairs [fb[c], fb[c+1]); split pair s is pair *n_whole + s.  If
+ *     *tail_clusters > 0, a second launch has that many clusters and cluster
+ *     c runs the second piece (key tiles [*split_at, n_kt)) of split pair c.
+ *   with_scratch != 0 (ag_attn_fwd_noalloc's schedule): *sched = 0, the
+ *     (pair, key tile) steps in *clusters equal contiguous runs (*whole = 1:
+ *     rounded to whole pairs); wb, fb unused.
+ * wb and fb are host arrays of 129 ints (written).  Statuses: AG_ERR_NULL
+ * for a NULL pointer; the size checks of ag_attn_fwd (H = 8, D = 128,
+ * block = 16); AG_ERR_SHAPE for B == 0, L == 0 or sm_pairs < 1.
+ */
+ag_status ag_attn_fwd_schedule(int64_t B, int64_t L, int sm_pairs, int with_scratch,
+                               int *sched, int *clusters, int *tail_clusters, int *whole,
+                               int *n_whole, int *split_at, int *wb, int *fb);
 
 /*
  * ag_attn_bwd -- gradients of ag_attn_fwd_ex's out for an upstream gradient

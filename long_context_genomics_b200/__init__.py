@@ -68,6 +68,10 @@ def _load() -> ctypes.CDLL:
     lib.ag_attn_fwd_launch_count.argtypes = [i64, i64, i64, i64, i64, f32,
                                              ctypes.POINTER(ctypes.c_int)]
     lib.ag_attn_fwd_launch_count.restype = ctypes.c_int
+    ip = ctypes.POINTER(ctypes.c_int)
+    lib.ag_attn_fwd_schedule.argtypes = [i64, i64, ctypes.c_int, ctypes.c_int, ip, ip, ip,
+                                         ip, ip, ip, ip, ip]
+    lib.ag_attn_fwd_schedule.restype = ctypes.c_int
     lib.ag_attn_bwd.argtypes = [vp, vp, vp, vp, i64, vp, vp, i64, i64, i64, i64, i64,
                                 i64, f32, vp, vp, vp, vp, vp, vp]
     lib.ag_attn_bwd.restype = ctypes.c_int

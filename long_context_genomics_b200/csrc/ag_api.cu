@@ -21,18 +21,11 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
-struct DeviceInfo {
-  bool ready = false;
-  bool sm100 = false;
-  int num_sms = 0;
-  unsigned *err = nullptr;  // device address of g_device_error_word
-  void *scratch = nullptr;  // attention split-pair scratch (one slot per SM)
-  void *static_scratch = nullptr;  // device address of g_static_attn_scratch
-};
-
 std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
 EncodeTiledFn g_encode = nullptr;
+
+}  // namespace
 
 // Per-device set-up, done once with that device current.
 ag_status device_info(DeviceInfo **out) {
@@ -65,20 +58,6 @@ ag_status device_info(DeviceInfo **out) {
   return AG_OK;
 }
 
-// The attention kernel's scratch, allocated with cudaMalloc on the first call
-// that needs it on this device and kept until the process exits.
-ag_status device_scratch(DeviceInfo *d, void **out) {
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (!d->scratch) {
-    void *p = nullptr;
-    const size_t bytes = attn_scratch_bytes(d->num_sms);
-    if (cudaMalloc(&p, bytes) != cudaSuccess) return AG_ERR_CUDA;
-    d->scratch = p;
-  }
-  *out = d->scratch;
-  return AG_OK;
-}
-
 ag_status get_encoder(EncodeTiledFn *fn) {
   std::lock_guard<std::mutex> lock(g_mu);
   if (!g_encode) {
@@ -91,28 +70,6 @@ ag_status get_encoder(EncodeTiledFn *fn) {
     g_encode = reinterpret_cast<EncodeTiledFn>(p);
   }
   *fn = g_encode;
-  return AG_OK;
-}
-
-// Scratch for ag_attn_fwd_noalloc: the same split-pair slots as the
-// allocated scratch, for at most kStaticScratchSlots clusters, in a file-scope
-// array that every device loading this library holds until the process exits.
-constexpr int kStaticScratchSlots = 148;
-constexpr size_t kStaticScratchBytes =
-    kStaticScratchSlots * (kAttnSlotOutBytes + kAttnSlotLseBytes);
-static __device__ __align__(256) unsigned char g_static_attn_scratch[kStaticScratchBytes];
-
-// Device address of g_static_attn_scratch for the current device, looked up
-// once per device (host code may not use the symbol itself as an address).
-ag_status static_scratch(DeviceInfo *d, void **out) {
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (!d->static_scratch) {
-    void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_static_attn_scratch) != cudaSuccess || !p)
-      return AG_ERR_CUDA;
-    d->static_scratch = p;
-  }
-  *out = d->static_scratch;
   return AG_OK;
 }
 
@@ -131,6 +88,8 @@ bool overlap(const void *a, uint64_t na, const void *b, uint64_t nb) {
 // A failure from an earlier asynchronous launch is sticky; it is reported
 // here rather than attributed to the next call.
 ag_status from_cuda(cudaError_t e) { return e == cudaSuccess ? AG_OK : AG_ERR_CUDA; }
+
+namespace {
 
 __global__ void wait_timeout_probe_kernel(uint64_t timeout_ns, unsigned *err) {
   __shared__ uint64_t bar;
@@ -196,16 +155,21 @@ ag_status ag_pair_bias_project(const float *pair, const float *W, float *bias,
   ag::DeviceInfo *dev = nullptr;
   ag_status st = ag::device_info(&dev);
   if (st != AG_OK) return st;
+  ag::EncodeTiledFn enc = nullptr;
+  st = ag::get_encoder(&enc);
+  if (st != AG_OK) return st;
   return ag::from_cuda(ag::launch_pair_bias_project(
-      pair, W, bias, P, dev->num_sms, dev->err, static_cast<cudaStream_t>(stream)));
+      pair, W, bias, P, dev->num_sms, dev->err, enc, static_cast<cudaStream_t>(stream)));
 }
+
+}  // extern "C"
 
 namespace ag {
 // Size and value checks shared by the attention entry points, in order:
 // shapes, then cap, then what the kernels support (including the work-step
 // bound: pairs of query tiles x key tiles must stay below 2^30).
-static ag_status check_attn_sizes(int64_t B, int64_t H, int64_t L, int64_t D,
-                                  int64_t block, float cap) {
+ag_status check_attn_sizes(int64_t B, int64_t H, int64_t L, int64_t D, int64_t block,
+                           float cap) {
   if (B < 0 || H <= 0 || L < 0 || D <= 0 || block <= 0) return AG_ERR_SHAPE;
   if (std::isnan(cap) || !(cap > 0.0f)) return AG_ERR_VALUE;
   if (H != 8 || D != 128 || block != 16 || L > 65536) return AG_ERR_UNSUPPORTED;
@@ -232,6 +196,8 @@ static ag_status check_value_width_and_bias_stride(int64_t B, int64_t H, int64_t
   return AG_OK;
 }
 }  // namespace ag
+
+extern "C" {
 
 ag_status ag_attn_fwd(const void *q, const void *k, const void *v,
                       const float *bias, int64_t B, int64_t H, int64_t L,
@@ -284,9 +250,6 @@ ag_status ag_attn_fwd_ex(const void *q, const void *k, const void *v,
   ag::EncodeTiledFn enc = nullptr;
   st = ag::get_encoder(&enc);
   if (st != AG_OK) return st;
-  void *scratch = nullptr;
-  st = ag::device_scratch(dev, &scratch);
-  if (st != AG_OK) return st;
   ag::AttnLaunch a;
   a.q = q;
   a.k = k;
@@ -301,69 +264,8 @@ ag_status ag_attn_fwd_ex(const void *q, const void *k, const void *v,
   a.cap = cap;
   a.err = dev->err;
   a.num_sms = dev->num_sms;
-  a.scratch = scratch;
-  a.scratch_slots = dev->num_sms;
-  a.encode = enc;
-  a.stream = static_cast<cudaStream_t>(stream);
-  return ag::from_cuda(ag::launch_attn_fwd(a));
-}
-
-ag_status ag_attn_fwd_noalloc(const void *q, const void *k, const void *v,
-                              const float *bias, int64_t B, int64_t H, int64_t L,
-                              int64_t D, int64_t block, float cap, float *out,
-                              float *lse, void *stream) {
-  // The same checks, in the same order, as ag_attn_fwd.
-  const ag_status vs = ag::check_attn_sizes(B, H, L, D, block, cap);
-  if (vs != AG_OK) return vs;
-  if (B == 0 || L == 0) return AG_OK;
-  if (!q || !k || !v || !bias || !out || !lse) return AG_ERR_NULL;
-  if (!ag::aligned(q, 16) || !ag::aligned(k, 16) || !ag::aligned(v, 16) ||
-      !ag::aligned(bias, 4) || !ag::aligned(out, 16) || !ag::aligned(lse, 4))
-    return AG_ERR_ALIGN;
-  const uint64_t P = static_cast<uint64_t>((L + block - 1) / block);
-  const uint64_t qb = static_cast<uint64_t>(B) * H * L * D * 2;
-  const uint64_t kb = static_cast<uint64_t>(B) * L * D * 2;
-  const uint64_t bb = static_cast<uint64_t>(H) * P * P * 4;
-  const uint64_t ob = static_cast<uint64_t>(B) * H * L * D * 4;
-  const uint64_t lb = static_cast<uint64_t>(B) * H * L * 4;
-  const void *ins[4] = {q, k, v, bias};
-  const uint64_t insz[4] = {qb, kb, kb, bb};
-  for (int t = 0; t < 4; ++t)
-    if (ag::overlap(out, ob, ins[t], insz[t]) || ag::overlap(lse, lb, ins[t], insz[t]))
-      return AG_ERR_ALIAS;
-  if (ag::overlap(out, ob, lse, lb)) return AG_ERR_ALIAS;
-  ag::DeviceInfo *dev = nullptr;
-  ag_status st = ag::device_info(&dev);
-  if (st != AG_OK) return st;
-  // One scratch slot per cluster; the grid is one 2-CTA cluster per SM pair
-  // (fewer for tiny problems).  A device whose grid would need more slots
-  // than the static buffer holds is refused rather than given a slower grid.
-  const int64_t steps = ag::attn_work_steps(B, L);
-  const int64_t pairs_of_sms = dev->num_sms / 2;
-  const int64_t slots = steps < pairs_of_sms ? steps : pairs_of_sms;
-  if (slots > ag::kStaticScratchSlots) return AG_ERR_SCRATCH;
-  ag::EncodeTiledFn enc = nullptr;
-  st = ag::get_encoder(&enc);
-  if (st != AG_OK) return st;
-  void *scratch = nullptr;
-  st = ag::static_scratch(dev, &scratch);
-  if (st != AG_OK) return st;
-  ag::AttnLaunch a;
-  a.q = q;
-  a.k = k;
-  a.v = v;
-  a.bias = bias;
-  a.bias_bstride = 0;
-  a.out = out;
-  a.lse = lse;
-  a.B = B;
-  a.L = L;
-  a.Dv = D;
-  a.cap = cap;
-  a.err = dev->err;
-  a.num_sms = dev->num_sms;
-  a.scratch = scratch;
-  a.scratch_slots = ag::kStaticScratchSlots;
+  a.scratch = nullptr;  // whole pairs or two launches: no scratch
+  a.scratch_slots = 0;
   a.encode = enc;
   a.stream = static_cast<cudaStream_t>(stream);
   return ag::from_cuda(ag::launch_attn_fwd(a));
@@ -382,9 +284,22 @@ ag_status ag_attn_fwd_launch_count(int64_t B, int64_t H, int64_t L, int64_t D,
   ag_status st = ag::device_info(&dev);
   if (st != AG_OK) return st;
   int n = 0;
-  st = ag::from_cuda(ag::attn_fwd_kernel_count(B, L, D, cap, dev->num_sms, dev->num_sms, &n));
+  st = ag::from_cuda(ag::attn_fwd_kernel_count(B, L, D, cap, dev->num_sms, 0, &n));
   if (st != AG_OK) return st;
   *count = n;
+  return AG_OK;
+}
+
+ag_status ag_attn_fwd_schedule(int64_t B, int64_t L, int sm_pairs, int with_scratch,
+                               int *sched, int *clusters, int *tail_clusters, int *whole,
+                               int *n_whole, int *split_at, int *wb, int *fb) {
+  if (!sched || !clusters || !tail_clusters || !whole || !n_whole || !split_at || !wb || !fb)
+    return AG_ERR_NULL;
+  const ag_status vs = ag::check_attn_sizes(B, 8, L, 128, 16, 5.0f);
+  if (vs != AG_OK) return vs;
+  if (B == 0 || L == 0 || sm_pairs < 1) return AG_ERR_SHAPE;
+  ag::attn_fwd_schedule(B, L, sm_pairs, with_scratch ? sm_pairs : 0, sched, clusters,
+                        tail_clusters, whole, n_whole, split_at, wb, fb);
   return AG_OK;
 }
 

@@ -13,37 +13,44 @@
 //    heads.  Every row of the tile shares one 16-position bias row block and
 //    all 8 heads consume the same K/V tile (multi-query sharing).
 //  * Two SMs work as a pair (a 2-CTA cluster) on a pair of query tiles: each
-//    CTA holds one tile, and one thread of the even CTA issues tcgen05.mma
-//    with cta_group::2, M = 256 rows over both SMs.  Each CTA stages only half
-//    of every K tile (64 of its 128 keys) and half of every V tile (DV/2 of
-//    the DV value columns), so each K/V byte crosses from L2 into one SM only
-//    and serves the 256 query rows of the pair, and one MMA instruction keeps
-//    both tensor cores busy.  DV (value width) is 128 or 192.
-//  * One persistent cluster per SM pair takes a contiguous, equal share of all
-//    (pair, key tile) steps; a pair whose key range is split between clusters
-//    is merged exactly from the pieces' partial results by log-sum-exp (see
-//    "Split pairs" below).
-//  * Inside each CTA: a producer warp streams its Q tile and a ring of K and V
-//    halves with TMA (no multicast); the softmax warpgroups own 32- or 64-key
-//    chunks of the key tiles (see "Softmax warpgroups").  In the odd CTA the MMA warp relays
-//    "loaded" to the even CTA (a cluster-scope arrive), so each CTA's copies
-//    complete on its own barriers and can be drained locally.
+//    CTA holds one tile, and tcgen05.mma with cta_group::2 covers M = 256 rows
+//    over both SMs.  Each CTA stages only half of every K tile (64 of its 128
+//    keys) and half of every V tile (DV/2 value columns), so each K/V byte
+//    crosses from L2 into one SM only and serves the 256 query rows of the
+//    pair.  DV (value width) is 128 or 192.
 //  * Tensor memory (per CTA): two 128-column S buffers (fp32 logits of
-//    alternate key tiles) and the DV-column O accumulator.  P is written as
-//    bf16 over part of its S buffer and fed to the PV product straight from
-//    tensor memory.  With S double-buffered the MMA order per key tile is
-//    PV(j), S(j+2): the logits a softmax warp needs next were computed while
-//    it worked on the current ones.
-//  * Bias: each softmax thread owns one row, so per key tile it needs just
-//    the two compact cells of its 32 keys, read from global (L2) one tile
-//    ahead and kept in registers; the 16x repeat is never built.
-//  * With a finite cap every logit lies in (-cap, cap), so the softmax uses
-//    the fixed shift m = cap (exact: softmax is shift invariant) and needs no
-//    running max and no rescaling of O.  cap > 40 (where exp(-2 cap) would
-//    underflow fp32) and cap = +inf use a running max with lazy rescaling.
+//    alternate key tiles), one or two 64-column P buffers (bf16 probabilities
+//    of a key tile) and the DV-column O accumulator.  Because P has buffers of
+//    its own, the logits S(j+2) can be computed as soon as the softmax has
+//    read S(j) into registers, long before PV(j) runs: the tensor core always
+//    holds the next logits when the softmax wants them.
+//  * Two MMA-issuing threads in the even CTA: one issues every S = Q K^T and
+//    one every O += P V, each with its own waits and commits, fed by separate
+//    K and V rings (TMA, no multicast).  In the odd CTA two relay threads
+//    forward "loaded" to the even CTA (cluster-scope arrives), so each CTA's
+//    copies complete on its own barriers and can be drained locally.
+//  * All four softmax warpgroups work on every key tile, 32 keys each; the
+//    bias of a thread's 32 keys is two compact cells, read from global (L2)
+//    one tile ahead and kept in registers: the 16x repeat is never built.
+//  * With a finite cap every logit lies in (-cap, cap), so the softmax uses a
+//    fixed shift (exact: softmax is shift invariant) and needs no running max
+//    and no rescaling of O.  cap > 40 (where exp(-2 cap) would underflow fp32)
+//    and cap = +inf use a running max with lazy rescaling.
+//  * Work is cut into segments (a pair of query tiles and a run of its key
+//    tiles).  Three schedules: whole pairs per cluster; "two phases", where
+//    some pairs are split into a first piece (first launch, result written to
+//    out/lse) and a second piece (second launch, programmatic dependent
+//    launch, merged with the first piece's result in its epilogue) so that
+//    the grid stays balanced without any scratch memory; and contiguous
+//    ranges of (pair, key tile) steps whose split pieces go through a
+//    caller-provided scratch buffer and a merge kernel.
 //  * Every mbarrier wait is bounded (sm100.cuh); on timeout the kernel records
 //    the wait site in the device error word, drains its own copies and MMAs,
 //    frees tensor memory and returns.
+#include <algorithm>
+#include <mutex>
+#include <vector>
+
 #include "ag_internal.h"
 #include "sm100.cuh"
 
@@ -56,16 +63,13 @@ constexpr int kKeys = static_cast<int>(kAttnKeyTile);  // keys per key tile
 static_assert(kKeys == 128, "the tile layout below assumes 128-key tiles");
 constexpr int kQTileBytes = 128 * kD * 2;     // this CTA's query tile (bf16)
 constexpr int kQHalfBytes = kQTileBytes / 2;  // one 64-wide (128-byte) half
-// A step load is what one key-tile step needs from this CTA: its half of a
-// V tile (128 keys x DV/2 value columns; VLayout below) and its half of the K
-// tile two steps ahead (64 keys x 128, two 64-wide halves of 8 KB), or, first in a
-// segment, the halves of the segment's first two K tiles.  A ring slot holds
-// two consecutive step loads, so the MMA thread waits for data and releases
-// it once per two steps (each mbarrier operation costs it about 180 cycles
-// while the tensor core is busy, measured).
-constexpr int kPartBytes = 16384;            // one K half
-constexpr int kKHalfBytes = kPartBytes / 2;  // a K half's 64-wide half
+constexpr int kKTileBytes = 64 * kD * 2;      // this CTA's 64 keys of a K tile
+constexpr int kKHalfBytes = kKTileBytes / 2;  // one 64-wide half of them
+// Ring slots hold two consecutive key tiles, so each issuing thread waits
+// for data and releases it once per two tiles (each mbarrier operation costs
+// the issuing thread about 180 cycles, measured).
 constexpr int kStages = 2;
+constexpr int kTilesPerSlot = 2;
 
 // This CTA's half of a V tile, 128 keys x DV/2 value columns, MN-major for
 // the PV product.  DV = 128: one 128-byte-swizzled 64-column box.  DV = 192
@@ -76,44 +80,53 @@ constexpr int kStages = 2;
 template <int DV> struct VLayout;
 template <> struct VLayout<128> {
   static constexpr int kBoxes = 1, kBoxCols = 64;
-  static constexpr int kPartBytes = 128 * 64 * 2;       // 16 KB
+  static constexpr int kTileBytes = 128 * 64 * 2;       // 16 KB
   static constexpr uint32_t kDescHi = desc_sw128_hi(1024);
   static constexpr uint32_t kAtomBytes = 16384;         // LBO (one atom: unused)
   static constexpr uint32_t kKStepBytes = 16 * 128;     // 16 keys x 128 B
 };
 template <> struct VLayout<192> {
   static constexpr int kBoxes = 3, kBoxCols = 32;
-  static constexpr int kPartBytes = 128 * 96 * 2;       // 24 KB
+  static constexpr int kTileBytes = 128 * 96 * 2;       // 24 KB
   static constexpr uint32_t kDescHi = desc_sw64_hi(512);
   static constexpr uint32_t kAtomBytes = 8192;          // LBO: 32-column atoms
   static constexpr uint32_t kKStepBytes = 16 * 64;      // 16 keys x 64 B
 };
-// A step load: a K half (part 0) and a V half or a second K half (part 1).
-template <int DV> constexpr int step_bytes() { return kPartBytes + VLayout<DV>::kPartBytes; }
-template <int DV> constexpr int slot_bytes() { return 2 * step_bytes<DV>(); }
-static_assert(step_bytes<128>() >= 2 * kPartBytes && step_bytes<192>() >= 2 * kPartBytes,
-              "step load 0 holds two K halves");
+constexpr int kKSlotBytes = kTilesPerSlot * kKTileBytes;
+template <int DV> constexpr int v_slot_bytes() {
+  return kTilesPerSlot * VLayout<DV>::kTileBytes;
+}
+
+// Tensor-memory columns: S buffer u at 128 u; P buffer p (bf16 pairs, 64
+// columns for 128 keys) at 256 + 64 p; O (DV columns) after the P buffers.
+// DV = 128: 2 S + 2 P + O = 512 columns; DV = 192: 2 S + 1 P + O = 512.
+template <int DV> struct Tmem {
+  static constexpr int kNP = DV == 128 ? 2 : 1;
+  static constexpr uint32_t kColP = 256;
+  static constexpr uint32_t kColO = 256 + 64 * kNP;
+};
+static_assert(Tmem<128>::kColO + 128 <= 512 && Tmem<192>::kColO + 192 <= 512,
+              "tensor memory budget");
+constexpr uint32_t kTmemCols = 512;
+
 constexpr int kWG = 4;                      // softmax warpgroups
 constexpr int kSoftThreads = 128 * kWG;
 constexpr int kSoftWarps = 4 * kWG;         // per CTA
 constexpr int kPairSoftWarps = 2 * kSoftWarps;
+constexpr int kWarpLoadQK = 4 * kWG;        // TMA: Q and K
+constexpr int kWarpIssueS = 4 * kWG + 1;    // even CTA: S issuer; odd: Q/K relay
+constexpr int kWarpIssuePV = 4 * kWG + 2;   // even CTA: PV issuer; odd: V relay
+constexpr int kWarpLoadV = 4 * kWG + 3;     // TMA: V
 constexpr int kNumWarps = 4 * kWG + 4;
 constexpr int kThreads = kNumWarps * 32;
-constexpr int kWarpLoad = 4 * kWG;          // TMA producer
-constexpr int kWarpMma = 4 * kWG + 1;       // MMA issuer (even CTA) / relay (odd)
 // Registers per thread: the launch gives every thread kRegsLaunch (the cap
 // for this block size, which ptxas allocates when setmaxnreg is present; the
-// launcher checks it); the producer warpgroup then drops to kRegsLow (with
-// fewer the MMA and relay threads spill).  The softmax keeps the launch count.
+// launcher checks it); the loader/issuer warpgroup then drops to kRegsLow.
+// The softmax keeps the launch count.
 constexpr uint32_t kRegsLaunch = 96;
 constexpr uint32_t kRegsLow = 88;
 static_assert(kSoftThreads * kRegsLaunch + 128 * kRegsLow <= kThreads * kRegsLaunch,
               "register split exceeds the launch allocation");
-constexpr uint32_t kTmemCols = 512;
-// Tensor-memory columns: S buffer u at 128 u, O at 256 (DV columns).  P (bf16
-// pairs) of chunk c (keys [32c, 32c + 32) of the tile) is written over the
-// first 16 columns of that chunk's own S columns, [32c, 32c + 16).
-constexpr uint32_t kColO = 256;
 constexpr uint32_t kIdescQK = idesc_bf16_f32(256, kKeys, 0);  // K-major B (K)
 template <int DV> constexpr uint32_t idesc_pv() { return idesc_bf16_f32(256, DV, 1); }
 constexpr float kLog2e = 1.4426950408889634f;
@@ -121,49 +134,65 @@ constexpr float kLn2 = 0.6931471805599453f;
 // Lazy rescale threshold (log2 units) for the running-max modes.
 constexpr float kRescaleThreshold = 8.0f;
 
-enum Mode { kStaticCap = 0, kOnlineCap = 1, kNoCap = 2 };
+// Softmax modes.  kStaticFast: finite cap up to kFastCapMax, tanh on the
+// special-function unit (tanh.approx, whose absolute error times the cap
+// bounds the logit error).  kStaticAcc: larger finite caps up to 40, the
+// capped logit from the logistic form below (every step to about 1e-7).
+// kOnline: cap > 40, the same logistic form with a running max.  kNoCap.
+enum Mode { kStaticFast = 0, kStaticAcc = 1, kOnline = 2, kNoCap = 3 };
 
 // Wait sites recorded in the device error word.
 enum Site : unsigned {
-  kSiteProdQ = 1, kSiteProdKV = 2, kSiteMmaQ = 3, kSiteMmaKV = 4,
-  kSiteMmaP = 5, kSiteSoftS = 6, kSiteSoftO = 7, kSiteDrain = 8,
-  kSiteXchg = 9, kSiteSoftPV = 10, kSiteRelay = 11
+  kSiteProdQ = 1, kSiteProdK = 2, kSiteIssueQ = 3, kSiteIssueK = 4,
+  kSiteIssueP = 5, kSiteSoftS = 6, kSiteSoftO = 7, kSiteDrain = 8,
+  kSiteXchg = 9, kSiteSoftPV = 10, kSiteRelay = 11, kSiteProdV = 12,
+  kSiteIssueV = 13, kSiteIssueSFree = 14
 };
 
-// Per-CTA barriers.  In the even CTA, q_full and kv_full also count the odd
-// CTA's relay (two arrivals: the local producer's, with the byte count, and
-// the relay's), so the MMA thread waits once for both halves of a load;
-// p_full is used in the even CTA only (the odd CTA's softmax warps arrive on
-// it remotely).  q_empty, kv_empty, s_full, pv_done and o_full are signalled
-// in both CTAs by the even CTA's MMA commits.
+// Per-CTA barriers.  In the even CTA, q_full, k_full and v_full also count
+// the odd CTA's relay (two arrivals: the local producer's, with the byte
+// count, and the relay's), so an issuing thread waits once for both halves
+// of a load; s_free and p_full are used in the even CTA only (the odd CTA's
+// softmax warps arrive on them remotely).  q_empty, k_empty, v_empty, s_full,
+// pv_done and o_full are signalled in both CTAs by the even CTA's commits.
 struct __align__(8) Barriers {
   uint64_t q_full, q_empty;
-  uint64_t kv_full[kStages], kv_empty[kStages];
-  // s_full / p_full by S buffer: a softmax may finish key tile j + 1 before
-  // the MMA warp has taken key tile j's arrivals.
-  uint64_t s_full[2], p_full[2];
-  uint64_t pv_done, o_full;
+  uint64_t k_full[kStages], k_empty[kStages];
+  uint64_t v_full[kStages], v_empty[kStages];
+  uint64_t s_full[2], s_free[2];
+  uint64_t p_full[2], pv_done[2];  // [Tmem<DV>::kNP] in use
+  uint64_t o_full;
   uint64_t xm, xd;  // row-max / row-sum exchange between the warpgroups
-  uint64_t drain;
+  uint64_t drain;   // both issuing threads' MMAs have completed
   uint32_t tmem_base;
   int abort;
-  int range_begin, range_end;  // this cluster's (pair, key tile) steps
 };
 
-// Softmax-side shared memory: row-max (per step, double-buffered by step
-// parity) and row-sum (per segment) exchange between the four chunks.
+// Softmax-side shared memory: row-max (per key tile, double-buffered by tile
+// parity) and row-sum (per segment) exchange between the four warpgroups.
 struct Xchg {
-  float mpart[2][kWG][128];  // [step parity][chunk][row]
-  float dpart[kWG][128];     // [chunk][row]
+  float mpart[2][kWG][128];  // [tile parity][warpgroup][row]
+  float dpart[kWG][128];     // [warpgroup][row]
 };
 
 template <int DV> constexpr size_t smem_bytes() {
-  return 1024 + static_cast<size_t>(kQTileBytes) +
-         kStages * static_cast<size_t>(slot_bytes<DV>()) + sizeof(Barriers) +
-         sizeof(Xchg);
+  return 1024 + static_cast<size_t>(kQTileBytes) + kStages * static_cast<size_t>(kKSlotBytes) +
+         kStages * static_cast<size_t>(v_slot_bytes<DV>()) + sizeof(Barriers) + sizeof(Xchg);
 }
 static_assert(smem_bytes<128>() <= 227 * 1024 && smem_bytes<192>() <= 227 * 1024,
               "shared memory budget");
+
+// --------------------------------------------------------------------------
+// Work schedules.  A segment is one pair of query tiles (an "item": batch
+// item b = item / pairs, query blocks 2 (item % pairs) and the next) and a
+// run [kb, ke) of its key tiles; every role of a cluster walks the same
+// segment sequence.
+enum Sched { kSchedRange = 0, kSchedUnits = 1, kSchedTail = 2 };
+// Where a segment's normalised result goes: out/lse (a whole pair, or the
+// first piece of a split one); this cluster's scratch slot (a later piece of
+// a split pair under kSchedRange, merged by attn_merge_kernel); or merged
+// into out/lse with the first piece's result (kSchedTail).
+enum Dest { kDestOut = 0, kDestScratch = 1, kDestMerge = 2 };
 
 struct Params {
   const float *bias;
@@ -171,36 +200,45 @@ struct Params {
   float *out;
   float *lse;
   unsigned *err;
-  // Split-pair scratch (see "Split pairs"): one slot per cluster.
-  float *ws_out;       // [clusters][2][128][DV] partial outputs
-  float *ws_lse;       // [clusters][2][128] partial log-sum-exps
+  float *ws_out;       // kSchedRange scratch: [clusters][2][128][DV] partial outputs
+  float *ws_lse;       //                      [clusters][2][128] partial log-sum-exps
   int L, P;
   int nb;          // 16-position query blocks per batch item, ceil(L / 16)
   int pairs;       // query-tile pairs per batch item: ceil(nb / 2)
   int n_items;     // B * pairs
   int n_kt;        // key tiles: ceil(L / 128)
   int last_valid;  // valid keys in the last key tile (1..128)
-  int whole;       // 1: cluster ranges hold whole pairs (no split pairs)
+  int sched;       // Sched
+  int whole;       // kSchedRange: cluster ranges hold whole pairs
+  int n_whole;     // kSchedUnits/Tail: items [0, n_whole) run whole; item
+                   // n_whole + s is split pair s
+  int split_at;    // split pairs: first piece key tiles [0, split_at), second
+                   // piece [split_at, n_kt)
   float qk_scale;  // multiplies q.k
   float bias_mul;  // multiplies the compact bias
   float A;         // capped modes: cap * log2(e)
+  float shift;     // static modes: the fixed shift (log2 units, an integer >= A)
+  // kSchedUnits: cluster c runs whole items [wb[c], wb[c+1]) and then the
+  // first pieces of split pairs [fb[c], fb[c+1]).
+  int wb[kAttnMaxClusters + 1];
+  int fb[kAttnMaxClusters + 1];
 };
 
-// --------------------------------------------------------------------------
-// Work split.  The W = n_items * n_kt (pair, key tile) steps are cut into
-// one contiguous range per cluster, [W c / G, W (c+1) / G) for cluster c of
-// G.  Both CTAs of a cluster walk the range as segments: one pair and a run
-// of its key tiles.  A pair covered by more than one cluster is "split".
 struct Segment {
-  int item, kb, ke;  // pair index and key tiles [kb, ke)
+  int item, kb, ke, dest;
+};
+
+struct Cursor {
+  int a, a_end, f, f_end;
 };
 
 __device__ __forceinline__ int num_clusters() { return static_cast<int>(gridDim.x >> 1); }
 __device__ __forceinline__ int cluster_index() { return static_cast<int>(blockIdx.x >> 1); }
 
-// W = n_items * n_kt <= 2^30 (checked by the launcher), so steps fit in int;
-// only the range bounds need a 64-bit product.  With p.whole the bounds are
-// rounded to whole pairs: cluster c gets pairs [n_items c / G, n_items (c+1) / G).
+// kSchedRange: the W = n_items * n_kt (pair, key tile) steps are cut into
+// one contiguous range per cluster, [W c / G, W (c+1) / G) for cluster c of G
+// (W <= 2^30, checked by the launcher; only the bounds need 64 bits).  With
+// p.whole the bounds are rounded to whole pairs.
 __device__ __forceinline__ int range_start(const Params &p, int c) {
   const long long G = num_clusters();
   if (p.whole)
@@ -208,41 +246,58 @@ __device__ __forceinline__ int range_start(const Params &p, int c) {
   return static_cast<int>(static_cast<long long>(p.n_items) * p.n_kt * c / G);
 }
 
-__device__ __forceinline__ Segment segment_at(const Params &p, int t, int end) {
-  Segment sg;
-  sg.item = t / p.n_kt;
-  sg.kb = t - sg.item * p.n_kt;
-  const int left = end - t;
-  sg.ke = left < p.n_kt - sg.kb ? sg.kb + left : p.n_kt;
-  return sg;
+__device__ __forceinline__ Cursor cursor_begin(const Params &p) {
+  const int c = cluster_index();
+  Cursor cu;
+  if (p.sched == kSchedRange) {
+    cu.a = range_start(p, c);
+    cu.a_end = range_start(p, c + 1);
+    cu.f = cu.f_end = 0;
+  } else if (p.sched == kSchedUnits) {
+    cu.a = p.wb[c];
+    cu.a_end = p.wb[c + 1];
+    cu.f = p.fb[c];
+    cu.f_end = p.fb[c + 1];
+  } else {  // kSchedTail: the second piece of split pair c
+    cu.a = c;
+    cu.a_end = c + 1;
+    cu.f = cu.f_end = 0;
+  }
+  return cu;
 }
 
-// K/V ring order, shared by the producers, the relay and the MMA warp: for a
-// segment with key tiles [kb, ke) (n of them), step load 0 holds K(kb) (part
-// 0) and K(kb+1) (part 1); step load i = 1 .. n holds K(kb+i+1) (part 0,
-// while it exists) and V(kb+i-1) (part 1).  S runs two key tiles ahead of PV.
-// Step loads 2d and 2d+1 share ring slot load d (the last may be alone).
-struct StepLoad {
-  int k_tile;  // K tile in part 0, or -1
-  int second;  // V tile (is_v) or K tile in part 1, or -1
-  bool is_v;
-};
-__device__ __forceinline__ StepLoad step_load(const Segment &sg, int i) {
-  const int n = sg.ke - sg.kb;
-  if (i == 0) return {sg.kb, n > 1 ? sg.kb + 1 : -1, false};
-  return {sg.kb + i + 1 < sg.ke ? sg.kb + i + 1 : -1, sg.kb + i - 1, true};
-}
-// f(first step load, last step load) for every ring slot load of the segment.
-template <typename F>
-__device__ __forceinline__ bool for_each_slot_load(const Segment &sg, F &&f) {
-  const int n = sg.ke - sg.kb;
-  bool ok = true;
-  for (int i = 0; i <= n && ok; i += 2) ok = f(i, i + 1 <= n ? i + 1 : i);
-  return ok;
+__device__ __forceinline__ bool next_segment(const Params &p, Cursor &cu, Segment &sg) {
+  if (p.sched == kSchedRange) {
+    if (cu.a >= cu.a_end) return false;
+    sg.item = cu.a / p.n_kt;
+    sg.kb = cu.a - sg.item * p.n_kt;
+    const int left = cu.a_end - cu.a;
+    sg.ke = left < p.n_kt - sg.kb ? sg.kb + left : p.n_kt;
+    sg.dest = sg.kb == 0 ? kDestOut : kDestScratch;
+    cu.a += sg.ke - sg.kb;
+    return true;
+  }
+  if (p.sched == kSchedUnits) {
+    if (cu.a < cu.a_end) {
+      sg = {cu.a, 0, p.n_kt, kDestOut};
+      ++cu.a;
+      return true;
+    }
+    if (cu.f < cu.f_end) {
+      sg = {p.n_whole + cu.f, 0, p.split_at, kDestOut};
+      ++cu.f;
+      return true;
+    }
+    return false;
+  }
+  if (cu.a >= cu.a_end) return false;
+  sg = {p.n_whole + cu.a, p.split_at, p.n_kt, kDestMerge};
+  ++cu.a;
+  return true;
 }
 
 // --------------------------------------------------------------------------
-// MMA issue helpers (single thread of the even CTA).
+// MMA issue helpers (issuing threads of the even CTA).
 
 // Shared-memory descriptors: every operand here has 8-row groups 1 KB apart,
 // so all share one high word; the low word (start address and leading
@@ -251,7 +306,7 @@ __device__ __forceinline__ bool for_each_slot_load(const Segment &sg, F &&f) {
 constexpr uint32_t kDescHi = desc_sw128_hi(1024);
 
 // S[256 x 128] = Q[256 x 128] K^T over the pair: eight K=16 steps over the two
-// 64-wide halves of each CTA's Q tile (16 KB apart) and K half (8 KB apart).
+// 64-wide halves of each CTA's Q tile (16 KB apart) and K tile (8 KB apart).
 __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_addr,
                                          uint32_t k_addr) {
   const uint32_t q_lo = desc_sw128_lo(q_addr, 16), k_lo = desc_sw128_lo(k_addr, 16);
@@ -264,19 +319,17 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_addr,
 }
 
 // O[256 x DV] (+)= P[256 x 128 keys] V[128 keys x DV]: P from each CTA's
-// tensor memory (bf16 pairs, 8 columns per 16 keys; keys 32c.. of chunk c
-// start at column 32c of the S buffer), V MN-major: each CTA holds DV/2 value
-// columns for all 128 keys (VLayout).
+// tensor memory (bf16 pairs, 8 columns per 16 keys, keys in column order),
+// V MN-major: each CTA holds DV/2 value columns for all 128 keys (VLayout).
 template <int DV>
-__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t s_tmem,
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem,
                                          uint32_t v_addr, bool accumulate) {
   using VL = VLayout<DV>;
   const uint32_t v_lo = desc_sw128_lo(v_addr, VL::kAtomBytes);
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk) {
-    umma2_ts_lo(d_tmem, s_tmem + 32 * (kk >> 1) + 8 * (kk & 1),
-                v_lo + ((kk * VL::kKStepBytes) >> 4), VL::kDescHi, idesc_pv<DV>(),
-                (accumulate || kk > 0) ? 1u : 0u);
+    umma2_ts_lo(d_tmem, p_tmem + 8 * kk, v_lo + ((kk * VL::kKStepBytes) >> 4), VL::kDescHi,
+                idesc_pv<DV>(), (accumulate || kk > 0) ? 1u : 0u);
   }
 }
 
@@ -298,181 +351,206 @@ __device__ __forceinline__ int tile_block(const Params &p, int I0, uint32_t rank
 }
 
 // --------------------------------------------------------------------------
-// Producer warp, lane 0 (each CTA): TMA loads of this CTA's Q tile and of its
-// halves of the K and V tiles.
-template <int DV>
-__device__ __forceinline__ void producer(const CUtensorMap *tm_q,
-                                         const CUtensorMap *tm_k,
-                                         const CUtensorMap *tm_v, uint8_t *q_s,
-                                         uint8_t *kv_s, Barriers *bars,
-                                         const Params &p, uint32_t rank,
-                                         volatile int *abort) {
+// Producer warps, lane 0 (each CTA): TMA loads of this CTA's Q tile and of
+// its halves of the K tiles (producer_qk), and of its halves of the V tiles
+// (producer_v).  Key tiles [j0, j0 + 2) of a segment share a ring slot.
+__device__ __forceinline__ void producer_qk(const CUtensorMap *tm_q, const CUtensorMap *tm_k,
+                                            uint8_t *q_s, uint8_t *k_s, Barriers *bars,
+                                            const Params &p, uint32_t rank,
+                                            volatile int *abort) {
   const uint64_t pol_q = l2_policy_evict_first();
-  const uint64_t pol_kv = l2_policy_evict_last();
-  uint32_t qcount = 0, kv = 0;
+  const uint64_t pol_k = l2_policy_evict_last();
+  uint32_t qc = 0, kl = 0;
   bool ok = true;
-  const int end = bars->range_end;
-  for (int t = bars->range_begin; t < end && ok;) {
-    const Segment sg = segment_at(p, t, end);
-    t += sg.ke - sg.kb;
+  Cursor cu = cursor_begin(p);
+  Segment sg;
+  while (ok && next_segment(p, cu, sg)) {
     const int b = sg.item / p.pairs;
     const int I0 = (sg.item % p.pairs) * 2;
-    ok = mbar_wait(&bars->q_empty, (qcount & 1u) ^ 1u, abort, p.err, kSiteProdQ);
+    ok = mbar_wait(&bars->q_empty, (qc & 1u) ^ 1u, abort, p.err, kSiteProdQ);
     if (!ok) break;
     mbar_arrive_expect_tx(&bars->q_full, kQTileBytes);
     const int qrow = tile_block(p, I0, rank) * 16;
     tma_load_4d(q_s, tm_q, &bars->q_full, 0, qrow, 0, b, pol_q);
     tma_load_4d(q_s + kQHalfBytes, tm_q, &bars->q_full, 64, qrow, 0, b, pol_q);
-    ++qcount;
-    ok = for_each_slot_load(sg, [&](int i0, int i1) {
-      const uint32_t slot = kv % kStages, ph = (kv / kStages) & 1u;
-      if (!mbar_wait(&bars->kv_empty[slot], ph ^ 1u, abort, p.err, kSiteProdKV))
-        return false;
-      uint32_t bytes = 0;
-      for (int i = i0; i <= i1; ++i) {
-        const StepLoad sl = step_load(sg, i);
-        bytes += (sl.k_tile >= 0 ? kPartBytes : 0) +
-                 (sl.second < 0 ? 0 : sl.is_v ? VLayout<DV>::kPartBytes : kPartBytes);
+    ++qc;
+    for (int j0 = sg.kb; j0 < sg.ke; j0 += kTilesPerSlot) {
+      const uint32_t slot = kl % kStages, ph = (kl / kStages) & 1u;
+      ok = mbar_wait(&bars->k_empty[slot], ph ^ 1u, abort, p.err, kSiteProdK);
+      if (!ok) break;
+      const int nt = sg.ke - j0 < kTilesPerSlot ? sg.ke - j0 : kTilesPerSlot;
+      mbar_arrive_expect_tx(&bars->k_full[slot], static_cast<uint32_t>(nt) * kKTileBytes);
+      for (int t = 0; t < nt; ++t) {
+        // Keys [128 j + 64 rank, +64), all 128 columns, as two 64-wide halves.
+        uint8_t *dst = k_s + slot * kKSlotBytes + t * kKTileBytes;
+        const int key0 = (j0 + t) * kKeys + 64 * static_cast<int>(rank);
+        tma_load_3d(dst, tm_k, &bars->k_full[slot], 0, key0, b, pol_k);
+        tma_load_3d(dst + kKHalfBytes, tm_k, &bars->k_full[slot], 64, key0, b, pol_k);
       }
-      mbar_arrive_expect_tx(&bars->kv_full[slot], bytes);
-      // A K half: keys [128 j + 64 rank, +64), all 128 columns.
-      auto load_k = [&](uint8_t *to, int j) {
-        const int key0 = j * kKeys + 64 * static_cast<int>(rank);
-        tma_load_3d(to, tm_k, &bars->kv_full[slot], 0, key0, b, pol_kv);
-        tma_load_3d(to + kKHalfBytes, tm_k, &bars->kv_full[slot], 64, key0, b, pol_kv);
-      };
-      for (int i = i0; i <= i1; ++i) {
-        const StepLoad sl = step_load(sg, i);
-        uint8_t *dst = kv_s + slot * slot_bytes<DV>() + (i & 1) * step_bytes<DV>();
-        if (sl.k_tile >= 0) load_k(dst, sl.k_tile);
-        if (sl.is_v) {  // keys [128 j, +128), value columns [DV/2 rank, +DV/2)
-#pragma unroll
-          for (int a = 0; a < VLayout<DV>::kBoxes; ++a)
-            tma_load_3d(dst + kPartBytes + a * VLayout<DV>::kAtomBytes, tm_v,
-                        &bars->kv_full[slot],
-                        (DV / 2) * static_cast<int>(rank) + a * VLayout<DV>::kBoxCols,
-                        sl.second * kKeys, b, pol_kv);
-        } else if (sl.second >= 0) {
-          load_k(dst + kPartBytes, sl.second);
-        }
-      }
-      ++kv;
-      return true;
-    });
+      ++kl;
+    }
   }
   // Every copy this thread started must land before the CTA exits.
-  if (qcount > 0) drain_wait(&bars->q_full, (qcount - 1) & 1u);
-  const uint32_t first = kv > kStages ? kv - kStages : 0;
-  for (uint32_t i = first; i < kv; ++i)
-    drain_wait(&bars->kv_full[i % kStages], (i / kStages) & 1u);
+  if (qc > 0) drain_wait(&bars->q_full, (qc - 1) & 1u);
+  for (uint32_t i = kl > kStages ? kl - kStages : 0; i < kl; ++i)
+    drain_wait(&bars->k_full[i % kStages], (i / kStages) & 1u);
+}
+
+template <int DV>
+__device__ __forceinline__ void producer_v(const CUtensorMap *tm_v, uint8_t *v_s,
+                                           Barriers *bars, const Params &p, uint32_t rank,
+                                           volatile int *abort) {
+  using VL = VLayout<DV>;
+  const uint64_t pol_v = l2_policy_evict_last();
+  uint32_t vl = 0;
+  bool ok = true;
+  Cursor cu = cursor_begin(p);
+  Segment sg;
+  while (ok && next_segment(p, cu, sg)) {
+    const int b = sg.item / p.pairs;
+    for (int j0 = sg.kb; j0 < sg.ke; j0 += kTilesPerSlot) {
+      const uint32_t slot = vl % kStages, ph = (vl / kStages) & 1u;
+      ok = mbar_wait(&bars->v_empty[slot], ph ^ 1u, abort, p.err, kSiteProdV);
+      if (!ok) break;
+      const int nt = sg.ke - j0 < kTilesPerSlot ? sg.ke - j0 : kTilesPerSlot;
+      mbar_arrive_expect_tx(&bars->v_full[slot], static_cast<uint32_t>(nt) * VL::kTileBytes);
+      for (int t = 0; t < nt; ++t) {
+        // Keys [128 j, +128), value columns [DV/2 rank, +DV/2).
+        uint8_t *dst = v_s + slot * v_slot_bytes<DV>() + t * VL::kTileBytes;
+#pragma unroll
+        for (int a = 0; a < VL::kBoxes; ++a)
+          tma_load_3d(dst + a * VL::kAtomBytes, tm_v, &bars->v_full[slot],
+                      (DV / 2) * static_cast<int>(rank) + a * VL::kBoxCols,
+                      (j0 + t) * kKeys, b, pol_v);
+      }
+      ++vl;
+    }
+  }
+  for (uint32_t i = vl > kStages ? vl - kStages : 0; i < vl; ++i)
+    drain_wait(&bars->v_full[i % kStages], (i / kStages) & 1u);
 }
 
 // --------------------------------------------------------------------------
-// MMA warp of the odd CTA, lane 0: tells the even CTA's MMA thread, in ring
-// order, that this CTA's half of each Q / K / V load has landed.
-__device__ __forceinline__ void relay(Barriers *bars, const Params &p,
-                                      volatile int *abort) {
+// Relays of the odd CTA, lane 0: tell the even CTA's issuing threads, in
+// ring order, that this CTA's half of each Q / K load (relay_qk) or V load
+// (relay_v) has landed.
+__device__ __forceinline__ void relay_qk(Barriers *bars, const Params &p, volatile int *abort) {
   const uint32_t q_leader = cluster_addr(&bars->q_full, 0);
-  uint32_t qcount = 0, kv = 0;
+  uint32_t qc = 0, kl = 0;
   bool ok = true;
-  const int end = bars->range_end;
-  for (int t = bars->range_begin; t < end && ok;) {
-    const Segment sg = segment_at(p, t, end);
-    t += sg.ke - sg.kb;
-    ok = mbar_wait(&bars->q_full, qcount & 1u, abort, p.err, kSiteRelay);
-    ++qcount;
+  Cursor cu = cursor_begin(p);
+  Segment sg;
+  while (ok && next_segment(p, cu, sg)) {
+    ok = mbar_wait(&bars->q_full, qc & 1u, abort, p.err, kSiteRelay);
+    ++qc;
     if (!ok) break;
     mbar_arrive_cluster(q_leader);
-    ok = for_each_slot_load(sg, [&](int, int) {
-      const uint32_t slot = kv % kStages;
-      if (!mbar_wait(&bars->kv_full[slot], (kv / kStages) & 1u, abort, p.err,
-                     kSiteRelay))
-        return false;
-      ++kv;
-      mbar_arrive_cluster(cluster_addr(&bars->kv_full[slot], 0));
-      return true;
-    });
+    for (int j0 = sg.kb; j0 < sg.ke; j0 += kTilesPerSlot) {
+      const uint32_t slot = kl % kStages;
+      ok = mbar_wait(&bars->k_full[slot], (kl / kStages) & 1u, abort, p.err, kSiteRelay);
+      if (!ok) break;
+      ++kl;
+      mbar_arrive_cluster(cluster_addr(&bars->k_full[slot], 0));
+    }
+  }
+}
+
+__device__ __forceinline__ void relay_v(Barriers *bars, const Params &p, volatile int *abort) {
+  uint32_t vl = 0;
+  bool ok = true;
+  Cursor cu = cursor_begin(p);
+  Segment sg;
+  while (ok && next_segment(p, cu, sg)) {
+    for (int j0 = sg.kb; j0 < sg.ke; j0 += kTilesPerSlot) {
+      const uint32_t slot = vl % kStages;
+      ok = mbar_wait(&bars->v_full[slot], (vl / kStages) & 1u, abort, p.err, kSiteRelay);
+      if (!ok) break;
+      ++vl;
+      mbar_arrive_cluster(cluster_addr(&bars->v_full[slot], 0));
+    }
   }
 }
 
 // --------------------------------------------------------------------------
-// MMA warp of the even CTA, lane 0: tcgen05.mma issuer for the pair.
-// kPvDone: also signal pv_done after every PV but the segment's last (the
-// running-max modes rescale O and must know when the previous PV finished).
-template <bool kPvDone, int DV>
-__device__ __forceinline__ void mma_issuer(uint8_t *q_s, uint8_t *kv_s,
-                                           Barriers *bars, uint32_t tmem,
-                                           const Params &p, volatile int *abort) {
-  const uint32_t q_addr = smem_u32(q_s);
-  const uint32_t kv_addr = smem_u32(kv_s);
-  uint32_t qcount = 0, kv = 0;
-  uint32_t pbits = 0;  // bit u: parity of the next p_full[u] phase
-  bool ok = true;
-  // Both halves of the next ring load: this CTA's copy and the peer's relay
-  // (both arrive on this CTA's kv_full).  The odd CTA's arrivals here (relay,
-  // softmax) are relaxed (see mbar_arrive_cluster), so these waits acquire at
-  // CTA scope: a cluster-scope acquire would order nothing more and costs
-  // about 180 cycles per wait on this thread (measured).
-  auto wait_kv = [&](uint32_t &slot) {
-    slot = kv % kStages;
-    const uint32_t ph = (kv / kStages) & 1u;
-    ++kv;
-    return mbar_wait(&bars->kv_full[slot], ph, abort, p.err, kSiteMmaKV);
-  };
-  const int end = bars->range_end;
-  for (int t = bars->range_begin; t < end && ok;) {
-    const Segment sg = segment_at(p, t, end);
-    t += sg.ke - sg.kb;
-    const int n = sg.ke - sg.kb;
-    ok = mbar_wait(&bars->q_full, qcount & 1u, abort, p.err, kSiteMmaQ);
-    ++qcount;
-    if (!ok) break;
-    // Step load 0: S(kb) into buffer 0 and S(kb+1) into buffer 1.
-    uint32_t slot;
-    ok = wait_kv(slot);
-    if (!ok) break;
-    tc_fence_after();
-    {
-      const uint32_t base = kv_addr + slot * slot_bytes<DV>();
-      for (int u = 0; u < 2 && u < n; ++u) {
-        issue_qk(tmem + 128u * u, q_addr, base + u * kPartBytes);
-        umma2_commit_both(&bars->s_full[u]);
-        if (u == n - 1) umma2_commit_both(&bars->q_empty);
-      }
-    }
+// Issuing threads of the even CTA.  The odd CTA's arrivals on their barriers
+// (relays, softmax) are relaxed (see mbar_arrive_cluster), so their waits
+// acquire at CTA scope: a cluster-scope acquire would order nothing more and
+// costs about 180 cycles per wait (measured).
 
-    // Step load i = j - kb + 1: V(j) in part 1, K(j+2) (while it exists) in
-    // part 0; a new ring slot starts at every even i.
+// S = Q K^T for every key tile, into S buffer (use count & 1), once the
+// softmax has read that buffer's previous logits (s_free).
+__device__ __forceinline__ void issuer_s(uint8_t *q_s, uint8_t *k_s, Barriers *bars,
+                                         uint32_t tmem, const Params &p,
+                                         volatile int *abort) {
+  const uint32_t q_addr = smem_u32(q_s), k_addr = smem_u32(k_s);
+  uint32_t qc = 0, kl = 0, su = 0;
+  bool ok = true;
+  Cursor cu = cursor_begin(p);
+  Segment sg;
+  while (ok && next_segment(p, cu, sg)) {
+    ok = mbar_wait(&bars->q_full, qc & 1u, abort, p.err, kSiteIssueQ);
+    ++qc;
+    if (!ok) break;
+    uint32_t slot = 0;
     for (int j = sg.kb; j < sg.ke; ++j) {
-      const int i = j - sg.kb + 1;
-      const uint32_t u = static_cast<uint32_t>(j - sg.kb) & 1u;
+      const int i = j - sg.kb;
       if ((i & 1) == 0) {
-        ok = wait_kv(slot);
+        slot = kl % kStages;
+        ok = mbar_wait(&bars->k_full[slot], (kl / kStages) & 1u, abort, p.err, kSiteIssueK);
+        ++kl;
         if (!ok) break;
       }
-      ok = mbar_wait(&bars->p_full[u], (pbits >> u) & 1u, abort, p.err, kSiteMmaP);
-      pbits ^= 1u << u;
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t base = kv_addr + slot * slot_bytes<DV>() + (i & 1) * step_bytes<DV>();
-      issue_pv<DV>(tmem + kColO, tmem + 128u * u, base + kPartBytes, j > sg.kb);
-      if (j + 1 == sg.ke)
-        umma2_commit_both(&bars->o_full);
-      else if (kPvDone)
-        umma2_commit_both(&bars->pv_done);
-      if (j + 2 < sg.ke) {
-        // S(j+2) over buffer u: issued after PV(j), which reads P(j) from the
-        // same columns (the tensor core runs one thread's MMAs in order).
-        issue_qk(tmem + 128u * u, q_addr, base);
-        umma2_commit_both(&bars->s_full[u]);
-        if (j + 3 == sg.ke) umma2_commit_both(&bars->q_empty);
+      const uint32_t sb = su & 1u, sn = su >> 1;
+      if (sn > 0) {
+        ok = mbar_wait(&bars->s_free[sb], (sn - 1) & 1u, abort, p.err, kSiteIssueSFree);
+        if (!ok) break;
       }
-      if ((i & 1) == 1 || j + 1 == sg.ke) umma2_commit_both(&bars->kv_empty[slot]);
+      tc_fence_after();
+      issue_qk(tmem + 128u * sb, q_addr, k_addr + slot * kKSlotBytes + (i & 1) * kKTileBytes);
+      umma2_commit_both(&bars->s_full[sb]);
+      if (j + 1 == sg.ke) umma2_commit_both(&bars->q_empty);
+      if ((i & 1) == 1 || j + 1 == sg.ke) umma2_commit_both(&bars->k_empty[slot]);
+      ++su;
     }
-    // A segment of one key tile: its only slot holds step loads 0 and 1 and
-    // was released above; otherwise the last slot was released in the loop.
   }
   // All MMAs this thread issued complete before tensor memory is released.
+  umma2_commit_self(&bars->drain);
+  drain_wait(&bars->drain, 0);
+}
+
+// O += P V for every key tile, once the softmax has written P (p_full).
+template <int DV>
+__device__ __forceinline__ void issuer_pv(uint8_t *v_s, Barriers *bars, uint32_t tmem,
+                                          const Params &p, volatile int *abort) {
+  using T = Tmem<DV>;
+  const uint32_t v_addr = smem_u32(v_s);
+  uint32_t vl = 0, pu = 0;
+  bool ok = true;
+  Cursor cu = cursor_begin(p);
+  Segment sg;
+  while (ok && next_segment(p, cu, sg)) {
+    uint32_t slot = 0;
+    for (int j = sg.kb; j < sg.ke; ++j) {
+      const int i = j - sg.kb;
+      if ((i & 1) == 0) {
+        slot = vl % kStages;
+        ok = mbar_wait(&bars->v_full[slot], (vl / kStages) & 1u, abort, p.err, kSiteIssueV);
+        ++vl;
+        if (!ok) break;
+      }
+      const uint32_t pb = pu % T::kNP, pn = pu / T::kNP;
+      ok = mbar_wait(&bars->p_full[pb], pn & 1u, abort, p.err, kSiteIssueP);
+      if (!ok) break;
+      tc_fence_after();
+      issue_pv<DV>(tmem + T::kColO, tmem + T::kColP + 64u * pb,
+                   v_addr + slot * v_slot_bytes<DV>() + (i & 1) * VLayout<DV>::kTileBytes,
+                   i > 0);
+      umma2_commit_both(&bars->pv_done[pb]);
+      if (j + 1 == sg.ke) umma2_commit_both(&bars->o_full);
+      if ((i & 1) == 1 || j + 1 == sg.ke) umma2_commit_both(&bars->v_empty[slot]);
+      ++pu;
+    }
+  }
   umma2_commit_self(&bars->drain);
   drain_wait(&bars->drain, 0);
 }
@@ -480,21 +558,27 @@ __device__ __forceinline__ void mma_issuer(uint8_t *q_s, uint8_t *kv_s,
 // --------------------------------------------------------------------------
 // Softmax warpgroups (each CTA, its own query tile).
 //
-// Thread r of a warpgroup owns tensor-memory lane r, i.e. row r of the tile.
-// Static-cap mode: warpgroups 2q and 2q+1 take the key tiles in S buffer q,
-// 64 keys each.  Running-max modes: warpgroup g takes keys [32g, 32g + 32) of
-// every key tile.  Either way a row's sum is split between four threads and
-// combined through shared memory once per work item (and, in the running-max
-// modes, its maximum once per key tile).  Each 32-key chunk's P goes over
-// the first 16 of its own S columns, so a warpgroup only ever overwrites S
-// columns it has already read itself.
+// Thread r of warpgroup g owns tensor-memory lane r, i.e. row r of the tile,
+// and keys [32 g, 32 g + 32) of every key tile.  A row's sum is split between
+// four threads and combined through shared memory once per segment (and, in
+// the running-max modes, its maximum once per key tile).
 
 // Softmax-side barriers count warps: each warp arrives once, from lane 0,
-// after __syncwarp has ordered its lanes' prior work (one arrival per warp
-// instead of 32 keeps the mbarrier off the shared-memory pipe).
+// after __syncwarp has ordered its lanes' prior work.
 __device__ __forceinline__ void warp_arrive(uint64_t *bar) {
   __syncwarp();
   if (lane_id() == 0) mbar_arrive(bar);
+}
+// The same on a barrier of the even CTA (local, or remote from the odd CTA).
+__device__ __forceinline__ void warp_arrive_leader(uint64_t *bar, uint32_t remote,
+                                                   uint32_t rank) {
+  __syncwarp();
+  if (lane_id() == 0) {
+    if (rank == 0)
+      mbar_arrive(bar);
+    else
+      mbar_arrive_cluster(remote);
+  }
 }
 
 // Publish this thread's value, then wait (bounded) until every softmax thread
@@ -508,7 +592,7 @@ __device__ __forceinline__ bool exchange(uint64_t *bar, uint32_t &count,
   return __all_sync(0xffffffffu, ok);
 }
 
-// The compact bias cells of chunk g of key tile j (two per 32-key chunk):
+// The compact bias cells of warpgroup g's 32 keys of key tile j:
 // bias[h, I, 8j + 2g + e] (0 past the end: those keys are masked).
 __device__ __forceinline__ void load_bias(const float *brow, int j, int g, int P,
                                           float (&bn)[2]) {
@@ -518,35 +602,52 @@ __device__ __forceinline__ void load_bias(const float *brow, int j, int g, int P
 }
 
 // Column pairs (out of every 8) whose exponential runs on the FMA pipe
-// (exp2_poly2) instead of the special-function unit.  The SFU still computes
-// every tanh, so it does 1 + (8 - kEmuPairs) / 8 operations per logit.
+// (exp2_poly2_fma) instead of the special-function unit, in kStaticFast.  The
+// SFU still computes every tanh, so it does 1 + (8 - kEmuPairs) / 8
+// operations per logit.
 #ifndef AG_EXP2_EMU_PAIRS
 #define AG_EXP2_EMU_PAIRS 6
 #endif
 constexpr int kEmuPairs = AG_EXP2_EMU_PAIRS;
 
-// Static-shift softmax of one 32-column chunk: p = 2^(A tanh(y) - A) with
-// y = s * qk_scale + b / cap, two columns at a time.  Adds the row sum into
-// acc and writes 16 bf16 pairs of P.  kMask zeroes columns >= nvalid (only
-// the last key tile of a ragged length needs it).
-template <bool kMask>
-__device__ __forceinline__ void chunk_static(const uint32_t (&s)[32], float b0,
-                                             float b1, float2 sc, float2 ap,
-                                             float2 an, int col0, int nvalid,
+// Constants of the static modes, per thread.
+struct StaticK {
+  float2 sc;     // multiplies s
+  float2 a;      // kStaticFast: A = cap log2(e); kStaticAcc: -2A
+  float2 nsh;    // kStaticFast: -shift (for the SFU pairs)
+  float2 km;     // 1.5 * 2^23 - shift (kStaticFast) or 1.5 * 2^23 (kStaticAcc)
+};
+
+// One thread's 32 keys of a key tile, static shift, log2 units:
+//   kStaticFast: t = tanh(y), p = 2^(A t - shift), y = s qk_scale + b / cap
+//   kStaticAcc:  e = 2^u, u = 2 log2(e) y; p = 2^(-2A / (1 + e))
+//     (cap (tanh y - 1) = -2 cap / (1 + e^{2y}); the fixed shift is A).
+// Adds the row sum into acc and packs 16 bf16 pairs of P.  kMask zeroes keys
+// >= nvalid (only the last key tile of a ragged length needs it).
+template <int MODE, bool kMask>
+__device__ __forceinline__ void chunk_static(const uint32_t (&s)[32], float b0, float b1,
+                                             const StaticK &k, int col0, int nvalid,
                                              float2 &acc, uint32_t (&pk)[16]) {
 #pragma unroll
   for (int e = 0; e < 16; ++e) {
     const float bb = e < 8 ? b0 : b1;
     const float2 y = __ffma2_rn(
-        make_float2(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1])), sc,
+        make_float2(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1])), k.sc,
         make_float2(bb, bb));
-    const float2 t = make_float2(tanh_approx(y.x), tanh_approx(y.y));
-    const float2 x = __ffma2_rn(t, ap, an);
     float2 pr;
-    if ((e & 7) < kEmuPairs) {
-      pr = exp2_poly2(x);
+    if constexpr (MODE == kStaticFast) {
+      const float2 t = make_float2(tanh_approx(y.x), tanh_approx(y.y));
+      if ((e & 7) < kEmuPairs) {
+        pr = exp2_poly2_fma(t, k.a, k.km);
+      } else {
+        const float2 x = __ffma2_rn(t, k.a, k.nsh);
+        pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+      }
     } else {
-      pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+      const float2 den = __fadd2_rn(make_float2(ex2_approx(y.x), ex2_approx(y.y)),
+                                    make_float2(1.f, 1.f));
+      const float2 r = make_float2(rcp_approx(den.x), rcp_approx(den.y));
+      pr = exp2_poly2_fma(r, k.a, k.km);
     }
     if (kMask) {
       if (col0 + 2 * e >= nvalid) pr.x = 0.f;
@@ -557,225 +658,204 @@ __device__ __forceinline__ void chunk_static(const uint32_t (&s)[32], float b0,
   }
 }
 
-// One key tile, static shift: S in, P out over the first 16 columns of this
-// warpgroup's chunk.  Returns the partial row sum.
-template <bool kMask>
-__device__ __forceinline__ float tile_static(uint32_t tS, int col0, float b0,
-                                             float b1, float2 sc, float2 ap,
-                                             float2 an, int nvalid) {
-  float2 acc = make_float2(0.f, 0.f);
-  uint32_t s[32], pk[16];
-  tmem_ld32(tS, s);
-  tmem_wait_ld(s);
-  chunk_static<kMask>(s, b0, b1, sc, ap, an, col0, nvalid, acc, pk);
-  tmem_st16(tS, pk);
-  return acc.x + acc.y;
+// A running-max mode's capped (or uncapped) logit of one key, log2 units.
+template <int MODE>
+__device__ __forceinline__ float online_logit(float s, float bb, const Params &p) {
+  const float y = fmaf(s, p.qk_scale, bb);
+  if constexpr (MODE == kOnline) {
+    // A tanh(y') = A (1 - 2 / (1 + e^{2y'})), with y = 2 log2(e) y'.
+    return fmaf(-2.f * p.A, rcp_approx(1.f + ex2_approx(y)), p.A);
+  } else {
+    return y;
+  }
 }
 
-// One key tile with a running maximum shared by the four threads of each row
-// (exchanged through shared memory).  When the maximum grows past the lazy
-// threshold, this warpgroup's DV/4 columns of O are rescaled, after the
-// previous PV into O has finished (pv_done).
-template <int MODE, int DV>
-__device__ __forceinline__ bool tile_online(uint32_t tS, uint32_t tO, int g,
-                                            int r, uint32_t par, bool o_live,
-                                            uint32_t pv_parity, float b0,
-                                            float b1, const Params &p, int nvalid,
-                                            Xchg *xc, Barriers *bars,
-                                            uint32_t &xcount, volatile int *abort,
-                                            float &m, float &d) {
-  uint32_t s[32];
-  float x[32];
-  tmem_ld32(tS, s);
+// Per-thread pipeline counters of the softmax role.
+struct SoftCounters {
+  uint32_t su = 0;  // S buffer uses (key tiles) so far
+  uint32_t pu = 0;  // P buffer uses so far
+  uint32_t ocount = 0, xmcount = 0, xdcount = 0;
+};
+
+// Waits for the S of the next key tile, loads this thread's 32 logits and
+// releases the S buffer to the S issuer.
+__device__ __forceinline__ bool load_s(Barriers *bars, uint32_t tmem, int g, uint32_t lane_base,
+                                       uint32_t rank, const uint32_t (&sf_remote)[2],
+                                       SoftCounters &c, const Params &p, volatile int *abort,
+                                       uint32_t (&s)[32]) {
+  const uint32_t sb = c.su & 1u, sph = (c.su >> 1) & 1u;
+  ++c.su;
+  const bool ok = mbar_wait(&bars->s_full[sb], sph, abort, p.err, kSiteSoftS);
+  if (!__all_sync(0xffffffffu, ok)) return false;
+  tc_fence_after();
+  tmem_ld32(tmem + 128u * sb + 32u * g + lane_base, s);
   tmem_wait_ld(s);
-  float mt = -INFINITY;
-#pragma unroll
-  for (int e = 0; e < 32; ++e) {
-    const float bb = e < 16 ? b0 : b1;
-    const float y = fmaf(__uint_as_float(s[e]), p.qk_scale, bb);
-    const float v = (MODE == kOnlineCap) ? p.A * tanh_approx(y) : y;
-    x[e] = (32 * g + e < nvalid) ? v : -INFINITY;
-    mt = fmaxf(mt, x[e]);
-  }
-  xc->mpart[par][g][r] = mt;
-  if (!exchange(&bars->xm, xcount, abort, p.err)) return false;
-#pragma unroll
-  for (int q = 0; q < kWG; ++q) mt = fmaxf(mt, xc->mpart[par][q][r]);
-  float factor = 1.f;
-  if (mt > m + kRescaleThreshold || m == -INFINITY) {
-    factor = (m == -INFINITY) ? 0.f : ex2_approx(m - mt);
-    m = mt;
-    d *= factor;
-  }
-  if (o_live && __any_sync(0xffffffffu, factor != 1.f)) {
-    const bool ok = mbar_wait(&bars->pv_done, pv_parity, abort, p.err, kSiteSoftPV);
-    if (!__all_sync(0xffffffffu, ok)) return false;
-    tc_fence_after();
-    uint32_t o[32];
-    tmem_ld32(tO, o);
-    tmem_wait_ld(o);
-#pragma unroll
-    for (int e = 0; e < 32; ++e)
-      o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
-    tmem_st32(tO, o);
-    if constexpr (DV == 192) {  // columns 32 .. 47 of this warpgroup's 48
-      uint32_t o2[16];
-      tmem_ld16(tO + 32, o2);
-      tmem_wait_ld16(o2);
-#pragma unroll
-      for (int e = 0; e < 16; ++e)
-        o2[e] = __float_as_uint(__uint_as_float(o2[e]) * factor);
-      tmem_st16(tO + 32, o2);
-    }
-  }
-  float acc = 0.f;
-  uint32_t pk[16];
-#pragma unroll
-  for (int e = 0; e < 16; ++e) {
-    const float p0 = ex2_approx(x[2 * e] - m);
-    const float p1 = ex2_approx(x[2 * e + 1] - m);
-    acc += p0 + p1;
-    pk[e] = pack_bf16x2(p0, p1);
-  }
-  tmem_st16(tS, pk);
-  d += acc;
+  tc_fence_before();
+  warp_arrive_leader(&bars->s_free[sb], sf_remote[sb], rank);
   return true;
 }
 
-// --------------------------------------------------------------------------
-// Split pairs.  Every segment of a split pair finishes like a whole pair but
-// over its own key range: a normalised partial output and the partial
-// log-sum-exp.  The first segment (key tile 0) writes them to out / lse, the
-// others to the scratch slot of their cluster (a cluster starts at most one
-// segment in the middle of a pair).  attn_merge_kernel, launched right after
-// on the same stream, then merges the pieces of every split pair:
-//   lse = log sum_s exp(lse_s),  out = sum_s exp(lse_s - lse) out_s.
-
-// Static-cap mode: the warps split into two groups that take alternate key
-// tiles (group q = warpgroups 2q, 2q+1 takes the tiles in S buffer q), each
-// warpgroup 64 keys of its group's tiles.  Both S buffers are then in work
-// at once, so one group's waits (for its logits, for its tensor-memory
-// stores, for its arrival) are covered by the other group's arithmetic.
-__device__ __forceinline__ void load_bias4(const float *brow, int j, int hk, int P,
-                                           float (&bn)[4]) {
-  const int J0 = j * 8 + hk * 4;
-#pragma unroll
-  for (int e = 0; e < 4; ++e) bn[e] = (J0 + e < P) ? __ldg(brow + J0 + e) : 0.f;
+// Writes this thread's 16 columns of P into the next P buffer (once the PV
+// that last read it has finished) and tells the PV issuer.
+template <int DV>
+__device__ __forceinline__ bool store_p(Barriers *bars, uint32_t tmem, int g,
+                                        uint32_t lane_base, uint32_t rank,
+                                        const uint32_t (&pf_remote)[2], SoftCounters &c,
+                                        const Params &p, volatile int *abort,
+                                        const uint32_t (&pk)[16]) {
+  using T = Tmem<DV>;
+  const uint32_t pb = c.pu % T::kNP, pn = c.pu / T::kNP;
+  ++c.pu;
+  if (pn > 0) {
+    const bool ok = mbar_wait(&bars->pv_done[pb], (pn - 1) & 1u, abort, p.err, kSiteSoftPV);
+    if (!__all_sync(0xffffffffu, ok)) return false;
+  }
+  tc_fence_after();
+  tmem_st16(tmem + T::kColP + 64u * pb + 16u * g + lane_base, pk);
+  tmem_wait_st();
+  tc_fence_before();
+  warp_arrive_leader(&bars->p_full[pb], pf_remote[pb], rank);
+  return true;
 }
 
+// Static-shift segment: every warpgroup takes 32 keys of every key tile.
+template <int MODE, int DV>
 __device__ __forceinline__ bool segment_static(const Segment &sg, const float *brow,
-                                               uint32_t tmem, uint32_t lane_base,
-                                               int g, const Params &p,
-                                               Barriers *bars, uint32_t rank,
-                                               uint32_t pf_remote, uint32_t &scount,
-                                               volatile int *abort, float &d) {
-  const int q = g >> 1, hk = g & 1;  // group (S buffer) and key half
-  const float2 sc = make_float2(p.qk_scale, p.qk_scale);
-  const float2 ap = make_float2(p.A, p.A), an = make_float2(-p.A, -p.A);
-  const int j0 = sg.kb + q;
-  // Bias cells of this group's next tile.  The cells of tile j + 2 are
-  // requested right after tile j's arrival (a load in flight would hold up
-  // that arrival); they land while the group waits for tile j + 2's logits.
-  float bc[4] = {0.f, 0.f, 0.f, 0.f};
-  if (j0 < sg.ke) load_bias4(brow, j0, hk, p.P, bc);
-  for (int j = j0; j < sg.ke; j += 2) {
-    const int nvalid = (j + 1 == p.n_kt) ? p.last_valid : kKeys;
-    bool ok = mbar_wait(&bars->s_full[q], scount & 1u, abort, p.err, kSiteSoftS);
-    ++scount;
-    if (!__all_sync(0xffffffffu, ok)) return false;
-    tc_fence_after();
-    const uint32_t tS = tmem + 128u * q + 64 * hk + lane_base;
-    const float m = p.bias_mul;
-    if (nvalid == kKeys) {
-      d += tile_static<false>(tS, 64 * hk, bc[0] * m, bc[1] * m, sc, ap, an, nvalid);
-      d += tile_static<false>(tS + 32, 64 * hk + 32, bc[2] * m, bc[3] * m, sc, ap, an,
-                              nvalid);
-    } else {
-      d += tile_static<true>(tS, 64 * hk, bc[0] * m, bc[1] * m, sc, ap, an, nvalid);
-      d += tile_static<true>(tS + 32, 64 * hk + 32, bc[2] * m, bc[3] * m, sc, ap, an,
-                             nvalid);
-    }
-    tmem_wait_st();
-    tc_fence_before();
-    __syncwarp();
-    if (lane_id() == 0) {
-      if (rank == 0)
-        mbar_arrive(&bars->p_full[q]);
-      else
-        mbar_arrive_cluster(pf_remote);
-    }
-    if (j + 2 < sg.ke) load_bias4(brow, j + 2, hk, p.P, bc);
+                                               uint32_t tmem, uint32_t lane_base, int g,
+                                               const Params &p, Barriers *bars,
+                                               uint32_t rank, const uint32_t (&sf_remote)[2],
+                                               const uint32_t (&pf_remote)[2],
+                                               SoftCounters &c, volatile int *abort,
+                                               float &d) {
+  StaticK k;
+  k.sc = make_float2(p.qk_scale, p.qk_scale);
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  if constexpr (MODE == kStaticFast) {
+    k.a = make_float2(p.A, p.A);
+    k.nsh = make_float2(-p.shift, -p.shift);
+    k.km = make_float2(kShift - p.shift, kShift - p.shift);
+  } else {
+    k.a = make_float2(-2.f * p.A, -2.f * p.A);
+    k.nsh = make_float2(0.f, 0.f);
+    k.km = make_float2(kShift, kShift);
   }
-  return true;
-}
-
-// Running-max modes: every warpgroup takes every key tile (32 keys each),
-// the four threads of a row sharing its maximum per tile.
-template <int MODE, int DV>
-__device__ __forceinline__ bool segment_online(const Segment &sg, const float *brow,
-                                               uint32_t tmem, uint32_t lane_base,
-                                               int g, int r, const Params &p,
-                                               Barriers *bars, Xchg *xc,
-                                               uint32_t rank, uint32_t pf_remote0,
-                                               uint32_t pf_remote1, uint32_t &scount0,
-                                               uint32_t &scount1, uint32_t &xmcount,
-                                               uint32_t pvd, volatile int *abort,
-                                               float &m, float &d) {
+  float2 acc = make_float2(0.f, 0.f);
   float bc[2], bn[2] = {0.f, 0.f};
   load_bias(brow, sg.kb, g, p.P, bc);
-  if (sg.kb + 1 < sg.ke) load_bias(brow, sg.kb + 1, g, p.P, bn);
   for (int j = sg.kb; j < sg.ke; ++j) {
-    const uint32_t u = static_cast<uint32_t>(j - sg.kb) & 1u;
+    if (j + 1 < sg.ke) load_bias(brow, j + 1, g, p.P, bn);
     const int nvalid = (j + 1 == p.n_kt) ? p.last_valid : kKeys;
+    uint32_t s[32], pk[16];
+    if (!load_s(bars, tmem, g, lane_base, rank, sf_remote, c, p, abort, s)) return false;
     const float b0 = bc[0] * p.bias_mul, b1 = bc[1] * p.bias_mul;
-    const uint32_t sphase = u ? scount1++ : scount0++;
-    bool ok = mbar_wait(&bars->s_full[u], sphase & 1u, abort, p.err, kSiteSoftS);
-    if (!__all_sync(0xffffffffu, ok)) return false;
-    tc_fence_after();
-    const uint32_t tS = tmem + 128u * u + 32 * g + lane_base;
-    const uint32_t tO = tmem + kColO + (DV / 4) * g + lane_base;
-    // PV(j-1) is pv_done phase pvd + (j - 1 - kb); PV(j-2) has finished
-    // (s_full(j) was committed after it), so that phase is the current or
-    // the last completed one and its parity identifies it.
-    const uint32_t pv_parity = (pvd + static_cast<uint32_t>(j - 1 - sg.kb)) & 1u;
-    if (!tile_online<MODE, DV>(tS, tO, g, r, u, j > sg.kb, pv_parity, b0, b1, p, nvalid,
-                           xc, bars, xmcount, abort, m, d))
-      return false;
-    tmem_wait_st();
-    tc_fence_before();
-    __syncwarp();
-    if (lane_id() == 0) {
-      if (rank == 0)
-        mbar_arrive(&bars->p_full[u]);
-      else
-        mbar_arrive_cluster(u ? pf_remote1 : pf_remote0);
-    }
+    if (nvalid == kKeys)
+      chunk_static<MODE, false>(s, b0, b1, k, 32 * g, nvalid, acc, pk);
+    else
+      chunk_static<MODE, true>(s, b0, b1, k, 32 * g, nvalid, acc, pk);
+    if (!store_p<DV>(bars, tmem, g, lane_base, rank, pf_remote, c, p, abort, pk)) return false;
     bc[0] = bn[0];
     bc[1] = bn[1];
-    if (j + 2 < sg.ke) load_bias(brow, j + 2, g, p.P, bn);
+  }
+  d = acc.x + acc.y;
+  return true;
+}
+
+// Running-max segment: the four threads of a row share its maximum per key
+// tile (through shared memory).  When the maximum grows past the lazy
+// threshold, this warpgroup's DV/4 columns of O are rescaled, after the
+// previous PV into O has finished.
+template <int MODE, int DV>
+__device__ __forceinline__ bool segment_online(const Segment &sg, const float *brow,
+                                               uint32_t tmem, uint32_t lane_base, int g, int r,
+                                               const Params &p, Barriers *bars, Xchg *xc,
+                                               uint32_t rank, const uint32_t (&sf_remote)[2],
+                                               const uint32_t (&pf_remote)[2],
+                                               SoftCounters &c, volatile int *abort,
+                                               float &m, float &d) {
+  using T = Tmem<DV>;
+  float bc[2], bn[2] = {0.f, 0.f};
+  load_bias(brow, sg.kb, g, p.P, bc);
+  for (int j = sg.kb; j < sg.ke; ++j) {
+    if (j + 1 < sg.ke) load_bias(brow, j + 1, g, p.P, bn);
+    const int nvalid = (j + 1 == p.n_kt) ? p.last_valid : kKeys;
+    const uint32_t par = c.su & 1u;
+    uint32_t s[32];
+    if (!load_s(bars, tmem, g, lane_base, rank, sf_remote, c, p, abort, s)) return false;
+    const float b0 = bc[0] * p.bias_mul, b1 = bc[1] * p.bias_mul;
+    float x[32];
+    float mt = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const float v = online_logit<MODE>(__uint_as_float(s[e]), e < 16 ? b0 : b1, p);
+      x[e] = (32 * g + e < nvalid) ? v : -INFINITY;
+      mt = fmaxf(mt, x[e]);
+    }
+    xc->mpart[par][g][r] = mt;
+    if (!exchange(&bars->xm, c.xmcount, abort, p.err)) return false;
+#pragma unroll
+    for (int q = 0; q < kWG; ++q) mt = fmaxf(mt, xc->mpart[par][q][r]);
+    float factor = 1.f;
+    if (mt > m + kRescaleThreshold || m == -INFINITY) {
+      factor = (m == -INFINITY) ? 0.f : ex2_approx(m - mt);
+      m = mt;
+      d *= factor;
+    }
+    if (j > sg.kb && __any_sync(0xffffffffu, factor != 1.f)) {
+      // PV(j - 1) used P buffer (pu - 1) % NP; it is that buffer's last phase.
+      const uint32_t prev = c.pu - 1;
+      const bool ok = mbar_wait(&bars->pv_done[prev % T::kNP], (prev / T::kNP) & 1u, abort,
+                                p.err, kSiteSoftPV);
+      if (!__all_sync(0xffffffffu, ok)) return false;
+      tc_fence_after();
+      const uint32_t tO = tmem + T::kColO + (DV / 4) * g + lane_base;
+      // This warpgroup's DV/4 columns, 16 at a time.
+#pragma unroll 1
+      for (int cc = 0; cc < DV / 4; cc += 16) {
+        uint32_t o[16];
+        tmem_ld16(tO + cc, o);
+        tmem_wait_ld16(o);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
+        tmem_st16(tO + cc, o);
+      }
+    }
+    float acc = 0.f;
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float p0 = ex2_approx(x[2 * e] - m);
+      const float p1 = ex2_approx(x[2 * e + 1] - m);
+      acc += p0 + p1;
+      pk[e] = pack_bf16x2(p0, p1);
+    }
+    d += acc;
+    // store_p waits for the stores above (tcgen05.wait::st) before arriving.
+    if (!store_p<DV>(bars, tmem, g, lane_base, rank, pf_remote, c, p, abort, pk)) return false;
+    bc[0] = bn[0];
+    bc[1] = bn[1];
   }
   return true;
 }
 
 template <int MODE, int DV>
-__device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc,
-                                             uint32_t tmem, const Params &p,
-                                             uint32_t rank, volatile int *abort) {
+__device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc, uint32_t tmem,
+                                             const Params &p, uint32_t rank,
+                                             volatile int *abort) {
+  using T = Tmem<DV>;
   const int g = threadIdx.x >> 7;         // warpgroup
   const int r = threadIdx.x & 127;        // tile row == tensor-memory lane
   const int h = r >> 4, il = r & 15;      // head, position inside the block
   const uint32_t lane_base = static_cast<uint32_t>(r >> 5) << 21;  // (32 * quarter) << 16
-  const uint32_t pf_remote0 = cluster_addr(&bars->p_full[0], 0);
-  const uint32_t pf_remote1 = cluster_addr(&bars->p_full[1], 0);
-  uint32_t scount0 = 0, scount1 = 0;  // s_full waits per S buffer
-  uint32_t ocount = 0, xmcount = 0, xdcount = 0;
-  uint32_t pvd = 0;  // pv_done phases completed before this segment
+  const uint32_t sf_remote[2] = {cluster_addr(&bars->s_free[0], 0),
+                                 cluster_addr(&bars->s_free[1], 0)};
+  const uint32_t pf_remote[2] = {cluster_addr(&bars->p_full[0], 0),
+                                 cluster_addr(&bars->p_full[1], 0)};
+  constexpr bool kStatic = (MODE == kStaticFast || MODE == kStaticAcc);
+  SoftCounters c;
   bool ok = true;
-  const int end = bars->range_end;
-
-  for (int t = bars->range_begin; t < end && ok;) {
-    const Segment sg = segment_at(p, t, end);
-    t += sg.ke - sg.kb;
+  Cursor cu = cursor_begin(p);
+  Segment sg;
+  while (ok && next_segment(p, cu, sg)) {
     const int b = sg.item / p.pairs;
     const int I0 = (sg.item % p.pairs) * 2;
     const int I = tile_block(p, I0, rank);
@@ -783,38 +863,45 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc,
     const int pos = I * 16 + il;  // this thread's query position
     const float *brow = p.bias + static_cast<long long>(b) * p.bias_bstride +
                         (static_cast<size_t>(h) * p.P + I) * p.P;
-    float m = (MODE == kStaticCap) ? p.A : -INFINITY;  // log2 units
+    float m = kStatic ? p.shift : -INFINITY;  // log2 units
     float d = 0.f;
-    if constexpr (MODE == kStaticCap) {
-      // A thread of group q only ever waits on S buffer q: scount0 counts
-      // those waits.
-      ok = segment_static(sg, brow, tmem, lane_base, g, p, bars, rank,
-                          (g >> 1) ? pf_remote1 : pf_remote0, scount0, abort, d);
+    if constexpr (kStatic) {
+      ok = segment_static<MODE, DV>(sg, brow, tmem, lane_base, g, p, bars, rank, sf_remote,
+                                    pf_remote, c, abort, d);
     } else {
       ok = segment_online<MODE, DV>(sg, brow, tmem, lane_base, g, r, p, bars, xc, rank,
-                                pf_remote0, pf_remote1, scount0, scount1, xmcount,
-                                pvd, abort, m, d);
+                                    sf_remote, pf_remote, c, abort, m, d);
     }
     if (!ok) break;
-    pvd += static_cast<uint32_t>(sg.ke - sg.kb - 1);
 
     // Epilogue: d = sum of the four warpgroups' partial sums; out = O / d
     // over this segment's keys (warpgroup g writes columns [g DV/4, (g+1)
-    // DV/4) of the row) and lse, to out / lse or, for a later piece of a
-    // split pair, to this cluster's scratch slot.  The copy of block I0 in an
-    // odd CTA past the end of an odd block count writes nothing.
-    ok = mbar_wait(&bars->o_full, ocount & 1u, abort, p.err, kSiteSoftO);
-    ++ocount;
-    if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+    // DV/4) of the row) and lse.  The copy of block I0 in an odd CTA past the
+    // end of an odd block count writes nothing.
+    ok = mbar_wait(&bars->o_full, c.ocount & 1u, abort, p.err, kSiteSoftO);
+    ++c.ocount;
+    if (!__all_sync(0xffffffffu, ok)) {
+      ok = false;
+      break;
+    }
     tc_fence_after();
+    const bool writes = valid && pos < p.L;  // rows past the end of a partial block: none
+    const size_t row = (static_cast<size_t>(b) * kH + h) * p.L + static_cast<size_t>(pos);
+    float lse_a = 0.f;
+    if (sg.dest == kDestMerge) {
+      // The first piece of this pair was written by the previous launch;
+      // every thread reads it before warpgroup 0 overwrites lse below (the
+      // exchange orders the two).
+      griddep_wait();
+      if (writes) lse_a = p.lse[row];
+    }
     xc->dpart[g][r] = d;
-    ok = exchange(&bars->xd, xdcount, abort, p.err);
+    ok = exchange(&bars->xd, c.xdcount, abort, p.err);
     if (!ok) break;
     float dsum = 0.f;
 #pragma unroll
     for (int q = 0; q < kWG; ++q) dsum += xc->dpart[q][r];
-    const float inv_d = 1.f / dsum;
-    const uint32_t tO = tmem + kColO + (DV / 4) * g + lane_base;
+    const uint32_t tO = tmem + T::kColO + (DV / 4) * g + lane_base;
     uint32_t o[32];
     tmem_ld32(tO, o);
     tmem_wait_ld(o);
@@ -823,38 +910,50 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc,
       tmem_ld16(tO + 32, o2);
       tmem_wait_ld16(o2);
     }
-    if (valid && pos < p.L) {  // rows past the end of a partial block: none
-      const size_t row = (static_cast<size_t>(b) * kH + h) * p.L +
-                         static_cast<size_t>(pos);
+    if (writes) {
+      const float lse_b = (m + lg2_approx(dsum)) * kLn2;
       float *orow_base;
       float *lse_dst;
-      if (sg.kb == 0) {
-        orow_base = p.out + row * DV;
-        lse_dst = p.lse + row;
-      } else {
-        const size_t slot =
-            (static_cast<size_t>(cluster_index()) * 2 + rank) * 128 + r;
+      if (sg.dest == kDestScratch) {
+        const size_t slot = (static_cast<size_t>(cluster_index()) * 2 + rank) * 128 + r;
         orow_base = p.ws_out + slot * DV;
         lse_dst = p.ws_lse + slot;
+      } else {
+        orow_base = p.out + row * DV;
+        lse_dst = p.lse + row;
       }
       float4 *orow = reinterpret_cast<float4 *>(orow_base + (DV / 4) * g);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        orow[e] = make_float4(__uint_as_float(o[4 * e]) * inv_d,
-                              __uint_as_float(o[4 * e + 1]) * inv_d,
-                              __uint_as_float(o[4 * e + 2]) * inv_d,
-                              __uint_as_float(o[4 * e + 3]) * inv_d);
+      float wb = 1.f / dsum, wa = 0.f, lse_w = lse_b;
+      if (sg.dest == kDestMerge) {
+        // Log-sum-exp merge with the first piece: lse = log(e^a + e^b),
+        // out = e^(a - lse) out_a + e^(b - lse) O_b / d_b.
+        const float M = fmaxf(lse_a, lse_b);
+        const float ea = ex2_approx((lse_a - M) * kLog2e);
+        const float eb = ex2_approx((lse_b - M) * kLog2e);
+        const float inv = 1.f / (ea + eb);
+        wa = ea * inv;
+        wb = eb * inv / dsum;
+        lse_w = M + lg2_approx(ea + eb) * kLn2;
       }
+      auto put = [&](int e, const uint32_t *v) {
+        float4 val = make_float4(__uint_as_float(v[0]) * wb, __uint_as_float(v[1]) * wb,
+                                 __uint_as_float(v[2]) * wb, __uint_as_float(v[3]) * wb);
+        if (sg.dest == kDestMerge) {
+          const float4 a = orow[e];
+          val.x = fmaf(wa, a.x, val.x);
+          val.y = fmaf(wa, a.y, val.y);
+          val.z = fmaf(wa, a.z, val.z);
+          val.w = fmaf(wa, a.w, val.w);
+        }
+        orow[e] = val;
+      };
+#pragma unroll
+      for (int e = 0; e < 8; ++e) put(e, o + 4 * e);
       if constexpr (DV == 192) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          orow[8 + e] = make_float4(__uint_as_float(o2[4 * e]) * inv_d,
-                                    __uint_as_float(o2[4 * e + 1]) * inv_d,
-                                    __uint_as_float(o2[4 * e + 2]) * inv_d,
-                                    __uint_as_float(o2[4 * e + 3]) * inv_d);
-        }
+        for (int e = 0; e < 4; ++e) put(8 + e, o2 + 4 * e);
       }
-      if (g == 0) *lse_dst = (m + lg2_approx(dsum)) * kLn2;
+      if (g == 0) *lse_dst = lse_w;
     }
     tc_fence_before();
   }
@@ -865,46 +964,50 @@ template <int MODE, int DV>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const Params p) {
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
-  uint8_t *q_s = smem_raw + pad;             // this CTA's query tile
-  uint8_t *kv_s = q_s + kQTileBytes;         // K/V ring
-  Barriers *bars = reinterpret_cast<Barriers *>(kv_s + kStages * slot_bytes<DV>());
-  auto *xc = reinterpret_cast<Xchg *>(reinterpret_cast<uint8_t *>(bars) +
-                                      sizeof(Barriers));
+  uint8_t *q_s = smem_raw + pad;                      // this CTA's query tile
+  uint8_t *k_s = q_s + kQTileBytes;                   // K ring
+  uint8_t *v_s = k_s + kStages * kKSlotBytes;         // V ring
+  Barriers *bars = reinterpret_cast<Barriers *>(v_s + kStages * v_slot_bytes<DV>());
+  auto *xc = reinterpret_cast<Xchg *>(reinterpret_cast<uint8_t *>(bars) + sizeof(Barriers));
   const int warp = threadIdx.x >> 5;
   const uint32_t rank = cluster_ctarank();
 
   if (threadIdx.x == 0) {
+    // A second launch of a two-phase schedule may start once every CTA of
+    // this grid has got here; it only reads this grid's results after
+    // griddepcontrol.wait.
+    griddep_launch_dependents();
     const uint32_t loads = rank == 0 ? 2 : 1;  // producer (+ relay, even CTA)
     mbar_init(&bars->q_full, loads);
     mbar_init(&bars->q_empty, 1);
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bars->kv_full[s], loads);
-      mbar_init(&bars->kv_empty[s], 1);
+      mbar_init(&bars->k_full[s], loads);
+      mbar_init(&bars->k_empty[s], 1);
+      mbar_init(&bars->v_full[s], loads);
+      mbar_init(&bars->v_empty[s], 1);
     }
     for (int u = 0; u < 2; ++u) {
       mbar_init(&bars->s_full[u], 1);
-      // Static cap: one warp group per S buffer; otherwise every warp.
-      mbar_init(&bars->p_full[u], MODE == kStaticCap ? kPairSoftWarps / 2 : kPairSoftWarps);
+      mbar_init(&bars->s_free[u], kPairSoftWarps);
+      mbar_init(&bars->p_full[u], kPairSoftWarps);
+      mbar_init(&bars->pv_done[u], 1);
     }
-    mbar_init(&bars->pv_done, 1);
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->xm, kSoftWarps);
     mbar_init(&bars->xd, kSoftWarps);
-    mbar_init(&bars->drain, 1);
+    mbar_init(&bars->drain, 2);
     bars->abort = 0;
-    bars->range_begin = range_start(p, cluster_index());
-    bars->range_end = range_start(p, cluster_index() + 1);
     fence_mbar_init();
   }
-  if (warp == kWarpLoad && lane_id() == 0) {
+  if (warp == kWarpLoadQK && lane_id() == 0) {
     prefetch_tensormap(&tm_q);
     prefetch_tensormap(&tm_k);
-    prefetch_tensormap(&tm_v);
   }
-  if (warp == kWarpMma) {
+  if (warp == kWarpLoadV && lane_id() == 0) prefetch_tensormap(&tm_v);
+  if (warp == kWarpIssueS) {
     tmem_alloc2(&bars->tmem_base, kTmemCols);
     tmem_relinquish2();
   }
@@ -916,15 +1019,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t tmem = bars->tmem_base;
   volatile int *abort = &bars->abort;
 
-  if (warp >= kWarpLoad) {
+  if (warp >= kWarpLoadQK) {
     regs_dec<kRegsLow>();
-    if (warp == kWarpLoad && lane_id() == 0) {
-      producer<DV>(&tm_q, &tm_k, &tm_v, q_s, kv_s, bars, p, rank, abort);
-    } else if (warp == kWarpMma && lane_id() == 0) {
-      if (rank == 0)
-        mma_issuer<MODE != kStaticCap, DV>(q_s, kv_s, bars, tmem, p, abort);
-      else
-        relay(bars, p, abort);
+    if (lane_id() == 0) {
+      if (warp == kWarpLoadQK) {
+        producer_qk(&tm_q, &tm_k, q_s, k_s, bars, p, rank, abort);
+      } else if (warp == kWarpLoadV) {
+        producer_v<DV>(&tm_v, v_s, bars, p, rank, abort);
+      } else if (warp == kWarpIssueS) {
+        if (rank == 0)
+          issuer_s(q_s, k_s, bars, tmem, p, abort);
+        else
+          relay_qk(bars, p, abort);
+      } else if (warp == kWarpIssuePV) {
+        if (rank == 0)
+          issuer_pv<DV>(v_s, bars, tmem, p, abort);
+        else
+          relay_v(bars, p, abort);
+      }
     }
   } else {
     softmax_role<MODE, DV>(bars, xc, tmem, p, rank, abort);
@@ -935,25 +1047,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   // done once every thread of both CTAs is here.
   tc_fence_before();
   cluster_sync();
-  if (warp == kWarpMma) {
+  if (warp == kWarpIssueS) {
     tc_fence_after();
     tmem_dealloc2(tmem, kTmemCols);
   }
 }
 
 // --------------------------------------------------------------------------
-// Split-pair merge.  kMergeBlocksPerBoundary blocks per cluster boundary; only
-// the boundary that is the first one inside a pair merges that pair.  One
-// warp per output row (query tile row / 128, row % 128): lane l merges the
-// 4-column groups l, l + 32, ... of the row's DV columns over the pieces, and
-// lane 0 writes the merged lse once every lane has read the first piece's.
+// Split-pair merge of kSchedRange.  Every segment of a split pair finishes
+// like a whole pair but over its own key range: a normalised partial output
+// and the partial log-sum-exp.  The first segment (key tile 0) writes them to
+// out / lse, the others to the scratch slot of their cluster (a cluster
+// starts at most one segment in the middle of a pair).  This kernel, launched
+// right after on the same stream, merges the pieces of every split pair:
+//   lse = log sum_s exp(lse_s),  out = sum_s exp(lse_s - lse) out_s.
+// kMergeBlocksPerBoundary blocks per cluster boundary; only the boundary that
+// is the first one inside a pair merges that pair.  One warp per output row
+// (query tile row / 128, row % 128): lane l merges the 4-column groups l,
+// l + 32, ... of the row's DV columns over the pieces, and lane 0 writes the
+// merged lse once every lane has read the first piece's.
 constexpr int kMergeThreads = 256;
 constexpr int kMergeRowsPerBlock = kMergeThreads / 32;
 constexpr int kMergeBlocksPerBoundary = 2 * 128 / kMergeRowsPerBlock;
 
 template <int DV>
 __global__ void __launch_bounds__(kMergeThreads)
-    attn_merge_kernel(const Params p, int grid) {
+    attn_merge_kernel(const __grid_constant__ Params p, int grid) {
   const int c = blockIdx.x / kMergeBlocksPerBoundary + 1;  // boundary between clusters c-1, c
   const int W = p.n_items * p.n_kt;
   auto start = [&](int cc) {
@@ -980,8 +1099,7 @@ __global__ void __launch_bounds__(kMergeThreads)
   const int h = r >> 4, il = r & 15;
   const int pos = (I0 + X) * 16 + il;
   if (pos >= p.L) return;  // past the end of a partial last block
-  const size_t row = (static_cast<size_t>(b) * kH + h) * p.L +
-                     static_cast<size_t>(pos);
+  const size_t row = (static_cast<size_t>(b) * kH + h) * p.L + static_cast<size_t>(pos);
   auto slot = [&](int s) {
     return (static_cast<size_t>(c_first + s) * 2 + X) * 128 + r;
   };
@@ -993,19 +1111,19 @@ __global__ void __launch_bounds__(kMergeThreads)
     sum += ex2_approx(((s == 0 ? p.lse[row] : p.ws_lse[slot(s)]) - M) * kLog2e);
   const float lse = M + lg2_approx(sum) * kLn2;
 #pragma unroll
-  for (int c = lane; c < DV / 4; c += 32) {
+  for (int cc = lane; cc < DV / 4; cc += 32) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int s = 0; s < n_seg; ++s) {
       const float l = s == 0 ? p.lse[row] : p.ws_lse[slot(s)];
       const float wgt = ex2_approx((l - lse) * kLog2e);
       const float4 v = reinterpret_cast<const float4 *>(
-          s == 0 ? p.out + row * DV : p.ws_out + slot(s) * DV)[c];
+          s == 0 ? p.out + row * DV : p.ws_out + slot(s) * DV)[cc];
       acc.x = fmaf(wgt, v.x, acc.x);
       acc.y = fmaf(wgt, v.y, acc.y);
       acc.z = fmaf(wgt, v.z, acc.z);
       acc.w = fmaf(wgt, v.w, acc.w);
     }
-    reinterpret_cast<float4 *>(p.out + row * DV)[c] = acc;
+    reinterpret_cast<float4 *>(p.out + row * DV)[cc] = acc;
   }
   __syncwarp();  // every lane has read p.lse[row]
   if (lane == 0) p.lse[row] = lse;
@@ -1014,7 +1132,7 @@ __global__ void __launch_bounds__(kMergeThreads)
 }  // namespace attn
 
 // --------------------------------------------------------------------------
-// Host launcher.
+// Host side.
 
 static bool encode_map(EncodeTiledFn enc, CUtensorMap *map, const void *base,
                        int rank, const cuuint64_t *dims,
@@ -1029,17 +1147,24 @@ static bool encode_map(EncodeTiledFn enc, CUtensorMap *map, const void *base,
   return r == CUDA_SUCCESS;
 }
 
+namespace {
+
 // One-time per-device setup of a kernel (mode, value width): shared-memory
 // opt-in, the register check, and how many 2-CTA clusters can be resident.
+// The per-device table is written under g_cfg_mu, so two host threads making
+// their first call on a device at once configure it once.
+std::mutex g_cfg_mu;
+constexpr int kCfgDevices = 64;
+
 template <int MODE, int DV>
-static cudaError_t configure_mode(int *max_clusters) {
-  static int configured[64] = {0};
-  static int clusters[64] = {0};
+cudaError_t configure_mode(int *max_clusters) {
+  static int clusters[kCfgDevices] = {0};  // 0: not configured yet
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!configured[dev]) {
+  if (dev < 0 || dev >= kCfgDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_cfg_mu);
+  if (clusters[dev] == 0) {
     // setmaxnreg.dec must lower the count the launch allocated: refuse a
     // build whose allocation is below the launch count the split assumes.
     cudaFuncAttributes fa;
@@ -1060,67 +1185,289 @@ static cudaError_t configure_mode(int *max_clusters) {
     if (e != cudaSuccess) return e;
     if (n < 1) return cudaErrorInvalidConfiguration;
     clusters[dev] = n;
-    configured[dev] = 1;
   }
   *max_clusters = clusters[dev];
   return cudaSuccess;
 }
 
-template <int MODE, int DV>
-static cudaError_t launch_mode(const CUtensorMap &tq, const CUtensorMap &tk,
-                               const CUtensorMap &tv, const attn::Params &p,
-                               int clusters, cudaStream_t stream) {
-  attn::attn_fwd_kernel<MODE, DV>
-      <<<2 * clusters, attn::kThreads, attn::smem_bytes<DV>(), stream>>>(tq, tk, tv, p);
-  return cudaGetLastError();
-}
-
 template <int DV>
-static cudaError_t configure_any(int mode, int *max_clusters) {
+cudaError_t configure_any(int mode, int *max_clusters) {
   using namespace attn;
   switch (mode) {
-    case kStaticCap: return configure_mode<kStaticCap, DV>(max_clusters);
-    case kOnlineCap: return configure_mode<kOnlineCap, DV>(max_clusters);
+    case kStaticFast: return configure_mode<kStaticFast, DV>(max_clusters);
+    case kStaticAcc: return configure_mode<kStaticAcc, DV>(max_clusters);
+    case kOnline: return configure_mode<kOnline, DV>(max_clusters);
     default: return configure_mode<kNoCap, DV>(max_clusters);
   }
 }
 
-// Grid of a call: one 2-CTA cluster per resident SM pair, never more
+// Largest cap that runs the kStaticFast softmax.
+constexpr float kFastCapMax = 10.0f;
+
+int attn_mode(float cap) {
+  using namespace attn;
+  if (std::isinf(cap)) return kNoCap;
+  if (cap <= kFastCapMax) return kStaticFast;
+  return cap <= 40.0f ? kStaticAcc : kOnline;
+}
+
+// --------------------------------------------------------------------------
+// Schedules.
+struct Plan {
+  int sched = attn::kSchedUnits;
+  int clusters = 0;       // first (or only) launch
+  int tail_clusters = 0;  // second launch of a two-phase schedule (0: none)
+  int whole = 1;          // kSchedRange: whole pairs (no merge kernel)
+  int n_whole = 0, split_at = 0;
+  std::vector<int> wb, fb;
+};
+
+// Whole pairs, as evenly as they go: cluster c takes items
+// [n c / G, n (c+1) / G).
+void plan_whole(int n_items, int G, Plan *pl) {
+  const int clusters = std::min(G, n_items);
+  pl->sched = attn::kSchedUnits;
+  pl->clusters = clusters;
+  pl->tail_clusters = 0;
+  pl->n_whole = n_items;
+  pl->split_at = 0;
+  pl->wb.assign(clusters + 1, 0);
+  pl->fb.assign(clusters + 1, 0);
+  for (int c = 0; c <= clusters; ++c)
+    pl->wb[c] = static_cast<int>(static_cast<long long>(n_items) * c / clusters);
+}
+
+// Two-phase packing check for a first launch of at most t key-tile steps per
+// cluster: nw whole pairs (n_kt steps each) and ns first pieces (a steps
+// each, a < n_kt) into G clusters.  Starts from the most whole pairs per
+// cluster and trades whole pairs for first pieces where a trade gains the
+// most (clusters at one level trade alike, so levels are counted, not
+// clusters).  On success gives the per-cluster counts.
+bool pack_first_launch(int t, int nw, int ns, int n_kt, int a, int G, std::vector<int> *x,
+                       std::vector<int> *y) {
+  const int xmax = t / n_kt;
+  if (static_cast<long long>(xmax) * G < nw) return false;
+  auto firsts = [&](int xx) { return (t - xx * n_kt) / a; };
+  std::vector<long long> cnt(xmax + 1, 0);  // clusters holding x whole pairs
+  cnt[xmax] = G;
+  long long spare = static_cast<long long>(xmax) * G - nw;  // removable wholes
+  long long have = static_cast<long long>(G) * firsts(xmax);
+  while (have < ns && spare > 0) {
+    int best = -1, gain = 0;
+    for (int xx = 1; xx <= xmax; ++xx) {
+      if (cnt[xx] == 0) continue;
+      const int g = firsts(xx - 1) - firsts(xx);
+      if (g > gain) {
+        gain = g;
+        best = xx;
+      }
+    }
+    if (best < 0) break;
+    const long long need = (ns - have + gain - 1) / gain;
+    const long long k = std::min({cnt[best], spare, need});
+    cnt[best] -= k;
+    cnt[best - 1] += k;
+    have += k * gain;
+    spare -= k;
+  }
+  if (have < ns) return false;
+  // Clusters in order of decreasing whole pairs; hand out exactly nw wholes
+  // and ns first pieces.
+  x->assign(G, 0);
+  y->assign(G, 0);
+  int c = 0;
+  for (int xx = xmax; xx >= 0; --xx)
+    for (long long i = 0; i < cnt[xx]; ++i) (*x)[c++] = xx;
+  int wl = nw, fl = ns;
+  for (int cc = 0; cc < G; ++cc) {
+    (*x)[cc] = std::min((*x)[cc], wl);
+    wl -= (*x)[cc];
+  }
+  for (int cc = 0; cc < G; ++cc) {
+    (*y)[cc] = std::min(firsts((*x)[cc]), fl);
+    fl -= (*y)[cc];
+  }
+  return wl == 0 && fl == 0;
+}
+
+// Extra cost of a second launch, in key-tile steps: its prologue (barriers,
+// tensor memory, the Q tile and the first logits) before the softmax runs.
+constexpr int kTailCostSteps = 4;
+
+// No-scratch schedule: whole pairs, or two phases when that beats them.
+void plan_no_scratch(int n_items, int n_kt, int G, Plan *pl) {
+  plan_whole(n_items, G, pl);
+  const long long whole_cost = static_cast<long long>((n_items + G - 1) / G) * n_kt;
+  if (n_kt < 2 || n_items > 8 * G || n_items <= G) return;
+  const int ns = G;  // one second piece per cluster of the second launch
+  const int nw = n_items - ns;
+  long long best = whole_cost;
+  int best_b = 0, best_t = 0;
+  for (int b = 1; b < n_kt; ++b) {
+    const int a = n_kt - b;
+    const long long hi = best - b - kTailCostSteps - 1;  // t must beat the best so far
+    const long long work = static_cast<long long>(nw) * n_kt + static_cast<long long>(ns) * a;
+    long long lo = (work + G - 1) / G;
+    if (lo > hi) continue;
+    std::vector<int> x, y;
+    if (!pack_first_launch(static_cast<int>(hi), nw, ns, n_kt, a, G, &x, &y)) continue;
+    long long l = lo, h = hi;  // smallest feasible t in [lo, hi]
+    while (l < h) {
+      const long long mid = (l + h) / 2;
+      if (pack_first_launch(static_cast<int>(mid), nw, ns, n_kt, a, G, &x, &y))
+        h = mid;
+      else
+        l = mid + 1;
+    }
+    const long long cost = l + b + kTailCostSteps;
+    if (cost < best) {
+      best = cost;
+      best_b = b;
+      best_t = static_cast<int>(l);
+    }
+  }
+  if (best_b == 0) return;
+  std::vector<int> x, y;
+  const int a = n_kt - best_b;
+  if (!pack_first_launch(best_t, nw, ns, n_kt, a, G, &x, &y)) return;
+  // Drop clusters with no work; ranges stay contiguous per kind.
+  std::vector<int> wb(1, 0), fb(1, 0);
+  for (int c = 0; c < G; ++c) {
+    if (x[c] == 0 && y[c] == 0) continue;
+    wb.push_back(wb.back() + x[c]);
+    fb.push_back(fb.back() + y[c]);
+  }
+  pl->sched = attn::kSchedUnits;
+  pl->clusters = static_cast<int>(wb.size()) - 1;
+  pl->tail_clusters = ns;
+  pl->n_whole = nw;
+  pl->split_at = a;
+  pl->wb = wb;
+  pl->fb = fb;
+}
+
+// Scratch schedule (kSchedRange): one cluster per SM pair, never more
 // clusters than (pair, key tile) steps or scratch slots.  Whole pairs per
 // cluster unless that leaves the grid badly balanced: a split pair costs a
 // second pass over its rows (partial results, then the merge), so whole pairs
 // win while the busiest cluster's extra work stays below kSplitGain pairs.
-static cudaError_t plan_grid(int mode, int dv, int n_items, int n_kt, int num_sms,
-                             int scratch_slots, int *clusters_out, int *whole_out) {
-  int max_clusters = 0;
-  cudaError_t e = dv == 192 ? configure_any<192>(mode, &max_clusters)
-                            : configure_any<128>(mode, &max_clusters);
-  if (e != cudaSuccess) return e;
+void plan_range(int n_items, int n_kt, int G, int scratch_slots, Plan *pl) {
+  int clusters = std::min(G, scratch_slots);
   const long long steps = static_cast<long long>(n_items) * n_kt;
-  if (steps > (1ll << 30)) return cudaErrorInvalidValue;
-  int clusters = num_sms / 2;
-  if (max_clusters < clusters) clusters = max_clusters;
-  if (scratch_slots < clusters) clusters = scratch_slots;
   if (steps < clusters) clusters = static_cast<int>(steps);
-  if (clusters < 1) return cudaErrorInvalidValue;
   constexpr double kSplitGain = 0.5;
   const long long per = (n_items + clusters - 1) / clusters;  // busiest cluster
   const double even = static_cast<double>(n_items) / clusters;
   const int whole = (per - even <= kSplitGain) ? 1 : 0;
   if (whole && n_items < clusters) clusters = n_items;
-  *clusters_out = clusters;
-  *whole_out = whole;
+  pl->sched = attn::kSchedRange;
+  pl->clusters = clusters;
+  pl->tail_clusters = 0;
+  pl->whole = whole;
+  pl->wb.clear();
+  pl->fb.clear();
+}
+
+// The schedule for n_items pairs of n_kt key tiles on G clusters: with
+// scratch slots, the range schedule; without, whole pairs or two phases.
+// Pure host logic (no CUDA call).
+Plan plan_for(int n_items, int n_kt, int G, int scratch_slots) {
+  Plan pl;
+  if (scratch_slots > 0)
+    plan_range(n_items, n_kt, G, scratch_slots, &pl);
+  else
+    plan_no_scratch(n_items, n_kt, std::min(G, kAttnMaxClusters), &pl);
+  return pl;
+}
+
+// Plans are cached per (items, key tiles, clusters, scratch slots): the
+// two-phase search costs more than a launch.
+struct PlanKey {
+  int n_items, n_kt, G, slots;
+  bool operator==(const PlanKey &o) const {
+    return n_items == o.n_items && n_kt == o.n_kt && G == o.G && slots == o.slots;
+  }
+};
+std::mutex g_plan_mu;
+std::vector<std::pair<PlanKey, Plan>> g_plans;
+
+cudaError_t make_plan(int mode, int dv, int n_items, int n_kt, int num_sms, int scratch_slots,
+                      Plan *pl) {
+  int max_clusters = 0;
+  cudaError_t e = dv == 192 ? configure_any<192>(mode, &max_clusters)
+                            : configure_any<128>(mode, &max_clusters);
+  if (e != cudaSuccess) return e;
+  const long long steps = static_cast<long long>(n_items) * n_kt;
+  if (steps > (1ll << 30) || steps < 1) return cudaErrorInvalidValue;
+  // One cluster per resident SM pair.  The range schedule needs no
+  // per-cluster table; the others carry per-cluster ranges in the kernel
+  // parameters, sized for kAttnMaxClusters (plan_for clamps them).
+  const int G = std::min(num_sms / 2, max_clusters);
+  if (G < 1) return cudaErrorInvalidValue;
+  const PlanKey key{n_items, n_kt, G, scratch_slots};
+  {
+    std::lock_guard<std::mutex> lock(g_plan_mu);
+    for (const auto &kv : g_plans)
+      if (kv.first == key) {
+        *pl = kv.second;
+        return cudaSuccess;
+      }
+  }
+  Plan fresh = plan_for(n_items, n_kt, G, scratch_slots);
+  if (fresh.clusters < 1 ||
+      (fresh.sched != attn::kSchedRange &&
+       (fresh.clusters > kAttnMaxClusters || fresh.tail_clusters > kAttnMaxClusters)))
+    return cudaErrorInvalidValue;
+  {
+    std::lock_guard<std::mutex> lock(g_plan_mu);
+    if (g_plans.size() >= 256) g_plans.erase(g_plans.begin());
+    g_plans.emplace_back(key, fresh);
+  }
+  *pl = fresh;
   return cudaSuccess;
 }
 
-static int attn_mode(float cap) {
-  using namespace attn;
-  if (isinf(cap)) return kNoCap;
-  return cap <= 40.0f ? kStaticCap : kOnlineCap;
+template <int MODE, int DV>
+cudaError_t launch_mode(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                        const attn::Params &p, int clusters, bool dependent,
+                        cudaStream_t stream) {
+  if (!dependent) {
+    attn::attn_fwd_kernel<MODE, DV>
+        <<<2 * clusters, attn::kThreads, attn::smem_bytes<DV>(), stream>>>(tq, tk, tv, p);
+    return cudaGetLastError();
+  }
+  // The second launch of a two-phase schedule: programmatic dependent launch,
+  // so its CTAs take the SMs that the first launch's CTAs leave.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  cfg.blockDim = dim3(attn::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = attn::smem_bytes<DV>();
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, attn::attn_fwd_kernel<MODE, DV>, tq, tk, tv, p);
 }
 
-cudaError_t attn_fwd_kernel_count(int64_t B, int64_t L, int64_t Dv, float cap,
-                                  int num_sms, int scratch_slots, int *count) {
+template <int DV>
+cudaError_t launch_dv(int mode, const CUtensorMap &tq, const CUtensorMap &tk,
+                      const CUtensorMap &tv, const attn::Params &p, int clusters,
+                      bool dependent, cudaStream_t stream) {
+  using namespace attn;
+  switch (mode) {
+    case kStaticFast: return launch_mode<kStaticFast, DV>(tq, tk, tv, p, clusters, dependent, stream);
+    case kStaticAcc: return launch_mode<kStaticAcc, DV>(tq, tk, tv, p, clusters, dependent, stream);
+    case kOnline: return launch_mode<kOnline, DV>(tq, tk, tv, p, clusters, dependent, stream);
+    default: return launch_mode<kNoCap, DV>(tq, tk, tv, p, clusters, dependent, stream);
+  }
+}
+
+}  // namespace
+
+cudaError_t attn_fwd_kernel_count(int64_t B, int64_t L, int64_t Dv, float cap, int num_sms,
+                                  int scratch_slots, int *count) {
   using namespace attn;
   if (B == 0 || L == 0) {
     *count = 0;
@@ -1129,17 +1476,53 @@ cudaError_t attn_fwd_kernel_count(int64_t B, int64_t L, int64_t Dv, float cap,
   const int nb = static_cast<int>((L + 15) / 16);
   const int n_items = static_cast<int>(B) * ((nb + 1) / 2);
   const int n_kt = static_cast<int>((L + kKeys - 1) / kKeys);
-  int clusters = 0, whole = 0;
-  cudaError_t e = plan_grid(attn_mode(cap), static_cast<int>(Dv), n_items, n_kt,
-                            num_sms, scratch_slots, &clusters, &whole);
+  Plan pl;
+  cudaError_t e = make_plan(attn_mode(cap), static_cast<int>(Dv), n_items, n_kt, num_sms,
+                            scratch_slots, &pl);
   if (e != cudaSuccess) return e;
-  *count = (clusters < 2 || whole) ? 1 : 2;
+  if (pl.sched == kSchedRange)
+    *count = (pl.clusters < 2 || pl.whole) ? 1 : 2;
+  else
+    *count = pl.tail_clusters > 0 ? 2 : 1;
   return cudaSuccess;
+}
+
+cudaError_t attn_fwd_clusters(int64_t B, int64_t L, int64_t Dv, float cap, int num_sms,
+                              int scratch_slots, int *clusters) {
+  const int nb = static_cast<int>((L + 15) / 16);
+  const int n_items = static_cast<int>(B) * ((nb + 1) / 2);
+  const int n_kt = static_cast<int>((L + attn::kKeys - 1) / attn::kKeys);
+  Plan pl;
+  cudaError_t e = make_plan(attn_mode(cap), static_cast<int>(Dv), n_items, n_kt, num_sms,
+                            scratch_slots, &pl);
+  if (e != cudaSuccess) return e;
+  *clusters = pl.clusters;
+  return cudaSuccess;
+}
+
+void attn_fwd_schedule(int64_t B, int64_t L, int sm_pairs, int scratch_slots, int *sched,
+                       int *clusters, int *tail_clusters, int *whole, int *n_whole,
+                       int *split_at, int *wb, int *fb) {
+  const int nb = static_cast<int>((L + 15) / 16);
+  const int n_items = static_cast<int>(B) * ((nb + 1) / 2);
+  const int n_kt = static_cast<int>((L + attn::kKeys - 1) / attn::kKeys);
+  const Plan pl = plan_for(n_items, n_kt, sm_pairs, scratch_slots);
+  *sched = pl.sched;
+  *clusters = pl.clusters;
+  *tail_clusters = pl.tail_clusters;
+  *whole = pl.whole;
+  *n_whole = pl.n_whole;
+  *split_at = pl.split_at;
+  for (int c = 0; c <= kAttnMaxClusters; ++c) {
+    wb[c] = c < static_cast<int>(pl.wb.size()) ? pl.wb[c] : 0;
+    fb[c] = c < static_cast<int>(pl.fb.size()) ? pl.fb[c] : 0;
+  }
 }
 
 cudaError_t launch_attn_fwd(const AttnLaunch &a) {
   using namespace attn;
   const int64_t B = a.B, L = a.L;
+  if (a.Dv != 128 && a.Dv != 192) return cudaErrorInvalidValue;
   CUtensorMap tq, tk, tv;
   {
     const cuuint64_t dims[4] = {kD, static_cast<cuuint64_t>(L), kH,
@@ -1175,6 +1558,8 @@ cudaError_t launch_attn_fwd(const AttnLaunch &a) {
   p.out = a.out;
   p.lse = a.lse;
   p.err = a.err;
+  p.ws_out = nullptr;
+  p.ws_lse = nullptr;
   p.L = static_cast<int>(L);
   p.P = static_cast<int>((L + 15) / 16);
   p.nb = p.P;
@@ -1183,49 +1568,67 @@ cudaError_t launch_attn_fwd(const AttnLaunch &a) {
   p.n_items = static_cast<int>(B) * p.pairs;
   p.n_kt = static_cast<int>((L + kKeys - 1) / kKeys);
   p.last_valid = static_cast<int>(L - static_cast<int64_t>(p.n_kt - 1) * kKeys);
+  if (static_cast<long long>(p.n_items) * p.n_kt != attn_work_steps(B, L))
+    return cudaErrorInvalidValue;
   const float cap = a.cap;
   const float inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(kD));
   const int mode = attn_mode(cap);
-  if (mode == kNoCap) {
-    p.qk_scale = inv_sqrt_d * kLog2e;
-    p.bias_mul = kLog2e;
-    p.A = 0.f;
-  } else {
-    p.qk_scale = inv_sqrt_d / cap;
-    p.bias_mul = 1.0f / cap;
-    p.A = cap * kLog2e;
+  switch (mode) {
+    case kNoCap:
+      p.qk_scale = inv_sqrt_d * kLog2e;
+      p.bias_mul = kLog2e;
+      p.A = 0.f;
+      p.shift = 0.f;
+      break;
+    case kStaticFast:
+      // y = z / cap; the shift is the smallest integer >= A (exp2_poly2_fma
+      // folds an integer shift into its coefficients).
+      p.qk_scale = inv_sqrt_d / cap;
+      p.bias_mul = 1.0f / cap;
+      p.A = cap * kLog2e;
+      p.shift = ceilf(p.A);
+      break;
+    default:  // kStaticAcc, kOnline: u = 2 log2(e) z / cap
+      p.qk_scale = 2.0f * kLog2e * inv_sqrt_d / cap;
+      p.bias_mul = 2.0f * kLog2e / cap;
+      p.A = cap * kLog2e;
+      p.shift = p.A;
+      break;
   }
-  if (a.Dv != 128 && a.Dv != 192) return cudaErrorInvalidValue;
   const int dv = static_cast<int>(a.Dv);
-  int clusters = 0;
-  cudaError_t e = plan_grid(mode, dv, p.n_items, p.n_kt, a.num_sms, a.scratch_slots,
-                            &clusters, &p.whole);
+  Plan pl;
+  cudaError_t e = make_plan(mode, dv, p.n_items, p.n_kt, a.num_sms, a.scratch ? a.scratch_slots : 0,
+                            &pl);
   if (e != cudaSuccess) return e;
-  if (static_cast<long long>(p.n_items) * p.n_kt != attn_work_steps(B, L))
-    return cudaErrorInvalidValue;
-  char *base = static_cast<char *>(a.scratch);
-  p.ws_out = reinterpret_cast<float *>(base);
-  p.ws_lse = reinterpret_cast<float *>(base + a.scratch_slots * kAttnSlotOutBytes);
-  if (dv == 192) {
-    switch (mode) {
-      case kStaticCap: e = launch_mode<kStaticCap, 192>(tq, tk, tv, p, clusters, a.stream); break;
-      case kOnlineCap: e = launch_mode<kOnlineCap, 192>(tq, tk, tv, p, clusters, a.stream); break;
-      default: e = launch_mode<kNoCap, 192>(tq, tk, tv, p, clusters, a.stream); break;
-    }
-  } else {
-    switch (mode) {
-      case kStaticCap: e = launch_mode<kStaticCap, 128>(tq, tk, tv, p, clusters, a.stream); break;
-      case kOnlineCap: e = launch_mode<kOnlineCap, 128>(tq, tk, tv, p, clusters, a.stream); break;
-      default: e = launch_mode<kNoCap, 128>(tq, tk, tv, p, clusters, a.stream); break;
-    }
+  p.sched = pl.sched;
+  p.whole = pl.whole;
+  p.n_whole = pl.n_whole;
+  p.split_at = pl.split_at;
+  for (int c = 0; c <= kAttnMaxClusters; ++c) {
+    p.wb[c] = c < static_cast<int>(pl.wb.size()) ? pl.wb[c] : 0;
+    p.fb[c] = c < static_cast<int>(pl.fb.size()) ? pl.fb[c] : 0;
   }
-  if (e != cudaSuccess || clusters < 2 || p.whole) return e;
-  const int merge_blocks = (clusters - 1) * kMergeBlocksPerBoundary;
-  if (dv == 192)
-    attn_merge_kernel<192><<<merge_blocks, kMergeThreads, 0, a.stream>>>(p, clusters);
-  else
-    attn_merge_kernel<128><<<merge_blocks, kMergeThreads, 0, a.stream>>>(p, clusters);
-  return cudaGetLastError();
+  if (pl.sched == kSchedRange) {
+    char *base = static_cast<char *>(a.scratch);
+    p.ws_out = reinterpret_cast<float *>(base);
+    p.ws_lse = reinterpret_cast<float *>(base + a.scratch_slots * kAttnSlotOutBytes);
+  }
+  e = dv == 192 ? launch_dv<192>(mode, tq, tk, tv, p, pl.clusters, false, a.stream)
+                : launch_dv<128>(mode, tq, tk, tv, p, pl.clusters, false, a.stream);
+  if (e != cudaSuccess) return e;
+  if (pl.sched == kSchedRange) {
+    if (pl.clusters < 2 || pl.whole) return cudaSuccess;
+    const int merge_blocks = (pl.clusters - 1) * kMergeBlocksPerBoundary;
+    if (dv == 192)
+      attn_merge_kernel<192><<<merge_blocks, kMergeThreads, 0, a.stream>>>(p, pl.clusters);
+    else
+      attn_merge_kernel<128><<<merge_blocks, kMergeThreads, 0, a.stream>>>(p, pl.clusters);
+    return cudaGetLastError();
+  }
+  if (pl.tail_clusters == 0) return cudaSuccess;
+  p.sched = kSchedTail;
+  return dv == 192 ? launch_dv<192>(mode, tq, tk, tv, p, pl.tail_clusters, true, a.stream)
+                   : launch_dv<128>(mode, tq, tk, tv, p, pl.tail_clusters, true, a.stream);
 }
 
 }  // namespace ag

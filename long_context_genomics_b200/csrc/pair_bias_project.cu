@@ -8,16 +8,20 @@
 // the attention kernel reads the compact result directly instead).
 //
 // Bound by HBM: 512 bytes of pair data per cell against 8 outputs.  A
-// persistent CTA per SM streams chunks of 64 consecutive cells (32 KB) into a
-// 4-stage shared-memory ring with untiled bulk copies issued by one producer
-// lane, so 128 KB per SM are in flight.  Eight consumer warps take 8 cells
-// each per chunk.  Lane l reads channels 4l..4l+3 of a cell (one conflict-free
-// 16-byte shared load per cell) and keeps W[4l..4l+3, 0..7] in registers
-// (products for two heads per packed fp32x2 instruction); the
-// 64 partial sums (8 heads x 8 cells) are reduced across the warp by a
-// butterfly reduce-scatter (offsets 16, 8, 4, 2, 1), after which lane l holds
-// the two finished values of head l/4 for cells 2(l%4) and 2(l%4)+1: a float2
-// store, eight consecutive cells per head across the warp.
+// persistent CTA per SM streams chunks of 32 consecutive cells (16 KB) into a
+// 12-stage shared-memory ring with TMA (one producer lane; the pair tensor is
+// seen as [cells, 128] fp32 rows, four 32-channel boxes per chunk with the
+// 128-byte swizzle), so up to 192 KB per SM are in flight.  Each of eight
+// consumer warps takes whole chunks: lane l owns cell l of the chunk and sums
+// its 128 channels for all 8 heads in registers (packed fp32x2 products, two
+// heads per instruction).  The swizzle puts the 16-byte channel group g of
+// cell l at group slot g ^ (l % 8) of its 128-byte row, so the eight lanes of
+// a shared-memory phase read eight different bank groups; W sits in shared
+// memory and every lane reads the same W row (a broadcast).  No cross-lane
+// reduction is needed, and lane l stores cell l of each head plane: 32
+// consecutive floats per store instruction.
+#include <mutex>
+
 #include "ag_internal.h"
 #include "sm100.cuh"
 
@@ -27,70 +31,69 @@ namespace proj {
 constexpr int kCp = 128;
 constexpr int kH = 8;
 constexpr int kCellBytes = kCp * 4;                  // 512
-constexpr int kChunkCells = 64;
-constexpr int kChunkBytes = kChunkCells * kCellBytes;  // 32 KB
-constexpr int kStages = 4;
-constexpr int kConsumerWarps = 8;                    // 8 cells each per chunk
+constexpr int kChunkCells = 32;                      // one cell per lane
+constexpr int kChunkBytes = kChunkCells * kCellBytes;  // 16 KB
+constexpr int kBoxBytes = kChunkCells * 128;         // 32 cells x 32 channels
+constexpr int kStages = 12;
+constexpr int kConsumerWarps = 8;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;  // + producer warp
-constexpr size_t kSmemBytes = 1024 + kStages * kChunkBytes + 2 * kStages * 8 + 16;
+constexpr int kWBytes = kCp * kH * 4;                // 4 KB
+constexpr size_t kSmemBytes = 1024 + kStages * kChunkBytes + kWBytes + 2 * kStages * 8 + 16;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
 enum Site : unsigned { kSiteFull = 20, kSiteEmpty = 21 };
 
-// One reduce-scatter level: lanes with bit `o` set keep the upper half of
-// the first 2*n values, the others the lower half; each adds its partner's
-// (two values per packed add).
-template <int n>
-__device__ __forceinline__ void rs_level(float (&a)[64], int o, bool upper) {
-#pragma unroll
-  for (int j = 0; j < n; j += 2) {
-    const float2 keep = upper ? make_float2(a[j + n], a[j + n + 1])
-                              : make_float2(a[j], a[j + 1]);
-    const float2 send = upper ? make_float2(a[j], a[j + 1])
-                              : make_float2(a[j + n], a[j + n + 1]);
-    const float2 recv = make_float2(__shfl_xor_sync(0xffffffffu, send.x, o),
-                                    __shfl_xor_sync(0xffffffffu, send.y, o));
-    const float2 sum = __fadd2_rn(keep, recv);
-    a[j] = sum.x;
-    a[j + 1] = sum.y;
-  }
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar,
+                                            int c0, int c1, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_"
+      "tx::bytes.L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1),
+      "l"(policy)
+      : "memory");
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    pair_bias_project_kernel(const float *__restrict__ pair,
+    pair_bias_project_kernel(const __grid_constant__ CUtensorMap tm_pair,
                              const float *__restrict__ W, float *__restrict__ bias,
-                             long long n_cells, int vec_store, unsigned *err) {
+                             long long n_cells, unsigned *err) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t *ring = smem_raw + pad;
-  uint64_t *full = reinterpret_cast<uint64_t *>(ring + kStages * kChunkBytes);
+  float *w_s = reinterpret_cast<float *>(ring + kStages * kChunkBytes);
+  uint64_t *full = reinterpret_cast<uint64_t *>(w_s + kCp * kH);
   uint64_t *empty = full + kStages;
   int *abort_flag = reinterpret_cast<int *>(empty + kStages);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kConsumerWarps);
+      mbar_init(&empty[s], 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
   }
+  for (int i = threadIdx.x; i < kCp * kH; i += kThreads) w_s[i] = __ldg(W + i);
   __syncthreads();
   volatile int *abort = abort_flag;
   const long long n_chunks = (n_cells + kChunkCells - 1) / kChunkCells;
 
   if (warp == kConsumerWarps) {
-    // Producer: one lane issues the bulk copies.
+    // Producer: one lane issues four 32-channel boxes per chunk.  Rows past
+    // the last cell are filled with zeros and their results never stored.
     if (lane == 0) {
+      prefetch_tensormap(&tm_pair);
       const uint64_t pol = l2_policy_evict_first();
       uint32_t it = 0;
       for (long long ch = blockIdx.x; ch < n_chunks; ch += gridDim.x, ++it) {
         const uint32_t slot = it % kStages, ph = (it / kStages) & 1u;
         if (!mbar_wait(&empty[slot], ph ^ 1u, abort, err, kSiteEmpty)) break;
-        const long long c0 = ch * kChunkCells;
-        const long long nc = n_cells - c0 < kChunkCells ? n_cells - c0 : kChunkCells;
-        const uint32_t bytes = static_cast<uint32_t>(nc) * kCellBytes;
-        mbar_arrive_expect_tx(&full[slot], bytes);
-        bulk_load(ring + slot * kChunkBytes, pair + c0 * kCp, bytes, &full[slot], pol);
+        mbar_arrive_expect_tx(&full[slot], kChunkBytes);
+        const int row = static_cast<int>(ch * kChunkCells);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          tma_load_2d(ring + slot * kChunkBytes + q * kBoxBytes, &tm_pair, &full[slot], 32 * q,
+                      row, pol);
       }
       // Every copy this thread started must land before the CTA exits.
       const uint32_t first = it > kStages ? it - kStages : 0;
@@ -102,59 +105,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // W[4l + i, h] for heads in pairs (2p, 2p + 1).
-    float2 w[4][kH / 2];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int hp = 0; hp < kH / 2; ++hp)
-        w[i][hp] = make_float2(__ldg(W + (4 * lane + i) * kH + 2 * hp),
-                               __ldg(W + (4 * lane + i) * kH + 2 * hp + 1));
-    const int h_out = lane >> 2;       // head this lane finishes
-    const int n_out = 2 * (lane & 3);  // first of its two cells
-    uint32_t it = 0;
-    for (long long ch = blockIdx.x; ch < n_chunks; ch += gridDim.x, ++it) {
+    // Consumer warp `warp` takes the CTA's chunks it = warp, warp + 8, ...
+    const float4 *w4 = reinterpret_cast<const float4 *>(w_s);  // W[c][0..3], W[c][4..7]
+    const uint32_t swz = static_cast<uint32_t>(lane & 7);
+    for (uint32_t it = warp;; it += kConsumerWarps) {
+      const long long ch = blockIdx.x + static_cast<long long>(it) * gridDim.x;
+      if (ch >= n_chunks) break;
       const uint32_t slot = it % kStages, ph = (it / kStages) & 1u;
       const bool ok = mbar_wait(&full[slot], ph, abort, err, kSiteFull);
       if (!__all_sync(0xffffffffu, ok)) break;
-      const long long c0 = ch * kChunkCells + warp * 8;  // this warp's 8 cells
-      const float4 *cells = reinterpret_cast<const float4 *>(
-          ring + slot * kChunkBytes + warp * 8 * kCellBytes);
-      float4 x[8];
+      const uint8_t *base = ring + slot * kChunkBytes + lane * 128;
+      float2 acc[kH / 2];
 #pragma unroll
-      for (int n = 0; n < 8; ++n)
-        x[n] = (c0 + n < n_cells) ? cells[n * (kCp / 4) + lane]
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int hp = 0; hp < kH / 2; ++hp) acc[hp] = make_float2(0.f, 0.f);
+      // Channel group g (channels 4g .. 4g+3): box g / 8, 16-byte slot
+      // (g % 8) ^ (lane % 8) of this lane's 128-byte row.
+#pragma unroll 8
+      for (int g = 0; g < kCp / 4; ++g) {
+        const float4 x = *reinterpret_cast<const float4 *>(
+            base + (g >> 3) * kBoxBytes + ((static_cast<uint32_t>(g & 7) ^ swz) << 4));
+        const float xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float4 wa = w4[(4 * g + k) * 2], wb = w4[(4 * g + k) * 2 + 1];
+          const float2 xx = make_float2(xs[k], xs[k]);
+          acc[0] = __ffma2_rn(xx, make_float2(wa.x, wa.y), acc[0]);
+          acc[1] = __ffma2_rn(xx, make_float2(wa.z, wa.w), acc[1]);
+          acc[2] = __ffma2_rn(xx, make_float2(wb.x, wb.y), acc[2]);
+          acc[3] = __ffma2_rn(xx, make_float2(wb.z, wb.w), acc[3]);
+        }
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[slot]);  // this warp is done with the slot
-      if (c0 >= n_cells) continue;
-      float a[64];  // a[h * 8 + n]: the same products and order as
-                    // fmaf(x.w, w3, fmaf(x.z, w2, fmaf(x.y, w1, x.x * w0))),
-                    // two heads per packed instruction
+      const long long cell = ch * kChunkCells + lane;
+      if (cell < n_cells) {
 #pragma unroll
-      for (int hp = 0; hp < kH / 2; ++hp)
-#pragma unroll
-        for (int n = 0; n < 8; ++n) {
-          float2 v = __fmul2_rn(make_float2(x[n].x, x[n].x), w[0][hp]);
-          v = __ffma2_rn(make_float2(x[n].y, x[n].y), w[1][hp], v);
-          v = __ffma2_rn(make_float2(x[n].z, x[n].z), w[2][hp], v);
-          v = __ffma2_rn(make_float2(x[n].w, x[n].w), w[3][hp], v);
-          a[(2 * hp) * 8 + n] = v.x;
-          a[(2 * hp + 1) * 8 + n] = v.y;
+        for (int hp = 0; hp < kH / 2; ++hp) {
+          __stcs(bias + (2 * hp) * n_cells + cell, acc[hp].x);
+          __stcs(bias + (2 * hp + 1) * n_cells + cell, acc[hp].y);
         }
-      rs_level<32>(a, 16, lane & 16);
-      rs_level<16>(a, 8, lane & 8);
-      rs_level<8>(a, 4, lane & 4);
-      rs_level<4>(a, 2, lane & 2);
-      rs_level<2>(a, 1, lane & 1);
-      // a[0], a[1]: head h_out, cells c0 + n_out and c0 + n_out + 1.
-      float *dst = bias + static_cast<long long>(h_out) * n_cells + c0 + n_out;
-      const long long cell = c0 + n_out;
-      if (vec_store && cell + 1 < n_cells) {
-        __stcs(reinterpret_cast<float2 *>(dst), make_float2(a[0], a[1]));
-      } else {
-        if (cell < n_cells) dst[0] = a[0];
-        if (cell + 1 < n_cells) dst[1] = a[1];
       }
     }
   }
@@ -163,30 +152,38 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace proj
 
-cudaError_t launch_pair_bias_project(const float *pair, const float *W,
-                                     float *bias, int64_t P, int num_sms,
-                                     unsigned *err, cudaStream_t stream) {
+cudaError_t launch_pair_bias_project(const float *pair, const float *W, float *bias,
+                                     int64_t P, int num_sms, unsigned *err,
+                                     EncodeTiledFn encode, cudaStream_t stream) {
   using namespace proj;
-  static int configured[64] = {0};
+  static std::once_flag once[64];
+  static cudaError_t once_err[64];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!configured[dev]) {
-    e = cudaFuncSetAttribute(pair_bias_project_kernel,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSmemBytes));
-    if (e != cudaSuccess) return e;
-    configured[dev] = 1;
-  }
+  std::call_once(once[dev], [&] {
+    once_err[dev] = cudaFuncSetAttribute(pair_bias_project_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kSmemBytes));
+  });
+  if (once_err[dev] != cudaSuccess) return once_err[dev];
   const long long n_cells = static_cast<long long>(P) * P;
+  // pair as a 2-D tensor: n_cells rows of 128 fp32 channels (512-byte rows).
+  CUtensorMap tm;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kCp), static_cast<cuuint64_t>(n_cells)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kCellBytes)};
+  const cuuint32_t box[2] = {32, kChunkCells};
+  const cuuint32_t estr[2] = {1, 1};
+  if (encode(&tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(pair), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
   const long long n_chunks = (n_cells + kChunkCells - 1) / kChunkCells;
   const long long grid = n_chunks < num_sms ? n_chunks : num_sms;
-  // float2 stores need an even cell count (then every head's plane starts
-  // 8-byte aligned, as does every even cell inside it).
-  const int vec_store = (n_cells % 2 == 0) ? 1 : 0;
-  pair_bias_project_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemBytes,
-                             stream>>>(pair, W, bias, n_cells, vec_store, err);
+  pair_bias_project_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, stream>>>(
+      tm, W, bias, n_cells, err);
   return cudaGetLastError();
 }
 

@@ -376,6 +376,24 @@ __device__ __forceinline__ float lg2_approx(float x) {
   asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// ---------------------------------------------------------------------------
+// Programmatic dependent launch.  A grid launched with programmatic stream
+// serialization may start while the grid before it on the stream still
+// runs, once every CTA of that grid has executed launch_dependents (or has
+// exited); griddep_wait then blocks the calling thread until the earlier grid
+// has completed and its memory writes are visible.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
 
 // 2^x on the FMA pipe (two lanes at once) for x in [-126, 0], used to take
 // part of the exponentials off the special-function unit.  Range reduction
@@ -397,6 +415,29 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   return make_float2(
       __int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
       __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
+// 2^(a t - m) on the FMA pipe (two lanes at once) for an integer m in
+// [0, 2^21) and a t - m in [-126, 0]: the same range reduction and
+// polynomial as exp2_poly2, with the product a t and the shift folded into
+// the reduction.  km = 1.5 * 2^23 - m is exact in fp32, so one fused
+// multiply-add rounded toward minus infinity gives T = km + floor(a t)
+// exactly (a t + km is exact before that rounding since |a t| < 2^22);
+// nf = km - T = -floor(a t) is exact, f = a t + nf lies in [0, 1), and the
+// low bits of T hold floor(a t) - m for the exponent.  Saves the separate
+// a t - m product of exp2_poly2(a t - m).
+__device__ __forceinline__ float2 exp2_poly2_fma(float2 t, float2 a, float2 km) {
+  constexpr float c0 = 0.9999252557754517f, c1 = 0.695833683013916f,
+                  c2 = 0.22606664896011353f, c3 = 0.07802490144968033f;
+  const float2 T = __ffma2_rd(a, t, km);
+  const float2 nf = __fadd2_rn(km, make_float2(-T.x, -T.y));
+  const float2 f = __ffma2_rn(a, t, nf);
+  float2 p = __ffma2_rn(make_float2(c3, c3), f, make_float2(c2, c2));
+  p = __ffma2_rn(p, f, make_float2(c1, c1));
+  p = __ffma2_rn(p, f, make_float2(c0, c0));
+  return make_float2(
+      __int_as_float(__float_as_int(p.x) + (__float_as_int(T.x) << 23)),
+      __int_as_float(__float_as_int(p.y) + (__float_as_int(T.y) << 23)));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -230,16 +230,82 @@ def test_cap_modes(ag, oracle_lib, cap):
     _compare(out, lse, ro, rl, f"cap={cap}")
 
 
-@pytest.mark.parametrize("cap", [5.0, 30.0, math.inf])
+@pytest.mark.parametrize("cap", [5.0, 10.0, 30.0, 40.0, 50.0, math.inf])
 def test_large_logits(ag, oracle_lib, cap):
     """q, k with std 3 and a bias of std 4: logits far beyond the cap
-    (saturated tanh) and, without a cap, a wide softmax range."""
+    (saturated tanh), a softmax dominated by a few keys at the large caps
+    (where an error in a logit passes straight into lse) and, without a cap,
+    a wide softmax range.  Caps 40 and 50 sit on either side of the switch
+    from the static shift to the running maximum."""
     inp = ag_inputs.random_case(1, 8, 640, 128, 128, 16, seed=77, bias_std=4.0,
                                 qk_std=3.0)
     out, lse = _gpu_attn(ag, inp, cap)
     ro, rl = oracle_lib.attn_fwd(inp["q"], inp["k"], inp["v"], inp["bias"],
                                  block=16, cap=cap)
     _compare(out, lse, ro, rl, f"large logits cap={cap}")
+
+
+@pytest.mark.parametrize("cap", [5.0, 10.0, 40.0, 50.0])
+def test_large_logits_full_context_sampled(ag, oracle_lib, cap):
+    """The same logit distribution at L = 8192 (8192 keys per softmax, the
+    two-launch schedule at B = 1), sampled rows against the oracle."""
+    inp = ag_inputs.random_case(1, 8, 8192, 128, 128, 16, seed=78, bias_std=4.0,
+                                qk_std=3.0)
+    out, lse = _gpu_attn(ag, inp, cap)
+    rows = ag_inputs.sample_rows(1, 8, 8192, 384, seed=int(cap)).numpy()
+    ro, rl = oracle_lib.attn_rows(inp["q"], inp["k"], inp["v"], inp["bias"], rows,
+                                  block=16, cap=cap)
+    b, h, i = rows[:, 0], rows[:, 1], rows[:, 2]
+    _compare(out[b, h, i], lse[b, h, i], ro, rl, f"large logits L=8192 cap={cap} sampled")
+
+
+def test_split_pairs_full_context(ag, oracle_lib):
+    """L = 8192, B = 1 on a 148-SM B200 runs two launches: the last 74 pairs
+    of query blocks (positions 5824..8191) have their keys split in two, the
+    second launch merging into the first's results.  Rows drawn from those
+    positions only, all heads, against the oracle."""
+    w = ag_inputs.WORKLOADS["full"]
+    inp = ag_inputs.make_inputs(w)
+    bias = ag.ag_pair_bias_project(_dev(inp["pair"]), _dev(inp["W"]))
+    out, lse = _gpu_attn(ag, inp, w.cap, bias=bias)
+    ref_bias = oracle_lib.pair_bias_project(inp["pair"], inp["W"])
+    g = torch.Generator().manual_seed(8)
+    pos = 5824 + torch.randperm(8192 - 5824, generator=g)[:64]
+    rows = np.array([(0, h, int(i)) for i in pos for h in range(8)] +
+                    [(0, h, i) for i in (5824, 5855, 5856, 8191) for h in range(8)])
+    ro, rl = oracle_lib.attn_rows(inp["q"], inp["k"], inp["v"], ref_bias, rows,
+                                  block=16, cap=w.cap)
+    b, h, i = rows[:, 0], rows[:, 1], rows[:, 2]
+    _compare(out[b, h, i], lse[b, h, i], ro, rl, "split pairs L=8192")
+
+
+def test_two_streams_at_once(ag, oracle_lib):
+    """Two different L = 8192 calls issued on two streams without waiting for
+    each other (the library keeps no shared scratch, so they may overlap on
+    the GPU): one B = 1 (two launches) and one B = 2 with its own bias per
+    item (whole pairs), each checked against the oracle on sampled rows."""
+    cases = [ag_inputs.random_case(1, 8, 8192, 128, 128, 16, seed=61),
+             ag_inputs.random_case(2, 8, 8192, 128, 128, 16, seed=62, batched_bias=True)]
+    dev = [{n: _dev(t) for n, t in c.items()} for c in cases]
+    outs = []
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    torch.cuda.synchronize()
+    for _ in range(3):  # several rounds so that the two calls really overlap
+        outs = []
+        for d, st in zip(dev, streams):
+            with torch.cuda.stream(st):
+                outs.append(ag.ag_attn_fwd(d["q"], d["k"], d["v"], d["bias"], cap=5.0,
+                                           stream=st))
+    torch.cuda.synchronize()
+    assert ag.ag_device_error(0) == 0
+    for n, (c, (o, l)) in enumerate(zip(cases, outs)):
+        B = c["q"].shape[0]
+        rows = ag_inputs.sample_rows(B, 8, 8192, 256, seed=70 + n).numpy()
+        ro, rl = oracle_lib.attn_rows(c["q"], c["k"], c["v"], c["bias"], rows, block=16,
+                                      cap=5.0)
+        b, h, i = rows[:, 0], rows[:, 1], rows[:, 2]
+        on, ln = o.double().cpu().numpy(), l.double().cpu().numpy()
+        _compare(on[b, h, i], ln[b, h, i], ro, rl, f"stream {n} B={B}")
 
 
 def test_maximum_length_sampled(ag, oracle_lib):
@@ -276,23 +342,52 @@ def test_deterministic_and_stream(ag):
     assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
 
 
-def test_no_quadratic_memory(ag):
-    """The call allocates nothing: peak device memory during it stays at the
-    inputs plus outputs (no L x L logits, no expanded bias)."""
-    w = ag_inputs.WORKLOADS["full"]
-    inp = ag_inputs.make_inputs(w)
-    q, k, v = _dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"])
-    bias = ag.ag_pair_bias_project(_dev(inp["pair"]), _dev(inp["W"]))
-    out = torch.empty(1, 8, w.L, 128, device="cuda")
-    lse = torch.empty(1, 8, w.L, device="cuda")
+_MEMORY_PROBE = r"""
+import json, sys, torch
+sys.path.insert(0, sys.argv[1])
+import ag_inputs
+import long_context_genomics_b200 as ag
+w = ag_inputs.WORKLOADS["full"]
+inp = ag_inputs.make_inputs(w)
+d = {n: t.cuda() for n, t in inp.items()}
+bias = ag.ag_pair_bias_project(d["pair"], d["W"])   # loads the library's other modules
+out = torch.empty(1, 8, w.L, 128, device="cuda")
+lse = torch.empty(1, 8, w.L, device="cuda")
+torch.cuda.synchronize()
+free = [torch.cuda.mem_get_info()[0]]
+for _ in range(2):
+    ag.ag_attn_fwd(d["q"], d["k"], d["v"], bias, cap=5.0, out=out, lse=lse)
     torch.cuda.synchronize()
-    torch.cuda.reset_peak_memory_stats()
-    base = torch.cuda.memory_allocated()
-    ag.ag_attn_fwd(q, k, v, bias, cap=5.0, out=out, lse=lse)
-    torch.cuda.synchronize()
-    assert torch.cuda.max_memory_allocated() == base
-    free, total = torch.cuda.mem_get_info()
-    assert free > 0 and total > 0
+    free.append(torch.cuda.mem_get_info()[0])
+assert ag.ag_device_error(0) == 0
+print(json.dumps({"free": free, "lse0": float(lse[0, 0, 0])}))
+"""
+
+
+def test_no_quadratic_memory():
+    """The attention allocates no device memory.  In a fresh process (so that
+    the call is the first on the device), free device memory as the driver
+    reports it (cudaMemGetInfo) before and after the first and the second
+    call at L = 8192: the first call may only load the kernels' code (lazy
+    module loading, well under 8 MiB; a single fp32 head of L x L logits
+    would be 256 MiB, the old split-pair scratch 29 MB); the second changes
+    nothing."""
+    import json
+    import os
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    res = subprocess.run([sys.executable, "-c", _MEMORY_PROBE, root], capture_output=True,
+                         text=True, timeout=300)
+    assert res.returncode == 0, res.stderr[-2000:]
+    rec = json.loads(res.stdout.strip().splitlines()[-1])
+    f0, f1, f2 = rec["free"]
+    print(f"free before {f0}, after first call {f1} (-{(f0 - f1) / 2**20:.2f} MiB), "
+          f"after second {f2}")
+    assert math.isfinite(rec["lse0"])
+    assert 0 <= f0 - f1 <= 8 << 20
+    assert f2 == f1
 
 
 def test_bounded_wait_reports_and_context_survives(ag, oracle_lib):

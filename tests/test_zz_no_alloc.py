@@ -1,14 +1,17 @@
 """ag_attn_fwd_noalloc: the attention entry point that allocates nothing.
 
-Some callers cannot let a library call cudaMalloc: code that must not touch
-the allocator while a CUDA graph is being captured, or a framework that has
-already handed all device memory to its own pool.  For them the library keeps
-its split-pair scratch in a static device array instead of allocating it on
-the first call.  This test calls that entry point through the C ABI and
-checks it against ag_attn_fwd (which allocates its scratch) on two calls in a
-row: a size that splits pairs between SMs (so the scratch is really used) and
-then a different size, which must not be affected by what the first call left
-in the shared static array.  This file sorts last so that a run stopping at
+Some callers cannot let a library allocate device memory: a framework that
+has already handed all device memory to its own pool, or a process whose
+device memory budget is fixed at start-up.  This entry point runs the
+attention on the range schedule, whose split pairs need scratch; the
+library keeps that scratch in a static device array compiled into it.  The
+test calls the entry point through the C ABI on two calls in a row, at two
+sizes whose range schedule splits pairs on a 148-SM B200 (L = 512: 64
+clusters of one step each; L = 1024: 74 clusters), so the second call runs
+on what the first left in the shared array.  Each result is checked against
+the float64 oracle and against ag_attn_fwd within the tolerances of the
+parity tests, and a repeated call must give the same bits and leave free
+device memory unchanged.  This file sorts last so that a run stopping at
 the first failure has already run every other test.
 """
 import ctypes
@@ -27,37 +30,67 @@ LSE_TOL = 1e-3
 
 
 @pytest.fixture(scope="module")
-def lib():
+def ag():
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
     import long_context_genomics_b200 as ag
 
-    return ag.lib
+    return ag
 
 
-def _call(fn, inp, cap):
-    q, k, v, bias = (inp[n].cuda().contiguous() for n in ("q", "k", "v", "bias"))
-    B, H, L, D = q.shape
-    out = torch.full((B, H, L, D), float("nan"), device="cuda")
-    lse = torch.full((B, H, L), float("nan"), device="cuda")
-    st = fn(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
-            ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(bias.data_ptr()),
+def _launch(fn, d, cap, out, lse):
+    B, H, L, D = d["q"].shape
+    st = fn(ctypes.c_void_p(d["q"].data_ptr()), ctypes.c_void_p(d["k"].data_ptr()),
+            ctypes.c_void_p(d["v"].data_ptr()), ctypes.c_void_p(d["bias"].data_ptr()),
             B, H, L, D, 16, ctypes.c_float(cap), ctypes.c_void_p(out.data_ptr()),
             ctypes.c_void_p(lse.data_ptr()),
             ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == 0, f"status {st}"
     torch.cuda.synchronize()
-    return out.double().cpu().numpy(), lse.double().cpu().numpy()
 
 
-@pytest.mark.parametrize("cases", [[(1, 512, 5.0, 31), (1, 2064, math.inf, 32)]])
-def test_noalloc_matches_allocating_entry_point(lib, cases):
+def _host(out, lse):
+    return out.cpu().double().numpy(), lse.cpu().double().numpy()
+
+
+def _splits_pairs(ag, B, L):
+    """Whether the range schedule of this call splits pairs (so the merge
+    kernel reads the static scratch) on this device."""
+    I = ctypes.c_int
+    outs = [I() for _ in range(6)]
+    wb, fb = (I * 129)(), (I * 129)()
+    pairs = torch.cuda.get_device_properties(0).multi_processor_count // 2
+    st = ag.lib.ag_attn_fwd_schedule(B, L, pairs, 1, *[ctypes.byref(x) for x in outs], wb, fb)
+    assert st == 0
+    sched, clusters, _, whole, _, _ = (x.value for x in outs)
+    return sched == 0 and clusters > 1 and not whole
+
+
+@pytest.mark.parametrize("cases", [[(1, 512, 5.0, 31), (1, 1024, math.inf, 32)]])
+def test_noalloc_matches_the_oracle_and_the_allocating_entry_point(ag, oracle_lib, cases):
     for B, L, cap, seed in cases:  # two calls in a row on the static scratch
         inp = ag_inputs.random_case(B, 8, L, 128, 128, 16, seed=seed)
-        ref_out, ref_lse = _call(lib.ag_attn_fwd, inp, cap)
-        out, lse = _call(lib.ag_attn_fwd_noalloc, inp, cap)
-        assert np.isfinite(out).all() and np.isfinite(lse).all()
-        eo = float(np.max(np.abs(out - ref_out)))
-        el = float(np.max(np.abs(lse - ref_lse)))
-        print(f"noalloc B={B} L={L} cap={cap}: max|dout|={eo:.3e} max|dlse|={el:.3e}")
-        assert eo <= OUT_TOL and el <= LSE_TOL
+        d = {n: t.cuda().contiguous() for n, t in inp.items()}
+        if torch.cuda.get_device_properties(0).multi_processor_count == 148:
+            assert _splits_pairs(ag, B, L), "the case must exercise the scratch"
+        nan = dict(device="cuda", dtype=torch.float32)
+        out, out2, out3 = (torch.full((B, 8, L, 128), float("nan"), **nan) for _ in range(3))
+        lse, lse2, lse3 = (torch.full((B, 8, L), float("nan"), **nan) for _ in range(3))
+        _launch(ag.lib.ag_attn_fwd_noalloc, d, cap, out, lse)
+        free = torch.cuda.mem_get_info()[0]
+        _launch(ag.lib.ag_attn_fwd_noalloc, d, cap, out2, lse2)
+        assert torch.cuda.mem_get_info()[0] == free, "a repeated call allocated memory"
+        assert ag.ag_device_error(0) == 0
+        _launch(ag.lib.ag_attn_fwd, d, cap, out3, lse3)
+        (o1, l1), (o2, l2) = _host(out, lse), _host(out2, lse2)
+        ref_out, ref_lse = _host(out3, lse3)
+        assert np.array_equal(o1, o2) and np.array_equal(l1, l2), "not reproducible"
+        oo, ol = oracle_lib.attn_fwd(inp["q"], inp["k"], inp["v"], inp["bias"], block=16,
+                                     cap=cap)
+        assert np.isfinite(o1).all() and np.isfinite(l1).all()
+        for what, (ro, rl) in (("oracle", (oo, ol)), ("ag_attn_fwd", (ref_out, ref_lse))):
+            eo = float(np.max(np.abs(o1 - ro)))
+            el = float(np.max(np.abs(l1 - rl)))
+            print(f"noalloc B={B} L={L} cap={cap} vs {what}: max|dout|={eo:.3e} "
+                  f"max|dlse|={el:.3e}")
+            assert eo <= OUT_TOL and el <= LSE_TOL
