@@ -282,6 +282,42 @@ def max_over_ranks(seconds: float, device, world: int) -> float:
     return float(t.item())
 
 
+def query_shard(L: int, world: int, rank: int) -> tuple:
+    """Rank r's query positions [q0, q1) when the L queries of a sequence are
+    split between the ranks: contiguous ranges, each a multiple of 32
+    positions (whole pairs of 16-position blocks) except the last, which
+    takes the remainder."""
+    unit = 32
+    units = -(-L // unit)
+    q0 = min(L, unit * (units * rank // world))
+    q1 = min(L, unit * (units * (rank + 1) // world))
+    return q0, q1
+
+
+def gather_keys(shard: torch.Tensor, world: int, out: torch.Tensor | None = None) -> torch.Tensor:
+    """All of a sequence's keys (or values) from every rank's contiguous
+    shard [B, L/world, D]: one all_gather, the shards placed in rank order
+    along the sequence.  out, if given, is the [B, L, D] result."""
+    B, Ls, D = shard.shape
+    if out is None:
+        out = torch.empty(B, world * Ls, D, dtype=shard.dtype, device=shard.device)
+    if world == 1:
+        out.copy_(shard)
+        return out
+    parts = [torch.empty_like(shard) for _ in range(world)]
+    torch.distributed.all_gather(parts, shard.contiguous())
+    for r, part in enumerate(parts):
+        out[:, r * Ls:(r + 1) * Ls].copy_(part)
+    return out
+
+
+def bias_rows(bias: torch.Tensor, q0: int, q1: int, block: int = 16) -> torch.Tensor:
+    """The bias rows of query positions [q0, q1) (q0 a multiple of block):
+    rows q0/block .. ceil(q1/block) of the last-but-one axis, contiguous."""
+    assert q0 % block == 0
+    return bias[..., q0 // block:-(-q1 // block), :].contiguous()
+
+
 def aggregate_rate(world: int, units_per_step: float, steps: int, seconds: float) -> float:
     """Whole-job throughput: the units all ranks processed over the slowest
     rank's time (weak scaling: every rank does the same work per step)."""
@@ -509,6 +545,88 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     print(json.dumps(line), flush=True)
 
 
+def run_sharded(args, rank: int, world: int, local_rank: int) -> None:
+    """One full-context problem split between the ranks by query position
+    (strong scaling).  Each rank holds its slab of queries, its rows of the
+    pair representation and a contiguous shard of the keys and values, as a
+    sequence-parallel model would; every step all-gathers K and V (NCCL),
+    projects its pair rows and runs the attention for its queries.  The
+    outputs stay sharded: no collective follows."""
+    import long_context_genomics_b200 as ag
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = config_layers(args.config)[0]
+    if len(config_layers(args.config)) != 1 or w.bias_mode != "pair":
+        raise SystemExit("--shard queries runs the single-layer projected workload (full)")
+    host = ag_inputs.make_inputs(w)       # every rank draws the same problem
+    q0, q1 = query_shard(w.L, world, rank)
+    k0, k1 = w.L * rank // world, w.L * (rank + 1) // world
+    if (w.L % world) or (w.L // world) % 16:
+        raise SystemExit("--shard queries needs L / world to be a multiple of 16")
+    q = host["q"][:, :, q0:q1].contiguous().to(dev)
+    k_shard = host["k"][:, k0:k1].contiguous().to(dev)
+    v_shard = host["v"][:, k0:k1].contiguous().to(dev)
+    pair = host["pair"][q0 // 16:-(-q1 // 16)].contiguous().to(dev)   # pair rows of the slab
+    W = host["W"].to(dev)
+    k_full = torch.empty(w.B, w.L, w.D, dtype=torch.bfloat16, device=dev)
+    v_full = torch.empty(w.B, w.L, w.Dv, dtype=torch.bfloat16, device=dev)
+    bias = torch.empty(w.H, pair.shape[0], w.P, device=dev)
+    out = torch.empty(w.B, w.H, q1 - q0, w.Dv, device=dev)
+    lse = torch.empty(w.B, w.H, q1 - q0, device=dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        gather_keys(k_shard, world, k_full)
+        gather_keys(v_shard, world, v_full)
+        ag.ag_pair_bias_project_rows(pair, W, bias=bias)
+        ag.ag_attn_fwd_query_slab(q, k_full, v_full, bias, cap=w.cap, out=out, lse=lse)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    barrier()
+    assert ag.ag_device_error(local_rank) == 0
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    time.sleep(0.3 if sampler else 0.0)
+    barrier()
+    t_wall0 = time.time()
+    for i in range(K):
+        flush.zero_()
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    barrier()
+    clocks = sampler.stop(t_wall0, time.time()) if sampler else None
+    total_s = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3, dev, world)
+    assert ag.ag_device_error(local_rank) == 0 and math.isfinite(float(lse[0, 0, 0]))
+    if rank != 0:
+        return
+    pk = peaks()
+    flops = w.attn_flops()                # the whole problem, split between the ranks
+    value = flops * K / total_s / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": 1e3 * total_s / K, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {**job_config(args.config, [w], 1),
+                   "parallelism": f"queries split over {world} GPUs (K/V all-gather)",
+                   "step": "all_gather K, V + ag_pair_bias_project_rows + "
+                           "ag_attn_fwd_query_slab"},
+        "pct_of_peak": 100.0 * value / world / pk["bf16_tflops"], "peak_source": pk["source"],
+        "gpu_launches": K * (1 + 2), "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def backward_flops(w) -> float:
     """Algorithmic FLOPs of one backward call, the usual count of five L x L
     products: S = Q K^T (recomputed), dP = dO V^T, dV = P^T dO, dQ = dS K,
@@ -600,6 +718,9 @@ def main() -> None:
                     help="with --path backward: which workload (default full, L=8192)")
     ap.add_argument("--config", choices=CONFIGS + ("all",), default="full",
                     help="forward workload (default full: L=8192, B=1, the headline line)")
+    ap.add_argument("--shard", choices=["replicas", "queries"], default="replicas",
+                    help="N > 1: independent problems per GPU (replicas, weak scaling) or "
+                         "one problem's queries split between the GPUs (strong scaling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.steps is None:
@@ -613,6 +734,8 @@ def main() -> None:
         ap.error("--workload applies to --path backward only")
     if args.path == "backward" and args.config != "full":
         ap.error("--config applies to --path forward")
+    if args.shard == "queries" and (args.config != "full" or args.impl != "ours"):
+        ap.error("--shard queries runs our kernels on the full workload")
     if args.path == "backward":
         run_backward(args)
         return
@@ -634,7 +757,11 @@ def main() -> None:
             backend="nccl", timeout=datetime.timedelta(seconds=120))
     try:
         for c in configs:
-            run_ours(argparse.Namespace(**{**vars(args), "config": c}), rank, world, local_rank)
+            a = argparse.Namespace(**{**vars(args), "config": c})
+            if args.shard == "queries":
+                run_sharded(a, rank, world, local_rank)
+            else:
+                run_ours(a, rank, world, local_rank)
             torch.cuda.empty_cache()
     finally:
         if world > 1:

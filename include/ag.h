@@ -79,6 +79,20 @@ ag_status ag_pair_bias_project(const float *pair, const float *W, float *bias,
                                int64_t P, int64_t Cp, int64_t H, void *stream);
 
 /*
+ * ag_pair_bias_project_rows -- the same projection for R rows of the pair
+ * representation (R <= P), e.g. the rows of the query positions one GPU
+ * holds when the queries are split between GPUs (see
+ * ag_attn_fwd_query_slab):
+ *   pair [R, P, Cp] -> bias [H, R, P],  bias[h, r, q] = sum_c pair[r, q, c] W[c, h]
+ * Same types, alignment and statuses as ag_pair_bias_project (R > 4096 is
+ * AG_ERR_UNSUPPORTED, R < 0 AG_ERR_SHAPE, R == 0 a no-op);
+ * ag_pair_bias_project is this call with R = P.
+ */
+ag_status ag_pair_bias_project_rows(const float *pair, const float *W, float *bias,
+                                    int64_t R, int64_t P, int64_t Cp, int64_t H,
+                                    void *stream);
+
+/*
  * ag_attn_fwd -- fused pair-bias multi-query attention forward.
  *
  * For b < B, h < H, query i < L, key j < L (page "Making Full-Context
@@ -157,6 +171,33 @@ ag_status ag_attn_fwd_ex(const void *q, const void *k, const void *v,
                          const float *bias, int64_t bias_batch_stride, int64_t B,
                          int64_t H, int64_t L, int64_t D, int64_t Dv, int64_t block,
                          float cap, float *out, float *lse, void *stream);
+
+/*
+ * ag_attn_fwd_query_slab -- ag_attn_fwd_ex for a slab of Lq consecutive query
+ * positions of sequences of L positions (so that the queries can be split
+ * between GPUs while every GPU holds all L keys and values: the sequence
+ * parallelism of the page "From Code to Cure: How AlphaGenome Decodes the
+ * 'Dark Matter' of DNA", section "The Architecture").
+ *
+ * Query i of this call is position q0 + i of its sequence for some q0 that
+ * is a multiple of block (the caller's choice; the call never sees q0):
+ *   q     [B, H, Lq, D]   the slab's queries
+ *   k     [B, L, D], v [B, L, Dv]   all keys and values
+ *   bias  [H, ceil(Lq / block), ceil(L / block)] per item: rows q0 / block ..
+ *         of the full [H, P, P] bias (one per item at bias_batch_stride,
+ *         0 or >= H * ceil(Lq / block) * ceil(L / block) floats)
+ *   out   [B, H, Lq, Dv], lse [B, H, Lq]   the slab's results
+ * Every query attends to all L keys, so the slab's rows equal the same rows
+ * of a full call (bit for bit when both calls run those rows as whole pairs;
+ * see ag_attn_fwd_schedule).  Lq == L with q0 = 0 is ag_attn_fwd_ex.
+ * Checks and statuses as ag_attn_fwd_ex, plus AG_ERR_SHAPE for Lq < 0 and
+ * AG_ERR_UNSUPPORTED for Lq > 65536; Lq == 0 is a no-op.
+ */
+ag_status ag_attn_fwd_query_slab(const void *q, const void *k, const void *v,
+                                 const float *bias, int64_t bias_batch_stride, int64_t B,
+                                 int64_t H, int64_t Lq, int64_t L, int64_t D, int64_t Dv,
+                                 int64_t block, float cap, float *out, float *lse,
+                                 void *stream);
 
 /*
  * ag_attn_fwd_noalloc -- the attention forward on the range schedule, for

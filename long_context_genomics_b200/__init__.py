@@ -53,6 +53,8 @@ def _load() -> ctypes.CDLL:
     lib.ag_version.restype = ctypes.c_int
     lib.ag_pair_bias_project.argtypes = [vp, vp, vp, i64, i64, i64, vp]
     lib.ag_pair_bias_project.restype = ctypes.c_int
+    lib.ag_pair_bias_project_rows.argtypes = [vp, vp, vp, i64, i64, i64, i64, vp]
+    lib.ag_pair_bias_project_rows.restype = ctypes.c_int
     lib.ag_attn_fwd.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, f32,
                                 vp, vp, vp]
     lib.ag_attn_fwd.restype = ctypes.c_int
@@ -62,6 +64,9 @@ def _load() -> ctypes.CDLL:
     lib.ag_attn_fwd_ex.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, i64,
                                    i64, f32, vp, vp, vp]
     lib.ag_attn_fwd_ex.restype = ctypes.c_int
+    lib.ag_attn_fwd_query_slab.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, i64,
+                                           i64, i64, f32, vp, vp, vp]
+    lib.ag_attn_fwd_query_slab.restype = ctypes.c_int
     lib.ag_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64,
                                         f32, vp, vp, vp]
     lib.ag_attn_fwd_noalloc.restype = ctypes.c_int
@@ -148,6 +153,29 @@ def ag_pair_bias_project(pair: torch.Tensor, W: torch.Tensor,
     return bias
 
 
+def ag_pair_bias_project_rows(pair: torch.Tensor, W: torch.Tensor,
+                              bias: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """bias[h,r,q] = sum_c pair[r,q,c] W[c,h] for a row slab pair[R,P,Cp]
+    (libag kernel); returns bias [H,R,P]."""
+    _check(pair, "pair", torch.float32, 3)
+    _check(W, "W", torch.float32, 2)
+    R, P, Cp = pair.shape
+    if W.shape[0] != Cp:
+        raise ValueError("pair must be [R,P,Cp] and W [Cp,H]")
+    H = W.shape[1]
+    if bias is None:
+        bias = torch.empty((H, R, P), dtype=torch.float32, device=pair.device)
+    _check(bias, "bias", torch.float32, 3)
+    if tuple(bias.shape) != (H, R, P):
+        raise ValueError("bias must be [H,R,P]")
+    with torch.cuda.device(_one_device(pair, W, bias)):
+        st = lib.ag_pair_bias_project_rows(pair.data_ptr(), W.data_ptr(), bias.data_ptr(),
+                                           R, P, Cp, H, _stream_ptr(stream))
+    if st != AG_OK:
+        raise AgError("ag_pair_bias_project_rows", st)
+    return bias
+
+
 def ag_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                 bias: torch.Tensor, cap: float = 5.0, block: int = 16,
                 out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
@@ -181,16 +209,53 @@ def ag_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     return out, lse
 
 
-def _bias_stride(bias: torch.Tensor, B: int, H: int, L: int, block: int) -> int:
-    """Batch stride (floats) of a [H,P,P] (0) or [B,H,P,P] bias, P = ceil(L/block)."""
+def ag_attn_fwd_query_slab(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                           bias: torch.Tensor, cap: float = 5.0, block: int = 16,
+                           out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                           stream=None):
+    """The attention rows of a slab of query positions (libag kernel).
+
+    q [B,H,Lq,D] holds positions q0 .. q0+Lq-1 (q0 a multiple of block) of
+    sequences whose keys and values k [B,L,D], v [B,L,Dv] are all given; bias
+    holds the slab's bias rows, [H, ceil(Lq/block), ceil(L/block)] (shared by
+    the batch) or [B, H, ceil(Lq/block), ceil(L/block)].  Returns
+    (out [B,H,Lq,Dv] fp32, lse [B,H,Lq] fp32)."""
+    _check(q, "q", torch.bfloat16, 4)
+    _check(k, "k", torch.bfloat16, 3)
+    _check(v, "v", torch.bfloat16, 3)
+    B, H, Lq, D = q.shape
+    L, Dv = k.shape[1], v.shape[-1]
+    if tuple(k.shape) != (B, L, D) or tuple(v.shape) != (B, L, Dv):
+        raise ValueError("k must be [B,L,D] and v [B,L,Dv] with q [B,H,Lq,D]")
+    bstride = _bias_stride(bias, B, H, L, block, rows=-(-Lq // block) if block > 0 else 0)
+    if out is None:
+        out = torch.empty((B, H, Lq, Dv), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
+    _check_out(out, lse, B, H, Lq, Dv)
+    with torch.cuda.device(_one_device(q, k, v, bias, out, lse)):
+        st = lib.ag_attn_fwd_query_slab(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), bias.data_ptr(), bstride, B, H, Lq, L,
+            D, Dv, int(block), float(cap), out.data_ptr(), lse.data_ptr(),
+            _stream_ptr(stream))
+    if st != AG_OK:
+        raise AgError("ag_attn_fwd_query_slab", st)
+    return out, lse
+
+
+def _bias_stride(bias: torch.Tensor, B: int, H: int, L: int, block: int,
+                 rows: int | None = None) -> int:
+    """Batch stride (floats) of a [H,R,P] (0) or [B,H,R,P] bias, P = ceil(L/block)
+    and R = rows (default P)."""
     if bias.dtype != torch.float32 or not bias.is_contiguous():
         raise ValueError("bias must be a contiguous float32 tensor")
     P = -(-L // block) if block > 0 else 0
-    if tuple(bias.shape) == (H, P, P):
+    R = P if rows is None else rows
+    if tuple(bias.shape) == (H, R, P):
         return 0
-    if tuple(bias.shape) == (B, H, P, P):
-        return H * P * P
-    raise ValueError(f"bias must be [{H},{P},{P}] or [{B},{H},{P},{P}], got {tuple(bias.shape)}")
+    if tuple(bias.shape) == (B, H, R, P):
+        return H * R * P
+    raise ValueError(f"bias must be [{H},{R},{P}] or [{B},{H},{R},{P}], got {tuple(bias.shape)}")
 
 
 def _check_out(out: torch.Tensor, lse: torch.Tensor, B: int, H: int, L: int, Dv: int):

@@ -141,13 +141,19 @@ int ag_version(void) { return 10000 * 0 + 100 * 1 + 0; }
 
 ag_status ag_pair_bias_project(const float *pair, const float *W, float *bias,
                                int64_t P, int64_t Cp, int64_t H, void *stream) {
-  if (P < 0 || Cp <= 0 || H <= 0) return AG_ERR_SHAPE;
-  if (Cp != 128 || H != 8 || P > 4096) return AG_ERR_UNSUPPORTED;
-  if (P == 0) return AG_OK;
+  return ag_pair_bias_project_rows(pair, W, bias, P, P, Cp, H, stream);
+}
+
+ag_status ag_pair_bias_project_rows(const float *pair, const float *W, float *bias,
+                                    int64_t R, int64_t P, int64_t Cp, int64_t H,
+                                    void *stream) {
+  if (R < 0 || P < 0 || Cp <= 0 || H <= 0) return AG_ERR_SHAPE;
+  if (Cp != 128 || H != 8 || P > 4096 || R > 4096) return AG_ERR_UNSUPPORTED;
+  if (P == 0 || R == 0) return AG_OK;
   if (!pair || !W || !bias) return AG_ERR_NULL;
   if (!ag::aligned(pair, 16) || !ag::aligned(W, 4) || !ag::aligned(bias, 8))
     return AG_ERR_ALIGN;
-  const uint64_t cells = static_cast<uint64_t>(P) * P;
+  const uint64_t cells = static_cast<uint64_t>(R) * P;
   const uint64_t bias_bytes = cells * H * 4;
   if (ag::overlap(bias, bias_bytes, pair, cells * Cp * 4) ||
       ag::overlap(bias, bias_bytes, W, static_cast<uint64_t>(Cp) * H * 4))
@@ -159,7 +165,8 @@ ag_status ag_pair_bias_project(const float *pair, const float *W, float *bias,
   st = ag::get_encoder(&enc);
   if (st != AG_OK) return st;
   return ag::from_cuda(ag::launch_pair_bias_project(
-      pair, W, bias, P, dev->num_sms, dev->err, enc, static_cast<cudaStream_t>(stream)));
+      pair, W, bias, static_cast<int64_t>(cells), dev->num_sms, dev->err, enc,
+      static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"
@@ -179,19 +186,20 @@ ag_status check_attn_sizes(int64_t B, int64_t H, int64_t L, int64_t D, int64_t b
   return AG_OK;
 }
 
-// The value width and the per-item bias stride (after check_attn_sizes).
-static ag_status check_value_width_and_bias_stride(int64_t B, int64_t H, int64_t L,
-                                                   int64_t Dv, int64_t block,
+// The value width and the per-item bias stride (after check_attn_sizes), for
+// a bias of `rows` rows of P cells per head.
+static ag_status check_value_width_and_bias_stride(int64_t B, int64_t H, int64_t rows,
+                                                   int64_t P, int64_t Dv,
                                                    int64_t bias_batch_stride) {
   if (Dv <= 0) return AG_ERR_SHAPE;
   if (Dv != 128 && Dv != 192) return AG_ERR_UNSUPPORTED;
-  const int64_t P = (L + block - 1) / block;
-  if (bias_batch_stride < 0 || (bias_batch_stride > 0 && bias_batch_stride < H * P * P))
+  const int64_t per_item = H * rows * P;
+  if (bias_batch_stride < 0 || (bias_batch_stride > 0 && bias_batch_stride < per_item))
     return AG_ERR_SHAPE;
-  // The items' bias span, (B - 1) * stride + H * P * P floats, must stay far
+  // The items' bias span, (B - 1) * stride + H * rows * P floats, must stay far
   // below 2^63 bytes so that the alias check and the kernel's offsets are exact.
   constexpr int64_t kMaxBiasSpan = int64_t(1) << 56;
-  if (B > 1 && bias_batch_stride > (kMaxBiasSpan - H * P * P) / (B - 1))
+  if (B > 1 && bias_batch_stride > (kMaxBiasSpan - per_item) / (B - 1))
     return AG_ERR_SHAPE;
   return AG_OK;
 }
@@ -220,24 +228,38 @@ ag_status ag_attn_fwd_ex(const void *q, const void *k, const void *v,
                          const float *bias, int64_t bias_batch_stride, int64_t B,
                          int64_t H, int64_t L, int64_t D, int64_t Dv, int64_t block,
                          float cap, float *out, float *lse, void *stream) {
+  return ag_attn_fwd_query_slab(q, k, v, bias, bias_batch_stride, B, H, L, L, D, Dv, block,
+                                cap, out, lse, stream);
+}
+
+ag_status ag_attn_fwd_query_slab(const void *q, const void *k, const void *v,
+                                 const float *bias, int64_t bias_batch_stride, int64_t B,
+                                 int64_t H, int64_t Lq, int64_t L, int64_t D, int64_t Dv,
+                                 int64_t block, float cap, float *out, float *lse,
+                                 void *stream) {
   const ag_status vs = ag::check_attn_sizes(B, H, L, D, block, cap);
   if (vs != AG_OK) return vs;
-  const ag_status ws = ag::check_value_width_and_bias_stride(B, H, L, Dv, block,
-                                                             bias_batch_stride);
-  if (ws != AG_OK) return ws;
+  if (Lq < 0) return AG_ERR_SHAPE;
+  if (Lq > 65536 || (B > 0 && Lq > 0 && B * Lq > (int64_t(1) << 28)) ||
+      (B > 0 && Lq > 0 && L > 0 && ag::attn_work_steps(B, Lq, L) > (int64_t(1) << 30)))
+    return AG_ERR_UNSUPPORTED;
   const int64_t P = (L + block - 1) / block;
-  if (B == 0 || L == 0) return AG_OK;
+  const int64_t rows = (Lq + block - 1) / block;
+  const ag_status ws =
+      ag::check_value_width_and_bias_stride(B, H, rows, P, Dv, bias_batch_stride);
+  if (ws != AG_OK) return ws;
+  if (B == 0 || L == 0 || Lq == 0) return AG_OK;
   if (!q || !k || !v || !bias || !out || !lse) return AG_ERR_NULL;
   if (!ag::aligned(q, 16) || !ag::aligned(k, 16) || !ag::aligned(v, 16) ||
       !ag::aligned(bias, 4) || !ag::aligned(out, 16) || !ag::aligned(lse, 4))
     return AG_ERR_ALIGN;
-  const uint64_t qb = static_cast<uint64_t>(B) * H * L * D * 2;
+  const uint64_t qb = static_cast<uint64_t>(B) * H * Lq * D * 2;
   const uint64_t kb = static_cast<uint64_t>(B) * L * D * 2;
   const uint64_t vb = static_cast<uint64_t>(B) * L * Dv * 2;
   const uint64_t bb = (static_cast<uint64_t>(B - 1) * bias_batch_stride +
-                       static_cast<uint64_t>(H) * P * P) * 4;
-  const uint64_t ob = static_cast<uint64_t>(B) * H * L * Dv * 4;
-  const uint64_t lb = static_cast<uint64_t>(B) * H * L * 4;
+                       static_cast<uint64_t>(H) * rows * P) * 4;
+  const uint64_t ob = static_cast<uint64_t>(B) * H * Lq * Dv * 4;
+  const uint64_t lb = static_cast<uint64_t>(B) * H * Lq * 4;
   const void *ins[4] = {q, k, v, bias};
   const uint64_t insz[4] = {qb, kb, vb, bb};
   for (int t = 0; t < 4; ++t)
@@ -260,6 +282,7 @@ ag_status ag_attn_fwd_ex(const void *q, const void *k, const void *v,
   a.lse = lse;
   a.B = B;
   a.L = L;
+  a.Lq = Lq;
   a.Dv = Dv;
   a.cap = cap;
   a.err = dev->err;
@@ -284,7 +307,7 @@ ag_status ag_attn_fwd_launch_count(int64_t B, int64_t H, int64_t L, int64_t D,
   ag_status st = ag::device_info(&dev);
   if (st != AG_OK) return st;
   int n = 0;
-  st = ag::from_cuda(ag::attn_fwd_kernel_count(B, L, D, cap, dev->num_sms, 0, &n));
+  st = ag::from_cuda(ag::attn_fwd_kernel_count(B, L, L, D, cap, dev->num_sms, 0, &n));
   if (st != AG_OK) return st;
   *count = n;
   return AG_OK;
@@ -310,7 +333,8 @@ ag_status ag_attn_bwd(const void *q, const void *k, const void *v, const float *
                       float *dbias, float *delta, void *stream) {
   ag_status st = ag::check_attn_sizes(B, H, L, D, block, cap);
   if (st != AG_OK) return st;
-  st = ag::check_value_width_and_bias_stride(B, H, L, Dv, block, bias_batch_stride);
+  const int64_t Pc = (L + block - 1) / block;
+  st = ag::check_value_width_and_bias_stride(B, H, Pc, Pc, Dv, bias_batch_stride);
   if (st != AG_OK) return st;
   if (B == 0 || L == 0) return AG_OK;
   if (!q || !k || !v || !bias || !lse || !dout || !dq || !dk || !dv || !dbias || !delta)

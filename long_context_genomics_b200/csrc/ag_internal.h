@@ -32,17 +32,19 @@ inline size_t attn_scratch_bytes(int slots) {
 constexpr int64_t kAttnKeyTile = 128;
 // Most 2-CTA clusters an attention launch uses (one per SM pair up to 256 SMs).
 constexpr int kAttnMaxClusters = 128;
-inline int64_t attn_work_steps(int64_t B, int64_t L) {
-  const int64_t blocks = (L + 15) / 16;  // the last may be partial
+inline int64_t attn_work_steps(int64_t B, int64_t Lq, int64_t L) {
+  const int64_t blocks = (Lq + 15) / 16;  // the last may be partial
   return B * ((blocks + 1) / 2) * ((L + kAttnKeyTile - 1) / kAttnKeyTile);
 }
+inline int64_t attn_work_steps(int64_t B, int64_t L) { return attn_work_steps(B, L, L); }
 
 struct AttnLaunch {
   const void *q, *k, *v;
   const float *bias;
   int64_t bias_bstride;  // floats between batch items' bias (0: shared)
   float *out, *lse;
-  int64_t B, L;
+  int64_t B, L;         // batch items, keys per item
+  int64_t Lq;           // query positions per item (rows of q, out and lse)
   int64_t Dv;           // value width: 128 or 192
   float cap;
   unsigned *err;        // device error word
@@ -62,7 +64,7 @@ cudaError_t launch_attn_fwd(const AttnLaunch &a);
 // How many kernels launch_attn_fwd launches for these sizes on the current
 // device (0 for an empty call, 1, or 2 when split pairs need the merge kernel
 // or a second launch); scratch_slots 0 for the schedules without scratch.
-cudaError_t attn_fwd_kernel_count(int64_t B, int64_t L, int64_t Dv, float cap,
+cudaError_t attn_fwd_kernel_count(int64_t B, int64_t Lq, int64_t L, int64_t Dv, float cap,
                                   int num_sms, int scratch_slots, int *count);
 // The schedule launch_attn_fwd uses for these sizes with sm_pairs resident
 // 2-CTA clusters (pure host logic): wb and fb hold kAttnMaxClusters + 1 ints.
@@ -88,8 +90,10 @@ struct AttnBwdLaunch {
 cudaError_t launch_attn_bwd(const AttnBwdLaunch &a);
 int attn_bwd_kernel_count();
 
+// Projects `cells` consecutive cells of 128 channels into 8 head planes of
+// `cells` floats each.
 cudaError_t launch_pair_bias_project(const float *pair, const float *W,
-                                     float *bias, int64_t P, int num_sms,
+                                     float *bias, int64_t cells, int num_sms,
                                      unsigned *err, EncodeTiledFn encode,
                                      cudaStream_t stream);
 

@@ -202,8 +202,11 @@ struct Params {
   unsigned *err;
   float *ws_out;       // kSchedRange scratch: [clusters][2][128][DV] partial outputs
   float *ws_lse;       //                      [clusters][2][128] partial log-sum-exps
-  int L, P;
-  int nb;          // 16-position query blocks per batch item, ceil(L / 16)
+  int L;           // keys per batch item
+  int Lq;          // query positions per batch item (rows of q, out, lse)
+  int P;           // bias cells per bias row, ceil(L / 16)
+  int bias_rows;   // bias rows per head in the bias array, ceil(Lq / 16)
+  int nb;          // 16-position query blocks per batch item, ceil(Lq / 16)
   int pairs;       // query-tile pairs per batch item: ceil(nb / 2)
   int n_items;     // B * pairs
   int n_kt;        // key tiles: ceil(L / 128)
@@ -862,7 +865,7 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc, uint32_t 
     const bool valid = I0 + static_cast<int>(rank) < p.nb;
     const int pos = I * 16 + il;  // this thread's query position
     const float *brow = p.bias + static_cast<long long>(b) * p.bias_bstride +
-                        (static_cast<size_t>(h) * p.P + I) * p.P;
+                        (static_cast<size_t>(h) * p.bias_rows + I) * p.P;
     float m = kStatic ? p.shift : -INFINITY;  // log2 units
     float d = 0.f;
     if constexpr (kStatic) {
@@ -885,8 +888,8 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc, uint32_t 
       break;
     }
     tc_fence_after();
-    const bool writes = valid && pos < p.L;  // rows past the end of a partial block: none
-    const size_t row = (static_cast<size_t>(b) * kH + h) * p.L + static_cast<size_t>(pos);
+    const bool writes = valid && pos < p.Lq;  // rows past the end of a partial block: none
+    const size_t row = (static_cast<size_t>(b) * kH + h) * p.Lq + static_cast<size_t>(pos);
     float lse_a = 0.f;
     if (sg.dest == kDestMerge) {
       // The first piece of this pair was written by the previous launch;
@@ -1098,8 +1101,8 @@ __global__ void __launch_bounds__(kMergeThreads)
   const int lane = static_cast<int>(threadIdx.x & 31);
   const int h = r >> 4, il = r & 15;
   const int pos = (I0 + X) * 16 + il;
-  if (pos >= p.L) return;  // past the end of a partial last block
-  const size_t row = (static_cast<size_t>(b) * kH + h) * p.L + static_cast<size_t>(pos);
+  if (pos >= p.Lq) return;  // past the end of a partial last block
+  const size_t row = (static_cast<size_t>(b) * kH + h) * p.Lq + static_cast<size_t>(pos);
   auto slot = [&](int s) {
     return (static_cast<size_t>(c_first + s) * 2 + X) * 128 + r;
   };
@@ -1466,14 +1469,14 @@ cudaError_t launch_dv(int mode, const CUtensorMap &tq, const CUtensorMap &tk,
 
 }  // namespace
 
-cudaError_t attn_fwd_kernel_count(int64_t B, int64_t L, int64_t Dv, float cap, int num_sms,
-                                  int scratch_slots, int *count) {
+cudaError_t attn_fwd_kernel_count(int64_t B, int64_t Lq, int64_t L, int64_t Dv, float cap,
+                                  int num_sms, int scratch_slots, int *count) {
   using namespace attn;
-  if (B == 0 || L == 0) {
+  if (B == 0 || L == 0 || Lq == 0) {
     *count = 0;
     return cudaSuccess;
   }
-  const int nb = static_cast<int>((L + 15) / 16);
+  const int nb = static_cast<int>((Lq + 15) / 16);
   const int n_items = static_cast<int>(B) * ((nb + 1) / 2);
   const int n_kt = static_cast<int>((L + kKeys - 1) / kKeys);
   Plan pl;
@@ -1521,14 +1524,14 @@ void attn_fwd_schedule(int64_t B, int64_t L, int sm_pairs, int scratch_slots, in
 
 cudaError_t launch_attn_fwd(const AttnLaunch &a) {
   using namespace attn;
-  const int64_t B = a.B, L = a.L;
+  const int64_t B = a.B, L = a.L, Lq = a.Lq;
   if (a.Dv != 128 && a.Dv != 192) return cudaErrorInvalidValue;
   CUtensorMap tq, tk, tv;
   {
-    const cuuint64_t dims[4] = {kD, static_cast<cuuint64_t>(L), kH,
+    const cuuint64_t dims[4] = {kD, static_cast<cuuint64_t>(Lq), kH,
                                 static_cast<cuuint64_t>(B)};
-    const cuuint64_t strides[3] = {kD * 2, static_cast<cuuint64_t>(L) * kD * 2,
-                                   static_cast<cuuint64_t>(L) * kD * 2 * kH};
+    const cuuint64_t strides[3] = {kD * 2, static_cast<cuuint64_t>(Lq) * kD * 2,
+                                   static_cast<cuuint64_t>(Lq) * kD * 2 * kH};
     const cuuint32_t box[4] = {64, 16, kH, 1};
     if (!encode_map(a.encode, &tq, a.q, 4, dims, strides, box))
       return cudaErrorInvalidValue;
@@ -1561,14 +1564,16 @@ cudaError_t launch_attn_fwd(const AttnLaunch &a) {
   p.ws_out = nullptr;
   p.ws_lse = nullptr;
   p.L = static_cast<int>(L);
+  p.Lq = static_cast<int>(Lq);
   p.P = static_cast<int>((L + 15) / 16);
-  p.nb = p.P;
+  p.nb = static_cast<int>((Lq + 15) / 16);
+  p.bias_rows = p.nb;
   p.bias_bstride = a.bias_bstride;
   p.pairs = (p.nb + 1) / 2;
   p.n_items = static_cast<int>(B) * p.pairs;
   p.n_kt = static_cast<int>((L + kKeys - 1) / kKeys);
   p.last_valid = static_cast<int>(L - static_cast<int64_t>(p.n_kt - 1) * kKeys);
-  if (static_cast<long long>(p.n_items) * p.n_kt != attn_work_steps(B, L))
+  if (static_cast<long long>(p.n_items) * p.n_kt != attn_work_steps(B, Lq, L))
     return cudaErrorInvalidValue;
   const float cap = a.cap;
   const float inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(kD));

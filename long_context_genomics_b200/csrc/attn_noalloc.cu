@@ -97,6 +97,7 @@ extern "C" ag_status ag_attn_fwd_noalloc(const void *q, const void *k, const voi
   a.lse = lse;
   a.B = B;
   a.L = L;
+  a.Lq = L;
   a.Dv = D;
   a.cap = cap;
   a.err = dev->err;

@@ -153,7 +153,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace proj
 
 cudaError_t launch_pair_bias_project(const float *pair, const float *W, float *bias,
-                                     int64_t P, int num_sms, unsigned *err,
+                                     int64_t cells, int num_sms, unsigned *err,
                                      EncodeTiledFn encode, cudaStream_t stream) {
   using namespace proj;
   static std::once_flag once[64];
@@ -168,7 +168,7 @@ cudaError_t launch_pair_bias_project(const float *pair, const float *W, float *b
                                          static_cast<int>(kSmemBytes));
   });
   if (once_err[dev] != cudaSuccess) return once_err[dev];
-  const long long n_cells = static_cast<long long>(P) * P;
+  const long long n_cells = cells;
   // pair as a 2-D tensor: n_cells rows of 128 fp32 channels (512-byte rows).
   CUtensorMap tm;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kCp), static_cast<cuuint64_t>(n_cells)};

@@ -395,37 +395,17 @@ __device__ __forceinline__ void griddep_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
-// 2^x on the FMA pipe (two lanes at once) for x in [-126, 0], used to take
-// part of the exponentials off the special-function unit.  Range reduction
-// x = j + f with j = floor(x): adding 1.5 * 2^23 with round-toward-minus-
-// infinity leaves j in the low mantissa bits of t (integers are exact there).
-// 2^f for f in [0, 1) is a degree-3 polynomial with minimax relative error
-// 7.5e-5 (coefficients fitted for this library), and 2^j is added into the
-// exponent field: the bits of t shifted left by 23 equal j << 23 modulo 2^32.
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
-  constexpr float c0 = 0.9999252557754517f, c1 = 0.695833683013916f,
-                  c2 = 0.22606664896011353f, c3 = 0.07802490144968033f;
-  const float2 t = __fadd2_rd(x, make_float2(kShift, kShift));
-  const float2 j = __fadd2_rn(t, make_float2(-kShift, -kShift));
-  const float2 f = __ffma2_rn(j, make_float2(-1.f, -1.f), x);
-  float2 p = __ffma2_rn(make_float2(c3, c3), f, make_float2(c2, c2));
-  p = __ffma2_rn(p, f, make_float2(c1, c1));
-  p = __ffma2_rn(p, f, make_float2(c0, c0));
-  return make_float2(
-      __int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
-      __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
-}
-
-// 2^(a t - m) on the FMA pipe (two lanes at once) for an integer m in
-// [0, 2^21) and a t - m in [-126, 0]: the same range reduction and
-// polynomial as exp2_poly2, with the product a t and the shift folded into
-// the reduction.  km = 1.5 * 2^23 - m is exact in fp32, so one fused
-// multiply-add rounded toward minus infinity gives T = km + floor(a t)
-// exactly (a t + km is exact before that rounding since |a t| < 2^22);
-// nf = km - T = -floor(a t) is exact, f = a t + nf lies in [0, 1), and the
-// low bits of T hold floor(a t) - m for the exponent.  Saves the separate
-// a t - m product of exp2_poly2(a t - m).
+// 2^(a t - m) on the FMA pipe (two lanes at once), used to take part of the
+// exponentials off the special-function unit; m is an integer in [0, 2^21)
+// and a t - m must lie in [-126, 0].  Range reduction a t = j + f with
+// j = floor(a t): km = 1.5 * 2^23 - m is exact in fp32 and a t + km is exact
+// before rounding (|a t| < 2^22), so one fused multiply-add rounded toward
+// minus infinity gives T = km + j, with j - m in the low mantissa bits of T
+// (integers are exact there); nf = km - T = -j is exact and f = a t + nf
+// lies in [0, 1).  2^f is a degree-3 polynomial with minimax relative error
+// 7.5e-5 (coefficients fitted for this library), and 2^(j - m) is added into
+// the exponent field: the bits of T shifted left by 23 equal (j - m) << 23
+// modulo 2^32.
 __device__ __forceinline__ float2 exp2_poly2_fma(float2 t, float2 a, float2 km) {
   constexpr float c0 = 0.9999252557754517f, c1 = 0.695833683013916f,
                   c2 = 0.22606664896011353f, c3 = 0.07802490144968033f;

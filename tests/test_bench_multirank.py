@@ -90,3 +90,51 @@ def test_single_rank_helpers():
     assert bench.rank_workload(base, 3).seed == base.seed + 3000
     assert bench.max_over_ranks(1.5, torch.device("cpu"), 1) == 1.5
     assert bench.aggregate_rate(1, 8.0, 5, 2.0) == 20.0
+
+
+def _shard_worker(rank: int, world: int, port: int, results):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    if ROOT not in sys.path:
+        sys.path.insert(0, ROOT)
+    import datetime
+
+    import ag_inputs
+    import bench
+
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        L = 160
+        inp = ag_inputs.random_case(2, 8, L, 128, 128, 16, seed=9, batched_bias=True)
+        # Keys and values arrive as contiguous sequence shards, one per rank.
+        k0, k1 = L * rank // world, L * (rank + 1) // world
+        k_full = bench.gather_keys(inp["k"][:, k0:k1].contiguous(), world)
+        v_full = bench.gather_keys(inp["v"][:, k0:k1].contiguous(), world)
+        q0, q1 = bench.query_shard(L, world, rank)
+        slab = bench.bias_rows(inp["bias"], q0, q1)
+        # Local query i of the slab must read the bias row of position q0 + i.
+        rows_ok = all(torch.equal(slab[:, :, i // 16], inp["bias"][:, :, (q0 + i) // 16])
+                      for i in range(q1 - q0))
+        results[rank] = {"k": torch.equal(k_full, inp["k"]), "v": torch.equal(v_full, inp["v"]),
+                         "range": (q0, q1), "rows_ok": rows_ok,
+                         "slab_rows": slab.shape[2]}
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def test_query_sharding_partition_gather_and_bias_rows():
+    """--shard queries on two gloo ranks: the query ranges partition [0, L) in
+    multiples of 32 positions, one all_gather rebuilds every key and value in
+    sequence order, and each rank's bias slab puts the row of position q0 + i
+    at local row i / 16."""
+    world, port = 2, _free_port()
+    results = mp.Manager().dict()
+    mp.spawn(_shard_worker, args=(world, port, results), nprocs=world, join=True)
+    got = [results[r] for r in range(world)]
+    assert all(g["k"] and g["v"] and g["rows_ok"] for g in got)
+    ranges = [g["range"] for g in got]
+    assert ranges[0][0] == 0 and ranges[-1][1] == 160
+    assert all(a[1] == b[0] for a, b in zip(ranges, ranges[1:]))
+    assert all(r[0] % 32 == 0 for r in ranges)
+    assert [g["slab_rows"] for g in got] == [-(-(r[1] - r[0]) // 16) for r in ranges]

@@ -308,6 +308,48 @@ def test_two_streams_at_once(ag, oracle_lib):
         _compare(on[b, h, i], ln[b, h, i], ro, rl, f"stream {n} B={B}")
 
 
+@pytest.mark.parametrize("starts", [(0, 1024), (0, 704, 1408)])
+def test_query_slabs_reproduce_the_full_call(ag, starts):
+    """Queries split into slabs (ag_attn_fwd_query_slab: the slab's q rows and
+    its bias rows, all keys): at L = 2048, B = 2 every call runs whole pairs of
+    query blocks, so each slab's rows equal the full call's bit for bit."""
+    B, L = 2, 2048
+    inp = ag_inputs.random_case(B, 8, L, 128, 128, 16, seed=41, batched_bias=True)
+    q, k, v, bias = (_dev(inp[n]) for n in ("q", "k", "v", "bias"))
+    out, lse = ag.ag_attn_fwd(q, k, v, bias, cap=5.0)
+    ends = starts[1:] + (L,)
+    for q0, q1 in zip(starts, ends):
+        so, sl = ag.ag_attn_fwd_query_slab(q[:, :, q0:q1].contiguous(), k, v,
+                                           bias[:, :, q0 // 16:-(-q1 // 16)].contiguous(),
+                                           cap=5.0)
+        torch.cuda.synchronize()
+        assert torch.equal(so, out[:, :, q0:q1]) and torch.equal(sl, lse[:, :, q0:q1]), \
+            f"slab [{q0}, {q1}) differs from the full call"
+    assert ag.ag_device_error(0) == 0
+
+
+def test_query_slabs_full_context(ag, oracle_lib):
+    """L = 8192 split into four slabs of 2048 queries, as four GPUs would hold
+    them: every slab against the oracle on sampled rows."""
+    L = 8192
+    inp = ag_inputs.random_case(1, 8, L, 128, 128, 16, seed=43)
+    q, k, v, bias = (_dev(inp[n]) for n in ("q", "k", "v", "bias"))
+    for r in range(4):
+        q0, q1 = 2048 * r, 2048 * (r + 1)
+        so, sl = ag.ag_attn_fwd_query_slab(q[:, :, q0:q1].contiguous(), k, v,
+                                           bias[:, q0 // 16:q1 // 16].contiguous(), cap=5.0)
+        torch.cuda.synchronize()
+        rows = ag_inputs.sample_rows(1, 8, 2048, 96, seed=r).numpy()
+        glob = rows.copy()
+        glob[:, 2] += q0
+        ro, rl = oracle_lib.attn_rows(inp["q"], inp["k"], inp["v"], inp["bias"], glob,
+                                      block=16, cap=5.0)
+        b, h, i = rows[:, 0], rows[:, 1], rows[:, 2]
+        _compare(so.double().cpu().numpy()[b, h, i], sl.double().cpu().numpy()[b, h, i],
+                 ro, rl, f"slab {r} of L=8192")
+    assert ag.ag_device_error(0) == 0
+
+
 def test_maximum_length_sampled(ag, oracle_lib):
     inp = ag_inputs.random_case(1, 8, 65536, 128, 128, 16, seed=5)
     out, lse = _gpu_attn(ag, inp, 5.0)
