@@ -318,6 +318,14 @@ def bias_rows(bias: torch.Tensor, q0: int, q1: int, block: int = 16) -> torch.Te
     return bias[..., q0 // block:-(-q1 // block), :].contiguous()
 
 
+def check_device(ag, device: int, where: str) -> None:
+    """Fails with the device error word's code (wait site << 8 | kind) if a
+    bounded wait in one of the kernels ran out."""
+    code = ag.ag_device_error(device)
+    if code:
+        raise RuntimeError(f"{where}: device error word {code:#x} (site {code >> 8})")
+
+
 def aggregate_rate(world: int, units_per_step: float, steps: int, seconds: float) -> float:
     """Whole-job throughput: the units all ranks processed over the slowest
     rank's time (weak scaling: every rank does the same work per step)."""
@@ -428,7 +436,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         flush.zero_()
         step()
     torch.cuda.synchronize()
-    assert ag.ag_device_error(local_rank) == 0
+    check_device(ag, local_rank, "after warm-up or timing")
 
     # ---- device-resident timing --------------------------------------------
     # Events per step: start, then after each layer's projection and after
@@ -457,7 +465,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
                for e in ev]
     attn_ms = [sum(e[1 + 2 * li].elapsed_time(e[2 + 2 * li]) for li in range(nl)) for e in ev]
     total_s = max_over_ranks(sum(step_ms) / 1e3, dev, world)
-    assert ag.ag_device_error(local_rank) == 0
+    check_device(ag, local_rank, "after warm-up or timing")
 
     # ---- end to end through the public API with host buffers ---------------
     names = _e2e_inputs(w0)
@@ -470,7 +478,8 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     barrier()
     e2e_s, e2e_lse = pipelined_e2e(ag, layers, pinned, dev, K)
     e2e_s = max_over_ranks(e2e_s, dev, world)
-    assert math.isfinite(float(e2e_lse.flatten()[0])) and ag.ag_device_error(local_rank) == 0
+    check_device(ag, local_rank, "e2e pipelined")
+    assert math.isfinite(float(e2e_lse.flatten()[0]))
     # (2) One layer at a time on one stream: upload, compute, download.
     ee = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     barrier()
@@ -486,7 +495,8 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         ee[i][1].record(stream)
     barrier()
     serial_s = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ee) / 1e3, dev, world)
-    assert math.isfinite(float(lse_h.flatten()[0])) and ag.ag_device_error(local_rank) == 0
+    check_device(ag, local_rank, "e2e serial")
+    assert math.isfinite(float(lse_h.flatten()[0]))
 
     if rank != 0:
         return
@@ -592,7 +602,7 @@ def run_sharded(args, rank: int, world: int, local_rank: int) -> None:
         flush.zero_()
         step()
     barrier()
-    assert ag.ag_device_error(local_rank) == 0
+    check_device(ag, local_rank, "after warm-up or timing")
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     sampler = ClockSampler(local_rank) if rank == 0 else None
@@ -607,7 +617,8 @@ def run_sharded(args, rank: int, world: int, local_rank: int) -> None:
     barrier()
     clocks = sampler.stop(t_wall0, time.time()) if sampler else None
     total_s = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3, dev, world)
-    assert ag.ag_device_error(local_rank) == 0 and math.isfinite(float(lse[0, 0, 0]))
+    check_device(ag, local_rank, "sharded timing")
+    assert math.isfinite(float(lse[0, 0, 0]))
     if rank != 0:
         return
     pk = peaks()
@@ -662,7 +673,7 @@ def run_backward(args) -> None:
         flush.zero_()
         ag.ag_attn_bwd(d["q"], d["k"], d["v"], bias, lse, dout, cap=w.cap)
     torch.cuda.synchronize()
-    assert ag.ag_device_error(0) == 0
+    check_device(ag, 0, "backward")
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     sampler = ClockSampler(0)
@@ -676,7 +687,7 @@ def run_backward(args) -> None:
         ev[i][1].record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop(t0, time.time())
-    assert ag.ag_device_error(0) == 0
+    check_device(ag, 0, "backward")
     ms = [e[0].elapsed_time(e[1]) for e in ev]
     mean_s = statistics.mean(ms) / 1e3
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
