@@ -703,7 +703,7 @@ def run_backward(args) -> None:
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {**workload_config(w), "step": "ag_attn_bwd (given the forward's lse)",
                    "parallelism": "single GPU"},
-        "gpu_launches": K * ag.ag_attn_bwd_launch_count(),
+        "gpu_launches": K * ag.ag_attn_bwd_launch_count(w.Dv),
         "roofline": {"kernel": "attn_bwd_q_kernel + attn_bwd_kv_kernel", "bound": "alu",
                      "achieved": alg, "peak": fp32_peak, "unit": "TFLOP/s",
                      "frac": alg / fp32_peak, "traffic": None,

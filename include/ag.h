@@ -292,13 +292,19 @@ ag_status ag_attn_fwd_schedule(int64_t B, int64_t L, int sm_pairs, int with_scra
  *   bias_batch_stride = 0 the one shared bias gets the sum over the items;
  *   otherwise item b's cells at dbias + b * bias_batch_stride, the padding
  *   between items untouched), delta [B,H,L].
- * Alignment: q, k, v 2 bytes, the float32 arrays 4 bytes (AG_ERR_ALIGN).
- *   No output may overlap an input or another output (AG_ERR_ALIAS).  Size
- *   and value checks and their statuses as ag_attn_fwd_ex; B == 0 or
- *   L == 0 is a no-op.
- * Two kernels on `stream` (asynchronous); no device memory is allocated;
- * every output value is written by one thread in a fixed order, so results
- * are bitwise reproducible.  The arithmetic is float32 on the CUDA cores.
+ * Alignment: q, k, v 2 bytes, the float32 arrays 4 bytes; with Dv == 128
+ *   also q, k, v, dout and dq 16 bytes (AG_ERR_ALIGN).  No output may
+ *   overlap an input or another output (AG_ERR_ALIAS).  Size and value
+ *   checks and their statuses as ag_attn_fwd_ex; B == 0 or L == 0 is a no-op.
+ * Asynchronous on `stream`; no device memory is allocated; every output
+ * value is written by one thread in a fixed order, so results are bitwise
+ * reproducible.
+ * Dv == 128 runs on the tensor cores (four kernels): dout is first split
+ *   into two bf16 halves (hi = bf16(dout), lo = bf16(dout - hi)) stored in
+ *   dq's memory (which the last kernel then overwrites with dq); the
+ *   products with dout, P and dS take each as such a pair, so that they
+ *   carry 16 significant bits, with fp32 accumulation.
+ * Dv == 192 runs two float32 CUDA-core kernels.
  */
 ag_status ag_attn_bwd(const void *q, const void *k, const void *v, const float *bias,
                       int64_t bias_batch_stride, const float *lse, const float *dout,
@@ -308,10 +314,12 @@ ag_status ag_attn_bwd(const void *q, const void *k, const void *v, const float *
 
 /*
  * ag_attn_bwd_launch_count -- how many kernels a non-empty ag_attn_bwd call
- * launches (a library convenience; the pages have no counterpart).  count
- * is a host pointer (AG_ERR_NULL if NULL).  Launches nothing.
+ * with value width Dv launches: 4 for Dv == 128, 2 for Dv == 192 (a library
+ * convenience; the pages have no counterpart).  count is a host pointer
+ * (AG_ERR_NULL if NULL); AG_ERR_SHAPE for Dv <= 0, AG_ERR_UNSUPPORTED for
+ * other widths.  Launches nothing.
  */
-ag_status ag_attn_bwd_launch_count(int *count);
+ag_status ag_attn_bwd_launch_count(int64_t Dv, int *count);
 
 /*
  * Device error word.  Every wait inside the kernels is bounded (about one

@@ -80,7 +80,7 @@ def _load() -> ctypes.CDLL:
     lib.ag_attn_bwd.argtypes = [vp, vp, vp, vp, i64, vp, vp, i64, i64, i64, i64, i64,
                                 i64, f32, vp, vp, vp, vp, vp, vp]
     lib.ag_attn_bwd.restype = ctypes.c_int
-    lib.ag_attn_bwd_launch_count.argtypes = [ctypes.POINTER(ctypes.c_int)]
+    lib.ag_attn_bwd_launch_count.argtypes = [i64, ctypes.POINTER(ctypes.c_int)]
     lib.ag_attn_bwd_launch_count.restype = ctypes.c_int
     lib.ag_device_error.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int),
                                     ctypes.c_int]
@@ -339,10 +339,10 @@ def ag_attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, bias: torch.T
     return dq, dk, dv, dbias, delta
 
 
-def ag_attn_bwd_launch_count() -> int:
-    """How many kernels a non-empty ag_attn_bwd call launches."""
+def ag_attn_bwd_launch_count(Dv: int = 128) -> int:
+    """How many kernels a non-empty ag_attn_bwd call with value width Dv launches."""
     n = ctypes.c_int(-1)
-    st = lib.ag_attn_bwd_launch_count(ctypes.byref(n))
+    st = lib.ag_attn_bwd_launch_count(int(Dv), ctypes.byref(n))
     if st != AG_OK:
         raise AgError("ag_attn_bwd_launch_count", st)
     return int(n.value)

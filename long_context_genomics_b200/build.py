@@ -18,7 +18,7 @@ CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libag.so")
 SOURCES = ["ag_api.cu", "attn_fwd_sm100.cu", "attn_noalloc.cu", "attn_bwd.cu",
-           "pair_bias_project.cu"]
+           "attn_bwd_sm100.cu", "pair_bias_project.cu"]
 HEADERS = ["sm100.cuh", "ag_internal.h", "attn_bwd_phases.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 

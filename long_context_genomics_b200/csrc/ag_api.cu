@@ -362,6 +362,11 @@ ag_status ag_attn_bwd(const void *q, const void *k, const void *v, const float *
     for (int u = o + 1; u < 5; ++u)
       if (ag::overlap(outs[o], outsz[o], outs[u], outsz[u])) return AG_ERR_ALIAS;
   }
+  // The tensor-core path (value width 128) reads q, k, v, dout and dq's
+  // staging planes with TMA or 16-byte vectors.
+  if (Dv == 128 && (!ag::aligned(q, 16) || !ag::aligned(k, 16) || !ag::aligned(v, 16) ||
+                    !ag::aligned(dout, 16) || !ag::aligned(dq, 16)))
+    return AG_ERR_ALIGN;
   ag::DeviceInfo *dev = nullptr;
   st = ag::device_info(&dev);
   if (st != AG_OK) return st;
@@ -384,12 +389,20 @@ ag_status ag_attn_bwd(const void *q, const void *k, const void *v, const float *
   a.Dv = Dv;
   a.cap = cap;
   a.stream = static_cast<cudaStream_t>(stream);
+  if (ag::attn_bwd_tc_supported(a)) {
+    ag::EncodeTiledFn enc = nullptr;
+    st = ag::get_encoder(&enc);
+    if (st != AG_OK) return st;
+    return ag::from_cuda(ag::launch_attn_bwd_tc(a, dev->num_sms, dev->err, enc));
+  }
   return ag::from_cuda(ag::launch_attn_bwd(a));
 }
 
-ag_status ag_attn_bwd_launch_count(int *count) {
+ag_status ag_attn_bwd_launch_count(int64_t Dv, int *count) {
   if (!count) return AG_ERR_NULL;
-  *count = ag::attn_bwd_kernel_count();
+  if (Dv <= 0) return AG_ERR_SHAPE;
+  if (Dv != 128 && Dv != 192) return AG_ERR_UNSUPPORTED;
+  *count = Dv == 128 ? 4 : ag::attn_bwd_kernel_count();
   return AG_OK;
 }
 

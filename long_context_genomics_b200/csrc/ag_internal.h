@@ -89,6 +89,12 @@ struct AttnBwdLaunch {
 };
 cudaError_t launch_attn_bwd(const AttnBwdLaunch &a);
 int attn_bwd_kernel_count();
+// Tensor-core backward (attn_bwd_sm100.cu): value width 128, q, k, v, dout
+// and dq 16-byte aligned; four launches (dout split, query pass 1, key pass,
+// query pass 2).  Uses dq as the staging place of dout's bf16 halves.
+bool attn_bwd_tc_supported(const AttnBwdLaunch &a);
+cudaError_t launch_attn_bwd_tc(const AttnBwdLaunch &a, int num_sms, unsigned *err,
+                               EncodeTiledFn encode);
 
 // Projects `cells` consecutive cells of 128 channels into 8 head planes of
 // `cells` floats each.

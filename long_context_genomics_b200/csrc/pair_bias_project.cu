@@ -11,8 +11,12 @@
 // persistent CTA per SM streams chunks of 32 consecutive cells (16 KB) into a
 // 12-stage shared-memory ring with TMA (one producer lane; the pair tensor is
 // seen as [cells, 128] fp32 rows, four 32-channel boxes per chunk with the
-// 128-byte swizzle), so up to 192 KB per SM are in flight.  Each of eight
-// consumer warps takes whole chunks: lane l owns cell l of the chunk and sums
+// 128-byte swizzle), so up to 192 KB per SM are in flight.  Each of six
+// consumer warps takes whole chunks (chunk n of the CTA goes to warp n % 6,
+// so warp w always uses ring slots w and w + 6 and waits for their phases in
+// order; a slot shared by warps would let a warp wait for a phase one ahead
+// of the slot's current one, which a parity wait cannot tell from the phase
+// before).  Lane l owns cell l of the chunk and sums
 // its 128 channels for all 8 heads in registers (packed fp32x2 products, two
 // heads per instruction).  The swizzle puts the 16-byte channel group g of
 // cell l at group slot g ^ (l % 8) of its 128-byte row, so the eight lanes of
@@ -35,7 +39,8 @@ constexpr int kChunkCells = 32;                      // one cell per lane
 constexpr int kChunkBytes = kChunkCells * kCellBytes;  // 16 KB
 constexpr int kBoxBytes = kChunkCells * 128;         // 32 cells x 32 channels
 constexpr int kStages = 12;
-constexpr int kConsumerWarps = 8;
+constexpr int kConsumerWarps = 6;
+static_assert(kStages % kConsumerWarps == 0, "each ring slot belongs to one consumer warp");
 constexpr int kThreads = (kConsumerWarps + 1) * 32;  // + producer warp
 constexpr int kWBytes = kCp * kH * 4;                // 4 KB
 constexpr size_t kSmemBytes = 1024 + kStages * kChunkBytes + kWBytes + 2 * kStages * 8 + 16;
@@ -105,7 +110,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // Consumer warp `warp` takes the CTA's chunks it = warp, warp + 8, ...
+    // Consumer warp `warp` takes the CTA's chunks it = warp, warp + 6, ...
     const float4 *w4 = reinterpret_cast<const float4 *>(w_s);  // W[c][0..3], W[c][4..7]
     const uint32_t swz = static_cast<uint32_t>(lane & 7);
     for (uint32_t it = warp;; it += kConsumerWarps) {

@@ -176,6 +176,11 @@ def test_backward_validation(ag):
         assert _bwd(ag, **{name: None}) == 1, name  # AG_ERR_NULL
     assert _bwd(ag, q=A16 + 1) == 3               # bf16 needs 2-byte alignment
     assert _bwd(ag, lse=A16 + 2) == 3             # fp32 needs 4-byte alignment
+    # Value width 128 (the tensor-core path): q, k, v, dout, dq 16-byte aligned.
+    for name in ("q", "k", "v", "dout", "dq"):
+        assert _bwd(ag, **{name: (A16 * 6 if name == "dout" else
+                                  A16 * 1000 if name == "dq" else
+                                  A16 * {"q": 1, "k": 2, "v": 3}[name]) + 4}) == 3, name
     # Outputs overlapping an input or one another.
     assert _bwd(ag, dq=A16 * 6) == 7              # dq on dout
     assert _bwd(ag, delta=A16 * 1000 + 64) == 7   # delta inside dq
@@ -184,6 +189,9 @@ def test_backward_validation(ag):
 
 def test_backward_launch_count(ag):
     n = ctypes.c_int(-1)
-    assert ag.lib.ag_attn_bwd_launch_count(ctypes.byref(n)) == 0 and n.value == 2
-    assert ag.lib.ag_attn_bwd_launch_count(None) == 1
-    assert ag.ag_attn_bwd_launch_count() == 2
+    assert ag.lib.ag_attn_bwd_launch_count(128, ctypes.byref(n)) == 0 and n.value == 4
+    assert ag.lib.ag_attn_bwd_launch_count(192, ctypes.byref(n)) == 0 and n.value == 2
+    assert ag.lib.ag_attn_bwd_launch_count(128, None) == 1   # AG_ERR_NULL
+    assert ag.lib.ag_attn_bwd_launch_count(0, ctypes.byref(n)) == 2
+    assert ag.lib.ag_attn_bwd_launch_count(96, ctypes.byref(n)) == 4
+    assert ag.ag_attn_bwd_launch_count() == 4 and ag.ag_attn_bwd_launch_count(192) == 2
