@@ -646,9 +646,15 @@ def backward_flops(w) -> float:
 
 
 def backward_executed_flops(w) -> float:
-    """FLOPs the two backward kernels execute: the delta pass 2 (D + Dv), the
-    dq pass 2 (D + Dv) + 2 D and the key kernel 2 (D + Dv) + 2 D + 2 Dv per
+    """FLOPs the backward kernels execute per call.  Value width 128 (tensor
+    cores, dout, P and dS each taken as a pair of bf16 halves): query pass 1
+    S + 2 dP, the key pass S^T + 2 dP^T + 3 dV + 2 dK, query pass 2
+    S + 2 dP + 2 dQ, i.e. 16 products of 2 L^2 x 128 per (item, head).
+    Value width 192 (CUDA cores): the delta pass 2 (D + Dv), the dq pass
+    2 (D + Dv) + 2 D and the key kernel 2 (D + Dv) + 2 D + 2 Dv per
     (item, head, query, key)."""
+    if w.Dv == 128:
+        return 2.0 * w.B * w.H * w.L * w.L * 128 * 16
     return 2.0 * w.B * w.H * w.L * w.L * (3 * (w.D + w.Dv) + 2 * w.D + w.Dv)
 
 
@@ -692,23 +698,34 @@ def run_backward(args) -> None:
     mean_s = statistics.mean(ms) / 1e3
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     max_mhz = (clocks or {}).get("sm_max_mhz") or 1965.0
-    # FP32 FMA pipe: 128 lanes per SM, 2 FLOPs per FMA, at the maximum SM clock.
-    fp32_peak = sms * 128 * 2 * max_mhz * 1e6 / 1e12
     alg = backward_flops(w) / mean_s / 1e12
     exe = backward_executed_flops(w) / mean_s / 1e12
+    if w.Dv == 128:
+        pk = peaks()
+        roof = {"kernel": "bwd_query_kernel x 2 + bwd_key_kernel (tcgen05)", "bound": "tensor",
+                "achieved": alg, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": alg / pk["bf16_tflops"], "traffic": None,
+                "peak_kind": "bf16 burst (" + pk["source"] + ")",
+                "executed_tflops": exe, "frac_executed": exe / pk["bf16_tflops"]}
+        dtype = "bf16"
+    else:
+        # FP32 FMA pipe: 128 lanes per SM, 2 FLOPs per FMA, at the maximum SM clock.
+        fp32_peak = sms * 128 * 2 * max_mhz * 1e6 / 1e12
+        roof = {"kernel": "attn_bwd_q_kernel + attn_bwd_kv_kernel", "bound": "alu",
+                "achieved": alg, "peak": fp32_peak, "unit": "TFLOP/s",
+                "frac": alg / fp32_peak, "traffic": None,
+                "peak_kind": f"fp32 FMA pipe, {sms} SMs x 128 lanes x 2 x {max_mhz:.0f} MHz",
+                "executed_tflops": exe, "frac_executed": exe / fp32_peak}
+        dtype = "f32"
     line = {
         "metric": f"pair-bias attention backward TFLOP/s at L={w.L}", "value": alg,
         "unit": "TFLOP/s", "n_gpus": 1, "steps": K, "warmup": args.warmup,
         "ms_per_step": 1e3 * mean_s, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "vs_baseline": None, "dtype": dtype, "data": "synthetic",
         "config": {**workload_config(w), "step": "ag_attn_bwd (given the forward's lse)",
                    "parallelism": "single GPU"},
         "gpu_launches": K * ag.ag_attn_bwd_launch_count(w.Dv),
-        "roofline": {"kernel": "attn_bwd_q_kernel + attn_bwd_kv_kernel", "bound": "alu",
-                     "achieved": alg, "peak": fp32_peak, "unit": "TFLOP/s",
-                     "frac": alg / fp32_peak, "traffic": None,
-                     "peak_kind": f"fp32 FMA pipe, {sms} SMs x 128 lanes x 2 x {max_mhz:.0f} MHz",
-                     "executed_tflops": exe, "frac_executed": exe / fp32_peak},
+        "roofline": roof,
         "ms": {"median": statistics.median(ms), "p95": sorted(ms)[int(0.95 * (K - 1))]},
         "clocks": clocks,
     }

@@ -707,7 +707,86 @@ __device__ __forceinline__ bool store_p(Barriers *bars, uint32_t tmem, int g,
   return true;
 }
 
-// Static-shift segment: every warpgroup takes 32 keys of every key tile.
+// Static-shift segment with alternating groups (value width 128): the warps
+// split into two groups that take alternate key tiles, group q = warpgroups
+// 2q and 2q + 1 taking the tiles in S buffer q (64 keys each per tile) and
+// writing P buffer q.  One group's waits (for its logits, for the previous
+// PV of its P buffer, for its tensor-memory loads and stores) are covered by
+// the other group's arithmetic, so the special-function unit stays busy.
+// A group only ever waits on its own S and P buffers' barriers, in order.
+template <int DV>
+__device__ __forceinline__ bool segment_static_grouped(const Segment &sg, const float *brow,
+                                                       uint32_t tmem, uint32_t lane_base, int g,
+                                                       const Params &p, Barriers *bars,
+                                                       uint32_t rank,
+                                                       const uint32_t (&sf_remote)[2],
+                                                       const uint32_t (&pf_remote)[2],
+                                                       SoftCounters &c, volatile int *abort,
+                                                       float &d) {
+  static_assert(Tmem<DV>::kNP == 2, "one P buffer per group");
+  using T = Tmem<DV>;
+  const int q = g >> 1, hk = g & 1;  // group (S and P buffer), key half
+  StaticK k;
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  k.sc = make_float2(p.qk_scale, p.qk_scale);
+  k.a = make_float2(p.A, p.A);
+  k.nsh = make_float2(-p.shift, -p.shift);
+  k.km = make_float2(kShift - p.shift, kShift - p.shift);
+  float2 acc = make_float2(0.f, 0.f);
+  // Key tile j of the segment is global tile c.su + (j - kb): buffer (that) & 1.
+  const int j0 = sg.kb + static_cast<int>((static_cast<uint32_t>(q) - c.su) & 1u);
+  float bc[4] = {0.f, 0.f, 0.f, 0.f};
+  auto load_bias4 = [&](int j) {
+    const int J0 = j * 8 + hk * 4;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) bc[e] = (J0 + e < p.P) ? __ldg(brow + J0 + e) : 0.f;
+  };
+  if (j0 < sg.ke) load_bias4(j0);
+  for (int j = j0; j < sg.ke; j += 2) {
+    const uint32_t n = (c.su + static_cast<uint32_t>(j - sg.kb)) >> 1;  // use of buffer q
+    const int nvalid = (j + 1 == p.n_kt) ? p.last_valid : kKeys;
+    bool ok = mbar_wait(&bars->s_full[q], n & 1u, abort, p.err, kSiteSoftS);
+    if (!__all_sync(0xffffffffu, ok)) return false;
+    tc_fence_after();
+    const uint32_t tS = tmem + 128u * q + 64u * hk + lane_base;
+    const uint32_t tP = tmem + T::kColP + 64u * q + 32u * hk + lane_base;
+    const float m = p.bias_mul;
+    uint32_t s[32], pk[16];
+    tmem_ld32(tS, s);
+    tmem_wait_ld(s);
+    if (nvalid == kKeys)
+      chunk_static<false>(s, bc[0] * m, bc[1] * m, k, 64 * hk, nvalid, acc, pk);
+    else
+      chunk_static<true>(s, bc[0] * m, bc[1] * m, k, 64 * hk, nvalid, acc, pk);
+    if (n > 0) {  // the PV that last read P buffer q
+      ok = mbar_wait(&bars->pv_done[q], (n - 1) & 1u, abort, p.err, kSiteSoftPV);
+      if (!__all_sync(0xffffffffu, ok)) return false;
+    }
+    tc_fence_after();
+    tmem_st16(tP, pk);  // the first 32 keys' probabilities
+    tmem_ld32(tS + 32, s);
+    tmem_wait_ld(s);
+    tc_fence_before();
+    warp_arrive_leader(&bars->s_free[q], sf_remote[q], rank);  // S(j) fully read
+    if (nvalid == kKeys)
+      chunk_static<false>(s, bc[2] * m, bc[3] * m, k, 64 * hk + 32, nvalid, acc, pk);
+    else
+      chunk_static<true>(s, bc[2] * m, bc[3] * m, k, 64 * hk + 32, nvalid, acc, pk);
+    if (j + 2 < sg.ke) load_bias4(j + 2);
+    tmem_st16(tP + 16, pk);
+    tmem_wait_st();
+    tc_fence_before();
+    warp_arrive_leader(&bars->p_full[q], pf_remote[q], rank);
+  }
+  const uint32_t tiles = static_cast<uint32_t>(sg.ke - sg.kb);
+  c.su += tiles;
+  c.pu += tiles;
+  d = acc.x + acc.y;
+  return true;
+}
+
+// Static-shift segment: every warpgroup takes 32 keys of every key tile
+// (value width 192, whose single P buffer both groups would share).
 template <int MODE, int DV>
 __device__ __forceinline__ bool segment_static(const Segment &sg, const float *brow,
                                                uint32_t tmem, uint32_t lane_base, int g,
@@ -848,7 +927,10 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc, uint32_t 
                         (static_cast<size_t>(h) * p.bias_rows + I) * p.P;
     float m = kStatic ? p.shift : -INFINITY;  // log2 units
     float d = 0.f;
-    if constexpr (kStatic) {
+    if constexpr (kStatic && DV == 128) {
+      ok = segment_static_grouped<DV>(sg, brow, tmem, lane_base, g, p, bars, rank, sf_remote,
+                                      pf_remote, c, abort, d);
+    } else if constexpr (kStatic) {
       ok = segment_static<MODE, DV>(sg, brow, tmem, lane_base, g, p, bars, rank, sf_remote,
                                     pf_remote, c, abort, d);
     } else {
@@ -972,10 +1054,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(&bars->v_full[s], loads);
       mbar_init(&bars->v_empty[s], 1);
     }
+    // Static cap at value width 128: one warp group per S and P buffer;
+    // otherwise every softmax warp takes part in every key tile.
+    constexpr uint32_t kSPArrivals =
+        (MODE == kStaticCap && DV == 128) ? kPairSoftWarps / 2 : kPairSoftWarps;
     for (int u = 0; u < 2; ++u) {
       mbar_init(&bars->s_full[u], 1);
-      mbar_init(&bars->s_free[u], kPairSoftWarps);
-      mbar_init(&bars->p_full[u], kPairSoftWarps);
+      mbar_init(&bars->s_free[u], kSPArrivals);
+      mbar_init(&bars->p_full[u], kSPArrivals);
       mbar_init(&bars->pv_done[u], 1);
     }
     mbar_init(&bars->o_full, 1);

@@ -27,10 +27,16 @@ def test_backward_flops_count_five_products():
                 "dQ = dS K": 2 * 128, "dK = dS^T Q": 2 * 128}
     pairs = 1 * 8 * 8192 * 8192
     assert bench.backward_flops(w) == pairs * sum(per_pair.values())
-    # The kernels recompute S and dP in three passes (delta, dq, dk/dv) and
-    # add the three gradient products once each.
-    executed = 3 * (2 * 128 + 2 * 128) + 2 * 128 + 2 * 128 + 2 * 128
-    assert bench.backward_executed_flops(w) == pairs * executed
+    # Value width 128, tensor cores: S and dP in three passes (delta, keys,
+    # dq), dout, P and dS each as two bf16 halves: pass 1 S + 2 dP, the key
+    # pass S + 2 dP + 3 dV + 2 dK, pass 2 S + 2 dP + 2 dQ.
+    executed = (1 + 2) + (1 + 2 + 3 + 2) + (1 + 2 + 2)
+    assert bench.backward_executed_flops(w) == pairs * 2 * 128 * executed
+    # Value width 192, CUDA cores: S and dP recomputed in three passes, the
+    # three gradient products once each.
+    w192 = ag_inputs.Workload("w192", B=1, L=8192, seed=0, Dv=192)
+    executed = 3 * (2 * 128 + 2 * 192) + 2 * 128 + 2 * 128 + 2 * 192
+    assert bench.backward_executed_flops(w192) == pairs * executed
 
 
 def test_workload_names_follow_the_bias_mode():
