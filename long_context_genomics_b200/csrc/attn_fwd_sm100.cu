@@ -604,12 +604,21 @@ __device__ __forceinline__ void load_bias(const float *brow, int j, int g, int P
   for (int e = 0; e < 2; ++e) bn[e] = (J0 + e < P) ? __ldg(brow + J0 + e) : 0.f;
 }
 
+// The compact bias cells of warpgroup half hk's 64 keys of key tile j:
+// bias[h, I, 8j + 4hk + e] (0 past the end: those keys are masked).
+__device__ __forceinline__ void load_bias4(const float *brow, int j, int hk, int P,
+                                           float (&bn)[4]) {
+  const int J0 = j * 8 + hk * 4;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) bn[e] = (J0 + e < P) ? __ldg(brow + J0 + e) : 0.f;
+}
+
 // Column pairs (out of every 8) whose exponential runs on the FMA pipe
 // (exp2_poly2_fma) instead of the special-function unit, in kStaticCap.  The
 // SFU still computes every tanh, so it does 1 + (8 - kEmuPairs) / 8
 // operations per logit.
 #ifndef AG_EXP2_EMU_PAIRS
-#define AG_EXP2_EMU_PAIRS 6
+#define AG_EXP2_EMU_PAIRS 5
 #endif
 constexpr int kEmuPairs = AG_EXP2_EMU_PAIRS;
 
@@ -625,12 +634,12 @@ struct StaticK {
 // t = tanh(y), p = 2^(A t - shift), y = s qk_scale + b / cap.  Adds the row
 // sum into acc and packs 16 bf16 pairs of P.  kMask zeroes keys >= nvalid
 // (only the last key tile of a ragged length needs it).
-template <bool kMask>
-__device__ __forceinline__ void chunk_static(const uint32_t (&s)[32], float b0, float b1,
+template <bool kMask, int N>
+__device__ __forceinline__ void chunk_static(const uint32_t (&s)[N], float b0, float b1,
                                              const StaticK &k, int col0, int nvalid,
-                                             float2 &acc, uint32_t (&pk)[16]) {
+                                             float2 &acc, uint32_t (&pk)[N / 2]) {
 #pragma unroll
-  for (int e = 0; e < 16; ++e) {
+  for (int e = 0; e < N / 2; ++e) {
     const float bb = e < 8 ? b0 : b1;
     const float2 y = __ffma2_rn(
         make_float2(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1])), k.sc,
@@ -680,7 +689,7 @@ __device__ __forceinline__ bool load_s(Barriers *bars, uint32_t tmem, int g, uin
   tmem_ld32(tmem + 128u * sb + 32u * g + lane_base, s);
   tmem_wait_ld(s);
   tc_fence_before();
-  warp_arrive_leader(&bars->s_free[sb], sf_remote[sb], rank);
+  warp_arrive_leader(&bars->s_free[sb], sb ? sf_remote[1] : sf_remote[0], rank);
   return true;
 }
 
@@ -703,7 +712,45 @@ __device__ __forceinline__ bool store_p(Barriers *bars, uint32_t tmem, int g,
   tmem_st16(tmem + T::kColP + 64u * pb + 16u * g + lane_base, pk);
   tmem_wait_st();
   tc_fence_before();
-  warp_arrive_leader(&bars->p_full[pb], pf_remote[pb], rank);
+  warp_arrive_leader(&bars->p_full[pb], pb ? pf_remote[1] : pf_remote[0], rank);
+  return true;
+}
+
+// One 64-key half tile of a grouped static segment (see below): tS and tP
+// address this warp's S and P columns, bc holds the four bias cells.
+template <bool kMask>
+__device__ __forceinline__ bool tile_grouped(uint32_t tS, uint32_t tP, const float (&bc)[4],
+                                             float m, const StaticK &k, int col0, int nvalid,
+                                             uint32_t n, int q, uint32_t sf_q, Barriers *bars,
+                                             uint32_t rank, const Params &p,
+                                             volatile int *abort, float2 &acc) {
+  uint32_t sa[16], sb[16], pk[8];
+  tmem_ld16(tS, sa);
+  tmem_wait_ld16(sa);
+  tmem_ld16(tS + 16u, sb);
+  chunk_static<kMask, 16>(sa, bc[0] * m, bc[0] * m, k, col0, nvalid, acc, pk);
+  if (n > 0) {  // the PV that last read P buffer q
+    const bool ok = mbar_wait(&bars->pv_done[q], (n - 1) & 1u, abort, p.err, kSiteSoftPV);
+    if (!__all_sync(0xffffffffu, ok)) {
+      tmem_wait_ld16(sb);
+      return false;
+    }
+  }
+  tc_fence_after();
+  tmem_st8(tP, pk);
+  tmem_wait_ld16(sb);
+  tmem_ld16(tS + 32u, sa);
+  chunk_static<kMask, 16>(sb, bc[1] * m, bc[1] * m, k, col0 + 16, nvalid, acc, pk);
+  tmem_st8(tP + 8u, pk);
+  tmem_wait_ld16(sa);
+  tmem_ld16(tS + 48u, sb);
+  chunk_static<kMask, 16>(sa, bc[2] * m, bc[2] * m, k, col0 + 32, nvalid, acc, pk);
+  tmem_st8(tP + 16u, pk);
+  tmem_wait_ld16(sb);
+  tc_fence_before();
+  warp_arrive_leader(&bars->s_free[q], sf_q, rank);  // S fully read
+  chunk_static<kMask, 16>(sb, bc[3] * m, bc[3] * m, k, col0 + 48, nvalid, acc, pk);
+  tmem_st8(tP + 24u, pk);
   return true;
 }
 
@@ -733,15 +780,14 @@ __device__ __forceinline__ bool segment_static_grouped(const Segment &sg, const 
   k.nsh = make_float2(-p.shift, -p.shift);
   k.km = make_float2(kShift - p.shift, kShift - p.shift);
   float2 acc = make_float2(0.f, 0.f);
+  // This group's barriers in the even CTA, as scalars (an array indexed by q
+  // would live in local memory).
+  const uint32_t sf_q = q ? sf_remote[1] : sf_remote[0];
+  const uint32_t pf_q = q ? pf_remote[1] : pf_remote[0];
   // Key tile j of the segment is global tile c.su + (j - kb): buffer (that) & 1.
   const int j0 = sg.kb + static_cast<int>((static_cast<uint32_t>(q) - c.su) & 1u);
   float bc[4] = {0.f, 0.f, 0.f, 0.f};
-  auto load_bias4 = [&](int j) {
-    const int J0 = j * 8 + hk * 4;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) bc[e] = (J0 + e < p.P) ? __ldg(brow + J0 + e) : 0.f;
-  };
-  if (j0 < sg.ke) load_bias4(j0);
+  if (j0 < sg.ke) load_bias4(brow, j0, hk, p.P, bc);
   for (int j = j0; j < sg.ke; j += 2) {
     const uint32_t n = (c.su + static_cast<uint32_t>(j - sg.kb)) >> 1;  // use of buffer q
     const int nvalid = (j + 1 == p.n_kt) ? p.last_valid : kKeys;
@@ -751,37 +797,56 @@ __device__ __forceinline__ bool segment_static_grouped(const Segment &sg, const 
     const uint32_t tS = tmem + 128u * q + 64u * hk + lane_base;
     const uint32_t tP = tmem + T::kColP + 64u * q + 32u * hk + lane_base;
     const float m = p.bias_mul;
-    uint32_t s[32], pk[16];
-    tmem_ld32(tS, s);
-    tmem_wait_ld(s);
+    // Four pieces of 16 keys (one bias cell each), the tensor-memory load of
+    // the next piece in flight while this one is computed.  The P buffer is
+    // written once the PV that last read it has finished; the S buffer is
+    // released once its last piece has arrived in registers.
     if (nvalid == kKeys)
-      chunk_static<false>(s, bc[0] * m, bc[1] * m, k, 64 * hk, nvalid, acc, pk);
+      ok = tile_grouped<false>(tS, tP, bc, m, k, 64 * hk, nvalid, n, q, sf_q, bars, rank, p,
+                               abort, acc);
     else
-      chunk_static<true>(s, bc[0] * m, bc[1] * m, k, 64 * hk, nvalid, acc, pk);
-    if (n > 0) {  // the PV that last read P buffer q
-      ok = mbar_wait(&bars->pv_done[q], (n - 1) & 1u, abort, p.err, kSiteSoftPV);
-      if (!__all_sync(0xffffffffu, ok)) return false;
-    }
-    tc_fence_after();
-    tmem_st16(tP, pk);  // the first 32 keys' probabilities
-    tmem_ld32(tS + 32, s);
-    tmem_wait_ld(s);
-    tc_fence_before();
-    warp_arrive_leader(&bars->s_free[q], sf_remote[q], rank);  // S(j) fully read
-    if (nvalid == kKeys)
-      chunk_static<false>(s, bc[2] * m, bc[3] * m, k, 64 * hk + 32, nvalid, acc, pk);
-    else
-      chunk_static<true>(s, bc[2] * m, bc[3] * m, k, 64 * hk + 32, nvalid, acc, pk);
-    if (j + 2 < sg.ke) load_bias4(j + 2);
-    tmem_st16(tP + 16, pk);
+      ok = tile_grouped<true>(tS, tP, bc, m, k, 64 * hk, nvalid, n, q, sf_q, bars, rank, p,
+                              abort, acc);
+    if (!ok) return false;
+    if (j + 2 < sg.ke) load_bias4(brow, j + 2, hk, p.P, bc);
     tmem_wait_st();
     tc_fence_before();
-    warp_arrive_leader(&bars->p_full[q], pf_remote[q], rank);
+    warp_arrive_leader(&bars->p_full[q], pf_q, rank);
   }
   const uint32_t tiles = static_cast<uint32_t>(sg.ke - sg.kb);
   c.su += tiles;
   c.pu += tiles;
   d = acc.x + acc.y;
+  return true;
+}
+
+// One warpgroup's 32 keys of a key tile in an ungrouped static segment:
+// tS and tP address this warp's S and P columns, bc holds the two bias cells.
+template <bool kMask>
+__device__ __forceinline__ bool tile_split(uint32_t tS, uint32_t tP, const float (&bc)[2],
+                                           float m, const StaticK &k, int col0, int nvalid,
+                                           uint32_t pn, uint32_t pb, uint32_t sb, uint32_t sfr,
+                                           Barriers *bars, uint32_t rank, const Params &p,
+                                           volatile int *abort, float2 &acc) {
+  uint32_t sa[16], sc[16], pk[8];
+  tmem_ld16(tS, sa);
+  tmem_wait_ld16(sa);
+  tmem_ld16(tS + 16u, sc);
+  chunk_static<kMask, 16>(sa, bc[0] * m, bc[0] * m, k, col0, nvalid, acc, pk);
+  if (pn > 0) {  // the PV that last read this P buffer
+    const bool ok = mbar_wait(&bars->pv_done[pb], (pn - 1) & 1u, abort, p.err, kSiteSoftPV);
+    if (!__all_sync(0xffffffffu, ok)) {
+      tmem_wait_ld16(sc);
+      return false;
+    }
+  }
+  tc_fence_after();
+  tmem_st8(tP, pk);
+  tmem_wait_ld16(sc);
+  tc_fence_before();
+  warp_arrive_leader(&bars->s_free[sb], sfr, rank);  // S fully read
+  chunk_static<kMask, 16>(sc, bc[1] * m, bc[1] * m, k, col0 + 16, nvalid, acc, pk);
+  tmem_st8(tP + 8u, pk);
   return true;
 }
 
@@ -795,6 +860,7 @@ __device__ __forceinline__ bool segment_static(const Segment &sg, const float *b
                                                const uint32_t (&pf_remote)[2],
                                                SoftCounters &c, volatile int *abort,
                                                float &d) {
+  using T = Tmem<DV>;
   StaticK k;
   constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
   k.sc = make_float2(p.qk_scale, p.qk_scale);
@@ -807,14 +873,28 @@ __device__ __forceinline__ bool segment_static(const Segment &sg, const float *b
   for (int j = sg.kb; j < sg.ke; ++j) {
     if (j + 1 < sg.ke) load_bias(brow, j + 1, g, p.P, bn);
     const int nvalid = (j + 1 == p.n_kt) ? p.last_valid : kKeys;
-    uint32_t s[32], pk[16];
-    if (!load_s(bars, tmem, g, lane_base, rank, sf_remote, c, p, abort, s)) return false;
-    const float b0 = bc[0] * p.bias_mul, b1 = bc[1] * p.bias_mul;
+    const uint32_t sb = c.su & 1u, sph = (c.su >> 1) & 1u;
+    ++c.su;
+    bool ok = mbar_wait(&bars->s_full[sb], sph, abort, p.err, kSiteSoftS);
+    if (!__all_sync(0xffffffffu, ok)) return false;
+    tc_fence_after();
+    const uint32_t tS = tmem + 128u * sb + 32u * g + lane_base;
+    const uint32_t pb = c.pu % T::kNP, pn = c.pu / T::kNP;
+    ++c.pu;
+    const uint32_t tP = tmem + T::kColP + 64u * pb + 16u * g + lane_base;
+    // Two pieces of 16 keys (one bias cell each), the second piece's
+    // tensor-memory load in flight while the first is computed.
+    const uint32_t sfr = sb ? sf_remote[1] : sf_remote[0];
     if (nvalid == kKeys)
-      chunk_static<false>(s, b0, b1, k, 32 * g, nvalid, acc, pk);
+      ok = tile_split<false>(tS, tP, bc, p.bias_mul, k, 32 * g, nvalid, pn, pb, sb, sfr, bars,
+                             rank, p, abort, acc);
     else
-      chunk_static<true>(s, b0, b1, k, 32 * g, nvalid, acc, pk);
-    if (!store_p<DV>(bars, tmem, g, lane_base, rank, pf_remote, c, p, abort, pk)) return false;
+      ok = tile_split<true>(tS, tP, bc, p.bias_mul, k, 32 * g, nvalid, pn, pb, sb, sfr, bars,
+                            rank, p, abort, acc);
+    if (!ok) return false;
+    tmem_wait_st();
+    tc_fence_before();
+    warp_arrive_leader(&bars->p_full[pb], pb ? pf_remote[1] : pf_remote[0], rank);
     bc[0] = bn[0];
     bc[1] = bn[1];
   }
@@ -967,57 +1047,55 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc, uint32_t 
 #pragma unroll
     for (int q = 0; q < kWG; ++q) dsum += xc->dpart[q][r];
     const uint32_t tO = tmem + T::kColO + (DV / 4) * g + lane_base;
-    uint32_t o[32];
-    tmem_ld32(tO, o);
-    tmem_wait_ld(o);
-    uint32_t o2[16];  // columns 32 .. 47 of this warpgroup's 48 (DV = 192)
-    if constexpr (DV == 192) {
-      tmem_ld16(tO + 32, o2);
-      tmem_wait_ld16(o2);
+    const float lse_b = (m + lg2_approx(dsum)) * kLn2;
+    float *orow_base;
+    float *lse_dst;
+    if (sg.dest == kDestScratch) {
+      const size_t slot = (static_cast<size_t>(cluster_index()) * 2 + rank) * 128 + r;
+      orow_base = p.ws_out + slot * DV;
+      lse_dst = p.ws_lse + slot;
+    } else {
+      orow_base = p.out + row * DV;
+      lse_dst = p.lse + row;
+    }
+    float4 *orow = reinterpret_cast<float4 *>(orow_base + (DV / 4) * g);
+    float wb = 1.f / dsum, wa = 0.f, lse_w = lse_b;
+    if (sg.dest == kDestMerge) {
+      // Log-sum-exp merge with the first piece: lse = log(e^a + e^b),
+      // out = e^(a - lse) out_a + e^(b - lse) O_b / d_b.
+      const float M = fmaxf(lse_a, lse_b);
+      const float ea = ex2_approx((lse_a - M) * kLog2e);
+      const float eb = ex2_approx((lse_b - M) * kLog2e);
+      const float inv = 1.f / (ea + eb);
+      wa = ea * inv;
+      wb = eb * inv / dsum;
+      lse_w = M + lg2_approx(ea + eb) * kLn2;
+    }
+    // This warpgroup's DV / 4 columns of the row, 16 at a time (every lane
+    // loads: tcgen05.ld is warp-wide; rows that do not exist store nothing).
+#pragma unroll 1
+    for (int c16 = 0; c16 < DV / 4 / 16; ++c16) {
+      uint32_t o[16];
+      tmem_ld16(tO + 16u * c16, o);
+      tmem_wait_ld16(o);
+      if (writes) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float4 val = make_float4(__uint_as_float(o[4 * e]) * wb, __uint_as_float(o[4 * e + 1]) * wb,
+                                   __uint_as_float(o[4 * e + 2]) * wb,
+                                   __uint_as_float(o[4 * e + 3]) * wb);
+          if (sg.dest == kDestMerge) {
+            const float4 av = orow[4 * c16 + e];
+            val.x = fmaf(wa, av.x, val.x);
+            val.y = fmaf(wa, av.y, val.y);
+            val.z = fmaf(wa, av.z, val.z);
+            val.w = fmaf(wa, av.w, val.w);
+          }
+          orow[4 * c16 + e] = val;
+        }
+      }
     }
     if (writes) {
-      const float lse_b = (m + lg2_approx(dsum)) * kLn2;
-      float *orow_base;
-      float *lse_dst;
-      if (sg.dest == kDestScratch) {
-        const size_t slot = (static_cast<size_t>(cluster_index()) * 2 + rank) * 128 + r;
-        orow_base = p.ws_out + slot * DV;
-        lse_dst = p.ws_lse + slot;
-      } else {
-        orow_base = p.out + row * DV;
-        lse_dst = p.lse + row;
-      }
-      float4 *orow = reinterpret_cast<float4 *>(orow_base + (DV / 4) * g);
-      float wb = 1.f / dsum, wa = 0.f, lse_w = lse_b;
-      if (sg.dest == kDestMerge) {
-        // Log-sum-exp merge with the first piece: lse = log(e^a + e^b),
-        // out = e^(a - lse) out_a + e^(b - lse) O_b / d_b.
-        const float M = fmaxf(lse_a, lse_b);
-        const float ea = ex2_approx((lse_a - M) * kLog2e);
-        const float eb = ex2_approx((lse_b - M) * kLog2e);
-        const float inv = 1.f / (ea + eb);
-        wa = ea * inv;
-        wb = eb * inv / dsum;
-        lse_w = M + lg2_approx(ea + eb) * kLn2;
-      }
-      auto put = [&](int e, const uint32_t *v) {
-        float4 val = make_float4(__uint_as_float(v[0]) * wb, __uint_as_float(v[1]) * wb,
-                                 __uint_as_float(v[2]) * wb, __uint_as_float(v[3]) * wb);
-        if (sg.dest == kDestMerge) {
-          const float4 a = orow[e];
-          val.x = fmaf(wa, a.x, val.x);
-          val.y = fmaf(wa, a.y, val.y);
-          val.z = fmaf(wa, a.z, val.z);
-          val.w = fmaf(wa, a.w, val.w);
-        }
-        orow[e] = val;
-      };
-#pragma unroll
-      for (int e = 0; e < 8; ++e) put(e, o + 4 * e);
-      if constexpr (DV == 192) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) put(8 + e, o2 + 4 * e);
-      }
       if (g == 0) *lse_dst = lse_w;
     }
     tc_fence_before();

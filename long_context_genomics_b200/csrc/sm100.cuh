@@ -69,10 +69,29 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   return ok != 0u;
 }
 
+// The same test, letting the hardware suspend the thread until the phase
+// completes or about hint_ns nanoseconds have passed, so that a waiting warp
+// does not take issue slots from the warps that compute.
+#ifndef AG_WAIT_HINT_NS
+#define AG_WAIT_HINT_NS 20000
+#endif
+__device__ __forceinline__ bool mbar_test_suspend(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "n"(AG_WAIT_HINT_NS)
+      : "memory");
+  return ok != 0u;
+}
+
 // Wait until the phase with the given parity has completed.  Bounded: gives
 // up after kWaitLimitNs, or as soon as another thread of the block has set
-// *abort.  On giving up it sets *abort, records `site` in the error word
-// (first writer wins) and returns false.
+// *abort (checked whenever the hardware returns from a suspended test, i.e.
+// at least every few tens of microseconds).  On giving up it sets *abort,
+// records `site` in the error word (first writer wins) and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
                                           volatile int *abort, unsigned *err,
                                           unsigned site,
@@ -81,7 +100,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
   if (mbar_test(a, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
+#if AG_WAIT_HINT_NS > 0
+    if (mbar_test_suspend(a, parity)) return true;
+#else
     if (mbar_test(a, parity)) return true;
+#endif
     if (*abort) return false;
     if (globaltimer_ns() - t0 > limit_ns) {
       *abort = 1;
@@ -464,6 +487,13 @@ __device__ __forceinline__ void griddep_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
+// bits(t) * 2^23 + bits(p) modulo 2^32, as one integer multiply-add.
+__device__ __forceinline__ int mad_shl23(float t, float p) {
+  int r;
+  asm("mad.lo.s32 %0, %1, 8388608, %2;" : "=r"(r) : "r"(__float_as_int(t)), "r"(__float_as_int(p)));
+  return r;
+}
+
 // 2^(a t - m) on the FMA pipe (two lanes at once), used to take part of the
 // exponentials off the special-function unit; m is an integer in [0, 2^21)
 // and a t - m must lie in [-126, 0].  Range reduction a t = j + f with
@@ -484,9 +514,7 @@ __device__ __forceinline__ float2 exp2_poly2_fma(float2 t, float2 a, float2 km) 
   float2 p = __ffma2_rn(make_float2(c3, c3), f, make_float2(c2, c2));
   p = __ffma2_rn(p, f, make_float2(c1, c1));
   p = __ffma2_rn(p, f, make_float2(c0, c0));
-  return make_float2(
-      __int_as_float(__float_as_int(p.x) + (__float_as_int(T.x) << 23)),
-      __int_as_float(__float_as_int(p.y) + (__float_as_int(T.y) << 23)));
+  return make_float2(__int_as_float(mad_shl23(T.x, p.x)), __int_as_float(mad_shl23(T.y, p.y)));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
