@@ -58,7 +58,7 @@ constexpr int kSubBytes = kSubRows * kD * 2;  // 16 KB (Q, dO hi or dO lo)
 constexpr int kSubHalf = kSubBytes / 2;       // 8 KB
 constexpr int kKStages = 3;                 // Q/dO ring of the key kernel
 constexpr int kSoftWarps = 16;
-constexpr int kThreads = 640;               // 16 softmax warps, producer, MMA, 2 idle
+constexpr int kThreads = 576;               // 16 softmax warps, producer, MMA
 constexpr int kWarpLoad = 16, kWarpMma = 17;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -171,13 +171,23 @@ __global__ void __launch_bounds__(256) bwd_split_kernel(const float *__restrict_
 // Query kernel.  Tile t = (item b, 16-position block I): rows h * 16 + il of
 // all 8 heads.  PASS 1: delta.  PASS 2: dq (needs delta).
 //
-// Tensor memory: S [0, 64), dP [64, 128), dS hi [128, 160), dS lo [160, 192),
-// dQ [256, 384).  Warpgroup g takes keys [16 g, 16 g + 16) of each 64-key
-// step; thread r of it owns row r.
+// The CTA's steps (64 keys of one of its tiles each) are numbered s = 0, 1,
+// ... across its tiles; step s uses K/V ring slot s % 3 and tensor-memory
+// buffer s % 3: S at columns [128 b, 128 b + 64), dP at [128 b + 64,
+// 128 b + 128).  Pass 2 writes dS (bf16 hi, lo) over the S columns it has
+// read, and dQ accumulates at [384, 512).  Warpgroup g takes keys
+// [16 g, 16 g + 16) of each step; thread r of it owns row r.  The tensor
+// core works up to two steps ahead of the softmax warps: S and dP of step
+// s + 2 are issued right after dQ of step s, into the buffer that dQ of
+// step s - 1 has finished reading.
+constexpr int kQBufs = kQStages;
 struct QBars {
   uint64_t q_full, q_empty;
   uint64_t kv_full[kQStages], kv_empty[kQStages];
-  uint64_t sp_full, sp_free, ds_full, ds_free, dq_full, xd, drain;
+  uint64_t sp_full[kQBufs];   // S and dP of the buffer's step are in tensor memory
+  uint64_t buf_free[kQBufs];  // the buffer's last step is done with it
+  uint64_t ds_full[kQBufs];   // pass 2: dS of the buffer's step is written
+  uint64_t dq_full, xd, drain;
   uint32_t tmem;
   int abort;
 };
@@ -202,6 +212,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int n_kt = (a.L + kQKeys - 1) / kQKeys;
   const int tiles = a.B * a.nb;
+  // This CTA's tiles are blockIdx.x, blockIdx.x + gridDim.x, ...
+  const int my_tiles =
+      static_cast<int>(blockIdx.x) < tiles
+          ? (tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                static_cast<int>(gridDim.x)
+          : 0;
+  const uint32_t total = static_cast<uint32_t>(my_tiles) * static_cast<uint32_t>(n_kt);
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -209,11 +226,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kQStages; ++s) {
       mbar_init(&bars->kv_full[s], 1);
       mbar_init(&bars->kv_empty[s], 1);
+      mbar_init(&bars->sp_full[s], 1);
+      // Pass 1: the softmax warps free a buffer once they have loaded it;
+      // pass 2: the tensor core, once dQ has read the dS written there.
+      mbar_init(&bars->buf_free[s], PASS == 1 ? kSoftWarps : 1);
+      mbar_init(&bars->ds_full[s], kSoftWarps);
     }
-    mbar_init(&bars->sp_full, 1);
-    mbar_init(&bars->sp_free, kSoftWarps);
-    mbar_init(&bars->ds_full, kSoftWarps);
-    mbar_init(&bars->ds_free, 1);
     mbar_init(&bars->dq_full, 1);
     mbar_init(&bars->xd, kSoftWarps);
     mbar_init(&bars->drain, 1);
@@ -271,59 +289,50 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane_id() == 0) {
       const uint32_t q_a = smem_u32(q_s), dh_a = smem_u32(dh_s), dl_a = smem_u32(dl_s);
       const uint32_t kv_a = smem_u32(kv_s);
-      const uint32_t tS = tmem, tP = tmem + 64, tDS = tmem + 128, tQ = tmem + 256;
-      uint32_t qc = 0, kl = 0, uses = 0, dsu = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-        ok = mbar_wait(&bars->q_full, qc & 1u, abort, a.err, kSiteQ);
-        ++qc;
-        if (!ok) break;
-        uint32_t prev_slot = 0;
-        for (int j = 0; j < n_kt; ++j, ++kl) {
-          const uint32_t s = kl % kQStages;
-          ok = mbar_wait(&bars->kv_full[s], (kl / kQStages) & 1u, abort, a.err, kSiteKV);
-          if (!ok) break;
-          if (uses > 0) {
-            ok = mbar_wait(&bars->sp_free, (uses - 1) & 1u, abort, a.err, kSiteSP);
-            if (!ok) break;
-          }
-          tc_fence_after();
-          const uint32_t ks = kv_a + s * 2 * kQKTileBytes, vs = ks + kQKTileBytes;
-          mma_kk(tS, q_a, kQHalf, ks, kQKHalf, kQKeys, false);         // S = Q K^T
-          mma_kk(tP, dh_a, kQHalf, vs, kQKHalf, kQKeys, false);        // dP = dO_hi V^T
-          mma_kk(tP, dl_a, kQHalf, vs, kQKHalf, kQKeys, true);         //    + dO_lo V^T
-          umma1_commit(&bars->sp_full);
-          ++uses;
-          if (j + 1 == n_kt) umma1_commit(&bars->q_empty);
-          if (PASS == 1) {
-            umma1_commit(&bars->kv_empty[s]);
-          } else if (j > 0) {
-            // dQ += dS(j-1) K(j-1), from hi and lo.
-            ok = mbar_wait(&bars->ds_full, dsu & 1u, abort, a.err, kSiteDS);
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t kp = kv_a + prev_slot * 2 * kQKTileBytes;
-            mma_tm(tQ, [&](int kk) { return tDS + 8 * kk; }, 4, kp, kQKHalf, j > 1);
-            mma_tm(tQ, [&](int kk) { return tDS + 32 + 8 * kk; }, 4, kp, kQKHalf, true);
-            umma1_commit(&bars->ds_free);
-            umma1_commit(&bars->kv_empty[prev_slot]);
-            ++dsu;
-          }
-          prev_slot = s;
+      const uint32_t tQ = tmem + 384;
+      const uint32_t nk = static_cast<uint32_t>(n_kt);
+      // S = Q K^T and dP = dO V^T (dO as hi + lo) of step s into buffer s % 3.
+      auto issue_sp = [&](uint32_t s) -> bool {
+        const uint32_t b = s % kQBufs, u = s / kQBufs, j = s % nk;
+        if (j == 0 && !mbar_wait(&bars->q_full, (s / nk) & 1u, abort, a.err, kSiteQ))
+          return false;
+        if (!mbar_wait(&bars->kv_full[b], u & 1u, abort, a.err, kSiteKV)) return false;
+        if (u > 0 && !mbar_wait(&bars->buf_free[b], (u - 1) & 1u, abort, a.err, kSiteSP))
+          return false;
+        tc_fence_after();
+        const uint32_t ks = kv_a + b * 2 * kQKTileBytes, vs = ks + kQKTileBytes;
+        const uint32_t tS = tmem + 128 * b, tP = tS + 64;
+        mma_kk(tS, q_a, kQHalf, ks, kQKHalf, kQKeys, false);   // S = Q K^T
+        mma_kk(tP, dh_a, kQHalf, vs, kQKHalf, kQKeys, false);  // dP = dO_hi V^T
+        mma_kk(tP, dl_a, kQHalf, vs, kQKHalf, kQKeys, true);   //    + dO_lo V^T
+        umma1_commit(&bars->sp_full[b]);
+        if (j + 1 == nk) umma1_commit(&bars->q_empty);
+        if (PASS == 1) umma1_commit(&bars->kv_empty[b]);
+        return true;
+      };
+      // dQ += dS K of step s, dS (hi, lo) over the S columns of its buffer.
+      auto issue_dq = [&](uint32_t s) -> bool {
+        const uint32_t b = s % kQBufs, u = s / kQBufs, j = s % nk;
+        if (!mbar_wait(&bars->ds_full[b], u & 1u, abort, a.err, kSiteDS)) return false;
+        tc_fence_after();
+        const uint32_t kp = kv_a + b * 2 * kQKTileBytes, tS = tmem + 128 * b;
+        mma_tm(tQ, [=](int kk) { return tS + 16 * kk; }, 4, kp, kQKHalf, j > 0);
+        mma_tm(tQ, [=](int kk) { return tS + 16 * kk + 8; }, 4, kp, kQKHalf, true);
+        umma1_commit(&bars->buf_free[b]);
+        umma1_commit(&bars->kv_empty[b]);
+        if (j + 1 == nk) umma1_commit(&bars->dq_full);
+        return true;
+      };
+      if (PASS == 1) {
+        for (uint32_t s = 0; s < total; ++s)
+          if (!issue_sp(s)) break;
+      } else {
+        bool ok = true;
+        for (uint32_t s = 0; s < 2 && s < total && ok; ++s) ok = issue_sp(s);
+        for (uint32_t s = 0; s < total && ok; ++s) {
+          ok = issue_dq(s);
+          if (ok && s + 2 < total) ok = issue_sp(s + 2);
         }
-        if (!ok) break;
-        if (PASS == 2) {
-          ok = mbar_wait(&bars->ds_full, dsu & 1u, abort, a.err, kSiteDS);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t kp = kv_a + prev_slot * 2 * kQKTileBytes;
-          mma_tm(tQ, [&](int kk) { return tDS + 8 * kk; }, 4, kp, kQKHalf, n_kt > 1);
-          mma_tm(tQ, [&](int kk) { return tDS + 32 + 8 * kk; }, 4, kp, kQKHalf, true);
-          umma1_commit(&bars->ds_free);
-          umma1_commit(&bars->kv_empty[prev_slot]);
-          ++dsu;
-        }
-        umma1_commit(&bars->dq_full);
       }
       umma1_commit(&bars->drain);
       drain(&bars->drain, 0);
@@ -332,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int g = threadIdx.x >> 7, r = threadIdx.x & 127;
     const int h = r >> 4, il = r & 15;
     const uint32_t lane_base = static_cast<uint32_t>(r >> 5) << 21;
-    uint32_t uses = 0, dsu = 0, qc = 0, xc = 0;
+    uint32_t s = 0, qc = 0, xc = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
       const int b = t / a.nb, I = t - b * a.nb;
@@ -344,21 +353,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float *brow = a.bias + static_cast<long long>(b) * a.bias_bstride +
                           (static_cast<size_t>(h) * a.P + I) * a.P;
       float acc = 0.f;
-      for (int j = 0; j < n_kt; ++j) {
+      for (int j = 0; j < n_kt; ++j, ++s) {
+        const uint32_t bf = s % kQBufs, u = s / kQBufs;
         const int key0 = kQKeys * j + 16 * g;  // this thread's 16 keys: one bias cell
         const float bj = key0 < a.L ? __ldg(brow + key0 / 16) : 0.f;
-        ok = mbar_wait(&bars->sp_full, uses & 1u, abort, a.err, kSiteSoft);
-        ++uses;
+        ok = mbar_wait(&bars->sp_full[bf], u & 1u, abort, a.err, kSiteSoft);
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
+        const uint32_t tS = tmem + 128 * bf + 16 * g + lane_base;
         uint32_t sv[16], pv[16];
-        tmem_ld16(tmem + 16 * g + lane_base, sv);
-        tmem_ld16(tmem + 64 + 16 * g + lane_base, pv);
+        tmem_ld16(tS, sv);
+        tmem_ld16(tS + 64, pv);
         tmem_wait_ld16(sv);
         tmem_wait_ld16(pv);
-        tc_fence_before();
-        warp_arrive(&bars->sp_free);
         if (PASS == 1) {
+          tc_fence_before();
+          warp_arrive(&bars->buf_free[bf]);
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const Logit lg = logit(__uint_as_float(sv[e]), bj, lse2, a);
@@ -370,33 +380,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 16; e += 2) {
             float ds2[2];
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const Logit lg = logit(__uint_as_float(sv[e + u]), bj, lse2, a);
-              const float ds = lg.p * (__uint_as_float(pv[e + u]) - del) * lg.dt;
-              ds2[u] = (key0 + e + u < a.L && row_ok) ? ds : 0.f;
+            for (int u2 = 0; u2 < 2; ++u2) {
+              const Logit lg = logit(__uint_as_float(sv[e + u2]), bj, lse2, a);
+              const float ds = lg.p * (__uint_as_float(pv[e + u2]) - del) * lg.dt;
+              ds2[u2] = (key0 + e + u2 < a.L && row_ok) ? ds : 0.f;
             }
             split2(ds2[0], ds2[1], hi[e / 2], lo[e / 2]);
           }
-          if (dsu > 0) {
-            ok = mbar_wait(&bars->ds_free, (dsu - 1) & 1u, abort, a.err, kSiteSoft);
-            if (!__all_sync(0xffffffffu, ok)) break;
-          }
-          ++dsu;
-          tc_fence_after();
-          tmem_st8(tmem + 128 + 8 * g + lane_base, hi);
-          tmem_st8(tmem + 160 + 8 * g + lane_base, lo);
+          // In place: this warp's lanes of the S columns it has just read.
+          tmem_st8(tS, hi);
+          tmem_st8(tS + 8, lo);
           tmem_wait_st();
           tc_fence_before();
-          warp_arrive(&bars->ds_full);
+          warp_arrive(&bars->ds_full[bf]);
         }
       }
       if (!ok) break;
-      // Tile epilogue: dq_full also tells that every S and dP of the tile
-      // has been read by the tensor core.
-      ok = mbar_wait(&bars->dq_full, qc & 1u, abort, a.err, kSiteEnd);
-      ++qc;
-      if (!__all_sync(0xffffffffu, ok)) break;
-      tc_fence_after();
       if (PASS == 1) {
         float *dp = dpart + (xc & 1u) * 512;
         dp[g * 128 + r] = acc;
@@ -406,9 +405,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!__all_sync(0xffffffffu, ok)) break;
         if (g == 0 && row_ok) a.delta[row] = dp[r] + dp[128 + r] + dp[256 + r] + dp[384 + r];
       } else {
-        // dq row: warpgroup g writes columns [32 g, 32 g + 32).
+        // dq row: warpgroup g writes columns [32 g, 32 g + 32).  dq_full also
+        // tells that every dS of the tile has been read.
+        ok = mbar_wait(&bars->dq_full, qc & 1u, abort, a.err, kSiteEnd);
+        ++qc;
+        if (!__all_sync(0xffffffffu, ok)) break;
+        tc_fence_after();
         uint32_t o[32];
-        tmem_ld32(tmem + 256 + 32 * g + lane_base, o);
+        tmem_ld32(tmem + 384 + 32 * g + lane_base, o);
         tmem_wait_ld(o);
         if (row_ok) {
           float4 *dst = reinterpret_cast<float4 *>(a.dq + row * kD + 32 * g);
@@ -419,8 +423,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                  __uint_as_float(o[4 * e + 2]) * sc,
                                  __uint_as_float(o[4 * e + 3]) * sc);
         }
+        tc_fence_before();
       }
-      tc_fence_before();
     }
   }
   __syncwarp();
@@ -438,14 +442,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 // item, each block as two 64-row steps (heads 0-3, then 4-7).  Per item:
 // K and V resident, a 3-stage ring of (Q, dO hi, dO lo) steps.
 //
-// Tensor memory (lane = key): S^T [0, 64), dP^T [64, 128), P^T hi [128,
-// 160), P^T lo [160, 192), dS^T hi [192, 224), dS^T lo [224, 256), dV [256,
-// 384), dK [384, 512).  Warpgroup g takes the step's rows [16 g, 16 g + 16):
-// head 4 (step & 1) + g, positions 0..15 of the block; thread r owns key r.
+// Tensor memory (lane = key): two step buffers b = s % 2 (s counts the
+// CTA's steps across items), S^T at [128 b, 128 b + 64) and dP^T at
+// [128 b + 64, 128 b + 128); the softmax warps write P^T (bf16 hi, lo) over
+// the S^T columns and dS^T (hi, lo) over the dP^T columns they have read.
+// dV [256, 384), dK [384, 512).  Warpgroup g takes the step's rows
+// [16 g, 16 g + 16): head 4 (step & 1) + g, positions 0..15 of the block;
+// thread r owns key r.  The tensor core issues, per step s: dK += dS^T Q
+// (then tells that the dS^T columns are read), dV += P^T dO (then the P^T
+// columns), and behind them dP^T and S^T of step s + 2 into the same
+// buffer, each after the wait for the columns it overwrites, so the waits
+// are covered by the products already queued.
 struct KBars {
   uint64_t kv_full, kv_free;
   uint64_t ring_full[kKStages], ring_empty[kKStages];
-  uint64_t sp_full, sp_free, pds_full, pds_free, acc_full, acc_free;
+  uint64_t sp_full[2];   // S^T and dP^T of the buffer's step are in tensor memory
+  uint64_t pds_full[2];  // P^T and dS^T of the buffer's step are written
+  uint64_t ds_read[2];   // dK has read the buffer's dS^T columns
+  uint64_t p_read[2];    // dV has read the buffer's P^T columns
+  uint64_t acc_full, acc_free;
   uint64_t peer;      // even CTA: the odd CTA's partial of the item is in dk/dv
   uint64_t peer_ack;  // odd CTA: the even CTA has read it
   uint64_t epi;       // every softmax warp of this CTA is through the item's dK, dV
@@ -512,10 +527,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(&bars->ring_full[s], 1);
       mbar_init(&bars->ring_empty[s], 1);
     }
-    mbar_init(&bars->sp_full, 1);
-    mbar_init(&bars->sp_free, kSoftWarps);
-    mbar_init(&bars->pds_full, kSoftWarps);
-    mbar_init(&bars->pds_free, 1);
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(&bars->sp_full[q], 1);
+      mbar_init(&bars->pds_full[q], kSoftWarps);
+      mbar_init(&bars->ds_read[q], 1);
+      mbar_init(&bars->p_read[q], 1);
+    }
     mbar_init(&bars->acc_full, 1);
     mbar_init(&bars->acc_free, kSoftWarps);
     mbar_init(&bars->peer, 1);
@@ -574,66 +591,71 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp == kWarpMma) {
     if (lane_id() == 0) {
       const uint32_t k_a = smem_u32(k_s), v_a = smem_u32(v_s), ring_a = smem_u32(ring);
-      const uint32_t tS = tmem, tP = tmem + 64, tV = tmem + 256, tK = tmem + 384;
-      uint32_t rc = 0, uses = 0, acc_count = 0;
-      bool ok = true, need_acc_free = false;
-      // dV += P^T dO, dK += dS^T Q for the step in ring stage st.
-      auto grads = [&](uint32_t st, bool first) -> bool {
-        if (need_acc_free) {
-          if (!mbar_wait(&bars->acc_free, (acc_count - 1) & 1u, abort, a.err, kSiteAcc))
-            return false;
-          need_acc_free = false;
-        }
-        tc_fence_after();
+      const uint32_t tV = tmem + 256, tK = tmem + 384;
+      const uint32_t ns = static_cast<uint32_t>(n_sub);
+      const uint32_t total = static_cast<uint32_t>(a.B) * ns;
+      // dP^T = V dO^T (dO as hi + lo) and S^T = K Q^T of step s into buffer
+      // s % 2, each once the products of step s - 2 have read the columns.
+      auto issue_sp = [&](uint32_t s) -> bool {
+        const uint32_t b = s & 1u, u = s >> 1, st = s % kKStages, n = s % ns, item = s / ns;
+        if (n == 0 && !mbar_wait(&bars->kv_full, item & 1u, abort, a.err, kSiteKV)) return false;
+        if (!mbar_wait(&bars->ring_full[st], (s / kKStages) & 1u, abort, a.err, kSiteRing))
+          return false;
         const uint32_t qs = ring_a + st * 3 * kSubBytes, dh = qs + kSubBytes, dl = dh + kSubBytes;
-        mma_tm(tV, [&](int kk) { return tmem + 128 + 8 * kk; }, 4, dh, kSubHalf, !first);
-        mma_tm(tV, [&](int kk) { return tmem + 128 + 8 * kk; }, 4, dl, kSubHalf, true);
-        mma_tm(tV, [&](int kk) { return tmem + 160 + 8 * kk; }, 4, dh, kSubHalf, true);
-        mma_tm(tK, [&](int kk) { return tmem + 192 + 8 * kk; }, 4, qs, kSubHalf, !first);
-        mma_tm(tK, [&](int kk) { return tmem + 224 + 8 * kk; }, 4, qs, kSubHalf, true);
-        umma1_commit(&bars->pds_free);
-        umma1_commit(&bars->ring_empty[st]);
+        const uint32_t tS = tmem + 128 * b, tP = tS + 64;
+        if (u > 0 && !mbar_wait(&bars->ds_read[b], (u - 1) & 1u, abort, a.err, kSiteSP))
+          return false;
+        tc_fence_after();
+        mma_kk(tP, v_a, kKHalf, dh, kSubHalf, kSubRows, false);  // dP^T = V dO_hi^T
+        mma_kk(tP, v_a, kKHalf, dl, kSubHalf, kSubRows, true);   //      + V dO_lo^T
+        if (u > 0 && !mbar_wait(&bars->p_read[b], (u - 1) & 1u, abort, a.err, kSiteSP))
+          return false;
+        tc_fence_after();
+        mma_kk(tS, k_a, kKHalf, qs, kSubHalf, kSubRows, false);  // S^T = K Q^T
+        umma1_commit(&bars->sp_full[b]);
+        if (n + 1 == ns) umma1_commit(&bars->kv_free);
         return true;
       };
-      for (int b = 0; b < a.B && ok; ++b) {
-        ok = mbar_wait(&bars->kv_full, static_cast<uint32_t>(b) & 1u, abort, a.err, kSiteKV);
-        if (!ok) break;
-        uint32_t prev = 0;
-        for (int n = 0; n < n_sub; ++n, ++rc) {
-          const uint32_t st = rc % kKStages;
-          ok = mbar_wait(&bars->ring_full[st], (rc / kKStages) & 1u, abort, a.err, kSiteRing);
-          if (!ok) break;
-          if (uses > 0) {
-            ok = mbar_wait(&bars->sp_free, (uses - 1) & 1u, abort, a.err, kSiteSP);
-            if (!ok) break;
-          }
-          tc_fence_after();
-          const uint32_t qs = ring_a + st * 3 * kSubBytes, dh = qs + kSubBytes, dl = dh + kSubBytes;
-          mma_kk(tS, k_a, kKHalf, qs, kSubHalf, kSubRows, false);   // S^T = K Q^T
-          mma_kk(tP, v_a, kKHalf, dh, kSubHalf, kSubRows, false);   // dP^T = V dO_hi^T
-          mma_kk(tP, v_a, kKHalf, dl, kSubHalf, kSubRows, true);    //      + V dO_lo^T
-          umma1_commit(&bars->sp_full);
-          if (n + 1 == n_sub) umma1_commit(&bars->kv_free);
-          ++uses;
-          if (n > 0) {
-            ok = mbar_wait(&bars->pds_full, (uses - 2) & 1u, abort, a.err, kSiteDS);
-            if (!ok || !grads(prev, n == 1)) {
-              ok = false;
-              break;
-            }
-          }
-          prev = st;
-        }
-        if (!ok) break;
-        if (n_sub > 0) {
-          ok = mbar_wait(&bars->pds_full, (uses - 1) & 1u, abort, a.err, kSiteDS);
-          if (!ok || !grads(prev, n_sub == 1)) break;
-        } else {
+      // dK += dS^T Q, dV += P^T dO (P^T and dS^T as hi + lo) of step s.
+      auto issue_g = [&](uint32_t s) -> bool {
+        const uint32_t b = s & 1u, u = s >> 1, st = s % kKStages, n = s % ns, item = s / ns;
+        if (!mbar_wait(&bars->pds_full[b], u & 1u, abort, a.err, kSiteDS)) return false;
+        if (n == 0 && item > 0 &&
+            !mbar_wait(&bars->acc_free, (item - 1) & 1u, abort, a.err, kSiteAcc))
+          return false;
+        tc_fence_after();
+        const uint32_t qs = ring_a + st * 3 * kSubBytes, dh = qs + kSubBytes, dl = dh + kSubBytes;
+        const uint32_t tS = tmem + 128 * b, tP = tS + 64;
+        const bool first = n == 0;
+        mma_tm(tK, [=](int kk) { return tP + 16 * kk; }, 4, qs, kSubHalf, !first);
+        mma_tm(tK, [=](int kk) { return tP + 16 * kk + 8; }, 4, qs, kSubHalf, true);
+        umma1_commit(&bars->ds_read[b]);
+        mma_tm(tV, [=](int kk) { return tS + 16 * kk; }, 4, dh, kSubHalf, !first);
+        mma_tm(tV, [=](int kk) { return tS + 16 * kk; }, 4, dl, kSubHalf, true);
+        mma_tm(tV, [=](int kk) { return tS + 16 * kk + 8; }, 4, dh, kSubHalf, true);
+        umma1_commit(&bars->p_read[b]);
+        umma1_commit(&bars->ring_empty[st]);
+        if (n + 1 == ns) umma1_commit(&bars->acc_full);
+        return true;
+      };
+      if (ns == 0) {
+        // No query blocks here: zero partials, but the same per-item handshakes.
+        for (int b = 0; b < a.B; ++b) {
+          if (!mbar_wait(&bars->kv_full, static_cast<uint32_t>(b) & 1u, abort, a.err, kSiteKV))
+            break;
           umma1_commit(&bars->kv_free);
+          if (b > 0 && !mbar_wait(&bars->acc_free, static_cast<uint32_t>(b - 1) & 1u, abort,
+                                  a.err, kSiteAcc))
+            break;
+          umma1_commit(&bars->acc_full);
         }
-        umma1_commit(&bars->acc_full);
-        ++acc_count;
-        need_acc_free = true;
+      } else {
+        bool ok = true;
+        for (uint32_t s = 0; s < 2 && s < total && ok; ++s) ok = issue_sp(s);
+        for (uint32_t s = 0; s < total && ok; ++s) {
+          ok = issue_g(s);
+          if (ok && s + 2 < total) ok = issue_sp(s + 2);
+        }
       }
       umma1_commit(&bars->drain);
       drain(&bars->drain, 0);
@@ -647,7 +669,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int wq = (r >> 5) & 3;  // this warp's 32 keys: key blocks 8 kt + 2 wq (+1)
     const uint32_t peer_even = cluster_addr(&bars->peer, 0);
     const uint32_t ack_odd = cluster_addr(&bars->peer_ack, 1);
-    uint32_t uses = 0, pdsu = 0, acc_count = 0;
+    uint32_t sc = 0, acc_count = 0;  // sc: the CTA's step counter
     bool ok = true;
     for (int b = 0; b < a.B && ok; ++b) {
       const float *bias_b = a.bias + static_cast<long long>(b) * a.bias_bstride;
@@ -659,17 +681,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int nrows = a.L - 16 * I < 16 ? a.L - 16 * I : 16;
         const float bj = key_ok ? __ldg(bias_b + (static_cast<size_t>(h) * a.P + I) * a.P + J)
                                 : 0.f;
-        ok = mbar_wait(&bars->sp_full, uses & 1u, abort, a.err, kSiteSoft);
-        ++uses;
+        const uint32_t bf = sc & 1u, u = sc >> 1;
+        ++sc;
+        ok = mbar_wait(&bars->sp_full[bf], u & 1u, abort, a.err, kSiteSoft);
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
+        const uint32_t tS = tmem + 128 * bf + 16 * g + lane_base, tP = tS + 64;
         uint32_t sv[16], pv[16];
-        tmem_ld16(tmem + 16 * g + lane_base, sv);
-        tmem_ld16(tmem + 64 + 16 * g + lane_base, pv);
+        tmem_ld16(tS, sv);
+        tmem_ld16(tP, pv);
         tmem_wait_ld16(sv);
         tmem_wait_ld16(pv);
-        tc_fence_before();
-        warp_arrive(&bars->sp_free);
         uint32_t ph[8], pl[8], sh[8], sl[8];
         float cell = 0.f;
 #pragma unroll
@@ -692,19 +714,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           split2(pp[0], pp[1], ph[e / 2], pl[e / 2]);
           split2(dd[0], dd[1], sh[e / 2], sl[e / 2]);
         }
-        if (pdsu > 0) {
-          ok = mbar_wait(&bars->pds_free, (pdsu - 1) & 1u, abort, a.err, kSiteSoft);
-          if (!__all_sync(0xffffffffu, ok)) break;
-        }
-        ++pdsu;
-        tc_fence_after();
-        tmem_st8(tmem + 128 + 8 * g + lane_base, ph);
-        tmem_st8(tmem + 160 + 8 * g + lane_base, pl);
-        tmem_st8(tmem + 192 + 8 * g + lane_base, sh);
-        tmem_st8(tmem + 224 + 8 * g + lane_base, sl);
+        // In place: this warp's lanes of the columns it has just read.
+        tmem_st8(tS, ph);
+        tmem_st8(tS + 8, pl);
+        tmem_st8(tP, sh);
+        tmem_st8(tP + 8, sl);
         tmem_wait_st();
         tc_fence_before();
-        warp_arrive(&bars->pds_full);
+        warp_arrive(&bars->pds_full[bf]);
         // dbias: sum the cell over its 16 keys (lanes 0-15, 16-31 of the warp).
 #pragma unroll
         for (int o = 8; o >= 1; o >>= 1) cell += __shfl_xor_sync(0xffffffffu, cell, o);

@@ -11,11 +11,11 @@
 // persistent CTA per SM streams chunks of 32 consecutive cells (16 KB) into a
 // 12-stage shared-memory ring with TMA (one producer lane; the pair tensor is
 // seen as [cells, 128] fp32 rows, four 32-channel boxes per chunk with the
-// 128-byte swizzle), so up to 192 KB per SM are in flight.  Each of six
-// consumer warps takes whole chunks (chunk n of the CTA goes to warp n % 6,
-// so warp w always uses ring slots w and w + 6 and waits for their phases in
-// order; a slot shared by warps would let a warp wait for a phase one ahead
-// of the slot's current one, which a parity wait cannot tell from the phase
+// 128-byte swizzle), so up to 192 KB per SM are in flight.  Each of twelve
+// consumer warps takes whole chunks (chunk n of the CTA goes to warp n % 12,
+// so warp w always uses ring slot w and waits for its phases in order; a
+// slot shared by warps would let a warp wait for a phase one ahead of the
+// slot's current one, which a parity wait cannot tell from the phase
 // before).  Lane l owns cell l of the chunk and sums
 // its 128 channels for all 8 heads in registers (packed fp32x2 products, two
 // heads per instruction).  The swizzle puts the 16-byte channel group g of
@@ -38,8 +38,18 @@ constexpr int kCellBytes = kCp * 4;                  // 512
 constexpr int kChunkCells = 32;                      // one cell per lane
 constexpr int kChunkBytes = kChunkCells * kCellBytes;  // 16 KB
 constexpr int kBoxBytes = kChunkCells * 128;         // 32 cells x 32 channels
-constexpr int kStages = 12;
-constexpr int kConsumerWarps = 6;
+#ifndef AG_PROJ_STAGES
+#define AG_PROJ_STAGES 12
+#endif
+#ifndef AG_PROJ_CTAS_PER_SM
+#define AG_PROJ_CTAS_PER_SM 1
+#endif
+#ifndef AG_PROJ_PROMO
+#define AG_PROJ_PROMO 2
+#endif
+constexpr int kStages = AG_PROJ_STAGES;
+constexpr int kConsumerWarps = AG_PROJ_STAGES;
+constexpr int kCtasPerSm = AG_PROJ_CTAS_PER_SM;
 static_assert(kStages % kConsumerWarps == 0, "each ring slot belongs to one consumer warp");
 constexpr int kThreads = (kConsumerWarps + 1) * 32;  // + producer warp
 constexpr int kWBytes = kCp * kH * 4;                // 4 KB
@@ -58,7 +68,7 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, u
       : "memory");
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
     pair_bias_project_kernel(const __grid_constant__ CUtensorMap tm_pair,
                              const float *__restrict__ W, float *__restrict__ bias,
                              long long n_cells, unsigned *err) {
@@ -110,7 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // Consumer warp `warp` takes the CTA's chunks it = warp, warp + 6, ...
+    // Consumer warp `warp` takes the CTA's chunks it = warp, warp + 12, ...
     const float4 *w4 = reinterpret_cast<const float4 *>(w_s);  // W[c][0..3], W[c][4..7]
     const uint32_t swz = static_cast<uint32_t>(lane & 7);
     for (uint32_t it = warp;; it += kConsumerWarps) {
@@ -182,11 +192,11 @@ cudaError_t launch_pair_bias_project(const float *pair, const float *W, float *b
   const cuuint32_t estr[2] = {1, 1};
   if (encode(&tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(pair), dims, strides,
              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             AG_PROJ_PROMO == 2 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B : AG_PROJ_PROMO == 1 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B : CU_TENSOR_MAP_L2_PROMOTION_NONE,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   const long long n_chunks = (n_cells + kChunkCells - 1) / kChunkCells;
-  const long long grid = n_chunks < num_sms ? n_chunks : num_sms;
+  const long long grid = n_chunks < kCtasPerSm * num_sms ? n_chunks : kCtasPerSm * num_sms;
   pair_bias_project_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, stream>>>(
       tm, W, bias, n_cells, err);
   return cudaGetLastError();
