@@ -58,8 +58,8 @@ constexpr int kSubBytes = kSubRows * kD * 2;  // 16 KB (Q, dO hi or dO lo)
 constexpr int kSubHalf = kSubBytes / 2;       // 8 KB
 constexpr int kKStages = 3;                 // Q/dO ring of the key kernel
 constexpr int kSoftWarps = 16;
-constexpr int kThreads = 576;               // 16 softmax warps, producer, MMA
-constexpr int kWarpLoad = 16, kWarpMma = 17;
+constexpr int kThreads = 608;               // 16 softmax warps, producer, 2 MMA issuers
+constexpr int kWarpLoad = 16, kWarpMma = 17, kWarpMma2 = 18;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -150,6 +150,146 @@ __device__ __forceinline__ Logit logit(float s, float bias, float lse2, const Ar
   return {ex2_approx(fmaf(y, kLog2e, -lse2)), 1.f};
 }
 
+// The same split by truncation, on the integer and FMA pipes only: hi keeps
+// the upper 16 bits of each value, lo the upper 16 bits of the exact
+// remainder, so hi + lo is within 2^-14 of the value (relative).  Element a
+// goes to the low half of each packed pair.
+__device__ __forceinline__ void split2t(float a, float b, uint32_t &hi, uint32_t &lo) {
+  const uint32_t ua = __float_as_uint(a), ub = __float_as_uint(b);
+  const float ra = a - __uint_as_float(ua & 0xffff0000u);
+  const float rb = b - __uint_as_float(ub & 0xffff0000u);
+  hi = __byte_perm(ua, ub, 0x7632);
+  lo = __byte_perm(__float_as_uint(ra), __float_as_uint(rb), 0x7632);
+}
+
+// 2^x for two values on the FMA pipe (exp2_poly2_fma with a = 1, m = 0),
+// x clamped below at -126 so that the result stays a normal number (the
+// clamp moves only values under 2^-126, which no gradient here can see).
+__device__ __forceinline__ float2 exp2_fma_pair(float x0, float x1) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  return exp2_poly2_fma(make_float2(fmaxf(x0, -126.f), fmaxf(x1, -126.f)),
+                        make_float2(1.f, 1.f), make_float2(kShift, kShift));
+}
+
+// Probabilities of two logits (raw products s0, s1; lse in log2 units l0,
+// l1), with the exponential on the FMA pipe (kEmu) or the special-function
+// unit; dt = 1 - t^2 (1 without a cap).
+template <bool kCapped, bool kEmu>
+__device__ __forceinline__ float2 prob_pair(float s0, float s1, float bias_term, float l0,
+                                            float l1, const Args &a, float2 &dt) {
+  const float y0 = fmaf(s0, a.qk_scale, bias_term), y1 = fmaf(s1, a.qk_scale, bias_term);
+  float x0, x1;
+  if (kCapped) {
+    const float t0 = tanh_approx(y0), t1 = tanh_approx(y1);
+    dt = make_float2(fmaf(-t0, t0, 1.f), fmaf(-t1, t1, 1.f));
+    x0 = fmaf(a.A, t0, -l0);
+    x1 = fmaf(a.A, t1, -l1);
+  } else {
+    dt = make_float2(1.f, 1.f);
+    x0 = fmaf(y0, kLog2e, -l0);
+    x1 = fmaf(y1, kLog2e, -l1);
+  }
+  if (kEmu) return exp2_fma_pair(x0, x1);
+  return make_float2(ex2_approx(x0), ex2_approx(x1));
+}
+
+// Exponential pairs (out of the 8 of a 16-logit step) on the FMA pipe, per
+// kernel: the delta pass is bound by the special-function unit, the others
+// by instruction issue.
+#ifndef AG_BWD_EMU_DELTA
+#define AG_BWD_EMU_DELTA 3
+#endif
+#ifndef AG_BWD_EMU_DQ
+#define AG_BWD_EMU_DQ 0
+#endif
+#ifndef AG_BWD_EMU_KEY
+#define AG_BWD_EMU_KEY 0
+#endif
+
+template <bool kCapped, int kEmu>
+__device__ __forceinline__ float2 prob_sel(int pair, float s0, float s1, float bias_term,
+                                           float l0, float l1, const Args &a, float2 &dt) {
+  if (pair < kEmu) return prob_pair<kCapped, true>(s0, s1, bias_term, l0, l1, a, dt);
+  return prob_pair<kCapped, false>(s0, s1, bias_term, l0, l1, a, dt);
+}
+
+// Query kernel, pass 1: sum over this thread's 16 keys of p dp for its row
+// (keys from nvalid on are past L when kMask).
+template <bool kCapped, bool kMask>
+__device__ __forceinline__ float delta_part(const uint32_t (&sv)[16], const uint32_t (&pv)[16],
+                                            float bias_term, float lse2, int nvalid,
+                                            const Args &a) {
+  float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+  for (int e = 0; e < 16; e += 2) {
+    float2 dt;
+    float2 p = prob_sel<kCapped, AG_BWD_EMU_DELTA>(e >> 1, __uint_as_float(sv[e]),
+                                                   __uint_as_float(sv[e + 1]), bias_term, lse2,
+                                                   lse2, a, dt);
+    if (kMask) {
+      p.x = e < nvalid ? p.x : 0.f;
+      p.y = e + 1 < nvalid ? p.y : 0.f;
+    }
+    acc0 = fmaf(p.x, __uint_as_float(pv[e]), acc0);
+    acc1 = fmaf(p.y, __uint_as_float(pv[e + 1]), acc1);
+  }
+  return acc0 + acc1;
+}
+
+// Query kernel, pass 2: ds = p (dp - delta) dt for this thread's row and 16
+// keys, split into bf16 hi and lo pairs.
+template <bool kCapped, bool kMask>
+__device__ __forceinline__ void ds_row(const uint32_t (&sv)[16], const uint32_t (&pv)[16],
+                                       float bias_term, float lse2, float del, int nvalid,
+                                       const Args &a, uint32_t (&hi)[8], uint32_t (&lo)[8]) {
+#pragma unroll
+  for (int e = 0; e < 16; e += 2) {
+    float2 dt;
+    const float2 p = prob_sel<kCapped, AG_BWD_EMU_DQ>(e >> 1, __uint_as_float(sv[e]),
+                                                      __uint_as_float(sv[e + 1]), bias_term,
+                                                      lse2, lse2, a, dt);
+    float d0 = p.x * (__uint_as_float(pv[e]) - del) * dt.x;
+    float d1 = p.y * (__uint_as_float(pv[e + 1]) - del) * dt.y;
+    if (kMask) {
+      d0 = e < nvalid ? d0 : 0.f;
+      d1 = e + 1 < nvalid ? d1 : 0.f;
+    }
+    split2t(d0, d1, hi[e >> 1], lo[e >> 1]);
+  }
+}
+
+// Key kernel: P and dS of this thread's key for 16 rows (lse2 of row e at
+// lr[e], delta at dr[e]: shared memory, the same for every lane), split into
+// bf16 hi and lo pairs; returns the sum of ds.
+template <bool kCapped>
+__device__ __forceinline__ float key_rows(const uint32_t (&sv)[16], const uint32_t (&pv)[16],
+                                          const float *lr, const float *dr, float bias_term,
+                                          const Args &a, uint32_t (&ph)[8], uint32_t (&pl)[8],
+                                          uint32_t (&sh)[8], uint32_t (&sl)[8]) {
+  const float4 *l4p = reinterpret_cast<const float4 *>(lr);
+  const float4 *d4p = reinterpret_cast<const float4 *>(dr);
+  float cell = 0.f;
+#pragma unroll
+  for (int e4 = 0; e4 < 4; ++e4) {
+    const float4 l4 = l4p[e4], d4 = d4p[e4];
+    const float la[4] = {l4.x, l4.y, l4.z, l4.w}, da[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      const int e = 4 * e4 + 2 * h2;
+      float2 dt;
+      const float2 p = prob_sel<kCapped, AG_BWD_EMU_KEY>(
+          e >> 1, __uint_as_float(sv[e]), __uint_as_float(sv[e + 1]), bias_term, la[2 * h2],
+          la[2 * h2 + 1], a, dt);
+      const float d0 = p.x * (__uint_as_float(pv[e]) - da[2 * h2]) * dt.x;
+      const float d1 = p.y * (__uint_as_float(pv[e + 1]) - da[2 * h2 + 1]) * dt.y;
+      cell += d0 + d1;
+      split2t(p.x, p.y, ph[e >> 1], pl[e >> 1]);
+      split2t(d0, d1, sh[e >> 1], sl[e >> 1]);
+    }
+  }
+  return cell;
+}
+
 // ---------------------------------------------------------------------------
 // dout -> hi, lo planes.  Row r of [B H L] rows (128 values) becomes 256
 // bf16 at bytes [512 r, 512 r + 512) of dq: hi first, then lo.
@@ -172,22 +312,33 @@ __global__ void __launch_bounds__(256) bwd_split_kernel(const float *__restrict_
 // all 8 heads.  PASS 1: delta.  PASS 2: dq (needs delta).
 //
 // The CTA's steps (64 keys of one of its tiles each) are numbered s = 0, 1,
-// ... across its tiles; step s uses K/V ring slot s % 3 and tensor-memory
-// buffer s % 3: S at columns [128 b, 128 b + 64), dP at [128 b + 64,
-// 128 b + 128).  Pass 2 writes dS (bf16 hi, lo) over the S columns it has
-// read, and dQ accumulates at [384, 512).  Warpgroup g takes keys
-// [16 g, 16 g + 16) of each step; thread r of it owns row r.  The tensor
-// core works up to two steps ahead of the softmax warps: S and dP of step
-// s + 2 are issued right after dQ of step s, into the buffer that dQ of
-// step s - 1 has finished reading.
-constexpr int kQBufs = kQStages;
+// ... across its tiles.  K and V come in separate 3-slot rings (slot s % 3):
+// V is free as soon as dP has been formed, K only after dQ.  Tensor memory
+// holds two step buffers b = s % 2, S at columns [128 b, 128 b + 64) and dP
+// at [128 b + 64, 128 b + 128); pass 2 writes dS (bf16 hi, lo) over the S
+// columns it has read, and dQ accumulates at [256, 384).
+//
+// The softmax warps form two groups of two warpgroups: group q takes the
+// steps of buffer q (s % 2 == q), so one group's waits for its logits and
+// for tensor-memory traffic are covered by the other group's arithmetic.
+// Warpgroup hg of a group takes keys [32 hg, 32 hg + 32) of the step (two
+// 16-key blocks, one bias cell each); thread r of it owns row r.
+//
+// The tensor core runs ahead of the softmax warps: pass 1 issues S and dP of
+// a step as soon as its buffer has been loaded by the softmax group; pass 2
+// issues, per step s, dQ of step s, then dP of step s + 2 (its columns were
+// read before dS of step s was written), then S of step s + 2 once dQ of
+// step s has read the columns -- a wait covered by the dP products queued.
+constexpr int kQBufs = 2;
+constexpr int kGroupWarps = kSoftWarps / 2;
 struct QBars {
   uint64_t q_full, q_empty;
-  uint64_t kv_full[kQStages], kv_empty[kQStages];
+  uint64_t k_full[kQStages], k_empty[kQStages], v_full[kQStages], v_empty[kQStages];
   uint64_t sp_full[kQBufs];   // S and dP of the buffer's step are in tensor memory
-  uint64_t buf_free[kQBufs];  // the buffer's last step is done with it
+  uint64_t buf_free[kQBufs];  // the buffer's S columns may be overwritten
   uint64_t ds_full[kQBufs];   // pass 2: dS of the buffer's step is written
-  uint64_t dq_full, xd, drain;
+  uint64_t dq_full, dq_free, xd;
+  uint64_t drain[2];  // per issuing thread: its last products have completed
   uint32_t tmem;
   int abort;
 };
@@ -203,8 +354,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *q_s = smem_raw + pad;                 // Q tile (32 KB)
   uint8_t *dh_s = q_s + kQTileBytes;             // dO hi tile
   uint8_t *dl_s = dh_s + kQTileBytes;            // dO lo tile
-  uint8_t *kv_s = dl_s + kQTileBytes;            // ring: K then V, 32 KB a slot
-  QBars *bars = reinterpret_cast<QBars *>(kv_s + kQStages * 2 * kQKTileBytes);
+  uint8_t *k_ring = dl_s + kQTileBytes;          // K ring, 16 KB a slot
+  uint8_t *v_ring = k_ring + kQStages * kQKTileBytes;  // V ring
+  QBars *bars = reinterpret_cast<QBars *>(v_ring + kQStages * kQKTileBytes);
   // Row-sum exchange between the warpgroups, double-buffered by tile parity:
   // a thread writes one tile's half only after every thread has passed the
   // previous tile's exchange, i.e. has read the half before.
@@ -221,20 +373,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t total = static_cast<uint32_t>(my_tiles) * static_cast<uint32_t>(n_kt);
 
   if (threadIdx.x == 0) {
+    // Both issuing threads read the Q/dO tile and write a step's S and dP.
     mbar_init(&bars->q_full, 1);
-    mbar_init(&bars->q_empty, 1);
+    mbar_init(&bars->q_empty, 2);
     for (int s = 0; s < kQStages; ++s) {
-      mbar_init(&bars->kv_full[s], 1);
-      mbar_init(&bars->kv_empty[s], 1);
-      mbar_init(&bars->sp_full[s], 1);
-      // Pass 1: the softmax warps free a buffer once they have loaded it;
-      // pass 2: the tensor core, once dQ has read the dS written there.
-      mbar_init(&bars->buf_free[s], PASS == 1 ? kSoftWarps : 1);
-      mbar_init(&bars->ds_full[s], kSoftWarps);
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
+    }
+    for (int b = 0; b < kQBufs; ++b) {
+      mbar_init(&bars->sp_full[b], 2);
+      // Pass 1: the buffer's group frees it once it has loaded it; pass 2:
+      // issuer 1, once dQ has read the dS written there.
+      mbar_init(&bars->buf_free[b], PASS == 1 ? kGroupWarps : 1);
+      mbar_init(&bars->ds_full[b], kGroupWarps);
     }
     mbar_init(&bars->dq_full, 1);
+    mbar_init(&bars->dq_free, kSoftWarps);
     mbar_init(&bars->xd, kSoftWarps);
-    mbar_init(&bars->drain, 1);
+    mbar_init(&bars->drain[0], 1);
+    mbar_init(&bars->drain[1], 1);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -268,62 +427,92 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ++qc;
         for (int j = 0; j < n_kt && ok; ++j, ++kl) {
-          const uint32_t s = kl % kQStages;
-          ok = mbar_wait(&bars->kv_empty[s], ((kl / kQStages) & 1u) ^ 1u, abort, a.err, kSiteKV);
+          const uint32_t s = kl % kQStages, ph = ((kl / kQStages) & 1u) ^ 1u;
+          // V first: its slot is freed earlier than K's.
+          ok = mbar_wait(&bars->v_empty[s], ph, abort, a.err, kSiteKV);
           if (!ok) break;
-          mbar_arrive_expect_tx(&bars->kv_full[s], 2 * kQKTileBytes);
-          uint8_t *ks = kv_s + s * 2 * kQKTileBytes;
-          for (int hf = 0; hf < 2; ++hf) {
-            tma_load_3d(ks + hf * kQKHalf, &tm_k, &bars->kv_full[s], 64 * hf, kQKeys * j, b,
+          mbar_arrive_expect_tx(&bars->v_full[s], kQKTileBytes);
+          uint8_t *vs = v_ring + s * kQKTileBytes;
+          for (int hf = 0; hf < 2; ++hf)
+            tma_load_3d(vs + hf * kQKHalf, &tm_v, &bars->v_full[s], 64 * hf, kQKeys * j, b,
                         pol_k);
-            tma_load_3d(ks + kQKTileBytes + hf * kQKHalf, &tm_v, &bars->kv_full[s], 64 * hf,
-                        kQKeys * j, b, pol_k);
-          }
+          ok = mbar_wait(&bars->k_empty[s], ph, abort, a.err, kSiteKV);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&bars->k_full[s], kQKTileBytes);
+          uint8_t *ks = k_ring + s * kQKTileBytes;
+          for (int hf = 0; hf < 2; ++hf)
+            tma_load_3d(ks + hf * kQKHalf, &tm_k, &bars->k_full[s], 64 * hf, kQKeys * j, b,
+                        pol_k);
         }
       }
       if (qc > 0) drain(&bars->q_full, (qc - 1) & 1u);
-      for (uint32_t i = kl > kQStages ? kl - kQStages : 0; i < kl; ++i)
-        drain(&bars->kv_full[i % kQStages], (i / kQStages) & 1u);
+      for (uint32_t i = kl > kQStages ? kl - kQStages : 0; i < kl; ++i) {
+        drain(&bars->v_full[i % kQStages], (i / kQStages) & 1u);
+        drain(&bars->k_full[i % kQStages], (i / kQStages) & 1u);
+      }
     }
-  } else if (warp == kWarpMma) {
+  } else if (warp == kWarpMma || warp == kWarpMma2) {
+    // Two issuing threads: issuer 0 forms dP, issuer 1 forms S and (pass 2)
+    // dQ from the dS written over S, so the dQ accumulator is fed by one
+    // thread in a fixed order.
     if (lane_id() == 0) {
+      const int who = warp - kWarpMma;
       const uint32_t q_a = smem_u32(q_s), dh_a = smem_u32(dh_s), dl_a = smem_u32(dl_s);
-      const uint32_t kv_a = smem_u32(kv_s);
-      const uint32_t tQ = tmem + 384;
+      const uint32_t k_a = smem_u32(k_ring), v_a = smem_u32(v_ring);
+      const uint32_t tQ = tmem + 256;
       const uint32_t nk = static_cast<uint32_t>(n_kt);
-      // S = Q K^T and dP = dO V^T (dO as hi + lo) of step s into buffer s % 3.
+      // Issuer 0: dP = dO V^T (dO as hi + lo) of step s into buffer s % 2,
+      // once the softmax warps have read the dP of the buffer's previous
+      // step.  Issuer 1: S = Q K^T, once the buffer's previous S (pass 1) or
+      // the dS over it (pass 2, read by dQ) is no longer needed.
       auto issue_sp = [&](uint32_t s) -> bool {
-        const uint32_t b = s % kQBufs, u = s / kQBufs, j = s % nk;
+        const uint32_t b = s % kQBufs, u = s / kQBufs, st = s % kQStages, j = s % nk;
+        const uint32_t rph = (s / kQStages) & 1u;
         if (j == 0 && !mbar_wait(&bars->q_full, (s / nk) & 1u, abort, a.err, kSiteQ))
           return false;
-        if (!mbar_wait(&bars->kv_full[b], u & 1u, abort, a.err, kSiteKV)) return false;
-        if (u > 0 && !mbar_wait(&bars->buf_free[b], (u - 1) & 1u, abort, a.err, kSiteSP))
-          return false;
-        tc_fence_after();
-        const uint32_t ks = kv_a + b * 2 * kQKTileBytes, vs = ks + kQKTileBytes;
-        const uint32_t tS = tmem + 128 * b, tP = tS + 64;
-        mma_kk(tS, q_a, kQHalf, ks, kQKHalf, kQKeys, false);   // S = Q K^T
-        mma_kk(tP, dh_a, kQHalf, vs, kQKHalf, kQKeys, false);  // dP = dO_hi V^T
-        mma_kk(tP, dl_a, kQHalf, vs, kQKHalf, kQKeys, true);   //    + dO_lo V^T
+        if (u > 0) {
+          uint64_t *prev = (PASS == 1 || who == 1) ? &bars->buf_free[b] : &bars->ds_full[b];
+          if (!mbar_wait(prev, (u - 1) & 1u, abort, a.err, kSiteSP)) return false;
+        }
+        if (who == 0) {
+          if (!mbar_wait(&bars->v_full[st], rph, abort, a.err, kSiteKV)) return false;
+          tc_fence_after();
+          const uint32_t vs = v_a + st * kQKTileBytes, tP = tmem + 128 * b + 64;
+          mma_kk(tP, dh_a, kQHalf, vs, kQKHalf, kQKeys, false);  // dP = dO_hi V^T
+          mma_kk(tP, dl_a, kQHalf, vs, kQKHalf, kQKeys, true);   //    + dO_lo V^T
+          umma1_commit(&bars->v_empty[st]);
+        } else {
+          if (!mbar_wait(&bars->k_full[st], rph, abort, a.err, kSiteKV)) return false;
+          tc_fence_after();
+          const uint32_t ks = k_a + st * kQKTileBytes, tS = tmem + 128 * b;
+          mma_kk(tS, q_a, kQHalf, ks, kQKHalf, kQKeys, false);   // S = Q K^T
+          if (PASS == 1) umma1_commit(&bars->k_empty[st]);
+        }
         umma1_commit(&bars->sp_full[b]);
         if (j + 1 == nk) umma1_commit(&bars->q_empty);
-        if (PASS == 1) umma1_commit(&bars->kv_empty[b]);
         return true;
       };
-      // dQ += dS K of step s, dS (hi, lo) over the S columns of its buffer.
+      // Issuer 1, pass 2: dQ += dS K of step s, dS (hi, lo) over the S
+      // columns of its buffer.
       auto issue_dq = [&](uint32_t s) -> bool {
-        const uint32_t b = s % kQBufs, u = s / kQBufs, j = s % nk;
+        const uint32_t b = s % kQBufs, u = s / kQBufs, st = s % kQStages, j = s % nk;
         if (!mbar_wait(&bars->ds_full[b], u & 1u, abort, a.err, kSiteDS)) return false;
+        // The tile's first dQ overwrites the accumulator: every softmax warp
+        // must have read the previous tile's.
+        const uint32_t tile = s / nk;
+        if (j == 0 && tile > 0 &&
+            !mbar_wait(&bars->dq_free, (tile - 1) & 1u, abort, a.err, kSiteEnd))
+          return false;
         tc_fence_after();
-        const uint32_t kp = kv_a + b * 2 * kQKTileBytes, tS = tmem + 128 * b;
+        const uint32_t kp = k_a + st * kQKTileBytes, tS = tmem + 128 * b;
         mma_tm(tQ, [=](int kk) { return tS + 16 * kk; }, 4, kp, kQKHalf, j > 0);
         mma_tm(tQ, [=](int kk) { return tS + 16 * kk + 8; }, 4, kp, kQKHalf, true);
         umma1_commit(&bars->buf_free[b]);
-        umma1_commit(&bars->kv_empty[b]);
+        umma1_commit(&bars->k_empty[st]);
         if (j + 1 == nk) umma1_commit(&bars->dq_full);
         return true;
       };
-      if (PASS == 1) {
+      if (PASS == 1 || who == 0) {
         for (uint32_t s = 0; s < total; ++s)
           if (!issue_sp(s)) break;
       } else {
@@ -334,65 +523,93 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ok && s + 2 < total) ok = issue_sp(s + 2);
         }
       }
-      umma1_commit(&bars->drain);
-      drain(&bars->drain, 0);
+      umma1_commit(&bars->drain[who]);
+      drain(&bars->drain[who], 0);
     }
   } else if (warp < kSoftWarps) {
     const int g = threadIdx.x >> 7, r = threadIdx.x & 127;
+    const int q = g >> 1, hg = g & 1;  // group (buffer), key half
     const int h = r >> 4, il = r & 15;
     const uint32_t lane_base = static_cast<uint32_t>(r >> 5) << 21;
-    uint32_t s = 0, qc = 0, xc = 0;
+    uint32_t qc = 0, xc = 0;
+    uint32_t s0 = 0;  // the CTA's step number of the tile's first step
     bool ok = true;
-    for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+    for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, s0 += static_cast<uint32_t>(n_kt)) {
       const int b = t / a.nb, I = t - b * a.nb;
       const int pos = 16 * I + il;
       const bool row_ok = pos < a.L;
       const size_t row = (static_cast<size_t>(b) * kH + h) * a.L + (row_ok ? pos : 0);
-      const float lse2 = row_ok ? a.lse[row] * kLog2e : 0.f;
+      // A row past L gets lse = +inf: its probabilities are 0 (its dO row,
+      // zero-filled, makes its ds 0 too).
+      const float lse2 = row_ok ? a.lse[row] * kLog2e : __int_as_float(0x7f800000);
       const float del = (PASS == 2 && row_ok) ? a.delta[row] : 0.f;
       const float *brow = a.bias + static_cast<long long>(b) * a.bias_bstride +
                           (static_cast<size_t>(h) * a.P + I) * a.P;
       float acc = 0.f;
-      for (int j = 0; j < n_kt; ++j, ++s) {
-        const uint32_t bf = s % kQBufs, u = s / kQBufs;
-        const int key0 = kQKeys * j + 16 * g;  // this thread's 16 keys: one bias cell
-        const float bj = key0 < a.L ? __ldg(brow + key0 / 16) : 0.f;
-        ok = mbar_wait(&bars->sp_full[bf], u & 1u, abort, a.err, kSiteSoft);
+      // This group's steps of the tile: j with (s0 + j) % 2 == q.
+      for (int j = static_cast<int>((static_cast<uint32_t>(q) - s0) & 1u); j < n_kt; j += 2) {
+        const uint32_t s = s0 + static_cast<uint32_t>(j), u = s / kQBufs;
+        const int key0 = kQKeys * j + 32 * hg;  // this thread's 32 keys: two bias cells
+        float bt[2];
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+          bt[k] = (key0 + 16 * k < a.L ? __ldg(brow + key0 / 16 + k) : 0.f) * a.bias_mul;
+        ok = mbar_wait(&bars->sp_full[q], u & 1u, abort, a.err, kSiteSoft);
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
-        const uint32_t tS = tmem + 128 * bf + 16 * g + lane_base;
-        uint32_t sv[16], pv[16];
-        tmem_ld16(tS, sv);
-        tmem_ld16(tS + 64, pv);
-        tmem_wait_ld16(sv);
-        tmem_wait_ld16(pv);
+        const uint32_t tS = tmem + 128 * q + 32 * hg + lane_base;
         if (PASS == 1) {
-          tc_fence_before();
-          warp_arrive(&bars->buf_free[bf]);
+          uint32_t sv[2][16], pv[2][16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const Logit lg = logit(__uint_as_float(sv[e]), bj, lse2, a);
-            if (key0 + e < a.L) acc = fmaf(lg.p, __uint_as_float(pv[e]), acc);
+          for (int k = 0; k < 2; ++k) {
+            tmem_ld16(tS + 16 * k, sv[k]);
+            tmem_ld16(tS + 64 + 16 * k, pv[k]);
+          }
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            tmem_wait_ld16(sv[k]);
+            tmem_wait_ld16(pv[k]);
+          }
+          tc_fence_before();
+          warp_arrive(&bars->buf_free[q]);
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const int nvalid = a.L - (key0 + 16 * k);  // keys of the 16 before L
+            if (nvalid >= 16)
+              acc += a.capped ? delta_part<true, false>(sv[k], pv[k], bt[k], lse2, nvalid, a)
+                              : delta_part<false, false>(sv[k], pv[k], bt[k], lse2, nvalid, a);
+            else
+              acc += a.capped ? delta_part<true, true>(sv[k], pv[k], bt[k], lse2, nvalid, a)
+                              : delta_part<false, true>(sv[k], pv[k], bt[k], lse2, nvalid, a);
           }
         } else {
-          uint32_t hi[8], lo[8];
-#pragma unroll
-          for (int e = 0; e < 16; e += 2) {
-            float ds2[2];
-#pragma unroll
-            for (int u2 = 0; u2 < 2; ++u2) {
-              const Logit lg = logit(__uint_as_float(sv[e + u2]), bj, lse2, a);
-              const float ds = lg.p * (__uint_as_float(pv[e + u2]) - del) * lg.dt;
-              ds2[u2] = (key0 + e + u2 < a.L && row_ok) ? ds : 0.f;
+#pragma unroll 1
+          for (int k = 0; k < 2; ++k) {
+            const int nvalid = a.L - (key0 + 16 * k);
+            const float bterm = k ? bt[1] : bt[0];
+            uint32_t sv[16], pv[16], hi[8], lo[8];
+            tmem_ld16(tS + 16 * k, sv);
+            tmem_ld16(tS + 64 + 16 * k, pv);
+            tmem_wait_ld16(sv);
+            tmem_wait_ld16(pv);
+            if (nvalid >= 16) {
+              if (a.capped)
+                ds_row<true, false>(sv, pv, bterm, lse2, del, nvalid, a, hi, lo);
+              else
+                ds_row<false, false>(sv, pv, bterm, lse2, del, nvalid, a, hi, lo);
+            } else {
+              if (a.capped)
+                ds_row<true, true>(sv, pv, bterm, lse2, del, nvalid, a, hi, lo);
+              else
+                ds_row<false, true>(sv, pv, bterm, lse2, del, nvalid, a, hi, lo);
             }
-            split2(ds2[0], ds2[1], hi[e / 2], lo[e / 2]);
+            // In place: this warp's lanes of the S columns it has just read.
+            tmem_st8(tS + 16 * k, hi);
+            tmem_st8(tS + 16 * k + 8, lo);
           }
-          // In place: this warp's lanes of the S columns it has just read.
-          tmem_st8(tS, hi);
-          tmem_st8(tS + 8, lo);
           tmem_wait_st();
           tc_fence_before();
-          warp_arrive(&bars->ds_full[bf]);
+          warp_arrive(&bars->ds_full[q]);
         }
       }
       if (!ok) break;
@@ -412,7 +629,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
         uint32_t o[32];
-        tmem_ld32(tmem + 384 + 32 * g + lane_base, o);
+        tmem_ld32((tmem + 256) + 32 * g + lane_base, o);
         tmem_wait_ld(o);
         if (row_ok) {
           float4 *dst = reinterpret_cast<float4 *>(a.dq + row * kD + 32 * g);
@@ -424,6 +641,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                  __uint_as_float(o[4 * e + 3]) * sc);
         }
         tc_fence_before();
+        warp_arrive(&bars->dq_free);
       }
     }
   }
@@ -464,10 +682,12 @@ struct KBars {
   uint64_t peer;      // even CTA: the odd CTA's partial of the item is in dk/dv
   uint64_t peer_ack;  // odd CTA: the even CTA has read it
   uint64_t epi;       // every softmax warp of this CTA is through the item's dK, dV
-  uint64_t drain;
+  uint64_t drain[2];  // per issuing thread: its last products have completed
   uint32_t tmem;
   int abort;
 };
+
+constexpr size_t kKBarsBytes = (sizeof(KBars) + 15) & ~static_cast<size_t>(15);
 
 __device__ __forceinline__ int block_begin(int nb, uint32_t rank) {
   return static_cast<int>((static_cast<long long>(nb) * rank) / 2);
@@ -521,24 +741,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int n_sub = 2 * (I1 - I0);  // steps per item
 
   if (threadIdx.x == 0) {
+    // Arrival counts: one commit per issuing thread where both read or
+    // write (ring stage, K/V, the step's S^T/dP^T, the accumulators).
     mbar_init(&bars->kv_full, 1);
-    mbar_init(&bars->kv_free, 1);
+    mbar_init(&bars->kv_free, 2);
     for (int s = 0; s < kKStages; ++s) {
       mbar_init(&bars->ring_full[s], 1);
-      mbar_init(&bars->ring_empty[s], 1);
+      mbar_init(&bars->ring_empty[s], 2);
     }
     for (int q = 0; q < 2; ++q) {
-      mbar_init(&bars->sp_full[q], 1);
-      mbar_init(&bars->pds_full[q], kSoftWarps);
+      mbar_init(&bars->sp_full[q], 2);
+      mbar_init(&bars->pds_full[q], kSoftWarps / 2);
       mbar_init(&bars->ds_read[q], 1);
       mbar_init(&bars->p_read[q], 1);
     }
-    mbar_init(&bars->acc_full, 1);
+    mbar_init(&bars->acc_full, 2);
     mbar_init(&bars->acc_free, kSoftWarps);
     mbar_init(&bars->peer, 1);
     mbar_init(&bars->peer_ack, 1);
     mbar_init(&bars->epi, kSoftWarps);
-    mbar_init(&bars->drain, 1);
+    mbar_init(&bars->drain[0], 1);
+    mbar_init(&bars->drain[1], 1);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -588,14 +811,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (uint32_t i = rc > kKStages ? rc - kKStages : 0; i < rc; ++i)
         drain(&bars->ring_full[i % kKStages], (i / kKStages) & 1u);
     }
-  } else if (warp == kWarpMma) {
+  } else if (warp == kWarpMma || warp == kWarpMma2) {
+    // Two issuing threads, one per chain of tensor-memory columns: issuer 0
+    // forms dP^T and, from the dS^T written over it, dK; issuer 1 forms S^T
+    // and, from the P^T written over it, dV.  Each accumulator is fed by one
+    // thread in a fixed order.
     if (lane_id() == 0) {
+      const int who = warp - kWarpMma;
       const uint32_t k_a = smem_u32(k_s), v_a = smem_u32(v_s), ring_a = smem_u32(ring);
       const uint32_t tV = tmem + 256, tK = tmem + 384;
       const uint32_t ns = static_cast<uint32_t>(n_sub);
       const uint32_t total = static_cast<uint32_t>(a.B) * ns;
-      // dP^T = V dO^T (dO as hi + lo) and S^T = K Q^T of step s into buffer
-      // s % 2, each once the products of step s - 2 have read the columns.
+      // Issuer 0: dP^T = V dO^T (dO as hi + lo); issuer 1: S^T = K Q^T; of
+      // step s into buffer s % 2, once this issuer's products of step s - 2
+      // have read the columns.
       auto issue_sp = [&](uint32_t s) -> bool {
         const uint32_t b = s & 1u, u = s >> 1, st = s % kKStages, n = s % ns, item = s / ns;
         if (n == 0 && !mbar_wait(&bars->kv_full, item & 1u, abort, a.err, kSiteKV)) return false;
@@ -603,20 +832,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           return false;
         const uint32_t qs = ring_a + st * 3 * kSubBytes, dh = qs + kSubBytes, dl = dh + kSubBytes;
         const uint32_t tS = tmem + 128 * b, tP = tS + 64;
-        if (u > 0 && !mbar_wait(&bars->ds_read[b], (u - 1) & 1u, abort, a.err, kSiteSP))
+        if (u > 0 && !mbar_wait(who == 0 ? &bars->ds_read[b] : &bars->p_read[b], (u - 1) & 1u,
+                                abort, a.err, kSiteSP))
           return false;
         tc_fence_after();
-        mma_kk(tP, v_a, kKHalf, dh, kSubHalf, kSubRows, false);  // dP^T = V dO_hi^T
-        mma_kk(tP, v_a, kKHalf, dl, kSubHalf, kSubRows, true);   //      + V dO_lo^T
-        if (u > 0 && !mbar_wait(&bars->p_read[b], (u - 1) & 1u, abort, a.err, kSiteSP))
-          return false;
-        tc_fence_after();
-        mma_kk(tS, k_a, kKHalf, qs, kSubHalf, kSubRows, false);  // S^T = K Q^T
+        if (who == 0) {
+          mma_kk(tP, v_a, kKHalf, dh, kSubHalf, kSubRows, false);  // dP^T = V dO_hi^T
+          mma_kk(tP, v_a, kKHalf, dl, kSubHalf, kSubRows, true);   //      + V dO_lo^T
+        } else {
+          mma_kk(tS, k_a, kKHalf, qs, kSubHalf, kSubRows, false);  // S^T = K Q^T
+        }
         umma1_commit(&bars->sp_full[b]);
         if (n + 1 == ns) umma1_commit(&bars->kv_free);
         return true;
       };
-      // dK += dS^T Q, dV += P^T dO (P^T and dS^T as hi + lo) of step s.
+      // Issuer 0: dK += dS^T Q; issuer 1: dV += P^T dO (P^T, dS^T and dO as
+      // hi + lo) of step s.
       auto issue_g = [&](uint32_t s) -> bool {
         const uint32_t b = s & 1u, u = s >> 1, st = s % kKStages, n = s % ns, item = s / ns;
         if (!mbar_wait(&bars->pds_full[b], u & 1u, abort, a.err, kSiteDS)) return false;
@@ -627,13 +858,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t qs = ring_a + st * 3 * kSubBytes, dh = qs + kSubBytes, dl = dh + kSubBytes;
         const uint32_t tS = tmem + 128 * b, tP = tS + 64;
         const bool first = n == 0;
-        mma_tm(tK, [=](int kk) { return tP + 16 * kk; }, 4, qs, kSubHalf, !first);
-        mma_tm(tK, [=](int kk) { return tP + 16 * kk + 8; }, 4, qs, kSubHalf, true);
-        umma1_commit(&bars->ds_read[b]);
-        mma_tm(tV, [=](int kk) { return tS + 16 * kk; }, 4, dh, kSubHalf, !first);
-        mma_tm(tV, [=](int kk) { return tS + 16 * kk; }, 4, dl, kSubHalf, true);
-        mma_tm(tV, [=](int kk) { return tS + 16 * kk + 8; }, 4, dh, kSubHalf, true);
-        umma1_commit(&bars->p_read[b]);
+        if (who == 0) {
+          mma_tm(tK, [=](int kk) { return tP + 16 * kk; }, 4, qs, kSubHalf, !first);
+          mma_tm(tK, [=](int kk) { return tP + 16 * kk + 8; }, 4, qs, kSubHalf, true);
+          umma1_commit(&bars->ds_read[b]);
+        } else {
+          mma_tm(tV, [=](int kk) { return tS + 16 * kk; }, 4, dh, kSubHalf, !first);
+          mma_tm(tV, [=](int kk) { return tS + 16 * kk; }, 4, dl, kSubHalf, true);
+          mma_tm(tV, [=](int kk) { return tS + 16 * kk + 8; }, 4, dh, kSubHalf, true);
+          umma1_commit(&bars->p_read[b]);
+        }
         umma1_commit(&bars->ring_empty[st]);
         if (n + 1 == ns) umma1_commit(&bars->acc_full);
         return true;
@@ -657,8 +891,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (ok && s + 2 < total) ok = issue_sp(s + 2);
         }
       }
-      umma1_commit(&bars->drain);
-      drain(&bars->drain, 0);
+      umma1_commit(&bars->drain[who]);
+      drain(&bars->drain[who], 0);
     }
   } else if (warp < kSoftWarps) {
     const int g = threadIdx.x >> 7, r = threadIdx.x & 127;  // r: key in the tile
@@ -669,70 +903,85 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int wq = (r >> 5) & 3;  // this warp's 32 keys: key blocks 8 kt + 2 wq (+1)
     const uint32_t peer_even = cluster_addr(&bars->peer, 0);
     const uint32_t ack_odd = cluster_addr(&bars->peer_ack, 1);
-    uint32_t sc = 0, acc_count = 0;  // sc: the CTA's step counter
+    // Two groups of two warpgroups: group q takes the steps of buffer q
+    // (n % 2 == q: heads 4 q .. 4 q + 3), warpgroup hg of it the rows of
+    // heads 4 q + 2 hg + k, k = 0, 1 (two 16-row blocks, one bias cell each).
+    const int q = g >> 1, hg = g & 1;
+    uint32_t uq = 0, acc_count = 0;  // uq: this group's steps so far
+    const int lane = static_cast<int>(lane_id());
+    // Per warp, two buffers of the step's 32 lse2 then 32 delta values (row
+    // 16 k + il: block k, position il).
+    float *rows = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(bars) + kKBarsBytes) +
+                  warp * 128;
+    // This lane's row of step n of item b (block lane / 16, position
+    // lane % 16): (lse2, delta); a row past L gets lse = +inf (its
+    // probabilities are 0) and delta 0.
+    auto row_value = [&](int b, int n) -> float2 {
+      const int I = I0 + (n >> 1), h = 4 * (n & 1) + 2 * hg + (lane >> 4), il = lane & 15;
+      const bool valid = 16 * I + il < a.L;
+      const size_t row = (static_cast<size_t>(b) * kH + h) * a.L + 16 * I + (valid ? il : 0);
+      return valid ? make_float2(__ldg(a.lse + row) * kLog2e, __ldg(a.delta + row))
+                   : make_float2(__int_as_float(0x7f800000), 0.f);
+    };
     bool ok = true;
     for (int b = 0; b < a.B && ok; ++b) {
       const float *bias_b = a.bias + static_cast<long long>(b) * a.bias_bstride;
       float *dbias_b = a.dbias + static_cast<long long>(b) * a.bias_bstride;
       const bool add_bias = a.bias_bstride == 0 && b > 0;  // shared bias: sum over items
-      for (int n = 0; n < n_sub; ++n) {
-        const int I = I0 + (n >> 1), h = 4 * (n & 1) + g;
-        const size_t row0 = (static_cast<size_t>(b) * kH + h) * a.L + 16 * I;
-        const int nrows = a.L - 16 * I < 16 ? a.L - 16 * I : 16;
-        const float bj = key_ok ? __ldg(bias_b + (static_cast<size_t>(h) * a.P + I) * a.P + J)
-                                : 0.f;
-        const uint32_t bf = sc & 1u, u = sc >> 1;
-        ++sc;
-        ok = mbar_wait(&bars->sp_full[bf], u & 1u, abort, a.err, kSiteSoft);
+      float2 rv_next = q < n_sub ? row_value(b, q) : make_float2(0.f, 0.f);
+      for (int n = q; n < n_sub; n += 2) {
+        const int I = I0 + (n >> 1), h0 = 4 * q + 2 * hg;
+        float bt[2];
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+          bt[k] = __ldg(bias_b + (static_cast<size_t>(h0 + k) * a.P + I) * a.P + J) * a.bias_mul;
+        float *rv = rows + 64 * (uq & 1u);
+        rv[lane] = rv_next.x;
+        rv[32 + lane] = rv_next.y;
+        __syncwarp();
+        if (n + 2 < n_sub) rv_next = row_value(b, n + 2);
+        ok = mbar_wait(&bars->sp_full[q], uq & 1u, abort, a.err, kSiteSoft);
+        ++uq;
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
-        const uint32_t tS = tmem + 128 * bf + 16 * g + lane_base, tP = tS + 64;
-        uint32_t sv[16], pv[16];
-        tmem_ld16(tS, sv);
-        tmem_ld16(tP, pv);
-        tmem_wait_ld16(sv);
-        tmem_wait_ld16(pv);
-        uint32_t ph[8], pl[8], sh[8], sl[8];
-        float cell = 0.f;
+#pragma unroll 1
+        for (int k = 0; k < 2; ++k) {
+          const uint32_t tS = tmem + 128 * q + 32 * hg + 16 * k + lane_base, tP = tS + 64;
+          uint32_t sv[16], pv[16];
+          tmem_ld16(tS, sv);
+          tmem_ld16(tP, pv);
+          tmem_wait_ld16(sv);
+          tmem_wait_ld16(pv);
+          uint32_t ph[8], pl[8], sh[8], sl[8];
+          // Keys past L (zero K rows) get probabilities too; they reach only
+          // their own dK, dV rows, which are not stored, and the bias cell
+          // sum, which leaves them out.
+          const float bterm = k ? bt[1] : bt[0];
+          float cell =
+              a.capped ? key_rows<true>(sv, pv, rv + 16 * k, rv + 32 + 16 * k, bterm, a, ph, pl,
+                                        sh, sl)
+                       : key_rows<false>(sv, pv, rv + 16 * k, rv + 32 + 16 * k, bterm, a, ph,
+                                         pl, sh, sl);
+          if (!key_ok) cell = 0.f;
+          // In place: this warp's lanes of the columns it has just read.
+          tmem_st8(tS, ph);
+          tmem_st8(tS + 8, pl);
+          tmem_st8(tP, sh);
+          tmem_st8(tP + 8, sl);
+          // dbias: sum the cell over its 16 keys (lanes 0-15, 16-31 of the warp).
 #pragma unroll
-        for (int e = 0; e < 16; e += 2) {
-          float pp[2], dd[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int il = e + u;
-            const bool ok_i = key_ok && il < nrows;
-            // Rows past L are clamped to the block's last row (the values
-            // are discarded): every load stays inside lse and delta.
-            const size_t ri = row0 + (il < nrows ? il : nrows - 1);
-            const float l2 = __ldg(a.lse + ri) * kLog2e;
-            const float dl = __ldg(a.delta + ri);
-            const Logit lg = logit(__uint_as_float(sv[il]), bj, l2, a);
-            pp[u] = ok_i ? lg.p : 0.f;
-            dd[u] = ok_i ? lg.p * (__uint_as_float(pv[il]) - dl) * lg.dt : 0.f;
-            cell += dd[u];
+          for (int o = 8; o >= 1; o >>= 1) cell += __shfl_xor_sync(0xffffffffu, cell, o);
+          if ((lane & 15) == 0) {
+            const int Jc = 8 * kt + 2 * wq + (lane >> 4);
+            if (Jc < a.P) {
+              float *dst = dbias_b + (static_cast<size_t>(h0 + k) * a.P + I) * a.P + Jc;
+              *dst = add_bias ? *dst + cell : cell;
+            }
           }
-          split2(pp[0], pp[1], ph[e / 2], pl[e / 2]);
-          split2(dd[0], dd[1], sh[e / 2], sl[e / 2]);
         }
-        // In place: this warp's lanes of the columns it has just read.
-        tmem_st8(tS, ph);
-        tmem_st8(tS + 8, pl);
-        tmem_st8(tP, sh);
-        tmem_st8(tP + 8, sl);
         tmem_wait_st();
         tc_fence_before();
-        warp_arrive(&bars->pds_full[bf]);
-        // dbias: sum the cell over its 16 keys (lanes 0-15, 16-31 of the warp).
-#pragma unroll
-        for (int o = 8; o >= 1; o >>= 1) cell += __shfl_xor_sync(0xffffffffu, cell, o);
-        const int lane = static_cast<int>(lane_id());
-        if ((lane & 15) == 0) {
-          const int Jc = 8 * kt + 2 * wq + (lane >> 4);
-          if (Jc < a.P) {
-            float *dst = dbias_b + (static_cast<size_t>(h) * a.P + I) * a.P + Jc;
-            *dst = add_bias ? *dst + cell : cell;
-          }
-        }
+        warp_arrive(&bars->pds_full[q]);
       }
       if (!ok) break;
       // Item epilogue: dK and dV of this CTA's half, then the pair's sum.
@@ -802,9 +1051,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
 }
 
-constexpr size_t kQuerySmem = 1024 + 3 * kQTileBytes + kQStages * 2 * kQKTileBytes +
+constexpr size_t kQuerySmem = 1024 + 3 * kQTileBytes + 2 * kQStages * kQKTileBytes +
                               sizeof(QBars) + 2 * 512 * sizeof(float);
-constexpr size_t kKeySmem = 1024 + 2 * kKTileBytes + kKStages * 3 * kSubBytes + sizeof(KBars);
+constexpr size_t kKeySmem = 1024 + 2 * kKTileBytes + kKStages * 3 * kSubBytes + kKBarsBytes +
+                            kSoftWarps * 128 * sizeof(float);
 static_assert(kQuerySmem <= 227 * 1024 && kKeySmem <= 227 * 1024, "shared memory budget");
 
 }  // namespace bwdtc
