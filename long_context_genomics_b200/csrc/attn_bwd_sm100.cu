@@ -100,7 +100,7 @@ __device__ __forceinline__ void mma_kk(uint32_t d, uint32_t a, uint32_t a_half, 
   for (int kk = 0; kk < 8; ++kk) {
     const uint32_t ao = ((kk >> 2) * a_half + (kk & 3) * 32) >> 4;
     const uint32_t bo = ((kk >> 2) * b_half + (kk & 3) * 32) >> 4;
-    umma1_ss_lo(d, a_lo + ao, kHi, b_lo + bo, kHi, idesc(N, 0), (acc || kk > 0) ? 1u : 0u);
+    umma1_ss_w(d, a_lo + ao, kHi, b_lo + bo, kHi, idesc(N, 0), (acc || kk > 0) ? 1u : 0u);
   }
 }
 
@@ -112,7 +112,7 @@ __device__ __forceinline__ void mma_tm(uint32_t d, ACol a_col, int nk, uint32_t 
                                        uint32_t b_atom, bool acc) {
   const uint32_t b_lo = desc_sw128_lo(b, b_atom);
   for (int kk = 0; kk < nk; ++kk)
-    umma1_ts_lo(d, a_col(kk), b_lo + ((kk * 16 * 128) >> 4), kHi, idesc(128, 1),
+    umma1_ts_w(d, a_col(kk), b_lo + ((kk * 16 * 128) >> 4), kHi, idesc(128, 1),
                 (acc || kk > 0) ? 1u : 0u);
 }
 
@@ -455,77 +455,75 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Two issuing threads: issuer 0 forms dP, issuer 1 forms S and (pass 2)
     // dQ from the dS written over S, so the dQ accumulator is fed by one
     // thread in a fixed order.
-    if (lane_id() == 0) {
-      const int who = warp - kWarpMma;
-      const uint32_t q_a = smem_u32(q_s), dh_a = smem_u32(dh_s), dl_a = smem_u32(dl_s);
-      const uint32_t k_a = smem_u32(k_ring), v_a = smem_u32(v_ring);
-      const uint32_t tQ = tmem + 256;
-      const uint32_t nk = static_cast<uint32_t>(n_kt);
-      // Issuer 0: dP = dO V^T (dO as hi + lo) of step s into buffer s % 2,
-      // once the softmax warps have read the dP of the buffer's previous
-      // step.  Issuer 1: S = Q K^T, once the buffer's previous S (pass 1) or
-      // the dS over it (pass 2, read by dQ) is no longer needed.
-      auto issue_sp = [&](uint32_t s) -> bool {
-        const uint32_t b = s % kQBufs, u = s / kQBufs, st = s % kQStages, j = s % nk;
-        const uint32_t rph = (s / kQStages) & 1u;
-        if (j == 0 && !mbar_wait(&bars->q_full, (s / nk) & 1u, abort, a.err, kSiteQ))
-          return false;
-        if (u > 0) {
-          uint64_t *prev = (PASS == 1 || who == 1) ? &bars->buf_free[b] : &bars->ds_full[b];
-          if (!mbar_wait(prev, (u - 1) & 1u, abort, a.err, kSiteSP)) return false;
-        }
-        if (who == 0) {
-          if (!mbar_wait(&bars->v_full[st], rph, abort, a.err, kSiteKV)) return false;
-          tc_fence_after();
-          const uint32_t vs = v_a + st * kQKTileBytes, tP = tmem + 128 * b + 64;
-          mma_kk(tP, dh_a, kQHalf, vs, kQKHalf, kQKeys, false);  // dP = dO_hi V^T
-          mma_kk(tP, dl_a, kQHalf, vs, kQKHalf, kQKeys, true);   //    + dO_lo V^T
-          umma1_commit(&bars->v_empty[st]);
-        } else {
-          if (!mbar_wait(&bars->k_full[st], rph, abort, a.err, kSiteKV)) return false;
-          tc_fence_after();
-          const uint32_t ks = k_a + st * kQKTileBytes, tS = tmem + 128 * b;
-          mma_kk(tS, q_a, kQHalf, ks, kQKHalf, kQKeys, false);   // S = Q K^T
-          if (PASS == 1) umma1_commit(&bars->k_empty[st]);
-        }
-        umma1_commit(&bars->sp_full[b]);
-        if (j + 1 == nk) umma1_commit(&bars->q_empty);
-        return true;
-      };
-      // Issuer 1, pass 2: dQ += dS K of step s, dS (hi, lo) over the S
-      // columns of its buffer.
-      auto issue_dq = [&](uint32_t s) -> bool {
-        const uint32_t b = s % kQBufs, u = s / kQBufs, st = s % kQStages, j = s % nk;
-        if (!mbar_wait(&bars->ds_full[b], u & 1u, abort, a.err, kSiteDS)) return false;
-        // The tile's first dQ overwrites the accumulator: every softmax warp
-        // must have read the previous tile's.
-        const uint32_t tile = s / nk;
-        if (j == 0 && tile > 0 &&
-            !mbar_wait(&bars->dq_free, (tile - 1) & 1u, abort, a.err, kSiteEnd))
-          return false;
-        tc_fence_after();
-        const uint32_t kp = k_a + st * kQKTileBytes, tS = tmem + 128 * b;
-        mma_tm(tQ, [=](int kk) { return tS + 16 * kk; }, 4, kp, kQKHalf, j > 0);
-        mma_tm(tQ, [=](int kk) { return tS + 16 * kk + 8; }, 4, kp, kQKHalf, true);
-        umma1_commit(&bars->buf_free[b]);
-        umma1_commit(&bars->k_empty[st]);
-        if (j + 1 == nk) umma1_commit(&bars->dq_full);
-        return true;
-      };
-      if (PASS == 1 || who == 0) {
-        for (uint32_t s = 0; s < total; ++s)
-          if (!issue_sp(s)) break;
-      } else {
-        bool ok = true;
-        for (uint32_t s = 0; s < 2 && s < total && ok; ++s) ok = issue_sp(s);
-        for (uint32_t s = 0; s < total && ok; ++s) {
-          ok = issue_dq(s);
-          if (ok && s + 2 < total) ok = issue_sp(s + 2);
-        }
+    const int who = warp - kWarpMma;
+    const uint32_t q_a = smem_u32(q_s), dh_a = smem_u32(dh_s), dl_a = smem_u32(dl_s);
+    const uint32_t k_a = smem_u32(k_ring), v_a = smem_u32(v_ring);
+    const uint32_t tQ = tmem + 256;
+    const uint32_t nk = static_cast<uint32_t>(n_kt);
+    // Issuer 0: dP = dO V^T (dO as hi + lo) of step s into buffer s % 2,
+    // once the softmax warps have read the dP of the buffer's previous
+    // step.  Issuer 1: S = Q K^T, once the buffer's previous S (pass 1) or
+    // the dS over it (pass 2, read by dQ) is no longer needed.
+    auto issue_sp = [&](uint32_t s) -> bool {
+      const uint32_t b = s % kQBufs, u = s / kQBufs, st = s % kQStages, j = s % nk;
+      const uint32_t rph = (s / kQStages) & 1u;
+      if (j == 0 && !mbar_wait_warp(&bars->q_full, (s / nk) & 1u, abort, a.err, kSiteQ))
+        return false;
+      if (u > 0) {
+        uint64_t *prev = (PASS == 1 || who == 1) ? &bars->buf_free[b] : &bars->ds_full[b];
+        if (!mbar_wait_warp(prev, (u - 1) & 1u, abort, a.err, kSiteSP)) return false;
       }
-      umma1_commit(&bars->drain[who]);
-      drain(&bars->drain[who], 0);
+      if (who == 0) {
+        if (!mbar_wait_warp(&bars->v_full[st], rph, abort, a.err, kSiteKV)) return false;
+        tc_fence_after();
+        const uint32_t vs = v_a + st * kQKTileBytes, tP = tmem + 128 * b + 64;
+        mma_kk(tP, dh_a, kQHalf, vs, kQKHalf, kQKeys, false);  // dP = dO_hi V^T
+        mma_kk(tP, dl_a, kQHalf, vs, kQKHalf, kQKeys, true);   //    + dO_lo V^T
+        umma1_commit_w(&bars->v_empty[st]);
+      } else {
+        if (!mbar_wait_warp(&bars->k_full[st], rph, abort, a.err, kSiteKV)) return false;
+        tc_fence_after();
+        const uint32_t ks = k_a + st * kQKTileBytes, tS = tmem + 128 * b;
+        mma_kk(tS, q_a, kQHalf, ks, kQKHalf, kQKeys, false);   // S = Q K^T
+        if (PASS == 1) umma1_commit_w(&bars->k_empty[st]);
+      }
+      umma1_commit_w(&bars->sp_full[b]);
+      if (j + 1 == nk) umma1_commit_w(&bars->q_empty);
+      return true;
+    };
+    // Issuer 1, pass 2: dQ += dS K of step s, dS (hi, lo) over the S
+    // columns of its buffer.
+    auto issue_dq = [&](uint32_t s) -> bool {
+      const uint32_t b = s % kQBufs, u = s / kQBufs, st = s % kQStages, j = s % nk;
+      if (!mbar_wait_warp(&bars->ds_full[b], u & 1u, abort, a.err, kSiteDS)) return false;
+      // The tile's first dQ overwrites the accumulator: every softmax warp
+      // must have read the previous tile's.
+      const uint32_t tile = s / nk;
+      if (j == 0 && tile > 0 &&
+          !mbar_wait_warp(&bars->dq_free, (tile - 1) & 1u, abort, a.err, kSiteEnd))
+        return false;
+      tc_fence_after();
+      const uint32_t kp = k_a + st * kQKTileBytes, tS = tmem + 128 * b;
+      mma_tm(tQ, [=](int kk) { return tS + 16 * kk; }, 4, kp, kQKHalf, j > 0);
+      mma_tm(tQ, [=](int kk) { return tS + 16 * kk + 8; }, 4, kp, kQKHalf, true);
+      umma1_commit_w(&bars->buf_free[b]);
+      umma1_commit_w(&bars->k_empty[st]);
+      if (j + 1 == nk) umma1_commit_w(&bars->dq_full);
+      return true;
+    };
+    if (PASS == 1 || who == 0) {
+      for (uint32_t s = 0; s < total; ++s)
+        if (!issue_sp(s)) break;
+    } else {
+      bool ok = true;
+      for (uint32_t s = 0; s < 2 && s < total && ok; ++s) ok = issue_sp(s);
+      for (uint32_t s = 0; s < total && ok; ++s) {
+        ok = issue_dq(s);
+        if (ok && s + 2 < total) ok = issue_sp(s + 2);
+      }
     }
+    umma1_commit_w(&bars->drain[who]);
+    drain(&bars->drain[who], 0);
   } else if (warp < kSoftWarps) {
     const int g = threadIdx.x >> 7, r = threadIdx.x & 127;
     const int q = g >> 1, hg = g & 1;  // group (buffer), key half
@@ -816,84 +814,82 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // forms dP^T and, from the dS^T written over it, dK; issuer 1 forms S^T
     // and, from the P^T written over it, dV.  Each accumulator is fed by one
     // thread in a fixed order.
-    if (lane_id() == 0) {
-      const int who = warp - kWarpMma;
-      const uint32_t k_a = smem_u32(k_s), v_a = smem_u32(v_s), ring_a = smem_u32(ring);
-      const uint32_t tV = tmem + 256, tK = tmem + 384;
-      const uint32_t ns = static_cast<uint32_t>(n_sub);
-      const uint32_t total = static_cast<uint32_t>(a.B) * ns;
-      // Issuer 0: dP^T = V dO^T (dO as hi + lo); issuer 1: S^T = K Q^T; of
-      // step s into buffer s % 2, once this issuer's products of step s - 2
-      // have read the columns.
-      auto issue_sp = [&](uint32_t s) -> bool {
-        const uint32_t b = s & 1u, u = s >> 1, st = s % kKStages, n = s % ns, item = s / ns;
-        if (n == 0 && !mbar_wait(&bars->kv_full, item & 1u, abort, a.err, kSiteKV)) return false;
-        if (!mbar_wait(&bars->ring_full[st], (s / kKStages) & 1u, abort, a.err, kSiteRing))
-          return false;
-        const uint32_t qs = ring_a + st * 3 * kSubBytes, dh = qs + kSubBytes, dl = dh + kSubBytes;
-        const uint32_t tS = tmem + 128 * b, tP = tS + 64;
-        if (u > 0 && !mbar_wait(who == 0 ? &bars->ds_read[b] : &bars->p_read[b], (u - 1) & 1u,
-                                abort, a.err, kSiteSP))
-          return false;
-        tc_fence_after();
-        if (who == 0) {
-          mma_kk(tP, v_a, kKHalf, dh, kSubHalf, kSubRows, false);  // dP^T = V dO_hi^T
-          mma_kk(tP, v_a, kKHalf, dl, kSubHalf, kSubRows, true);   //      + V dO_lo^T
-        } else {
-          mma_kk(tS, k_a, kKHalf, qs, kSubHalf, kSubRows, false);  // S^T = K Q^T
-        }
-        umma1_commit(&bars->sp_full[b]);
-        if (n + 1 == ns) umma1_commit(&bars->kv_free);
-        return true;
-      };
-      // Issuer 0: dK += dS^T Q; issuer 1: dV += P^T dO (P^T, dS^T and dO as
-      // hi + lo) of step s.
-      auto issue_g = [&](uint32_t s) -> bool {
-        const uint32_t b = s & 1u, u = s >> 1, st = s % kKStages, n = s % ns, item = s / ns;
-        if (!mbar_wait(&bars->pds_full[b], u & 1u, abort, a.err, kSiteDS)) return false;
-        if (n == 0 && item > 0 &&
-            !mbar_wait(&bars->acc_free, (item - 1) & 1u, abort, a.err, kSiteAcc))
-          return false;
-        tc_fence_after();
-        const uint32_t qs = ring_a + st * 3 * kSubBytes, dh = qs + kSubBytes, dl = dh + kSubBytes;
-        const uint32_t tS = tmem + 128 * b, tP = tS + 64;
-        const bool first = n == 0;
-        if (who == 0) {
-          mma_tm(tK, [=](int kk) { return tP + 16 * kk; }, 4, qs, kSubHalf, !first);
-          mma_tm(tK, [=](int kk) { return tP + 16 * kk + 8; }, 4, qs, kSubHalf, true);
-          umma1_commit(&bars->ds_read[b]);
-        } else {
-          mma_tm(tV, [=](int kk) { return tS + 16 * kk; }, 4, dh, kSubHalf, !first);
-          mma_tm(tV, [=](int kk) { return tS + 16 * kk; }, 4, dl, kSubHalf, true);
-          mma_tm(tV, [=](int kk) { return tS + 16 * kk + 8; }, 4, dh, kSubHalf, true);
-          umma1_commit(&bars->p_read[b]);
-        }
-        umma1_commit(&bars->ring_empty[st]);
-        if (n + 1 == ns) umma1_commit(&bars->acc_full);
-        return true;
-      };
-      if (ns == 0) {
-        // No query blocks here: zero partials, but the same per-item handshakes.
-        for (int b = 0; b < a.B; ++b) {
-          if (!mbar_wait(&bars->kv_full, static_cast<uint32_t>(b) & 1u, abort, a.err, kSiteKV))
-            break;
-          umma1_commit(&bars->kv_free);
-          if (b > 0 && !mbar_wait(&bars->acc_free, static_cast<uint32_t>(b - 1) & 1u, abort,
-                                  a.err, kSiteAcc))
-            break;
-          umma1_commit(&bars->acc_full);
-        }
+    const int who = warp - kWarpMma;
+    const uint32_t k_a = smem_u32(k_s), v_a = smem_u32(v_s), ring_a = smem_u32(ring);
+    const uint32_t tV = tmem + 256, tK = tmem + 384;
+    const uint32_t ns = static_cast<uint32_t>(n_sub);
+    const uint32_t total = static_cast<uint32_t>(a.B) * ns;
+    // Issuer 0: dP^T = V dO^T (dO as hi + lo); issuer 1: S^T = K Q^T; of
+    // step s into buffer s % 2, once this issuer's products of step s - 2
+    // have read the columns.
+    auto issue_sp = [&](uint32_t s) -> bool {
+      const uint32_t b = s & 1u, u = s >> 1, st = s % kKStages, n = s % ns, item = s / ns;
+      if (n == 0 && !mbar_wait_warp(&bars->kv_full, item & 1u, abort, a.err, kSiteKV)) return false;
+      if (!mbar_wait_warp(&bars->ring_full[st], (s / kKStages) & 1u, abort, a.err, kSiteRing))
+        return false;
+      const uint32_t qs = ring_a + st * 3 * kSubBytes, dh = qs + kSubBytes, dl = dh + kSubBytes;
+      const uint32_t tS = tmem + 128 * b, tP = tS + 64;
+      if (u > 0 && !mbar_wait_warp(who == 0 ? &bars->ds_read[b] : &bars->p_read[b], (u - 1) & 1u,
+                              abort, a.err, kSiteSP))
+        return false;
+      tc_fence_after();
+      if (who == 0) {
+        mma_kk(tP, v_a, kKHalf, dh, kSubHalf, kSubRows, false);  // dP^T = V dO_hi^T
+        mma_kk(tP, v_a, kKHalf, dl, kSubHalf, kSubRows, true);   //      + V dO_lo^T
       } else {
-        bool ok = true;
-        for (uint32_t s = 0; s < 2 && s < total && ok; ++s) ok = issue_sp(s);
-        for (uint32_t s = 0; s < total && ok; ++s) {
-          ok = issue_g(s);
-          if (ok && s + 2 < total) ok = issue_sp(s + 2);
-        }
+        mma_kk(tS, k_a, kKHalf, qs, kSubHalf, kSubRows, false);  // S^T = K Q^T
       }
-      umma1_commit(&bars->drain[who]);
-      drain(&bars->drain[who], 0);
+      umma1_commit_w(&bars->sp_full[b]);
+      if (n + 1 == ns) umma1_commit_w(&bars->kv_free);
+      return true;
+    };
+    // Issuer 0: dK += dS^T Q; issuer 1: dV += P^T dO (P^T, dS^T and dO as
+    // hi + lo) of step s.
+    auto issue_g = [&](uint32_t s) -> bool {
+      const uint32_t b = s & 1u, u = s >> 1, st = s % kKStages, n = s % ns, item = s / ns;
+      if (!mbar_wait_warp(&bars->pds_full[b], u & 1u, abort, a.err, kSiteDS)) return false;
+      if (n == 0 && item > 0 &&
+          !mbar_wait_warp(&bars->acc_free, (item - 1) & 1u, abort, a.err, kSiteAcc))
+        return false;
+      tc_fence_after();
+      const uint32_t qs = ring_a + st * 3 * kSubBytes, dh = qs + kSubBytes, dl = dh + kSubBytes;
+      const uint32_t tS = tmem + 128 * b, tP = tS + 64;
+      const bool first = n == 0;
+      if (who == 0) {
+        mma_tm(tK, [=](int kk) { return tP + 16 * kk; }, 4, qs, kSubHalf, !first);
+        mma_tm(tK, [=](int kk) { return tP + 16 * kk + 8; }, 4, qs, kSubHalf, true);
+        umma1_commit_w(&bars->ds_read[b]);
+      } else {
+        mma_tm(tV, [=](int kk) { return tS + 16 * kk; }, 4, dh, kSubHalf, !first);
+        mma_tm(tV, [=](int kk) { return tS + 16 * kk; }, 4, dl, kSubHalf, true);
+        mma_tm(tV, [=](int kk) { return tS + 16 * kk + 8; }, 4, dh, kSubHalf, true);
+        umma1_commit_w(&bars->p_read[b]);
+      }
+      umma1_commit_w(&bars->ring_empty[st]);
+      if (n + 1 == ns) umma1_commit_w(&bars->acc_full);
+      return true;
+    };
+    if (ns == 0) {
+      // No query blocks here: zero partials, but the same per-item handshakes.
+      for (int b = 0; b < a.B; ++b) {
+        if (!mbar_wait_warp(&bars->kv_full, static_cast<uint32_t>(b) & 1u, abort, a.err, kSiteKV))
+          break;
+        umma1_commit_w(&bars->kv_free);
+        if (b > 0 && !mbar_wait_warp(&bars->acc_free, static_cast<uint32_t>(b - 1) & 1u, abort,
+                                a.err, kSiteAcc))
+          break;
+        umma1_commit_w(&bars->acc_full);
+      }
+    } else {
+      bool ok = true;
+      for (uint32_t s = 0; s < 2 && s < total && ok; ++s) ok = issue_sp(s);
+      for (uint32_t s = 0; s < total && ok; ++s) {
+        ok = issue_g(s);
+        if (ok && s + 2 < total) ok = issue_sp(s + 2);
+      }
     }
+    umma1_commit_w(&bars->drain[who]);
+    drain(&bars->drain[who], 0);
   } else if (warp < kSoftWarps) {
     const int g = threadIdx.x >> 7, r = threadIdx.x & 127;  // r: key in the tile
     const uint32_t lane_base = static_cast<uint32_t>(r >> 5) << 21;

@@ -317,7 +317,7 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_addr,
   for (int kk = 0; kk < 8; ++kk) {
     const uint32_t qo = ((kk >> 2) * kQHalfBytes + (kk & 3) * 32) >> 4;
     const uint32_t ko = ((kk >> 2) * kKHalfBytes + (kk & 3) * 32) >> 4;
-    umma2_ss_lo(d_tmem, q_lo + qo, k_lo + ko, kDescHi, kIdescQK, kk > 0 ? 1u : 0u);
+    umma2_ss_w(d_tmem, q_lo + qo, k_lo + ko, kDescHi, kIdescQK, kk > 0 ? 1u : 0u);
   }
 }
 
@@ -331,8 +331,8 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem,
   const uint32_t v_lo = desc_sw128_lo(v_addr, VL::kAtomBytes);
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk) {
-    umma2_ts_lo(d_tmem, p_tmem + 8 * kk, v_lo + ((kk * VL::kKStepBytes) >> 4), VL::kDescHi,
-                idesc_pv<DV>(), (accumulate || kk > 0) ? 1u : 0u);
+    umma2_ts_w(d_tmem, p_tmem + 8 * kk, v_lo + ((kk * VL::kKStepBytes) >> 4), VL::kDescHi,
+               idesc_pv<DV>(), (accumulate || kk > 0) ? 1u : 0u);
   }
 }
 
@@ -475,7 +475,8 @@ __device__ __forceinline__ void relay_v(Barriers *bars, const Params &p, volatil
 }
 
 // --------------------------------------------------------------------------
-// Issuing threads of the even CTA.  The odd CTA's arrivals on their barriers
+// Issuing warps of the even CTA (every lane waits; one elected lane issues).
+// The odd CTA's arrivals on their barriers
 // (relays, softmax) are relaxed (see mbar_arrive_cluster), so their waits
 // acquire at CTA scope: a cluster-scope acquire would order nothing more and
 // costs about 180 cycles per wait (measured).
@@ -491,7 +492,7 @@ __device__ __forceinline__ void issuer_s(uint8_t *q_s, uint8_t *k_s, Barriers *b
   Cursor cu = cursor_begin(p);
   Segment sg;
   while (ok && next_segment(p, cu, sg)) {
-    ok = mbar_wait(&bars->q_full, qc & 1u, abort, p.err, kSiteIssueQ);
+    ok = mbar_wait_warp(&bars->q_full, qc & 1u, abort, p.err, kSiteIssueQ);
     ++qc;
     if (!ok) break;
     uint32_t slot = 0;
@@ -499,25 +500,25 @@ __device__ __forceinline__ void issuer_s(uint8_t *q_s, uint8_t *k_s, Barriers *b
       const int i = j - sg.kb;
       if ((i & 1) == 0) {
         slot = kl % kStages;
-        ok = mbar_wait(&bars->k_full[slot], (kl / kStages) & 1u, abort, p.err, kSiteIssueK);
+        ok = mbar_wait_warp(&bars->k_full[slot], (kl / kStages) & 1u, abort, p.err, kSiteIssueK);
         ++kl;
         if (!ok) break;
       }
       const uint32_t sb = su & 1u, sn = su >> 1;
       if (sn > 0) {
-        ok = mbar_wait(&bars->s_free[sb], (sn - 1) & 1u, abort, p.err, kSiteIssueSFree);
+        ok = mbar_wait_warp(&bars->s_free[sb], (sn - 1) & 1u, abort, p.err, kSiteIssueSFree);
         if (!ok) break;
       }
       tc_fence_after();
       issue_qk(tmem + 128u * sb, q_addr, k_addr + slot * kKSlotBytes + (i & 1) * kKTileBytes);
-      umma2_commit_both(&bars->s_full[sb]);
-      if (j + 1 == sg.ke) umma2_commit_both(&bars->q_empty);
-      if ((i & 1) == 1 || j + 1 == sg.ke) umma2_commit_both(&bars->k_empty[slot]);
+      umma2_commit_both_w(&bars->s_full[sb]);
+      if (j + 1 == sg.ke) umma2_commit_both_w(&bars->q_empty);
+      if ((i & 1) == 1 || j + 1 == sg.ke) umma2_commit_both_w(&bars->k_empty[slot]);
       ++su;
     }
   }
   // All MMAs this thread issued complete before tensor memory is released.
-  umma2_commit_self(&bars->drain);
+  umma2_commit_self_w(&bars->drain);
   drain_wait(&bars->drain, 0);
 }
 
@@ -537,24 +538,24 @@ __device__ __forceinline__ void issuer_pv(uint8_t *v_s, Barriers *bars, uint32_t
       const int i = j - sg.kb;
       if ((i & 1) == 0) {
         slot = vl % kStages;
-        ok = mbar_wait(&bars->v_full[slot], (vl / kStages) & 1u, abort, p.err, kSiteIssueV);
+        ok = mbar_wait_warp(&bars->v_full[slot], (vl / kStages) & 1u, abort, p.err, kSiteIssueV);
         ++vl;
         if (!ok) break;
       }
       const uint32_t pb = pu % T::kNP, pn = pu / T::kNP;
-      ok = mbar_wait(&bars->p_full[pb], pn & 1u, abort, p.err, kSiteIssueP);
+      ok = mbar_wait_warp(&bars->p_full[pb], pn & 1u, abort, p.err, kSiteIssueP);
       if (!ok) break;
       tc_fence_after();
       issue_pv<DV>(tmem + T::kColO, tmem + T::kColP + 64u * pb,
                    v_addr + slot * v_slot_bytes<DV>() + (i & 1) * VLayout<DV>::kTileBytes,
                    i > 0);
-      umma2_commit_both(&bars->pv_done[pb]);
-      if (j + 1 == sg.ke) umma2_commit_both(&bars->o_full);
-      if ((i & 1) == 1 || j + 1 == sg.ke) umma2_commit_both(&bars->v_empty[slot]);
+      umma2_commit_both_w(&bars->pv_done[pb]);
+      if (j + 1 == sg.ke) umma2_commit_both_w(&bars->o_full);
+      if ((i & 1) == 1 || j + 1 == sg.ke) umma2_commit_both_w(&bars->v_empty[slot]);
       ++pu;
     }
   }
-  umma2_commit_self(&bars->drain);
+  umma2_commit_self_w(&bars->drain);
   drain_wait(&bars->drain, 0);
 }
 
@@ -1168,21 +1169,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   if (warp >= kWarpLoadQK) {
     regs_dec<kRegsLow>();
-    if (lane_id() == 0) {
+    if (rank == 0 && warp == kWarpIssueS) {
+      issuer_s(q_s, k_s, bars, tmem, p, abort);  // the whole warp: elected issue
+    } else if (rank == 0 && warp == kWarpIssuePV) {
+      issuer_pv<DV>(v_s, bars, tmem, p, abort);
+    } else if (lane_id() == 0) {
       if (warp == kWarpLoadQK) {
         producer_qk(&tm_q, &tm_k, q_s, k_s, bars, p, rank, abort);
       } else if (warp == kWarpLoadV) {
         producer_v<DV>(&tm_v, v_s, bars, p, rank, abort);
       } else if (warp == kWarpIssueS) {
-        if (rank == 0)
-          issuer_s(q_s, k_s, bars, tmem, p, abort);
-        else
-          relay_qk(bars, p, abort);
+        relay_qk(bars, p, abort);
       } else if (warp == kWarpIssuePV) {
-        if (rank == 0)
-          issuer_pv<DV>(v_s, bars, tmem, p, abort);
-        else
-          relay_v(bars, p, abort);
+        relay_v(bars, p, abort);
       }
     }
   } else {
