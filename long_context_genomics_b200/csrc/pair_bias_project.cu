@@ -38,18 +38,11 @@ constexpr int kCellBytes = kCp * 4;                  // 512
 constexpr int kChunkCells = 32;                      // one cell per lane
 constexpr int kChunkBytes = kChunkCells * kCellBytes;  // 16 KB
 constexpr int kBoxBytes = kChunkCells * 128;         // 32 cells x 32 channels
-#ifndef AG_PROJ_STAGES
-#define AG_PROJ_STAGES 12
-#endif
-#ifndef AG_PROJ_CTAS_PER_SM
-#define AG_PROJ_CTAS_PER_SM 1
-#endif
-#ifndef AG_PROJ_PROMO
-#define AG_PROJ_PROMO 2
-#endif
-constexpr int kStages = AG_PROJ_STAGES;
-constexpr int kConsumerWarps = AG_PROJ_STAGES;
-constexpr int kCtasPerSm = AG_PROJ_CTAS_PER_SM;
+// Measured on B200 at P = 512 (134 MB): 12 stages of 16 KB per SM reach the
+// same time as 6 of 32 KB; fewer bytes in flight are slower, and two or three
+// CTAs per SM with the same bytes in flight are slower too.
+constexpr int kStages = 12;
+constexpr int kConsumerWarps = 12;
 static_assert(kStages % kConsumerWarps == 0, "each ring slot belongs to one consumer warp");
 constexpr int kThreads = (kConsumerWarps + 1) * 32;  // + producer warp
 constexpr int kWBytes = kCp * kH * 4;                // 4 KB
@@ -68,7 +61,7 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, u
       : "memory");
 }
 
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+__global__ void __launch_bounds__(kThreads, 1)
     pair_bias_project_kernel(const __grid_constant__ CUtensorMap tm_pair,
                              const float *__restrict__ W, float *__restrict__ bias,
                              long long n_cells, unsigned *err) {
@@ -192,11 +185,11 @@ cudaError_t launch_pair_bias_project(const float *pair, const float *W, float *b
   const cuuint32_t estr[2] = {1, 1};
   if (encode(&tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(pair), dims, strides,
              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             AG_PROJ_PROMO == 2 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B : AG_PROJ_PROMO == 1 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B : CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   const long long n_chunks = (n_cells + kChunkCells - 1) / kChunkCells;
-  const long long grid = n_chunks < kCtasPerSm * num_sms ? n_chunks : kCtasPerSm * num_sms;
+  const long long grid = n_chunks < num_sms ? n_chunks : num_sms;
   pair_bias_project_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, stream>>>(
       tm, W, bias, n_cells, err);
   return cudaGetLastError();
