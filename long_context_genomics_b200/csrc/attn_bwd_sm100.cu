@@ -314,29 +314,36 @@ __global__ void __launch_bounds__(256) bwd_split_kernel(const float *__restrict_
 // The CTA's steps (64 keys of one of its tiles each) are numbered s = 0, 1,
 // ... across its tiles.  K and V come in separate 3-slot rings (slot s % 3):
 // V is free as soon as dP has been formed, K only after dQ.  Tensor memory
-// holds two step buffers b = s % 2, S at columns [128 b, 128 b + 64) and dP
-// at [128 b + 64, 128 b + 128); pass 2 writes dS (bf16 hi, lo) over the S
-// columns it has read, and dQ accumulates at [256, 384).
+// holds step buffers b = s % nb (nb = 4 in pass 1, 2 in pass 2), S at
+// columns [128 b, 128 b + 64) and dP at [128 b + 64, 128 b + 128); pass 2
+// writes dS (bf16 hi, lo) over the S columns it has read, and dQ accumulates
+// at [256, 384).
 //
 // The softmax warps form two groups of two warpgroups: group q takes the
-// steps of buffer q (s % 2 == q), so one group's waits for its logits and
-// for tensor-memory traffic are covered by the other group's arithmetic.
+// steps s % 2 == q (so the buffers b % 2 == q), and one group's waits for its
+// logits and for tensor-memory traffic are covered by the other group's
+// arithmetic.
 // Warpgroup hg of a group takes keys [32 hg, 32 hg + 32) of the step (two
 // 16-key blocks, one bias cell each); thread r of it owns row r.
 //
 // The tensor core runs ahead of the softmax warps: pass 1 issues S and dP of
-// a step as soon as its buffer has been loaded by the softmax group; pass 2
+// a step as soon as its buffer has been loaded by the softmax group (up to
+// two of each group's steps ahead); pass 2
 // issues, per step s, dQ of step s, then dP of step s + 2 (its columns were
 // read before dS of step s was written), then S of step s + 2 once dQ of
 // step s has read the columns -- a wait covered by the dP products queued.
-constexpr int kQBufs = 2;
+constexpr int kQBufsMax = 4;
+// Step buffers: four in pass 1 (two per softmax group, so the tensor core
+// can run two of a group's steps ahead), two in pass 2 (dQ takes the rest).
+template <int PASS>
+constexpr int q_bufs() { return PASS == 1 ? 4 : 2; }
 constexpr int kGroupWarps = kSoftWarps / 2;
 struct QBars {
   uint64_t q_full, q_empty;
   uint64_t k_full[kQStages], k_empty[kQStages], v_full[kQStages], v_empty[kQStages];
-  uint64_t sp_full[kQBufs];   // S and dP of the buffer's step are in tensor memory
-  uint64_t buf_free[kQBufs];  // the buffer's S columns may be overwritten
-  uint64_t ds_full[kQBufs];   // pass 2: dS of the buffer's step is written
+  uint64_t sp_full[kQBufsMax];   // S and dP of the buffer's step are in tensor memory
+  uint64_t buf_free[kQBufsMax];  // the buffer's S columns may be overwritten
+  uint64_t ds_full[kQBufsMax];   // pass 2: dS of the buffer's step is written
   uint64_t dq_full, dq_free, xd;
   uint64_t drain[2];  // per issuing thread: its last products have completed
   uint32_t tmem;
@@ -349,6 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                      const __grid_constant__ CUtensorMap tm_do,
                      const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ Args a) {
+  constexpr int kQBufs = q_bufs<PASS>();
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t *q_s = smem_raw + pad;                 // Q tile (32 KB)
@@ -552,10 +560,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int k = 0; k < 2; ++k)
           bt[k] = (key0 + 16 * k < a.L ? __ldg(brow + key0 / 16 + k) : 0.f) * a.bias_mul;
-        ok = mbar_wait(&bars->sp_full[q], u & 1u, abort, a.err, kSiteSoft);
+        const uint32_t bf = s % kQBufs;  // a buffer of this group (bf % 2 == q)
+        ok = mbar_wait(&bars->sp_full[bf], u & 1u, abort, a.err, kSiteSoft);
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
-        const uint32_t tS = tmem + 128 * q + 32 * hg + lane_base;
+        const uint32_t tS = tmem + 128 * bf + 32 * hg + lane_base;
         if (PASS == 1) {
           uint32_t sv[2][16], pv[2][16];
 #pragma unroll
@@ -569,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_wait_ld16(pv[k]);
           }
           tc_fence_before();
-          warp_arrive(&bars->buf_free[q]);
+          warp_arrive(&bars->buf_free[bf]);
 #pragma unroll
           for (int k = 0; k < 2; ++k) {
             const int nvalid = a.L - (key0 + 16 * k);  // keys of the 16 before L
@@ -607,7 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tmem_wait_st();
           tc_fence_before();
-          warp_arrive(&bars->ds_full[q]);
+          warp_arrive(&bars->ds_full[bf]);
         }
       }
       if (!ok) break;
