@@ -590,25 +590,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                               : delta_part<false, true>(sv[k], pv[k], bt[k], lse2, nvalid, a);
           }
         } else {
-#pragma unroll 1
+          // Both blocks' loads in flight at once; each block's dS is written
+          // over its own S columns as soon as it is formed.
+          uint32_t sv[2][16], pv[2][16];
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            tmem_ld16(tS + 16 * k, sv[k]);
+            tmem_ld16(tS + 64 + 16 * k, pv[k]);
+          }
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            tmem_wait_ld16(sv[k]);
+            tmem_wait_ld16(pv[k]);
+          }
+#pragma unroll
           for (int k = 0; k < 2; ++k) {
             const int nvalid = a.L - (key0 + 16 * k);
-            const float bterm = k ? bt[1] : bt[0];
-            uint32_t sv[16], pv[16], hi[8], lo[8];
-            tmem_ld16(tS + 16 * k, sv);
-            tmem_ld16(tS + 64 + 16 * k, pv);
-            tmem_wait_ld16(sv);
-            tmem_wait_ld16(pv);
+            uint32_t hi[8], lo[8];
             if (nvalid >= 16) {
               if (a.capped)
-                ds_row<true, false>(sv, pv, bterm, lse2, del, nvalid, a, hi, lo);
+                ds_row<true, false>(sv[k], pv[k], bt[k], lse2, del, nvalid, a, hi, lo);
               else
-                ds_row<false, false>(sv, pv, bterm, lse2, del, nvalid, a, hi, lo);
+                ds_row<false, false>(sv[k], pv[k], bt[k], lse2, del, nvalid, a, hi, lo);
             } else {
               if (a.capped)
-                ds_row<true, true>(sv, pv, bterm, lse2, del, nvalid, a, hi, lo);
+                ds_row<true, true>(sv[k], pv[k], bt[k], lse2, del, nvalid, a, hi, lo);
               else
-                ds_row<false, true>(sv, pv, bterm, lse2, del, nvalid, a, hi, lo);
+                ds_row<false, true>(sv[k], pv[k], bt[k], lse2, del, nvalid, a, hi, lo);
             }
             // In place: this warp's lanes of the S columns it has just read.
             tmem_st8(tS + 16 * k, hi);
