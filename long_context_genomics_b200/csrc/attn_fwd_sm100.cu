@@ -175,9 +175,21 @@ struct Xchg {
   float dpart[kWG][128];     // [warpgroup][row]
 };
 
+// Epilogue staging (value width 128): per softmax warp, 32 rows x 16 fp32
+// columns, rows padded to 20 floats (80 bytes) so that both the row-wise
+// writes and the column-wise reads of a shared-memory phase hit 8 distinct
+// 16-byte bank groups (one 2-way pair on the reads).  With it the output is
+// stored 64 contiguous bytes per row per 4 lanes instead of 16 bytes per lane
+// at a 512-byte stride.  Value width 192 has no room for it and stores
+// directly.
+constexpr int kStageRow = 20;
+template <int DV> constexpr size_t stage_bytes() {
+  return DV == 128 ? static_cast<size_t>(kSoftThreads / 32) * 32 * kStageRow * 4 : 0;
+}
+constexpr size_t kBarsXchgBytes = (sizeof(Barriers) + sizeof(Xchg) + 15) & ~static_cast<size_t>(15);
 template <int DV> constexpr size_t smem_bytes() {
   return 1024 + static_cast<size_t>(kQTileBytes) + kStages * static_cast<size_t>(kKSlotBytes) +
-         kStages * static_cast<size_t>(v_slot_bytes<DV>()) + sizeof(Barriers) + sizeof(Xchg);
+         kStages * static_cast<size_t>(v_slot_bytes<DV>()) + kBarsXchgBytes + stage_bytes<DV>();
 }
 static_assert(smem_bytes<128>() <= 227 * 1024 && smem_bytes<192>() <= 227 * 1024,
               "shared memory budget");
@@ -981,7 +993,7 @@ __device__ __forceinline__ bool segment_online(const Segment &sg, const float *b
 }
 
 template <int MODE, int DV>
-__device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc, uint32_t tmem,
+__device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc, float *stage, uint32_t tmem,
                                              const Params &p, uint32_t rank,
                                              volatile int *abort) {
   using T = Tmem<DV>;
@@ -1072,27 +1084,77 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc, uint32_t 
       wb = eb * inv / dsum;
       lse_w = M + lg2_approx(ea + eb) * kLn2;
     }
-    // This warpgroup's DV / 4 columns of the row, 16 at a time (every lane
-    // loads: tcgen05.ld is warp-wide; rows that do not exist store nothing).
+    if constexpr (DV == 128) {
+      // This warpgroup's 32 columns of its warp's 32 rows, 16 columns at a
+      // time: scaled into the warp's staging rows, then stored by groups of
+      // four lanes, one 64-byte row segment each.
+      const int lane = static_cast<int>(lane_id());
+      float *slot = stage + (threadIdx.x >> 5) * (32 * kStageRow);
+      const int r0 = r - lane;  // the warp's first tile row
 #pragma unroll 1
-    for (int c16 = 0; c16 < DV / 4 / 16; ++c16) {
-      uint32_t o[16];
-      tmem_ld16(tO + 16u * c16, o);
-      tmem_wait_ld16(o);
-      if (writes) {
+      for (int c16 = 0; c16 < 2; ++c16) {
+        uint32_t o[16];
+        tmem_ld16(tO + 16u * c16, o);
+        tmem_wait_ld16(o);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float4 val = make_float4(__uint_as_float(o[4 * e]) * wb, __uint_as_float(o[4 * e + 1]) * wb,
-                                   __uint_as_float(o[4 * e + 2]) * wb,
-                                   __uint_as_float(o[4 * e + 3]) * wb);
-          if (sg.dest == kDestMerge) {
-            const float4 av = orow[4 * c16 + e];
-            val.x = fmaf(wa, av.x, val.x);
-            val.y = fmaf(wa, av.y, val.y);
-            val.z = fmaf(wa, av.z, val.z);
-            val.w = fmaf(wa, av.w, val.w);
+        for (int e = 0; e < 4; ++e)
+          *reinterpret_cast<float4 *>(slot + lane * kStageRow + 4 * e) =
+              make_float4(__uint_as_float(o[4 * e]) * wb, __uint_as_float(o[4 * e + 1]) * wb,
+                          __uint_as_float(o[4 * e + 2]) * wb, __uint_as_float(o[4 * e + 3]) * wb);
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int rr = 8 * k + (lane >> 2), cc = lane & 3;  // staging row, float4 column
+          float4 val = *reinterpret_cast<const float4 *>(slot + rr * kStageRow + 4 * cc);
+          const int rt = r0 + rr;  // tile row
+          const int pos_t = I * 16 + (rt & 15);
+          const float wa_t = __shfl_sync(0xffffffffu, wa, rr);
+          if (valid && pos_t < p.Lq) {
+            float *dst_row;
+            if (sg.dest == kDestScratch) {
+              const size_t slot_row = (static_cast<size_t>(cluster_index()) * 2 + rank) * 128 + rt;
+              dst_row = p.ws_out + slot_row * DV;
+            } else {
+              const size_t row_t = (static_cast<size_t>(b) * kH + (rt >> 4)) * p.Lq +
+                                   static_cast<size_t>(pos_t);
+              dst_row = p.out + row_t * DV;
+            }
+            float4 *dst = reinterpret_cast<float4 *>(dst_row + 32 * g + 16 * c16) + cc;
+            if (sg.dest == kDestMerge) {
+              const float4 av = *dst;
+              val.x = fmaf(wa_t, av.x, val.x);
+              val.y = fmaf(wa_t, av.y, val.y);
+              val.z = fmaf(wa_t, av.z, val.z);
+              val.w = fmaf(wa_t, av.w, val.w);
+            }
+            *dst = val;
           }
-          orow[4 * c16 + e] = val;
+        }
+        __syncwarp();
+      }
+    } else {
+      // This warpgroup's DV / 4 columns of the row, 16 at a time (every lane
+      // loads: tcgen05.ld is warp-wide; rows that do not exist store nothing).
+#pragma unroll 1
+      for (int c16 = 0; c16 < DV / 4 / 16; ++c16) {
+        uint32_t o[16];
+        tmem_ld16(tO + 16u * c16, o);
+        tmem_wait_ld16(o);
+        if (writes) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float4 val =
+                make_float4(__uint_as_float(o[4 * e]) * wb, __uint_as_float(o[4 * e + 1]) * wb,
+                            __uint_as_float(o[4 * e + 2]) * wb, __uint_as_float(o[4 * e + 3]) * wb);
+            if (sg.dest == kDestMerge) {
+              const float4 av = orow[4 * c16 + e];
+              val.x = fmaf(wa, av.x, val.x);
+              val.y = fmaf(wa, av.y, val.y);
+              val.z = fmaf(wa, av.z, val.z);
+              val.w = fmaf(wa, av.w, val.w);
+            }
+            orow[4 * c16 + e] = val;
+          }
         }
       }
     }
@@ -1116,6 +1178,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint8_t *v_s = k_s + kStages * kKSlotBytes;         // V ring
   Barriers *bars = reinterpret_cast<Barriers *>(v_s + kStages * v_slot_bytes<DV>());
   auto *xc = reinterpret_cast<Xchg *>(reinterpret_cast<uint8_t *>(bars) + sizeof(Barriers));
+  float *stage = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(bars) + kBarsXchgBytes);
   const int warp = threadIdx.x >> 5;
   const uint32_t rank = cluster_ctarank();
 
@@ -1185,7 +1248,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    softmax_role<MODE, DV>(bars, xc, tmem, p, rank, abort);
+    softmax_role<MODE, DV>(bars, xc, stage, tmem, p, rank, abort);
   }
   __syncwarp();
   // No CTA leaves while the other may still use its shared or tensor memory:
