@@ -51,15 +51,6 @@ static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
 enum Site : unsigned { kSiteFull = 20, kSiteEmpty = 21 };
 
-__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar,
-                                            int c0, int c1, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_"
-      "tx::bytes.L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1),
-      "l"(policy)
-      : "memory");
-}
 
 __global__ void __launch_bounds__(kThreads, 1)
     pair_bias_project_kernel(const __grid_constant__ CUtensorMap tm_pair,

@@ -136,6 +136,15 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   return p;
 }
 
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar,
+                                            int c0, int c1, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_"
+      "tx::bytes.L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1),
+      "l"(policy)
+      : "memory");
+}
 __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map,
                                             uint64_t *bar, int c0, int c1,
                                             int c2, uint64_t policy) {
@@ -270,8 +279,47 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
                    cluster_bar)
                : "memory");
 }
+// Arrive on an mbarrier of any CTA of the cluster with release semantics at
+// cluster scope: this thread's earlier writes (shared memory of either CTA
+// included) are visible to a thread that observes the phase with an acquire
+// at cluster scope.
+__device__ __forceinline__ void mbar_arrive_cluster_release(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
+                   cluster_bar)
+               : "memory");
+}
+// Store one float into shared memory of any CTA of the cluster.
+__device__ __forceinline__ void st_cluster_f32(uint32_t cluster_addr_, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(cluster_addr_), "f"(v) : "memory");
+}
+// mbar_wait with acquire at cluster scope, for phases whose arrivals
+// release data written by the other CTA of the cluster.  Bounded like
+// mbar_wait.
+__device__ __forceinline__ bool mbar_wait_acq_cluster(uint64_t *bar, uint32_t parity,
+                                                      volatile int *abort, unsigned *err,
+                                                      unsigned site) {
+  const uint32_t a = smem_u32(bar);
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(a), "r"(parity)
+        : "memory");
+    if (ok) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      *abort = 1;
+      if (err) atomicCAS(err, 0u, (site << 8) | kErrTimeout);
+      return false;
+    }
+  }
+}
 // tcgen05 with .cta_group::2: one warp of each CTA of the pair allocates
-// (and later frees) the same columns in both CTAs' tensor memory; one thread
+// (and later frees) the same columns in both CTAs' tensor memory; one elected lane
 // of the even CTA issues MMAs of M = 256 whose A rows 0..127 come from the
 // even CTA and rows 128..255 from the odd one (shared-memory descriptors and
 // tensor-memory addresses name the same offsets in both), whose B columns
@@ -292,45 +340,6 @@ __device__ __forceinline__ void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr),
                "r"(ncols)
                : "memory");
-}
-__device__ __forceinline__ void umma2_ss_lo(uint32_t d_tmem, uint32_t a_lo,
-                                            uint32_t b_lo, uint32_t hi,
-                                            uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
-      "mov.b64 da, {%1, %3};\n\t"
-      "mov.b64 db, {%2, %3};\n\t"
-      "setp.ne.b32 p, %5, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], da, db, %4, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_lo), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void umma2_ts_lo(uint32_t d_tmem, uint32_t a_tmem,
-                                            uint32_t b_lo, uint32_t hi,
-                                            uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
-      "mov.b64 db, {%2, %3};\n\t"
-      "setp.ne.b32 p, %5, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], db, %4, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// Arrive (once) on the mbarrier at the same offset in both CTAs of the pair
-// when every tcgen05 operation this thread issued so far has completed.
-__device__ __forceinline__ void umma2_commit_both(uint64_t *bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster."
-      "multicast::cluster.b64 [%0], %1;" ::"r"(smem_u32(bar)),
-      "h"(static_cast<uint16_t>(3))
-      : "memory");
-}
-// The same, on this CTA's barrier only.
-__device__ __forceinline__ void umma2_commit_self(uint64_t *bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 "
-      "[%0];" ::"r"(smem_u32(bar))
-      : "memory");
 }
 
 // Warp-wide forms of the MMA and commit issue: the whole warp, converged,
@@ -362,6 +371,9 @@ __device__ __forceinline__ void umma2_ts_w(uint32_t d_tmem, uint32_t a_tmem, uin
       "r"(a_tmem), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// Commits: arrive (once) when every tcgen05 operation the issuing lane
+// started so far has completed, on the barrier at the same offset in both
+// CTAs of the pair (_both), or on this CTA's only (_self, umma1_commit_w).
 __device__ __forceinline__ void umma2_commit_both_w(uint64_t *bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
@@ -426,37 +438,6 @@ __device__ __forceinline__ void tmem_dealloc1(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr),
                "r"(ncols)
                : "memory");
-}
-__device__ __forceinline__ void umma1_ss_lo(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi,
-                                            uint32_t b_lo, uint32_t b_hi, uint32_t idesc,
-                                            uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
-      "mov.b64 da, {%1, %2};\n\t"
-      "mov.b64 db, {%3, %4};\n\t"
-      "setp.ne.b32 p, %6, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void umma1_ts_lo(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
-                                            uint32_t b_hi, uint32_t idesc,
-                                            uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
-      "mov.b64 db, {%2, %3};\n\t"
-      "setp.ne.b32 p, %5, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// Arrive (once) on this CTA's mbarrier when every tcgen05 operation this
-// thread issued so far has completed.
-__device__ __forceinline__ void umma1_commit(uint64_t *bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-          smem_u32(bar))
-      : "memory");
 }
 
 // Tensor-memory loads/stores, 32 lanes x 32-bit, repeated along columns.
