@@ -279,45 +279,6 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
                    cluster_bar)
                : "memory");
 }
-// Arrive on an mbarrier of any CTA of the cluster with release semantics at
-// cluster scope: this thread's earlier writes (shared memory of either CTA
-// included) are visible to a thread that observes the phase with an acquire
-// at cluster scope.
-__device__ __forceinline__ void mbar_arrive_cluster_release(uint32_t cluster_bar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
-                   cluster_bar)
-               : "memory");
-}
-// Store one float into shared memory of any CTA of the cluster.
-__device__ __forceinline__ void st_cluster_f32(uint32_t cluster_addr_, float v) {
-  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(cluster_addr_), "f"(v) : "memory");
-}
-// mbar_wait with acquire at cluster scope, for phases whose arrivals
-// release data written by the other CTA of the cluster.  Bounded like
-// mbar_wait.
-__device__ __forceinline__ bool mbar_wait_acq_cluster(uint64_t *bar, uint32_t parity,
-                                                      volatile int *abort, unsigned *err,
-                                                      unsigned site) {
-  const uint32_t a = smem_u32(bar);
-  const uint64_t t0 = globaltimer_ns();
-  while (true) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(a), "r"(parity)
-        : "memory");
-    if (ok) return true;
-    if (*abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-      *abort = 1;
-      if (err) atomicCAS(err, 0u, (site << 8) | kErrTimeout);
-      return false;
-    }
-  }
-}
 // tcgen05 with .cta_group::2: one warp of each CTA of the pair allocates
 // (and later frees) the same columns in both CTAs' tensor memory; one elected lane
 // of the even CTA issues MMAs of M = 256 whose A rows 0..127 come from the
