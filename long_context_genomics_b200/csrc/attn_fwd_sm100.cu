@@ -105,6 +105,15 @@ template <int DV> struct Tmem {
   static constexpr uint32_t kColP = 256;
   static constexpr uint32_t kColO = 256 + 64 * kNP;
 };
+// Static cap at value width 128 ("P in place"): three 128-column step
+// buffers b = t % 3 at [128 b, 128 b + 128), the softmax writing each 64-key
+// half's P (bf16 pairs, 32 columns) over the first columns of that half's
+// logits, and O at [384, 512).  S of tile t waits for PV of tile t - 3 (the
+// buffer's last reader) instead of for the softmax, so the logits of a warp
+// group's next tile are usually ready before the group asks for them.
+constexpr uint32_t kIPBufs = 3;
+constexpr uint32_t kIPColO = 384;
+template <int MODE, int DV> constexpr bool p_in_place() { return MODE == 0 && DV == 128; }
 static_assert(Tmem<128>::kColO + 128 <= 512 && Tmem<192>::kColO + 192 <= 512,
               "tensor memory budget");
 constexpr uint32_t kTmemCols = 512;
@@ -159,8 +168,8 @@ struct __align__(8) Barriers {
   uint64_t q_full, q_empty;
   uint64_t k_full[kStages], k_empty[kStages];
   uint64_t v_full[kStages], v_empty[kStages];
-  uint64_t s_full[2], s_free[2];
-  uint64_t p_full[2], pv_done[2];  // [Tmem<DV>::kNP] in use
+  uint64_t s_full[3], s_free[2];
+  uint64_t p_full[3], pv_done[3];  // three in use with P in place, else [Tmem<DV>::kNP]
   uint64_t o_full;
   uint64_t xm, xd;  // row-max / row-sum exchange between the warpgroups
   uint64_t drain;   // both issuing threads' MMAs have completed
@@ -348,6 +357,20 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem,
   }
 }
 
+// The same for P in place (value width 128): keys 16 kk .. 16 kk + 15 are
+// in the half kk / 4 of the step buffer, at its column 64 (kk / 4) + 8 (kk % 4).
+__device__ __forceinline__ void issue_pv_in_place(uint32_t d_tmem, uint32_t buf_tmem,
+                                                  uint32_t v_addr, bool accumulate) {
+  using VL = VLayout<128>;
+  const uint32_t v_lo = desc_sw128_lo(v_addr, VL::kAtomBytes);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    umma2_ts_w(d_tmem, buf_tmem + 64 * (kk >> 2) + 8 * (kk & 3),
+               v_lo + ((kk * VL::kKStepBytes) >> 4), VL::kDescHi, idesc_pv<128>(),
+               (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
 // Bounded wait used while draining: ignores the abort flag, records nothing.
 __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
   const uint32_t a = smem_u32(bar);
@@ -495,9 +518,11 @@ __device__ __forceinline__ void relay_v(Barriers *bars, const Params &p, volatil
 
 // S = Q K^T for every key tile, into S buffer (use count & 1), once the
 // softmax has read that buffer's previous logits (s_free).
+template <bool kIP>
 __device__ __forceinline__ void issuer_s(uint8_t *q_s, uint8_t *k_s, Barriers *bars,
                                          uint32_t tmem, const Params &p,
                                          volatile int *abort) {
+  constexpr uint32_t kBufs = kIP ? kIPBufs : 2;
   const uint32_t q_addr = smem_u32(q_s), k_addr = smem_u32(k_s);
   uint32_t qc = 0, kl = 0, su = 0;
   bool ok = true;
@@ -516,9 +541,12 @@ __device__ __forceinline__ void issuer_s(uint8_t *q_s, uint8_t *k_s, Barriers *b
         ++kl;
         if (!ok) break;
       }
-      const uint32_t sb = su & 1u, sn = su >> 1;
+      const uint32_t sb = su % kBufs, sn = su / kBufs;
       if (sn > 0) {
-        ok = mbar_wait_warp(&bars->s_free[sb], (sn - 1) & 1u, abort, p.err, kSiteIssueSFree);
+        // The buffer's previous logits are no longer needed: read by the
+        // softmax (s_free), or, with P in place, read by PV as P (pv_done).
+        ok = mbar_wait_warp(kIP ? &bars->pv_done[sb] : &bars->s_free[sb], (sn - 1) & 1u, abort,
+                            p.err, kSiteIssueSFree);
         if (!ok) break;
       }
       tc_fence_after();
@@ -535,10 +563,11 @@ __device__ __forceinline__ void issuer_s(uint8_t *q_s, uint8_t *k_s, Barriers *b
 }
 
 // O += P V for every key tile, once the softmax has written P (p_full).
-template <int DV>
+template <int DV, bool kIP>
 __device__ __forceinline__ void issuer_pv(uint8_t *v_s, Barriers *bars, uint32_t tmem,
                                           const Params &p, volatile int *abort) {
   using T = Tmem<DV>;
+  constexpr uint32_t kBufs = kIP ? kIPBufs : T::kNP;
   const uint32_t v_addr = smem_u32(v_s);
   uint32_t vl = 0, pu = 0;
   bool ok = true;
@@ -554,13 +583,15 @@ __device__ __forceinline__ void issuer_pv(uint8_t *v_s, Barriers *bars, uint32_t
         ++vl;
         if (!ok) break;
       }
-      const uint32_t pb = pu % T::kNP, pn = pu / T::kNP;
+      const uint32_t pb = pu % kBufs, pn = pu / kBufs;
       ok = mbar_wait_warp(&bars->p_full[pb], pn & 1u, abort, p.err, kSiteIssueP);
       if (!ok) break;
       tc_fence_after();
-      issue_pv<DV>(tmem + T::kColO, tmem + T::kColP + 64u * pb,
-                   v_addr + slot * v_slot_bytes<DV>() + (i & 1) * VLayout<DV>::kTileBytes,
-                   i > 0);
+      const uint32_t va = v_addr + slot * v_slot_bytes<DV>() + (i & 1) * VLayout<DV>::kTileBytes;
+      if constexpr (kIP)
+        issue_pv_in_place(tmem + kIPColO, tmem + 128u * pb, va, i > 0);
+      else
+        issue_pv<DV>(tmem + T::kColO, tmem + T::kColP + 64u * pb, va, i > 0);
       umma2_commit_both_w(&bars->pv_done[pb]);
       if (j + 1 == sg.ke) umma2_commit_both_w(&bars->o_full);
       if ((i & 1) == 1 || j + 1 == sg.ke) umma2_commit_both_w(&bars->v_empty[slot]);
@@ -732,60 +763,49 @@ __device__ __forceinline__ bool store_p(Barriers *bars, uint32_t tmem, int g,
 // One 64-key half tile of a grouped static segment (see below): tS and tP
 // address this warp's S and P columns, bc holds the four bias cells.
 template <bool kMask>
-__device__ __forceinline__ bool tile_grouped(uint32_t tS, uint32_t tP, const float (&bc)[4],
-                                             float m, const StaticK &k, int col0, int nvalid,
-                                             uint32_t n, int q, uint32_t sf_q, Barriers *bars,
-                                             uint32_t rank, const Params &p,
-                                             volatile int *abort, float2 &acc) {
+__device__ __forceinline__ void tile_grouped(uint32_t tS, const float (&bc)[4], float m,
+                                             const StaticK &k, int col0, int nvalid,
+                                             float2 &acc) {
+  // P piece c (8 columns) goes over columns 8 c .. 8 c + 7 of this half's
+  // logits, which pieces 0 .. c have already brought into registers; piece
+  // c + 1 (columns 16 c + 16 ..) is being loaded meanwhile.
   uint32_t sa[16], sb[16], pk[8];
   tmem_ld16(tS, sa);
   tmem_wait_ld16(sa);
   tmem_ld16(tS + 16u, sb);
   chunk_static<kMask, 16>(sa, bc[0] * m, bc[0] * m, k, col0, nvalid, acc, pk);
-  if (n > 0) {  // the PV that last read P buffer q
-    const bool ok = mbar_wait(&bars->pv_done[q], (n - 1) & 1u, abort, p.err, kSiteSoftPV);
-    if (!__all_sync(0xffffffffu, ok)) {
-      tmem_wait_ld16(sb);
-      return false;
-    }
-  }
-  tc_fence_after();
-  tmem_st8(tP, pk);
+  tmem_st8(tS, pk);
   tmem_wait_ld16(sb);
   tmem_ld16(tS + 32u, sa);
   chunk_static<kMask, 16>(sb, bc[1] * m, bc[1] * m, k, col0 + 16, nvalid, acc, pk);
-  tmem_st8(tP + 8u, pk);
+  tmem_st8(tS + 8u, pk);
   tmem_wait_ld16(sa);
   tmem_ld16(tS + 48u, sb);
   chunk_static<kMask, 16>(sa, bc[2] * m, bc[2] * m, k, col0 + 32, nvalid, acc, pk);
-  tmem_st8(tP + 16u, pk);
+  tmem_st8(tS + 16u, pk);
   tmem_wait_ld16(sb);
-  tc_fence_before();
-  warp_arrive_leader(&bars->s_free[q], sf_q, rank);  // S fully read
   chunk_static<kMask, 16>(sb, bc[3] * m, bc[3] * m, k, col0 + 48, nvalid, acc, pk);
-  tmem_st8(tP + 24u, pk);
-  return true;
+  tmem_st8(tS + 24u, pk);
 }
 
-// Static-shift segment with alternating groups (value width 128): the warps
-// split into two groups that take alternate key tiles, group q = warpgroups
-// 2q and 2q + 1 taking the tiles in S buffer q (64 keys each per tile) and
-// writing P buffer q.  One group's waits (for its logits, for the previous
-// PV of its P buffer, for its tensor-memory loads and stores) are covered by
-// the other group's arithmetic, so the special-function unit stays busy.
-// A group only ever waits on its own S and P buffers' barriers, in order.
+// Static-shift segment with alternating groups (value width 128, P in
+// place): the warps split into two groups that take alternate key tiles,
+// group q = warpgroups 2q and 2q + 1, warpgroup hk of it the 64 keys
+// [64 hk, 64 hk + 64) of the tile; tile t's logits are in step buffer t % 3
+// and its P goes over them.  One group's waits (for its logits, for its
+// tensor-memory loads and stores) are covered by the other group's
+// arithmetic, so the special-function unit stays busy.  A group waits for
+// the s_full phases of its own tiles in order; the phase of the buffer's
+// previous tile (the other group's) has completed by then, because the
+// logits of the group's own previous tile, issued later, have.
 template <int DV>
 __device__ __forceinline__ bool segment_static_grouped(const Segment &sg, const float *brow,
                                                        uint32_t tmem, uint32_t lane_base, int g,
                                                        const Params &p, Barriers *bars,
-                                                       uint32_t rank,
-                                                       const uint32_t (&sf_remote)[2],
-                                                       const uint32_t (&pf_remote)[2],
-                                                       SoftCounters &c, volatile int *abort,
-                                                       float &d) {
-  static_assert(Tmem<DV>::kNP == 2, "one P buffer per group");
-  using T = Tmem<DV>;
-  const int q = g >> 1, hk = g & 1;  // group (S and P buffer), key half
+                                                       uint32_t rank, SoftCounters &c,
+                                                       volatile int *abort, float &d) {
+  static_assert(DV == 128, "P in place: value width 128");
+  const int q = g >> 1, hk = g & 1;  // group, key half
   StaticK k;
   constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
   k.sc = make_float2(p.qk_scale, p.qk_scale);
@@ -793,38 +813,31 @@ __device__ __forceinline__ bool segment_static_grouped(const Segment &sg, const 
   k.nsh = make_float2(-p.shift, -p.shift);
   k.km = make_float2(kShift - p.shift, kShift - p.shift);
   float2 acc = make_float2(0.f, 0.f);
-  // This group's barriers in the even CTA, as scalars (an array indexed by q
-  // would live in local memory).
-  const uint32_t sf_q = q ? sf_remote[1] : sf_remote[0];
-  const uint32_t pf_q = q ? pf_remote[1] : pf_remote[0];
-  // Key tile j of the segment is global tile c.su + (j - kb): buffer (that) & 1.
+  const uint32_t pf0 = cluster_addr(&bars->p_full[0], 0);  // the even CTA's p_full
+  // Key tile j of the segment is global tile c.su + (j - kb); the group takes
+  // the tiles of its parity.
   const int j0 = sg.kb + static_cast<int>((static_cast<uint32_t>(q) - c.su) & 1u);
   float bc[4] = {0.f, 0.f, 0.f, 0.f};
   if (j0 < sg.ke) load_bias4(brow, j0, hk, p.P, bc);
   for (int j = j0; j < sg.ke; j += 2) {
-    const uint32_t n = (c.su + static_cast<uint32_t>(j - sg.kb)) >> 1;  // use of buffer q
+    const uint32_t tile = c.su + static_cast<uint32_t>(j - sg.kb);
+    const uint32_t b = tile % kIPBufs, u = tile / kIPBufs;
     const int nvalid = (j + 1 == p.n_kt) ? p.last_valid : kKeys;
-    bool ok = mbar_wait(&bars->s_full[q], n & 1u, abort, p.err, kSiteSoftS);
+    bool ok = mbar_wait(&bars->s_full[b], u & 1u, abort, p.err, kSiteSoftS);
     if (!__all_sync(0xffffffffu, ok)) return false;
     tc_fence_after();
-    const uint32_t tS = tmem + 128u * q + 64u * hk + lane_base;
-    const uint32_t tP = tmem + T::kColP + 64u * q + 32u * hk + lane_base;
+    const uint32_t tS = tmem + 128u * b + 64u * hk + lane_base;
     const float m = p.bias_mul;
     // Four pieces of 16 keys (one bias cell each), the tensor-memory load of
-    // the next piece in flight while this one is computed.  The P buffer is
-    // written once the PV that last read it has finished; the S buffer is
-    // released once its last piece has arrived in registers.
+    // the next piece in flight while this one is computed.
     if (nvalid == kKeys)
-      ok = tile_grouped<false>(tS, tP, bc, m, k, 64 * hk, nvalid, n, q, sf_q, bars, rank, p,
-                               abort, acc);
+      tile_grouped<false>(tS, bc, m, k, 64 * hk, nvalid, acc);
     else
-      ok = tile_grouped<true>(tS, tP, bc, m, k, 64 * hk, nvalid, n, q, sf_q, bars, rank, p,
-                              abort, acc);
-    if (!ok) return false;
+      tile_grouped<true>(tS, bc, m, k, 64 * hk, nvalid, acc);
     if (j + 2 < sg.ke) load_bias4(brow, j + 2, hk, p.P, bc);
     tmem_wait_st();
     tc_fence_before();
-    warp_arrive_leader(&bars->p_full[q], pf_q, rank);
+    warp_arrive_leader(&bars->p_full[b], pf0 + 8u * b, rank);
   }
   const uint32_t tiles = static_cast<uint32_t>(sg.ke - sg.kb);
   c.su += tiles;
@@ -1021,8 +1034,7 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc, float *st
     float m = kStatic ? p.shift : -INFINITY;  // log2 units
     float d = 0.f;
     if constexpr (kStatic && DV == 128) {
-      ok = segment_static_grouped<DV>(sg, brow, tmem, lane_base, g, p, bars, rank, sf_remote,
-                                      pf_remote, c, abort, d);
+      ok = segment_static_grouped<DV>(sg, brow, tmem, lane_base, g, p, bars, rank, c, abort, d);
     } else if constexpr (kStatic) {
       ok = segment_static<MODE, DV>(sg, brow, tmem, lane_base, g, p, bars, rank, sf_remote,
                                     pf_remote, c, abort, d);
@@ -1200,9 +1212,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // otherwise every softmax warp takes part in every key tile.
     constexpr uint32_t kSPArrivals =
         (MODE == kStaticCap && DV == 128) ? kPairSoftWarps / 2 : kPairSoftWarps;
-    for (int u = 0; u < 2; ++u) {
+    for (int u = 0; u < 3; ++u) {
       mbar_init(&bars->s_full[u], 1);
-      mbar_init(&bars->s_free[u], kSPArrivals);
+      if (u < 2) mbar_init(&bars->s_free[u], kSPArrivals);
       mbar_init(&bars->p_full[u], kSPArrivals);
       mbar_init(&bars->pv_done[u], 1);
     }
@@ -1233,9 +1245,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (warp >= kWarpLoadQK) {
     regs_dec<kRegsLow>();
     if (rank == 0 && warp == kWarpIssueS) {
-      issuer_s(q_s, k_s, bars, tmem, p, abort);  // the whole warp: elected issue
+      issuer_s<p_in_place<MODE, DV>()>(q_s, k_s, bars, tmem, p, abort);  // the whole warp
     } else if (rank == 0 && warp == kWarpIssuePV) {
-      issuer_pv<DV>(v_s, bars, tmem, p, abort);
+      issuer_pv<DV, p_in_place<MODE, DV>()>(v_s, bars, tmem, p, abort);
     } else if (lane_id() == 0) {
       if (warp == kWarpLoadQK) {
         producer_qk(&tm_q, &tm_k, q_s, k_s, bars, p, rank, abort);
