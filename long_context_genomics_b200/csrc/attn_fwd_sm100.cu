@@ -1242,7 +1242,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t tmem = bars->tmem_base;
   volatile int *abort = &bars->abort;
 
-  if (warp >= kWarpLoadQK) {
+  if (warp >= kSoftWarps) {  // the four role warps
     regs_dec<kRegsLow>();
     if (rank == 0 && warp == kWarpIssueS) {
       issuer_s<p_in_place<MODE, DV>()>(q_s, k_s, bars, tmem, p, abort);  // the whole warp
