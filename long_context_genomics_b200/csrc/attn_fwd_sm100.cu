@@ -65,9 +65,9 @@ constexpr int kQTileBytes = 128 * kD * 2;     // this CTA's query tile (bf16)
 constexpr int kQHalfBytes = kQTileBytes / 2;  // one 64-wide (128-byte) half
 constexpr int kKTileBytes = 64 * kD * 2;      // this CTA's 64 keys of a K tile
 constexpr int kKHalfBytes = kKTileBytes / 2;  // one 64-wide half of them
-// Ring slots hold two consecutive key tiles, so each issuing thread waits
-// for data and releases it once per two tiles (each mbarrier operation costs
-// the issuing thread about 180 cycles, measured).
+// K ring slots hold two consecutive key tiles, so the S issuer waits for
+// data and releases it once per two tiles (each mbarrier operation costs the
+// issuing thread about 180 cycles, measured).
 constexpr int kStages = 2;
 constexpr int kTilesPerSlot = 2;
 
@@ -93,8 +93,15 @@ template <> struct VLayout<192> {
   static constexpr uint32_t kKStepBytes = 16 * 64;      // 16 keys x 64 B
 };
 constexpr int kKSlotBytes = kTilesPerSlot * kKTileBytes;
+// The V ring: value width 128 keeps three one-tile slots (48 KB instead of
+// 64 KB, which leaves room for the epilogue's staging of out); value width
+// 192 two two-tile slots.  V tiles are needed a few tiles after their K tile
+// (PV trails S), so the shallower ring still covers the load latency.
+template <int DV> constexpr int v_stages() { return DV == 128 ? 3 : 2; }
+template <int DV> constexpr int v_tiles_per_slot() { return DV == 128 ? 1 : 2; }
+constexpr int kVStagesMax = 3;
 template <int DV> constexpr int v_slot_bytes() {
-  return kTilesPerSlot * VLayout<DV>::kTileBytes;
+  return v_tiles_per_slot<DV>() * VLayout<DV>::kTileBytes;
 }
 
 // Tensor-memory columns: S buffer u at 128 u; P buffer p (bf16 pairs, 64
@@ -167,7 +174,7 @@ enum Site : unsigned {
 struct __align__(8) Barriers {
   uint64_t q_full, q_empty;
   uint64_t k_full[kStages], k_empty[kStages];
-  uint64_t v_full[kStages], v_empty[kStages];
+  uint64_t v_full[kVStagesMax], v_empty[kVStagesMax];  // [v_stages<DV>()] in use
   uint64_t s_full[3], s_free[2];
   uint64_t p_full[3], pv_done[3];  // three in use with P in place, else [Tmem<DV>::kNP]
   uint64_t o_full;
@@ -184,21 +191,27 @@ struct Xchg {
   float dpart[kWG][128];     // [warpgroup][row]
 };
 
-// Epilogue staging (value width 128): per softmax warp, 32 rows x 16 fp32
-// columns, rows padded to 20 floats (80 bytes) so that both the row-wise
-// writes and the column-wise reads of a shared-memory phase hit 8 distinct
-// 16-byte bank groups (one 2-way pair on the reads).  With it the output is
-// stored 64 contiguous bytes per row per 4 lanes instead of 16 bytes per lane
-// at a 512-byte stride.  Value width 192 has no room for it and stores
-// directly.
+// Epilogue staging (value width 128): 4 KB per softmax warp, 1024-byte
+// aligned.  A segment that writes out directly stages the warp's 32 rows x
+// 32 columns of it there in the TMA 128-byte swizzle (row l at 128 l,
+// 16-byte chunk c at (c ^ (l & 7)) 16: every 8 lanes of a 16-byte store hit
+// all 32 banks) and one lane stores the box with a bulk tensor copy, which
+// runs on while the warp goes on to the next segment.  The other segments
+// (merge with a first piece, scratch) stage 16 columns at a time in rows
+// padded to 20 floats and store them with plain 16-byte stores, 64
+// contiguous bytes per row per 4 lanes.  Value width 192 has no room for
+// staging and stores directly.
 constexpr int kStageRow = 20;
+constexpr int kStageWarpFloats = 1024;  // 4 KB
 template <int DV> constexpr size_t stage_bytes() {
-  return DV == 128 ? static_cast<size_t>(kSoftThreads / 32) * 32 * kStageRow * 4 : 0;
+  return DV == 128 ? static_cast<size_t>(kSoftThreads / 32) * kStageWarpFloats * 4 : 0;
 }
+static_assert(32 * kStageRow <= kStageWarpFloats, "padded staging fits a warp's slot");
 constexpr size_t kBarsXchgBytes = (sizeof(Barriers) + sizeof(Xchg) + 15) & ~static_cast<size_t>(15);
 template <int DV> constexpr size_t smem_bytes() {
   return 1024 + static_cast<size_t>(kQTileBytes) + kStages * static_cast<size_t>(kKSlotBytes) +
-         kStages * static_cast<size_t>(v_slot_bytes<DV>()) + kBarsXchgBytes + stage_bytes<DV>();
+         v_stages<DV>() * static_cast<size_t>(v_slot_bytes<DV>()) + stage_bytes<DV>() +
+         kBarsXchgBytes;
 }
 static_assert(smem_bytes<128>() <= 227 * 1024 && smem_bytes<192>() <= 227 * 1024,
               "shared memory budget");
@@ -439,6 +452,7 @@ __device__ __forceinline__ void producer_v(const CUtensorMap *tm_v, uint8_t *v_s
                                            Barriers *bars, const Params &p, uint32_t rank,
                                            volatile int *abort) {
   using VL = VLayout<DV>;
+  constexpr int kVS = v_stages<DV>(), kVT = v_tiles_per_slot<DV>();
   const uint64_t pol_v = l2_policy_evict_last();
   uint32_t vl = 0;
   bool ok = true;
@@ -446,11 +460,11 @@ __device__ __forceinline__ void producer_v(const CUtensorMap *tm_v, uint8_t *v_s
   Segment sg;
   while (ok && next_segment(p, cu, sg)) {
     const int b = sg.item / p.pairs;
-    for (int j0 = sg.kb; j0 < sg.ke; j0 += kTilesPerSlot) {
-      const uint32_t slot = vl % kStages, ph = (vl / kStages) & 1u;
+    for (int j0 = sg.kb; j0 < sg.ke; j0 += kVT) {
+      const uint32_t slot = vl % kVS, ph = (vl / kVS) & 1u;
       ok = mbar_wait(&bars->v_empty[slot], ph ^ 1u, abort, p.err, kSiteProdV);
       if (!ok) break;
-      const int nt = sg.ke - j0 < kTilesPerSlot ? sg.ke - j0 : kTilesPerSlot;
+      const int nt = sg.ke - j0 < kVT ? sg.ke - j0 : kVT;
       mbar_arrive_expect_tx(&bars->v_full[slot], static_cast<uint32_t>(nt) * VL::kTileBytes);
       for (int t = 0; t < nt; ++t) {
         // Keys [128 j, +128), value columns [DV/2 rank, +DV/2).
@@ -464,8 +478,8 @@ __device__ __forceinline__ void producer_v(const CUtensorMap *tm_v, uint8_t *v_s
       ++vl;
     }
   }
-  for (uint32_t i = vl > kStages ? vl - kStages : 0; i < vl; ++i)
-    drain_wait(&bars->v_full[i % kStages], (i / kStages) & 1u);
+  for (uint32_t i = vl > kVS ? vl - kVS : 0; i < vl; ++i)
+    drain_wait(&bars->v_full[i % kVS], (i / kVS) & 1u);
 }
 
 // --------------------------------------------------------------------------
@@ -493,15 +507,17 @@ __device__ __forceinline__ void relay_qk(Barriers *bars, const Params &p, volati
   }
 }
 
+template <int DV>
 __device__ __forceinline__ void relay_v(Barriers *bars, const Params &p, volatile int *abort) {
+  constexpr int kVS = v_stages<DV>(), kVT = v_tiles_per_slot<DV>();
   uint32_t vl = 0;
   bool ok = true;
   Cursor cu = cursor_begin(p);
   Segment sg;
   while (ok && next_segment(p, cu, sg)) {
-    for (int j0 = sg.kb; j0 < sg.ke; j0 += kTilesPerSlot) {
-      const uint32_t slot = vl % kStages;
-      ok = mbar_wait(&bars->v_full[slot], (vl / kStages) & 1u, abort, p.err, kSiteRelay);
+    for (int j0 = sg.kb; j0 < sg.ke; j0 += kVT) {
+      const uint32_t slot = vl % kVS;
+      ok = mbar_wait(&bars->v_full[slot], (vl / kVS) & 1u, abort, p.err, kSiteRelay);
       if (!ok) break;
       ++vl;
       mbar_arrive_cluster(cluster_addr(&bars->v_full[slot], 0));
@@ -568,6 +584,7 @@ __device__ __forceinline__ void issuer_pv(uint8_t *v_s, Barriers *bars, uint32_t
                                           const Params &p, volatile int *abort) {
   using T = Tmem<DV>;
   constexpr uint32_t kBufs = kIP ? kIPBufs : T::kNP;
+  constexpr int kVS = v_stages<DV>(), kVT = v_tiles_per_slot<DV>();
   const uint32_t v_addr = smem_u32(v_s);
   uint32_t vl = 0, pu = 0;
   bool ok = true;
@@ -577,9 +594,9 @@ __device__ __forceinline__ void issuer_pv(uint8_t *v_s, Barriers *bars, uint32_t
     uint32_t slot = 0;
     for (int j = sg.kb; j < sg.ke; ++j) {
       const int i = j - sg.kb;
-      if ((i & 1) == 0) {
-        slot = vl % kStages;
-        ok = mbar_wait_warp(&bars->v_full[slot], (vl / kStages) & 1u, abort, p.err, kSiteIssueV);
+      if (i % kVT == 0) {
+        slot = vl % kVS;
+        ok = mbar_wait_warp(&bars->v_full[slot], (vl / kVS) & 1u, abort, p.err, kSiteIssueV);
         ++vl;
         if (!ok) break;
       }
@@ -587,14 +604,15 @@ __device__ __forceinline__ void issuer_pv(uint8_t *v_s, Barriers *bars, uint32_t
       ok = mbar_wait_warp(&bars->p_full[pb], pn & 1u, abort, p.err, kSiteIssueP);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t va = v_addr + slot * v_slot_bytes<DV>() + (i & 1) * VLayout<DV>::kTileBytes;
+      const uint32_t va =
+          v_addr + slot * v_slot_bytes<DV>() + (i % kVT) * VLayout<DV>::kTileBytes;
       if constexpr (kIP)
         issue_pv_in_place(tmem + kIPColO, tmem + 128u * pb, va, i > 0);
       else
         issue_pv<DV>(tmem + T::kColO, tmem + T::kColP + 64u * pb, va, i > 0);
       umma2_commit_both_w(&bars->pv_done[pb]);
       if (j + 1 == sg.ke) umma2_commit_both_w(&bars->o_full);
-      if ((i & 1) == 1 || j + 1 == sg.ke) umma2_commit_both_w(&bars->v_empty[slot]);
+      if (i % kVT == kVT - 1 || j + 1 == sg.ke) umma2_commit_both_w(&bars->v_empty[slot]);
       ++pu;
     }
   }
@@ -1007,8 +1025,8 @@ __device__ __forceinline__ bool segment_online(const Segment &sg, const float *b
 
 template <int MODE, int DV>
 __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc, float *stage, uint32_t tmem,
-                                             const Params &p, uint32_t rank,
-                                             volatile int *abort) {
+                                             const CUtensorMap *tm_o, const Params &p,
+                                             uint32_t rank, volatile int *abort) {
   using T = Tmem<DV>;
   const int g = threadIdx.x >> 7;         // warpgroup
   const int r = threadIdx.x & 127;        // tile row == tensor-memory lane
@@ -1097,52 +1115,83 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc, float *st
       lse_w = M + lg2_approx(ea + eb) * kLn2;
     }
     if constexpr (DV == 128) {
-      // This warpgroup's 32 columns of its warp's 32 rows, 16 columns at a
-      // time: scaled into the warp's staging rows, then stored by groups of
-      // four lanes, one 64-byte row segment each.
       const int lane = static_cast<int>(lane_id());
-      float *slot = stage + (threadIdx.x >> 5) * (32 * kStageRow);
+      float *slot = stage + (threadIdx.x >> 5) * kStageWarpFloats;
       const int r0 = r - lane;  // the warp's first tile row
-#pragma unroll 1
-      for (int c16 = 0; c16 < 2; ++c16) {
-        uint32_t o[16];
-        tmem_ld16(tO + 16u * c16, o);
-        tmem_wait_ld16(o);
+      // The bulk store of this warp's previous segment has read the slot.
+      if (lane == 0) bulk_wait_read_all();
+      __syncwarp();
+      if (sg.dest == kDestOut) {
+        // This warpgroup's 32 columns of the warp's 32 rows (heads 2 (warp
+        // % 4) and + 1, positions 16 I .. 16 I + 15): scaled into the slot
+        // in the 128-byte swizzle, then one bulk tensor store.  Rows past Lq
+        // lie outside the tensor and are not written.
+        if (valid) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          *reinterpret_cast<float4 *>(slot + lane * kStageRow + 4 * e) =
-              make_float4(__uint_as_float(o[4 * e]) * wb, __uint_as_float(o[4 * e + 1]) * wb,
-                          __uint_as_float(o[4 * e + 2]) * wb, __uint_as_float(o[4 * e + 3]) * wb);
-        __syncwarp();
+          for (int c16 = 0; c16 < 2; ++c16) {
+            uint32_t o[16];
+            tmem_ld16(tO + 16u * c16, o);
+            tmem_wait_ld16(o);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int rr = 8 * k + (lane >> 2), cc = lane & 3;  // staging row, float4 column
-          float4 val = *reinterpret_cast<const float4 *>(slot + rr * kStageRow + 4 * cc);
-          const int rt = r0 + rr;  // tile row
-          const int pos_t = I * 16 + (rt & 15);
-          const float wa_t = __shfl_sync(0xffffffffu, wa, rr);
-          if (valid && pos_t < p.Lq) {
-            float *dst_row;
-            if (sg.dest == kDestScratch) {
-              const size_t slot_row = (static_cast<size_t>(cluster_index()) * 2 + rank) * 128 + rt;
-              dst_row = p.ws_out + slot_row * DV;
-            } else {
-              const size_t row_t = (static_cast<size_t>(b) * kH + (rt >> 4)) * p.Lq +
-                                   static_cast<size_t>(pos_t);
-              dst_row = p.out + row_t * DV;
+            for (int e = 0; e < 4; ++e) {
+              const int chunk = (4 * c16 + e) ^ (lane & 7);
+              *reinterpret_cast<float4 *>(slot + 32 * lane + 4 * chunk) = make_float4(
+                  __uint_as_float(o[4 * e]) * wb, __uint_as_float(o[4 * e + 1]) * wb,
+                  __uint_as_float(o[4 * e + 2]) * wb, __uint_as_float(o[4 * e + 3]) * wb);
             }
-            float4 *dst = reinterpret_cast<float4 *>(dst_row + 32 * g + 16 * c16) + cc;
-            if (sg.dest == kDestMerge) {
-              const float4 av = *dst;
-              val.x = fmaf(wa_t, av.x, val.x);
-              val.y = fmaf(wa_t, av.y, val.y);
-              val.z = fmaf(wa_t, av.z, val.z);
-              val.w = fmaf(wa_t, av.w, val.w);
-            }
-            *dst = val;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_4d(tm_o, slot, 32 * g, I * 16, 2 * ((threadIdx.x >> 5) & 3), b);
+            bulk_commit_group();
           }
         }
-        __syncwarp();
+      } else {
+        // This warpgroup's 32 columns of its warp's 32 rows, 16 columns at a
+        // time: scaled into the warp's staging rows, then stored by groups of
+        // four lanes, one 64-byte row segment each.
+#pragma unroll 1
+        for (int c16 = 0; c16 < 2; ++c16) {
+          uint32_t o[16];
+          tmem_ld16(tO + 16u * c16, o);
+          tmem_wait_ld16(o);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            *reinterpret_cast<float4 *>(slot + lane * kStageRow + 4 * e) =
+                make_float4(__uint_as_float(o[4 * e]) * wb, __uint_as_float(o[4 * e + 1]) * wb,
+                            __uint_as_float(o[4 * e + 2]) * wb, __uint_as_float(o[4 * e + 3]) * wb);
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int rr = 8 * k + (lane >> 2), cc = lane & 3;  // staging row, float4 column
+            float4 val = *reinterpret_cast<const float4 *>(slot + rr * kStageRow + 4 * cc);
+            const int rt = r0 + rr;  // tile row
+            const int pos_t = I * 16 + (rt & 15);
+            const float wa_t = __shfl_sync(0xffffffffu, wa, rr);
+            if (valid && pos_t < p.Lq) {
+              float *dst_row;
+              if (sg.dest == kDestScratch) {
+                const size_t slot_row = (static_cast<size_t>(cluster_index()) * 2 + rank) * 128 + rt;
+                dst_row = p.ws_out + slot_row * DV;
+              } else {
+                const size_t row_t = (static_cast<size_t>(b) * kH + (rt >> 4)) * p.Lq +
+                                     static_cast<size_t>(pos_t);
+                dst_row = p.out + row_t * DV;
+              }
+              float4 *dst = reinterpret_cast<float4 *>(dst_row + 32 * g + 16 * c16) + cc;
+              if (sg.dest == kDestMerge) {
+                const float4 av = *dst;
+                val.x = fmaf(wa_t, av.x, val.x);
+                val.y = fmaf(wa_t, av.y, val.y);
+                val.z = fmaf(wa_t, av.z, val.z);
+                val.w = fmaf(wa_t, av.w, val.w);
+              }
+              *dst = val;
+            }
+          }
+          __syncwarp();
+        }
       }
     } else {
       // This warpgroup's DV / 4 columns of the row, 16 at a time (every lane
@@ -1175,6 +1224,11 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc, float *st
     }
     tc_fence_before();
   }
+  if constexpr (DV == 128) {
+    // Every bulk store this warp started completes before the CTA exits.
+    if (lane_id() == 0) bulk_wait_all();
+    __syncwarp();
+  }
 }
 
 // --------------------------------------------------------------------------
@@ -1182,15 +1236,17 @@ template <int MODE, int DV>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ Params p) {
+                    const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t *q_s = smem_raw + pad;                      // this CTA's query tile
   uint8_t *k_s = q_s + kQTileBytes;                   // K ring
   uint8_t *v_s = k_s + kStages * kKSlotBytes;         // V ring
-  Barriers *bars = reinterpret_cast<Barriers *>(v_s + kStages * v_slot_bytes<DV>());
+  float *stage = reinterpret_cast<float *>(v_s + v_stages<DV>() * v_slot_bytes<DV>());
+  Barriers *bars = reinterpret_cast<Barriers *>(reinterpret_cast<uint8_t *>(stage) +
+                                                stage_bytes<DV>());
   auto *xc = reinterpret_cast<Xchg *>(reinterpret_cast<uint8_t *>(bars) + sizeof(Barriers));
-  float *stage = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(bars) + kBarsXchgBytes);
   const int warp = threadIdx.x >> 5;
   const uint32_t rank = cluster_ctarank();
 
@@ -1205,6 +1261,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars->k_full[s], loads);
       mbar_init(&bars->k_empty[s], 1);
+    }
+    for (int s = 0; s < v_stages<DV>(); ++s) {
       mbar_init(&bars->v_full[s], loads);
       mbar_init(&bars->v_empty[s], 1);
     }
@@ -1256,11 +1314,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       } else if (warp == kWarpIssueS) {
         relay_qk(bars, p, abort);
       } else if (warp == kWarpIssuePV) {
-        relay_v(bars, p, abort);
+        relay_v<DV>(bars, p, abort);
       }
     }
   } else {
-    softmax_role<MODE, DV>(bars, xc, stage, tmem, p, rank, abort);
+    softmax_role<MODE, DV>(bars, xc, stage, tmem, &tm_o, p, rank, abort);
   }
   __syncwarp();
   // No CTA leaves while the other may still use its shared or tensor memory:
@@ -1358,9 +1416,10 @@ __global__ void __launch_bounds__(kMergeThreads)
 static bool encode_map(EncodeTiledFn enc, CUtensorMap *map, const void *base,
                        int rank, const cuuint64_t *dims,
                        const cuuint64_t *strides, const cuuint32_t *box,
-                       CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
+                       CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B,
+                       CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank,
+  CUresult r = enc(map, dtype, rank,
                    const_cast<void *>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -1647,11 +1706,11 @@ cudaError_t make_plan(int mode, int dv, int n_items, int n_kt, int num_sms, int 
 
 template <int MODE, int DV>
 cudaError_t launch_mode(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                        const attn::Params &p, int clusters, bool dependent,
-                        cudaStream_t stream) {
+                        const CUtensorMap &to, const attn::Params &p, int clusters,
+                        bool dependent, cudaStream_t stream) {
   if (!dependent) {
     attn::attn_fwd_kernel<MODE, DV>
-        <<<2 * clusters, attn::kThreads, attn::smem_bytes<DV>(), stream>>>(tq, tk, tv, p);
+        <<<2 * clusters, attn::kThreads, attn::smem_bytes<DV>(), stream>>>(tq, tk, tv, to, p);
     return cudaGetLastError();
   }
   // The second launch of a two-phase schedule: programmatic dependent launch,
@@ -1666,18 +1725,20 @@ cudaError_t launch_mode(const CUtensorMap &tq, const CUtensorMap &tk, const CUte
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, attn::attn_fwd_kernel<MODE, DV>, tq, tk, tv, p);
+  return cudaLaunchKernelEx(&cfg, attn::attn_fwd_kernel<MODE, DV>, tq, tk, tv, to, p);
 }
 
 template <int DV>
 cudaError_t launch_dv(int mode, const CUtensorMap &tq, const CUtensorMap &tk,
-                      const CUtensorMap &tv, const attn::Params &p, int clusters,
-                      bool dependent, cudaStream_t stream) {
+                      const CUtensorMap &tv, const CUtensorMap &to, const attn::Params &p,
+                      int clusters, bool dependent, cudaStream_t stream) {
   using namespace attn;
   switch (mode) {
-    case kStaticCap: return launch_mode<kStaticCap, DV>(tq, tk, tv, p, clusters, dependent, stream);
-    case kOnlineCap: return launch_mode<kOnlineCap, DV>(tq, tk, tv, p, clusters, dependent, stream);
-    default: return launch_mode<kNoCap, DV>(tq, tk, tv, p, clusters, dependent, stream);
+    case kStaticCap:
+      return launch_mode<kStaticCap, DV>(tq, tk, tv, to, p, clusters, dependent, stream);
+    case kOnlineCap:
+      return launch_mode<kOnlineCap, DV>(tq, tk, tv, to, p, clusters, dependent, stream);
+    default: return launch_mode<kNoCap, DV>(tq, tk, tv, to, p, clusters, dependent, stream);
   }
 }
 
@@ -1770,6 +1831,20 @@ cudaError_t launch_attn_fwd(const AttnLaunch &a) {
                     dv192 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   }
+  // out [B, H, Lq, Dv] fp32, stored by the value-width-128 epilogue one box
+  // of 32 columns x 16 positions x 2 heads per softmax warp (128-byte rows,
+  // 128-byte swizzle).  Value width 192 stores directly and never reads it.
+  CUtensorMap to = tq;
+  if (a.Dv == 128) {
+    const cuuint64_t odims[4] = {128, static_cast<cuuint64_t>(Lq), kH,
+                                 static_cast<cuuint64_t>(B)};
+    const cuuint64_t ostrides[3] = {128 * 4, static_cast<cuuint64_t>(Lq) * 128 * 4,
+                                    static_cast<cuuint64_t>(Lq) * 128 * 4 * kH};
+    const cuuint32_t obox[4] = {32, 16, 2, 1};
+    if (!encode_map(a.encode, &to, a.out, 4, odims, ostrides, obox, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_DATA_TYPE_FLOAT32))
+      return cudaErrorInvalidValue;
+  }
   Params p;
   p.bias = a.bias;
   p.out = a.out;
@@ -1827,8 +1902,8 @@ cudaError_t launch_attn_fwd(const AttnLaunch &a) {
     p.ws_out = reinterpret_cast<float *>(base);
     p.ws_lse = reinterpret_cast<float *>(base + a.scratch_slots * kAttnSlotOutBytes);
   }
-  e = dv == 192 ? launch_dv<192>(mode, tq, tk, tv, p, pl.clusters, false, a.stream)
-                : launch_dv<128>(mode, tq, tk, tv, p, pl.clusters, false, a.stream);
+  e = dv == 192 ? launch_dv<192>(mode, tq, tk, tv, to, p, pl.clusters, false, a.stream)
+                : launch_dv<128>(mode, tq, tk, tv, to, p, pl.clusters, false, a.stream);
   if (e != cudaSuccess) return e;
   if (pl.sched == kSchedRange) {
     if (pl.clusters < 2 || pl.whole) return cudaSuccess;
@@ -1841,8 +1916,8 @@ cudaError_t launch_attn_fwd(const AttnLaunch &a) {
   }
   if (pl.tail_clusters == 0) return cudaSuccess;
   p.sched = kSchedTail;
-  return dv == 192 ? launch_dv<192>(mode, tq, tk, tv, p, pl.tail_clusters, true, a.stream)
-                   : launch_dv<128>(mode, tq, tk, tv, p, pl.tail_clusters, true, a.stream);
+  return dv == 192 ? launch_dv<192>(mode, tq, tk, tv, to, p, pl.tail_clusters, true, a.stream)
+                   : launch_dv<128>(mode, tq, tk, tv, to, p, pl.tail_clusters, true, a.stream);
 }
 
 }  // namespace ag
