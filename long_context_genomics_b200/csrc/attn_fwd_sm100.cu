@@ -188,7 +188,7 @@ struct __align__(8) Barriers {
 // parity) and row-sum (per segment) exchange between the four warpgroups.
 struct Xchg {
   float mpart[2][kWG][128];  // [tile parity][warpgroup][row]
-  float dpart[kWG][128];     // [warpgroup][row]
+  float dpart[2][kWG][128];  // [segment parity][warpgroup][row]
 };
 
 // Epilogue staging (value width 128): 4 KB per softmax warp, 1024-byte
@@ -1066,13 +1066,6 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc, float *st
     // over this segment's keys (warpgroup g writes columns [g DV/4, (g+1)
     // DV/4) of the row) and lse.  The copy of block I0 in an odd CTA past the
     // end of an odd block count writes nothing.
-    ok = mbar_wait(&bars->o_full, c.ocount & 1u, abort, p.err, kSiteSoftO);
-    ++c.ocount;
-    if (!__all_sync(0xffffffffu, ok)) {
-      ok = false;
-      break;
-    }
-    tc_fence_after();
     const bool writes = valid && pos < p.Lq;  // rows past the end of a partial block: none
     const size_t row = (static_cast<size_t>(b) * kH + h) * p.Lq + static_cast<size_t>(pos);
     float lse_a = 0.f;
@@ -1083,12 +1076,26 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc, float *st
       griddep_wait();
       if (writes) lse_a = p.lse[row];
     }
-    xc->dpart[g][r] = d;
-    ok = exchange(&bars->xd, c.xdcount, abort, p.err);
-    if (!ok) break;
+    // The partial sums are published before the wait for the last PV, so
+    // the exchange has normally completed when O is ready.  Double-buffered
+    // by segment parity: a warp writes the buffer of segment n + 2 only after
+    // the exchange of segment n + 1, which every warp joins after reading
+    // segment n's.
+    float(*dp)[128] = xc->dpart[c.xdcount & 1u];
+    dp[g][r] = d;
+    warp_arrive(&bars->xd);
+    ok = mbar_wait(&bars->o_full, c.ocount & 1u, abort, p.err, kSiteSoftO);
+    ++c.ocount;
+    if (ok) ok = mbar_wait(&bars->xd, c.xdcount & 1u, abort, p.err, kSiteXchg);
+    ++c.xdcount;
+    if (!__all_sync(0xffffffffu, ok)) {
+      ok = false;
+      break;
+    }
+    tc_fence_after();
     float dsum = 0.f;
 #pragma unroll
-    for (int q = 0; q < kWG; ++q) dsum += xc->dpart[q][r];
+    for (int q = 0; q < kWG; ++q) dsum += dp[q][r];
     const uint32_t tO = tmem + T::kColO + (DV / 4) * g + lane_base;
     const float lse_b = (m + lg2_approx(dsum)) * kLn2;
     float *orow_base;
