@@ -104,9 +104,10 @@ template <int DV> constexpr int v_slot_bytes() {
   return v_tiles_per_slot<DV>() * VLayout<DV>::kTileBytes;
 }
 
-// Tensor-memory columns: S buffer u at 128 u; P buffer p (bf16 pairs, 64
-// columns for 128 keys) at 256 + 64 p; O (DV columns) after the P buffers.
-// DV = 128: 2 S + 2 P + O = 512 columns; DV = 192: 2 S + 1 P + O = 512.
+// Tensor-memory columns of the running-max modes and of value width 192: S
+// buffer u at 128 u; P buffer p (bf16 pairs, 64 columns for 128 keys) at
+// 256 + 64 p; O (DV columns) after the P buffers.  DV = 128: 2 S + 2 P + O =
+// 512 columns; DV = 192: 2 S + 1 P + O = 512.
 template <int DV> struct Tmem {
   static constexpr int kNP = DV == 128 ? 2 : 1;
   static constexpr uint32_t kColP = 256;
@@ -120,6 +121,7 @@ template <int DV> struct Tmem {
 // group's next tile are usually ready before the group asks for them.
 constexpr uint32_t kIPBufs = 3;
 constexpr uint32_t kIPColO = 384;
+// The fixed-shift mode (mode 0, kStaticCap below) at value width 128.
 template <int MODE, int DV> constexpr bool p_in_place() { return MODE == 0 && DV == 128; }
 static_assert(Tmem<128>::kColO + 128 <= 512 && Tmem<192>::kColO + 192 <= 512,
               "tensor memory budget");
@@ -532,8 +534,10 @@ __device__ __forceinline__ void relay_v(Barriers *bars, const Params &p, volatil
 // acquire at CTA scope: a cluster-scope acquire would order nothing more and
 // costs about 180 cycles per wait (measured).
 
-// S = Q K^T for every key tile, into S buffer (use count & 1), once the
-// softmax has read that buffer's previous logits (s_free).
+// S = Q K^T for every key tile, into step buffer (use count) % 2, once the
+// softmax has read that buffer's previous logits (s_free); with P in place
+// into buffer (use count) % 3, once PV has read the P written over that
+// buffer's previous logits (pv_done).
 template <bool kIP>
 __device__ __forceinline__ void issuer_s(uint8_t *q_s, uint8_t *k_s, Barriers *bars,
                                          uint32_t tmem, const Params &p,
