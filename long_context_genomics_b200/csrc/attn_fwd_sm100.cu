@@ -1581,11 +1581,21 @@ bool pack_first_launch(int t, int nw, int ns, int n_kt, int a, int G, std::vecto
 // Extra cost of a second launch, in key-tile steps: its prologue (barriers,
 // tensor memory, the Q tile and the first logits) before the softmax runs.
 constexpr int kTailCostSteps = 4;
+// Extra cost of every segment (a whole pair or a piece), in key-tile steps:
+// the drain of its last PV, the epilogue and the restart of the step-buffer
+// pipeline, about 7,000-9,000 cycles against 1,790 per steady-state step.
+// With it the planner stops cutting a cluster's work into many short first
+// pieces (measured at B = 1: L = 4096 89.2 -> 80.0 us, L = 6144 160.8 ->
+// 154.8 us, L = 8192 249.8 -> 248.8 us, against a model without it).
+constexpr int kSegCostSteps = 5;
 
-// No-scratch schedule: whole pairs, or two phases when that beats them.
+// No-scratch schedule: whole pairs, or two phases when that beats them.  A
+// plan's cost is its critical path in key-tile steps, every segment counted
+// kSegCostSteps longer.
 void plan_no_scratch(int n_items, int n_kt, int G, Plan *pl) {
   plan_whole(n_items, G, pl);
-  const long long whole_cost = static_cast<long long>((n_items + G - 1) / G) * n_kt;
+  constexpr int c = kSegCostSteps;
+  const long long whole_cost = static_cast<long long>((n_items + G - 1) / G) * (n_kt + c);
   if (n_kt < 2 || n_items > 8 * G || n_items <= G) return;
   const int ns = G;  // one second piece per cluster of the second launch
   const int nw = n_items - ns;
@@ -1593,21 +1603,22 @@ void plan_no_scratch(int n_items, int n_kt, int G, Plan *pl) {
   int best_b = 0, best_t = 0;
   for (int b = 1; b < n_kt; ++b) {
     const int a = n_kt - b;
-    const long long hi = best - b - kTailCostSteps - 1;  // t must beat the best so far
-    const long long work = static_cast<long long>(nw) * n_kt + static_cast<long long>(ns) * a;
+    const long long hi = best - (b + c) - kTailCostSteps - 1;  // t must beat the best so far
+    const long long work =
+        static_cast<long long>(nw) * (n_kt + c) + static_cast<long long>(ns) * (a + c);
     long long lo = (work + G - 1) / G;
     if (lo > hi) continue;
     std::vector<int> x, y;
-    if (!pack_first_launch(static_cast<int>(hi), nw, ns, n_kt, a, G, &x, &y)) continue;
+    if (!pack_first_launch(static_cast<int>(hi), nw, ns, n_kt + c, a + c, G, &x, &y)) continue;
     long long l = lo, h = hi;  // smallest feasible t in [lo, hi]
     while (l < h) {
       const long long mid = (l + h) / 2;
-      if (pack_first_launch(static_cast<int>(mid), nw, ns, n_kt, a, G, &x, &y))
+      if (pack_first_launch(static_cast<int>(mid), nw, ns, n_kt + c, a + c, G, &x, &y))
         h = mid;
       else
         l = mid + 1;
     }
-    const long long cost = l + b + kTailCostSteps;
+    const long long cost = l + (b + c) + kTailCostSteps;
     if (cost < best) {
       best = cost;
       best_b = b;
@@ -1617,7 +1628,7 @@ void plan_no_scratch(int n_items, int n_kt, int G, Plan *pl) {
   if (best_b == 0) return;
   std::vector<int> x, y;
   const int a = n_kt - best_b;
-  if (!pack_first_launch(best_t, nw, ns, n_kt, a, G, &x, &y)) return;
+  if (!pack_first_launch(best_t, nw, ns, n_kt + c, a + c, G, &x, &y)) return;
   // Drop clusters with no work; ranges stay contiguous per kind.
   std::vector<int> wb(1, 0), fb(1, 0);
   for (int c = 0; c < G; ++c) {

@@ -71,16 +71,22 @@ def test_no_scratch_schedule_covers_every_step_once(lib, B, L, pairs):
     assert all(v == 1 for v in steps)
 
 
+SEG_COST = 5   # the planner's cost of one segment, in key-tile steps
+TAIL_COST = 4  # and of the second launch's start
+
+
 @pytest.mark.parametrize("B,L", CASES)
 def test_no_scratch_schedule_is_never_worse_than_whole_pairs(lib, B, L):
     """Two phases are chosen only when their critical path (first launch's
-    busiest cluster plus the second piece) beats whole pairs."""
+    busiest cluster plus the second piece, every segment counted SEG_COST
+    steps longer) beats whole pairs."""
     items, n_kt = sizes(B, L)
     s = schedule(lib, B, L, 74)
-    whole_cost = math.ceil(items / 74) * n_kt
+    whole_cost = math.ceil(items / 74) * (n_kt + SEG_COST)
     cl, wb, fb, a = s["clusters"], s["wb"], s["fb"], s["split_at"]
-    first = max((wb[c + 1] - wb[c]) * n_kt + (fb[c + 1] - fb[c]) * a for c in range(cl))
-    cost = first + (n_kt - a if s["tail"] else 0)
+    first = max((wb[c + 1] - wb[c]) * (n_kt + SEG_COST) + (fb[c + 1] - fb[c]) * (a + SEG_COST)
+                for c in range(cl))
+    cost = first + (n_kt - a + SEG_COST + TAIL_COST if s["tail"] else 0)
     assert cost <= whole_cost
     if not s["tail"]:
         assert first == whole_cost
@@ -89,12 +95,19 @@ def test_no_scratch_schedule_is_never_worse_than_whole_pairs(lib, B, L):
 def test_full_context_schedule_on_a_b200(lib):
     """L = 8192, B = 1 on 74 SM pairs: 256 pairs do not divide over 74, so
     whole pairs would cost 4 x 64 = 256 key-tile steps on the busiest pair;
-    the two-phase schedule costs 192 + 32 (the ideal is 16384 / 74 = 221.4)."""
+    the two-phase schedule costs 192 + 34 (the ideal is 16384 / 74 = 221.4),
+    with at most 4 segments on a cluster of the first launch."""
     s = schedule(lib, 1, 8192, 74)
-    assert s["tail"] == 74 and s["split_at"] == 32 and s["n_whole"] == 182
-    loads = [(s["wb"][c + 1] - s["wb"][c]) * 64 + (s["fb"][c + 1] - s["fb"][c]) * 32
+    assert s["tail"] == 74 and s["split_at"] == 30 and s["n_whole"] == 182
+    loads = [(s["wb"][c + 1] - s["wb"][c]) * 64 + (s["fb"][c + 1] - s["fb"][c]) * 30
              for c in range(s["clusters"])]
-    assert max(loads) == 192
+    segs = [(s["wb"][c + 1] - s["wb"][c]) + (s["fb"][c + 1] - s["fb"][c])
+            for c in range(s["clusters"])]
+    assert max(loads) == 192 and max(segs) == 4
+    # L = 4096: 128 pairs of 32 steps; cutting them would add segments that
+    # cost more than they balance, so whole pairs (2 per cluster).
+    s1 = schedule(lib, 1, 4096, 74)
+    assert s1["tail"] == 0 and s1["clusters"] == 74
     # The nine-layer stack's B = 2 divides almost evenly (512 / 74 = 6.92): whole pairs.
     s2 = schedule(lib, 2, 8192, 74)
     assert s2["tail"] == 0 and s2["clusters"] == 74
