@@ -18,24 +18,33 @@
 //    keys) and half of every V tile (DV/2 value columns), so each K/V byte
 //    crosses from L2 into one SM only and serves the 256 query rows of the
 //    pair.  DV (value width) is 128 or 192.
-//  * Tensor memory (per CTA): two 128-column S buffers (fp32 logits of
-//    alternate key tiles), one or two 64-column P buffers (bf16 probabilities
-//    of a key tile) and the DV-column O accumulator.  Because P has buffers of
-//    its own, the logits S(j+2) can be computed as soon as the softmax has
-//    read S(j) into registers, long before PV(j) runs: the tensor core always
-//    holds the next logits when the softmax wants them.
-//  * Two MMA-issuing threads in the even CTA: one issues every S = Q K^T and
-//    one every O += P V, each with its own waits and commits, fed by separate
-//    K and V rings (TMA, no multicast).  In the odd CTA two relay threads
-//    forward "loaded" to the even CTA (cluster-scope arrives), so each CTA's
-//    copies complete on its own barriers and can be drained locally.
-//  * All four softmax warpgroups work on every key tile, 32 keys each; the
-//    bias of a thread's 32 keys is two compact cells, read from global (L2)
-//    one tile ahead and kept in registers: the 16x repeat is never built.
+//  * Tensor memory (per CTA), fixed-shift mode at value width 128: three
+//    128-column step buffers (fp32 logits of key tile t in buffer t % 3, the
+//    bf16 probabilities then written over the logits already read) and the
+//    128-column O accumulator; the logits of tile t wait only for the PV of
+//    tile t - 3.  Running-max modes and value width 192: two S buffers, one
+//    or two P buffers of their own and the DV-column O.
+//  * Two MMA-issuing warps in the even CTA (an elect.sync-chosen lane
+//    issues): one issues every S = Q K^T and one every O += P V, each with its
+//    own waits and commits, fed by separate K and V rings (TMA, no
+//    multicast).  In the odd CTA two relay threads forward "loaded" to the
+//    even CTA (cluster-scope arrives), so each CTA's copies complete on its
+//    own barriers and can be drained locally.
+//  * Fixed-shift mode at value width 128: the 16 softmax warps form two
+//    groups on alternate key tiles, each warpgroup of a group 64 keys of the
+//    tile, so one group's waits are covered by the other's arithmetic.
+//    Otherwise all four warpgroups work on every key tile, 32 keys each.  The
+//    bias of a thread's keys is one compact cell per 16 keys, read from
+//    global (L2) a tile ahead and kept in registers: the 16x repeat is never
+//    built.
 //  * With a finite cap every logit lies in (-cap, cap), so the softmax uses a
 //    fixed shift (exact: softmax is shift invariant) and needs no running max
-//    and no rescaling of O.  cap > 40 (where exp(-2 cap) would underflow fp32)
-//    and cap = +inf use a running max with lazy rescaling.
+//    and no rescaling of O (cap <= 60: beyond, the probabilities of a row
+//    span more than fp32's range).  Larger caps and cap = +inf use a running
+//    max with lazy rescaling.
+//  * Epilogue at value width 128: each warp stages its 32 x 32 block of out
+//    in shared memory and writes it with one bulk tensor store, which drains
+//    while the warps go on to the next pair.
 //  * Work is cut into segments (a pair of query tiles and a run of its key
 //    tiles).  Three schedules: whole pairs per cluster; "two phases", where
 //    some pairs are split into a first piece (first launch, result written to
@@ -152,8 +161,8 @@ constexpr float kLn2 = 0.6931471805599453f;
 // Lazy rescale threshold (log2 units) for the running-max modes.
 constexpr float kRescaleThreshold = 8.0f;
 
-// Softmax modes.  kStaticCap: finite cap up to 40, fixed shift.  kOnlineCap:
-// cap > 40, running max.  kNoCap: no soft cap, running max.  The capped
+// Softmax modes.  kStaticCap: finite cap up to 60, fixed shift.  kOnlineCap:
+// cap > 60, running max.  kNoCap: no soft cap, running max.  The capped
 // modes take tanh from the special-function unit (tanh.approx.f32, measured
 // on B200 over |y| <= 12: relative error below 1e-5, absolute below 8e-6, so
 // the capped logit's error stays below 1e-5 min(cap, |y cap|)).
@@ -256,7 +265,7 @@ struct Params {
   float qk_scale;  // multiplies q.k
   float bias_mul;  // multiplies the compact bias
   float A;         // capped modes: cap * log2(e)
-  float shift;     // static modes: the fixed shift (log2 units, an integer >= A)
+  float shift;     // static modes: the fixed shift (log2 units, an integer; see attn_mode)
   // kSchedUnits: cluster c runs whole items [wb[c], wb[c+1]) and then the
   // first pieces of split pairs [fb[c], fb[c+1]).
   int wb[kAttnMaxClusters + 1];
@@ -1491,12 +1500,24 @@ cudaError_t configure_any(int mode, int *max_clusters) {
   }
 }
 
-// The static shift needs every exp(L - cap) of a row, down to exp(-2 cap),
-// to stay a normal fp32 number: cap <= 40.
+// The fixed shift s (log2 units) puts every probability 2^(A t - s) of a row,
+// A = cap log2(e) and t in (-1, 1), in (2^(-A-s), 2^(A-s)).  The smallest
+// must stay a normal fp32 number (the row's largest probability may be that
+// small, and the exponent insertion of exp2_poly2_fma must not leave the
+// exponent field) and the largest, times L and |v|, must not overflow the
+// sums.  s = ceil(A) (probabilities up to 1) meets both up to A = 60; above,
+// s = 120 - ceil(A) keeps the exponents in [-120, 2 ceil(A) - 120], which
+// stays far from overflow up to cap = 60 (A = 86.6, probabilities below
+// 2^54).  Larger caps run the running maximum.
 int attn_mode(float cap) {
   using namespace attn;
   if (std::isinf(cap)) return kNoCap;
-  return cap <= 40.0f ? kStaticCap : kOnlineCap;
+  return cap <= 60.0f ? kStaticCap : kOnlineCap;
+}
+
+float attn_static_shift(float A) {
+  const float ca = ceilf(A);
+  return ca <= 60.0f ? ca : 120.0f - ca;
 }
 
 // --------------------------------------------------------------------------
@@ -1897,13 +1918,13 @@ cudaError_t launch_attn_fwd(const AttnLaunch &a) {
       p.shift = 0.f;
       break;
     default:
-      // y = z / cap, logits A tanh(y) in log2 units.  The static shift is the
-      // smallest integer >= A (exp2_poly2_fma folds an integer shift into
-      // its range reduction).
+      // y = z / cap, logits A tanh(y) in log2 units.  The static shift is an
+      // integer (exp2_poly2_fma folds it into its range reduction): the
+      // smallest integer >= A, or 120 - that above A = 60 (attn_mode).
       p.qk_scale = inv_sqrt_d / cap;
       p.bias_mul = 1.0f / cap;
       p.A = cap * kLog2e;
-      p.shift = ceilf(p.A);
+      p.shift = attn_static_shift(p.A);
       break;
   }
   const int dv = static_cast<int>(a.Dv);

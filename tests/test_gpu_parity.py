@@ -219,10 +219,10 @@ def test_strided_bias_with_padding_between_items(ag, oracle_lib):
              "padded per-item bias")
 
 
-@pytest.mark.parametrize("cap", [1.0, 5.0, 10.0, 30.0, 40.0, 50.0, 1e4, math.inf])
+@pytest.mark.parametrize("cap", [1.0, 5.0, 10.0, 30.0, 40.0, 50.0, 60.0, 61.0, 1e4, math.inf])
 def test_cap_modes(ag, oracle_lib, cap):
-    """Static shift (cap <= 40), running max with the cap (cap > 40) and no
-    cap at all."""
+    """Static shift (cap <= 60; shift ceil(cap log2 e) up to cap 41.6, then
+    120 - that), running max with the cap (cap > 60) and no cap at all."""
     inp = ag_inputs.random_case(2, 8, 512, 128, 128, 16, seed=int(min(cap, 1e6)) + 3)
     out, lse = _gpu_attn(ag, inp, cap)
     ro, rl = oracle_lib.attn_fwd(inp["q"], inp["k"], inp["v"], inp["bias"],
@@ -230,13 +230,14 @@ def test_cap_modes(ag, oracle_lib, cap):
     _compare(out, lse, ro, rl, f"cap={cap}")
 
 
-@pytest.mark.parametrize("cap", [5.0, 10.0, 30.0, 40.0, 50.0, math.inf])
+@pytest.mark.parametrize("cap", [5.0, 10.0, 30.0, 40.0, 50.0, 60.0, 61.0, math.inf])
 def test_large_logits(ag, oracle_lib, cap):
     """q, k with std 3 and a bias of std 4: logits far beyond the cap
     (saturated tanh), a softmax dominated by a few keys at the large caps
     (where an error in a logit passes straight into lse) and, without a cap,
     a wide softmax range.  Caps 40 and 50 sit on either side of the switch
-    from the static shift to the running maximum."""
+    between the two shifts of the static mode, 60 and 61 on either side of
+    the switch to the running maximum."""
     inp = ag_inputs.random_case(1, 8, 640, 128, 128, 16, seed=77, bias_std=4.0,
                                 qk_std=3.0)
     out, lse = _gpu_attn(ag, inp, cap)
@@ -245,7 +246,7 @@ def test_large_logits(ag, oracle_lib, cap):
     _compare(out, lse, ro, rl, f"large logits cap={cap}")
 
 
-@pytest.mark.parametrize("cap", [5.0, 10.0, 40.0, 50.0])
+@pytest.mark.parametrize("cap", [5.0, 10.0, 40.0, 50.0, 60.0, 61.0])
 def test_large_logits_full_context_sampled(ag, oracle_lib, cap):
     """The same logit distribution at L = 8192 (8192 keys per softmax, the
     two-launch schedule at B = 1), sampled rows against the oracle."""
