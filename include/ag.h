@@ -132,7 +132,11 @@ ag_status ag_pair_bias_project_rows(const float *pair, const float *W, float *bi
  * piece runs in a second launch on the same stream (programmatic dependent
  * launch, so it starts on the SMs the first launch frees) and merges the
  * first piece's result with its own by log-sum-exp.  No scratch memory is
- * used, so calls on different streams may overlap freely.
+ * used, so calls on different streams may overlap freely.  The softmax
+ * shifts by a fixed amount for cap <= 60 (the soft cap bounds every logit);
+ * for a larger cap or no cap (value width 128) a first pass writes every
+ * row's largest logit into lse and the main kernel then shifts each row by
+ * it, over whole pairs (value width 192: a running maximum).
  */
 ag_status ag_attn_fwd(const void *q, const void *k, const void *v,
                       const float *bias, int64_t B, int64_t H, int64_t L,
@@ -235,12 +239,13 @@ ag_status ag_attn_fwd_noalloc(const void *q, const void *k, const void *v,
  * ag_attn_fwd_launch_count -- how many kernels ag_attn_fwd (and
  * ag_attn_fwd_strided_bias, ag_attn_fwd_ex) launches for these sizes on the
  * current device: 0 for an empty call, 1, or 2 when some pairs of query tiles
- * have their keys split in two and a second launch merges them (a library
- * convenience for callers that count launches; the pages have no
- * counterpart).  Same size and value checks, and statuses, as ag_attn_fwd;
- * count is a host pointer (AG_ERR_NULL if NULL).  Launches nothing.  The
- * count holds at either value width: both widths run one CTA per SM, so
- * they get the same grid.
+ * have their keys split in two and a second launch merges them; for a cap
+ * above 60 or no cap, the first pass of row maxima (1 or 2 launches) plus
+ * the main kernel (a library convenience for callers that count launches;
+ * the pages have no counterpart).  Same size and value checks, and
+ * statuses, as ag_attn_fwd; count is a host pointer (AG_ERR_NULL if NULL).
+ * Launches nothing.  The count is for value width D (128); at value width
+ * 192 the caps above 60 run the running maximum, 1 or 2 launches.
  */
 ag_status ag_attn_fwd_launch_count(int64_t B, int64_t H, int64_t L, int64_t D,
                                    int64_t block, float cap, int *count);

@@ -68,6 +68,25 @@ namespace attn {
 
 constexpr int kH = 8;
 constexpr int kD = 128;
+
+// Softmax modes (see the comment before attn_mode for the choice).
+//   kStaticCap:   finite cap up to 60, fixed shift (no row maximum needed).
+//   kOnlineCap:   cap > 60, running maximum with lazy rescaling.
+//   kNoCap:       no soft cap, running maximum.
+//   kRowMax:      first pass of the two-pass schedule (value width 128, cap
+//                 > 60 or none): each row's largest logit, into lse.
+//   kRowShift:    second pass without a cap: the fixed-shift kernel with the
+//                 row's own shift ceil(max) read from lse.
+//   kRowShiftCap: the same with the soft cap (cap > 60).
+enum Mode {
+  kStaticCap = 0, kOnlineCap = 1, kNoCap = 2, kRowMax = 3, kRowShift = 4, kRowShiftCap = 5
+};
+template <int MODE> constexpr bool fixed_shift() {
+  return MODE == kStaticCap || MODE == kRowShift || MODE == kRowShiftCap;
+}
+template <int MODE> constexpr bool row_shift() {
+  return MODE == kRowShift || MODE == kRowShiftCap;
+}
 constexpr int kKeys = static_cast<int>(kAttnKeyTile);  // keys per key tile
 static_assert(kKeys == 128, "the tile layout below assumes 128-key tiles");
 constexpr int kQTileBytes = 128 * kD * 2;     // this CTA's query tile (bf16)
@@ -129,9 +148,13 @@ template <int DV> struct Tmem {
 // buffer's last reader) instead of for the softmax, so the logits of a warp
 // group's next tile are usually ready before the group asks for them.
 constexpr uint32_t kIPBufs = 3;
+// The first pass of the two-pass schedule has no P and no O: four S buffers.
+constexpr uint32_t kRowMaxBufs = 4;
 constexpr uint32_t kIPColO = 384;
-// The fixed-shift mode (mode 0, kStaticCap below) at value width 128.
-template <int MODE, int DV> constexpr bool p_in_place() { return MODE == 0 && DV == 128; }
+// The fixed-shift modes at value width 128.
+template <int MODE, int DV> constexpr bool p_in_place() {
+  return fixed_shift<MODE>() && DV == 128;
+}
 static_assert(Tmem<128>::kColO + 128 <= 512 && Tmem<192>::kColO + 192 <= 512,
               "tensor memory budget");
 constexpr uint32_t kTmemCols = 512;
@@ -161,12 +184,9 @@ constexpr float kLn2 = 0.6931471805599453f;
 // Lazy rescale threshold (log2 units) for the running-max modes.
 constexpr float kRescaleThreshold = 8.0f;
 
-// Softmax modes.  kStaticCap: finite cap up to 60, fixed shift.  kOnlineCap:
-// cap > 60, running max.  kNoCap: no soft cap, running max.  The capped
-// modes take tanh from the special-function unit (tanh.approx.f32, measured
-// on B200 over |y| <= 12: relative error below 1e-5, absolute below 8e-6, so
-// the capped logit's error stays below 1e-5 min(cap, |y cap|)).
-enum Mode { kStaticCap = 0, kOnlineCap = 1, kNoCap = 2 };
+// The capped modes take tanh from the special-function unit (tanh.approx.f32,
+// measured on B200 over |y| <= 12: relative error below 1e-5, absolute below
+// 8e-6, so the capped logit's error stays below 1e-5 min(cap, |y cap|)).
 
 // Wait sites recorded in the device error word.
 enum Site : unsigned {
@@ -186,7 +206,7 @@ struct __align__(8) Barriers {
   uint64_t q_full, q_empty;
   uint64_t k_full[kStages], k_empty[kStages];
   uint64_t v_full[kVStagesMax], v_empty[kVStagesMax];  // [v_stages<DV>()] in use
-  uint64_t s_full[3], s_free[2];
+  uint64_t s_full[kRowMaxBufs], s_free[kRowMaxBufs];  // [3] / [2] / [4] in use (see issuer_s)
   uint64_t p_full[3], pv_done[3];  // three in use with P in place, else [Tmem<DV>::kNP]
   uint64_t o_full;
   uint64_t xm, xd;  // row-max / row-sum exchange between the warpgroups
@@ -591,6 +611,48 @@ __device__ __forceinline__ void issuer_s(uint8_t *q_s, uint8_t *k_s, Barriers *b
   drain_wait(&bars->drain, 0);
 }
 
+// S for the first pass of the two-pass schedule (kRowMax): a step is one K
+// ring slot (two key tiles, or one at the end of a segment), issued into the
+// 256-column buffer pair step % 2 and committed once, so the issuing thread
+// waits and commits once per two tiles; the softmax releases a pair
+// (s_free[pair]) once it has read both tiles' logits.
+__device__ __forceinline__ void issuer_rowmax(uint8_t *q_s, uint8_t *k_s, Barriers *bars,
+                                              uint32_t tmem, const Params &p,
+                                              volatile int *abort) {
+  const uint32_t q_addr = smem_u32(q_s), k_addr = smem_u32(k_s);
+  uint32_t qc = 0, kl = 0, st = 0;
+  bool ok = true;
+  Cursor cu = cursor_begin(p);
+  Segment sg;
+  while (ok && next_segment(p, cu, sg)) {
+    ok = mbar_wait_warp(&bars->q_full, qc & 1u, abort, p.err, kSiteIssueQ);
+    ++qc;
+    if (!ok) break;
+    for (int j0 = sg.kb; j0 < sg.ke; j0 += kTilesPerSlot) {
+      const int nt = sg.ke - j0 < kTilesPerSlot ? sg.ke - j0 : kTilesPerSlot;
+      const uint32_t slot = kl % kStages;
+      ok = mbar_wait_warp(&bars->k_full[slot], (kl / kStages) & 1u, abort, p.err, kSiteIssueK);
+      ++kl;
+      if (!ok) break;
+      const uint32_t b = st & 1u, n = st >> 1;
+      if (n > 0) {
+        ok = mbar_wait_warp(&bars->s_free[b], (n - 1) & 1u, abort, p.err, kSiteIssueSFree);
+        if (!ok) break;
+      }
+      tc_fence_after();
+      for (int t = 0; t < nt; ++t)
+        issue_qk(tmem + 256u * b + 128u * static_cast<uint32_t>(t), q_addr,
+                 k_addr + slot * kKSlotBytes + t * kKTileBytes);
+      umma2_commit_both_w(&bars->s_full[b]);
+      if (j0 + nt == sg.ke) umma2_commit_both_w(&bars->q_empty);
+      umma2_commit_both_w(&bars->k_empty[slot]);
+      ++st;
+    }
+  }
+  umma2_commit_self_w(&bars->drain);
+  drain_wait(&bars->drain, 0);
+}
+
 // O += P V for every key tile, once the softmax has written P (p_full).
 template <int DV, bool kIP>
 __device__ __forceinline__ void issuer_pv(uint8_t *v_s, Barriers *bars, uint32_t tmem,
@@ -700,16 +762,22 @@ constexpr int kEmuPairs = AG_EXP2_EMU_PAIRS;
 // Constants of the static mode, per thread.
 struct StaticK {
   float2 sc;     // multiplies s
-  float2 a;      // A = cap log2(e)
+  float2 a;      // A = cap log2(e) (1 without a cap)
   float2 nsh;    // -shift (for the SFU pairs)
   float2 km;     // 1.5 * 2^23 - shift (exp2_poly2_fma)
+  float tmin;    // row shifts: the smallest t for exp2_poly2_fma, (shift - 126) / A
 };
 
-// One thread's 32 keys of a key tile, static shift, log2 units:
-// t = tanh(y), p = 2^(A t - shift), y = s qk_scale + b / cap.  Adds the row
-// sum into acc and packs 16 bf16 pairs of P.  kMask zeroes keys >= nvalid
-// (only the last key tile of a ragged length needs it).
-template <bool kMask, int N>
+// One thread's N keys of a key tile, fixed shift, log2 units:
+// t = tanh(y) (or t = y without a cap, MODE kRowShift), p = 2^(A t - shift),
+// y = s qk_scale + b / cap.  Adds the row sum into acc and packs N/2 bf16
+// pairs of P.  kMask zeroes keys >= nvalid (only the last key tile of a
+// ragged length needs it).  With a row's own shift the exponent A t - shift
+// has no lower bound, so the FMA-pipe exponential takes t no smaller than
+// k.tmin (probabilities below 2^-126, which cannot move a row sum whose
+// largest term is at least 1/2, become 2^-126); the special-function unit's
+// ex2 flushes them to zero by itself.
+template <bool kMask, int N, int MODE = kStaticCap>
 __device__ __forceinline__ void chunk_static(const uint32_t (&s)[N], float b0, float b1,
                                              const StaticK &k, int col0, int nvalid,
                                              float2 &acc, uint32_t (&pk)[N / 2]) {
@@ -719,10 +787,13 @@ __device__ __forceinline__ void chunk_static(const uint32_t (&s)[N], float b0, f
     const float2 y = __ffma2_rn(
         make_float2(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1])), k.sc,
         make_float2(bb, bb));
-    const float2 t = make_float2(tanh_approx(y.x), tanh_approx(y.y));
+    const float2 t = MODE == kRowShift ? y : make_float2(tanh_approx(y.x), tanh_approx(y.y));
     float2 pr;
     if ((e & 7) < kEmuPairs) {
-      pr = exp2_poly2_fma(t, k.a, k.km);
+      if constexpr (row_shift<MODE>())
+        pr = exp2_poly2_fma(make_float2(fmaxf(t.x, k.tmin), fmaxf(t.y, k.tmin)), k.a, k.km);
+      else
+        pr = exp2_poly2_fma(t, k.a, k.km);
     } else {
       const float2 x = __ffma2_rn(t, k.a, k.nsh);
       pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
@@ -793,7 +864,7 @@ __device__ __forceinline__ bool store_p(Barriers *bars, uint32_t tmem, int g,
 
 // One 64-key half tile of a grouped static segment (see below): tS and tP
 // address this warp's S and P columns, bc holds the four bias cells.
-template <bool kMask>
+template <bool kMask, int MODE>
 __device__ __forceinline__ void tile_grouped(uint32_t tS, const float (&bc)[4], float m,
                                              const StaticK &k, int col0, int nvalid,
                                              float2 &acc) {
@@ -804,18 +875,18 @@ __device__ __forceinline__ void tile_grouped(uint32_t tS, const float (&bc)[4], 
   tmem_ld16(tS, sa);
   tmem_wait_ld16(sa);
   tmem_ld16(tS + 16u, sb);
-  chunk_static<kMask, 16>(sa, bc[0] * m, bc[0] * m, k, col0, nvalid, acc, pk);
+  chunk_static<kMask, 16, MODE>(sa, bc[0] * m, bc[0] * m, k, col0, nvalid, acc, pk);
   tmem_st8(tS, pk);
   tmem_wait_ld16(sb);
   tmem_ld16(tS + 32u, sa);
-  chunk_static<kMask, 16>(sb, bc[1] * m, bc[1] * m, k, col0 + 16, nvalid, acc, pk);
+  chunk_static<kMask, 16, MODE>(sb, bc[1] * m, bc[1] * m, k, col0 + 16, nvalid, acc, pk);
   tmem_st8(tS + 8u, pk);
   tmem_wait_ld16(sa);
   tmem_ld16(tS + 48u, sb);
-  chunk_static<kMask, 16>(sa, bc[2] * m, bc[2] * m, k, col0 + 32, nvalid, acc, pk);
+  chunk_static<kMask, 16, MODE>(sa, bc[2] * m, bc[2] * m, k, col0 + 32, nvalid, acc, pk);
   tmem_st8(tS + 16u, pk);
   tmem_wait_ld16(sb);
-  chunk_static<kMask, 16>(sb, bc[3] * m, bc[3] * m, k, col0 + 48, nvalid, acc, pk);
+  chunk_static<kMask, 16, MODE>(sb, bc[3] * m, bc[3] * m, k, col0 + 48, nvalid, acc, pk);
   tmem_st8(tS + 24u, pk);
 }
 
@@ -829,20 +900,26 @@ __device__ __forceinline__ void tile_grouped(uint32_t tS, const float (&bc)[4], 
 // the s_full phases of its own tiles in order; the phase of the buffer's
 // previous tile (the other group's) has completed by then, because the
 // logits of the group's own previous tile, issued later, have.
-template <int DV>
+//
+// shift: this thread's row's shift (p.shift, or the row's own one in the
+// row-shift modes; an integer).
+template <int MODE, int DV>
 __device__ __forceinline__ bool segment_static_grouped(const Segment &sg, const float *brow,
                                                        uint32_t tmem, uint32_t lane_base, int g,
                                                        const Params &p, Barriers *bars,
                                                        uint32_t rank, SoftCounters &c,
-                                                       volatile int *abort, float &d) {
+                                                       volatile int *abort, float shift,
+                                                       float &d) {
   static_assert(DV == 128, "P in place: value width 128");
   const int q = g >> 1, hk = g & 1;  // group, key half
   StaticK k;
   constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  const float A = MODE == kRowShift ? 1.f : p.A;
   k.sc = make_float2(p.qk_scale, p.qk_scale);
-  k.a = make_float2(p.A, p.A);
-  k.nsh = make_float2(-p.shift, -p.shift);
-  k.km = make_float2(kShift - p.shift, kShift - p.shift);
+  k.a = make_float2(A, A);
+  k.nsh = make_float2(-shift, -shift);
+  k.km = make_float2(kShift - shift, kShift - shift);
+  k.tmin = (shift - 126.f) / A;
   float2 acc = make_float2(0.f, 0.f);
   const uint32_t pf0 = cluster_addr(&bars->p_full[0], 0);  // the even CTA's p_full
   // Key tile j of the segment is global tile c.su + (j - kb); the group takes
@@ -862,9 +939,9 @@ __device__ __forceinline__ bool segment_static_grouped(const Segment &sg, const 
     // Four pieces of 16 keys (one bias cell each), the tensor-memory load of
     // the next piece in flight while this one is computed.
     if (nvalid == kKeys)
-      tile_grouped<false>(tS, bc, m, k, 64 * hk, nvalid, acc);
+      tile_grouped<false, MODE>(tS, bc, m, k, 64 * hk, nvalid, acc);
     else
-      tile_grouped<true>(tS, bc, m, k, 64 * hk, nvalid, acc);
+      tile_grouped<true, MODE>(tS, bc, m, k, 64 * hk, nvalid, acc);
     if (j + 2 < sg.ke) load_bias4(brow, j + 2, hk, p.P, bc);
     tmem_wait_st();
     tc_fence_before();
@@ -959,6 +1036,50 @@ __device__ __forceinline__ bool segment_static(const Segment &sg, const float *b
   return true;
 }
 
+// First pass of the two-pass schedule (kRowMax): the row's largest biased
+// score y = s qk_scale + b bias_mul over this segment's keys, every
+// warpgroup 32 keys of every key tile, in the steps of issuer_rowmax (the
+// buffer pair released once both tiles' logits are in registers).  No P, no
+// PV.  c.su counts steps.
+__device__ __forceinline__ bool segment_rowmax(const Segment &sg, const float *brow,
+                                               uint32_t tmem, uint32_t lane_base, int g,
+                                               const Params &p, Barriers *bars, uint32_t rank,
+                                               SoftCounters &c, volatile int *abort,
+                                               float &ymax) {
+  const uint32_t sf0 = cluster_addr(&bars->s_free[0], 0);  // the even CTA's s_free
+  for (int j0 = sg.kb; j0 < sg.ke; j0 += kTilesPerSlot) {
+    const int nt = sg.ke - j0 < kTilesPerSlot ? sg.ke - j0 : kTilesPerSlot;
+    const uint32_t b = c.su & 1u, ph = (c.su >> 1) & 1u;
+    ++c.su;
+    float bc[kTilesPerSlot][2];
+#pragma unroll
+    for (int t = 0; t < kTilesPerSlot; ++t)
+      if (t < nt) load_bias(brow, j0 + t, g, p.P, bc[t]);
+    const bool okw = mbar_wait(&bars->s_full[b], ph, abort, p.err, kSiteSoftS);
+    if (!__all_sync(0xffffffffu, okw)) return false;
+    tc_fence_after();
+#pragma unroll
+    for (int t = 0; t < kTilesPerSlot; ++t) {
+      if (t < nt) {
+        uint32_t s[32];
+        tmem_ld32(tmem + 256u * b + 128u * t + 32u * g + lane_base, s);
+        tmem_wait_ld(s);
+        const int j = j0 + t;
+        const int nvalid = (j + 1 == p.n_kt) ? p.last_valid : kKeys;
+        const float b0 = bc[t][0] * p.bias_mul, b1 = bc[t][1] * p.bias_mul;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float y = fmaf(__uint_as_float(s[e]), p.qk_scale, e < 16 ? b0 : b1);
+          if (32 * g + e < nvalid) ymax = fmaxf(ymax, y);
+        }
+      }
+    }
+    tc_fence_before();
+    warp_arrive_leader(&bars->s_free[b], sf0 + 8u * b, rank);
+  }
+  return true;
+}
+
 // Running-max segment: the four threads of a row share its maximum per key
 // tile (through shared memory).  When the maximum grows past the lazy
 // threshold, this warpgroup's DV/4 columns of O are rescaled, after the
@@ -1049,7 +1170,7 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc, float *st
                                  cluster_addr(&bars->s_free[1], 0)};
   const uint32_t pf_remote[2] = {cluster_addr(&bars->p_full[0], 0),
                                  cluster_addr(&bars->p_full[1], 0)};
-  constexpr bool kStatic = (MODE == kStaticCap);
+  constexpr bool kStatic = fixed_shift<MODE>();
   SoftCounters c;
   bool ok = true;
   Cursor cu = cursor_begin(p);
@@ -1062,10 +1183,41 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc, float *st
     const int pos = I * 16 + il;  // this thread's query position
     const float *brow = p.bias + static_cast<long long>(b) * p.bias_bstride +
                         (static_cast<size_t>(h) * p.bias_rows + I) * p.P;
-    float m = kStatic ? p.shift : -INFINITY;  // log2 units
+    const bool writes = valid && pos < p.Lq;  // rows past the end of a partial block: none
+    const size_t row = (static_cast<size_t>(b) * kH + h) * p.Lq + static_cast<size_t>(pos);
+    if constexpr (MODE == kRowMax) {
+      // First pass: the row's largest logit (log2 units) into lse, for the
+      // second pass's shift.  cap tanh is increasing, so the largest capped
+      // logit is the cap of the largest biased score.
+      float ymax = -INFINITY;
+      ok = segment_rowmax(sg, brow, tmem, lane_base, g, p, bars, rank, c, abort, ymax);
+      if (!ok) break;
+      // Double-buffered by segment parity, like the row sums below.
+      float(*mp)[128] = xc->mpart[c.xmcount & 1u];
+      mp[g][r] = ymax;
+      ok = exchange(&bars->xm, c.xmcount, abort, p.err);
+      if (!ok) break;
+      float mx = mp[0][r];
+#pragma unroll
+      for (int q = 1; q < kWG; ++q) mx = fmaxf(mx, mp[q][r]);
+      float mrow = p.A > 0.f ? p.A * tanh_approx(mx) : mx;
+      if (sg.dest == kDestMerge) {
+        // Second piece of a split pair: the first piece's maximum is in lse.
+        griddep_wait();
+        if (writes) mrow = fmaxf(mrow, p.lse[row]);
+      }
+      if (writes && g == 0) p.lse[row] = mrow;
+      continue;
+    }
+    // The fixed shift: p.shift, or with row shifts the smallest integer at or
+    // above the row's largest logit, which the first pass left in lse.
+    float shift = p.shift;
+    if constexpr (row_shift<MODE>()) shift = writes ? ceilf(p.lse[row]) : 0.f;
+    float m = kStatic ? shift : -INFINITY;  // log2 units
     float d = 0.f;
     if constexpr (kStatic && DV == 128) {
-      ok = segment_static_grouped<DV>(sg, brow, tmem, lane_base, g, p, bars, rank, c, abort, d);
+      ok = segment_static_grouped<MODE, DV>(sg, brow, tmem, lane_base, g, p, bars, rank, c,
+                                            abort, shift, d);
     } else if constexpr (kStatic) {
       ok = segment_static<MODE, DV>(sg, brow, tmem, lane_base, g, p, bars, rank, sf_remote,
                                     pf_remote, c, abort, d);
@@ -1079,8 +1231,6 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc, float *st
     // over this segment's keys (warpgroup g writes columns [g DV/4, (g+1)
     // DV/4) of the row) and lse.  The copy of block I0 in an odd CTA past the
     // end of an odd block count writes nothing.
-    const bool writes = valid && pos < p.Lq;  // rows past the end of a partial block: none
-    const size_t row = (static_cast<size_t>(b) * kH + h) * p.Lq + static_cast<size_t>(pos);
     float lse_a = 0.f;
     if (sg.dest == kDestMerge) {
       // The first piece of this pair was written by the previous launch;
@@ -1289,12 +1439,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // Static cap at value width 128: one warp group per S and P buffer;
     // otherwise every softmax warp takes part in every key tile.
     constexpr uint32_t kSPArrivals =
-        (MODE == kStaticCap && DV == 128) ? kPairSoftWarps / 2 : kPairSoftWarps;
-    for (int u = 0; u < 3; ++u) {
+        p_in_place<MODE, DV>() ? kPairSoftWarps / 2 : kPairSoftWarps;
+    for (int u = 0; u < static_cast<int>(kRowMaxBufs); ++u) {
       mbar_init(&bars->s_full[u], 1);
-      if (u < 2) mbar_init(&bars->s_free[u], kSPArrivals);
-      mbar_init(&bars->p_full[u], kSPArrivals);
-      mbar_init(&bars->pv_done[u], 1);
+      mbar_init(&bars->s_free[u], kSPArrivals);
+      if (u < 3) {
+        mbar_init(&bars->p_full[u], kSPArrivals);
+        mbar_init(&bars->pv_done[u], 1);
+      }
     }
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->xm, kSoftWarps);
@@ -1323,18 +1475,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (warp >= kSoftWarps) {  // the four role warps
     regs_dec<kRegsLow>();
     if (rank == 0 && warp == kWarpIssueS) {
-      issuer_s<p_in_place<MODE, DV>()>(q_s, k_s, bars, tmem, p, abort);  // the whole warp
+      // The whole warp.
+      if constexpr (MODE == kRowMax)
+        issuer_rowmax(q_s, k_s, bars, tmem, p, abort);
+      else
+        issuer_s<p_in_place<MODE, DV>()>(q_s, k_s, bars, tmem, p, abort);
     } else if (rank == 0 && warp == kWarpIssuePV) {
-      issuer_pv<DV, p_in_place<MODE, DV>()>(v_s, bars, tmem, p, abort);
+      if constexpr (MODE == kRowMax) {
+        // No PV in the first pass; the drain still counts this warp.
+        umma2_commit_self_w(&bars->drain);
+        drain_wait(&bars->drain, 0);
+      } else {
+        issuer_pv<DV, p_in_place<MODE, DV>()>(v_s, bars, tmem, p, abort);
+      }
     } else if (lane_id() == 0) {
       if (warp == kWarpLoadQK) {
         producer_qk(&tm_q, &tm_k, q_s, k_s, bars, p, rank, abort);
       } else if (warp == kWarpLoadV) {
-        producer_v<DV>(&tm_v, v_s, bars, p, rank, abort);
+        if constexpr (MODE != kRowMax) producer_v<DV>(&tm_v, v_s, bars, p, rank, abort);
       } else if (warp == kWarpIssueS) {
         relay_qk(bars, p, abort);
       } else if (warp == kWarpIssuePV) {
-        relay_v<DV>(bars, p, abort);
+        if constexpr (MODE != kRowMax) relay_v<DV>(bars, p, abort);
       }
     }
   } else {
@@ -1493,6 +1655,14 @@ cudaError_t configure_mode(int *max_clusters) {
 template <int DV>
 cudaError_t configure_any(int mode, int *max_clusters) {
   using namespace attn;
+  if constexpr (DV == 128) {
+    switch (mode) {
+      case kRowMax: return configure_mode<kRowMax, DV>(max_clusters);
+      case kRowShift: return configure_mode<kRowShift, DV>(max_clusters);
+      case kRowShiftCap: return configure_mode<kRowShiftCap, DV>(max_clusters);
+      default: break;
+    }
+  }
   switch (mode) {
     case kStaticCap: return configure_mode<kStaticCap, DV>(max_clusters);
     case kOnlineCap: return configure_mode<kOnlineCap, DV>(max_clusters);
@@ -1518,6 +1688,21 @@ int attn_mode(float cap) {
 float attn_static_shift(float A) {
   const float ca = ceilf(A);
   return ca <= 60.0f ? ca : 120.0f - ca;
+}
+
+// Value width 128 without scratch runs the caps beyond the fixed shift's
+// range (cap > 60, and no cap) in two passes over whole pairs of query
+// tiles: kRowMax writes every row's largest logit into lse, then the
+// fixed-shift kernel runs with each row's own shift ceil(max) (kRowShift,
+// kRowShiftCap), instead of the running maximum, whose exchange of the
+// maxima between the four warpgroups on every key tile costs about twice the
+// time.  Whole pairs, because a split pair's second piece would need the
+// maximum after the first piece has overwritten lse.
+bool attn_two_pass(int mode, int dv, bool scratch) {
+  return (mode == attn::kOnlineCap || mode == attn::kNoCap) && dv == 128 && !scratch;
+}
+int attn_second_pass_mode(int mode) {
+  return mode == attn::kNoCap ? attn::kRowShift : attn::kRowShiftCap;
 }
 
 // --------------------------------------------------------------------------
@@ -1703,9 +1888,10 @@ Plan plan_for(int n_items, int n_kt, int G, int scratch_slots) {
 // Plans are cached per (items, key tiles, clusters, scratch slots): the
 // two-phase search costs more than a launch.
 struct PlanKey {
-  int n_items, n_kt, G, slots;
+  int n_items, n_kt, G, slots, whole_only;
   bool operator==(const PlanKey &o) const {
-    return n_items == o.n_items && n_kt == o.n_kt && G == o.G && slots == o.slots;
+    return n_items == o.n_items && n_kt == o.n_kt && G == o.G && slots == o.slots &&
+           whole_only == o.whole_only;
   }
 };
 std::mutex g_plan_mu;
@@ -1714,6 +1900,13 @@ std::vector<std::pair<PlanKey, Plan>> g_plans;
 cudaError_t make_plan(int mode, int dv, int n_items, int n_kt, int num_sms, int scratch_slots,
                       Plan *pl) {
   int max_clusters = 0;
+  const bool two_pass = attn_two_pass(mode, dv, scratch_slots > 0);
+  if (two_pass) {
+    int first = 0;
+    cudaError_t e1 = configure_any<128>(attn::kRowMax, &first);
+    if (e1 != cudaSuccess) return e1;
+    mode = attn_second_pass_mode(mode);
+  }
   cudaError_t e = dv == 192 ? configure_any<192>(mode, &max_clusters)
                             : configure_any<128>(mode, &max_clusters);
   if (e != cudaSuccess) return e;
@@ -1724,7 +1917,7 @@ cudaError_t make_plan(int mode, int dv, int n_items, int n_kt, int num_sms, int 
   // parameters, sized for kAttnMaxClusters (plan_for clamps them).
   const int G = std::min(num_sms / 2, max_clusters);
   if (G < 1) return cudaErrorInvalidValue;
-  const PlanKey key{n_items, n_kt, G, scratch_slots};
+  const PlanKey key{n_items, n_kt, G, scratch_slots, two_pass ? 1 : 0};
   {
     std::lock_guard<std::mutex> lock(g_plan_mu);
     for (const auto &kv : g_plans)
@@ -1733,7 +1926,11 @@ cudaError_t make_plan(int mode, int dv, int n_items, int n_kt, int num_sms, int 
         return cudaSuccess;
       }
   }
-  Plan fresh = plan_for(n_items, n_kt, G, scratch_slots);
+  Plan fresh;
+  if (two_pass)
+    plan_whole(n_items, std::min(G, kAttnMaxClusters), &fresh);
+  else
+    fresh = plan_for(n_items, n_kt, G, scratch_slots);
   if (fresh.clusters < 1 ||
       (fresh.sched != attn::kSchedRange &&
        (fresh.clusters > kAttnMaxClusters || fresh.tail_clusters > kAttnMaxClusters)))
@@ -1776,6 +1973,17 @@ cudaError_t launch_dv(int mode, const CUtensorMap &tq, const CUtensorMap &tk,
                       const CUtensorMap &tv, const CUtensorMap &to, const attn::Params &p,
                       int clusters, bool dependent, cudaStream_t stream) {
   using namespace attn;
+  if constexpr (DV == 128) {
+    switch (mode) {
+      case kRowMax:
+        return launch_mode<kRowMax, DV>(tq, tk, tv, to, p, clusters, dependent, stream);
+      case kRowShift:
+        return launch_mode<kRowShift, DV>(tq, tk, tv, to, p, clusters, dependent, stream);
+      case kRowShiftCap:
+        return launch_mode<kRowShiftCap, DV>(tq, tk, tv, to, p, clusters, dependent, stream);
+      default: break;
+    }
+  }
   switch (mode) {
     case kStaticCap:
       return launch_mode<kStaticCap, DV>(tq, tk, tv, to, p, clusters, dependent, stream);
@@ -1801,7 +2009,13 @@ cudaError_t attn_fwd_kernel_count(int64_t B, int64_t Lq, int64_t L, int64_t Dv, 
   cudaError_t e = make_plan(attn_mode(cap), static_cast<int>(Dv), n_items, n_kt, num_sms,
                             scratch_slots, &pl);
   if (e != cudaSuccess) return e;
-  if (pl.sched == kSchedRange)
+  if (attn_two_pass(attn_mode(cap), static_cast<int>(Dv), scratch_slots > 0)) {
+    // The row maxima (one or two launches), then the row-shift kernel.
+    Plan p1;
+    e = make_plan(kRowMax, static_cast<int>(Dv), n_items, n_kt, num_sms, 0, &p1);
+    if (e != cudaSuccess) return e;
+    *count = (p1.tail_clusters > 0 ? 2 : 1) + 1;
+  } else if (pl.sched == kSchedRange)
     *count = (pl.clusters < 2 || pl.whole) ? 1 : 2;
   else
     *count = pl.tail_clusters > 0 ? 2 : 1;
@@ -1944,6 +2158,31 @@ cudaError_t launch_attn_fwd(const AttnLaunch &a) {
     char *base = static_cast<char *>(a.scratch);
     p.ws_out = reinterpret_cast<float *>(base);
     p.ws_lse = reinterpret_cast<float *>(base + a.scratch_slots * kAttnSlotOutBytes);
+  }
+  if (attn_two_pass(mode, dv, a.scratch != nullptr)) {
+    // The row maxima (on the usual schedule, split pairs merged by maximum),
+    // then the row-shift kernel on whole pairs (make_plan's plan for mode).
+    Plan p1;
+    e = make_plan(kRowMax, dv, p.n_items, p.n_kt, a.num_sms, 0, &p1);
+    if (e != cudaSuccess) return e;
+    Params q1 = p;
+    q1.sched = p1.sched;
+    q1.whole = p1.whole;
+    q1.n_whole = p1.n_whole;
+    q1.split_at = p1.split_at;
+    for (int c = 0; c <= kAttnMaxClusters; ++c) {
+      q1.wb[c] = c < static_cast<int>(p1.wb.size()) ? p1.wb[c] : 0;
+      q1.fb[c] = c < static_cast<int>(p1.fb.size()) ? p1.fb[c] : 0;
+    }
+    e = launch_dv<128>(kRowMax, tq, tk, tv, to, q1, p1.clusters, false, a.stream);
+    if (e != cudaSuccess) return e;
+    if (p1.tail_clusters > 0) {
+      q1.sched = kSchedTail;
+      e = launch_dv<128>(kRowMax, tq, tk, tv, to, q1, p1.tail_clusters, true, a.stream);
+      if (e != cudaSuccess) return e;
+    }
+    return launch_dv<128>(attn_second_pass_mode(mode), tq, tk, tv, to, p, pl.clusters, false,
+                          a.stream);
   }
   e = dv == 192 ? launch_dv<192>(mode, tq, tk, tv, to, p, pl.clusters, false, a.stream)
                 : launch_dv<128>(mode, tq, tk, tv, to, p, pl.clusters, false, a.stream);

@@ -457,3 +457,7 @@ def test_launch_count_matches_the_grid_policy(ag):
         assert ag.ag_attn_fwd_launch_count(B, L) in (1, 2)
     if torch.cuda.get_device_properties(0).multi_processor_count == 148:
         assert ag.ag_attn_fwd_launch_count(1, 8192) == 2
+        # cap > 60 or none: the row maxima (split like the main kernel: two
+        # launches) and the row-shift kernel on whole pairs.
+        assert ag.ag_attn_fwd_launch_count(1, 8192, cap=math.inf) == 3
+        assert ag.ag_attn_fwd_launch_count(1, 8192, cap=61.0) == 3
