@@ -148,8 +148,6 @@ template <int DV> struct Tmem {
 // buffer's last reader) instead of for the softmax, so the logits of a warp
 // group's next tile are usually ready before the group asks for them.
 constexpr uint32_t kIPBufs = 3;
-// The first pass of the two-pass schedule has no P and no O: four S buffers.
-constexpr uint32_t kRowMaxBufs = 4;
 constexpr uint32_t kIPColO = 384;
 // The fixed-shift modes at value width 128.
 template <int MODE, int DV> constexpr bool p_in_place() {
@@ -206,7 +204,7 @@ struct __align__(8) Barriers {
   uint64_t q_full, q_empty;
   uint64_t k_full[kStages], k_empty[kStages];
   uint64_t v_full[kVStagesMax], v_empty[kVStagesMax];  // [v_stages<DV>()] in use
-  uint64_t s_full[kRowMaxBufs], s_free[kRowMaxBufs];  // [3] / [2] / [4] in use (see issuer_s)
+  uint64_t s_full[3], s_free[2];  // s_full: three in use with P in place, else two
   uint64_t p_full[3], pv_done[3];  // three in use with P in place, else [Tmem<DV>::kNP]
   uint64_t o_full;
   uint64_t xm, xd;  // row-max / row-sum exchange between the warpgroups
@@ -1440,13 +1438,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // otherwise every softmax warp takes part in every key tile.
     constexpr uint32_t kSPArrivals =
         p_in_place<MODE, DV>() ? kPairSoftWarps / 2 : kPairSoftWarps;
-    for (int u = 0; u < static_cast<int>(kRowMaxBufs); ++u) {
+    for (int u = 0; u < 3; ++u) {
       mbar_init(&bars->s_full[u], 1);
-      mbar_init(&bars->s_free[u], kSPArrivals);
-      if (u < 3) {
-        mbar_init(&bars->p_full[u], kSPArrivals);
-        mbar_init(&bars->pv_done[u], 1);
-      }
+      if (u < 2) mbar_init(&bars->s_free[u], kSPArrivals);
+      mbar_init(&bars->p_full[u], kSPArrivals);
+      mbar_init(&bars->pv_done[u], 1);
     }
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->xm, kSoftWarps);
