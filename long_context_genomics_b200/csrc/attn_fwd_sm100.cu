@@ -913,11 +913,12 @@ __device__ __forceinline__ bool segment_static_grouped(const Segment &sg, const 
   StaticK k;
   constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
   const float A = MODE == kRowShift ? 1.f : p.A;
+  const float sh = row_shift<MODE>() ? shift : p.shift;
   k.sc = make_float2(p.qk_scale, p.qk_scale);
   k.a = make_float2(A, A);
-  k.nsh = make_float2(-shift, -shift);
-  k.km = make_float2(kShift - shift, kShift - shift);
-  k.tmin = (shift - 126.f) / A;
+  k.nsh = make_float2(-sh, -sh);
+  k.km = make_float2(kShift - sh, kShift - sh);
+  k.tmin = row_shift<MODE>() ? (sh - 126.f) / A : 0.f;
   float2 acc = make_float2(0.f, 0.f);
   const uint32_t pf0 = cluster_addr(&bars->p_full[0], 0);  // the even CTA's p_full
   // Key tile j of the segment is global tile c.su + (j - kb); the group takes
@@ -1181,9 +1182,9 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc, float *st
     const int pos = I * 16 + il;  // this thread's query position
     const float *brow = p.bias + static_cast<long long>(b) * p.bias_bstride +
                         (static_cast<size_t>(h) * p.bias_rows + I) * p.P;
-    const bool writes = valid && pos < p.Lq;  // rows past the end of a partial block: none
-    const size_t row = (static_cast<size_t>(b) * kH + h) * p.Lq + static_cast<size_t>(pos);
     if constexpr (MODE == kRowMax) {
+      const bool writes = valid && pos < p.Lq;
+      const size_t row = (static_cast<size_t>(b) * kH + h) * p.Lq + static_cast<size_t>(pos);
       // First pass: the row's largest logit (log2 units) into lse, for the
       // second pass's shift.  cap tanh is increasing, so the largest capped
       // logit is the cap of the largest biased score.
@@ -1210,7 +1211,10 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc, float *st
     // The fixed shift: p.shift, or with row shifts the smallest integer at or
     // above the row's largest logit, which the first pass left in lse.
     float shift = p.shift;
-    if constexpr (row_shift<MODE>()) shift = writes ? ceilf(p.lse[row]) : 0.f;
+    if constexpr (row_shift<MODE>()) {
+      const size_t row = (static_cast<size_t>(b) * kH + h) * p.Lq + static_cast<size_t>(pos);
+      shift = (valid && pos < p.Lq) ? ceilf(p.lse[row]) : 0.f;
+    }
     float m = kStatic ? shift : -INFINITY;  // log2 units
     float d = 0.f;
     if constexpr (kStatic && DV == 128) {
@@ -1229,6 +1233,8 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc, float *st
     // over this segment's keys (warpgroup g writes columns [g DV/4, (g+1)
     // DV/4) of the row) and lse.  The copy of block I0 in an odd CTA past the
     // end of an odd block count writes nothing.
+    const bool writes = valid && pos < p.Lq;  // rows past the end of a partial block: none
+    const size_t row = (static_cast<size_t>(b) * kH + h) * p.Lq + static_cast<size_t>(pos);
     float lse_a = 0.f;
     if (sg.dest == kDestMerge) {
       // The first piece of this pair was written by the previous launch;
