@@ -1057,19 +1057,35 @@ __device__ __forceinline__ bool segment_rowmax(const Segment &sg, const float *b
     const bool okw = mbar_wait(&bars->s_full[b], ph, abort, p.err, kSiteSoftS);
     if (!__all_sync(0xffffffffu, okw)) return false;
     tc_fence_after();
+    // Both tiles' logits in flight together.
+    uint32_t s[kTilesPerSlot][32];
+    const uint32_t t0 = tmem + 256u * b + 32u * g + lane_base;
+    tmem_ld32(t0, s[0]);
+    if (nt > 1) tmem_ld32(t0 + 128u, s[1]);
+    tmem_wait_ld(s[0]);
+    if (nt > 1) tmem_wait_ld(s[1]);
 #pragma unroll
     for (int t = 0; t < kTilesPerSlot; ++t) {
       if (t < nt) {
-        uint32_t s[32];
-        tmem_ld32(tmem + 256u * b + 128u * t + 32u * g + lane_base, s);
-        tmem_wait_ld(s);
         const int j = j0 + t;
         const int nvalid = (j + 1 == p.n_kt) ? p.last_valid : kKeys;
         const float b0 = bc[t][0] * p.bias_mul, b1 = bc[t][1] * p.bias_mul;
+        if (32 * g + 32 <= nvalid) {
+          // qk_scale > 0 and one bias cell per 16 keys: the largest score of
+          // a 16-key piece comes from its largest logit.
+          float m0 = __uint_as_float(s[t][0]), m1 = __uint_as_float(s[t][16]);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float y = fmaf(__uint_as_float(s[e]), p.qk_scale, e < 16 ? b0 : b1);
-          if (32 * g + e < nvalid) ymax = fmaxf(ymax, y);
+          for (int e = 1; e < 16; ++e) {
+            m0 = fmaxf(m0, __uint_as_float(s[t][e]));
+            m1 = fmaxf(m1, __uint_as_float(s[t][16 + e]));
+          }
+          ymax = fmaxf(ymax, fmaxf(fmaf(m0, p.qk_scale, b0), fmaf(m1, p.qk_scale, b1)));
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float y = fmaf(__uint_as_float(s[t][e]), p.qk_scale, e < 16 ? b0 : b1);
+            if (32 * g + e < nvalid) ymax = fmaxf(ymax, y);
+          }
         }
       }
     }
