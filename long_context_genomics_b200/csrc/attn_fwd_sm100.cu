@@ -191,7 +191,7 @@ enum Site : unsigned {
   kSiteProdQ = 1, kSiteProdK = 2, kSiteIssueQ = 3, kSiteIssueK = 4,
   kSiteIssueP = 5, kSiteSoftS = 6, kSiteSoftO = 7, kSiteDrain = 8,
   kSiteXchg = 9, kSiteSoftPV = 10, kSiteRelay = 11, kSiteProdV = 12,
-  kSiteIssueV = 13, kSiteIssueSFree = 14
+  kSiteIssueV = 13, kSiteIssueSFree = 14, kSiteIssueOFree = 15
 };
 
 // Per-CTA barriers.  In the even CTA, q_full, k_full and v_full also count
@@ -200,13 +200,15 @@ enum Site : unsigned {
 // of a load; s_free and p_full are used in the even CTA only (the odd CTA's
 // softmax warps arrive on them remotely).  q_empty, k_empty, v_empty, s_full,
 // pv_done and o_full are signalled in both CTAs by the even CTA's commits.
+// o_free (even CTA, P in place) counts every softmax warp of the pair once
+// per segment, after its last read of O.
 struct __align__(8) Barriers {
   uint64_t q_full, q_empty;
   uint64_t k_full[kStages], k_empty[kStages];
   uint64_t v_full[kVStagesMax], v_empty[kVStagesMax];  // [v_stages<DV>()] in use
   uint64_t s_full[3], s_free[2];  // s_full: three in use with P in place, else two
   uint64_t p_full[3], pv_done[3];  // three in use with P in place, else [Tmem<DV>::kNP]
-  uint64_t o_full;
+  uint64_t o_full, o_free;
   uint64_t xm, xd;  // row-max / row-sum exchange between the warpgroups
   uint64_t drain;   // both issuing threads' MMAs have completed
   uint32_t tmem_base;
@@ -659,7 +661,7 @@ __device__ __forceinline__ void issuer_pv(uint8_t *v_s, Barriers *bars, uint32_t
   constexpr uint32_t kBufs = kIP ? kIPBufs : T::kNP;
   constexpr int kVS = v_stages<DV>(), kVT = v_tiles_per_slot<DV>();
   const uint32_t v_addr = smem_u32(v_s);
-  uint32_t vl = 0, pu = 0;
+  uint32_t vl = 0, pu = 0, seg = 0;
   bool ok = true;
   Cursor cu = cursor_begin(p);
   Segment sg;
@@ -676,6 +678,14 @@ __device__ __forceinline__ void issuer_pv(uint8_t *v_s, Barriers *bars, uint32_t
       const uint32_t pb = pu % kBufs, pn = pu / kBufs;
       ok = mbar_wait_warp(&bars->p_full[pb], pn & 1u, abort, p.err, kSiteIssueP);
       if (!ok) break;
+      if (kIP && i == 0 && seg > 0) {
+        // The first PV of a segment overwrites O.  With P in place the two
+        // softmax groups take alternate tiles, so the P of this tile does not
+        // imply that the other group has read the previous segment's O: wait
+        // until every softmax warp of the pair has.
+        ok = mbar_wait_warp(&bars->o_free, (seg - 1) & 1u, abort, p.err, kSiteIssueOFree);
+        if (!ok) break;
+      }
       tc_fence_after();
       const uint32_t va =
           v_addr + slot * v_slot_bytes<DV>() + (i % kVT) * VLayout<DV>::kTileBytes;
@@ -688,6 +698,7 @@ __device__ __forceinline__ void issuer_pv(uint8_t *v_s, Barriers *bars, uint32_t
       if (i % kVT == kVT - 1 || j + 1 == sg.ke) umma2_commit_both_w(&bars->v_empty[slot]);
       ++pu;
     }
+    ++seg;
   }
   umma2_commit_self_w(&bars->drain);
   drain_wait(&bars->drain, 0);
@@ -1308,6 +1319,14 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc, float *st
       const int lane = static_cast<int>(lane_id());
       float *slot = stage + (threadIdx.x >> 5) * kStageWarpFloats;
       const int r0 = r - lane;  // the warp's first tile row
+      // Once this warp's reads of O have completed (tcgen05.wait::ld), the
+      // PV issuer may start the next segment's O over it.
+      auto release_o = [&] {
+        if constexpr (p_in_place<MODE, DV>()) {
+          tc_fence_before();
+          warp_arrive_leader(&bars->o_free, cluster_addr(&bars->o_free, 0), rank);
+        }
+      };
       // The bulk store of this warp's previous segment has read the slot.
       if (lane == 0) bulk_wait_read_all();
       __syncwarp();
@@ -1330,6 +1349,9 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc, float *st
                   __uint_as_float(o[4 * e + 2]) * wb, __uint_as_float(o[4 * e + 3]) * wb);
             }
           }
+        }
+        release_o();
+        if (valid) {
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
@@ -1382,6 +1404,7 @@ __device__ __forceinline__ void softmax_role(Barriers *bars, Xchg *xc, float *st
           }
           __syncwarp();
         }
+        release_o();
       }
     } else {
       // This warpgroup's DV / 4 columns of the row, 16 at a time (every lane
@@ -1467,6 +1490,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(&bars->pv_done[u], 1);
     }
     mbar_init(&bars->o_full, 1);
+    mbar_init(&bars->o_free, kPairSoftWarps);
     mbar_init(&bars->xm, kSoftWarps);
     mbar_init(&bars->xd, kSoftWarps);
     mbar_init(&bars->drain, 2);
