@@ -127,6 +127,20 @@ def test_ragged_and_odd_shapes(ag, oracle_lib, B, L, cap):
     _compare(out, lse, ro, rl, f"B={B} L={L} cap={cap}")
 
 
+@pytest.mark.parametrize("B,L", [(160, 128), (48, 250)])
+@pytest.mark.parametrize("cap", [5.0, 50.0, math.inf])
+def test_many_short_segments_per_cluster(ag, oracle_lib, B, L, cap):
+    """Many items of one or two key tiles: every cluster runs several short
+    segments in a row, so the output accumulator is read out and restarted
+    many times per launch, and with one-tile segments each softmax group
+    owns every other segment's only tile."""
+    inp = ag_inputs.random_case(B, 8, L, 128, 128, 16, seed=B * 1000 + L + 7)
+    out, lse = _gpu_attn(ag, inp, cap)
+    ro, rl = oracle_lib.attn_fwd(inp["q"], inp["k"], inp["v"], inp["bias"],
+                                 block=16, cap=cap)
+    _compare(out, lse, ro, rl, f"B={B} L={L} cap={cap}")
+
+
 @pytest.mark.parametrize("B,L", [(1, 1), (1, 17), (2, 100), (1, 1000), (3, 2049),
                                  (1, 4095)])
 @pytest.mark.parametrize("cap", [5.0, 50.0, math.inf])
