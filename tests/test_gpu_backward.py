@@ -59,6 +59,8 @@ def _close(name, got, want):
     (3, 64, 128, 5.0, True),
     (2, 16, 128, 5.0, False),       # one query block: one CTA of the key pair has none
     (1, 1000, 128, 40.0, False),    # many steps per tile and per key CTA, ragged end
+    (160, 128, 128, 5.0, False),    # many items: accumulators restarted many times per CTA
+    (48, 250, 128, math.inf, True), # many ragged items, one bias per item, no cap
 ])
 def test_backward_parity(ag, oracle_lib, B, L, Dv, cap, batched):
     c = ag_inputs.random_case(B, 8, L, 128, Dv, 16, seed=L + B, batched_bias=batched)
