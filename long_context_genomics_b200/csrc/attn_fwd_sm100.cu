@@ -169,12 +169,18 @@ constexpr int kNumWarps = 4 * kWG + 4;
 constexpr int kThreads = kNumWarps * 32;
 // Registers per thread: the launch gives every thread kRegsLaunch (the cap
 // for this block size, which ptxas allocates when setmaxnreg is present; the
-// launcher checks it); the loader/issuer warpgroup then drops to kRegsLow.
-// The softmax keeps the launch count.
+// launcher refuses a build with fewer); the loader/issuer warpgroup then
+// drops to kRegsLow and the four softmax warpgroups rise to kRegsHigh out of
+// what it released (ptxas then compiles the softmax without spills).  The
+// split must fit the launch allocation, or the increase would wait forever:
+// 128 x 56 + 512 x 104 = 60,416 <= 640 x 96 = 61,440.
 constexpr uint32_t kRegsLaunch = 96;
-constexpr uint32_t kRegsLow = 88;
-static_assert(kSoftThreads * kRegsLaunch + 128 * kRegsLow <= kThreads * kRegsLaunch,
+constexpr uint32_t kRegsLow = 56;
+constexpr uint32_t kRegsHigh = 104;
+static_assert(kSoftThreads * kRegsHigh + 128 * kRegsLow <= kThreads * kRegsLaunch,
               "register split exceeds the launch allocation");
+static_assert(kRegsLow % 8 == 0 && kRegsHigh % 8 == 0 && kRegsLow >= 24 && kRegsHigh <= 256,
+              "setmaxnreg counts are multiples of 8 in [24, 256]");
 constexpr uint32_t kIdescQK = idesc_bf16_f32(256, kKeys, 0);  // K-major B (K)
 template <int DV> constexpr uint32_t idesc_pv() { return idesc_bf16_f32(256, DV, 1); }
 constexpr float kLog2e = 1.4426950408889634f;
@@ -1542,6 +1548,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
     }
   } else {
+    regs_inc<kRegsHigh>();  // covered by the role warpgroup's decrease above
     softmax_role<MODE, DV>(bars, xc, stage, tmem, &tm_o, p, rank, abort);
   }
   __syncwarp();

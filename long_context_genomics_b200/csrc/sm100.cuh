@@ -230,13 +230,19 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
 
 // ---------------------------------------------------------------------------
 // tcgen05: tensor memory and the 5th-generation tensor core.
-// Per-warpgroup register release (every warp of the warpgroup executes the
-// same instruction): lowers the warpgroup's register count below the launch
-// allocation.  (The matching increase is not used: an increase that the
-// decreases cannot cover waits forever.)
+// Per-warpgroup register counts (every warp of the warpgroup executes the
+// same instruction).  regs_dec lowers the warpgroup's count below the launch
+// allocation; regs_inc raises it, taking registers that other warpgroups of
+// the block have released, and waits until they have: an increase that the
+// decreases cannot cover waits forever, so a caller checks the split against
+// the block's launch allocation (threads x registers at launch).
 template <uint32_t kRegs>
 __device__ __forceinline__ void regs_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+template <uint32_t kRegs>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
 }
 
 __device__ __forceinline__ void tc_fence_before() {
